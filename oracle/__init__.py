@@ -1,0 +1,228 @@
+"""fp64 CPU oracle of the gated delta rule — TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may import
+this package.  It shares no code with the CUDA library (``gated_deltanet_linear_18_b200``) and the
+library never imports it.  The arithmetic lives in ``gdn_oracle.c`` (plain C, double precision,
+token by token); this module only compiles it with gcc and marshals numpy arrays.
+
+Functions and the passages they follow (page titles; the C file's header has the detail):
+  * ``gated_delta``       — "L'attention hybride", section "La récurrence" (symbols alpha, beta, I)
+                            with the gated delta rule S_t = a S (I - b k k^T) + b v k^T, o = S q.
+  * ``decode_steps``      — "Chapitre 16 ... Kimi K3", 16.3: read the state, output, update;
+                            the recurrence applied to one token per call.
+  * ``causal_conv_silu``  — "L'attention hybride", "Le décompte" (4 taps per channel, no bias)
+                            and "Les briques d'un réseau de neurones", 2. (SiLU).
+  * ``l2_normalize``      — q/k normalisation of the layer's prologue (the pages give no eps;
+                            the caller passes one).
+  * ``gated_rmsnorm``     — "L'attention hybride" (swish output gate, one 128-wide gain) and
+                            "Les briques d'un réseau de neurones", 4. (RMSNorm, eps 1e-5).
+  * ``layer_forward``     — composition of the above.  Parity unpinned beyond its pinned parts:
+                            the pages print no worked example of a whole layer.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from typing import Optional, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "gdn_oracle.c")
+_OUT_DIR = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_OUT_DIR, "liboracle_gdn.so")
+_GCC = ["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-fno-fast-math", "-ffp-contract=off"]
+_lock = threading.Lock()
+_default = None
+
+
+def compile_source(src_path: str, out_path: str) -> str:
+    """gcc a C oracle source into a shared library (IEEE fp64: no fast-math, no contraction)."""
+    os.makedirs(os.path.dirname(out_path), exist_ok=True)
+    tmp = out_path + f".tmp{os.getpid()}"
+    subprocess.check_call(_GCC + ["-o", tmp, src_path, "-lm", "-lpthread"])
+    os.replace(tmp, out_path)
+    return out_path
+
+
+def build(force: bool = False) -> str:
+    """Compile ``gdn_oracle.c`` into ``oracle/_build`` when missing or older than the source."""
+    stale = (not os.path.exists(_LIB_PATH)
+             or os.path.getmtime(_LIB_PATH) < os.path.getmtime(SOURCE))
+    if force or stale:
+        compile_source(SOURCE, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _f64(x) -> Optional[np.ndarray]:
+    """Widen a tensor/array to C-contiguous float64 (bf16 and fp32 widen exactly)."""
+    if x is None:
+        return None
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().to("cpu", torch.float64).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a: Optional[np.ndarray]):
+    if a is None:
+        return ctypes.POINTER(ctypes.c_double)()
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def default_threads() -> int:
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:  # pragma: no cover
+        return max(1, os.cpu_count() or 1)
+
+
+class OracleLib:
+    """ctypes view of one compiled oracle library (the default one, or a test's variant)."""
+
+    def __init__(self, path: str):
+        lib = ctypes.CDLL(path)
+        P = ctypes.POINTER(ctypes.c_double)
+        L, I, D = ctypes.c_long, ctypes.c_int, ctypes.c_double
+        lib.oracle_gated_delta.argtypes = [P, P, P, P, P, P, P, P, L, L, I, I, I, I, D, I]
+        lib.oracle_gated_delta.restype = I
+        lib.oracle_causal_conv_silu.argtypes = [P, P, P, L, L, L]
+        lib.oracle_causal_conv_silu.restype = None
+        lib.oracle_l2_normalize.argtypes = [P, P, L, I, D]
+        lib.oracle_l2_normalize.restype = None
+        lib.oracle_gated_rmsnorm.argtypes = [P, P, P, P, L, I, D]
+        lib.oracle_gated_rmsnorm.restype = None
+        self.lib = lib
+        self.path = path
+
+    # -- the recurrence ---------------------------------------------------------------------
+    def gated_delta(self, q, k, v, log_alpha, beta, S0=None, scale: float = 1.0,
+                    threads: Optional[int] = None, want_state: bool = True
+                    ) -> Tuple[np.ndarray, Optional[np.ndarray]]:
+        """Token-by-token recurrence.  q,k [B,T,Hk,dk]; v [B,T,Hv,dv]; gates [B,T,Hv];
+        S0 [B,Hv,dk,dv] holding S^T, or None for the zero state.
+        Returns (o [B,T,Hv,dv], S_T [B,Hv,dk,dv] holding S^T), fp64."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        la, be, s0 = _f64(log_alpha), _f64(beta), _f64(S0)
+        B, T, Hk, dk = q.shape
+        Hv, dv = v.shape[2], v.shape[3]
+        assert k.shape == q.shape and v.shape[:2] == (B, T)
+        assert la.shape == (B, T, Hv) == be.shape
+        if s0 is not None:
+            assert s0.shape == (B, Hv, dk, dv)
+        o = np.zeros((B, T, Hv, dv), dtype=np.float64)
+        sT = np.zeros((B, Hv, dk, dv), dtype=np.float64) if want_state else None
+        rc = self.lib.oracle_gated_delta(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(be),
+                                         _ptr(s0), _ptr(o), _ptr(sT), B, T, Hk, Hv, dk, dv,
+                                         float(scale), int(threads or default_threads()))
+        if rc != 0:
+            raise ValueError("oracle_gated_delta rejected the sizes")
+        return o, sT
+
+    def decode_steps(self, q, k, v, log_alpha, beta, S0, scale: float = 1.0,
+                     threads: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray]:
+        """``steps`` consecutive single-token steps over N sequences: q,k [steps,N,Hk,dk];
+        v [steps,N,Hv,dv]; gates [steps,N,Hv]; S0 [N,Hv,dk,dv].  Each step reads the state,
+        writes its output and the updated state.  Returns (o [steps,N,Hv,dv], final state)."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        la, be, S = _f64(log_alpha), _f64(beta), _f64(S0)
+        outs = []
+        for s in range(q.shape[0]):
+            o, S = self.gated_delta(q[s][:, None], k[s][:, None], v[s][:, None],
+                                    la[s][:, None], be[s][:, None], S, scale=scale,
+                                    threads=threads)
+            outs.append(o[:, 0])
+        return np.stack(outs), S
+
+    # -- prologue / epilogue pieces -----------------------------------------------------------
+    def causal_conv_silu(self, x, w) -> np.ndarray:
+        """x [B,T,C]; w [C,4], tap 3 on the current token; zero history.  SiLU(conv(x))."""
+        x, w = _f64(x), _f64(w)
+        B, T, C = x.shape
+        assert w.shape == (C, 4)
+        y = np.zeros_like(x)
+        self.lib.oracle_causal_conv_silu(_ptr(x), _ptr(w), _ptr(y), B, T, C)
+        return y
+
+    def l2_normalize(self, x, eps: float) -> np.ndarray:
+        """x / sqrt(sum x^2 + eps) over the last dimension."""
+        x = _f64(x)
+        d = x.shape[-1]
+        y = np.zeros_like(x)
+        self.lib.oracle_l2_normalize(_ptr(x), _ptr(y), x.size // d, d, float(eps))
+        return y
+
+    def gated_rmsnorm(self, o, z, w, eps: float) -> np.ndarray:
+        """o / sqrt(mean(o^2) + eps) * w * z * sigmoid(z) over the last dimension."""
+        o, z, w = _f64(o), _f64(z), _f64(w)
+        d = o.shape[-1]
+        assert z.shape == o.shape and w.shape == (d,)
+        y = np.zeros_like(o)
+        self.lib.oracle_gated_rmsnorm(_ptr(o), _ptr(z), _ptr(w), _ptr(y), o.size // d, d,
+                                      float(eps))
+        return y
+
+    def prologue(self, q_raw, k_raw, v_raw, wq, wk, wv, Hk: int, Hv: int, dk: int, dv: int,
+                 l2_eps: float):
+        """Conv(4 taps) + SiLU on the q, k, v channels, then L2 normalisation of each q and k
+        head.  Inputs [B,T,H*d]; returns q,k [B,T,Hk,dk], v [B,T,Hv,dv] (fp64)."""
+        qc = self.causal_conv_silu(q_raw, wq)
+        kc = self.causal_conv_silu(k_raw, wk)
+        vc = self.causal_conv_silu(v_raw, wv)
+        B, T = qc.shape[:2]
+        q = self.l2_normalize(qc.reshape(B, T, Hk, dk), l2_eps)
+        k = self.l2_normalize(kc.reshape(B, T, Hk, dk), l2_eps)
+        return q, k, vc.reshape(B, T, Hv, dv)
+
+    def layer_forward(self, q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w,
+                      Hk: int, Hv: int, dk: int, dv: int, l2_eps: float = 1e-6,
+                      norm_eps: float = 1e-5, scale: float = 1.0,
+                      threads: Optional[int] = None):
+        """Prologue -> recurrence -> gated RMSNorm.  Returns (y [B,T,Hv,dv], S_T)."""
+        q, k, v = self.prologue(q_raw, k_raw, v_raw, wq, wk, wv, Hk, Hv, dk, dv, l2_eps)
+        o, sT = self.gated_delta(q, k, v, log_alpha, beta, S0, scale=scale, threads=threads)
+        B, T = o.shape[:2]
+        y = self.gated_rmsnorm(o, _f64(z).reshape(B, T, Hv, dv), norm_w, norm_eps)
+        return y, sT
+
+
+def get() -> OracleLib:
+    """The default oracle (compiled on first use)."""
+    global _default
+    with _lock:
+        if _default is None:
+            _default = OracleLib(build())
+    return _default
+
+
+def gated_delta(*a, **kw):
+    return get().gated_delta(*a, **kw)
+
+
+def decode_steps(*a, **kw):
+    return get().decode_steps(*a, **kw)
+
+
+def causal_conv_silu(*a, **kw):
+    return get().causal_conv_silu(*a, **kw)
+
+
+def l2_normalize(*a, **kw):
+    return get().l2_normalize(*a, **kw)
+
+
+def gated_rmsnorm(*a, **kw):
+    return get().gated_rmsnorm(*a, **kw)
+
+
+def prologue(*a, **kw):
+    return get().prologue(*a, **kw)
+
+
+def layer_forward(*a, **kw):
+    return get().layer_forward(*a, **kw)

@@ -1,0 +1,275 @@
+"""Pins of the fp64 oracle against what the pages and mathematics fix (not against itself).
+
+Each ``pin_*`` takes an ``oracle.OracleLib`` and raises ``AssertionError`` when the oracle breaks
+the pinned fact.  ``test_oracle_pins.py`` runs them on the real oracle; ``test_oracle_mutants.py``
+runs them on deliberately broken copies to show that each plausible mistake is caught.
+
+Sources (page titles):
+  [HYB] "L'attention hybride", section "La récurrence": alpha_t in ]0,1[ fades the whole state;
+        beta_t in ]0,1[ replaces precisely the association bound to k_t; I is the identity.
+        Section "L'état, en mémoire": the state has the same size for a thousand tokens or a
+        million.
+  [KIMI] "Chapitre 16 - Assembler un système de type Kimi K3": 16.2 blocks hand the state on
+        (256 prompt tokens in blocks of 64 make four blocks); 16.3 a decode step reads the fixed
+        state, outputs and updates it; 16.4 the linear memory is a compressed state that can be
+        corrected.
+  [BRK] "Les briques d'un réseau de neurones", 2. sigmoid / SiLU, 4. RMSNorm.
+"""
+from __future__ import annotations
+
+import numpy as np
+from scipy.special import expit
+
+
+def _unit(x):
+    return x / np.linalg.norm(x, axis=-1, keepdims=True)
+
+
+def _rand(seed, B=1, T=8, Hk=1, Hv=1, dk=4, dv=4, unit_k=True, s0=0.5):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, T, Hk, dk))
+    k = rng.standard_normal((B, T, Hk, dk))
+    if unit_k:
+        q, k = _unit(q), _unit(k)
+    v = rng.standard_normal((B, T, Hv, dv))
+    la = -np.log1p(np.exp(rng.standard_normal((B, T, Hv)))) * 0.3      # alpha in (0, 1)
+    be = expit(rng.standard_normal((B, T, Hv)))                          # beta in (0, 1)
+    S0 = rng.standard_normal((B, Hv, dk, dv)) * s0 if s0 else None
+    return q, k, v, la, be, S0
+
+
+def _heads(G, Hv):
+    return [h // G for h in range(Hv)]
+
+
+# ---------------------------------------------------------------------------------------------
+# recurrence
+# ---------------------------------------------------------------------------------------------
+
+def pin_identity_when_alpha1_beta0(orc):
+    """alpha = 1, beta = 0: nothing fades and nothing is written, so S_t = S0 for every t and
+    o_t = S0 q_t (closed form; the state stored transposed means o = M0^T q)."""
+    q, k, v, la, be, S0 = _rand(1, B=2, T=9, Hk=2, Hv=4, dk=5, dv=3)
+    la[:] = 0.0
+    be[:] = 0.0
+    o, sT = orc.gated_delta(q, k, v, la, be, S0)
+    assert np.array_equal(sT, S0)
+    G = 2
+    for h in range(4):
+        expect = np.einsum("bid,bti->btd", S0[:, h], q[:, :, h // G])
+        np.testing.assert_allclose(o[:, :, h], expect, rtol=1e-13, atol=1e-13)
+
+
+def pin_pure_decay_when_beta0(orc):
+    """beta = 0: S_t = (prod_{s<=t} alpha_s) S0, so o_t = (prod_{s<=t} alpha_s) S0 q_t."""
+    q, k, v, la, be, S0 = _rand(2, B=1, T=12, Hk=1, Hv=2, dk=4, dv=6)
+    be[:] = 0.0
+    o, sT = orc.gated_delta(q, k, v, la, be, S0)
+    decay = np.exp(np.cumsum(la, axis=1))                                # [B, T, Hv]
+    for h in range(2):
+        np.testing.assert_allclose(sT[:, h], S0[:, h] * decay[:, -1, h][:, None, None],
+                                   rtol=1e-12, atol=1e-14)
+        expect = np.einsum("bid,bti->btd", S0[:, h], q[:, :, 0]) * decay[:, :, h][..., None]
+        np.testing.assert_allclose(o[:, :, h], expect, rtol=1e-12, atol=1e-14)
+
+
+def pin_exact_retrieval_orthonormal_keys(orc):
+    """alpha = 1, beta = 1 and orthonormal keys k_t = e_{pi(t)}: each write replaces the value
+    bound to its key, so S k_i = v_i exactly for every key written, whatever S0 held; querying
+    with the key just written returns its value ([HYB] role of beta; [KIMI] 16.4)."""
+    d = 8
+    rng = np.random.default_rng(3)
+    perm = rng.permutation(d)
+    T = d
+    k = np.zeros((1, T, 1, d))
+    k[0, np.arange(T), 0, perm] = 1.0
+    q = k.copy()
+    v = rng.standard_normal((1, T, 1, d))
+    la = np.zeros((1, T, 1))
+    be = np.ones((1, T, 1))
+    S0 = rng.standard_normal((1, 1, d, d))
+    o, sT = orc.gated_delta(q, k, v, la, be, S0)
+    np.testing.assert_allclose(o[0, :, 0], v[0, :, 0], rtol=0, atol=1e-14)
+    # S e_j is row j of the stored S^T
+    np.testing.assert_allclose(sT[0, 0][perm], v[0, :, 0], rtol=0, atol=1e-14)
+
+
+def pin_overwrite_same_key(orc):
+    """Writing a second value under the same unit key with beta = 1 replaces the first one:
+    S k = v2 afterwards (the memory is correctable, [KIMI] 16.4; [HYB] role of beta)."""
+    rng = np.random.default_rng(4)
+    dk, dv = 6, 5
+    kk = _unit(rng.standard_normal(dk))
+    k = np.stack([kk, kk])[None, :, None, :]
+    q = k.copy()
+    v = rng.standard_normal((1, 2, 1, dv))
+    la = np.zeros((1, 2, 1))
+    be = np.ones((1, 2, 1))
+    S0 = rng.standard_normal((1, 1, dk, dv))
+    o, sT = orc.gated_delta(q, k, v, la, be, S0)
+    np.testing.assert_allclose(o[0, 1, 0], v[0, 1, 0], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(sT[0, 0].T @ kk, v[0, 1, 0], rtol=0, atol=1e-13)
+
+
+def pin_bruteforce_unrolled_products(orc):
+    """On tiny inputs the recurrence equals its unrolled solution built from explicit d_k x d_k
+    transition matrices A_t = alpha_t (I - beta_t k_t k_t^T):
+        S_t = S0 A_1 ... A_t + sum_{s<=t} beta_s v_s k_s^T A_{s+1} ... A_t,  o_t = scale S_t q_t.
+    Keys are not normalised here; GQA uses 2 value heads per key head."""
+    B, T, Hk, Hv, dk, dv = 2, 7, 1, 2, 3, 4
+    q, k, v, la, be, S0 = _rand(5, B=B, T=T, Hk=Hk, Hv=Hv, dk=dk, dv=dv, unit_k=False)
+    scale = 0.75
+    o, sT = orc.gated_delta(q, k, v, la, be, S0, scale=scale)
+    I = np.eye(dk)
+    for b in range(B):
+        for h in range(Hv):
+            hk = h // (Hv // Hk)
+            A = [np.exp(la[b, t, h]) * (I - be[b, t, h] * np.outer(k[b, t, hk], k[b, t, hk]))
+                 for t in range(T)]
+            for t in range(T):
+                prod = I.copy()
+                for s in range(t + 1):
+                    prod = prod @ A[s]
+                S = S0[b, h].T @ prod
+                for s in range(t + 1):
+                    tail = I.copy()
+                    for r in range(s + 1, t + 1):
+                        tail = tail @ A[r]
+                    S = S + be[b, s, h] * np.outer(v[b, s, h], k[b, s, hk]) @ tail
+                np.testing.assert_allclose(o[b, t, h], scale * S @ q[b, t, hk],
+                                           rtol=1e-11, atol=1e-12)
+            np.testing.assert_allclose(sT[b, h], S.T, rtol=1e-11, atol=1e-12)
+
+
+def pin_frobenius_bound(orc):
+    """For unit keys and alpha, beta in (0, 1): ||S_t||_F <= alpha_t ||S_{t-1}||_F + beta_t ||v_t||,
+    because I - beta k k^T has eigenvalues {1, 1 - beta} and ||beta v k^T||_F = beta ||v||."""
+    T, d = 300, 16
+    q, k, v, la, be, S0 = _rand(6, T=T, dk=d, dv=d, s0=0.3)
+    S = S0
+    prev = np.linalg.norm(S0)
+    for t in range(T):
+        sl = slice(t, t + 1)
+        _, S = orc.gated_delta(q[:, sl], k[:, sl], v[:, sl], la[:, sl], be[:, sl], S)
+        now = np.linalg.norm(S)
+        bound = np.exp(la[0, t, 0]) * prev + be[0, t, 0] * np.linalg.norm(v[0, t, 0])
+        assert now <= bound * (1 + 1e-12) + 1e-14, (t, now, bound)
+        prev = now
+
+
+def pin_gqa_equals_repeated_key_heads(orc):
+    """Hv/Hk value heads share one key head ([HYB] three value heads per key head): the result
+    equals giving every value head its own copy of its key/query head (contiguous groups)."""
+    q, k, v, la, be, S0 = _rand(7, B=2, T=10, Hk=2, Hv=6, dk=4, dv=3)
+    o, sT = orc.gated_delta(q, k, v, la, be, S0)
+    qr, kr = np.repeat(q, 3, axis=2), np.repeat(k, 3, axis=2)
+    o2, sT2 = orc.gated_delta(qr, kr, v, la, be, S0)
+    assert np.array_equal(o, o2) and np.array_equal(sT, sT2)
+
+
+def pin_scale_is_linear_in_output_only(orc):
+    """The query scale multiplies o and leaves the state untouched."""
+    q, k, v, la, be, S0 = _rand(8, T=6, dk=4, dv=4)
+    o1, s1 = orc.gated_delta(q, k, v, la, be, S0, scale=1.0)
+    o2, s2 = orc.gated_delta(q, k, v, la, be, S0, scale=0.25)
+    assert np.array_equal(s1, s2)
+    np.testing.assert_allclose(o2, 0.25 * o1, rtol=1e-14, atol=1e-15)
+
+
+def pin_split_run_equals_one_run(orc):
+    """Handing the state from one call to the next (S_T of one as S0 of the next) gives the same
+    result as one call: 256 prompt tokens as four blocks of 64 ([KIMI] 16.2)."""
+    q, k, v, la, be, S0 = _rand(9, B=1, T=256, Hk=1, Hv=2, dk=4, dv=4)
+    o, sT = orc.gated_delta(q, k, v, la, be, S0)
+    S = S0
+    parts = []
+    for c in range(4):
+        sl = slice(64 * c, 64 * (c + 1))
+        oc, S = orc.gated_delta(q[:, sl], k[:, sl], v[:, sl], la[:, sl], be[:, sl], S)
+        parts.append(oc)
+    assert np.array_equal(np.concatenate(parts, axis=1), o) and np.array_equal(S, sT)
+
+
+def pin_state_size_constant_in_T(orc):
+    """The state keeps its shape and size whatever the number of tokens ([HYB] L'état)."""
+    shapes = set()
+    for T in (1, 17, 300):
+        q, k, v, la, be, S0 = _rand(10, T=T, dk=4, dv=3, s0=0)
+        _, sT = orc.gated_delta(q, k, v, la, be, S0)
+        shapes.add((sT.shape, sT.nbytes))
+    assert shapes == {((1, 1, 4, 3), 1 * 1 * 4 * 3 * 8)}
+
+
+def pin_decode_steps_equal_recurrence(orc):
+    """Five decode steps (read state, output, update: [KIMI] 16.3) equal one five-token call."""
+    N, T = 3, 5
+    q, k, v, la, be, S0 = _rand(11, B=N, T=T, Hk=1, Hv=2, dk=4, dv=4)
+    o, sT = orc.gated_delta(q, k, v, la, be, S0)
+    sw = lambda x: np.swapaxes(x, 0, 1)
+    od, Sd = orc.decode_steps(sw(q), sw(k), sw(v), sw(la), sw(be), S0)
+    assert np.array_equal(sw(od), o) and np.array_equal(Sd, sT)
+
+
+# ---------------------------------------------------------------------------------------------
+# prologue / epilogue
+# ---------------------------------------------------------------------------------------------
+
+def pin_conv_equals_library_convolution(orc):
+    """Causal depthwise conv with 4 taps and zero history equals numpy's full convolution of each
+    channel with its reversed taps, cut to the first T outputs; then SiLU = x * expit(x)."""
+    rng = np.random.default_rng(12)
+    B, T, C = 2, 20, 5
+    x = rng.standard_normal((B, T, C))
+    w = rng.standard_normal((C, 4)) * 0.5
+    y = orc.causal_conv_silu(x, w)
+    for b in range(B):
+        for c in range(C):
+            pre = np.convolve(x[b, :, c], w[c, ::-1])[:T]
+            np.testing.assert_allclose(y[b, :, c], pre * expit(pre), rtol=1e-13, atol=1e-15)
+
+
+def pin_silu_textbook(orc):
+    """With taps (0, 0, 0, 1) the prologue is SiLU(x) = x sigmoid(x) ([BRK] 2.): SiLU(0) = 0,
+    SiLU(x) -> x for large x, -> 0 for very negative x."""
+    x = np.array([[-40.0, -3.0, -0.5, 0.0, 0.5, 3.0, 40.0]])[..., None]       # [1, 7, 1]
+    w = np.array([[0.0, 0.0, 0.0, 1.0]])
+    y = orc.causal_conv_silu(x, w)[0, :, 0]
+    np.testing.assert_allclose(y, x[0, :, 0] * expit(x[0, :, 0]), rtol=1e-14, atol=1e-300)
+    assert y[3] == 0.0 and abs(y[6] - 40.0) < 1e-12 and -1e-15 < y[0] < 0.0
+
+
+def pin_l2_unit_norm(orc):
+    """After x / sqrt(|x|^2 + eps): the norm is 1 when eps = 0 and sqrt(s / (s + eps)) else."""
+    rng = np.random.default_rng(13)
+    x = rng.standard_normal((50, 7)) * rng.uniform(0.01, 10, size=(50, 1))
+    y0 = orc.l2_normalize(x, 0.0)
+    np.testing.assert_allclose(np.linalg.norm(y0, axis=1), 1.0, rtol=1e-14)
+    eps = 0.37
+    s = (x ** 2).sum(axis=1)
+    y1 = orc.l2_normalize(x, eps)
+    np.testing.assert_allclose(np.linalg.norm(y1, axis=1), np.sqrt(s / (s + eps)), rtol=1e-13)
+    np.testing.assert_allclose(y1 / np.linalg.norm(y1, axis=1, keepdims=True),
+                               x / np.linalg.norm(x, axis=1, keepdims=True), rtol=1e-13)
+
+
+def pin_gated_rmsnorm_closed_form(orc):
+    """RMSNorm(o) w SiLU(z) ([BRK] 4., swish gate of [HYB]): with w = 1 and z = 50 (SiLU(50) = 50 in
+    fp64) the mean square of y/50 is ms / (ms + eps); the gain scales coordinates; z = 0 gives 0;
+    the gate is SiLU, so z = -1 multiplies by -sigmoid(-1)."""
+    rng = np.random.default_rng(14)
+    rows, d, eps = 40, 8, 0.05
+    o = rng.standard_normal((rows, d)) * rng.uniform(0.05, 3, size=(rows, 1))
+    ms = (o ** 2).mean(axis=1)
+    y = orc.gated_rmsnorm(o, np.full_like(o, 50.0), np.ones(d), eps)
+    np.testing.assert_allclose(((y / 50.0) ** 2).mean(axis=1), ms / (ms + eps), rtol=1e-13)
+    np.testing.assert_allclose(y / np.linalg.norm(y, axis=1, keepdims=True),
+                               o / np.linalg.norm(o, axis=1, keepdims=True), rtol=1e-13)
+    w = np.arange(1, d + 1, dtype=np.float64)
+    y2 = orc.gated_rmsnorm(o, np.full_like(o, 50.0), w, eps)
+    np.testing.assert_allclose(y2, y * w, rtol=1e-14)
+    assert np.all(orc.gated_rmsnorm(o, np.zeros_like(o), np.ones(d), eps) == 0.0)
+    ym = orc.gated_rmsnorm(o, np.full_like(o, -1.0), np.ones(d), eps)
+    np.testing.assert_allclose(ym, -expit(-1.0) * y / 50.0, rtol=1e-13)
+
+
+ALL_PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]

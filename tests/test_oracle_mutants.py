@@ -1,0 +1,69 @@
+"""Plant plausible mistakes in copies of the C oracle and check that the pins catch every one.
+
+Each mutant is one textual edit of ``oracle/gdn_oracle.c`` (a dropped term, a wrong sign, a wrong
+index or head mapping, a transposed read, a wrong tap order, a wrong normalisation), compiled into
+a temporary library on the CPU.  A mutant that passes all pins would mean the pins cannot tell that
+mistake from the method, so the test fails.
+"""
+import os
+
+import pytest
+
+import oracle
+import oracle_pins
+
+MUTANTS = {
+    "drop_beta_in_erase": ("x = S[(long)a * dk + c] - beta * Sk[a] * k[c];",
+                           "x = S[(long)a * dk + c] - Sk[a] * k[c];"),
+    "wrong_sign_erase": ("x = S[(long)a * dk + c] - beta * Sk[a] * k[c];",
+                         "x = S[(long)a * dk + c] + beta * Sk[a] * k[c];"),
+    "decay_also_on_write": ("S[(long)a * dk + c] = alpha * x + beta * v[a] * k[c];",
+                            "S[(long)a * dk + c] = alpha * (x + beta * v[a] * k[c]);"),
+    "drop_write_term": ("S[(long)a * dk + c] = alpha * x + beta * v[a] * k[c];",
+                        "S[(long)a * dk + c] = alpha * x;"),
+    "log_alpha_as_alpha": ("const double alpha = exp(J->log_alpha[(b * J->T + t) * Hv + h]);",
+                           "const double alpha = 1.0 + J->log_alpha[(b * J->T + t) * Hv + h];"),
+    "transposed_S0_read": ("J->S0[(((long)b * Hv + h) * dk + c) * dv + a]",
+                           "J->S0[(((long)b * Hv + h) * dv + a) * dk + c]"),
+    "transposed_S_T_write": ("J->S_T[(((long)b * Hv + h) * dk + c) * dv + a] =",
+                             "J->S_T[(((long)b * Hv + h) * dv + a) * dk + c] ="),
+    "gqa_interleaved_heads": ("const int hk = h / (Hv / Hk);", "const int hk = h % Hk;"),
+    "erase_with_query": ("for (int c = 0; c < dk; ++c) acc += S[(long)a * dk + c] * k[c];\n"
+                         "            Sk[a] = acc;",
+                         "for (int c = 0; c < dk; ++c) acc += S[(long)a * dk + c] * q[c];\n"
+                         "            Sk[a] = acc;"),
+    "output_reads_key": ("for (int c = 0; c < dk; ++c) acc += S[(long)a * dk + c] * q[c];\n"
+                         "            o[a] = J->scale * acc;",
+                         "for (int c = 0; c < dk; ++c) acc += S[(long)a * dk + c] * k[c];\n"
+                         "            o[a] = J->scale * acc;"),
+    "output_ignores_scale": ("o[a] = J->scale * acc;", "o[a] = acc;"),
+    "conv_taps_reversed": ("acc += w[c * 4 + j] * x[(b * T + s) * C + c];",
+                           "acc += w[c * 4 + (3 - j)] * x[(b * T + s) * C + c];"),
+    "conv_off_by_one": ("const long s = t - 3 + j;", "const long s = t - 4 + j;"),
+    "conv_no_silu": ("y[(b * T + t) * C + c] = acc * sigmoid(acc);",
+                     "y[(b * T + t) * C + c] = acc;"),
+    "l2_eps_outside_sqrt": ("const double inv = 1.0 / sqrt(ss + eps);",
+                            "const double inv = 1.0 / (sqrt(ss) + eps);"),
+    "rms_sum_not_mean": ("const double inv = 1.0 / sqrt(ss / d + eps);",
+                         "const double inv = 1.0 / sqrt(ss + eps);"),
+    "gate_sigmoid_not_silu": ("* (zz * sigmoid(zz));", "* sigmoid(zz);"),
+    "gain_ignored": ("y[r * d + i] = (o[r * d + i] * inv) * w[i] * (zz * sigmoid(zz));",
+                     "y[r * d + i] = (o[r * d + i] * inv) * (zz * sigmoid(zz));"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, tmp_path):
+    before, after = MUTANTS[name]
+    src = open(oracle.SOURCE).read()
+    assert src.count(before) == 1, f"mutation site of {name} not unique in the oracle source"
+    path = tmp_path / f"{name}.c"
+    path.write_text(src.replace(before, after))
+    lib = oracle.OracleLib(oracle.compile_source(str(path), str(tmp_path / f"{name}.so")))
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(lib)
+        except AssertionError:
+            caught.append(pin.__name__)
+    assert caught, f"no pin catches the mutant {name}"
