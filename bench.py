@@ -1,0 +1,537 @@
+#!/usr/bin/env python
+"""Benchmark of the gated delta rule library on B200 (one JSON line on stdout, rank 0).
+
+Headline: the chunked forward (gdn_chunk_fwd) on the prefill workload — B=4, T=2048, 16 key heads
+shared by 48 value heads, d_k = d_v = 128, chunk 64, bf16 q/k/v, fp32 gates and state, S0 = 0 —
+in tokens/s, with its fraction of the HBM/tensor roofline.  Secondary lines in the same JSON
+object: the decode step (256 sequences, GB/s of state traffic against the HBM peak), the long
+context forward (B1 T65536) and the fused 8:1 layer (B2 T8192 Hv128).
+
+Every step runs with its inputs resident in HBM; an L2 flush (a 256 MiB write, outside the timed
+events) separates timed steps.  Device time comes from CUDA events on the launching stream.  Under
+torchrun each rank runs an independent replica of the workload (the path shards over sequences and
+heads with no exchange), a barrier brackets the timed region and the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the only reference this build has) on the host cores,
+on a bounded sample of the same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import gdn_inputs as gi  # noqa: E402
+
+METRIC = "gated-delta fwd tokens/s & % roofline; decode-step state GB/s vs HBM peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "source": "fallback"}
+
+
+# ------------------------------------------------------------------------------------------------
+# algorithmic work (bytes and FLOPs per call)
+# ------------------------------------------------------------------------------------------------
+
+def fwd_bytes(w: gi.Workload, s0: bool, s_t: bool, layer: bool = False) -> int:
+    """HBM bytes a one-pass forward must move: inputs once, outputs once, nothing intermediate."""
+    s = 2 if w.dtype == "bf16" else 4
+    tok = w.B * w.T
+    per_tok = 2 * w.Hk * w.dk * s + w.Hv * w.dv * (s + s) + 8 * w.Hv
+    if layer:   # raw q, k, v and z in, y out; conv taps and the norm gain once
+        per_tok += w.Hv * w.dv * s
+    extra = (2 * w.Hk * w.dk + w.Hv * w.dv) * 16 + w.dv * 4 if layer else 0
+    return tok * per_tok + w.B * w.Hv * w.dk * w.dv * 4 * (int(s0) + int(s_t)) + extra
+
+
+def fwd_flops(w: gi.Workload) -> float:
+    """Dense work of the chunked form per token and value head: 6 dk dv (state products) +
+    2C(dk + 2 dv) (intra-chunk products) + 4 C dk / G (shared q.k and k.k) + C^2/3 (solve)."""
+    C, G = w.chunk, w.Hv // w.Hk
+    per = 6 * w.dk * w.dv + 2 * C * (w.dk + 2 * w.dv) + 4 * C * w.dk / G + C * C / 3
+    return float(w.B * w.T * w.Hv * per)
+
+
+def decode_bytes(w: gi.Workload) -> int:
+    s = 2 if w.dtype == "bf16" else 4
+    N = w.B
+    return 2 * N * w.Hv * w.dk * w.dv * 4 + N * (2 * w.Hk * w.dk * s + 2 * w.Hv * w.dv * s
+                                                 + 8 * w.Hv)
+
+
+# ------------------------------------------------------------------------------------------------
+# helpers
+# ------------------------------------------------------------------------------------------------
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_deltanet_linear_18_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f).get(kernel, {}).get(workload)
+    if not rec or rec.get("source_sha") != kernel_source_sha():
+        return None
+    return rec.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region (every 200 ms)."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+class Flusher:
+    """Writes 256 MiB (twice the 126 MB L2) so the next step starts with a cold L2."""
+
+    def __init__(self, dev):
+        self.buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        self.v = 0
+
+    def __call__(self):
+        self.v = (self.v + 1) & 0xFF
+        self.buf.fill_(self.v)
+
+
+def time_steps(fn, steps: int, warmup: int, flush: Flusher, launches_per_step: int):
+    """W untimed steps, then K steps each timed with CUDA events on the current stream with an L2
+    flush between them (outside the events).  Returns per-step milliseconds."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for a, b in evs:
+        flush()
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+# ------------------------------------------------------------------------------------------------
+# workloads
+# ------------------------------------------------------------------------------------------------
+
+def prefill_fn(gdn, d, w):
+    o = torch.empty_like(d["v"])
+    sT = torch.empty(w.B, w.Hv, w.dk, w.dv, device=d["v"].device, dtype=torch.float32)
+
+    def step():
+        gdn.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
+                      chunk=w.chunk, out=o, state_out=sT)
+    return step
+
+
+def to_dev(x, dev):
+    return {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+
+
+def bench_prefill_like(gdn, name, dev, steps, warmup, flush, peaks):
+    w = gi.WORKLOADS[name]
+    x = gi.make_inputs(w)
+    d = to_dev(x, dev)
+    ms = time_steps(prefill_fn(gdn, d, w), steps, warmup, flush, 1)
+    t = statistics.mean(ms) / 1e3
+    B = fwd_bytes(w, x["S0"] is not None, True)
+    F = fwd_flops(w)
+    t_roof = max(B / (peaks["hbm_gbs"] * 1e9), F / (peaks["bf16_tflops"] * 1e12))
+    return w, x, d, ms, {
+        "value": w.B * w.T / t, "unit": "tokens/s", "ms_per_step": t * 1e3,
+        "hbm_gbs": B / t / 1e9, "tflops": F / t / 1e12, "roofline_frac": t_roof / t,
+        "variant": gdn.chunk_fwd_variant(w.dk, w.dv, w.chunk, w.torch_dtype),
+        "workload": workload_name(w)}
+
+
+def workload_name(w: gi.Workload) -> str:
+    s = f"{w.name} B{w.B} T{w.T} Hk{w.Hk} Hv{w.Hv} dk{w.dk} dv{w.dv} chunk{w.chunk} {w.dtype}"
+    if w.s0_std:
+        s += f" S0~N(0,{w.s0_std})"
+    if w.steps:
+        s = f"{w.name} N{w.B} Hk{w.Hk} Hv{w.Hv} dk{w.dk} dv{w.dv} {w.dtype} {w.steps} steps"
+    return s
+
+
+def bench_decode(gdn, dev, warmup, flush, peaks):
+    w = gi.WORKLOADS["decode"]
+    x = gi.make_decode_inputs(w)
+    d = to_dev(x, dev)
+    S = d["S0"].clone()
+    o = torch.empty(w.B, w.Hv, w.dv, device=dev, dtype=w.torch_dtype)
+    state = {"s": 0}
+
+    def step():
+        s = state["s"] % w.steps
+        gdn.decode_step(d["q"][s], d["k"][s], d["v"][s], d["log_alpha"][s], d["beta"][s], S,
+                        out=o)
+        state["s"] += 1
+    # the state (805 MB) is far larger than L2: consecutive steps need no flush
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(w.steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    t = a.elapsed_time(b) / 1e3 / w.steps
+    by = decode_bytes(w)
+    return {"value": by / t / 1e9, "unit": "GB/s", "us_per_step": t * 1e6,
+            "tokens_per_s": w.B / t, "roofline_frac": by / t / 1e9 / peaks["hbm_gbs"],
+            "bytes_per_step": by, "workload": workload_name(w)}
+
+
+def bench_layer(gdn, dev, warmup, flush, peaks, steps=3):
+    w = gi.WORKLOADS["layer_8to1"]
+    x = gi.make_layer_inputs(w)
+    d = to_dev(x, dev)
+    y = torch.empty(w.B, w.T, w.Hv, w.dv, device=dev, dtype=w.torch_dtype)
+    ws_bytes = gdn.layer_workspace_bytes(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv, w.chunk,
+                                         w.torch_dtype)
+    ws = torch.empty(max(ws_bytes, 1), device=dev, dtype=torch.uint8)
+
+    def step():
+        gdn.layer_fwd(d["q_raw"], d["k_raw"], d["v_raw"], d["z"], d["conv_wq"], d["conv_wk"],
+                      d["conv_wv"], d["log_alpha"], d["beta"], d["S0"], d["norm_w"], Hk=w.Hk,
+                      Hv=w.Hv, dk=w.dk, dv=w.dv, chunk=w.chunk, workspace=ws)
+    ms = time_steps(step, steps, warmup, flush, 3)
+    t = statistics.mean(ms) / 1e3
+    B = fwd_bytes(w, False, True, layer=True)
+    F = fwd_flops(w)
+    t_roof = max(B / (peaks["hbm_gbs"] * 1e9), F / (peaks["bf16_tflops"] * 1e12))
+    return {"value": w.B * w.T / t, "unit": "tokens/s", "ms_per_step": t * 1e3,
+            "hbm_gbs": B / t / 1e9, "roofline_frac": t_roof / t, "workspace_bytes": ws_bytes,
+            "workload": workload_name(w)}
+
+
+def e2e_prefill(gdn, x, w, dev, steps):
+    """Same metric through the public call with pinned host buffers: H2D of the step's inputs,
+    the call, D2H of o and S_T, all inside the timed region."""
+    names = ["q", "k", "v", "log_alpha", "beta"]
+    host = {n: x[n].pin_memory() for n in names}
+    dbuf = {n: torch.empty_like(x[n], device=dev) for n in names}
+    o_h = torch.empty(w.B, w.T, w.Hv, w.dv, dtype=w.torch_dtype).pin_memory()
+    s_h = torch.empty(w.B, w.Hv, w.dk, w.dv, dtype=torch.float32).pin_memory()
+    o_d = torch.empty(o_h.shape, dtype=o_h.dtype, device=dev)
+    s_d = torch.empty(s_h.shape, dtype=s_h.dtype, device=dev)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o_h.numel() * o_h.element_size() + s_h.numel() * s_h.element_size()
+
+    def step():
+        for n in names:
+            dbuf[n].copy_(host[n], non_blocking=True)
+        gdn.chunk_fwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["log_alpha"], dbuf["beta"], None,
+                      chunk=w.chunk, out=o_d, state_out=s_d)
+        o_h.copy_(o_d, non_blocking=True)
+        s_h.copy_(s_d, non_blocking=True)
+    step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    t = a.elapsed_time(b) / 1e3 / steps
+    return {"value": w.B * w.T / t, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h}
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle baseline
+# ------------------------------------------------------------------------------------------------
+
+def oracle_sample_rate(x, w, target_s: float):
+    """Tokens/s of the fp64 oracle on this host, on a bounded sample: the first `nh` value heads
+    of batch 0 over all T tokens, nh calibrated to take about `target_s` seconds; scaled to the
+    full workload's tokens by the fraction of (batch, head) recurrences processed."""
+    import oracle
+    threads = oracle.default_threads()
+
+    def run(nh):
+        G = w.Hv // w.Hk
+        nk = (nh + G - 1) // G
+        t0 = time.perf_counter()
+        oracle.gated_delta(x["q"][:1, :, :nk], x["k"][:1, :, :nk], x["v"][:1, :, :nh],
+                           x["log_alpha"][:1, :, :nh], x["beta"][:1, :, :nh], None,
+                           threads=threads)
+        return time.perf_counter() - t0
+    nh = min(w.Hv, threads)
+    t = run(nh)
+    per_round = t
+    rounds = max(1, min(int(target_s / max(per_round, 1e-3)), (w.B * w.Hv) // max(nh, 1)))
+    heads = min(w.Hv, nh * rounds)
+    t = run(heads)
+    frac = heads / (w.B * w.Hv)
+    return {"value": w.B * w.T * frac / t, "unit": "tokens/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"fp64 token-by-token recurrence on batch 0, value heads 0..{heads - 1} of "
+                      f"{workload_name(w)} ({heads} of {w.B * w.Hv} head recurrences, "
+                      f"{t:.1f} s); tokens/s scaled by that fraction",
+            "seconds": t}
+
+
+def cpu_name():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+# ------------------------------------------------------------------------------------------------
+# main
+# ------------------------------------------------------------------------------------------------
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the fp64 oracle on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    w = gi.WORKLOADS["prefill"]
+    x = gi.make_inputs(w)
+    import oracle
+    threads = oracle.default_threads()
+    G = w.Hv // w.Hk
+    nh = min(w.Hv, max(G, threads))          # one bounded sample per step: nh heads of batch 0
+    nk = (nh + G - 1) // G
+
+    def step():
+        oracle.gated_delta(x["q"][:1, :, :nk], x["k"][:1, :, :nk], x["v"][:1, :, :nh],
+                           x["log_alpha"][:1, :, :nh], x["beta"][:1, :, :nh], None,
+                           threads=threads)
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    t = (time.perf_counter() - t0) / args.steps
+    frac = nh / (w.B * w.Hv)
+    value = w.B * w.T * frac / t
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": workload_name(w), "global_batch": w.B, "seq_len": w.T,
+                       "parallelism": "host threads over (batch, head) recurrences"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
+                             "kind": "oracle", "cpu": cpu_name(),
+                             "sample": f"per step: value heads 0..{nh - 1} of batch 0 over all "
+                                       f"{w.T} tokens ({nh} of {w.B * w.Hv} recurrences); "
+                                       f"tokens/s scaled by that fraction"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the decode / long-context / layer lines")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world, rank, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    import gated_deltanet_linear_18_b200 as gdn
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    gdn.lib()
+    peaks = load_peaks()
+    flush = Flusher(dev)
+
+    w = gi.WORKLOADS["prefill"]
+    x = gi.make_inputs(w)
+    d = to_dev(x, dev)
+    step = prefill_fn(gdn, d, w)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        ms = time_steps(step, args.steps, 0, flush, 1)
+    torch.cuda.synchronize()
+    t_step = sum(ms) / len(ms) / 1e3
+    if world > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([t_step], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_step = float(tt.item())
+        dist.barrier()
+    gdn.check_error(dev)
+
+    B = fwd_bytes(w, False, True)
+    F = fwd_flops(w)
+    t_hbm = B / (peaks["hbm_gbs"] * 1e9)
+    t_ten = F / (peaks["bf16_tflops"] * 1e12)
+    hbm_bound = t_hbm >= t_ten
+    variant = gdn.chunk_fwd_variant(w.dk, w.dv, w.chunk, w.torch_dtype)
+    kname = "gdn_chunk_fwd_tc" if variant == "tcgen05" else "chunk_fwd_simt_kernel"
+    roof = {"bound": "hbm" if hbm_bound else "tensor",
+            "achieved": (B / t_step / 1e9) if hbm_bound else (F / t_step / 1e12),
+            "peak": peaks["hbm_gbs"] if hbm_bound else peaks["bf16_tflops"],
+            "unit": "GB/s" if hbm_bound else "TFLOP/s",
+            "traffic": recorded_traffic(kname, "prefill"),
+            "kernel": kname, "algorithmic_bytes": B, "algorithmic_flops": F,
+            "peak_source": peaks.get("source", "measured") + (" burst" if not hbm_bound else ""),
+            "other_bound_frac": (t_ten / t_step) if hbm_bound else (t_hbm / t_step)}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+
+    line = {"metric": METRIC, "value": w.B * w.T * world / t_step, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": workload_name(w), "global_batch": w.B * world,
+                       "seq_len": w.T, "parallelism": f"replicas x{world} (no exchange)",
+                       "kernel_variant": variant,
+                       "l2": "256 MiB write between timed steps (outside the events)"},
+            "roofline": roof, "gpu_launches": args.steps * 1,
+            "clocks": clocks.summary()}
+
+    e2e = e2e_prefill(gdn, x, w, dev, steps=max(3, min(args.steps, 10)))
+    if world > 1:   # whole-job e2e: every rank ran its replica; the slowest one sets the time
+        import torch.distributed as dist
+        tt = torch.tensor([w.B * w.T / e2e["value"]], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e["value"] = w.B * w.T * world / float(tt.item())
+    line["e2e"] = e2e
+    if rank == 0:
+        if not args.no_secondary:
+            sec = {}
+            sec["decode"] = bench_decode(gdn, dev, args.warmup, flush, peaks)
+            del d
+            torch.cuda.empty_cache()
+            _, xl, dl, _, sec["long_context"] = bench_prefill_like(
+                gdn, "long_context", dev, 3, 3, flush, peaks)
+            del xl, dl
+            torch.cuda.empty_cache()
+            sec["layer_8to1"] = bench_layer(gdn, dev, 3, flush, peaks)
+            line["secondary"] = sec
+        if not args.no_cpu_baseline and world == 1:
+            cb = oracle_sample_rate(x, w, target_s=10.0)
+            cb["cpu"] = cpu_name()
+            line["cpu_baseline"] = cb
+        line["peaks"] = {k: peaks.get(k) for k in ("hbm_gbs", "bf16_tflops",
+                                                   "bf16_tflops_sustained", "source")}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,234 @@
+"""Python binding of ``libgdn.so``, the gated delta rule (Gated DeltaNet) library for B200.
+
+Argument marshalling only: every step of the computation runs in the library's CUDA kernels,
+behind the C ABI declared in ``include/gdn.h``.  PyTorch supplies device memory and the current
+stream.  There is no fallback: if the library is missing or a call fails, these functions raise.
+
+Layouts (contiguous, last index fastest): q, k [B,T,Hk,dk]; v, o [B,T,Hv,dv]; log_alpha, beta
+[B,T,Hv] fp32; states [B,Hv,dk,dv] fp32 holding S transposed (d_v contiguous).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = ["GdnError", "lib", "library_path", "chunk_fwd", "chunk_fwd_variant", "decode_step",
+           "prologue", "out_norm", "layer_fwd", "layer_workspace_bytes", "check_error",
+           "STATUS", "VARIANTS"]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libgdn.so")
+_lib = None
+
+STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED", 3: "GDN_ERR_CUDA",
+          4: "GDN_ERR_TIMEOUT"}
+VARIANTS = {"auto": 0, "simt": 1, "tcgen05": 2}
+_DTYPES = {torch.float32: 0, torch.bfloat16: 1}
+
+
+class GdnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} returned {STATUS.get(status, status)}")
+        self.status = status
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """Load libgdn.so (built in-tree by ``__graft_entry__.build()``); raise if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with __graft_entry__.build()")
+        L = ctypes.CDLL(_LIB_PATH)
+        P, I, F, LL, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_longlong, \
+            ctypes.c_size_t
+        L.gdn_status_string.argtypes = [I]
+        L.gdn_status_string.restype = ctypes.c_char_p
+        L.gdn_version.argtypes = []
+        L.gdn_version.restype = I
+        L.gdn_check_error.argtypes = [P]
+        L.gdn_check_error.restype = I
+        L.gdn_chunk_fwd.argtypes = [P] * 8 + [I] * 7 + [F, I, P]
+        L.gdn_chunk_fwd.restype = I
+        L.gdn_chunk_fwd_ex.argtypes = [P] * 8 + [I] * 7 + [F, I, I, P]
+        L.gdn_chunk_fwd_ex.restype = I
+        L.gdn_chunk_fwd_variant.argtypes = [I, I, I, I]
+        L.gdn_chunk_fwd_variant.restype = I
+        L.gdn_decode_step.argtypes = [P] * 7 + [I] * 5 + [F, I, P]
+        L.gdn_decode_step.restype = I
+        L.gdn_prologue.argtypes = [P] * 9 + [I] * 6 + [F, I, P]
+        L.gdn_prologue.restype = I
+        L.gdn_out_norm.argtypes = [P, P, P, P, LL, I, F, I, P]
+        L.gdn_out_norm.restype = I
+        L.gdn_layer_fwd.argtypes = [P] * 14 + [SZ] + [I] * 7 + [F, F, F, I, P]
+        L.gdn_layer_fwd.restype = I
+        L.gdn_layer_workspace_bytes.argtypes = [I] * 7 + [I]
+        L.gdn_layer_workspace_bytes.restype = SZ
+        _lib = L
+    return _lib
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(dev: torch.device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise GdnError(fn, status)
+
+
+def _dev(*ts: Optional[torch.Tensor]) -> torch.device:
+    dev = None
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors")
+        if not t.is_contiguous():
+            raise ValueError("all tensors must be contiguous")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError("all tensors must be on one device")
+    return dev
+
+
+def _f32(*ts):
+    for t in ts:
+        if t is not None and t.dtype != torch.float32:
+            raise ValueError("gates, states and weights must be float32")
+
+
+def _io_dtype(t: torch.Tensor) -> int:
+    if t.dtype not in _DTYPES:
+        raise ValueError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+    return _DTYPES[t.dtype]
+
+
+def chunk_fwd_variant(dk: int, dv: int, chunk: int, dtype: torch.dtype) -> str:
+    """Which kernel family ``chunk_fwd`` runs for these sizes: 'simt' or 'tcgen05'."""
+    v = lib().gdn_chunk_fwd_variant(dk, dv, chunk, _DTYPES[dtype])
+    return {1: "simt", 2: "tcgen05"}[v]
+
+
+def chunk_fwd(q, k, v, log_alpha, beta, S0=None, *, chunk: int = 64, scale: float = 1.0,
+              out: Optional[torch.Tensor] = None, state_out: Optional[torch.Tensor] = None,
+              want_state: bool = True, variant: str = "auto"
+              ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunked prefill forward: returns (o [B,T,Hv,dv], S_T [B,Hv,dk,dv] or None)."""
+    B, T, Hk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    if k.shape != q.shape or v.shape[:2] != (B, T) or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v shapes/dtypes disagree")
+    if log_alpha.shape != (B, T, Hv) or beta.shape != (B, T, Hv):
+        raise ValueError("gates must be [B, T, Hv]")
+    _f32(log_alpha, beta, S0)
+    o = torch.empty_like(v) if out is None else out
+    sT = None
+    if want_state:
+        sT = torch.empty(B, Hv, dk, dv, device=q.device, dtype=torch.float32) \
+            if state_out is None else state_out
+    dev = _dev(q, k, v, log_alpha, beta, S0, o, sT)
+    with torch.cuda.device(dev):
+        st = lib().gdn_chunk_fwd_ex(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(S0), _p(o),
+                                    _p(sT), B, T, Hk, Hv, dk, dv, chunk, float(scale),
+                                    _io_dtype(q), VARIANTS[variant], _stream(dev))
+    _check("gdn_chunk_fwd", st)
+    return o, sT
+
+
+def decode_step(q, k, v, log_alpha, beta, S, *, scale: float = 1.0,
+                out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One decode step: q,k [N,Hk,dk]; v [N,Hv,dv]; gates [N,Hv]; S [N,Hv,dk,dv] updated in
+    place.  Returns o [N,Hv,dv]."""
+    N, Hk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    if k.shape != q.shape or v.shape[0] != N or S.shape != (N, Hv, dk, dv):
+        raise ValueError("decode shapes disagree")
+    _f32(log_alpha, beta, S)
+    o = torch.empty_like(v) if out is None else out
+    dev = _dev(q, k, v, log_alpha, beta, S, o)
+    with torch.cuda.device(dev):
+        st = lib().gdn_decode_step(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(S), _p(o),
+                                   N, Hk, Hv, dk, dv, float(scale), _io_dtype(q), _stream(dev))
+    _check("gdn_decode_step", st)
+    return o
+
+
+def prologue(q_raw, k_raw, v_raw, wq, wk, wv, Hk: int, Hv: int, dk: int, dv: int,
+             l2_eps: float = 1e-6):
+    """Conv(4 taps) + SiLU + L2-normalisation of q/k heads.  Returns (q, k, v) shaped
+    [B,T,Hk,dk], [B,T,Hk,dk], [B,T,Hv,dv]."""
+    B, T = q_raw.shape[:2]
+    _f32(wq, wk, wv)
+    q = torch.empty(B, T, Hk, dk, device=q_raw.device, dtype=q_raw.dtype)
+    k = torch.empty_like(q)
+    v = torch.empty(B, T, Hv, dv, device=q_raw.device, dtype=q_raw.dtype)
+    dev = _dev(q_raw, k_raw, v_raw, wq, wk, wv, q, k, v)
+    with torch.cuda.device(dev):
+        st = lib().gdn_prologue(_p(q_raw), _p(k_raw), _p(v_raw), _p(wq), _p(wk), _p(wv), _p(q),
+                                _p(k), _p(v), B, T, Hk, Hv, dk, dv, float(l2_eps),
+                                _io_dtype(q_raw), _stream(dev))
+    _check("gdn_prologue", st)
+    return q, k, v
+
+
+def out_norm(o, z, w, eps: float = 1e-5) -> torch.Tensor:
+    """y = RMSNorm(o) * w * SiLU(z) over the last dimension."""
+    if z.shape != o.shape or z.dtype != o.dtype:
+        raise ValueError("o and z must agree")
+    _f32(w)
+    dv = o.shape[-1]
+    y = torch.empty_like(o)
+    dev = _dev(o, z, w, y)
+    with torch.cuda.device(dev):
+        st = lib().gdn_out_norm(_p(o), _p(z), _p(w), _p(y), o.numel() // dv, dv, float(eps),
+                                _io_dtype(o), _stream(dev))
+    _check("gdn_out_norm", st)
+    return y
+
+
+def layer_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, dtype) -> int:
+    return int(lib().gdn_layer_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, _DTYPES[dtype]))
+
+
+def layer_fwd(q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, *, Hk: int,
+              Hv: int, dk: int, dv: int, chunk: int = 64, scale: float = 1.0,
+              l2_eps: float = 1e-6, norm_eps: float = 1e-5, want_state: bool = True,
+              workspace: Optional[torch.Tensor] = None):
+    """Whole layer between the projections: returns (y [B,T,Hv,dv], S_T or None)."""
+    B, T = q_raw.shape[:2]
+    _f32(wq, wk, wv, log_alpha, beta, S0, norm_w)
+    y = torch.empty(B, T, Hv, dv, device=q_raw.device, dtype=q_raw.dtype)
+    sT = torch.empty(B, Hv, dk, dv, device=q_raw.device, dtype=torch.float32) \
+        if want_state else None
+    need = layer_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, q_raw.dtype)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, device=q_raw.device, dtype=torch.uint8)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    dev = _dev(q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, y, sT)
+    with torch.cuda.device(dev):
+        st = lib().gdn_layer_fwd(_p(q_raw), _p(k_raw), _p(v_raw), _p(z), _p(wq), _p(wk), _p(wv),
+                                 _p(log_alpha), _p(beta), _p(S0), _p(norm_w), _p(y), _p(sT),
+                                 _p(workspace), wbytes, B, T, Hk, Hv, dk, dv, chunk,
+                                 float(scale), float(l2_eps), float(norm_eps),
+                                 _io_dtype(q_raw), _stream(dev))
+    _check("gdn_layer_fwd", st)
+    return y, sT
+
+
+def check_error(device: Optional[torch.device] = None):
+    """Synchronise the current stream and raise if a kernel recorded a timed-out wait."""
+    dev = device or torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        _check("gdn_check_error", lib().gdn_check_error(_stream(dev)))

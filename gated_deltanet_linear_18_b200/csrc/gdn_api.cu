@@ -1,0 +1,307 @@
+// C ABI of the gated delta rule library (declared in include/gdn.h): argument validation,
+// kernel selection and launches.  All kernels of the library are compiled in this one unit.
+#include <stdint.h>
+#include <string.h>
+
+#include "gdn.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "elementwise.cuh"
+#include "simt_chunk.cuh"
+#include "tc_chunk.cuh"
+
+using namespace gdn;
+
+namespace {
+
+constexpr int kVersion = 10000;   // 1.0.0
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool opt_aligned16(const void* p) { return p == nullptr || aligned16(p); }
+bool supported_dim(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+bool supported_chunk(int c) { return c == 16 || c == 32 || c == 64; }
+bool valid_dtype(gdn_dtype t) { return t == GDN_F32 || t == GDN_BF16; }
+
+gdn_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------------------------
+// SIMT chunked forward dispatch: DK in {16,32,64,128} x C in {16,32,64}, dv tiles of 16 columns.
+// ---------------------------------------------------------------------------------------------
+template <int DK, int C, typename Tio>
+gdn_status simt_launch(const void* q, const void* k, const void* v, const float* la,
+                       const float* be, const float* S0, void* o, float* S_T, int B, int T,
+                       int Hk, int Hv, int dv, float scale, cudaStream_t st) {
+  constexpr int DVT = 16;
+  auto kern = chunk_fwd_simt_kernel<DK, DVT, C, Tio>;
+  const size_t smem = simt_chunk_smem_floats<DK, DVT, C>() * sizeof(float);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return GDN_ERR_CUDA;
+  dim3 grid(dv / DVT, Hv, B);
+  kern<<<grid, kSimtThreads, smem, st>>>(
+      static_cast<const Tio*>(q), static_cast<const Tio*>(k), static_cast<const Tio*>(v), la,
+      be, S0, static_cast<Tio*>(o), S_T, T, Hk, Hv, dv, scale);
+  return launch_status();
+}
+
+template <typename Tio>
+gdn_status simt_dispatch(int dk, int chunk, const void* q, const void* k, const void* v,
+                         const float* la, const float* be, const float* S0, void* o, float* S_T,
+                         int B, int T, int Hk, int Hv, int dv, float scale, cudaStream_t st) {
+#define GDN_SIMT_CASE(DK_, C_)                                                             \
+  if (dk == DK_ && chunk == C_)                                                            \
+    return simt_launch<DK_, C_, Tio>(q, k, v, la, be, S0, o, S_T, B, T, Hk, Hv, dv, scale, st);
+  GDN_SIMT_CASE(16, 16) GDN_SIMT_CASE(16, 32) GDN_SIMT_CASE(16, 64)
+  GDN_SIMT_CASE(32, 16) GDN_SIMT_CASE(32, 32) GDN_SIMT_CASE(32, 64)
+  GDN_SIMT_CASE(64, 16) GDN_SIMT_CASE(64, 32) GDN_SIMT_CASE(64, 64)
+  GDN_SIMT_CASE(128, 16) GDN_SIMT_CASE(128, 32) GDN_SIMT_CASE(128, 64)
+#undef GDN_SIMT_CASE
+  return GDN_ERR_UNSUPPORTED;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Decode dispatch over (dk, dv)
+// ---------------------------------------------------------------------------------------------
+template <int DK, int DV, typename Tio>
+gdn_status decode_launch(const void* q, const void* k, const void* v, const float* la,
+                         const float* be, float* S, void* o, int N, int Hk, int Hv, float scale,
+                         cudaStream_t st) {
+  using Sh = DecodeShape<DK, DV>;
+  decode_step_kernel<DK, DV, Tio><<<(unsigned)((long)N * Hv), Sh::NT, 0, st>>>(
+      static_cast<const Tio*>(q), static_cast<const Tio*>(k), static_cast<const Tio*>(v), la,
+      be, S, static_cast<Tio*>(o), Hk, Hv, scale);
+  return launch_status();
+}
+
+template <typename Tio, int DK>
+gdn_status decode_dispatch_dv(int dv, const void* q, const void* k, const void* v,
+                              const float* la, const float* be, float* S, void* o, int N, int Hk,
+                              int Hv, float scale, cudaStream_t st) {
+  switch (dv) {
+    case 16: return decode_launch<DK, 16, Tio>(q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
+    case 32: return decode_launch<DK, 32, Tio>(q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
+    case 64: return decode_launch<DK, 64, Tio>(q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
+    case 128: return decode_launch<DK, 128, Tio>(q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
+  }
+  return GDN_ERR_UNSUPPORTED;
+}
+
+template <typename Tio>
+gdn_status decode_dispatch(int dk, int dv, const void* q, const void* k, const void* v,
+                           const float* la, const float* be, float* S, void* o, int N, int Hk,
+                           int Hv, float scale, cudaStream_t st) {
+  switch (dk) {
+    case 16: return decode_dispatch_dv<Tio, 16>(dv, q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
+    case 32: return decode_dispatch_dv<Tio, 32>(dv, q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
+    case 64: return decode_dispatch_dv<Tio, 64>(dv, q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
+    case 128:
+      return decode_dispatch_dv<Tio, 128>(dv, q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
+  }
+  return GDN_ERR_UNSUPPORTED;
+}
+
+gdn_status validate_heads(int Hk, int Hv, int dk, int dv) {
+  if (Hk <= 0 || Hv <= 0 || dk <= 0 || dv <= 0 || Hv % Hk != 0) return GDN_ERR_INVALID_ARG;
+  if (Hv > 65535) return GDN_ERR_UNSUPPORTED;
+  if (!supported_dim(dk) || !supported_dim(dv)) return GDN_ERR_UNSUPPORTED;
+  return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gdn_status_string(gdn_status s) {
+  switch (s) {
+    case GDN_OK: return "GDN_OK";
+    case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG";
+    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+    case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+    case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+  }
+  return "GDN_ERR_UNKNOWN";
+}
+
+int gdn_version(void) { return kVersion; }
+
+gdn_status gdn_check_error(gdn_stream_t stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return GDN_ERR_CUDA;
+  unsigned int word = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return GDN_ERR_CUDA;
+  if (word != 0 && cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  return (word & kErrTimeout) ? GDN_ERR_TIMEOUT : GDN_OK;
+}
+
+gdn_variant gdn_chunk_fwd_variant(int dk, int dv, int chunk, gdn_dtype dtype) {
+  if (tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16)) return GDN_VARIANT_TCGEN05;
+  return GDN_VARIANT_SIMT;
+}
+
+gdn_status gdn_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* log_alpha,
+                            const float* beta, const float* S0, void* o, float* S_T, int B,
+                            int T, int Hk, int Hv, int dk, int dv, int chunk, float scale,
+                            gdn_dtype dtype, gdn_variant variant, gdn_stream_t stream) {
+  if (B < 0 || T < 0 || !valid_dtype(dtype)) return GDN_ERR_INVALID_ARG;
+  if (variant != GDN_VARIANT_AUTO && variant != GDN_VARIANT_SIMT &&
+      variant != GDN_VARIANT_TCGEN05)
+    return GDN_ERR_INVALID_ARG;
+  gdn_status s = validate_heads(Hk, Hv, dk, dv);
+  if (s != GDN_OK) return s;
+  if (chunk <= 0) return GDN_ERR_INVALID_ARG;
+  if (!supported_chunk(chunk)) return GDN_ERR_UNSUPPORTED;
+  if (B > 65535) return GDN_ERR_UNSUPPORTED;
+  const bool work = (long)B * T > 0;
+  if (work && (!q || !k || !v || !log_alpha || !beta || !o)) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(q) && q) return GDN_ERR_INVALID_ARG;
+  if (!opt_aligned16(k) || !opt_aligned16(v) || !opt_aligned16(o) ||
+      !opt_aligned16(log_alpha) || !opt_aligned16(beta) || !opt_aligned16(S0) ||
+      !opt_aligned16(S_T))
+    return GDN_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (B == 0) return GDN_OK;
+  if (T == 0) {     // no token: the state is handed through unchanged (or is the zero state)
+    if (!S_T) return GDN_OK;
+    const size_t bytes = (size_t)B * Hv * dk * dv * sizeof(float);
+    cudaError_t e = S0 ? cudaMemcpyAsync(S_T, S0, bytes, cudaMemcpyDeviceToDevice, st)
+                       : cudaMemsetAsync(S_T, 0, bytes, st);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+  }
+  const bool tc_ok = tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16);
+  if (variant == GDN_VARIANT_TCGEN05 && !tc_ok) return GDN_ERR_UNSUPPORTED;
+  if (tc_ok && variant != GDN_VARIANT_SIMT)
+    return tc_chunk_launch(q, k, v, log_alpha, beta, S0, o, S_T, B, T, Hk, Hv, scale, st);
+  if (dtype == GDN_F32)
+    return simt_dispatch<float>(dk, chunk, q, k, v, log_alpha, beta, S0, o, S_T, B, T, Hk, Hv,
+                                dv, scale, st);
+  return simt_dispatch<__nv_bfloat16>(dk, chunk, q, k, v, log_alpha, beta, S0, o, S_T, B, T, Hk,
+                                      Hv, dv, scale, st);
+}
+
+gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* log_alpha,
+                         const float* beta, const float* S0, void* o, float* S_T, int B, int T,
+                         int Hk, int Hv, int dk, int dv, int chunk, float scale,
+                         gdn_dtype dtype, gdn_stream_t stream) {
+  return gdn_chunk_fwd_ex(q, k, v, log_alpha, beta, S0, o, S_T, B, T, Hk, Hv, dk, dv, chunk,
+                          scale, dtype, GDN_VARIANT_AUTO, stream);
+}
+
+gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const float* log_alpha,
+                           const float* beta, float* S, void* o, int N, int Hk, int Hv, int dk,
+                           int dv, float scale, gdn_dtype dtype, gdn_stream_t stream) {
+  if (N < 0 || !valid_dtype(dtype)) return GDN_ERR_INVALID_ARG;
+  gdn_status s = validate_heads(Hk, Hv, dk, dv);
+  if (s != GDN_OK) return s;
+  if (N == 0) return GDN_OK;
+  if (!q || !k || !v || !log_alpha || !beta || !S || !o) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha) ||
+      !aligned16(beta) || !aligned16(S) || !aligned16(o))
+    return GDN_ERR_INVALID_ARG;
+  if ((long)N * Hv > 0x7fffffffL) return GDN_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == GDN_F32)
+    return decode_dispatch<float>(dk, dv, q, k, v, log_alpha, beta, S, o, N, Hk, Hv, scale, st);
+  return decode_dispatch<__nv_bfloat16>(dk, dv, q, k, v, log_alpha, beta, S, o, N, Hk, Hv, scale,
+                                        st);
+}
+
+gdn_status gdn_prologue(const void* q_raw, const void* k_raw, const void* v_raw, const float* wq,
+                        const float* wk, const float* wv, void* q, void* k, void* v, int B, int T,
+                        int Hk, int Hv, int dk, int dv, float l2_eps, gdn_dtype dtype,
+                        gdn_stream_t stream) {
+  if (B < 0 || T < 0 || !valid_dtype(dtype) || !(l2_eps >= 0.f)) return GDN_ERR_INVALID_ARG;
+  gdn_status s = validate_heads(Hk, Hv, dk, dv);
+  if (s != GDN_OK) return s;
+  if ((long)B * T == 0) return GDN_OK;
+  if (B > 65535 || 2L * Hk + Hv > 65535) return GDN_ERR_UNSUPPORTED;
+  const void* ptrs[] = {q_raw, k_raw, v_raw, wq, wk, wv, q, k, v};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return GDN_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  dim3 grid((T + kPrologueTokens - 1) / kPrologueTokens, 2 * Hk + Hv, B);
+  if (dtype == GDN_F32)
+    prologue_kernel<float><<<grid, 128, 0, st>>>(
+        (const float*)q_raw, (const float*)k_raw, (const float*)v_raw, wq, wk, wv, (float*)q,
+        (float*)k, (float*)v, T, Hk, Hv, dk, dv, l2_eps);
+  else
+    prologue_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(
+        (const __nv_bfloat16*)q_raw, (const __nv_bfloat16*)k_raw, (const __nv_bfloat16*)v_raw,
+        wq, wk, wv, (__nv_bfloat16*)q, (__nv_bfloat16*)k, (__nv_bfloat16*)v, T, Hk, Hv, dk, dv,
+        l2_eps);
+  return launch_status();
+}
+
+gdn_status gdn_out_norm(const void* o, const void* z, const float* w, void* y, long long rows,
+                        int dv, float eps, gdn_dtype dtype, gdn_stream_t stream) {
+  if (rows < 0 || !valid_dtype(dtype) || dv <= 0 || !(eps >= 0.f)) return GDN_ERR_INVALID_ARG;
+  if (!supported_dim(dv)) return GDN_ERR_UNSUPPORTED;
+  if (rows == 0) return GDN_OK;
+  if (!o || !z || !w || !y || !aligned16(o) || !aligned16(z) || !aligned16(w) || !aligned16(y))
+    return GDN_ERR_INVALID_ARG;
+  const long long blocks = (rows + 7) / 8;
+  if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == GDN_F32)
+    out_norm_kernel<float><<<(unsigned)blocks, 256, 0, st>>>((const float*)o, (const float*)z, w,
+                                                             (float*)y, rows, dv, eps);
+  else
+    out_norm_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
+        (const __nv_bfloat16*)o, (const __nv_bfloat16*)z, w, (__nv_bfloat16*)y, rows, dv, eps);
+  return launch_status();
+}
+
+size_t gdn_layer_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, int chunk,
+                                 gdn_dtype dtype) {
+  (void)chunk;
+  if (B <= 0 || T <= 0 || Hk <= 0 || Hv <= 0 || dk <= 0 || dv <= 0) return 0;
+  const size_t el = dtype == GDN_F32 ? 4 : 2;
+  const size_t tok = (size_t)B * T;
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  // normalised q, k, convolved v and the pre-norm output o
+  return 2 * up(tok * Hk * dk * el) + 2 * up(tok * Hv * dv * el);
+}
+
+gdn_status gdn_layer_fwd(const void* q_raw, const void* k_raw, const void* v_raw, const void* z,
+                         const float* wq, const float* wk, const float* wv,
+                         const float* log_alpha, const float* beta, const float* S0,
+                         const float* norm_w, void* y, float* S_T, void* workspace,
+                         size_t workspace_bytes, int B, int T, int Hk, int Hv, int dk, int dv,
+                         int chunk, float scale, float l2_eps, float norm_eps, gdn_dtype dtype,
+                         gdn_stream_t stream) {
+  if (B < 0 || T < 0 || !valid_dtype(dtype)) return GDN_ERR_INVALID_ARG;
+  gdn_status s = validate_heads(Hk, Hv, dk, dv);
+  if (s != GDN_OK) return s;
+  if (chunk <= 0) return GDN_ERR_INVALID_ARG;
+  if (!supported_chunk(chunk)) return GDN_ERR_UNSUPPORTED;
+  const size_t need = gdn_layer_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, dtype);
+  if ((long)B * T > 0) {
+    if (!z || !norm_w || !y || !aligned16(z) || !aligned16(norm_w) || !aligned16(y))
+      return GDN_ERR_INVALID_ARG;
+    if (need > 0 && (!workspace || workspace_bytes < need ||
+                     (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0))
+      return GDN_ERR_INVALID_ARG;
+  }
+  if ((long)B * T == 0)
+    return gdn_chunk_fwd(nullptr, nullptr, nullptr, nullptr, nullptr, S0, nullptr, S_T, B, T, Hk,
+                         Hv, dk, dv, chunk, scale, dtype, stream);
+  const size_t el = dtype == GDN_F32 ? 4 : 2;
+  const size_t tok = (size_t)B * T;
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  char* ws = static_cast<char*>(workspace);
+  void* qn = ws;
+  void* kn = ws + up(tok * Hk * dk * el);
+  void* vc = ws + 2 * up(tok * Hk * dk * el);
+  void* o = ws + 2 * up(tok * Hk * dk * el) + up(tok * Hv * dv * el);
+  s = gdn_prologue(q_raw, k_raw, v_raw, wq, wk, wv, qn, kn, vc, B, T, Hk, Hv, dk, dv, l2_eps,
+                   dtype, stream);
+  if (s != GDN_OK) return s;
+  s = gdn_chunk_fwd(qn, kn, vc, log_alpha, beta, S0, o, S_T, B, T, Hk, Hv, dk, dv, chunk, scale,
+                    dtype, stream);
+  if (s != GDN_OK) return s;
+  return gdn_out_norm(o, z, norm_w, y, (long long)tok * Hv, dv, norm_eps, dtype, stream);
+}
+
+}  // extern "C"

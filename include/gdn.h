@@ -1,0 +1,179 @@
+/*
+ * gdn.h — C ABI of the gated delta rule (Gated DeltaNet) library for NVIDIA B200 (sm_100a).
+ *
+ * What it computes.  Per value head, a d_v x d_k fp32 state S evolves token by token as
+ *
+ *      S_t = alpha_t * S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,    o_t = scale * S_t q_t
+ *
+ * ("L'attention hybride", section "La récurrence": alpha_t in ]0,1[ fades the whole state,
+ * beta_t in ]0,1[ replaces the association bound to k_t, I is the identity; the equation itself
+ * did not survive the page's extraction and is the gated delta rule written with those symbols).
+ * Key/query heads are shared by groups of Hv/Hk consecutive value heads (same page, "La
+ * dissymétrie 16 / 48": 16 key heads for 48 value heads; 16 for 128 in the "Max" variant): value
+ * head h reads key head h / (Hv/Hk).  The state is kept in fp32 whatever the input dtype (same
+ * page, "Le float32 n'est pas un détail").
+ *
+ * Layouts (row-major, last index contiguous, no padding, no strides):
+ *   q, k        [B, T, Hk, dk]        dtype given by `dtype`
+ *   v, o        [B, T, Hv, dv]        dtype given by `dtype`
+ *   log_alpha   [B, T, Hv]  float     alpha = exp(log_alpha), expected in ]0, 1]
+ *   beta        [B, T, Hv]  float     expected in [0, 1]
+ *   S0, S_T, S  [B, Hv, dk, dv] float, holding S transposed: S_store[b][h][i][j] = S[j][i]
+ *               (i over d_k, j over d_v; d_v contiguous)
+ *
+ * Pointers.  Every tensor pointer is a DEVICE pointer (cudaMalloc'd or equivalent) on the device
+ * current for the calling thread, unless a comment says otherwise.  The caller owns every
+ * buffer; the library keeps no pointer after a call returns and allocates no device memory,
+ * except one 4-byte device error word per device, created statically with the library.
+ * Outputs must not overlap inputs, except S in gdn_decode_step, which is read and written in
+ * place.  Device pointers must be 16-byte aligned.
+ *
+ * Streams.  `stream` is a cudaStream_t (NULL = the legacy default stream).  Each compute call
+ * validates its arguments synchronously, enqueues its kernels on `stream` and returns without
+ * waiting; results are ready when the stream reaches that point.
+ *
+ * Errors.  Calls return gdn_status and never abort, throw or trap.  GDN_ERR_INVALID_ARG: a null
+ * required pointer, a non-positive size, Hv not a multiple of Hk, misalignment, or an
+ * unsupported enum value; nothing is enqueued.  GDN_ERR_UNSUPPORTED: valid sizes this build has
+ * no kernel for (dk, dv not in {16, 32, 64, 128}, chunk not in {16, 32, 64}); nothing enqueued.
+ * GDN_ERR_CUDA: a CUDA call failed (e.g. the launch); the CUDA error is left for
+ * cudaGetLastError.  GDN_ERR_TIMEOUT is reported by gdn_check_error when a kernel gave up on a
+ * bounded wait (it then skipped the rest of its work; its outputs are undefined).
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared here so that this header needs no CUDA include. */
+typedef struct CUstream_st *gdn_stream_t;
+
+typedef enum {
+  GDN_OK = 0,
+  GDN_ERR_INVALID_ARG = 1,
+  GDN_ERR_UNSUPPORTED = 2,
+  GDN_ERR_CUDA = 3,
+  GDN_ERR_TIMEOUT = 4
+} gdn_status;
+
+/* Storage type of q, k, v, o (and z, y, raw projections).  Gates and states are always fp32. */
+typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
+
+/* Kernel family for gdn_chunk_fwd_ex.  AUTO picks TCGEN05 when it supports the call
+ * (bf16, dk = dv = 128, chunk = 64), else SIMT. */
+typedef enum { GDN_VARIANT_AUTO = 0, GDN_VARIANT_SIMT = 1, GDN_VARIANT_TCGEN05 = 2 } gdn_variant;
+
+/* Static string naming a status (host only, no CUDA call). */
+GDN_API const char *gdn_status_string(gdn_status s);
+
+/* Library ABI version (host only): major * 10000 + minor * 100 + patch. */
+GDN_API int gdn_version(void);
+
+/* Waits for `stream`, then reads and clears the current device's error word.  Returns
+ * GDN_ERR_TIMEOUT if a kernel recorded a timed-out wait since the last check, GDN_ERR_CUDA if
+ * the synchronisation failed, else GDN_OK. */
+GDN_API gdn_status gdn_check_error(gdn_stream_t stream);
+
+/*
+ * Chunked prefill forward ("Chapitre 16 - Assembler un système de type Kimi K3", 16.2: each block
+ * of `chunk` tokens is processed with matrix operations and the state is handed to the next
+ * block).  Computes o for all T tokens and the state after token T-1.
+ *   S0   may be NULL: the zero state of a fresh request (16.1: the working state is reset for
+ *        the next request).  Otherwise the state after the previous call, so that splitting a
+ *        sequence over calls gives the same result as one call.
+ *   S_T  may be NULL when the final state is not wanted.
+ *   T    need not be a multiple of `chunk`; the ragged last block is masked.
+ *   scale multiplies q (o = scale * S q).
+ * Exact in real arithmetic for any chunk size; the chunk size only reorders rounding.
+ */
+GDN_API gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v,
+                         const float *log_alpha, const float *beta, const float *S0,
+                         void *o, float *S_T,
+                         int B, int T, int Hk, int Hv, int dk, int dv, int chunk,
+                         float scale, gdn_dtype dtype, gdn_stream_t stream);
+
+/* gdn_chunk_fwd with an explicit kernel family.  GDN_ERR_UNSUPPORTED if the requested family has
+ * no kernel for these sizes/dtype. */
+GDN_API gdn_status gdn_chunk_fwd_ex(const void *q, const void *k, const void *v,
+                            const float *log_alpha, const float *beta, const float *S0,
+                            void *o, float *S_T,
+                            int B, int T, int Hk, int Hv, int dk, int dv, int chunk,
+                            float scale, gdn_dtype dtype, gdn_variant variant,
+                            gdn_stream_t stream);
+
+/* The family gdn_chunk_fwd would run for these sizes (host only, no CUDA call). */
+GDN_API gdn_variant gdn_chunk_fwd_variant(int dk, int dv, int chunk, gdn_dtype dtype);
+
+/*
+ * One decode step for N independent sequences ("Chapitre 16 ...", 16.3: read the fixed state,
+ * compute the output, update the state).  q, k [N, Hk, dk]; v, o [N, Hv, dv]; log_alpha, beta
+ * [N, Hv]; S [N, Hv, dk, dv] (S transposed, fp32) is read and overwritten in place with the
+ * state after the token.  o_t reads the updated state.
+ */
+GDN_API gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
+                           const float *log_alpha, const float *beta, float *S, void *o,
+                           int N, int Hk, int Hv, int dk, int dv, float scale,
+                           gdn_dtype dtype, gdn_stream_t stream);
+
+/*
+ * Layer prologue: causal depthwise convolution with 4 taps and no bias, then SiLU, on the q, k
+ * and v channels; then each q and k head is divided by sqrt(sum of squares + l2_eps).
+ * ("L'attention hybride", "Le décompte": conv kernel 4 over the q, k, v channels, 4 weights per
+ * channel; "Les briques d'un réseau de neurones", 2.: SiLU(x) = x sigmoid(x).)
+ *   q_raw, k_raw [B, T, Hk*dk]; v_raw [B, T, Hv*dv]         (dtype)
+ *   wq, wk [Hk*dk, 4]; wv [Hv*dv, 4] float: tap 3 multiplies the current token, tap 0 the token
+ *        three steps back; positions before t = 0 are zeros (no carried conv state).
+ *   q, k [B, T, Hk, dk]; v [B, T, Hv, dv]                    (dtype, outputs)
+ */
+GDN_API gdn_status gdn_prologue(const void *q_raw, const void *k_raw, const void *v_raw,
+                        const float *wq, const float *wk, const float *wv,
+                        void *q, void *k, void *v,
+                        int B, int T, int Hk, int Hv, int dk, int dv, float l2_eps,
+                        gdn_dtype dtype, gdn_stream_t stream);
+
+/*
+ * Output gate: y = o / sqrt(mean(o^2) + eps) * w (.) SiLU(z) for each row of dv values
+ * ("L'attention hybride": swish output gate and one normalisation gain of 128 shared by all
+ * heads; "Les briques d'un réseau de neurones", 4.: RMSNorm).
+ *   o, z, y [rows, dv] (dtype); w [dv] float.
+ */
+GDN_API gdn_status gdn_out_norm(const void *o, const void *z, const float *w, void *y,
+                        long long rows, int dv, float eps, gdn_dtype dtype,
+                        gdn_stream_t stream);
+
+/*
+ * Whole layer between the projections: gdn_prologue -> gdn_chunk_fwd -> gdn_out_norm.
+ *   q_raw, k_raw [B, T, Hk*dk]; v_raw, z [B, T, Hv*dv] (dtype); wq, wk, wv conv taps as in
+ *   gdn_prologue; log_alpha, beta [B, T, Hv]; S0 nullable; norm_w [dv];
+ *   y [B, T, Hv, dv] (dtype, output); S_T nullable (output).
+ *   workspace: device scratch of at least gdn_layer_workspace_bytes(...) bytes, 256-byte
+ *   aligned, or NULL when that size is 0.  Its contents are undefined after the call.
+ */
+GDN_API gdn_status gdn_layer_fwd(const void *q_raw, const void *k_raw, const void *v_raw,
+                         const void *z, const float *wq, const float *wk, const float *wv,
+                         const float *log_alpha, const float *beta, const float *S0,
+                         const float *norm_w, void *y, float *S_T,
+                         void *workspace, size_t workspace_bytes,
+                         int B, int T, int Hk, int Hv, int dk, int dv, int chunk,
+                         float scale, float l2_eps, float norm_eps,
+                         gdn_dtype dtype, gdn_stream_t stream);
+
+/* Scratch bytes gdn_layer_fwd needs for these sizes (host only, no CUDA call); 0 if none. */
+GDN_API size_t gdn_layer_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, int chunk,
+                                 gdn_dtype dtype);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

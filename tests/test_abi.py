@@ -1,0 +1,107 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol include/gdn.h declares, and its
+host-only logic (status strings, variant choice, workspace sizing, argument validation that rejects
+bad calls before any CUDA call) behaves as documented."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from gated_deltanet_linear_18_b200 import _build
+    _build.build()
+    import gated_deltanet_linear_18_b200 as g
+    return g.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"GDN_API\s+[\w\s\*]+?\b(gdn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_calls():
+    names = declared_functions()
+    for must in ("gdn_prologue", "gdn_chunk_fwd", "gdn_decode_step", "gdn_out_norm",
+                 "gdn_layer_fwd", "gdn_status_string", "gdn_check_error"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings_and_version(L):
+    assert L.gdn_status_string(0) == b"GDN_OK"
+    assert L.gdn_status_string(4) == b"GDN_ERR_TIMEOUT"
+    assert L.gdn_status_string(99) == b"GDN_ERR_UNKNOWN"
+    assert L.gdn_version() >= 10000
+
+
+def test_variant_choice(L):
+    # bf16 / d128 / chunk 64 goes to the tensor-core family once it exists; fp32 never does
+    assert L.gdn_chunk_fwd_variant(16, 16, 16, 0) == 1
+    assert L.gdn_chunk_fwd_variant(128, 128, 64, 0) == 1
+    assert L.gdn_chunk_fwd_variant(128, 128, 64, 1) in (1, 2)
+
+
+def test_workspace_bytes(L):
+    n = L.gdn_layer_workspace_bytes(2, 100, 2, 4, 16, 32, 16, 1)
+    up = lambda x: (x + 255) // 256 * 256
+    assert n == 2 * up(2 * 100 * 2 * 16 * 2) + 2 * up(2 * 100 * 4 * 32 * 2)
+    assert L.gdn_layer_workspace_bytes(0, 100, 2, 4, 16, 32, 16, 1) == 0
+
+
+P = ctypes.c_void_p
+FAKE = P(0x1000)          # never dereferenced: validation fails or returns before any CUDA call
+
+
+def chunk(L, B=1, T=64, Hk=2, Hv=2, dk=16, dv=16, C=16, dtype=0, q=FAKE, o=FAKE, variant=0):
+    return L.gdn_chunk_fwd_ex(q, FAKE, FAKE, FAKE, FAKE, None, o, None, B, T, Hk, Hv, dk, dv, C,
+                              1.0, dtype, variant, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(B=-1), 1), (dict(T=-5), 1), (dict(Hk=0), 1), (dict(Hv=3), 1),   # Hv % Hk != 0
+    (dict(dk=0), 1), (dict(C=0), 1), (dict(dtype=7), 1), (dict(variant=9), 1),
+    (dict(q=None), 1), (dict(o=None), 1), (dict(q=P(0x1004)), 1),        # null / misaligned
+    (dict(dk=48), 2), (dict(dv=256), 2), (dict(C=128), 2), (dict(C=8), 2),
+    (dict(variant=2, dtype=0), 2),                                        # no tcgen05 fp32 kernel
+    (dict(B=0), 0),                                                       # empty batch: no work
+])
+def test_chunk_fwd_validation(L, kw, expect):
+    assert chunk(L, **kw) == expect
+
+
+def test_decode_validation(L):
+    f = L.gdn_decode_step
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, -1, 2, 2, 16, 16, 1.0, 0, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 3, 16, 16, 1.0, 0, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 4, 2, 2, 16, 16, 1.0, 0, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 2, 24, 16, 1.0, 0, None) == 2
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, 2, 16, 16, 1.0, 0, None) == 0
+
+
+def test_prologue_and_out_norm_validation(L):
+    assert L.gdn_prologue(*([FAKE] * 9), 1, 8, 2, 4, 16, 16, -1.0, 1, None) == 1   # eps < 0
+    assert L.gdn_prologue(*([FAKE] * 8), None, 1, 8, 2, 4, 16, 16, 1e-6, 1, None) == 1
+    assert L.gdn_prologue(*([FAKE] * 9), 1, 0, 2, 4, 16, 16, 1e-6, 1, None) == 0     # T = 0
+    assert L.gdn_out_norm(FAKE, FAKE, FAKE, FAKE, 10, 100, 1e-5, 1, None) == 2
+    assert L.gdn_out_norm(FAKE, FAKE, None, FAKE, 10, 128, 1e-5, 1, None) == 1
+    assert L.gdn_out_norm(FAKE, FAKE, FAKE, FAKE, 0, 128, 1e-5, 1, None) == 0
+
+
+def test_layer_validation(L):
+    args = [FAKE] * 13
+    # workspace missing although one is needed
+    assert L.gdn_layer_fwd(*args, None, 0, 1, 8, 2, 4, 16, 16, 16, 1.0, 1e-6, 1e-5, 1,
+                           None) == 1
+    # misaligned workspace
+    assert L.gdn_layer_fwd(*args, P(0x1010), 1 << 30, 1, 8, 2, 4, 16, 16, 16, 1.0, 1e-6, 1e-5,
+                           1, None) == 1

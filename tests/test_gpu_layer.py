@@ -1,0 +1,100 @@
+"""Parity of the layer prologue, the gated RMSNorm epilogue and the whole layer with the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import gdn_inputs as gi
+import gated_deltanet_linear_18_b200 as gdn
+from gpu_util import TOL_BF16_OUT, TOL_BF16_STATE, TOL_F32_ABS, max_abs, np64, rel_rms, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def layer_w(**kw):
+    return gi.WORKLOADS["layer_8to1"].with_sizes(**kw)
+
+
+@pytest.mark.parametrize("dtype,T,dk,dv", [("f32", 70, 16, 32), ("f32", 131, 64, 64),
+                                           ("bf16", 200, 128, 128), ("bf16", 3, 128, 128)])
+def test_prologue(orc, dtype, T, dk, dv):
+    w = layer_w(B=2, T=T, Hk=2, Hv=4, dk=dk, dv=dv, dtype=dtype, seed=T)
+    x = gi.make_layer_inputs(w)
+    d = to_dev(x)
+    q, k, v = gdn.prologue(d["q_raw"], d["k_raw"], d["v_raw"], d["conv_wq"], d["conv_wk"],
+                           d["conv_wv"], w.Hk, w.Hv, w.dk, w.dv, l2_eps=w.l2_eps)
+    torch.cuda.synchronize()
+    qr, kr, vr = orc.prologue(x["q_raw"], x["k_raw"], x["v_raw"], x["conv_wq"], x["conv_wk"],
+                              x["conv_wv"], w.Hk, w.Hv, w.dk, w.dv, w.l2_eps)
+    if dtype == "f32":
+        for g, r in ((q, qr), (k, kr), (v, vr)):
+            assert max_abs(g, r) <= 1e-5
+    else:   # one bf16 rounding of each output: relative error 2^-8 at most
+        for g, r in ((q, qr), (k, kr), (v, vr)):
+            assert np.all(np.abs(np64(g) - r) <= 2.0 ** -8 * np.abs(r) + 1e-6)
+
+
+@pytest.mark.parametrize("dtype,dv", [("f32", 16), ("f32", 128), ("bf16", 64), ("bf16", 128)])
+def test_out_norm(orc, dtype, dv):
+    g = torch.Generator().manual_seed(dv)
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    o = (torch.randn(37, 3, dv, generator=g) * 2).to(tdt)
+    z = torch.randn(37, 3, dv, generator=g).to(tdt)
+    w = torch.rand(dv, generator=g) + 0.5
+    y = gdn.out_norm(o.cuda(), z.cuda(), w.cuda(), eps=1e-5)
+    torch.cuda.synchronize()
+    ref = orc.gated_rmsnorm(o, z, w, 1e-5)
+    if dtype == "f32":
+        assert max_abs(y, ref) <= 1e-5
+    else:
+        assert np.all(np.abs(np64(y) - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-6)
+
+
+def _layer(x, w):
+    d = to_dev(x)
+    y, sT = gdn.layer_fwd(d["q_raw"], d["k_raw"], d["v_raw"], d["z"], d["conv_wq"], d["conv_wk"],
+                          d["conv_wv"], d["log_alpha"], d["beta"], d["S0"], d["norm_w"],
+                          Hk=w.Hk, Hv=w.Hv, dk=w.dk, dv=w.dv, chunk=w.chunk,
+                          l2_eps=w.l2_eps, norm_eps=w.norm_eps)
+    torch.cuda.synchronize()
+    gdn.check_error()
+    return y, sT
+
+
+def _ref_layer(orc, x, w, b=None, h=None):
+    """Oracle of the whole layer, optionally for one (batch, value head) only (channel slices)."""
+    if h is None:
+        return orc.layer_forward(x["q_raw"], x["k_raw"], x["v_raw"], x["z"], x["conv_wq"],
+                                 x["conv_wk"], x["conv_wv"], x["log_alpha"], x["beta"], x["S0"],
+                                 x["norm_w"], w.Hk, w.Hv, w.dk, w.dv, w.l2_eps, w.norm_eps)
+    hk = h // (w.Hv // w.Hk)
+    qs, vs = slice(hk * w.dk, (hk + 1) * w.dk), slice(h * w.dv, (h + 1) * w.dv)
+    bb = slice(b, b + 1)
+    s0 = None if x["S0"] is None else x["S0"][bb, h:h + 1]
+    return orc.layer_forward(x["q_raw"][bb, :, qs], x["k_raw"][bb, :, qs], x["v_raw"][bb, :, vs],
+                             x["z"][bb, :, vs], x["conv_wq"][qs], x["conv_wk"][qs],
+                             x["conv_wv"][vs], x["log_alpha"][bb, :, h:h + 1],
+                             x["beta"][bb, :, h:h + 1], s0, x["norm_w"], 1, 1, w.dk, w.dv,
+                             w.l2_eps, w.norm_eps)
+
+
+def test_layer_small(orc):
+    w = layer_w(B=2, T=150, Hk=2, Hv=16, seed=31, s0_std=0.02)
+    x = gi.make_layer_inputs(w)
+    y, sT = _layer(x, w)
+    y_ref, s_ref = _ref_layer(orc, x, w)
+    assert rel_rms(y, y_ref) <= TOL_BF16_OUT, rel_rms(y, y_ref)
+    assert rel_rms(sT, s_ref) <= TOL_BF16_STATE, rel_rms(sT, s_ref)
+
+
+def test_layer_full_size_sampled(orc):
+    """The 8:1 full layer at full size (B2 T8192 Hk16 Hv128); sampled (batch, head) pairs."""
+    w = gi.WORKLOADS["layer_8to1"]
+    x = gi.make_layer_inputs(w)
+    y, sT = _layer(x, w)
+    y, sT = y.cpu(), sT.cpu()
+    for b, h in ((0, 0), (1, 77), (1, 127)):
+        y_ref, s_ref = _ref_layer(orc, x, w, b, h)
+        e_y = rel_rms(y[b:b + 1, :, h:h + 1], y_ref)
+        e_s = rel_rms(sT[b:b + 1, h:h + 1], s_ref)
+        assert e_y <= TOL_BF16_OUT, (b, h, e_y)
+        assert e_s <= TOL_BF16_STATE, (b, h, e_s)
