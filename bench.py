@@ -326,32 +326,25 @@ def e2e_prefill(gdn, x, w, dev, steps):
 # ------------------------------------------------------------------------------------------------
 
 def oracle_sample_rate(x, w, target_s: float):
-    """Tokens/s of the fp64 oracle on this host, on a bounded sample: the first `nh` value heads
-    of batch 0 over all T tokens, nh calibrated to take about `target_s` seconds; scaled to the
-    full workload's tokens by the fraction of (batch, head) recurrences processed."""
+    """Tokens/s of the fp64 oracle on this host's cores.  Batch 0 (all heads) calibrates; then
+    the whole workload runs if that is estimated under 30 s, else the first `nb` batches with nb
+    chosen for about `target_s` seconds; tokens/s counts the tokens actually processed."""
     import oracle
     threads = oracle.default_threads()
 
-    def run(nh):
-        G = w.Hv // w.Hk
-        nk = (nh + G - 1) // G
+    def run(nb):
         t0 = time.perf_counter()
-        oracle.gated_delta(x["q"][:1, :, :nk], x["k"][:1, :, :nk], x["v"][:1, :, :nh],
-                           x["log_alpha"][:1, :, :nh], x["beta"][:1, :, :nh], None,
+        oracle.gated_delta(x["q"][:nb], x["k"][:nb], x["v"][:nb], x["log_alpha"][:nb],
+                           x["beta"][:nb], None if x["S0"] is None else x["S0"][:nb],
                            threads=threads)
         return time.perf_counter() - t0
-    nh = min(w.Hv, threads)
-    t = run(nh)
-    per_round = t
-    rounds = max(1, min(int(target_s / max(per_round, 1e-3)), (w.B * w.Hv) // max(nh, 1)))
-    heads = min(w.Hv, nh * rounds)
-    t = run(heads)
-    frac = heads / (w.B * w.Hv)
-    return {"value": w.B * w.T * frac / t, "unit": "tokens/s", "cores": threads,
-            "kind": "oracle",
-            "sample": f"fp64 token-by-token recurrence on batch 0, value heads 0..{heads - 1} of "
-                      f"{workload_name(w)} ({heads} of {w.B * w.Hv} head recurrences, "
-                      f"{t:.1f} s); tokens/s scaled by that fraction",
+    t1 = run(1)
+    nb = w.B if t1 * w.B <= 30.0 else max(1, min(w.B, int(target_s / max(t1, 1e-3))))
+    t = run(nb) if nb > 1 else t1
+    return {"value": nb * w.T / t, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"fp64 token-by-token recurrence over batches 0..{nb - 1} (all {w.Hv} "
+                      f"heads, all {w.T} tokens) of {workload_name(w)}: {nb * w.T} tokens in "
+                      f"{t:.1f} s on {threads} threads",
             "seconds": t}
 
 
@@ -391,8 +384,8 @@ def run_reference(args, world, rank):
     import oracle
     threads = oracle.default_threads()
     G = w.Hv // w.Hk
-    nh = min(w.Hv, max(G, threads))          # one bounded sample per step: nh heads of batch 0
-    nk = (nh + G - 1) // G
+    nk = max(1, min(w.Hk, threads // G))     # one bounded sample per step: nk key-head groups
+    nh = nk * G
 
     def step():
         oracle.gated_delta(x["q"][:1, :, :nk], x["k"][:1, :, :nk], x["v"][:1, :, :nh],

@@ -6,7 +6,7 @@ import torch
 import gdn_inputs as gi
 import gated_deltanet_linear_18_b200 as gdn
 from gpu_util import (TOL_BF16_OUT, TOL_BF16_STATE, TOL_F32_ABS, frob_rel, max_abs, np64,
-                      rel_rms, to_dev)
+                      out_err, rel_rms, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -61,7 +61,7 @@ def test_bf16_d128_small(orc, variant, T):
     w, x = small_bf16(T=T, seed=T)
     o, sT = run(x, 64, variant=variant)
     o_ref, s_ref = ref(orc, x)
-    assert rel_rms(o, o_ref) <= TOL_BF16_OUT, rel_rms(o, o_ref)
+    assert out_err(o, o_ref) <= TOL_BF16_OUT, (out_err(o, o_ref), rel_rms(o, o_ref))
     assert rel_rms(sT, s_ref) <= TOL_BF16_STATE, rel_rms(sT, s_ref)
 
 
@@ -73,7 +73,7 @@ def test_bf16_zero_state_and_no_state_out(orc):
     torch.cuda.synchronize()
     assert sT is None
     o_ref, _ = ref(orc, x)
-    assert rel_rms(o, o_ref) <= TOL_BF16_OUT
+    assert out_err(o, o_ref) <= TOL_BF16_OUT
 
 
 def test_split_run_equals_one_run():
@@ -129,7 +129,7 @@ def test_degenerate_gates(orc):
     o, sT = run(x, 64)
     o_ref, s_ref = ref(orc, x)
     assert max_abs(sT, s_ref) <= 1e-6
-    assert rel_rms(o, o_ref) <= TOL_BF16_OUT
+    assert out_err(o, o_ref) <= TOL_BF16_OUT
 
 
 def test_nan_propagates():
@@ -151,8 +151,8 @@ def _sampled_heads(orc, x, o, sT, heads, Hk, Hv):
                                        x["log_alpha"][b:b + 1, :, h:h + 1],
                                        x["beta"][b:b + 1, :, h:h + 1], s0)
         go, gs = o[b:b + 1, :, h:h + 1], sT[b:b + 1, h:h + 1]
-        e_o, e_s = rel_rms(go, o_ref), rel_rms(gs, s_ref)
-        assert e_o <= TOL_BF16_OUT, (b, h, e_o, frob_rel(go, o_ref))
+        e_o, e_s = out_err(go, o_ref), rel_rms(gs, s_ref)
+        assert e_o <= TOL_BF16_OUT, (b, h, e_o, rel_rms(go, o_ref), frob_rel(go, o_ref))
         assert e_s <= TOL_BF16_STATE, (b, h, e_s, frob_rel(gs, s_ref))
 
 
