@@ -83,15 +83,15 @@ prologue_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
   }
 }
 
-// One warp per row of dv <= 128 values.
-template <typename Tio>
+// One warp per row of dv <= 128 values.  `o` may be wider than z / y (the layer keeps o in fp32).
+template <typename To, typename Tio>
 __global__ void __launch_bounds__(256)
-out_norm_kernel(const Tio* __restrict__ o, const Tio* __restrict__ z, const float* __restrict__ w,
+out_norm_kernel(const To* __restrict__ o, const Tio* __restrict__ z, const float* __restrict__ w,
                 Tio* __restrict__ y, long long rows, int dv, float eps) {
   const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
-  const Tio* orow = o + row * dv;
+  const To* orow = o + row * dv;
   const Tio* zrow = z + row * dv;
   float ov[4];
   float ss = 0.f;

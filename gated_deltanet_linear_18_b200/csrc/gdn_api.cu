@@ -18,6 +18,8 @@ constexpr int kVersion = 10000;   // 1.0.0
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool opt_aligned16(const void* p) { return p == nullptr || aligned16(p); }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+bool opt_aligned4(const void* p) { return p == nullptr || aligned4(p); }
 bool supported_dim(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 bool supported_chunk(int c) { return c == 16 || c == 32 || c == 64; }
 bool valid_dtype(gdn_dtype t) { return t == GDN_F32 || t == GDN_BF16; }
@@ -29,12 +31,12 @@ gdn_status launch_status() {
 // ---------------------------------------------------------------------------------------------
 // SIMT chunked forward dispatch: DK in {16,32,64,128} x C in {16,32,64}, dv tiles of 16 columns.
 // ---------------------------------------------------------------------------------------------
-template <int DK, int C, typename Tio>
+template <int DK, int C, typename Tio, typename Tout>
 gdn_status simt_launch(const void* q, const void* k, const void* v, const float* la,
                        const float* be, const float* S0, void* o, float* S_T, int B, int T,
                        int Hk, int Hv, int dv, float scale, cudaStream_t st) {
   constexpr int DVT = 16;
-  auto kern = chunk_fwd_simt_kernel<DK, DVT, C, Tio>;
+  auto kern = chunk_fwd_simt_kernel<DK, DVT, C, Tio, Tout>;
   const size_t smem = simt_chunk_smem_floats<DK, DVT, C>() * sizeof(float);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
@@ -42,17 +44,18 @@ gdn_status simt_launch(const void* q, const void* k, const void* v, const float*
   dim3 grid(dv / DVT, Hv, B);
   kern<<<grid, kSimtThreads, smem, st>>>(
       static_cast<const Tio*>(q), static_cast<const Tio*>(k), static_cast<const Tio*>(v), la,
-      be, S0, static_cast<Tio*>(o), S_T, T, Hk, Hv, dv, scale);
+      be, S0, static_cast<Tout*>(o), S_T, T, Hk, Hv, dv, scale);
   return launch_status();
 }
 
-template <typename Tio>
+template <typename Tio, typename Tout = Tio>
 gdn_status simt_dispatch(int dk, int chunk, const void* q, const void* k, const void* v,
                          const float* la, const float* be, const float* S0, void* o, float* S_T,
                          int B, int T, int Hk, int Hv, int dv, float scale, cudaStream_t st) {
 #define GDN_SIMT_CASE(DK_, C_)                                                             \
   if (dk == DK_ && chunk == C_)                                                            \
-    return simt_launch<DK_, C_, Tio>(q, k, v, la, be, S0, o, S_T, B, T, Hk, Hv, dv, scale, st);
+    return simt_launch<DK_, C_, Tio, Tout>(q, k, v, la, be, S0, o, S_T, B, T, Hk, Hv, dv, scale, \
+                                           st);
   GDN_SIMT_CASE(16, 16) GDN_SIMT_CASE(16, 32) GDN_SIMT_CASE(16, 64)
   GDN_SIMT_CASE(32, 16) GDN_SIMT_CASE(32, 32) GDN_SIMT_CASE(32, 64)
   GDN_SIMT_CASE(64, 16) GDN_SIMT_CASE(64, 32) GDN_SIMT_CASE(64, 64)
@@ -100,6 +103,20 @@ gdn_status decode_dispatch(int dk, int dv, const void* q, const void* k, const v
       return decode_dispatch_dv<Tio, 128>(dv, q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
   }
   return GDN_ERR_UNSUPPORTED;
+}
+
+// The recurrence inside gdn_layer_fwd: inputs in `dtype`, output o in fp32.
+gdn_status layer_chunk_fwd(const void* q, const void* k, const void* v, const float* la,
+                           const float* be, const float* S0, float* o, float* S_T, int B, int T,
+                           int Hk, int Hv, int dk, int dv, int chunk, float scale,
+                           gdn_dtype dtype, cudaStream_t st) {
+  if (tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16))
+    return tc_chunk_launch_f32out(q, k, v, la, be, S0, o, S_T, B, T, Hk, Hv, scale, st);
+  if (dtype == GDN_F32)
+    return simt_dispatch<float, float>(dk, chunk, q, k, v, la, be, S0, o, S_T, B, T, Hk, Hv, dv,
+                                       scale, st);
+  return simt_dispatch<__nv_bfloat16, float>(dk, chunk, q, k, v, la, be, S0, o, S_T, B, T, Hk,
+                                             Hv, dv, scale, st);
 }
 
 gdn_status validate_heads(int Hk, int Hv, int dk, int dv) {
@@ -156,9 +173,8 @@ gdn_status gdn_chunk_fwd_ex(const void* q, const void* k, const void* v, const f
   if (B > 65535) return GDN_ERR_UNSUPPORTED;
   const bool work = (long)B * T > 0;
   if (work && (!q || !k || !v || !log_alpha || !beta || !o)) return GDN_ERR_INVALID_ARG;
-  if (!aligned16(q) && q) return GDN_ERR_INVALID_ARG;
-  if (!opt_aligned16(k) || !opt_aligned16(v) || !opt_aligned16(o) ||
-      !opt_aligned16(log_alpha) || !opt_aligned16(beta) || !opt_aligned16(S0) ||
+  if (!opt_aligned16(q) || !opt_aligned16(k) || !opt_aligned16(v) || !opt_aligned16(o) ||
+      !opt_aligned4(log_alpha) || !opt_aligned4(beta) || !opt_aligned16(S0) ||
       !opt_aligned16(S_T))
     return GDN_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -197,8 +213,8 @@ gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const fl
   if (s != GDN_OK) return s;
   if (N == 0) return GDN_OK;
   if (!q || !k || !v || !log_alpha || !beta || !S || !o) return GDN_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha) ||
-      !aligned16(beta) || !aligned16(S) || !aligned16(o))
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned4(log_alpha) ||
+      !aligned4(beta) || !aligned16(S) || !aligned16(o))
     return GDN_ERR_INVALID_ARG;
   if ((long)N * Hv > 0x7fffffffL) return GDN_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -217,9 +233,11 @@ gdn_status gdn_prologue(const void* q_raw, const void* k_raw, const void* v_raw,
   if (s != GDN_OK) return s;
   if ((long)B * T == 0) return GDN_OK;
   if (B > 65535 || 2L * Hk + Hv > 65535) return GDN_ERR_UNSUPPORTED;
-  const void* ptrs[] = {q_raw, k_raw, v_raw, wq, wk, wv, q, k, v};
+  const void* ptrs[] = {q_raw, k_raw, v_raw, q, k, v};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return GDN_ERR_INVALID_ARG;
+  if (!wq || !wk || !wv || !aligned4(wq) || !aligned4(wk) || !aligned4(wv))
+    return GDN_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   dim3 grid((T + kPrologueTokens - 1) / kPrologueTokens, 2 * Hk + Hv, B);
   if (dtype == GDN_F32)
@@ -239,16 +257,16 @@ gdn_status gdn_out_norm(const void* o, const void* z, const float* w, void* y, l
   if (rows < 0 || !valid_dtype(dtype) || dv <= 0 || !(eps >= 0.f)) return GDN_ERR_INVALID_ARG;
   if (!supported_dim(dv)) return GDN_ERR_UNSUPPORTED;
   if (rows == 0) return GDN_OK;
-  if (!o || !z || !w || !y || !aligned16(o) || !aligned16(z) || !aligned16(w) || !aligned16(y))
+  if (!o || !z || !w || !y || !aligned16(o) || !aligned16(z) || !aligned4(w) || !aligned16(y))
     return GDN_ERR_INVALID_ARG;
   const long long blocks = (rows + 7) / 8;
   if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == GDN_F32)
-    out_norm_kernel<float><<<(unsigned)blocks, 256, 0, st>>>((const float*)o, (const float*)z, w,
-                                                             (float*)y, rows, dv, eps);
+    out_norm_kernel<float, float><<<(unsigned)blocks, 256, 0, st>>>(
+        (const float*)o, (const float*)z, w, (float*)y, rows, dv, eps);
   else
-    out_norm_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
+    out_norm_kernel<__nv_bfloat16, __nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
         (const __nv_bfloat16*)o, (const __nv_bfloat16*)z, w, (__nv_bfloat16*)y, rows, dv, eps);
   return launch_status();
 }
@@ -260,8 +278,8 @@ size_t gdn_layer_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, i
   const size_t el = dtype == GDN_F32 ? 4 : 2;
   const size_t tok = (size_t)B * T;
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-  // normalised q, k, convolved v and the pre-norm output o
-  return 2 * up(tok * Hk * dk * el) + 2 * up(tok * Hv * dv * el);
+  // normalised q, k and convolved v in the storage dtype; the pre-norm output o in fp32
+  return 2 * up(tok * Hk * dk * el) + up(tok * Hv * dv * el) + up(tok * Hv * dv * 4);
 }
 
 gdn_status gdn_layer_fwd(const void* q_raw, const void* k_raw, const void* v_raw, const void* z,
@@ -278,7 +296,7 @@ gdn_status gdn_layer_fwd(const void* q_raw, const void* k_raw, const void* v_raw
   if (!supported_chunk(chunk)) return GDN_ERR_UNSUPPORTED;
   const size_t need = gdn_layer_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, dtype);
   if ((long)B * T > 0) {
-    if (!z || !norm_w || !y || !aligned16(z) || !aligned16(norm_w) || !aligned16(y))
+    if (!z || !norm_w || !y || !aligned16(z) || !aligned4(norm_w) || !aligned16(y))
       return GDN_ERR_INVALID_ARG;
     if (need > 0 && (!workspace || workspace_bytes < need ||
                      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0))
@@ -298,10 +316,21 @@ gdn_status gdn_layer_fwd(const void* q_raw, const void* k_raw, const void* v_raw
   s = gdn_prologue(q_raw, k_raw, v_raw, wq, wk, wv, qn, kn, vc, B, T, Hk, Hv, dk, dv, l2_eps,
                    dtype, stream);
   if (s != GDN_OK) return s;
-  s = gdn_chunk_fwd(qn, kn, vc, log_alpha, beta, S0, o, S_T, B, T, Hk, Hv, dk, dv, chunk, scale,
-                    dtype, stream);
+  // the recurrence writes o in fp32 so that the gated norm reads it unrounded
+  s = layer_chunk_fwd(qn, kn, vc, log_alpha, beta, S0, static_cast<float*>(o), S_T, B, T, Hk, Hv,
+                      dk, dv, chunk, scale, dtype, reinterpret_cast<cudaStream_t>(stream));
   if (s != GDN_OK) return s;
-  return gdn_out_norm(o, z, norm_w, y, (long long)tok * Hv, dv, norm_eps, dtype, stream);
+  const long long rows = (long long)tok * Hv;
+  const long long blocks = (rows + 7) / 8;
+  if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == GDN_F32)
+    out_norm_kernel<float, float><<<(unsigned)blocks, 256, 0, st>>>(
+        (const float*)o, (const float*)z, norm_w, (float*)y, rows, dv, norm_eps);
+  else
+    out_norm_kernel<float, __nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
+        (const float*)o, (const __nv_bfloat16*)z, norm_w, (__nv_bfloat16*)y, rows, dv, norm_eps);
+  return launch_status();
 }
 
 }  // extern "C"

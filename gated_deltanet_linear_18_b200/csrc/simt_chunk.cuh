@@ -27,12 +27,12 @@ constexpr size_t simt_chunk_smem_floats() {
   return 3 * C * DK + DK * DVT + 2 * C * DVT + 3 * C * C + 4 * C;
 }
 
-template <int DK, int DVT, int C, typename Tio>
+template <int DK, int DVT, int C, typename Tio, typename Tout>
 __global__ void __launch_bounds__(kSimtThreads)
 chunk_fwd_simt_kernel(const Tio* __restrict__ q, const Tio* __restrict__ k,
                       const Tio* __restrict__ v, const float* __restrict__ log_alpha,
                       const float* __restrict__ beta, const float* __restrict__ S0,
-                      Tio* __restrict__ o, float* __restrict__ S_T, int T, int Hk, int Hv,
+                      Tout* __restrict__ o, float* __restrict__ S_T, int T, int Hk, int Hv,
                       int dv, float scale) {
   constexpr int NT = kSimtThreads;
   const int j0 = blockIdx.x * DVT;
@@ -162,7 +162,7 @@ chunk_fwd_simt_kernel(const Tio* __restrict__ q, const Tio* __restrict__ k,
         for (int d = 0; d < DK; ++d) qm += sQ[i * DK + d] * sM[d * DVT + n];
         float pd = 0.f;
         for (int j = 0; j <= i; ++j) pd += sP[i * C + j] * sV[j * DVT + n];
-        o[((b * T + t0 + i) * Hv + h) * (long)dv + j0 + n] = from_f<Tio>(sGam[i] * qm + pd);
+        o[((b * T + t0 + i) * Hv + h) * (long)dv + j0 + n] = from_f<Tout>(sGam[i] * qm + pd);
       }
     }
     __syncthreads();

@@ -13,4 +13,10 @@ inline gdn_status tc_chunk_launch(const void*, const void*, const void*, const f
   return GDN_ERR_UNSUPPORTED;
 }
 
+inline gdn_status tc_chunk_launch_f32out(const void*, const void*, const void*, const float*,
+                                         const float*, const float*, float*, float*, int, int,
+                                         int, int, float, cudaStream_t) {
+  return GDN_ERR_UNSUPPORTED;
+}
+
 }  // namespace gdn

@@ -26,7 +26,8 @@
  * buffer; the library keeps no pointer after a call returns and allocates no device memory,
  * except one 4-byte device error word per device, created statically with the library.
  * Outputs must not overlap inputs, except S in gdn_decode_step, which is read and written in
- * place.  Device pointers must be 16-byte aligned.
+ * place.  Tensor pointers (q, k, v, o, z, y, states, raw projections, workspace) must be 16-byte
+ * aligned; gate and weight pointers (log_alpha, beta, conv taps, norm gain) 4-byte aligned.
  *
  * Streams.  `stream` is a cudaStream_t (NULL = the legacy default stream).  Each compute call
  * validates its arguments synchronously, enqueues its kernels on `stream` and returns without

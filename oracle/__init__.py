@@ -17,7 +17,12 @@ Functions and the passages they follow (page titles; the C file's header has the
   * ``gated_rmsnorm``     — "L'attention hybride" (swish output gate, one 128-wide gain) and
                             "Les briques d'un réseau de neurones", 4. (RMSNorm, eps 1e-5).
   * ``layer_forward``     — composition of the above.  Parity unpinned beyond its pinned parts:
-                            the pages print no worked example of a whole layer.
+                            the pages print no worked example of a whole layer.  With
+                            ``act_dtype="bf16"`` the prologue's outputs are rounded to bf16
+                            (round to nearest even) before the recurrence, because every
+                            activation of the model but the state is BF16 ("L'attention
+                            hybride", "Le float32 n'est pas un détail").
+  * ``round_bf16``        — that rounding, written from the bf16 format (8 significant bits).
 """
 from __future__ import annotations
 
@@ -73,6 +78,15 @@ def _ptr(a: Optional[np.ndarray]):
     if a is None:
         return ctypes.POINTER(ctypes.c_double)()
     return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def round_bf16(a) -> np.ndarray:
+    """Round float64 values to the nearest bf16 value (ties to even), returned as float64.
+    bf16 keeps 8 significant bits: a = m * 2^e with 0.5 <= |m| < 1 becomes rint(m * 2^8) * 2^(e-8).
+    (The values here stay far inside bf16's normal exponent range.)"""
+    a = np.asarray(a, dtype=np.float64)
+    m, e = np.frexp(a)
+    return np.ldexp(np.rint(m * 256.0), e - 8)
 
 
 def default_threads() -> int:
@@ -182,9 +196,14 @@ class OracleLib:
     def layer_forward(self, q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w,
                       Hk: int, Hv: int, dk: int, dv: int, l2_eps: float = 1e-6,
                       norm_eps: float = 1e-5, scale: float = 1.0,
-                      threads: Optional[int] = None):
-        """Prologue -> recurrence -> gated RMSNorm.  Returns (y [B,T,Hv,dv], S_T)."""
+                      threads: Optional[int] = None, act_dtype: str = "f64"):
+        """Prologue -> recurrence -> gated RMSNorm.  Returns (y [B,T,Hv,dv], S_T).
+        act_dtype "bf16" rounds the prologue outputs (the recurrence's q, k, v) to bf16."""
         q, k, v = self.prologue(q_raw, k_raw, v_raw, wq, wk, wv, Hk, Hv, dk, dv, l2_eps)
+        if act_dtype == "bf16":
+            q, k, v = round_bf16(q), round_bf16(k), round_bf16(v)
+        elif act_dtype != "f64":
+            raise ValueError(act_dtype)
         o, sT = self.gated_delta(q, k, v, log_alpha, beta, S0, scale=scale, threads=threads)
         B, T = o.shape[:2]
         y = self.gated_rmsnorm(o, _f64(z).reshape(B, T, Hv, dv), norm_w, norm_eps)

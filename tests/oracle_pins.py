@@ -272,4 +272,19 @@ def pin_gated_rmsnorm_closed_form(orc):
     np.testing.assert_allclose(ym, -expit(-1.0) * y / 50.0, rtol=1e-13)
 
 
+def pin_round_bf16_matches_library(orc):
+    """The oracle's bf16 rounding (used for the layer's BF16 activations) equals torch's
+    float32 -> bfloat16 conversion (round to nearest even) on values exactly representable in
+    float32, including ties and values near powers of two."""
+    import oracle
+    import torch
+    rng = np.random.default_rng(15)
+    a = rng.standard_normal(20000) * np.exp2(rng.integers(-20, 20, 20000))
+    a32 = a.astype(np.float32).astype(np.float64)
+    ties = (np.arange(1, 200) * 2 + 1) * np.exp2(-9.0)          # exactly halfway between bf16s
+    x = np.concatenate([a32, ties, -ties, [0.0, 1.0, -2.0, 1.0 + 2.0 ** -8]])
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(oracle.round_bf16(x), ref)
+
+
 ALL_PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]

@@ -62,11 +62,15 @@ def _layer(x, w):
 
 
 def _ref_layer(orc, x, w, b=None, h=None):
-    """Oracle of the whole layer, optionally for one (batch, value head) only (channel slices)."""
+    """Oracle of the whole layer, optionally for one (batch, value head) only (channel slices).
+    For bf16 workloads the recurrence's q, k, v are the prologue's outputs rounded to bf16: the
+    model keeps every activation but the state in BF16 ("L'attention hybride", "Le float32 n'est
+    pas un détail"), so a bf16 layer hands bf16 q, k, v to the recurrence."""
     if h is None:
         return orc.layer_forward(x["q_raw"], x["k_raw"], x["v_raw"], x["z"], x["conv_wq"],
                                  x["conv_wk"], x["conv_wv"], x["log_alpha"], x["beta"], x["S0"],
-                                 x["norm_w"], w.Hk, w.Hv, w.dk, w.dv, w.l2_eps, w.norm_eps)
+                                 x["norm_w"], w.Hk, w.Hv, w.dk, w.dv, w.l2_eps, w.norm_eps,
+                                 act_dtype=w.dtype)
     hk = h // (w.Hv // w.Hk)
     qs, vs = slice(hk * w.dk, (hk + 1) * w.dk), slice(h * w.dv, (h + 1) * w.dv)
     bb = slice(b, b + 1)
@@ -75,7 +79,7 @@ def _ref_layer(orc, x, w, b=None, h=None):
                              x["z"][bb, :, vs], x["conv_wq"][qs], x["conv_wk"][qs],
                              x["conv_wv"][vs], x["log_alpha"][bb, :, h:h + 1],
                              x["beta"][bb, :, h:h + 1], s0, x["norm_w"], 1, 1, w.dk, w.dv,
-                             w.l2_eps, w.norm_eps)
+                             w.l2_eps, w.norm_eps, act_dtype=w.dtype)
 
 
 def test_layer_small(orc):
