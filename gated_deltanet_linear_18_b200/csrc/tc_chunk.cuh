@@ -1,34 +1,36 @@
 // Chunked forward of the gated delta rule on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
 // Shapes: d_k = d_v = 128, chunk C = 64, bf16 q/k/v, fp32 gates and state.
 //
-// Per value head and chunk, with the chunk-start state M = S^T (128 x 128, fp32) the chunk form of
+// Per value head and chunk, with the chunk-start state M = S^T (128 x 128, fp32), the chunk form of
 // the recurrence ("Chapitre 16 - Assembler un système de type Kimi K3", 16.2: matrix operations
 // inside each block, state handed from block to block) is computed as
 //   state-independent part (one per chunk, shared by both halves of the state):
-//     G = cumsum(log alpha), gamma = exp(G), S = [Q; K] K^T               (MMA, 128 x 64 x 128)
+//     G = cumsum(log alpha), gamma = exp(G), S = [Q; K] K^T                (bf16 MMA, 128x64x128)
 //     P = lower_incl(exp(G_i - G_j) q_i.k_j) * scale,  A = strict_lower(beta_i exp(G_i - G_j) k_i.k_j)
-//     T = (I + A)^-1 (fp32, blocked by 16), T_b = T diag(beta)
-//     A2 = [P T_b; T_b] = [P; I] T_b                                        (MMA, 128 x 64 x 64)
-//     Ktil = diag(exp(G_last - G)) K
+//     T = (I + A)^-1 (fp32, blocked by 16),  T_b = T diag(beta)
+//     A2 = [P T_b; T_b]                     (P T_b: tf32 MMA, 64x64x64)
 //   state-dependent chain, for each 64-column half of M independently:
-//     X = [Q; K] M                         (MMA, 128 x 64 x 128)
-//     R' = V - diag(gamma) (K M)           (rows 64..127 of X)
-//     Y = A2 R' = [P Delta; Delta]         (MMA, 128 x 64 x 64), Delta = T_b (V - diag(gamma) K M)
+//     X = [Q; K] M                           (bf16 MMA, 128x64x128)
+//     R' = V - diag(gamma) (K M)             (rows 64..127 of X)
+//     Y = A2 R' = [P Delta; Delta]           (tf32 MMA, 128x64x64), Delta = T_b (V - diag(gamma) K M)
 //     o = diag(gamma) scale (Q M) + P Delta  (rows 0..63 of X and Y)
-//     M <- gamma_last M + Ktil^T Delta     (MMA, 128 x 64 x 64; fp32 master copy in registers)
+//     M <- gamma_last M + K^T (ktil Delta),  ktil = exp(G_last - G)
+//                                            (bf16 MMA on a two-term bf16 split of ktil Delta)
 // which is the token recurrence reorganised exactly (Delta's rows are beta_t (v_t - alpha_t
-// S_{t-1} k_t)).  MMA operands are bf16, every accumulation and the master state are fp32.
+// S_{t-1} k_t)).  Accumulations and the master state are fp32.  The operands that carry the state
+// through the chain (A2, R', ktil Delta) use tf32 or a hi+lo bf16 pair: with plain bf16 there the
+// state's largest entries drift by a few percent of its RMS.
 //
 // One CTA per (batch, value head), 512 threads in specialised warps:
-//   warp 0        TMA producer (Q, K tiles double-buffered, V single-buffered)
-//   warp 1        TMEM owner; issues the state-independent MMAs (S and A2)
+//   warp 0        TMA producer (Q, K tiles double-buffered; each V half in its own buffer)
+//   warp 1        TMEM owner; issues the state-independent MMAs (S and P T_b)
 //   warps 2, 3    issue the chain MMAs of state half 0 / half 1
-//   warps 4-7     "pre" warpgroup: gates, P / A, the triangular solve, A2 and Ktil tiles
+//   warps 4-7     "pre" warpgroup: gates, A, the triangular solve, P, T_b and A2
 //   warps 8-11    chain warpgroup of half 0 (dv columns 0..63); warps 12-15 of half 1
 // so the state-independent work of chunk c+1 overlaps the chain of chunk c, and the two halves'
 // chains interleave on the tensor pipe.  Every wait is bounded (2 s): on expiry the CTA records
-// GDN's timeout bit, every role leaves its loop at the next uniform check point, in-flight TMA
-// loads and MMAs are drained, TMEM is released and the kernel returns.
+// the library's timeout bit, every role leaves its loop at the next uniform check point, in-flight
+// TMA loads and MMAs are drained, TMEM is released and the kernel returns.
 #pragma once
 
 #include <cuda.h>
@@ -42,64 +44,79 @@ namespace tcf {
 
 constexpr int C = 64;
 constexpr int kThreads = 512;
-constexpr uint64_t kBudgetNs = 2000000000ull;
+constexpr uint64_t kBudgetNs = 4000000000ull;   // wait budget in SM cycles (about 2 s)
 
 // shared memory map (bytes from a 1024-aligned base); every MMA tile is 128-byte swizzled
 constexpr uint32_t OFF_QK = 0;          // 2 stages x 32 KB: kb0 [Q 64 rows | K 64 rows], kb1 [...]
 constexpr uint32_t QK_STAGE = 32768;
-constexpr uint32_t OFF_V = 65536;       // 16 KB: dv block 0 [64 rows x 128 B], dv block 1
-constexpr uint32_t OFF_A2 = 81920;      // 16 KB: 128 rows x 128 B, K-major
-constexpr uint32_t OFF_PI = 98304;      // 16 KB: rows 0..63 P (bf16), rows 64..127 identity
-constexpr uint32_t OFF_KT = 114688;     // 16 KB: Ktil, dk block 0 [64 rows x 128 B], dk block 1
-constexpr uint32_t OFF_RD = 131072;     // 2 x 8 KB: per half, R' then Delta [64 rows x 128 B]
-constexpr uint32_t OFF_MB = 147456;     // 2 x 16 KB: per half, bf16 M [128 rows x 128 B]
-constexpr uint32_t OFF_TB = 180224;     // 8 KB: T_b bf16 [64 rows x 128 B]
-constexpr int LDA = 68;                 // fp32 row stride of the solve matrices
-constexpr uint32_t OFF_SA = 188416;     // 64 x 68 fp32: A, then D A (block rows)
-constexpr uint32_t OFF_ST = 205824;     // 64 x 68 fp32: T
-constexpr uint32_t OFF_GB = 223232;     // 3 slots x 1 KB: G[64], gamma[64], ktil[64], beta[64]
-constexpr uint32_t OFF_BAR = 226304;
+constexpr uint32_t OFF_V = 65536;       // per half 8 KB: V[t][64 dv] bf16
+constexpr uint32_t OFF_RD = 81920;      // per half 16 KB: R' tf32 [dv block][64 t][128 B], then
+                                        // ktil Delta bf16 hi [64 t][128 B] + lo [64 t][128 B]
+constexpr uint32_t OFF_A2 = 114688;     // 32 KB: A2 tf32, [K block][128 rows][128 B]
+constexpr uint32_t OFF_MB = 147456;     // per half 16 KB: bf16 M [128 dk rows][128 B]
+constexpr uint32_t OFF_W = 180224;      // 32 KB: solve scratch, then P (tf32) and T_b (tf32)
+constexpr uint32_t OFF_WT = OFF_W + 16384;   // T_b, [dv block][64 rows][128 B]
+constexpr uint32_t SOLVE_T = 12800;     // byte offset of T inside the solve scratch
+constexpr uint32_t OFF_GB = 212992;     // 3 slots x 1 KB: G[64], gamma[64], ktil[64], beta[64]
+constexpr uint32_t OFF_BAR = 216064;
 constexpr int NBAR = 40;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;   // +0 TMEM base, +4 abort flag
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+static_assert(2 * SOLVE_T <= 32768, "solve scratch");
 
 // TMEM columns (512 allocated, 128 lanes x 32 bit)
 constexpr uint32_t TM_S = 0, TM_PT = 64, TM_X = 128, TM_Y = 256, TM_D3 = 384;
 
 // mbarriers
 enum : int {
-  B_QK_FULL = 0, B_IN_EMPTY = 2, B_V_FULL = 4, B_V_EMPTY = 5, B_S_FULL = 6, B_S_EMPTY = 7,
-  B_PT_READY = 8, B_PT_FULL = 9, B_PT_EMPTY = 10, B_PRE_FULL = 11, B_A2_EMPTY = 12,
-  B_KT_EMPTY = 13, B_GATE = 14, B_HALF = 17, B_DRAIN = 35
+  B_QK_FULL = 0, B_IN_EMPTY = 2, B_S_FULL = 4, B_S_EMPTY = 5, B_PT_READY = 6, B_PT_FULL = 7,
+  B_PT_EMPTY = 8, B_PRE_FULL = 9, B_A2_EMPTY = 10, B_GATE = 11, B_HALF = 14, B_DRAIN = 36
 };
 enum : int {
   H_X_FULL = 0, H_X_EMPTY, H_R_FULL, H_Y_FULL, H_Y_EMPTY, H_D_FULL, H_D3_FULL, H_D3_EMPTY,
-  H_M_READY, H_COUNT
+  H_M_READY, H_V_FULL, H_V_EMPTY, H_COUNT
 };
 static_assert(B_HALF + 2 * H_COUNT == B_DRAIN && B_DRAIN + 3 <= NBAR, "barrier map");
 
 constexpr uint32_t ID_S = tc::idesc_bf16(128, 64, false, false);
-constexpr uint32_t ID_PT = tc::idesc_bf16(128, 64, false, true);
+constexpr uint32_t ID_PT = tc::idesc_tf32(64, 64, false, true);
 constexpr uint32_t ID_X = tc::idesc_bf16(128, 64, false, true);
-constexpr uint32_t ID_Y = tc::idesc_bf16(128, 64, false, true);
+constexpr uint32_t ID_Y = tc::idesc_tf32(128, 64, false, true);
 constexpr uint32_t ID_U = tc::idesc_bf16(128, 64, true, true);
 
-// ------------------------------------------------------------------------------------------
-// pre warpgroup helpers
-// ------------------------------------------------------------------------------------------
+// Optional per-chunk timestamps for studying the pipeline (compiled only with GDN_TC_TRACE):
+// slot (block, chunk, event) of a caller-provided buffer receives clock64().
+#ifdef GDN_TC_TRACE
+__device__ unsigned long long* g_tc_trace = nullptr;
+#define GDN_TRACE(c, ev)                                                              \
+  do {                                                                                \
+    if (g_tc_trace) g_tc_trace[((size_t)blockIdx.x * nC + (c)) * 64 + (ev)] = clock64(); \
+  } while (0)
+#else
+#define GDN_TRACE(c, ev) do {} while (0)
+#endif
 
-// out[0..3] += sum_k X[xr][xc + k] * Y[yr + k][yc .. yc+3] for k < 16 (fp32, shared memory).
-__device__ __forceinline__ void strip16(const float* X, int xr, int xc, const float* Y, int yr,
-                                        int yc, float (&acc)[4]) {
+// ------------------------------------------------------------------------------------------
+// triangular solve on 16 x 16 blocks stored packed: block (i, k), i >= k, at index
+// i(i+1)/2 + k, 16 rows of 20 floats (4 floats of padding against bank conflicts)
+// ------------------------------------------------------------------------------------------
+constexpr int BLD = 20, BSZ = 16 * BLD;
+__device__ __forceinline__ float* blk(float* base, int i, int k) {
+  return base + (i * (i + 1) / 2 + k) * BSZ;
+}
+
+// acc[0..3] += sum_k X[xr][k] * Y[k][yc .. yc+3], k < 16, X and Y 16 x 16 blocks.
+__device__ __forceinline__ void strip16(const float* X, int xr, const float* Y, int yc,
+                                        float (&acc)[4]) {
 #pragma unroll
   for (int k4 = 0; k4 < 16; k4 += 4) {
-    const float4 xa = *reinterpret_cast<const float4*>(&X[xr * LDA + xc + k4]);
+    const float4 xa = *reinterpret_cast<const float4*>(&X[xr * BLD + k4]);
     const float xs[4] = {xa.x, xa.y, xa.z, xa.w};
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
-      const float4 y = *reinterpret_cast<const float4*>(&Y[(yr + k4 + kk) * LDA + yc]);
+      const float4 y = *reinterpret_cast<const float4*>(&Y[(k4 + kk) * BLD + yc]);
       acc[0] = fmaf(xs[kk], y.x, acc[0]);
       acc[1] = fmaf(xs[kk], y.y, acc[1]);
       acc[2] = fmaf(xs[kk], y.z, acc[2]);
@@ -108,88 +125,86 @@ __device__ __forceinline__ void strip16(const float* X, int xr, int xc, const fl
   }
 }
 
-// T = (I + A)^-1 for a 64 x 64 strictly lower A, by 16 x 16 blocks (128 threads, barrier id 1):
-//   D_b = (I + A_bb)^-1 (forward substitution, one column per thread);
+// T = (I + A)^-1 for a 64 x 64 strictly lower A (128 threads, named barrier 1):
+//   D_b = (I + A_bb)^-1 by forward substitution (one column per thread);
 //   At_ik = D_i A_ik;  U = (I + At)^-1 by block forward substitution (U_ii = I);  T_ik = U_ik D_k.
-// (I + A = blockdiag(I + A_bb) (I + At), so T = U D.)  sA is overwritten by At.
+// (I + A = blockdiag(I + A_bb) (I + At), so T = U D.)  sA is overwritten with At.
 __device__ void solve_unit_lower(float* sA, float* sT, int ptid) {
   if (ptid < 64) {
-    const int ob = 16 * (ptid >> 4), c = ptid & 15;
+    const int b = ptid >> 4, c = ptid & 15;
+    const float* Ab = blk(sA, b, b);
     float x[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       float acc = (i == c) ? 1.f : 0.f;
 #pragma unroll
-      for (int j = 0; j < i; ++j) acc = fmaf(-sA[(ob + i) * LDA + ob + j], x[j], acc);
+      for (int j = 0; j < i; ++j) acc = fmaf(-Ab[i * BLD + j], x[j], acc);
       x[i] = acc;
     }
+    float* Tb = blk(sT, b, b);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) sT[(ob + i) * LDA + ob + c] = x[i];
+    for (int i = 0; i < 16; ++i) Tb[i * BLD + c] = x[i];
   }
   tc::named_bar(1, 128);
-  // At_ik = D_i A_ik for the six blocks below the diagonal
   // block index bi = 0..5 -> (i, k) = (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
   auto blk_i = [](int bi) { return bi < 1 ? 1 : (bi < 3 ? 2 : 3); };
   auto blk_k = [](int bi, int i) { return bi - i * (i - 1) / 2; };
   float r1[3][4];
 #pragma unroll
-  for (int m = 0; m < 3; ++m) {
+  for (int m = 0; m < 3; ++m) {                       // At_ik = D_i A_ik
     const int id = ptid + 128 * m, bi = id >> 6, r = (id >> 2) & 15, cs = id & 3;
     const int i = blk_i(bi), k = blk_k(bi, i);
     r1[m][0] = r1[m][1] = r1[m][2] = r1[m][3] = 0.f;
-    strip16(sT, 16 * i + r, 16 * i, sA, 16 * i, 16 * k + 4 * cs, r1[m]);
+    strip16(blk(sT, i, i), r, blk(sA, i, k), 4 * cs, r1[m]);
   }
   tc::named_bar(1, 128);
 #pragma unroll
   for (int m = 0; m < 3; ++m) {
     const int id = ptid + 128 * m, bi = id >> 6, r = (id >> 2) & 15, cs = id & 3;
     const int i = blk_i(bi), k = blk_k(bi, i);
-    *reinterpret_cast<float4*>(&sA[(16 * i + r) * LDA + 16 * k + 4 * cs]) =
+    *reinterpret_cast<float4*>(&blk(sA, i, k)[r * BLD + 4 * cs]) =
         make_float4(r1[m][0], r1[m][1], r1[m][2], r1[m][3]);
   }
   tc::named_bar(1, 128);
-  // U_20 = -At_20 + At_21 At_10; U_31 = -At_31 + At_32 At_21; V_30 = -At_30 + At_31 At_10
-  // (stored in T's blocks (2,0), (3,1), (3,0), which nothing reads in this round)
+  // U_20 = -At_20 + At_21 At_10;  U_31 = -At_31 + At_32 At_21;  V_30 = -At_30 + At_31 At_10
   for (int id = ptid; id < 192; id += 128) {
     const int bi = id >> 6, r = (id >> 2) & 15, cs = id & 3;
     const int oi = bi == 0 ? 2 : 3, ok = bi == 1 ? 1 : 0;      // output block (oi, ok)
-    const int xi = oi, xk = bi == 0 ? 1 : (bi == 1 ? 2 : 1);    // X = At_(xi, xk)
-    const int yi = xk, yk = ok;                                  // Y = At_(yi, yk)
-    float acc[4];
-    const float4 base = *reinterpret_cast<const float4*>(&sA[(16 * oi + r) * LDA + 16 * ok + 4 * cs]);
-    acc[0] = -base.x; acc[1] = -base.y; acc[2] = -base.z; acc[3] = -base.w;
-    strip16(sA, 16 * xi + r, 16 * xk, sA, 16 * yi, 16 * yk + 4 * cs, acc);
-    *reinterpret_cast<float4*>(&sT[(16 * oi + r) * LDA + 16 * ok + 4 * cs]) =
+    const int xk = bi == 1 ? 2 : 1;                             // X = At_(oi, xk), Y = At_(xk, ok)
+    const float4 base = *reinterpret_cast<const float4*>(&blk(sA, oi, ok)[r * BLD + 4 * cs]);
+    float acc[4] = {-base.x, -base.y, -base.z, -base.w};
+    strip16(blk(sA, oi, xk), r, blk(sA, xk, ok), 4 * cs, acc);
+    *reinterpret_cast<float4*>(&blk(sT, oi, ok)[r * BLD + 4 * cs]) =
         make_float4(acc[0], acc[1], acc[2], acc[3]);
   }
   tc::named_bar(1, 128);
-  // U_30 = V_30 - At_32 U_20
-  if (ptid < 64) {
+  if (ptid < 64) {                                    // U_30 = V_30 - At_32 U_20
     const int r = ptid >> 2, cs = ptid & 3;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    strip16(sA, 48 + r, 32, sT, 32, 4 * cs, acc);
-    float4* dst = reinterpret_cast<float4*>(&sT[(48 + r) * LDA + 4 * cs]);
+    strip16(blk(sA, 3, 2), r, blk(sT, 2, 0), 4 * cs, acc);
+    float4* dst = reinterpret_cast<float4*>(&blk(sT, 3, 0)[r * BLD + 4 * cs]);
     const float4 v30 = *dst;
     *dst = make_float4(v30.x - acc[0], v30.y - acc[1], v30.z - acc[2], v30.w - acc[3]);
   }
   tc::named_bar(1, 128);
-  // T_ik = U_ik D_k, with U_10 = -At_10, U_21 = -At_21, U_32 = -At_32
   float r4[3][4];
 #pragma unroll
-  for (int m = 0; m < 3; ++m) {
+  for (int m = 0; m < 3; ++m) {                       // T_ik = U_ik D_k (U = -At next to diag)
     const int id = ptid + 128 * m, bi = id >> 6, r = (id >> 2) & 15, cs = id & 3;
     const int i = blk_i(bi), k = blk_k(bi, i);
-    const bool sub = (i == k + 1);                     // U on the first sub-diagonal is -At
+    const bool sub = (i == k + 1);
     r4[m][0] = r4[m][1] = r4[m][2] = r4[m][3] = 0.f;
-    strip16(sub ? sA : sT, 16 * i + r, 16 * k, sT, 16 * k, 16 * k + 4 * cs, r4[m]);
-    if (sub) { r4[m][0] = -r4[m][0]; r4[m][1] = -r4[m][1]; r4[m][2] = -r4[m][2]; r4[m][3] = -r4[m][3]; }
+    strip16(sub ? blk(sA, i, k) : blk(sT, i, k), r, blk(sT, k, k), 4 * cs, r4[m]);
+    if (sub) {
+      r4[m][0] = -r4[m][0]; r4[m][1] = -r4[m][1]; r4[m][2] = -r4[m][2]; r4[m][3] = -r4[m][3];
+    }
   }
   tc::named_bar(1, 128);
 #pragma unroll
   for (int m = 0; m < 3; ++m) {
     const int id = ptid + 128 * m, bi = id >> 6, r = (id >> 2) & 15, cs = id & 3;
     const int i = blk_i(bi), k = blk_k(bi, i);
-    *reinterpret_cast<float4*>(&sT[(16 * i + r) * LDA + 16 * k + 4 * cs]) =
+    *reinterpret_cast<float4*>(&blk(sT, i, k)[r * BLD + 4 * cs]) =
         make_float4(r4[m][0], r4[m][1], r4[m][2], r4[m][3]);
   }
   tc::named_bar(1, 128);
@@ -241,6 +256,11 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Four fp32 values rounded to tf32, stored as one 16-byte chunk.
+__device__ __forceinline__ void st_tf32x4(uint32_t addr, float a, float b, float c, float d) {
+  tc::st_shared_v4(addr, tc::to_tf32(a), tc::to_tf32(b), tc::to_tf32(c), tc::to_tf32(d));
+}
+
 // ------------------------------------------------------------------------------------------
 // the kernel
 // ------------------------------------------------------------------------------------------
@@ -266,10 +286,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(bar(B_QK_FULL + s), 1);
-      tc::mbar_init(bar(B_IN_EMPTY + s), 4);
+      tc::mbar_init(bar(B_IN_EMPTY + s), 5);
     }
-    tc::mbar_init(bar(B_V_FULL), 1);
-    tc::mbar_init(bar(B_V_EMPTY), 2);
     tc::mbar_init(bar(B_S_FULL), 1);
     tc::mbar_init(bar(B_S_EMPTY), 1);
     tc::mbar_init(bar(B_PT_READY), 1);
@@ -277,7 +295,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     tc::mbar_init(bar(B_PT_EMPTY), 1);
     tc::mbar_init(bar(B_PRE_FULL), 1);
     tc::mbar_init(bar(B_A2_EMPTY), 2);
-    tc::mbar_init(bar(B_KT_EMPTY), 2);
     for (int i = 0; i < 3; ++i) tc::mbar_init(bar(B_GATE + i), 1);
     for (int hh = 0; hh < 2; ++hh) {
       const int hb = B_HALF + H_COUNT * hh;
@@ -290,6 +307,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       tc::mbar_init(bar(hb + H_D3_FULL), 1);
       tc::mbar_init(bar(hb + H_D3_EMPTY), 1);
       tc::mbar_init(bar(hb + H_M_READY), 1);
+      tc::mbar_init(bar(hb + H_V_FULL), 1);
+      tc::mbar_init(bar(hb + H_V_EMPTY), 1);
     }
     for (int i = 0; i < 3; ++i) tc::mbar_init(bar(B_DRAIN + i), 1);
     *abort_flag = 0;
@@ -312,7 +331,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   if (warp == 0) {
     // ------------------------------- TMA producer -------------------------------------------
     if (lane == 0) {
-      int armed_qk[2] = {-1, -1}, armed_v = -1;
+      int armed_qk[2] = {-1, -1}, armed_v[2] = {-1, -1};
       bool ok = true;
       for (int c = 0; c < nC && ok; ++c) {
         const int s = c & 1, t0 = c * C;
@@ -325,23 +344,28 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         tc::tma_load_4d(dst + 16384, &tmq, bar(B_QK_FULL + s), 64, hk, t0, bq);
         tc::tma_load_4d(dst + 24576, &tmk, bar(B_QK_FULL + s), 64, hk, t0, bq);
         armed_qk[s] = c;
-        if (c >= 1) ok = tc::mbar_wait(bar(B_V_EMPTY), (c - 1) & 1, abort_flag, kBudgetNs);
-        if (!ok) break;
-        tc::mbar_arrive_expect_tx(bar(B_V_FULL), 16384);
-        tc::tma_load_4d(sb + OFF_V, &tmv, bar(B_V_FULL), 0, h, t0, bq);
-        tc::tma_load_4d(sb + OFF_V + 8192, &tmv, bar(B_V_FULL), 64, h, t0, bq);
-        armed_v = c;
+        for (int hh = 0; hh < 2 && ok; ++hh) {
+          const int hb = B_HALF + H_COUNT * hh;
+          if (c >= 1) ok = tc::mbar_wait(bar(hb + H_V_EMPTY), (c - 1) & 1, abort_flag, kBudgetNs);
+          if (!ok) break;
+          tc::mbar_arrive_expect_tx(bar(hb + H_V_FULL), 8192);
+          tc::tma_load_4d(sb + OFF_V + hh * 8192, &tmv, bar(hb + H_V_FULL), 64 * hh, h, t0, bq);
+          armed_v[hh] = c;
+        }
       }
       if (!ok) {   // let every load already issued land before the CTA can leave
         volatile int never = 0;
         for (int s = 0; s < 2; ++s)
           if (armed_qk[s] >= 0)
             tc::mbar_wait(bar(B_QK_FULL + s), (armed_qk[s] >> 1) & 1, &never, kBudgetNs / 4);
-        if (armed_v >= 0) tc::mbar_wait(bar(B_V_FULL), armed_v & 1, &never, kBudgetNs / 4);
+        for (int hh = 0; hh < 2; ++hh)
+          if (armed_v[hh] >= 0)
+            tc::mbar_wait(bar(B_HALF + H_COUNT * hh + H_V_FULL), armed_v[hh] & 1, &never,
+                          kBudgetNs / 4);
       }
     }
   } else if (warp == 1) {
-    // -------------------- state-independent MMAs: S = [Q;K] K^T, A2 = [P; I] T_b -------------
+    // -------------------- state-independent MMAs: S = [Q;K] K^T and P T_b --------------------
     if (lane == 0) {
       auto issue_S = [&](int c) -> bool {
         const int s = c & 1;
@@ -367,9 +391,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         if (!ok) break;
         tc::tc_fence_after();
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          tc::mma_bf16(tmem + TM_PT, tc::sdesc_sw128(sb + OFF_PI + ks * 32, 16, 1024),
-                       tc::sdesc_sw128(sb + OFF_TB + ks * 2048, 8192, 1024), ID_PT, ks > 0);
+        for (int ks = 0; ks < 8; ++ks)   // P (64 x 64, K-major) x T_b (64 x 64, MN-major), tf32
+          tc::mma_tf32(tmem + TM_PT,
+                       tc::sdesc_sw128(sb + OFF_W + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024),
+                       tc::sdesc_sw128_b32(sb + OFF_WT + ks * 1024, 8192), ID_PT, ks > 0);
         tc::mma_commit(bar(B_PT_FULL));
         if (c + 1 < nC) ok = issue_S(c + 1);
       }
@@ -381,12 +406,12 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     // -------------------------- chain MMAs of one state half ---------------------------------
     if (lane == 0) {
       const int hh = warp - 2, hb = B_HALF + H_COUNT * hh;
-      const uint32_t mb = sb + OFF_MB + hh * 16384, rd = sb + OFF_RD + hh * 8192;
+      const uint32_t mb = sb + OFF_MB + hh * 16384, rd = sb + OFF_RD + hh * 16384;
       bool ok = true;
       for (int c = 0; c < nC && ok; ++c) {
         const int s = c & 1;
         const uint32_t qk = sb + OFF_QK + s * QK_STAGE;
-        // X = [Q; K] M_half
+        // X = [Q; K] M_half                                                      (bf16)
         ok = tc::mbar_wait(bar(B_QK_FULL + s), (c >> 1) & 1, abort_flag, kBudgetNs) &&
              tc::mbar_wait(bar(hb + H_M_READY), c & 1, abort_flag, kBudgetNs) &&
              (c == 0 || tc::mbar_wait(bar(hb + H_X_EMPTY), (c - 1) & 1, abort_flag, kBudgetNs));
@@ -399,29 +424,35 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
                        tc::sdesc_sw128(mb + ks * 2048, 16384, 1024), ID_X, ks > 0);
         tc::mma_commit(bar(hb + H_X_FULL));
         tc::mma_commit(bar(B_IN_EMPTY + s));
-        // Y = A2 R'
+        GDN_TRACE(c, 10 + 4 * hh);
+        // Y = A2 R'                                                              (tf32)
         ok = tc::mbar_wait(bar(hb + H_R_FULL), c & 1, abort_flag, kBudgetNs) &&
              tc::mbar_wait(bar(B_PRE_FULL), c & 1, abort_flag, kBudgetNs) &&
              (c == 0 || tc::mbar_wait(bar(hb + H_Y_EMPTY), (c - 1) & 1, abort_flag, kBudgetNs));
         if (!ok) break;
         tc::tc_fence_after();
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          tc::mma_bf16(tmem + TM_Y + 64 * hh, tc::sdesc_sw128(sb + OFF_A2 + ks * 32, 16, 1024),
-                       tc::sdesc_sw128(rd + ks * 2048, 8192, 1024), ID_Y, ks > 0);
+        for (int ks = 0; ks < 8; ++ks)
+          tc::mma_tf32(tmem + TM_Y + 64 * hh,
+                       tc::sdesc_sw128(sb + OFF_A2 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
+                       tc::sdesc_sw128_b32(rd + ks * 1024, 8192), ID_Y, ks > 0);
         tc::mma_commit(bar(hb + H_Y_FULL));
         tc::mma_commit(bar(B_A2_EMPTY));
-        // D3 = Ktil^T Delta
+        GDN_TRACE(c, 11 + 4 * hh);
+        // D3 = K^T (ktil Delta)_hi + K^T (ktil Delta)_lo                         (bf16)
         ok = tc::mbar_wait(bar(hb + H_D_FULL), c & 1, abort_flag, kBudgetNs) &&
              (c == 0 || tc::mbar_wait(bar(hb + H_D3_EMPTY), (c - 1) & 1, abort_flag, kBudgetNs));
         if (!ok) break;
         tc::tc_fence_after();
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          tc::mma_bf16(tmem + TM_D3 + 64 * hh, tc::sdesc_sw128(sb + OFF_KT + ks * 2048, 8192, 1024),
-                       tc::sdesc_sw128(rd + ks * 2048, 8192, 1024), ID_U, ks > 0);
+        for (int ks = 0; ks < 8; ++ks)
+          tc::mma_bf16(tmem + TM_D3 + 64 * hh,
+                       tc::sdesc_sw128(qk + 8192 + (ks & 3) * 2048, 16384, 1024),
+                       tc::sdesc_sw128(rd + (ks >> 2) * 8192 + (ks & 3) * 2048, 8192, 1024), ID_U,
+                       ks > 0);
         tc::mma_commit(bar(hb + H_D3_FULL));
-        tc::mma_commit(bar(B_KT_EMPTY));
+        tc::mma_commit(bar(B_IN_EMPTY + s));
+        GDN_TRACE(c, 12 + 4 * hh);
       }
       tc::mma_commit(bar(B_DRAIN + 1 + hh));
       volatile int never = 0;
@@ -430,30 +461,28 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   } else if (warp < 8) {
     // ------------------------------- pre warpgroup -------------------------------------------
     const int ptid = threadIdx.x - 128;                 // = TMEM lane of this thread
-    const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-    float* sA = reinterpret_cast<float*>(smem + OFF_SA);
-    float* sT = reinterpret_cast<float*>(smem + OFF_ST);
-    if (ptid >= 64) {   // identity rows of [P; I], written once
-      const int r = ptid, j1 = ptid - 64;
-#pragma unroll
-      for (int cc = 0; cc < 8; ++cc) {
-        uint32_t w[4] = {0u, 0u, 0u, 0u};
-        if ((j1 >> 3) == cc) w[(j1 & 7) >> 1] = (j1 & 1) ? 0x3F800000u : 0x00003F80u;
-        tc::st_shared_v4(sb + OFF_PI + tc::sw128(r, cc), w[0], w[1], w[2], w[3]);
-      }
-    }
+    const int q = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
+    float* sA = reinterpret_cast<float*>(smem + OFF_W);
+    float* sT = reinterpret_cast<float*>(smem + OFF_W + SOLVE_T);
+    float pla0 = 0.f, pla1 = 0.f, pbe0 = 0.f, pbe1 = 0.f;   // gates of the next chunk (warp 4)
+    auto load_gates = [&](int c) {
+      const long ta = (long)c * C + 2 * lane, tb = ta + 1;
+      pla0 = pla1 = pbe0 = pbe1 = 0.f;
+      if (ta < T) { pla0 = log_alpha[((long)bq * T + ta) * Hv + h]; pbe0 = beta[((long)bq * T + ta) * Hv + h]; }
+      if (tb < T) { pla1 = log_alpha[((long)bq * T + tb) * Hv + h]; pbe1 = beta[((long)bq * T + tb) * Hv + h]; }
+    };
+    if (ptid < 32) load_gates(0);
     for (int c = 0; c < nC; ++c) {
-      const int s = c & 1, slot = c % 3;
-      const long t0 = (long)c * C;
+      const int slot = c % 3;
+      if (ptid == 0) GDN_TRACE(c, 0);
       float* gG = reinterpret_cast<float*>(smem + OFF_GB + slot * 1024);
       float* gGam = gG + 64;
       float* gKt = gG + 128;
       float* gBeta = gG + 192;
       if (ptid < 32) {          // gates of this chunk: lane l holds tokens 2l, 2l+1
-        float la0 = 0.f, la1 = 0.f, be0 = 0.f, be1 = 0.f;
-        const long ta = t0 + 2 * lane, tb = ta + 1;
-        if (ta < T) { la0 = log_alpha[((long)bq * T + ta) * Hv + h]; be0 = beta[((long)bq * T + ta) * Hv + h]; }
-        if (tb < T) { la1 = log_alpha[((long)bq * T + tb) * Hv + h]; be1 = beta[((long)bq * T + tb) * Hv + h]; }
+        const float la0 = pla0, la1 = pla1, be0 = pbe0, be1 = pbe1;
+        if (c + 1 < nC) load_gates(c + 1);
         float incl = la0 + la1;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
@@ -471,115 +500,129 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         if (lane == 0) tc::mbar_arrive(bar(B_GATE + slot));
       }
       tc::named_bar(1, 128);
-      // S row -> P row (rows 0..63) or A row (rows 64..127)
+      if (ptid == 0) GDN_TRACE(c, 1);
+      // A rows (threads 64..127): A[t][j] = beta_t exp(G_t - G_j) (k_t . k_j), j < t
       tc::mbar_wait(bar(B_S_FULL), c & 1, abort_flag, kBudgetNs);
+      if (ptid == 0) GDN_TRACE(c, 2);
       tc::tc_fence_after();
-      float sv[64];
       {
-        float a16[16];
+        float sv[32];
+        const int t = ptid - 64, ti = t >> 4, tr = t & 15;
+        const float gt = ptid >= 64 ? gG[t] : 0.f, bt = ptid >= 64 ? gBeta[t] : 0.f;
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          tmem_ld16(tmem + lane_off + TM_S + 16 * p, a16);
+        for (int p = 0; p < 2; ++p) {
+          tc::tmem_ld32(tmem + lane_off + TM_S + 32 * p, sv);
           tc::tmem_wait_ld();
+          if (ptid >= 64) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) sv[16 * p + i] = a16[i];
+            for (int kb2 = 0; kb2 < 2; ++kb2) {
+              const int kb = 2 * p + kb2;
+              if (kb <= ti) {
+                float* dst = blk(sA, ti, kb) + tr * BLD;
+#pragma unroll
+                for (int e4 = 0; e4 < 16; e4 += 4) {
+                  float a[4];
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) {
+                    const int j = 16 * kb + e4 + e;
+                    a[e] = (j < t) ? bt * __expf(gt - gG[j]) * sv[16 * kb2 + e4 + e] : 0.f;
+                  }
+                  *reinterpret_cast<float4*>(dst + e4) = make_float4(a[0], a[1], a[2], a[3]);
+                }
+              }
+            }
+          }
+        }
+      }
+      tc::named_bar(1, 128);
+      if (ptid == 0) GDN_TRACE(c, 3);
+      solve_unit_lower(sA, sT, ptid);
+      if (ptid == 0) GDN_TRACE(c, 4);
+      // T_b = T diag(beta): row k = ptid/2, columns n0..n0+31 (one tf32 column block)
+      float tb[32];
+      const int kr = ptid >> 1, nb = ptid & 1;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int n = 32 * nb + e;
+        tb[e] = (n <= kr) ? blk(sT, kr >> 4, n >> 4)[(kr & 15) * BLD + (n & 15)] * gBeta[n] : 0.f;
+      }
+      if (c >= 1) tc::mbar_wait(bar(B_A2_EMPTY), (c - 1) & 1, abort_flag, kBudgetNs);
+      tc::named_bar(1, 128);                     // the solve scratch is free from here on
+      {
+        // T_b as the MN-major B operand of P T_b (32-byte chunks), and as rows 64..127 of the
+        // K-major A2 (16-byte chunks)
+        const uint32_t tb_base = sb + OFF_WT + nb * 8192;
+        const uint32_t a2_row = sb + OFF_A2 + nb * 16384 + (64 + kr) * 128;
+#pragma unroll
+        for (int c32 = 0; c32 < 4; ++c32) {
+          const uint32_t a = tb_base + tc::sw128_b32(kr, c32);
+          st_tf32x4(a, tb[8 * c32], tb[8 * c32 + 1], tb[8 * c32 + 2], tb[8 * c32 + 3]);
+          st_tf32x4(a + 16, tb[8 * c32 + 4], tb[8 * c32 + 5], tb[8 * c32 + 6], tb[8 * c32 + 7]);
+        }
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc)
+          st_tf32x4(a2_row + ((cc ^ (kr & 7)) << 4), tb[4 * cc], tb[4 * cc + 1], tb[4 * cc + 2],
+                    tb[4 * cc + 3]);
+      }
+      // P rows (threads 0..63): P[t][j] = exp(G_t - G_j) (q_t . k_j) scale, j <= t
+      {
+        float sv[32];
+        const int t = ptid;
+        const float gt = ptid < 64 ? gG[t] : 0.f;
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+          tc::tmem_ld32(tmem + lane_off + TM_S + 32 * p, sv);
+          tc::tmem_wait_ld();
+          if (ptid < 64) {
+            const uint32_t prow = sb + OFF_W + p * 8192 + t * 128;
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) {
+              float v[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int j = 32 * p + 4 * cc + e;
+                v[e] = (j <= t) ? __expf(gt - gG[j]) * sv[4 * cc + e] * scale : 0.f;
+              }
+              st_tf32x4(prow + ((cc ^ (t & 7)) << 4), v[0], v[1], v[2], v[3]);
+            }
+          }
         }
       }
       tc::tc_fence_before();
-      tc::named_bar(1, 128);
-      if (ptid == 0) tc::mbar_arrive(bar(B_S_EMPTY));
-      if (ptid < 64) {
-        const int t = ptid;
-        const float gt = gG[t];
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          float pv[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int j = 8 * cc + e;
-            pv[e] = (j <= t) ? expf(gt - gG[j]) * sv[j] * scale : 0.f;
-          }
-          tc::st_shared_v4(sb + OFF_PI + tc::sw128(t, cc), tc::pack_bf16(pv[0], pv[1]),
-                           tc::pack_bf16(pv[2], pv[3]), tc::pack_bf16(pv[4], pv[5]),
-                           tc::pack_bf16(pv[6], pv[7]));
-        }
-      } else {
-        const int t = ptid - 64;
-        const float gt = gG[t], bt = gBeta[t];
-#pragma unroll
-        for (int j4 = 0; j4 < 64; j4 += 4) {
-          float4 av;
-          av.x = (j4 + 0 < t) ? bt * expf(gt - gG[j4 + 0]) * sv[j4 + 0] : 0.f;
-          av.y = (j4 + 1 < t) ? bt * expf(gt - gG[j4 + 1]) * sv[j4 + 1] : 0.f;
-          av.z = (j4 + 2 < t) ? bt * expf(gt - gG[j4 + 2]) * sv[j4 + 2] : 0.f;
-          av.w = (j4 + 3 < t) ? bt * expf(gt - gG[j4 + 3]) * sv[j4 + 3] : 0.f;
-          *reinterpret_cast<float4*>(&sA[t * LDA + j4]) = av;
-        }
-      }
-      tc::named_bar(1, 128);
-      solve_unit_lower(sA, sT, ptid);
-      {   // T_b = T diag(beta) as the bf16 B operand of [P; I] T_b (row k, 64 columns)
-        const int k = ptid >> 1, n0 = (ptid & 1) * 32;
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          float tv[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int n = n0 + 8 * cc + e;
-            tv[e] = (n <= k) ? sT[k * LDA + n] * gBeta[n] : 0.f;
-          }
-          tc::st_shared_v4(sb + OFF_TB + tc::sw128(k, (n0 >> 3) + cc), tc::pack_bf16(tv[0], tv[1]),
-                           tc::pack_bf16(tv[2], tv[3]), tc::pack_bf16(tv[4], tv[5]),
-                           tc::pack_bf16(tv[6], tv[7]));
-        }
-      }
       tc::fence_proxy_async_smem();
       tc::named_bar(1, 128);
-      if (ptid == 0) tc::mbar_arrive(bar(B_PT_READY));
-      // A2 = [P T_b; T_b] from TMEM, Ktil from the K tile
+      if (ptid == 0) {
+        tc::mbar_arrive(bar(B_S_EMPTY));
+        tc::mbar_arrive(bar(B_PT_READY));
+        GDN_TRACE(c, 6);
+      }
+      // A2 rows 0..63 = P T_b (64-row MMA: row r sits in lane (r % 16) + 32 (r / 16))
       tc::mbar_wait(bar(B_PT_FULL), c & 1, abort_flag, kBudgetNs);
+      if (ptid == 0) GDN_TRACE(c, 7);
       tc::tc_fence_after();
-      float pt[64];
       {
-        float a16[16];
+        float pv[32];
+        const int r = 16 * q + lane;
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          tmem_ld16(tmem + lane_off + TM_PT + 16 * p, a16);
+        for (int p = 0; p < 2; ++p) {
+          tc::tmem_ld32(tmem + lane_off + TM_PT + 32 * p, pv);
           tc::tmem_wait_ld();
+          if (lane < 16) {
+            const uint32_t a2_row = sb + OFF_A2 + p * 16384 + r * 128;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) pt[16 * p + i] = a16[i];
+            for (int cc = 0; cc < 8; ++cc)
+              st_tf32x4(a2_row + ((cc ^ (r & 7)) << 4), pv[4 * cc], pv[4 * cc + 1], pv[4 * cc + 2],
+                        pv[4 * cc + 3]);
+          }
         }
       }
       tc::tc_fence_before();
-      if (c >= 1) tc::mbar_wait(bar(B_A2_EMPTY), (c - 1) & 1, abort_flag, kBudgetNs);
-#pragma unroll
-      for (int cc = 0; cc < 8; ++cc)
-        tc::st_shared_v4(sb + OFF_A2 + tc::sw128(ptid, cc), tc::pack_bf16(pt[8 * cc], pt[8 * cc + 1]),
-                         tc::pack_bf16(pt[8 * cc + 2], pt[8 * cc + 3]),
-                         tc::pack_bf16(pt[8 * cc + 4], pt[8 * cc + 5]),
-                         tc::pack_bf16(pt[8 * cc + 6], pt[8 * cc + 7]));
-      tc::mbar_wait(bar(B_QK_FULL + s), (c >> 1) & 1, abort_flag, kBudgetNs);
-      if (c >= 1) tc::mbar_wait(bar(B_KT_EMPTY), (c - 1) & 1, abort_flag, kBudgetNs);
-      {
-        const int t = ptid >> 1, kb = ptid & 1;
-        const float f = gKt[t];
-        const uint32_t src = sb + OFF_QK + s * QK_STAGE + kb * 16384 + 8192 + t * 128;
-        const uint32_t dst = sb + OFF_KT + kb * 8192 + t * 128;
-#pragma unroll
-        for (int pc = 0; pc < 8; ++pc) {   // same swizzle on both sides: copy chunk positions
-          const uint4 u = tc::ld_shared_v4(src + pc * 16);
-          tc::st_shared_v4(dst + pc * 16, tc::pack_bf16(tc::bf16lo(u.x) * f, tc::bf16hi(u.x) * f),
-                           tc::pack_bf16(tc::bf16lo(u.y) * f, tc::bf16hi(u.y) * f),
-                           tc::pack_bf16(tc::bf16lo(u.z) * f, tc::bf16hi(u.z) * f),
-                           tc::pack_bf16(tc::bf16lo(u.w) * f, tc::bf16hi(u.w) * f));
-        }
-      }
       tc::fence_proxy_async_smem();
       const bool stop = vote_abort(1, 128, abort_flag);
       if (ptid == 0) {
         tc::mbar_arrive(bar(B_PRE_FULL));
-        tc::mbar_arrive(bar(B_IN_EMPTY + s));
         tc::mbar_arrive(bar(B_PT_EMPTY));
+        GDN_TRACE(c, 8);
       }
       if (stop) break;
     }
@@ -588,7 +631,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     const int hh = (warp - 8) >> 2, q = warp & 3, r = 32 * q + lane;
     const int hb = B_HALF + H_COUNT * hh;
     const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
-    const uint32_t mb = sb + OFF_MB + hh * 16384, rd = sb + OFF_RD + hh * 8192;
+    const uint32_t mb = sb + OFF_MB + hh * 16384, rd = sb + OFF_RD + hh * 16384;
+    const uint32_t vb = sb + OFF_V + hh * 8192;
     const uint32_t id_wg = 2 + 3 * hh, id_lo = 3 + 3 * hh, id_hi = 4 + 3 * hh;
     const long head = (long)bq * Hv + h;
     float M[64];
@@ -617,42 +661,50 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       const int slot = c % 3;
       const long t0 = (long)c * C;
       const float* gGam = reinterpret_cast<const float*>(smem + OFF_GB + slot * 1024) + 64;
+      const float* gKt = gGam + 64;
       if (q >= 2) {
-        // R' = V - gamma (K M) for token t, then Delta
+        // R' = V - gamma (K M) for token t (tf32), then ktil Delta as bf16 hi + lo
         const int t = r - 64;
         tc::mbar_wait(bar(hb + H_X_FULL), c & 1, abort_flag, kBudgetNs);
         tc::mbar_wait(bar(B_GATE + slot), (c / 3) & 1, abort_flag, kBudgetNs);
-        tc::mbar_wait(bar(B_V_FULL), c & 1, abort_flag, kBudgetNs);
+        tc::mbar_wait(bar(hb + H_V_FULL), c & 1, abort_flag, kBudgetNs);
+        if (q == 2 && lane == 0) GDN_TRACE(c, 20 + 10 * hh);
         tc::tc_fence_after();
         const float g = gGam[t];
-        const uint32_t vrow = sb + OFF_V + hh * 8192;
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
+        for (int p = 0; p < 4; ++p) {          // 16 columns: dv 16p .. 16p+15 of this half
           float x[16];
           tmem_ld16(tmem + lane_off + TM_X + 64 * hh + 16 * p, x);
           tc::tmem_wait_ld();
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
-            const int cc = 2 * p + half;
-            const uint4 u = tc::ld_shared_v4(vrow + tc::sw128(t, cc));
+            const int cc = 2 * p + half;       // bf16 chunk of V (8 values)
+            const uint4 u = tc::ld_shared_v4(vb + tc::sw128(t, cc));
             const float* xx = x + 8 * half;
-            tc::st_shared_v4(rd + tc::sw128(t, cc),
-                             tc::pack_bf16(tc::bf16lo(u.x) - g * xx[0], tc::bf16hi(u.x) - g * xx[1]),
-                             tc::pack_bf16(tc::bf16lo(u.y) - g * xx[2], tc::bf16hi(u.y) - g * xx[3]),
-                             tc::pack_bf16(tc::bf16lo(u.z) - g * xx[4], tc::bf16hi(u.z) - g * xx[5]),
-                             tc::pack_bf16(tc::bf16lo(u.w) - g * xx[6], tc::bf16hi(u.w) - g * xx[7]));
+            const float rv[8] = {tc::bf16lo(u.x) - g * xx[0], tc::bf16hi(u.x) - g * xx[1],
+                                 tc::bf16lo(u.y) - g * xx[2], tc::bf16hi(u.y) - g * xx[3],
+                                 tc::bf16lo(u.z) - g * xx[4], tc::bf16hi(u.z) - g * xx[5],
+                                 tc::bf16lo(u.w) - g * xx[6], tc::bf16hi(u.w) - g * xx[7]};
+            // MN-major tf32 layout: dv block nb = col / 32, 32-byte chunk (col % 32) / 8
+            const int col = 8 * cc, nb = col >> 5, c32 = (col & 31) >> 3;
+            const uint32_t a = rd + nb * 8192 + tc::sw128_b32(t, c32);
+            st_tf32x4(a, rv[0], rv[1], rv[2], rv[3]);
+            st_tf32x4(a + 16, rv[4], rv[5], rv[6], rv[7]);
           }
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
         tc::named_bar(id_hi, 64);
         if (q == 2 && lane == 0) {
+          GDN_TRACE(c, 21 + 10 * hh);
           tc::mbar_arrive(bar(hb + H_R_FULL));
-          tc::mbar_arrive(bar(B_V_EMPTY));
+          tc::mbar_arrive(bar(hb + H_V_EMPTY));
           tc::mbar_arrive(bar(hb + H_X_EMPTY));
         }
         tc::mbar_wait(bar(hb + H_Y_FULL), c & 1, abort_flag, kBudgetNs);
+        if (q == 2 && lane == 0) GDN_TRACE(c, 22 + 10 * hh);
         tc::tc_fence_after();
+        const float kt = gKt[t];
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
           float y[16];
@@ -660,16 +712,21 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
           tc::tmem_wait_ld();
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
-            const float* yy = y + 8 * half;
-            tc::st_shared_v4(rd + tc::sw128(t, 2 * p + half), tc::pack_bf16(yy[0], yy[1]),
-                             tc::pack_bf16(yy[2], yy[3]), tc::pack_bf16(yy[4], yy[5]),
-                             tc::pack_bf16(yy[6], yy[7]));
+            float hi[8], lo[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) tc::split_bf16(kt * y[8 * half + e], hi[e], lo[e]);
+            const uint32_t sw = tc::sw128(t, 2 * p + half);
+            tc::st_shared_v4(rd + sw, tc::pack_bf16(hi[0], hi[1]), tc::pack_bf16(hi[2], hi[3]),
+                             tc::pack_bf16(hi[4], hi[5]), tc::pack_bf16(hi[6], hi[7]));
+            tc::st_shared_v4(rd + 8192 + sw, tc::pack_bf16(lo[0], lo[1]), tc::pack_bf16(lo[2], lo[3]),
+                             tc::pack_bf16(lo[4], lo[5]), tc::pack_bf16(lo[6], lo[7]));
           }
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
         tc::named_bar(id_hi, 64);
         if (q == 2 && lane == 0) {
+          GDN_TRACE(c, 23 + 10 * hh);
           tc::mbar_arrive(bar(hb + H_D_FULL));
           tc::mbar_arrive(bar(hb + H_Y_EMPTY));
         }
@@ -679,6 +736,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         tc::mbar_wait(bar(hb + H_X_FULL), c & 1, abort_flag, kBudgetNs);
         tc::mbar_wait(bar(B_GATE + slot), (c / 3) & 1, abort_flag, kBudgetNs);
         tc::mbar_wait(bar(hb + H_Y_FULL), c & 1, abort_flag, kBudgetNs);
+        if (q == 0 && lane == 0) GDN_TRACE(c, 24 + 10 * hh);
         tc::tc_fence_after();
         const float g = gGam[t] * scale;
         const bool valid = t0 + t < T;
@@ -696,12 +754,14 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         tc::tc_fence_before();
         tc::named_bar(id_lo, 64);
         if (q == 0 && lane == 0) {
+          GDN_TRACE(c, 25 + 10 * hh);
           tc::mbar_arrive(bar(hb + H_X_EMPTY));
           tc::mbar_arrive(bar(hb + H_Y_EMPTY));
         }
       }
-      // M <- gamma_last M + Ktil^T Delta  (row r of this half), and its bf16 copy for the MMAs
+      // M <- gamma_last M + K^T (ktil Delta)  (row r of this half), and its bf16 copy
       tc::mbar_wait(bar(hb + H_D3_FULL), c & 1, abort_flag, kBudgetNs);
+      if (q == 0 && lane == 0) GDN_TRACE(c, 26 + 10 * hh);
       tc::tc_fence_after();
       const float gl = gGam[63];
 #pragma unroll
@@ -723,6 +783,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       tc::tc_fence_before();
       const bool stop = vote_abort(id_wg, 128, abort_flag);
       if (q == 0 && lane == 0) {
+        GDN_TRACE(c, 27 + 10 * hh);
         tc::mbar_arrive(bar(hb + H_D3_EMPTY));
         tc::mbar_arrive(bar(hb + H_M_READY));
       }
@@ -795,6 +856,12 @@ gdn_status launch(const void* q, const void* k, const void* v, const float* la, 
 }
 
 }  // namespace tcf
+
+#ifdef GDN_TC_TRACE
+extern "C" GDN_API void gdn_debug_set_trace(void* p) {
+  cudaMemcpyToSymbol(tcf::g_tc_trace, &p, sizeof(p));
+}
+#endif
 
 inline bool tc_chunk_supported(int dk, int dv, int chunk, bool bf16) {
   return bf16 && dk == 128 && dv == 128 && chunk == tcf::C;

@@ -8,8 +8,11 @@
 //   K) in 1024-byte groups of 8 rows (stride byte offset = 1024); an MN-major operand is rows of
 //   64 MN-contiguous bf16, one row per K index, 8-row groups 1024 bytes apart (stride byte
 //   offset) and 64-wide MN blocks `lbo` bytes apart (leading byte offset).
+//   MN-major operands of 32-bit elements (tf32) use the other 128-byte layout (type 1): 32-byte
+//   chunks XORed with (row & 3), so K rows come in 512-byte groups of 4.
 //   instruction descriptor (kind::f16): [4,6) D format (1 = f32), [7,10) A format (1 = bf16),
-//   [10,13) B format, [15] A MN-major, [16] B MN-major, [17,23) N >> 3, [24,29) M >> 4.
+//   [10,13) B format, [15] A MN-major, [16] B MN-major, [17,23) N >> 3, [24,29) M >> 4;
+//   kind::tf32 uses format 2 for A and B.
 #pragma once
 
 #include <stdint.h>
@@ -45,6 +48,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Same, but the thread may be suspended in hardware until the phase completes or `hint_ns`
+// passes, so waiting warps take no issue slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
@@ -54,16 +71,17 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Bounded wait: returns false if `abort` was raised by another thread or if `budget_ns` passed
-// (then it raises `abort` itself).  Never spins forever.
+// Bounded wait: returns false if `abort` was raised by another thread or once `budget_cycles`
+// SM clock cycles passed (it then raises `abort` itself).  Never spins forever: each poll
+// suspends the thread for up to 50 us unless the phase completes first.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                          uint64_t budget_ns) {
+                                          uint64_t budget_cycles) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  const long long t0 = clock64();
   for (;;) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 50000u)) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > budget_ns) {
+    if ((uint64_t)(clock64() - t0) > budget_cycles) {
       *abort = 1;
       return false;
     }
@@ -117,13 +135,24 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem desc] * B[smem desc], bf16 inputs, fp32 accumulate; one thread issues.
+// D[tmem] (+)= A[smem desc] * B[smem desc], bf16 inputs (K = 16 per instruction), fp32
+// accumulate; one thread issues.
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                          uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Same with tf32 inputs read from fp32 words (K = 8 per instruction).
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
@@ -157,24 +186,48 @@ __device__ __forceinline__ void tmem_wait_ld() {
 // ---------------------------------------------------------------------------------------------
 // descriptors
 // ---------------------------------------------------------------------------------------------
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
+                                          uint32_t layout) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
   d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
   d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
   d |= (uint64_t)1 << 46;     // descriptor version for sm_100
-  d |= (uint64_t)2 << 61;     // 128-byte swizzle
+  d |= (uint64_t)layout << 61;
   return d;
+}
+// 128-byte swizzle, 16-byte chunks (bf16 operands, K-major tf32 operands)
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return sdesc(saddr, lbo, sbo, 2);
+}
+// 128-byte swizzle on 32-byte chunks (MN-major tf32 operands); K groups of 4 rows (512 bytes)
+__device__ __forceinline__ uint64_t sdesc_sw128_b32(uint32_t saddr, uint32_t lbo) {
+  return sdesc(saddr, lbo, 512, 1);
 }
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) |
          ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// kind::tf32: A and B format 2 (tf32), D format f32.
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((a_mn ? 1u : 0u) << 15) |
+         ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// Round an fp32 value to tf32 (nearest, ties away), kept in an fp32 word with 13 low bits zero.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
 }
 
 // Byte offset of 16-byte chunk `c` (0..7) of row `r` in a 128-byte-swizzled tile whose base is
 // 1024-byte aligned: the chunk index is XORed with the row's position in its 8-row group.
 __device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t c) {
   return r * 128u + ((c ^ (r & 7u)) << 4);
+}
+// Byte offset of 32-byte chunk `c` (0..3) of row `r` in the 32-byte-chunk layout (type 1).
+__device__ __forceinline__ uint32_t sw128_b32(uint32_t r, uint32_t c) {
+  return r * 128u + ((c ^ (r & 3u)) << 5);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -194,6 +247,11 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
                : "r"(addr)
                : "memory");
   return v;
+}
+// Split x into a bf16 head and the bf16 rounding of its remainder: x ~= hi + lo to ~2^-16.
+__device__ __forceinline__ void split_bf16(float x, float& hi, float& lo) {
+  hi = __bfloat162float(__float2bfloat16_rn(x));
+  lo = x - hi;
 }
 __device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
