@@ -57,8 +57,10 @@ constexpr uint32_t OFF_MB = 147456;     // per half 16 KB: bf16 M [128 dk rows][
 constexpr uint32_t OFF_W = 180224;      // 32 KB: solve scratch, then P (tf32) and T_b (tf32)
 constexpr uint32_t OFF_WT = OFF_W + 16384;   // T_b, [dv block][64 rows][128 B]
 constexpr uint32_t SOLVE_T = 12800;     // byte offset of T inside the solve scratch
-constexpr uint32_t OFF_GB = 212992;     // 3 slots x 1 KB: G[64], gamma[64], ktil[64], beta[64]
-constexpr uint32_t OFF_BAR = 216064;
+constexpr uint32_t OFF_GB = 212992;     // 3 slots x 2 KB: G log2(e)[64], gamma[64], ktil[64],
+                                        // beta[64], E[4][64] (E[b][j] = exp(G_16b - G_j), j < 16b)
+constexpr uint32_t GB_SLOT = 2048;
+constexpr uint32_t OFF_BAR = OFF_GB + 3 * GB_SLOT;
 constexpr int NBAR = 40;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;   // +0 TMEM base, +4 abort flag
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16;
@@ -129,23 +131,24 @@ __device__ __forceinline__ void strip16(const float* X, int xr, const float* Y, 
 //   D_b = (I + A_bb)^-1 by forward substitution (one column per thread);
 //   At_ik = D_i A_ik;  U = (I + At)^-1 by block forward substitution (U_ii = I);  T_ik = U_ik D_k.
 // (I + A = blockdiag(I + A_bb) (I + At), so T = U D.)  sA is overwritten with At.
-__device__ void solve_unit_lower(float* sA, float* sT, int ptid) {
+__device__ void solve_unit_lower(float* sA, float* sT, int ptid, int c, int nC) {
   if (ptid < 64) {
-    const int b = ptid >> 4, c = ptid & 15;
+    const int b = ptid >> 4, col = ptid & 15;
     const float* Ab = blk(sA, b, b);
     float x[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      float acc = (i == c) ? 1.f : 0.f;
+      float acc = (i == col) ? 1.f : 0.f;
 #pragma unroll
       for (int j = 0; j < i; ++j) acc = fmaf(-Ab[i * BLD + j], x[j], acc);
       x[i] = acc;
     }
     float* Tb = blk(sT, b, b);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) Tb[i * BLD + c] = x[i];
+    for (int i = 0; i < 16; ++i) Tb[i * BLD + col] = x[i];
   }
   tc::named_bar(1, 128);
+  if (ptid == 0) GDN_TRACE(c, 44);
   // block index bi = 0..5 -> (i, k) = (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
   auto blk_i = [](int bi) { return bi < 1 ? 1 : (bi < 3 ? 2 : 3); };
   auto blk_k = [](int bi, int i) { return bi - i * (i - 1) / 2; };
@@ -166,6 +169,7 @@ __device__ void solve_unit_lower(float* sA, float* sT, int ptid) {
         make_float4(r1[m][0], r1[m][1], r1[m][2], r1[m][3]);
   }
   tc::named_bar(1, 128);
+  if (ptid == 0) GDN_TRACE(c, 45);
   // U_20 = -At_20 + At_21 At_10;  U_31 = -At_31 + At_32 At_21;  V_30 = -At_30 + At_31 At_10
   for (int id = ptid; id < 192; id += 128) {
     const int bi = id >> 6, r = (id >> 2) & 15, cs = id & 3;
@@ -187,6 +191,7 @@ __device__ void solve_unit_lower(float* sA, float* sT, int ptid) {
     *dst = make_float4(v30.x - acc[0], v30.y - acc[1], v30.z - acc[2], v30.w - acc[3]);
   }
   tc::named_bar(1, 128);
+  if (ptid == 0) GDN_TRACE(c, 46);
   float r4[3][4];
 #pragma unroll
   for (int m = 0; m < 3; ++m) {                       // T_ik = U_ik D_k (U = -At next to diag)
@@ -271,9 +276,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
                     const float* __restrict__ beta, const float* __restrict__ S0,
                     Tout* __restrict__ o, float* __restrict__ S_T, int T, int Hk, int Hv,
                     float scale) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // Offsetting the __shared__ array itself (not a round trip through an integer) keeps every
+  // access below a shared-memory access (ld/st.shared), not a generic one.
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sb = tc::smem_u32(smem);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -476,10 +482,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     for (int c = 0; c < nC; ++c) {
       const int slot = c % 3;
       if (ptid == 0) GDN_TRACE(c, 0);
-      float* gG = reinterpret_cast<float*>(smem + OFF_GB + slot * 1024);
+      float* gG = reinterpret_cast<float*>(smem + OFF_GB + slot * GB_SLOT);
       float* gGam = gG + 64;
       float* gKt = gG + 128;
       float* gBeta = gG + 192;
+      float* gE = gG + 256;
       if (ptid < 32) {          // gates of this chunk: lane l holds tokens 2l, 2l+1
         const float la0 = pla0, la1 = pla1, be0 = pbe0, be1 = pbe1;
         if (c + 1 < nC) load_gates(c + 1);
@@ -491,52 +498,105 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         }
         const float g1 = incl, g0 = incl - la1;
         const float gl = __shfl_sync(0xffffffffu, incl, 31);
-        gG[2 * lane] = g0;             gG[2 * lane + 1] = g1;
+        constexpr float kLog2e = 1.4426950408889634f;
+        gG[2 * lane] = g0 * kLog2e;    gG[2 * lane + 1] = g1 * kLog2e;
         gGam[2 * lane] = expf(g0);     gGam[2 * lane + 1] = expf(g1);
         gKt[2 * lane] = expf(gl - g0); gKt[2 * lane + 1] = expf(gl - g1);
         gBeta[2 * lane] = be0;         gBeta[2 * lane + 1] = be1;
+        // block factors E[b][j] = exp(G_16b - G_j) for j < 16b (each <= 1: G never increases)
+#pragma unroll
+        for (int b = 1; b < 4; ++b) {
+          const float gb = __shfl_sync(0xffffffffu, g0, 8 * b) * kLog2e;   // G at token 16b
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int j = 2 * lane + e;
+            const float gj = (e ? g1 : g0) * kLog2e;
+            gE[64 * b + j] = (j < 16 * b) ? tc::ex2(gb - gj) : 0.f;
+          }
+        }
         __syncwarp();
         __threadfence_block();
         if (lane == 0) tc::mbar_arrive(bar(B_GATE + slot));
       }
       tc::named_bar(1, 128);
       if (ptid == 0) GDN_TRACE(c, 1);
-      // A rows (threads 64..127): A[t][j] = beta_t exp(G_t - G_j) (k_t . k_j), j < t
+      // Rows of S: threads 0..63 hold (q_t . k_j), threads 64..127 hold (k_t . k_j).  Both
+      // halves turn their row into P or A at once; exp(G_t - G_j) = 2^(G'_t - G'_j), G' = G log2 e.
+      //   P[t][j] = exp(G_t - G_j) (q_t . k_j) scale, j <= t  (kept in the same TMEM row, as fp32,
+      //             until the solve scratch is free for the tf32 copy)
+      //   A[t][j] = beta_t exp(G_t - G_j) (k_t . k_j),  j < t  (into the packed solve blocks)
       tc::mbar_wait(bar(B_S_FULL), c & 1, abort_flag, kBudgetNs);
       if (ptid == 0) GDN_TRACE(c, 2);
       tc::tc_fence_after();
       {
-        float sv[32];
-        const int t = ptid - 64, ti = t >> 4, tr = t & 15;
-        const float gt = ptid >= 64 ? gG[t] : 0.f, bt = ptid >= 64 ? gBeta[t] : 0.f;
+        const bool is_p = ptid < 64;
+        const int t = is_p ? ptid : ptid - 64, ti = t >> 4, tr = t & 15;
+        const float gt = gG[t];
+        const float coef = is_p ? scale : gBeta[t];
+        // exp(G_t - G_j): inside t's 16-token block directly; across blocks as
+        // exp(G_t - G_16ti) * E[ti][j] (both factors <= 1)
+        const float et = tc::ex2(gt - gG[16 * ti]);
+        const float4* g4 = reinterpret_cast<const float4*>(gG);
+        const float4* e4p = reinterpret_cast<const float4*>(gE + 64 * ti);
+        const int lim = is_p ? t + 1 : t;            // column j is kept when j < lim
 #pragma unroll
         for (int p = 0; p < 2; ++p) {
+          float sv[32];
           tc::tmem_ld32(tmem + lane_off + TM_S + 32 * p, sv);
           tc::tmem_wait_ld();
-          if (ptid >= 64) {
+          if (ptid == 64 + 48) GDN_TRACE(c, 53 + 2 * p);
+#pragma unroll
+          for (int kb2 = 0; kb2 < 2; ++kb2) {
+            const int kb = 2 * p + kb2;
+            float* v = sv + 16 * kb2;
+            if (kb < ti) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float4 e = e4p[4 * kb + i];
+                v[4 * i] *= coef * et * e.x;     v[4 * i + 1] *= coef * et * e.y;
+                v[4 * i + 2] *= coef * et * e.z; v[4 * i + 3] *= coef * et * e.w;
+              }
+            } else if (kb == ti) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float4 g = g4[4 * kb + i];
+                const float gj[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int j = 16 * kb + 4 * i + e;
+                  v[4 * i + e] = (j < lim) ? coef * tc::ex2(gt - gj[e]) * v[4 * i + e] : 0.f;
+                }
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) v[e] = 0.f;
+            }
+          }
+          if (is_p) {
+            tc::tmem_st32(tmem + lane_off + TM_S + 32 * p, sv);
+          } else {
 #pragma unroll
             for (int kb2 = 0; kb2 < 2; ++kb2) {
               const int kb = 2 * p + kb2;
               if (kb <= ti) {
                 float* dst = blk(sA, ti, kb) + tr * BLD;
 #pragma unroll
-                for (int e4 = 0; e4 < 16; e4 += 4) {
-                  float a[4];
-#pragma unroll
-                  for (int e = 0; e < 4; ++e) {
-                    const int j = 16 * kb + e4 + e;
-                    a[e] = (j < t) ? bt * __expf(gt - gG[j]) * sv[16 * kb2 + e4 + e] : 0.f;
-                  }
-                  *reinterpret_cast<float4*>(dst + e4) = make_float4(a[0], a[1], a[2], a[3]);
-                }
+                for (int e4 = 0; e4 < 16; e4 += 4)
+                  *reinterpret_cast<float4*>(dst + e4) =
+                      make_float4(sv[16 * kb2 + e4], sv[16 * kb2 + e4 + 1], sv[16 * kb2 + e4 + 2],
+                                  sv[16 * kb2 + e4 + 3]);
               }
             }
           }
+          if (ptid == 64 + 48) GDN_TRACE(c, 54 + 2 * p);
         }
+        if (is_p) tc::tmem_wait_st();
+        if (ptid == 48) GDN_TRACE(c, 57);
       }
+      tc::tc_fence_before();
       tc::named_bar(1, 128);
       if (ptid == 0) GDN_TRACE(c, 3);
-      solve_unit_lower(sA, sT, ptid);
+      solve_unit_lower(sA, sT, ptid, c, nC);
       if (ptid == 0) GDN_TRACE(c, 4);
       // T_b = T diag(beta): row k = ptid/2, columns n0..n0+31 (one tf32 column block)
       float tb[32];
@@ -546,8 +606,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         const int n = 32 * nb + e;
         tb[e] = (n <= kr) ? blk(sT, kr >> 4, n >> 4)[(kr & 15) * BLD + (n & 15)] * gBeta[n] : 0.f;
       }
+      if (ptid == 0) GDN_TRACE(c, 48);
       if (c >= 1) tc::mbar_wait(bar(B_A2_EMPTY), (c - 1) & 1, abort_flag, kBudgetNs);
+      if (ptid == 0) GDN_TRACE(c, 49);
       tc::named_bar(1, 128);                     // the solve scratch is free from here on
+      if (ptid == 0) GDN_TRACE(c, 50);
       {
         // T_b as the MN-major B operand of P T_b (32-byte chunks), and as rows 64..127 of the
         // K-major A2 (16-byte chunks)
@@ -564,30 +627,24 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
           st_tf32x4(a2_row + ((cc ^ (kr & 7)) << 4), tb[4 * cc], tb[4 * cc + 1], tb[4 * cc + 2],
                     tb[4 * cc + 3]);
       }
-      // P rows (threads 0..63): P[t][j] = exp(G_t - G_j) (q_t . k_j) scale, j <= t
-      {
-        float sv[32];
+      if (ptid == 0) GDN_TRACE(c, 51);
+      // P rows (threads 0..63, warps 4 and 5): back from TMEM, rounded to tf32, into the K-major
+      // A operand of P T_b
+      if (ptid < 64) {
         const int t = ptid;
-        const float gt = ptid < 64 ? gG[t] : 0.f;
 #pragma unroll
         for (int p = 0; p < 2; ++p) {
-          tc::tmem_ld32(tmem + lane_off + TM_S + 32 * p, sv);
+          float pv[32];
+          tc::tmem_ld32(tmem + lane_off + TM_S + 32 * p, pv);
           tc::tmem_wait_ld();
-          if (ptid < 64) {
-            const uint32_t prow = sb + OFF_W + p * 8192 + t * 128;
+          const uint32_t prow = sb + OFF_W + p * 8192 + t * 128;
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-              float v[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int j = 32 * p + 4 * cc + e;
-                v[e] = (j <= t) ? __expf(gt - gG[j]) * sv[4 * cc + e] * scale : 0.f;
-              }
-              st_tf32x4(prow + ((cc ^ (t & 7)) << 4), v[0], v[1], v[2], v[3]);
-            }
-          }
+          for (int cc = 0; cc < 8; ++cc)
+            st_tf32x4(prow + ((cc ^ (t & 7)) << 4), pv[4 * cc], pv[4 * cc + 1], pv[4 * cc + 2],
+                      pv[4 * cc + 3]);
         }
       }
+      if (ptid == 0) GDN_TRACE(c, 52);
       tc::tc_fence_before();
       tc::fence_proxy_async_smem();
       tc::named_bar(1, 128);
@@ -660,7 +717,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     for (int c = 0; c < nC; ++c) {
       const int slot = c % 3;
       const long t0 = (long)c * C;
-      const float* gGam = reinterpret_cast<const float*>(smem + OFF_GB + slot * 1024) + 64;
+      const float* gGam = reinterpret_cast<const float*>(smem + OFF_GB + slot * GB_SLOT) + 64;
       const float* gKt = gGam + 64;
       if (q >= 2) {
         // R' = V - gamma (K M) for token t (tf32), then ktil Delta as bf16 hi + lo
@@ -747,10 +804,13 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
           tmem_ld16(tmem + lane_off + TM_X + 64 * hh + 16 * p, x);
           tmem_ld16(tmem + lane_off + TM_Y + 64 * hh + 16 * p, y);
           tc::tmem_wait_ld();
+          if (p == 0 && hh == 0 && q == 0 && lane == 0) GDN_TRACE(c, 58);
 #pragma unroll
           for (int i = 0; i < 16; ++i) y[i] = fmaf(g, x[i], y[i]);
           if (valid) store16<Tout>(orow + 16 * p, y);
+          if (p == 0 && hh == 0 && q == 0 && lane == 0) GDN_TRACE(c, 59);
         }
+        if (hh == 0 && q == 0 && lane == 0) GDN_TRACE(c, 60);
         tc::tc_fence_before();
         tc::named_bar(id_lo, 64);
         if (q == 0 && lane == 0) {
