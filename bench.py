@@ -415,6 +415,23 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def profile_case(args):
+    """A few launches of the chunked forward on one workload, nothing else (for profilers)."""
+    import gated_deltanet_linear_18_b200 as gdn
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = gi.WORKLOADS[args.profile_case]
+    kw = {k: v for k, v in (("B", args.B), ("T", args.T)) if v is not None}
+    if kw:
+        w = w.with_sizes(**kw)
+    step = prefill_fn(gdn, to_dev(gi.make_inputs(w), dev), w)
+    for _ in range(args.steps):
+        step()
+    torch.cuda.synchronize()
+    gdn.check_error(dev)
+    print(json.dumps({"profile_case": workload_name(w), "launches": args.steps}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -424,7 +441,14 @@ def main():
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the decode / long-context / layer lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", metavar="WORKLOAD", default=None,
+                    help="no timing: run the chunked forward --steps times on WORKLOAD (sizes "
+                         "from --B/--T) and exit; a small, fixed command for ncu captures")
+    ap.add_argument("--B", type=int, default=None)
+    ap.add_argument("--T", type=int, default=None)
     args = ap.parse_args()
+    if args.profile_case:
+        return profile_case(args)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 

@@ -12,10 +12,48 @@
 
 namespace gdn {
 
-constexpr int kPrologueTokens = 64;     // tokens per CTA
-constexpr int kPrologueGroup = 8;       // tokens reduced together per barrier
+constexpr int kPrologueTokens = 256;    // tokens per CTA
 
-// grid: (ceil(T / 64), 2*Hk + Hv, B); block: 128 threads, thread = channel within the head.
+// Vectors of 16 bytes: 8 bf16 or 4 fp32 values.
+template <typename T> struct Vec16;
+template <> struct Vec16<float> {
+  static constexpr int N = 4;
+  static __device__ __forceinline__ void load(const float* p, float (&v)[4]) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  }
+  static __device__ __forceinline__ void store(float* p, const float (&v)[4]) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+};
+template <> struct Vec16<__nv_bfloat16> {
+  static constexpr int N = 8;
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[8]) {
+    const uint4 a = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[8]) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+      w[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+};
+
+__device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
+
+// grid: (ceil(T / 256), 2*Hk + Hv, B); block: 128 threads.  A head row of d channels is held by
+// L = d / N threads (N channels each, one 16-byte load per token); the 128 / L row groups of the
+// CTA take consecutive spans of 256 L / 128 tokens, each span starting from its own 3-token conv
+// history.  The L2 norm of a q or k row is a shuffle reduction over its L threads.
 template <typename Tio>
 __global__ void __launch_bounds__(128)
 prologue_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
@@ -23,9 +61,9 @@ prologue_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
                 const float* __restrict__ wk, const float* __restrict__ wv,
                 Tio* __restrict__ yq, Tio* __restrict__ yk, Tio* __restrict__ yv, int T, int Hk,
                 int Hv, int dk, int dv, float eps) {
+  constexpr int N = Vec16<Tio>::N;
   const int slot = blockIdx.y;
   const long b = blockIdx.z;
-  const int c = threadIdx.x;
   const Tio* x;
   const float* w;
   Tio* y;
@@ -38,52 +76,76 @@ prologue_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
   } else {
     x = xv; w = wv; y = yv; d = dv; head = slot - 2 * Hk; width = Hv * dv; l2 = false;
   }
-  const bool active = c < d;
-  const long ch = (long)head * d + c;
-  float w0 = 0.f, w1 = 0.f, w2 = 0.f, w3 = 0.f;
-  if (active) { w0 = w[ch * 4 + 0]; w1 = w[ch * 4 + 1]; w2 = w[ch * 4 + 2]; w3 = w[ch * 4 + 3]; }
-
-  const long t0 = (long)blockIdx.x * kPrologueTokens;
-  const long tend = min((long)T, t0 + kPrologueTokens);
-  auto load = [&](long t) -> float {
-    return (active && t >= 0 && t < T) ? to_f(x[(b * T + t) * width + ch]) : 0.f;
-  };
-  float h3 = load(t0 - 3), h2 = load(t0 - 2), h1 = load(t0 - 1);   // x[t-3], x[t-2], x[t-1]
-
-  __shared__ float red[2][kPrologueGroup][4];
-  int buf = 0;
-  for (long tg = t0; tg < tend; tg += kPrologueGroup) {
-    float yv_[kPrologueGroup];
+  const int L = d / N;                        // 2 .. 32, a power of two
+  const int grp = threadIdx.x / L, lc = threadIdx.x % L;
+  const int span = kPrologueTokens * L / 128;
+  const long c0 = (long)head * d + lc * N;    // first channel of this thread
+  float wt[N][4];
 #pragma unroll
-    for (int g = 0; g < kPrologueGroup; ++g) {
-      const float xt = load(tg + g);
-      const float pre = w0 * h3 + w1 * h2 + w2 * h1 + w3 * xt;
-      h3 = h2; h2 = h1; h1 = xt;
-      yv_[g] = active ? pre * sigmoidf_(pre) : 0.f;
+  for (int i = 0; i < N; ++i)                 // weights need only 4-byte alignment
+#pragma unroll
+    for (int j = 0; j < 4; ++j) wt[i][j] = w[(c0 + i) * 4 + j];
+  const long ts = (long)blockIdx.x * kPrologueTokens + (long)grp * span;
+  auto load = [&](long t, float (&v)[N]) {
+    if (t >= 0 && t < T) {
+      Vec16<Tio>::load(x + (b * T + t) * width + c0, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < N; ++i) v[i] = 0.f;
+    }
+  };
+  float h3[N], h2[N], h1[N];                  // x[t-3], x[t-2], x[t-1]
+  load(ts - 3, h3);
+  load(ts - 2, h2);
+  load(ts - 1, h1);
+#pragma unroll 4
+  for (int i = 0; i < span; ++i) {            // same trip count for every thread of the warp
+    const long t = ts + i;
+    float xt[N], yv_[N];
+    load(t, xt);
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+      const float pre = wt[j][0] * h3[j] + wt[j][1] * h2[j] + wt[j][2] * h1[j] + wt[j][3] * xt[j];
+      h3[j] = h2[j]; h2[j] = h1[j]; h1[j] = xt[j];
+      yv_[j] = silu_fast(pre);
+      ss += yv_[j] * yv_[j];
     }
     if (l2) {
+      for (int o = L >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float inv = rsqrtf(ss + eps);
 #pragma unroll
-      for (int g = 0; g < kPrologueGroup; ++g) {
-        const float s = warp_sum(yv_[g] * yv_[g]);
-        if ((c & 31) == 0) red[buf][g][c >> 5] = s;
-      }
-      __syncthreads();
-#pragma unroll
-      for (int g = 0; g < kPrologueGroup; ++g) {
-        const float ss = red[buf][g][0] + red[buf][g][1] + red[buf][g][2] + red[buf][g][3];
-        yv_[g] *= rsqrtf(ss + eps);
-      }
-      buf ^= 1;
+      for (int j = 0; j < N; ++j) yv_[j] *= inv;
     }
-    if (active) {
-#pragma unroll
-      for (int g = 0; g < kPrologueGroup; ++g)
-        if (tg + g < tend) y[(b * T + tg + g) * width + ch] = from_f<Tio>(yv_[g]);
-    }
+    if (t < T) Vec16<Tio>::store(y + (b * T + t) * width + c0, yv_);
   }
 }
 
-// One warp per row of dv <= 128 values.  `o` may be wider than z / y (the layer keeps o in fp32).
+// One warp per row of dv <= 128 values, 4 consecutive channels per lane.  `o` may be wider than
+// z / y (the layer keeps o in fp32).
+template <typename T4> struct Vec4;
+template <> struct Vec4<float> {
+  static __device__ __forceinline__ void load(const float* p, float (&v)[4]) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  }
+  static __device__ __forceinline__ void store(float* p, const float (&v)[4]) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+};
+template <> struct Vec4<__nv_bfloat16> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[4]) {
+    const uint2 a = *reinterpret_cast<const uint2*>(p);
+    v[0] = __uint_as_float(a.x << 16); v[1] = __uint_as_float(a.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(a.y << 16); v[3] = __uint_as_float(a.y & 0xFFFF0000u);
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[4]) {
+    __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]), h1 = __floats2bfloat162_rn(v[2], v[3]);
+    *reinterpret_cast<uint2*>(p) =
+        make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
+  }
+};
+
 template <typename To, typename Tio>
 __global__ void __launch_bounds__(256)
 out_norm_kernel(const To* __restrict__ o, const Tio* __restrict__ z, const float* __restrict__ w,
@@ -91,25 +153,22 @@ out_norm_kernel(const To* __restrict__ o, const Tio* __restrict__ z, const float
   const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
-  const To* orow = o + row * dv;
-  const Tio* zrow = z + row * dv;
-  float ov[4];
-  float ss = 0.f;
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const int cidx = lane + 32 * e;
-    ov[e] = cidx < dv ? to_f(orow[cidx]) : 0.f;
-    ss += ov[e] * ov[e];
+  const int c = 4 * lane;
+  const bool active = c < dv;
+  float ov[4] = {0.f, 0.f, 0.f, 0.f}, zv[4] = {0.f, 0.f, 0.f, 0.f};
+  if (active) {
+    Vec4<To>::load(o + row * dv + c, ov);
+    Vec4<Tio>::load(z + row * dv + c, zv);
   }
+  float ss = (ov[0] * ov[0] + ov[1] * ov[1]) + (ov[2] * ov[2] + ov[3] * ov[3]);
   ss = warp_sum(ss);
   const float inv = rsqrtf(ss / dv + eps);
+  if (active) {
+    const float ww[4] = {w[c], w[c + 1], w[c + 2], w[c + 3]};
+    float yv[4];
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const int cidx = lane + 32 * e;
-    if (cidx < dv) {
-      const float zz = to_f(zrow[cidx]);
-      y[row * dv + cidx] = from_f<Tio>(ov[e] * inv * w[cidx] * (zz * sigmoidf_(zz)));
-    }
+    for (int e = 0; e < 4; ++e) yv[e] = ov[e] * inv * ww[e] * silu_fast(zv[e]);
+    Vec4<Tio>::store(y + row * dv + c, yv);
   }
 }
 

@@ -132,13 +132,22 @@ def test_degenerate_gates(orc):
     assert out_err(o, o_ref) <= TOL_BF16_OUT
 
 
-def test_nan_propagates():
-    """A NaN in v reaches the output of that head (no silent masking)."""
-    w, x = small_bf16(T=64, seed=9)
-    x["v"][0, 5, 1, 3] = float("nan")
-    o, sT = run(x, 64)
-    assert torch.isnan(o[0, 5:, 1]).any()
-    assert not torch.isnan(o[1]).any()
+@pytest.mark.parametrize("variant", ["simt", "auto"])
+@pytest.mark.parametrize("what,idx,val", [("v", (0, 5, 1, 3), float("nan")),
+                                          ("v", (0, 70, 1, 100), float("inf")),
+                                          ("k", (0, 5, 0, 3), float("nan")),
+                                          ("log_alpha", (0, 9, 1), float("nan"))])
+def test_nonfinite_propagates(variant, what, idx, val):
+    """A NaN or infinity in one head's input reaches that head's later outputs and final state as
+    non-finite values (no silent masking) and leaves every other sequence finite."""
+    w, x = small_bf16(T=130, seed=9)
+    x[what][idx] = val
+    o, sT = run(x, 64, variant=variant)
+    h = 1 if what != "k" else 0                  # value head 1, or key head 0 (value heads 0..2)
+    t = idx[1]
+    assert not torch.isfinite(o[0, t:, h].float()).all()
+    assert not torch.isfinite(sT[0, h]).all()
+    assert torch.isfinite(o[1].float()).all() and torch.isfinite(sT[1]).all()
 
 
 def _sampled_heads(orc, x, o, sT, heads, Hk, Hv):

@@ -5,7 +5,8 @@ import torch
 
 import gdn_inputs as gi
 import gated_deltanet_linear_18_b200 as gdn
-from gpu_util import TOL_BF16_OUT, TOL_BF16_STATE, TOL_F32_ABS, max_abs, np64, out_err, rel_rms
+from gpu_util import (TOL_BF16_OUT, TOL_BF16_STATE, TOL_F32_ABS, halfulp_bf16, max_abs, np64,
+                      out_err, rel_rms)
 
 pytestmark = pytest.mark.gpu
 
@@ -48,7 +49,7 @@ def test_decode_full_size_sampled(orc):
         assert rel_rms(S[n:n + 1], S_ref) <= TOL_BF16_STATE
 
 
-def test_decode_equals_chunk_fwd():
+def test_decode_equals_chunk_fwd(orc):
     """A run of decode steps and one chunked call over the same tokens agree (16.3 vs 16.2)."""
     w = gi.WORKLOADS["decode"].with_sizes(B=3, Hk=2, Hv=6, steps=70, seed=21)
     x = gi.make_decode_inputs(w)
@@ -58,8 +59,17 @@ def test_decode_equals_chunk_fwd():
     o_chk, S_chk = gdn.chunk_fwd(sw(d["q"]), sw(d["k"]), sw(d["v"]), sw(d["log_alpha"]),
                                  sw(d["beta"]), d["S0"], chunk=64)
     torch.cuda.synchronize()
-    assert rel_rms(o_dec, np64(sw(o_chk))) <= TOL_BF16_OUT
-    assert rel_rms(S_dec, np64(S_chk)) <= TOL_BF16_STATE
+    o_chk, S_chk = sw(o_chk).cpu(), S_chk.cpu()
+    # both against the oracle, then against each other: two bf16 results within the bound of the
+    # same exact value may sit a full bf16 ulp apart, so the mutual check allows both roundings
+    o_ref, S_ref = orc.decode_steps(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"])
+    for o, S in ((o_dec, S_dec), (o_chk, S_chk)):
+        assert out_err(o, o_ref) <= TOL_BF16_OUT
+        assert rel_rms(S, S_ref) <= TOL_BF16_STATE
+    a, b = np64(o_dec), np64(o_chk)
+    excess = np.maximum(np.abs(a - b) - 2 * halfulp_bf16(b), 0.0)
+    assert excess.max() / np.sqrt(np.mean(o_ref ** 2)) <= 2 * TOL_BF16_OUT
+    assert rel_rms(S_dec, np64(S_chk)) <= 2 * TOL_BF16_STATE
 
 
 def test_in_place_state_size_constant():
