@@ -83,7 +83,7 @@ constexpr uint32_t TM_S = 0, TM_PT = 64, TM_X = 128, TM_Y = 256, TM_M = 384;
 enum : int {
   B_QK_FULL = 0, B_IN_EMPTY = 2, B_S_FULL = 4, B_S_EMPTY, B_PT_READY, B_PT_FULL, B_PT_EMPTY,
   B_PRE_FULL, B_A2_EMPTY, B_GATE, B_X_FULL = B_GATE + 3, B_R_FULL, B_Y_FULL, B_D_FULL, B_D3_FULL,
-  B_M_READY, B_V_FULL, B_V_EMPTY, B_O_DONE, B_DRAIN, B_END = B_DRAIN + 2
+  B_M_READY, B_V_FULL, B_V_EMPTY, B_O_DONE, B_M_SCALED, B_DRAIN, B_END = B_DRAIN + 2
 };
 static_assert(B_END <= NBAR, "barrier map");
 
@@ -117,34 +117,68 @@ __device__ __forceinline__ uint32_t at(uint32_t blk_base, int r, int c) {
   return blk_base + (uint32_t)((r * BLD + c) * 4);
 }
 
-// acc[0..3] += sum_k X[xr][k] * Y[k][yc .. yc+3], k < 16, X and Y 16 x 16 blocks.
-__device__ __forceinline__ void strip16(uint32_t X, int xr, uint32_t Y, int yc, float (&acc)[4]) {
-#pragma unroll
-  for (int k4 = 0; k4 < 16; k4 += 4) {
-    const float4 xa = tc::lds4(at(X, xr, k4));
-    const float xs[4] = {xa.x, xa.y, xa.z, xa.w};
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      const float4 y = tc::lds4(at(Y, k4 + kk, yc));
-      acc[0] = fmaf(xs[kk], y.x, acc[0]);
-      acc[1] = fmaf(xs[kk], y.y, acc[1]);
-      acc[2] = fmaf(xs[kk], y.z, acc[2]);
-      acc[3] = fmaf(xs[kk], y.w, acc[3]);
-    }
-  }
-}
-
 // block index bi = 0..5 -> (i, k) = (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
 __device__ __forceinline__ int blk_i(int bi) { return bi < 1 ? 1 : (bi < 3 ? 2 : 3); }
 __device__ __forceinline__ int blk_k(int bi, int i) { return bi - i * (i - 1) / 2; }
 
-// T = (I + A)^-1 for a 64 x 64 strictly lower A (128 threads, named barrier 1), blocked by 16:
-//   D_b = (I + A_bb)^-1 by forward substitution (one column per thread);
-//   At_ik = D_i A_ik;  U = (I + At)^-1 (U_ii = I; At is block-nilpotent, so U is closed-form in
-//   At's blocks);  T_ik = U_ik D_k.   (I + A = blockdiag(I + A_bb) (I + At), so T = U D.)
-// On return the off-diagonal blocks of T are in `tv` (three 1 x 4 strips per thread, item m at
-// id = ptid + 128 m: block bi = id / 64, row (id / 4) % 16, columns 4 (id % 4) ..) and the
-// diagonal blocks D_b are in sT.  sA's blocks are overwritten.
+// Warp-level tf32 MMA: d (16 x 8 C fragment) += a (16 x 8) b (8 x 8).  Fragments (lane = 4 g + t):
+// a = {A[g][t], A[g+8][t], A[g][t+4], A[g+8][t+4]}, b = {B[t][g], B[t+4][g]},
+// d = {D[g][2t], D[g][2t+1], D[g+8][2t], D[g+8][2t+1]}.
+__device__ __forceinline__ void mma_m16n8k8_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                                 uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// x = hi + lo + e with hi, lo tf32 (truncated), |e| < 2^-20 |x|.
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+  hi = __float_as_uint(x) & 0xFFFFE000u;
+  lo = __float_as_uint(x - __uint_as_float(hi)) & 0xFFFFE000u;
+}
+// acc (C fragment of rows 0..15, columns n0 .. n0+7) += X Y[:, n0 .. n0+7] for 16 x 16 packed
+// blocks X and Y, as lo.hi + hi.lo + hi.hi tf32 products (fp32-level accuracy).
+__device__ __forceinline__ void mma_blk(uint32_t X, uint32_t Y, int n0, int g, int t,
+                                        float (&acc)[4]) {
+#pragma unroll
+  for (int kk = 0; kk < 16; kk += 8) {
+    uint32_t ah[4], al[4], bh0, bl0, bh1, bl1;
+    split_tf32(tc::lds1(at(X, g, kk + t)), ah[0], al[0]);
+    split_tf32(tc::lds1(at(X, g + 8, kk + t)), ah[1], al[1]);
+    split_tf32(tc::lds1(at(X, g, kk + t + 4)), ah[2], al[2]);
+    split_tf32(tc::lds1(at(X, g + 8, kk + t + 4)), ah[3], al[3]);
+    split_tf32(tc::lds1(at(Y, kk + t, n0 + g)), bh0, bl0);
+    split_tf32(tc::lds1(at(Y, kk + t + 4, n0 + g)), bh1, bl1);
+    mma_m16n8k8_tf32(acc, al, bh0, bh1);
+    mma_m16n8k8_tf32(acc, ah, bl0, bl1);
+    mma_m16n8k8_tf32(acc, ah, bh0, bh1);
+  }
+}
+__device__ __forceinline__ float2 lds2(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void sts2(uint32_t addr, float a, float b) {
+  asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
+}
+__device__ __forceinline__ void ld_frag(uint32_t B, int n0, int g, int t, float (&c)[4]) {
+  const float2 a = lds2(at(B, g, n0 + 2 * t)), b = lds2(at(B, g + 8, n0 + 2 * t));
+  c[0] = a.x; c[1] = a.y; c[2] = b.x; c[3] = b.y;
+}
+__device__ __forceinline__ void st_frag(uint32_t B, int n0, int g, int t, const float (&c)[4]) {
+  sts2(at(B, g, n0 + 2 * t), c[0], c[1]);
+  sts2(at(B, g + 8, n0 + 2 * t), c[2], c[3]);
+}
+
+// T = (I + A)^-1 for a 64 x 64 strictly lower A (128 threads = 4 warps, named barrier 1), blocked
+// by 16:  D_b = (I + A_bb)^-1 by forward substitution (one column per thread);  At_ik = D_i A_ik;
+// U = (I + At)^-1 (U_ii = I; At is block-nilpotent, so U is closed-form in At's blocks);
+// T_ik = U_ik D_k.   (I + A = blockdiag(I + A_bb) (I + At), so T = U D.)  The block products run
+// as warp MMAs on 16 x 8 half blocks.  On return the off-diagonal blocks of T are in `tv`: item m
+// of warp w is half block hp = w + 4 m (block bi = hp / 2, columns 8 (hp % 2) ..) as a C fragment;
+// the diagonal blocks D_b are in sT.  sA's blocks are overwritten.
 __device__ __forceinline__ void solve_unit_lower(uint32_t sA, uint32_t sT, int ptid, float (&tv)[3][4]) {
   if (ptid < 64) {                                    // D_b, column `col` of block b
     const int b = ptid >> 4, col = ptid & 15;
@@ -171,43 +205,51 @@ __device__ __forceinline__ void solve_unit_lower(uint32_t sA, uint32_t sT, int p
     for (int i = 0; i < 16; ++i) tc::sts1(at(Tb, i, col), x[i]);
   }
   tc::named_bar(1, 128);
+  const int w = ptid >> 5, lane = ptid & 31, g = lane >> 2, t = lane & 3;
 #pragma unroll
   for (int m = 0; m < 3; ++m) {                       // At_ik = D_i A_ik, into T's off-diagonal
-    const int id = ptid + 128 * m, bi = id >> 6, r = (id >> 2) & 15, cs = id & 3;
+    const int hp = w + 4 * m, bi = hp >> 1, n0 = (hp & 1) * 8;
     const int i = blk_i(bi), k = blk_k(bi, i);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    strip16(blk(sT, i, i), r, blk(sA, i, k), 4 * cs, acc);
-    tc::sts4(at(blk(sT, i, k), r, 4 * cs), make_float4(acc[0], acc[1], acc[2], acc[3]));
+    mma_blk(blk(sT, i, i), blk(sA, i, k), n0, g, t, acc);
+    st_frag(blk(sT, i, k), n0, g, t, acc);
   }
   tc::named_bar(1, 128);
   // U_20 = -At_20 + At_21 At_10;  U_31 = -At_31 + At_32 At_21;  V_30 = -At_30 + At_31 At_10
   // (into sA's blocks (2,0), (3,1), (3,0); A itself is no longer needed)
-  for (int id = ptid; id < 192; id += 128) {
-    const int bi = id >> 6, r = (id >> 2) & 15, cs = id & 3;
-    const int oi = bi == 0 ? 2 : 3, ok = bi == 1 ? 1 : 0;      // output block (oi, ok)
-    const int xk = bi == 1 ? 2 : 1;                             // X = At_(oi, xk), Y = At_(xk, ok)
-    const float4 base = tc::lds4(at(blk(sT, oi, ok), r, 4 * cs));
-    float acc[4] = {-base.x, -base.y, -base.z, -base.w};
-    strip16(blk(sT, oi, xk), r, blk(sT, xk, ok), 4 * cs, acc);
-    tc::sts4(at(blk(sA, oi, ok), r, 4 * cs), make_float4(acc[0], acc[1], acc[2], acc[3]));
+#pragma unroll
+  for (int m = 0; m < 2; ++m) {
+    const int hp = w + 4 * m;
+    if (hp < 6) {
+      const int bi = hp >> 1, n0 = (hp & 1) * 8;
+      const int oi = bi == 0 ? 2 : 3, ok = bi == 1 ? 1 : 0;    // output block (oi, ok)
+      const int xk = bi == 1 ? 2 : 1;                           // X = At_(oi, xk), Y = At_(xk, ok)
+      float acc[4];
+      ld_frag(blk(sT, oi, ok), n0, g, t, acc);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[e] = -acc[e];
+      mma_blk(blk(sT, oi, xk), blk(sT, xk, ok), n0, g, t, acc);
+      st_frag(blk(sA, oi, ok), n0, g, t, acc);
+    }
   }
   tc::named_bar(1, 128);
-  if (ptid < 64) {                                    // U_30 = V_30 - At_32 U_20
-    const int r = ptid >> 2, cs = ptid & 3;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    strip16(blk(sT, 3, 2), r, blk(sA, 2, 0), 4 * cs, acc);
-    const uint32_t dst = at(blk(sA, 3, 0), r, 4 * cs);
-    const float4 v30 = tc::lds4(dst);
-    tc::sts4(dst, make_float4(v30.x - acc[0], v30.y - acc[1], v30.z - acc[2], v30.w - acc[3]));
+  if (w < 2) {                                        // U_30 = V_30 - At_32 U_20
+    const int n0 = 8 * w;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, v[4];
+    mma_blk(blk(sT, 3, 2), blk(sA, 2, 0), n0, g, t, acc);
+    ld_frag(blk(sA, 3, 0), n0, g, t, v);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) v[e] -= acc[e];
+    st_frag(blk(sA, 3, 0), n0, g, t, v);
   }
   tc::named_bar(1, 128);
 #pragma unroll
   for (int m = 0; m < 3; ++m) {                       // T_ik = U_ik D_k (U = -At next to diag)
-    const int id = ptid + 128 * m, bi = id >> 6, r = (id >> 2) & 15, cs = id & 3;
+    const int hp = w + 4 * m, bi = hp >> 1, n0 = (hp & 1) * 8;
     const int i = blk_i(bi), k = blk_k(bi, i);
     const bool sub = (i == k + 1);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    strip16(sub ? blk(sT, i, k) : blk(sA, i, k), r, blk(sT, k, k), 4 * cs, acc);
+    mma_blk(sub ? blk(sT, i, k) : blk(sA, i, k), blk(sT, k, k), n0, g, t, acc);
     const float sg = sub ? -1.f : 1.f;
 #pragma unroll
     for (int e = 0; e < 4; ++e) tv[m][e] = sg * acc[e];
@@ -303,6 +345,19 @@ __device__ __forceinline__ void store_tb(uint32_t sb, int kr, int n, float4 v) {
             v);
 }
 
+// Same for two values (columns n, n + 1, n even).
+__device__ __forceinline__ void store_tb2(uint32_t sb, int kr, int n, float a, float b) {
+  uint32_t h, l;
+  split2(a, b, h, l);
+  const uint32_t a2 = sb + OFF_A2 + (64 + kr) * 128 + (((n >> 3) ^ (kr & 7)) << 4) + (n & 7) * 2;
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(a2), "r"(h) : "memory");
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(a2 + 16384), "r"(l) : "memory");
+  const uint32_t wt = sb + OFF_WT + (n >> 5) * 8192 + kr * 128 +
+                      ((((n & 31) >> 3) ^ (kr & 3)) << 5) + (n & 7) * 4;
+  asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(wt), "r"(tc::to_tf32(a)), "r"(tc::to_tf32(b))
+               : "memory");
+}
+
 // ------------------------------------------------------------------------------------------
 // the kernel
 // ------------------------------------------------------------------------------------------
@@ -339,7 +394,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
                         B_A2_EMPTY, B_GATE, B_GATE + 1, B_GATE + 2, B_X_FULL, B_Y_FULL, B_D3_FULL,
                         B_V_FULL, B_DRAIN, B_DRAIN + 1};
     for (int i : ones) tc::mbar_init(bar(i), 1);
-    const int twos[] = {B_R_FULL, B_D_FULL, B_M_READY, B_V_EMPTY, B_O_DONE};
+    const int twos[] = {B_R_FULL, B_D_FULL, B_M_READY, B_V_EMPTY, B_O_DONE, B_M_SCALED};
     for (int i : twos) tc::mbar_init(bar(i), 2);   // one arrive per column half
     *abort_flag = 0;
     tc::fence_barrier_init();
@@ -466,7 +521,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         tc::mma_commit(bar(B_A2_EMPTY));
         GDN_TRACE(c, 21);
         // M += K^T (ktil Delta)_hi + K^T (ktil Delta)_lo  (TMEM holds gamma_last M)  (bf16)
-        ok = tc::mbar_wait(bar(B_D_FULL), c & 1, abort_flag, kBudget);
+        ok = tc::mbar_wait(bar(B_D_FULL), c & 1, abort_flag, kBudget) &&
+             tc::mbar_wait(bar(B_M_SCALED), c & 1, abort_flag, kBudget);
         if (!ok) break;
         tc::tc_fence_after();
 #pragma unroll
@@ -518,6 +574,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       gGam[2 * lane] = expf(g0);     gGam[2 * lane + 1] = expf(g1);
       gKt[2 * lane] = expf(gl - g0); gKt[2 * lane + 1] = expf(gl - g1);
       gBeta[2 * lane] = be0;         gBeta[2 * lane + 1] = be1;
+      if (lane == 0) *reinterpret_cast<volatile int*>(gE) = 0;   // non-finite A flag (E[0] unused)
       // block factors E[b][j] = exp(G_16b - G_j) for j < 16b (each <= 1: G never increases)
 #pragma unroll
       for (int b = 1; b < 4; ++b) {
@@ -600,6 +657,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
           if (is_p) {
             tc::tmem_st32(tmem + lane_off + TM_S + 32 * p, sv);
           } else {
+            float sum = 0.f;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) sum += sv[e];
+            if (nonfinite(sum)) *reinterpret_cast<volatile int*>(const_cast<float*>(gE)) = 1;
 #pragma unroll
             for (int kb2 = 0; kb2 < 2; ++kb2) {
               const int kb = 2 * p + kb2;
@@ -622,15 +683,19 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       float tv[3][4];
       solve_unit_lower(sA, sT, ptid, tv);
       if (ptid == 0) GDN_TRACE(c, 3);
-      // T_b = T diag(beta): off-diagonal strips from the solve, diagonal strips from sT
-      float4 toff[3], tdg[2];
+      // T_b = T diag(beta): off-diagonal half blocks from the solve (C fragments), diagonal
+      // strips from sT
+      const int pw = ptid >> 5, pg = (ptid & 31) >> 2, pt = ptid & 3;
+      float toff[3][4];
 #pragma unroll
       for (int m = 0; m < 3; ++m) {
-        const int id = ptid + 128 * m, bi = id >> 6, cs = id & 3;
+        const int hp = pw + 4 * m, bi = hp >> 1, n0 = (hp & 1) * 8;
         const int k = blk_k(bi, blk_i(bi));
-        const float4 be = tc::lds4(gbeta_u + 4 * (16 * k + 4 * cs));
-        toff[m] = make_float4(tv[m][0] * be.x, tv[m][1] * be.y, tv[m][2] * be.z, tv[m][3] * be.w);
+        const float2 be = lds2(gbeta_u + 4 * (16 * k + n0 + 2 * pt));
+        toff[m][0] = tv[m][0] * be.x; toff[m][1] = tv[m][1] * be.y;
+        toff[m][2] = tv[m][2] * be.x; toff[m][3] = tv[m][3] * be.y;
       }
+      float4 tdg[2];
 #pragma unroll
       for (int m = 0; m < 2; ++m) {
         const int id = ptid + 128 * m, b = id >> 6, r = (id >> 2) & 15, cs = id & 3;
@@ -648,17 +713,23 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       {
         float sum = 0.f;
 #pragma unroll
-        for (int m = 0; m < 3; ++m) sum += (toff[m].x + toff[m].y) + (toff[m].z + toff[m].w);
+        for (int m = 0; m < 3; ++m) sum += (toff[m][0] + toff[m][1]) + (toff[m][2] + toff[m][3]);
 #pragma unroll
         for (int m = 0; m < 2; ++m) sum += (tdg[m].x + tdg[m].y) + (tdg[m].z + tdg[m].w);
-        const bool bad = nonfinite(sum);
+        // a non-finite A (the warp MMAs of the solve may drop a NaN) is flagged by its rows
+        const bool bad = nonfinite(sum) || *reinterpret_cast<volatile const int*>(gG + 256) != 0;
         const float4 inf4 = make_float4(kInf, kInf, kInf, kInf);
 #pragma unroll
         for (int m = 0; m < 3; ++m) {
-          const int id = ptid + 128 * m, bi = id >> 6, r = (id >> 2) & 15, cs = id & 3;
+          const int hp = pw + 4 * m, bi = hp >> 1, n0 = (hp & 1) * 8;
           const int i = blk_i(bi), k = blk_k(bi, i);
-          store_tb(sb, 16 * i + r, 16 * k + 4 * cs, bad ? inf4 : toff[m]);   // below the diagonal
-          store_tb(sb, 16 * k + r, 16 * i + 4 * cs, make_float4(0.f, 0.f, 0.f, 0.f));   // above
+#pragma unroll
+          for (int h8 = 0; h8 < 2; ++h8) {
+            const int n = 16 * k + n0 + 2 * pt;
+            store_tb2(sb, 16 * i + pg + 8 * h8, n, bad ? kInf : toff[m][2 * h8],
+                      bad ? kInf : toff[m][2 * h8 + 1]);                    // below the diagonal
+            store_tb2(sb, 16 * k + pg + 8 * h8, 16 * i + n0 + 2 * pt, 0.f, 0.f);   // above
+          }
         }
 #pragma unroll
         for (int m = 0; m < 2; ++m) {
@@ -773,7 +844,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
       stop = vote_abort(id_wg, 128, abort_flag);
-      if (leader) tc::mbar_arrive(bar(B_M_READY));
+      if (leader) {
+        tc::mbar_arrive(bar(B_M_READY));
+        tc::mbar_arrive(bar(B_M_SCALED));
+      }
     }
 
     for (int c = 0; c < nC && !stop; ++c) {
@@ -900,29 +974,32 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
           GDN_TRACE(c, 36 + ev);
         }
       }
-      // M <- gamma_last M + K^T (ktil Delta) is now in TMEM (row r of this half); keep its bf16
-      // copy for the next X and scale it by the next chunk's gamma_last for the next update
+      // M <- gamma_last M + K^T (ktil Delta) is now in TMEM (row r of this half).  Its bf16 pair
+      // goes out first (the next X needs it); then TMEM is scaled by the next chunk's
+      // gamma_last for the next update, which waits for that separately.
       tc::mbar_wait(bar(B_D3_FULL), c & 1, abort_flag, kBudget);
       if (leader) GDN_TRACE(c, 37 + ev);
       tc::tc_fence_after();
       if (c + 1 < nC) {
+        float m[64];
+        tmem_ld64(tmem + lane_off + TM_M + tcol, m);
         tc::mbar_wait(bar(B_GATE + (c + 1) % 3), ((c + 1) / 3) & 1, abort_flag, kBudget);
         const float gl = gslot(c + 1)[64 + 63];
+        tc::tmem_wait_ld();
         if (leader && hh == 0) GDN_TRACE(c, 50);
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
-          float m[32];
-          tc::tmem_ld32(tmem + lane_off + TM_M + tcol + 32 * p, m);
-          tc::tmem_wait_ld();
-          if (p == 0 && leader && hh == 0) GDN_TRACE(c, 51);
-          store_m32(m, p);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) m[i] *= gl;
-          tc::tmem_st32(tmem + lane_off + TM_M + tcol + 32 * p, m);
-          if (p == 0 && leader && hh == 0) GDN_TRACE(c, 52);
+        store_m32(*reinterpret_cast<const float(*)[32]>(&m[0]), 0);
+        store_m32(*reinterpret_cast<const float(*)[32]>(&m[32]), 1);
+        tc::fence_proxy_async_smem();
+        tc::named_bar(id_wg, 128);
+        if (leader) {
+          GDN_TRACE(c, 38 + ev);
+          tc::mbar_arrive(bar(B_M_READY));
         }
+#pragma unroll
+        for (int i = 0; i < 64; ++i) m[i] *= gl;
+        tmem_st64(tmem + lane_off + TM_M + tcol, m);
         tc::tmem_wait_st();
-        if (leader && hh == 0) GDN_TRACE(c, 53);
+        if (leader && hh == 0) GDN_TRACE(c, 51);
       } else if (S_T && !*abort_flag) {
         float m[64];
         tmem_ld64(tmem + lane_off + TM_M + tcol, m);
@@ -932,13 +1009,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         for (int i = 0; i < 16; ++i)
           dst[i] = make_float4(m[4 * i], m[4 * i + 1], m[4 * i + 2], m[4 * i + 3]);
       }
-      tc::fence_proxy_async_smem();
       tc::tc_fence_before();
-      if (leader && hh == 0) GDN_TRACE(c, 54);
       stop = vote_abort(id_wg, 128, abort_flag);
       if (leader) {
-        GDN_TRACE(c, 38 + ev);
-        tc::mbar_arrive(bar(B_M_READY));
+        if (hh == 0) GDN_TRACE(c, 52);
+        tc::mbar_arrive(bar(B_M_SCALED));
       }
     }
     if (leader) tc::bulk_wait_all();               // every o tile has reached global memory
