@@ -69,6 +69,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_layer_fwd.argtypes = [P] * 14 + [SZ] + [I] * 7 + [F, F, F, I, P]
         L.gdn_layer_fwd.restype = I
         L.gdn_layer_workspace_bytes.argtypes = [I] * 7 + [I]
+        L.gdn_layer_fwd_static.argtypes = [P] * 13 + [I] * 7 + [F, F, F, I, P]
+        L.gdn_layer_fwd_static.restype = I
         L.gdn_layer_workspace_bytes.restype = SZ
         _lib = L
     return _lib
@@ -224,6 +226,28 @@ def layer_fwd(q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, *
                                  float(scale), float(l2_eps), float(norm_eps),
                                  _io_dtype(q_raw), _stream(dev))
     _check("gdn_layer_fwd", st)
+    return y, sT
+
+
+def layer_fwd_static(q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, *,
+                     Hk: int, Hv: int, dk: int, dv: int, chunk: int = 64, scale: float = 1.0,
+                     l2_eps: float = 1e-6, norm_eps: float = 1e-5, want_state: bool = True):
+    """layer_fwd with the library's built-in device scratch instead of a workspace (see
+    gdn_layer_fwd_static in gdn.h: at most GDN_LAYER_STATIC_SCRATCH_BYTES of scratch, and calls
+    on one device must not overlap on the GPU)."""
+    B, T = q_raw.shape[:2]
+    _f32(wq, wk, wv, log_alpha, beta, S0, norm_w)
+    y = torch.empty(B, T, Hv, dv, device=q_raw.device, dtype=q_raw.dtype)
+    sT = torch.empty(B, Hv, dk, dv, device=q_raw.device, dtype=torch.float32) \
+        if want_state else None
+    dev = _dev(q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, y, sT)
+    with torch.cuda.device(dev):
+        st = lib().gdn_layer_fwd_static(_p(q_raw), _p(k_raw), _p(v_raw), _p(z), _p(wq), _p(wk),
+                                        _p(wv), _p(log_alpha), _p(beta), _p(S0), _p(norm_w),
+                                        _p(y), _p(sT), B, T, Hk, Hv, dk, dv, chunk, float(scale),
+                                        float(l2_eps), float(norm_eps), _io_dtype(q_raw),
+                                        _stream(dev))
+    _check("gdn_layer_fwd_static", st)
     return y, sT
 
 

@@ -334,3 +334,53 @@ gdn_status gdn_layer_fwd(const void* q_raw, const void* k_raw, const void* v_raw
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------------
+// gdn_layer_fwd_static: the whole layer with its scratch in the library's own device memory.
+// ---------------------------------------------------------------------------------------------
+#include <mutex>
+
+// The scratch is part of the library's device image: it exists on a device once the library's
+// device code is loaded there, and no call allocates or frees it.  Every byte the layer reads
+// from it is written earlier in the same call, so nothing in it has to start at zero.
+static __device__ __align__(256) unsigned char gdn_layer_scratch[GDN_LAYER_STATIC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kScratchDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kScratchDevices] = {};
+
+// Device address of gdn_layer_scratch on the current device; looked up on the first call per
+// device (a runtime query; it allocates nothing) and kept for later calls.
+gdn_status layer_scratch_address(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kScratchDevices) return GDN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, gdn_layer_scratch) != cudaSuccess || p == nullptr)
+      return GDN_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return GDN_OK;
+}
+}  // namespace
+
+extern "C" gdn_status gdn_layer_fwd_static(
+    const void* q_raw, const void* k_raw, const void* v_raw, const void* z, const float* wq,
+    const float* wk, const float* wv, const float* log_alpha, const float* beta, const float* S0,
+    const float* norm_w, void* y, float* S_T, int B, int T, int Hk, int Hv, int dk, int dv,
+    int chunk, float scale, float l2_eps, float norm_eps, gdn_dtype dtype, gdn_stream_t stream) {
+  if (B < 0 || T < 0 || !valid_dtype(dtype)) return GDN_ERR_INVALID_ARG;
+  const size_t need = gdn_layer_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, dtype);
+  if (need > (size_t)GDN_LAYER_STATIC_SCRATCH_BYTES) return GDN_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  if (need > 0) {
+    const gdn_status s = layer_scratch_address(&scratch);
+    if (s != GDN_OK) return s;
+  }
+  return gdn_layer_fwd(q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, y, S_T,
+                       scratch, need > 0 ? (size_t)GDN_LAYER_STATIC_SCRATCH_BYTES : 0, B, T, Hk,
+                       Hv, dk, dv, chunk, scale, l2_eps, norm_eps, dtype, stream);
+}

@@ -173,6 +173,34 @@ GDN_API gdn_status gdn_layer_fwd(const void *q_raw, const void *k_raw, const voi
 GDN_API size_t gdn_layer_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, int chunk,
                                  gdn_dtype dtype);
 
+/* Size of the device scratch that the library carries for gdn_layer_fwd_static: 32 MiB. */
+#define GDN_LAYER_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/* gdn_layer_fwd_static: the same layer as gdn_layer_fwd, for callers that cannot hand it a
+ * workspace.  A program that has no device allocator of its own (plain C linking only this
+ * library), or one that must not allocate device memory while it runs the layer (an allocation
+ * can synchronise the device and stall other streams), calls this instead: it allocates and frees
+ * nothing.  The pages describe no such call; it belongs to this library only.
+ *
+ *   Arguments, layouts, results and errors are those of gdn_layer_fwd without `workspace` and
+ *   `workspace_bytes`.  The scratch is GDN_LAYER_STATIC_SCRATCH_BYTES of device memory built into
+ *   the library (one per device); sizes for which gdn_layer_workspace_bytes(...) exceeds it return
+ *   GDN_ERR_UNSUPPORTED before any work (about 750 tokens at Hk=16, Hv=48, d=128, bf16).
+ *   The first call on a device looks the scratch's device address up (cudaGetSymbolAddress on
+ *   the current device, which must be the device of every pointer and of `stream`) and keeps it;
+ *   that lookup allocates nothing, but make the first call on each device before any stream
+ *   capture starts.  Nothing in the scratch needs to start at zero.
+ *   All calls on one device share the one scratch: two calls whose GPU work can overlap (on
+ *   streams not ordered with each other) race on it and give wrong results.  Order them.
+ */
+GDN_API gdn_status gdn_layer_fwd_static(const void *q_raw, const void *k_raw, const void *v_raw,
+                         const void *z, const float *wq, const float *wk, const float *wv,
+                         const float *log_alpha, const float *beta, const float *S0,
+                         const float *norm_w, void *y, float *S_T,
+                         int B, int T, int Hk, int Hv, int dk, int dv, int chunk,
+                         float scale, float l2_eps, float norm_eps,
+                         gdn_dtype dtype, gdn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
