@@ -101,8 +101,14 @@ __device__ unsigned long long* g_tc_trace = nullptr;
   do {                                                                                \
     if (g_tc_trace) g_tc_trace[((size_t)blockIdx.x * nC + (c)) * 64 + (ev)] = clock64(); \
   } while (0)
+// same with the global nanosecond timer (comparable across SMs)
+#define GDN_TRACE_G(c, ev)                                                            \
+  do {                                                                                \
+    if (g_tc_trace) g_tc_trace[((size_t)blockIdx.x * nC + (c)) * 64 + (ev)] = tc::globaltimer_ns(); \
+  } while (0)
 #else
 #define GDN_TRACE(c, ev) do {} while (0)
+#define GDN_TRACE_G(c, ev) do {} while (0)
 #endif
 
 // ------------------------------------------------------------------------------------------
@@ -126,8 +132,7 @@ __device__ __forceinline__ int blk_k(int bi, int i) { return bi - i * (i - 1) / 
 // d = {D[g][2t], D[g][2t+1], D[g+8][2t], D[g+8][2t+1]}.
 __device__ __forceinline__ void mma_m16n8k8_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                                  uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+  asm("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
       "{%8, %9}, {%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
@@ -137,22 +142,35 @@ __device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) 
   hi = __float_as_uint(x) & 0xFFFFE000u;
   lo = __float_as_uint(x - __uint_as_float(hi)) & 0xFFFFE000u;
 }
-// acc (C fragment of rows 0..15, columns n0 .. n0+7) += X Y[:, n0 .. n0+7] for 16 x 16 packed
-// blocks X and Y, as lo.hi + hi.lo + hi.hi tf32 products (fp32-level accuracy).
-__device__ __forceinline__ void mma_blk(uint32_t X, uint32_t Y, int n0, int g, int t,
-                                        float (&acc)[4]) {
+// One 16 x 16 x 16 product X Y[:, n0 .. n0+7] of packed blocks (a 16 x 8 half block of the result).
+struct Tile {
+  uint32_t X, Y;
+  int n0;
+};
+// acc[m] (C fragments) += X_m Y_m[:, n0_m ..] for N independent tiles, as lo.hi + hi.lo + hi.hi
+// tf32 products (fp32-level accuracy), one k half at a time; the MMAs of the N tiles interleave.
+template <int N>
+__device__ __forceinline__ void mma_tiles(const Tile (&tl)[N], int g, int t, float (&acc)[N][4]) {
 #pragma unroll
   for (int kk = 0; kk < 16; kk += 8) {
-    uint32_t ah[4], al[4], bh0, bl0, bh1, bl1;
-    split_tf32(tc::lds1(at(X, g, kk + t)), ah[0], al[0]);
-    split_tf32(tc::lds1(at(X, g + 8, kk + t)), ah[1], al[1]);
-    split_tf32(tc::lds1(at(X, g, kk + t + 4)), ah[2], al[2]);
-    split_tf32(tc::lds1(at(X, g + 8, kk + t + 4)), ah[3], al[3]);
-    split_tf32(tc::lds1(at(Y, kk + t, n0 + g)), bh0, bl0);
-    split_tf32(tc::lds1(at(Y, kk + t + 4, n0 + g)), bh1, bl1);
-    mma_m16n8k8_tf32(acc, al, bh0, bh1);
-    mma_m16n8k8_tf32(acc, ah, bl0, bl1);
-    mma_m16n8k8_tf32(acc, ah, bh0, bh1);
+    uint32_t ah[N][4], al[N][4], bh[N][2], bl[N][2];
+#pragma unroll
+    for (int m = 0; m < N; ++m) {
+      const uint32_t X = tl[m].X, Y = tl[m].Y;
+      const int n0 = tl[m].n0;
+      split_tf32(tc::lds1(at(X, g, kk + t)), ah[m][0], al[m][0]);
+      split_tf32(tc::lds1(at(X, g + 8, kk + t)), ah[m][1], al[m][1]);
+      split_tf32(tc::lds1(at(X, g, kk + t + 4)), ah[m][2], al[m][2]);
+      split_tf32(tc::lds1(at(X, g + 8, kk + t + 4)), ah[m][3], al[m][3]);
+      split_tf32(tc::lds1(at(Y, kk + t, n0 + g)), bh[m][0], bl[m][0]);
+      split_tf32(tc::lds1(at(Y, kk + t + 4, n0 + g)), bh[m][1], bl[m][1]);
+    }
+#pragma unroll
+    for (int m = 0; m < N; ++m) mma_m16n8k8_tf32(acc[m], al[m], bh[m][0], bh[m][1]);
+#pragma unroll
+    for (int m = 0; m < N; ++m) mma_m16n8k8_tf32(acc[m], ah[m], bl[m][0], bl[m][1]);
+#pragma unroll
+    for (int m = 0; m < N; ++m) mma_m16n8k8_tf32(acc[m], ah[m], bh[m][0], bh[m][1]);
   }
 }
 __device__ __forceinline__ float2 lds2(uint32_t addr) {
@@ -179,7 +197,8 @@ __device__ __forceinline__ void st_frag(uint32_t B, int n0, int g, int t, const 
 // as warp MMAs on 16 x 8 half blocks.  On return the off-diagonal blocks of T are in `tv`: item m
 // of warp w is half block hp = w + 4 m (block bi = hp / 2, columns 8 (hp % 2) ..) as a C fragment;
 // the diagonal blocks D_b are in sT.  sA's blocks are overwritten.
-__device__ __forceinline__ void solve_unit_lower(uint32_t sA, uint32_t sT, int ptid, float (&tv)[3][4]) {
+__device__ __forceinline__ void solve_unit_lower(uint32_t sA, uint32_t sT, int ptid, float (&tv)[3][4],
+                                                 [[maybe_unused]] int c, [[maybe_unused]] int nC) {
   if (ptid < 64) {                                    // D_b, column `col` of block b
     const int b = ptid >> 4, col = ptid & 15;
     const uint32_t Ab = blk(sA, b, b);
@@ -205,54 +224,84 @@ __device__ __forceinline__ void solve_unit_lower(uint32_t sA, uint32_t sT, int p
     for (int i = 0; i < 16; ++i) tc::sts1(at(Tb, i, col), x[i]);
   }
   tc::named_bar(1, 128);
+  if (ptid == 0) GDN_TRACE(c, 9);
   const int w = ptid >> 5, lane = ptid & 31, g = lane >> 2, t = lane & 3;
+  {                                                   // At_ik = D_i A_ik, into T's off-diagonal
+    Tile tl[3];
+    float acc[3][4] = {};
 #pragma unroll
-  for (int m = 0; m < 3; ++m) {                       // At_ik = D_i A_ik, into T's off-diagonal
-    const int hp = w + 4 * m, bi = hp >> 1, n0 = (hp & 1) * 8;
-    const int i = blk_i(bi), k = blk_k(bi, i);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    mma_blk(blk(sT, i, i), blk(sA, i, k), n0, g, t, acc);
-    st_frag(blk(sT, i, k), n0, g, t, acc);
-  }
-  tc::named_bar(1, 128);
-  // U_20 = -At_20 + At_21 At_10;  U_31 = -At_31 + At_32 At_21;  V_30 = -At_30 + At_31 At_10
-  // (into sA's blocks (2,0), (3,1), (3,0); A itself is no longer needed)
+    for (int m = 0; m < 3; ++m) {
+      const int hp = w + 4 * m, bi = hp >> 1, n0 = (hp & 1) * 8;
+      const int i = blk_i(bi), k = blk_k(bi, i);
+      tl[m] = Tile{blk(sT, i, i), blk(sA, i, k), n0};
+    }
+    mma_tiles(tl, g, t, acc);
 #pragma unroll
-  for (int m = 0; m < 2; ++m) {
-    const int hp = w + 4 * m;
-    if (hp < 6) {
-      const int bi = hp >> 1, n0 = (hp & 1) * 8;
-      const int oi = bi == 0 ? 2 : 3, ok = bi == 1 ? 1 : 0;    // output block (oi, ok)
-      const int xk = bi == 1 ? 2 : 1;                           // X = At_(oi, xk), Y = At_(xk, ok)
-      float acc[4];
-      ld_frag(blk(sT, oi, ok), n0, g, t, acc);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[e] = -acc[e];
-      mma_blk(blk(sT, oi, xk), blk(sT, xk, ok), n0, g, t, acc);
-      st_frag(blk(sA, oi, ok), n0, g, t, acc);
+    for (int m = 0; m < 3; ++m) {
+      const int hp = w + 4 * m, bi = hp >> 1, n0 = (hp & 1) * 8;
+      const int i = blk_i(bi), k = blk_k(bi, i);
+      st_frag(blk(sT, i, k), n0, g, t, acc[m]);
     }
   }
   tc::named_bar(1, 128);
+  if (ptid == 0) GDN_TRACE(c, 13);
+  // U_20 = -At_20 + At_21 At_10;  U_31 = -At_31 + At_32 At_21;  V_30 = -At_30 + At_31 At_10
+  // (into sA's blocks (2,0), (3,1), (3,0); A itself is no longer needed).  Half blocks w, w + 4.
+  {
+    const int nt = w < 2 ? 2 : 1;                     // warp-uniform
+    Tile tl[2];
+    float acc[2][4];
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const int hp = m < nt ? w + 4 * m : w, bi = hp >> 1, n0 = (hp & 1) * 8;
+      const int oi = bi == 0 ? 2 : 3, ok = bi == 1 ? 1 : 0;    // output block (oi, ok)
+      const int xk = bi == 1 ? 2 : 1;                           // X = At_(oi, xk), Y = At_(xk, ok)
+      ld_frag(blk(sT, oi, ok), n0, g, t, acc[m]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[m][e] = -acc[m][e];
+      tl[m] = Tile{blk(sT, oi, xk), blk(sT, xk, ok), n0};
+    }
+    mma_tiles(tl, g, t, acc);
+#pragma unroll
+    for (int m = 0; m < 2; ++m)
+      if (m < nt) {
+        const int hp = w + 4 * m, bi = hp >> 1, n0 = (hp & 1) * 8;
+        const int oi = bi == 0 ? 2 : 3, ok = bi == 1 ? 1 : 0;
+        st_frag(blk(sA, oi, ok), n0, g, t, acc[m]);
+      }
+  }
+  tc::named_bar(1, 128);
+  if (ptid == 0) GDN_TRACE(c, 14);
   if (w < 2) {                                        // U_30 = V_30 - At_32 U_20
     const int n0 = 8 * w;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f}, v[4];
-    mma_blk(blk(sT, 3, 2), blk(sA, 2, 0), n0, g, t, acc);
+    const Tile tl[1] = {Tile{blk(sT, 3, 2), blk(sA, 2, 0), n0}};
+    float acc[1][4] = {}, v[4];
     ld_frag(blk(sA, 3, 0), n0, g, t, v);
+    mma_tiles(tl, g, t, acc);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) v[e] -= acc[e];
+    for (int e = 0; e < 4; ++e) v[e] -= acc[0][e];
     st_frag(blk(sA, 3, 0), n0, g, t, v);
   }
   tc::named_bar(1, 128);
+  if (ptid == 0) GDN_TRACE(c, 15);
+  {                                                   // T_ik = U_ik D_k (U = -At next to diag)
+    Tile tl[3];
+    float acc[3][4] = {};
 #pragma unroll
-  for (int m = 0; m < 3; ++m) {                       // T_ik = U_ik D_k (U = -At next to diag)
-    const int hp = w + 4 * m, bi = hp >> 1, n0 = (hp & 1) * 8;
-    const int i = blk_i(bi), k = blk_k(bi, i);
-    const bool sub = (i == k + 1);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    mma_blk(sub ? blk(sT, i, k) : blk(sA, i, k), blk(sT, k, k), n0, g, t, acc);
-    const float sg = sub ? -1.f : 1.f;
+    for (int m = 0; m < 3; ++m) {
+      const int hp = w + 4 * m, bi = hp >> 1, n0 = (hp & 1) * 8;
+      const int i = blk_i(bi), k = blk_k(bi, i);
+      tl[m] = Tile{(i == k + 1) ? blk(sT, i, k) : blk(sA, i, k), blk(sT, k, k), n0};
+    }
+    mma_tiles(tl, g, t, acc);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) tv[m][e] = sg * acc[e];
+    for (int m = 0; m < 3; ++m) {
+      const int hp = w + 4 * m, bi = hp >> 1;
+      const int i = blk_i(bi), k = blk_k(bi, i);
+      const float sg = (i == k + 1) ? -1.f : 1.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) tv[m][e] = sg * acc[m][e];
+    }
   }
 }
 
@@ -369,6 +418,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
                     const float* __restrict__ S0, float* __restrict__ S_T, int T, int Hk, int Hv,
                     float scale) {
   constexpr bool kF32 = sizeof(Tout) == 4;
+  // X takes M as a hi + lo bf16 pair when o is fp32 (the layer, whose gated norm magnifies o's
+  // error); a bf16 o carries its own rounding, and one round-to-nearest bf16 copy of M suffices.
+  constexpr bool kSplitX = kF32;
   // Offsetting the __shared__ array itself (not a round trip through an integer) keeps every
   // access below a shared-memory access (ld/st.shared), not a generic one.
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -413,6 +465,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC);
+  if (threadIdx.x == 0) GDN_TRACE_G(0, 10);
 
   if (warp == 0) {
     // ------------------------------- TMA producer -------------------------------------------
@@ -496,7 +549,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         if (!ok) break;
         tc::tc_fence_after();
 #pragma unroll
-        for (int ks = 0; ks < 16; ++ks)
+        for (int ks = 0; ks < (kSplitX ? 16 : 8); ++ks)
           tc::mma_bf16(tmem + TM_X,
                        tc::sdesc_sw128(qk + ((ks >> 2) & 1) * 16384 + (ks & 3) * 32, 16, 1024),
                        tc::sdesc_sw128(sb + (ks < 8 ? OFF_MB : OFF_RD) + (ks & 7) * 2048, 16384, 1024),
@@ -681,7 +734,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       tc::named_bar(1, 128);
       if (ptid == 0) GDN_TRACE(c, 2);
       float tv[3][4];
-      solve_unit_lower(sA, sT, ptid, tv);
+      solve_unit_lower(sA, sT, ptid, tv, c, nC);
       if (ptid == 0) GDN_TRACE(c, 3);
       // T_b = T diag(beta): off-diagonal half blocks from the solve (C fragments), diagonal
       // strips from sT
@@ -810,13 +863,19 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     const long head = (long)bq * Hv + h;
     const bool leader = (q == 0 && lane == 0);
     [[maybe_unused]] const int ev = 10 * hh;
-    // 32 columns (32p ..) of M row r (this half) as two bf16 terms, hi into Mb and lo into the R'
-    // buffer, for the X MMA
+    // 32 columns (32p ..) of M row r (this half) for the X MMA: one round-to-nearest bf16 copy in Mb,
+    // or (kSplitX) a hi + lo pair, hi into Mb and lo into the R' buffer
     auto store_m32 = [&](const float (&m)[32], int p) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const uint32_t sw = tc::sw128(r, 4 * p + j);
-        st_split8(mb + sw, rd + sw, m + 8 * j);
+        if constexpr (kSplitX) {
+          st_split8(mb + sw, rd + sw, m + 8 * j);
+        } else {
+          const float* v = m + 8 * j;
+          tc::st_shared_v4(mb + sw, tc::pack_bf16(v[0], v[1]), tc::pack_bf16(v[2], v[3]),
+                           tc::pack_bf16(v[4], v[5]), tc::pack_bf16(v[6], v[7]));
+        }
       }
     };
     bool stop = false;
@@ -1021,6 +1080,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
 
   tc::tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) GDN_TRACE_G(nC - 1, 11);
   if (threadIdx.x == 0 && *abort_flag) record_error(kErrTimeout);
   if (warp == 1) {
     tc::tc_fence_after();
