@@ -30,7 +30,8 @@
 //   warp 0        TMA producer (Q, K tiles double-buffered; V single-buffered)
 //   warp 1        TMEM owner; issues the state-independent MMAs (S and P T_b)
 //   warp 2        issues the chain MMAs (X, Y and the state update)
-//   warps 4-7     "pre" warpgroup: gates (one chunk ahead), A, P, the triangular solve, T_b, A2
+//   warps 4-7     "pre" warpgroup: gates (one chunk ahead), A, P, the triangular solve, T_b
+//                 (A2's rows P T_b are written by the chain's O warps once their MMA is done)
 //   warps 8-11    chain warpgroup of value columns 0..63; warps 12-15 of columns 64..127
 // so the state-independent work of chunk c+1 overlaps the chain of chunk c.  The fp32 master state
 // lives in TMEM (the update MMA accumulates onto it); o leaves through shared memory and TMA
@@ -88,7 +89,7 @@ enum : int {
 static_assert(B_END <= NBAR, "barrier map");
 
 constexpr uint32_t ID_S = tc::idesc_bf16(128, 64, false, false);
-constexpr uint32_t ID_PT = tc::idesc_tf32(64, 64, false, true);
+constexpr uint32_t ID_PT = tc::idesc_tf32(128, 64, false, true);   // rows 64..127 unused
 constexpr uint32_t ID_X = tc::idesc_bf16(128, 128, false, true);
 constexpr uint32_t ID_Y = tc::idesc_bf16(128, 128, false, true);
 constexpr uint32_t ID_U = tc::idesc_bf16(128, 128, true, true);
@@ -442,12 +443,14 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       tc::mbar_init(bar(B_QK_FULL + s), 1);
       tc::mbar_init(bar(B_IN_EMPTY + s), 3);     // S, X and state-update MMAs read the tile
     }
-    const int ones[] = {B_S_FULL, B_S_EMPTY, B_PT_READY, B_PT_FULL, B_PT_EMPTY, B_PRE_FULL,
-                        B_A2_EMPTY, B_GATE, B_GATE + 1, B_GATE + 2, B_X_FULL, B_Y_FULL, B_D3_FULL,
-                        B_V_FULL, B_DRAIN, B_DRAIN + 1};
+    const int ones[] = {B_S_FULL, B_S_EMPTY, B_PT_READY, B_PT_FULL, B_A2_EMPTY, B_GATE,
+                        B_GATE + 1, B_GATE + 2, B_X_FULL, B_Y_FULL, B_D3_FULL, B_V_FULL, B_DRAIN,
+                        B_DRAIN + 1};
     for (int i : ones) tc::mbar_init(bar(i), 1);
-    const int twos[] = {B_R_FULL, B_D_FULL, B_M_READY, B_V_EMPTY, B_O_DONE, B_M_SCALED};
+    const int twos[] = {B_R_FULL, B_D_FULL, B_M_READY, B_V_EMPTY, B_O_DONE, B_M_SCALED,
+                        B_PT_EMPTY};
     for (int i : twos) tc::mbar_init(bar(i), 2);   // one arrive per column half
+    tc::mbar_init(bar(B_PRE_FULL), 3);             // T_b rows (pre) + P T_b rows (each half)
     *abort_flag = 0;
     tc::fence_barrier_init();
   }
@@ -825,30 +828,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         GDN_TRACE(c, 6);
       }
       if (ptid < 32 && c + 1 < nC) publish_gates(c + 1);
-      // A2 rows 0..63 = P T_b (64-row MMA: row r sits in lane (r % 16) + 32 (r / 16))
-      tc::mbar_wait(bar(B_PT_FULL), c & 1, abort_flag, kBudget);
-      if (ptid == 0) GDN_TRACE(c, 7);
-      tc::tc_fence_after();
-      {
-        float pv[64];
-        const int r = 16 * q + lane;
-        tmem_ld64(tmem + lane_off + TM_PT, pv);
-        tc::tmem_wait_ld();
-        if (lane < 16) {
-          const uint32_t a2_row = sb + OFF_A2 + r * 128;
-#pragma unroll
-          for (int cc = 0; cc < 8; ++cc) {
-            const uint32_t sw = (cc ^ (r & 7)) << 4;
-            st_split8(a2_row + sw, a2_row + 16384 + sw, pv + 8 * cc);
-          }
-        }
-      }
-      tc::tc_fence_before();
-      tc::fence_proxy_async_smem();
+      // A2 rows 0..63 = P T_b are written by the chain's O warps once the MMA is done
       stop = vote_abort(1, 128, abort_flag);
       if (ptid == 0) {
         tc::mbar_arrive(bar(B_PRE_FULL));
-        tc::mbar_arrive(bar(B_PT_EMPTY));
         GDN_TRACE(c, 8);
       }
     }
@@ -876,6 +859,31 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
           tc::st_shared_v4(mb + sw, tc::pack_bf16(v[0], v[1]), tc::pack_bf16(v[2], v[3]),
                            tc::pack_bf16(v[4], v[5]), tc::pack_bf16(v[6], v[7]));
         }
+      }
+    };
+    // A2 rows 0..63 = P T_b of chunk cn (O warps, q < 2): row r = TMEM lane r, this half takes
+    // columns 32 hh .. 32 hh + 31 of the 64
+    auto a2_top = [&](int cn) {
+      tc::mbar_wait(bar(B_PT_FULL), cn & 1, abort_flag, kBudget);
+      if (cn >= 1) tc::mbar_wait(bar(B_O_DONE), (cn - 1) & 1, abort_flag, kBudget);
+      if (leader && hh == 0) GDN_TRACE(cn, 16);
+      tc::tc_fence_after();
+      float pv[32];
+      tc::tmem_ld32(tmem + lane_off + TM_PT + 32 * hh, pv);
+      tc::tmem_wait_ld();
+      const uint32_t a2_row = sb + OFF_A2 + r * 128;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t sw = ((4 * hh + j) ^ (r & 7)) << 4;
+        st_split8(a2_row + sw, a2_row + 16384 + sw, pv + 8 * j);
+      }
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      tc::named_bar(id_lo, 64);
+      if (leader) {
+        if (hh == 0) GDN_TRACE(cn, 17);
+        tc::mbar_arrive(bar(B_PT_EMPTY));
+        tc::mbar_arrive(bar(B_PRE_FULL));
       }
     };
     bool stop = false;
@@ -907,6 +915,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         tc::mbar_arrive(bar(B_M_READY));
         tc::mbar_arrive(bar(B_M_SCALED));
       }
+      if (!stop && q < 2) a2_top(0);
     }
 
     for (int c = 0; c < nC && !stop; ++c) {
@@ -1074,6 +1083,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         if (hh == 0) GDN_TRACE(c, 52);
         tc::mbar_arrive(bar(B_M_SCALED));
       }
+      if (!stop && q < 2 && c + 1 < nC) a2_top(c + 1);
     }
     if (leader) tc::bulk_wait_all();               // every o tile has reached global memory
   }
