@@ -149,7 +149,7 @@ struct Tile {
   int n0;
 };
 // acc[m] (C fragments) += X_m Y_m[:, n0_m ..] for N independent tiles, as lo.hi + hi.lo + hi.hi
-// tf32 products (fp32-level accuracy), one k half at a time; the MMAs of the N tiles interleave.
+// tf32 products (fp32-level accuracy), one k half at a time; the MMAs of the tiles interleave.
 template <int N>
 __device__ __forceinline__ void mma_tiles(const Tile (&tl)[N], int g, int t, float (&acc)[N][4]) {
 #pragma unroll
@@ -239,13 +239,13 @@ __device__ __forceinline__ void solve_unit_lower(uint32_t sA, uint32_t sT, int p
     mma_tiles(tl, g, t, acc);
 #pragma unroll
     for (int m = 0; m < 3; ++m) {
-      const int hp = w + 4 * m, bi = hp >> 1, n0 = (hp & 1) * 8;
+      const int bi = (w + 4 * m) >> 1;
       const int i = blk_i(bi), k = blk_k(bi, i);
-      st_frag(blk(sT, i, k), n0, g, t, acc[m]);
+      st_frag(blk(sT, i, k), tl[m].n0, g, t, acc[m]);
     }
   }
   tc::named_bar(1, 128);
-  if (ptid == 0) GDN_TRACE(c, 13);
+  if (ptid == 0) GDN_TRACE(c, 23);
   // U_20 = -At_20 + At_21 At_10;  U_31 = -At_31 + At_32 At_21;  V_30 = -At_30 + At_31 At_10
   // (into sA's blocks (2,0), (3,1), (3,0); A itself is no longer needed).  Half blocks w, w + 4.
   {
@@ -266,13 +266,13 @@ __device__ __forceinline__ void solve_unit_lower(uint32_t sA, uint32_t sT, int p
 #pragma unroll
     for (int m = 0; m < 2; ++m)
       if (m < nt) {
-        const int hp = w + 4 * m, bi = hp >> 1, n0 = (hp & 1) * 8;
+        const int bi = (w + 4 * m) >> 1;
         const int oi = bi == 0 ? 2 : 3, ok = bi == 1 ? 1 : 0;
-        st_frag(blk(sA, oi, ok), n0, g, t, acc[m]);
+        st_frag(blk(sA, oi, ok), tl[m].n0, g, t, acc[m]);
       }
   }
   tc::named_bar(1, 128);
-  if (ptid == 0) GDN_TRACE(c, 14);
+  if (ptid == 0) GDN_TRACE(c, 24);
   if (w < 2) {                                        // U_30 = V_30 - At_32 U_20
     const int n0 = 8 * w;
     const Tile tl[1] = {Tile{blk(sT, 3, 2), blk(sA, 2, 0), n0}};
@@ -284,7 +284,7 @@ __device__ __forceinline__ void solve_unit_lower(uint32_t sA, uint32_t sT, int p
     st_frag(blk(sA, 3, 0), n0, g, t, v);
   }
   tc::named_bar(1, 128);
-  if (ptid == 0) GDN_TRACE(c, 15);
+  if (ptid == 0) GDN_TRACE(c, 25);
   {                                                   // T_ik = U_ik D_k (U = -At next to diag)
     Tile tl[3];
     float acc[3][4] = {};
@@ -297,13 +297,14 @@ __device__ __forceinline__ void solve_unit_lower(uint32_t sA, uint32_t sT, int p
     mma_tiles(tl, g, t, acc);
 #pragma unroll
     for (int m = 0; m < 3; ++m) {
-      const int hp = w + 4 * m, bi = hp >> 1;
+      const int bi = (w + 4 * m) >> 1;
       const int i = blk_i(bi), k = blk_k(bi, i);
       const float sg = (i == k + 1) ? -1.f : 1.f;
 #pragma unroll
       for (int e = 0; e < 4; ++e) tv[m][e] = sg * acc[m][e];
     }
   }
+  if (ptid == 0) GDN_TRACE(c, 26);
 }
 
 __device__ __forceinline__ bool vote_abort(uint32_t id, uint32_t n, volatile int* abort) {
@@ -332,6 +333,15 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
       : "memory");
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+// Store 16 consecutive fp32 TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16};" ::"r"(taddr),
+      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]),
+      "f"(v[8]), "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15])
+      : "memory");
 }
 // 64 consecutive fp32 TMEM columns of this thread's lane (no wait).
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
@@ -511,7 +521,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
           return false;
         tc::tc_fence_after();
         const uint32_t qk = sb + OFF_QK + s * QK_STAGE;
-#pragma unroll
+#pragma unroll 1
         for (int ks = 0; ks < 8; ++ks) {
           const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
           tc::mma_bf16(tmem + TM_S, tc::sdesc_sw128(qk + off, 16, 1024),
@@ -527,7 +537,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
              (c == 0 || tc::mbar_wait(bar(B_PT_EMPTY), (c - 1) & 1, abort_flag, kBudget));
         if (!ok) break;
         tc::tc_fence_after();
-#pragma unroll
+#pragma unroll 1
         for (int ks = 0; ks < 8; ++ks)   // P (64 x 64, K-major) x T_b (64 x 64, MN-major), tf32
           tc::mma_tf32(tmem + TM_PT,
                        tc::sdesc_sw128(sb + OFF_W + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024),
@@ -551,7 +561,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
              tc::mbar_wait(bar(B_M_READY), c & 1, abort_flag, kBudget);
         if (!ok) break;
         tc::tc_fence_after();
-#pragma unroll
+#pragma unroll 1
         for (int ks = 0; ks < (kSplitX ? 16 : 8); ++ks)
           tc::mma_bf16(tmem + TM_X,
                        tc::sdesc_sw128(qk + ((ks >> 2) & 1) * 16384 + (ks & 3) * 32, 16, 1024),
@@ -565,14 +575,14 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
              tc::mbar_wait(bar(B_PRE_FULL), c & 1, abort_flag, kBudget);
         if (!ok) break;
         tc::tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-#pragma unroll
-          for (int term = 0; term < 3; ++term)
-            tc::mma_bf16(tmem + TM_Y,
-                         tc::sdesc_sw128(sb + OFF_A2 + (term == 1 ? 16384 : 0) + ks * 32, 16, 1024),
-                         tc::sdesc_sw128(sb + OFF_RD + (term == 2 ? 8192 : 0) + ks * 2048, 16384, 1024),
-                         ID_Y, (ks | term) > 0);
+#pragma unroll 1
+        for (int i = 0; i < 12; ++i) {
+          const int ks = i / 3, term = i - 3 * ks;
+          tc::mma_bf16(tmem + TM_Y,
+                       tc::sdesc_sw128(sb + OFF_A2 + (term == 1 ? 16384 : 0) + ks * 32, 16, 1024),
+                       tc::sdesc_sw128(sb + OFF_RD + (term == 2 ? 8192 : 0) + ks * 2048, 16384, 1024),
+                       ID_Y, i > 0);
+        }
         tc::mma_commit(bar(B_Y_FULL));
         tc::mma_commit(bar(B_A2_EMPTY));
         GDN_TRACE(c, 21);
@@ -581,7 +591,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
              tc::mbar_wait(bar(B_M_SCALED), c & 1, abort_flag, kBudget);
         if (!ok) break;
         tc::tc_fence_after();
-#pragma unroll
+#pragma unroll 1
         for (int ks = 0; ks < 8; ++ks)
           tc::mma_bf16(tmem + TM_M, tc::sdesc_sw128(qk + 8192 + (ks & 3) * 2048, 16384, 1024),
                        tc::sdesc_sw128(sb + OFF_RD + (ks >> 2) * 8192 + (ks & 3) * 2048, 16384, 1024),
@@ -627,8 +637,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       const float gl = __shfl_sync(0xffffffffu, incl, 31);
       constexpr float kLog2e = 1.4426950408889634f;
       gG[2 * lane] = g0 * kLog2e;    gG[2 * lane + 1] = g1 * kLog2e;
-      gGam[2 * lane] = expf(g0);     gGam[2 * lane + 1] = expf(g1);
-      gKt[2 * lane] = expf(gl - g0); gKt[2 * lane + 1] = expf(gl - g1);
+      gGam[2 * lane] = tc::ex2(g0 * kLog2e);     gGam[2 * lane + 1] = tc::ex2(g1 * kLog2e);
+      gKt[2 * lane] = tc::ex2((gl - g0) * kLog2e); gKt[2 * lane + 1] = tc::ex2((gl - g1) * kLog2e);
       gBeta[2 * lane] = be0;         gBeta[2 * lane + 1] = be1;
       if (lane == 0) *reinterpret_cast<volatile int*>(gE) = 0;   // non-finite A flag (E[0] unused)
       // block factors E[b][j] = exp(G_16b - G_j) for j < 16b (each <= 1: G never increases)
@@ -677,7 +687,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         const float4* g4 = reinterpret_cast<const float4*>(gG);
         const float4* e4p = reinterpret_cast<const float4*>(gE + 64 * ti);
         const int lim = is_p ? t + 1 : t;            // column j is kept when j < lim
-#pragma unroll
+#pragma unroll 1
         for (int p = 0; p < 2; ++p) {                // columns 32p .. 32p+31
           float sv[32];
           tc::tmem_ld32(tmem + lane_off + TM_S + 32 * p, sv);
@@ -797,22 +807,22 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       // A operand of P T_b
       if (ptid < 64) {
         const int t = ptid;
-        float pv[64];
-        tmem_ld64(tmem + lane_off + TM_S, pv);
-        tc::tmem_wait_ld();
         float sum = 0.f;
-#pragma unroll
+#pragma unroll 1
         for (int p = 0; p < 2; ++p) {
+          float pv[32];
+          tc::tmem_ld32(tmem + lane_off + TM_S + 32 * p, pv);
+          tc::tmem_wait_ld();
           const uint32_t prow = sb + OFF_W + p * 8192 + t * 128;
 #pragma unroll
           for (int cc = 0; cc < 8; ++cc) {
-            const float* v = pv + 32 * p + 4 * cc;
+            const float* v = pv + 4 * cc;
             sum += (v[0] + v[1]) + (v[2] + v[3]);
             st_tf32x4(prow + ((cc ^ (t & 7)) << 4), v[0], v[1], v[2], v[3]);
           }
         }
         if (nonfinite(sum)) {
-#pragma unroll
+#pragma unroll 1
           for (int p = 0; p < 2; ++p)
 #pragma unroll
             for (int cc = 0; cc < 8; ++cc)
@@ -930,7 +940,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         if (q == 2 && lane == 0) GDN_TRACE(c, 30 + ev);
         tc::tc_fence_after();
         const float g = gGam[t];
-#pragma unroll
+#pragma unroll 1
         for (int p = 0; p < 2; ++p) {            // value columns 32p .. 32p+31 of this half
           float x[32];
           tc::tmem_ld32(tmem + lane_off + TM_X + tcol + 32 * p, x);
@@ -968,7 +978,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         if (q == 2 && lane == 0) GDN_TRACE(c, 32 + ev);
         tc::tc_fence_after();
         const float kt = gKt[t];
-#pragma unroll
+#pragma unroll 1
         for (int p = 0; p < 2; ++p) {
           float y[32];
           tc::tmem_ld32(tmem + lane_off + TM_Y + tcol + 32 * p, y);
@@ -1002,7 +1012,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         const float g = gGam[t] * scale;
         // bf16: one [64 t][64 dv] tile per half; fp32: two [64 t][32 dv] tiles per half
         const uint32_t stage = sb + OFF_A2 + hh * (kF32 ? 16384 : 8192);
-#pragma unroll
+#pragma unroll 1
         for (int p = 0; p < 4; ++p) {            // value columns 16p .. 16p+15 of this half
           float x[16], y[16];
           tmem_ld16(tmem + lane_off + TM_X + tcol + 16 * p, x);
