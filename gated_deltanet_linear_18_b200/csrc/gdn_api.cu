@@ -3,6 +3,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "gdn.h"
 #include "common.cuh"
 #include "decode.cuh"
@@ -105,18 +107,46 @@ gdn_status decode_dispatch(int dk, int dv, const void* q, const void* k, const v
   return GDN_ERR_UNSUPPORTED;
 }
 
-// The recurrence inside gdn_layer_fwd: inputs in `dtype`, output o in fp32.
+// The recurrence inside gdn_layer_fwd: inputs in `dtype`, output o in fp32; `scratch` is the
+// tensor-core forward's hand-over buffer (part of the layer workspace).
 gdn_status layer_chunk_fwd(const void* q, const void* k, const void* v, const float* la,
                            const float* be, const float* S0, float* o, float* S_T, int B, int T,
                            int Hk, int Hv, int dk, int dv, int chunk, float scale,
-                           gdn_dtype dtype, cudaStream_t st) {
+                           gdn_dtype dtype, void* scratch, cudaStream_t st) {
   if (tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16))
-    return tc_chunk_launch_f32out(q, k, v, la, be, S0, o, S_T, B, T, Hk, Hv, scale, st);
+    return tc_chunk_launch_f32out(q, k, v, la, be, S0, o, S_T, B, T, Hk, Hv, scale, scratch, st);
   if (dtype == GDN_F32)
     return simt_dispatch<float, float>(dk, chunk, q, k, v, la, be, S0, o, S_T, B, T, Hk, Hv, dv,
                                        scale, st);
   return simt_dispatch<__nv_bfloat16, float>(dk, chunk, q, k, v, la, be, S0, o, S_T, B, T, Hk,
                                              Hv, dv, scale, st);
+}
+
+// The tensor-core forward's scratch comes from a library-private stream-ordered memory pool per
+// device that keeps its memory between calls (so a repeated call reuses it without a new
+// device allocation).
+std::mutex g_pool_mu;
+cudaMemPool_t g_pools[64] = {};
+
+gdn_status scratch_pool(cudaMemPool_t* out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GDN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_pool_mu);
+  if (!g_pools[dev]) {
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.handleTypes = cudaMemHandleTypeNone;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t p = nullptr;
+    if (cudaMemPoolCreate(&p, &props) != cudaSuccess) return GDN_ERR_CUDA;
+    uint64_t keep = ~0ull;
+    if (cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess)
+      return GDN_ERR_CUDA;
+    g_pools[dev] = p;
+  }
+  *out = g_pools[dev];
+  return GDN_OK;
 }
 
 gdn_status validate_heads(int Hk, int Hv, int dk, int dv) {
@@ -188,8 +218,18 @@ gdn_status gdn_chunk_fwd_ex(const void* q, const void* k, const void* v, const f
   }
   const bool tc_ok = tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16);
   if (variant == GDN_VARIANT_TCGEN05 && !tc_ok) return GDN_ERR_UNSUPPORTED;
-  if (tc_ok && variant != GDN_VARIANT_SIMT)
-    return tc_chunk_launch(q, k, v, log_alpha, beta, S0, o, S_T, B, T, Hk, Hv, scale, st);
+  if (tc_ok && variant != GDN_VARIANT_SIMT) {
+    cudaMemPool_t pool = nullptr;
+    s = scratch_pool(&pool);
+    if (s != GDN_OK) return s;
+    void* scratch = nullptr;
+    if (cudaMallocFromPoolAsync(&scratch, tc_chunk_scratch_bytes(B, T, Hv), pool, st) !=
+        cudaSuccess)
+      return GDN_ERR_CUDA;
+    s = tc_chunk_launch(q, k, v, log_alpha, beta, S0, o, S_T, B, T, Hk, Hv, scale, scratch, st);
+    const cudaError_t e = cudaFreeAsync(scratch, st);   // ordered after the kernels
+    return s != GDN_OK ? s : (e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA);
+  }
   if (dtype == GDN_F32)
     return simt_dispatch<float>(dk, chunk, q, k, v, log_alpha, beta, S0, o, S_T, B, T, Hk, Hv,
                                 dv, scale, st);
@@ -278,8 +318,11 @@ size_t gdn_layer_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, i
   const size_t el = dtype == GDN_F32 ? 4 : 2;
   const size_t tok = (size_t)B * T;
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-  // normalised q, k and convolved v in the storage dtype; the pre-norm output o in fp32
-  return 2 * up(tok * Hk * dk * el) + up(tok * Hv * dv * el) + up(tok * Hv * dv * 4);
+  // normalised q, k and convolved v in the storage dtype; the pre-norm output o in fp32; the
+  // tensor-core forward's hand-over buffer when that forward runs
+  const size_t tc = tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16)
+                        ? up(tc_chunk_scratch_bytes(B, T, Hv)) : 0;
+  return 2 * up(tok * Hk * dk * el) + up(tok * Hv * dv * el) + up(tok * Hv * dv * 4) + tc;
 }
 
 gdn_status gdn_layer_fwd(const void* q_raw, const void* k_raw, const void* v_raw, const void* z,
@@ -313,12 +356,14 @@ gdn_status gdn_layer_fwd(const void* q_raw, const void* k_raw, const void* v_raw
   void* kn = ws + up(tok * Hk * dk * el);
   void* vc = ws + 2 * up(tok * Hk * dk * el);
   void* o = ws + 2 * up(tok * Hk * dk * el) + up(tok * Hv * dv * el);
+  void* tc_scratch = static_cast<char*>(o) + up(tok * Hv * dv * 4);
   s = gdn_prologue(q_raw, k_raw, v_raw, wq, wk, wv, qn, kn, vc, B, T, Hk, Hv, dk, dv, l2_eps,
                    dtype, stream);
   if (s != GDN_OK) return s;
   // the recurrence writes o in fp32 so that the gated norm reads it unrounded
   s = layer_chunk_fwd(qn, kn, vc, log_alpha, beta, S0, static_cast<float*>(o), S_T, B, T, Hk, Hv,
-                      dk, dv, chunk, scale, dtype, reinterpret_cast<cudaStream_t>(stream));
+                      dk, dv, chunk, scale, dtype, tc_scratch,
+                      reinterpret_cast<cudaStream_t>(stream));
   if (s != GDN_OK) return s;
   const long long rows = (long long)tok * Hv;
   const long long blocks = (rows + 7) / 8;
@@ -338,7 +383,6 @@ gdn_status gdn_layer_fwd(const void* q_raw, const void* k_raw, const void* v_raw
 // ---------------------------------------------------------------------------------------------
 // gdn_layer_fwd_static: the whole layer with its scratch in the library's own device memory.
 // ---------------------------------------------------------------------------------------------
-#include <mutex>
 
 // The scratch is part of the library's device image: it exists on a device once the library's
 // device code is loaded there, and no call allocates or frees it.  Every byte the layer reads

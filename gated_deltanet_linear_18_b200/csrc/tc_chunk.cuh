@@ -419,6 +419,139 @@ __device__ __forceinline__ void store_tb2(uint32_t sb, int kr, int n, float a, f
 }
 
 // ------------------------------------------------------------------------------------------
+// pre-pass: T_b = (I + A)^-1 diag(beta) of every (batch, value head, chunk), independently
+// ------------------------------------------------------------------------------------------
+// T_b depends on nothing across chunks, so it is computed ahead of the recurrence by many small
+// CTAs at once and handed over through HBM as 10 packed 16 x 16 blocks (block (i, k), i >= k, at
+// index i(i+1)/2 + k, rows of 16 floats): 10 KB per chunk.  A = strict_lower(beta_i exp(G_i - G_j)
+// k_i . k_j) with k_i . k_j from bf16 warp MMAs (exact products, fp32 sums) and the blocked solve
+// above.  A chunk whose A holds a NaN or an infinity gets T_b = +inf everywhere (the solve's
+// warp MMAs may drop a NaN operand), so the recurrence still sees a non-finite value.
+constexpr int kTbFloats = 10 * 256;                 // floats per chunk
+constexpr int PP_THREADS = 128;
+constexpr int PP_KROW = 136;                        // K tile row stride in bf16 (272 bytes)
+constexpr uint32_t PP_OFF_G = 64 * PP_KROW * 2;     // 17408: G log2(e)[64], beta[64], flag
+constexpr uint32_t PP_OFF_A = PP_OFF_G + 1024;      // 18432: solve scratch, A then T
+constexpr uint32_t PP_SMEM = PP_OFF_A + 2 * SOLVE_T;   // 44032
+static_assert(PP_OFF_A % 16 == 0, "solve scratch alignment");
+
+__device__ __forceinline__ void mma_m16n8k16_bf16(float (&d)[4], const uint32_t (&a)[4],
+                                                  uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// grid (nC, Hv, B), 128 threads.
+__global__ void __launch_bounds__(PP_THREADS)
+tb_prepass_kernel(const __nv_bfloat16* __restrict__ k, const float* __restrict__ log_alpha,
+                  const float* __restrict__ beta, float* __restrict__ Tb, int T, int Hk, int Hv) {
+  extern __shared__ __align__(16) uint8_t pp_smem[];
+  const uint32_t sb = tc::smem_u32(pp_smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
+  const int c = blockIdx.x, h = blockIdx.y, bq = blockIdx.z, nC = gridDim.x;
+  const int hk = h / (Hv / Hk);
+  const long t0 = (long)c * C;
+  float* gG = reinterpret_cast<float*>(pp_smem + PP_OFF_G);
+  float* gB = gG + 64;
+  volatile int* flag = reinterpret_cast<volatile int*>(gG + 128);
+  const uint32_t sA = sb + PP_OFF_A, sT = sA + SOLVE_T;
+
+  // K tile, rows past T zero
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int idx = tid + PP_THREADS * i, row = idx >> 4, ch = idx & 15;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (t0 + row < T)
+      v = *reinterpret_cast<const uint4*>(k + (((long)bq * T + t0 + row) * Hk + hk) * 128 + ch * 8);
+    *reinterpret_cast<uint4*>(pp_smem + row * PP_KROW * 2 + ch * 16) = v;
+  }
+  // gates: G = cumsum(log alpha) over the chunk (log2-scaled), beta; zero past T
+  if (tid < 64) {
+    const long tt = t0 + tid;
+    const float la = tt < T ? log_alpha[((long)bq * T + tt) * Hv + h] : 0.f;
+    gB[tid] = tt < T ? beta[((long)bq * T + tt) * Hv + h] : 0.f;
+    float incl = la;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const float n = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += n;
+    }
+    gG[tid] = incl;
+  }
+  if (tid == 0) *flag = 0;
+  __syncthreads();
+  if (tid >= 32 && tid < 64) gG[tid] += gG[31];       // carry of the first 32 tokens
+  __syncthreads();
+  if (tid < 64) gG[tid] *= 1.4426950408889634f;
+  __syncthreads();
+
+  // k_t . k_j for the 20 16 x 8 tiles of the lower block triangle (tile (mi, ni) with
+  // 8 ni < 16 (mi + 1)), five per warp, then A = strict_lower(beta_t 2^(G'_t - G'_j) k_t . k_j)
+  // into the packed solve blocks
+  bool bad = false;
+#pragma unroll 1
+  for (int m = 0; m < 5; ++m) {
+    const int tile = warp + 4 * m;
+    // tile -> (mi, ni): mi = 0 holds tiles 0..1, mi = 1 tiles 2..5, mi = 2 tiles 6..11, mi = 3 12..19
+    const int mi = tile < 2 ? 0 : (tile < 6 ? 1 : (tile < 12 ? 2 : 3));
+    const int ni = tile - (mi == 0 ? 0 : (mi == 1 ? 2 : (mi == 2 ? 6 : 12)));
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint8_t* ra0 = pp_smem + (16 * mi + g) * PP_KROW * 2;
+    const uint8_t* ra1 = ra0 + 8 * PP_KROW * 2;
+    const uint8_t* rb = pp_smem + (8 * ni + g) * PP_KROW * 2;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const int kc = 16 * ks + 2 * t4;             // bf16 column of this lane's pair
+      const uint32_t a[4] = {*reinterpret_cast<const uint32_t*>(ra0 + kc * 2),
+                             *reinterpret_cast<const uint32_t*>(ra1 + kc * 2),
+                             *reinterpret_cast<const uint32_t*>(ra0 + (kc + 8) * 2),
+                             *reinterpret_cast<const uint32_t*>(ra1 + (kc + 8) * 2)};
+      mma_m16n8k16_bf16(acc, a, *reinterpret_cast<const uint32_t*>(rb + kc * 2),
+                        *reinterpret_cast<const uint32_t*>(rb + (kc + 8) * 2));
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int t = 16 * mi + g + 8 * (e >> 1), j = 8 * ni + 2 * t4 + (e & 1);
+      const float a = j < t ? gB[t] * tc::ex2(gG[t] - gG[j]) * acc[e] : 0.f;
+      bad |= !(fabsf(a) <= 3.402823466e38f);
+      tc::sts1(at(blk(sA, t >> 4, j >> 4), t & 15, j & 15), a);
+    }
+  }
+  if (bad) *flag = 1;
+  tc::named_bar(1, PP_THREADS);
+
+  float tv[3][4];
+  solve_unit_lower(sA, sT, tid, tv, c, nC);
+  const bool poison = *flag != 0;
+
+  // T_b = T diag(beta): off-diagonal half blocks (C fragments of the solve), diagonal blocks
+  float* out = Tb + (((long)bq * Hv + h) * nC + c) * kTbFloats;
+#pragma unroll
+  for (int m = 0; m < 3; ++m) {
+    const int hp = warp + 4 * m, bi = hp >> 1, n0 = (hp & 1) * 8;
+    const int i = blk_i(bi), kk = blk_k(bi, i);
+    const int col = n0 + 2 * t4;
+    const float b0 = gB[16 * kk + col], b1 = gB[16 * kk + col + 1];
+    float* ob = out + (i * (i + 1) / 2 + kk) * 256;
+    const float2 r0 = poison ? make_float2(kInf, kInf) : make_float2(tv[m][0] * b0, tv[m][1] * b1);
+    const float2 r1 = poison ? make_float2(kInf, kInf) : make_float2(tv[m][2] * b0, tv[m][3] * b1);
+    *reinterpret_cast<float2*>(ob + g * 16 + col) = r0;
+    *reinterpret_cast<float2*>(ob + (g + 8) * 16 + col) = r1;
+  }
+#pragma unroll
+  for (int m = 0; m < 2; ++m) {
+    const int id = tid + PP_THREADS * m, b = id >> 6, r = (id >> 2) & 15, cs = id & 3;
+    const float4 d = tc::lds4(at(blk(sT, b, b), r, 4 * cs));
+    const float4 be = *reinterpret_cast<const float4*>(gB + 16 * b + 4 * cs);
+    const float4 v = poison ? make_float4(kInf, kInf, kInf, kInf)
+                            : make_float4(d.x * be.x, d.y * be.y, d.z * be.z, d.w * be.w);
+    *reinterpret_cast<float4*>(out + (b * (b + 1) / 2 + b) * 256 + r * 16 + 4 * cs) = v;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
 // the kernel
 // ------------------------------------------------------------------------------------------
 template <typename Tout>
@@ -426,8 +559,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
                     const float* __restrict__ log_alpha, const float* __restrict__ beta,
-                    const float* __restrict__ S0, float* __restrict__ S_T, int T, int Hk, int Hv,
-                    float scale) {
+                    const float* __restrict__ Tb, const float* __restrict__ S0,
+                    float* __restrict__ S_T, int T, int Hk, int Hv, float scale) {
   constexpr bool kF32 = sizeof(Tout) == 4;
   // X takes M as a hi + lo bf16 pair when o is fp32 (the layer, whose gated norm magnifies o's
   // error); a bf16 o carries its own rounding, and one round-to-nearest bf16 copy of M suffices.
@@ -611,7 +744,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     const int ptid = threadIdx.x - 128;                 // = TMEM lane of this thread
     const int q = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
-    const uint32_t sA = sb + OFF_W, sT = sb + OFF_W + SOLVE_T;
     // gates, computed by warp 4 one chunk ahead: lane l holds tokens 2l, 2l+1 of the next chunk
     float pla0 = 0.f, pla1 = 0.f, pbe0 = 0.f, pbe1 = 0.f;
     auto load_gates = [&](int c) {
@@ -640,7 +772,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       gGam[2 * lane] = tc::ex2(g0 * kLog2e);     gGam[2 * lane + 1] = tc::ex2(g1 * kLog2e);
       gKt[2 * lane] = tc::ex2((gl - g0) * kLog2e); gKt[2 * lane + 1] = tc::ex2((gl - g1) * kLog2e);
       gBeta[2 * lane] = be0;         gBeta[2 * lane + 1] = be1;
-      if (lane == 0) *reinterpret_cast<volatile int*>(gE) = 0;   // non-finite A flag (E[0] unused)
       // block factors E[b][j] = exp(G_16b - G_j) for j < 16b (each <= 1: G never increases)
 #pragma unroll
       for (int b = 1; b < 4; ++b) {
@@ -656,6 +787,17 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       if (lane == 0) tc::mbar_arrive(bar(B_GATE + c % 3));   // release: orders the stores above
       if (c + 1 < nC) load_gates(c + 1);                      // after the arrive, never before it
     };
+    // T_b of a chunk from the pre-pass: this thread's items id = ptid + 128 m (m < 5) of the 640
+    // float4 of the 10 packed blocks (block id / 64, row (id / 4) % 16, columns 4 (id % 4) ..),
+    // loaded one chunk ahead
+    float4 tbv[5];
+    auto load_tb = [&](int cc) {
+      const float4* src =
+          reinterpret_cast<const float4*>(Tb + (((long)bq * Hv + h) * nC + cc) * kTbFloats);
+#pragma unroll
+      for (int m = 0; m < 5; ++m) tbv[m] = src[ptid + 128 * m];
+    };
+    load_tb(0);
     if (ptid < 32) {
       load_gates(0);
       publish_gates(0);
@@ -664,35 +806,26 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     for (int c = 0; c < nC && !stop; ++c) {
       if (ptid == 0) GDN_TRACE(c, 0);
       const float* gG = gslot(c);
-      const float* gBeta = gG + 192;
       const float* gE = gG + 256;
-      const uint32_t gbeta_u = tc::smem_u32(gBeta);
       tc::mbar_wait(bar(B_GATE + c % 3), (c / 3) & 1, abort_flag, kBudget);
       tc::mbar_wait(bar(B_S_FULL), c & 1, abort_flag, kBudget);
       if (ptid == 0) GDN_TRACE(c, 1);
       tc::tc_fence_after();
-      // Rows of S: threads 0..63 hold (q_t . k_j), threads 64..127 hold (k_t . k_j).  Both
-      // halves turn their row into P or A at once; exp(G_t - G_j) = 2^(G'_t - G'_j), G' = G log2 e.
-      //   P[t][j] = exp(G_t - G_j) (q_t . k_j) scale, j <= t  (kept in the same TMEM row, as fp32,
-      //             until the solve scratch is free for the tf32 copy)
-      //   A[t][j] = beta_t exp(G_t - G_j) (k_t . k_j),  j < t  (into the packed solve blocks)
-      {
-        const bool is_p = ptid < 64;
-        const int t = is_p ? ptid : ptid - 64, ti = t >> 4, tr = t & 15;
+      // Rows 0..63 of S hold (q_t . k_j): P[t][j] = exp(G_t - G_j) (q_t . k_j) scale for j <= t,
+      // kept in the same TMEM row as fp32 until it goes out as the tf32 A operand of P T_b;
+      // exp(G_t - G_j) = 2^(G'_t - G'_j), G' = G log2 e, inside t's 16-token block directly and
+      // across blocks as 2^(G'_t - G'_16ti) E[ti][j] (both factors <= 1)
+      if (ptid < 64) {
+        const int t = ptid, ti = t >> 4;
         const float gt = gG[t];
-        const float coef = is_p ? scale : gBeta[t];
-        // exp(G_t - G_j): inside t's 16-token block directly; across blocks as
-        // exp(G_t - G_16ti) * E[ti][j] (both factors <= 1)
-        const float rowf = coef * tc::ex2(gt - gG[16 * ti]);
+        const float rowf = scale * tc::ex2(gt - gG[16 * ti]);
         const float4* g4 = reinterpret_cast<const float4*>(gG);
         const float4* e4p = reinterpret_cast<const float4*>(gE + 64 * ti);
-        const int lim = is_p ? t + 1 : t;            // column j is kept when j < lim
 #pragma unroll 1
         for (int p = 0; p < 2; ++p) {                // columns 32p .. 32p+31
           float sv[32];
           tc::tmem_ld32(tmem + lane_off + TM_S + 32 * p, sv);
           tc::tmem_wait_ld();
-          if (p == 0 && ptid == 64) GDN_TRACE(c, 62);
 #pragma unroll
           for (int kb2 = 0; kb2 < 2; ++kb2) {
             const int kb = 2 * p + kb2;
@@ -712,7 +845,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                   const int j = 16 * kb + 4 * i + e;
-                  v[4 * i + e] = (j < lim) ? coef * tc::ex2(gt - gj[e]) * v[4 * i + e] : 0.f;
+                  v[4 * i + e] = (j <= t) ? scale * tc::ex2(gt - gj[e]) * v[4 * i + e] : 0.f;
                 }
               }
             } else {
@@ -720,89 +853,39 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
               for (int e = 0; e < 16; ++e) v[e] = 0.f;
             }
           }
-          if (is_p) {
-            tc::tmem_st32(tmem + lane_off + TM_S + 32 * p, sv);
-          } else {
-            float sum = 0.f;
-#pragma unroll
-            for (int e = 0; e < 32; ++e) sum += sv[e];
-            if (nonfinite(sum)) *reinterpret_cast<volatile int*>(const_cast<float*>(gE)) = 1;
-#pragma unroll
-            for (int kb2 = 0; kb2 < 2; ++kb2) {
-              const int kb = 2 * p + kb2;
-              if (kb <= ti) {
-                const uint32_t dst = at(blk(sA, ti, kb), tr, 0);
-#pragma unroll
-                for (int e4 = 0; e4 < 16; e4 += 4)
-                  tc::sts4(dst + 4 * e4, make_float4(sv[16 * kb2 + e4], sv[16 * kb2 + e4 + 1],
-                                                     sv[16 * kb2 + e4 + 2], sv[16 * kb2 + e4 + 3]));
-              }
-            }
-          }
+          tc::tmem_st32(tmem + lane_off + TM_S + 32 * p, sv);
         }
-        if (ptid == 64) GDN_TRACE(c, 63);
-        if (is_p) tc::tmem_wait_st();
+        tc::tmem_wait_st();
       }
-      tc::tc_fence_before();
-      tc::named_bar(1, 128);
       if (ptid == 0) GDN_TRACE(c, 2);
-      float tv[3][4];
-      solve_unit_lower(sA, sT, ptid, tv, c, nC);
-      if (ptid == 0) GDN_TRACE(c, 3);
-      // T_b = T diag(beta): off-diagonal half blocks from the solve (C fragments), diagonal
-      // strips from sT
-      const int pw = ptid >> 5, pg = (ptid & 31) >> 2, pt = ptid & 3;
-      float toff[3][4];
+      float4 cur[5];
 #pragma unroll
-      for (int m = 0; m < 3; ++m) {
-        const int hp = pw + 4 * m, bi = hp >> 1, n0 = (hp & 1) * 8;
-        const int k = blk_k(bi, blk_i(bi));
-        const float2 be = lds2(gbeta_u + 4 * (16 * k + n0 + 2 * pt));
-        toff[m][0] = tv[m][0] * be.x; toff[m][1] = tv[m][1] * be.y;
-        toff[m][2] = tv[m][2] * be.x; toff[m][3] = tv[m][3] * be.y;
-      }
-      float4 tdg[2];
-#pragma unroll
-      for (int m = 0; m < 2; ++m) {
-        const int id = ptid + 128 * m, b = id >> 6, r = (id >> 2) & 15, cs = id & 3;
-        const float4 d = tc::lds4(at(blk(sT, b, b), r, 4 * cs));
-        const float4 be = tc::lds4(gbeta_u + 4 * (16 * b + 4 * cs));
-        tdg[m] = make_float4(d.x * be.x, d.y * be.y, d.z * be.z, d.w * be.w);
-      }
+      for (int m = 0; m < 5; ++m) cur[m] = tbv[m];
+      if (c + 1 < nC) load_tb(c + 1);
       if (c >= 1) {   // A2 (and the o tile staged in it) is free once Y and the o stores are done
         tc::mbar_wait(bar(B_A2_EMPTY), (c - 1) & 1, abort_flag, kBudget);
         tc::mbar_wait(bar(B_O_DONE), (c - 1) & 1, abort_flag, kBudget);
       }
       if (ptid == 0) GDN_TRACE(c, 4);
-      tc::named_bar(1, 128);                     // the solve scratch is free from here on
-      if (ptid == 0) GDN_TRACE(c, 5);
+      // T_b into A2's rows 64..127 (bf16 hi / lo) and into the B operand of P T_b (tf32), zero
+      // above the diagonal; the P T_b operands of the previous chunk are free (S of this chunk
+      // was issued after, and completed after, that MMA)
       {
         float sum = 0.f;
 #pragma unroll
-        for (int m = 0; m < 3; ++m) sum += (toff[m][0] + toff[m][1]) + (toff[m][2] + toff[m][3]);
-#pragma unroll
-        for (int m = 0; m < 2; ++m) sum += (tdg[m].x + tdg[m].y) + (tdg[m].z + tdg[m].w);
-        // a non-finite A (the warp MMAs of the solve may drop a NaN) is flagged by its rows
-        const bool bad = nonfinite(sum) || *reinterpret_cast<volatile const int*>(gG + 256) != 0;
+        for (int m = 0; m < 5; ++m) sum += (cur[m].x + cur[m].y) + (cur[m].z + cur[m].w);
+        const bool bad = nonfinite(sum);
         const float4 inf4 = make_float4(kInf, kInf, kInf, kInf);
 #pragma unroll
-        for (int m = 0; m < 3; ++m) {
-          const int hp = pw + 4 * m, bi = hp >> 1, n0 = (hp & 1) * 8;
-          const int i = blk_i(bi), k = blk_k(bi, i);
-#pragma unroll
-          for (int h8 = 0; h8 < 2; ++h8) {
-            const int n = 16 * k + n0 + 2 * pt;
-            store_tb2(sb, 16 * i + pg + 8 * h8, n, bad ? kInf : toff[m][2 * h8],
-                      bad ? kInf : toff[m][2 * h8 + 1]);                    // below the diagonal
-            store_tb2(sb, 16 * k + pg + 8 * h8, 16 * i + n0 + 2 * pt, 0.f, 0.f);   // above
-          }
-        }
-#pragma unroll
-        for (int m = 0; m < 2; ++m) {
-          const int id = ptid + 128 * m, b = id >> 6, r = (id >> 2) & 15, cs = id & 3;
-          store_tb(sb, 16 * b + r, 16 * b + 4 * cs, bad ? inf4 : tdg[m]);
+        for (int m = 0; m < 5; ++m) {
+          const int id = ptid + 128 * m, bb = id >> 6, r = (id >> 2) & 15, cs = id & 3;
+          const int i = bb >= 6 ? 3 : (bb >= 3 ? 2 : (bb >= 1 ? 1 : 0));
+          const int k = bb - i * (i + 1) / 2;
+          store_tb(sb, 16 * i + r, 16 * k + 4 * cs, bad ? inf4 : cur[m]);
+          if (i > k) store_tb(sb, 16 * k + r, 16 * i + 4 * cs, make_float4(0.f, 0.f, 0.f, 0.f));
         }
       }
+      if (ptid == 0) GDN_TRACE(c, 5);
       // P rows (threads 0..63, warps 4 and 5): back from TMEM, rounded to tf32, into the K-major
       // A operand of P T_b
       if (ptid < 64) {
@@ -1140,10 +1223,16 @@ inline bool make_tile_map(CUtensorMap* m, const void* base, int H, int T, int B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Bytes of the T_b hand-over buffer between the pre-pass and the recurrence.
+inline size_t scratch_bytes(int B, int T, int Hv) {
+  const size_t nC = (size_t)(T + C - 1) / C;
+  return (size_t)B * Hv * nC * kTbFloats * sizeof(float);
+}
+
 template <typename Tout>
 gdn_status launch(const void* q, const void* k, const void* v, const float* la, const float* be,
                   const float* S0, Tout* o, float* S_T, int B, int T, int Hk, int Hv, float scale,
-                  cudaStream_t st) {
+                  float* tb, cudaStream_t st) {
   CUtensorMap mq, mk, mv, mo;
   if (!make_tile_map(&mq, q, Hk, T, B, false) || !make_tile_map(&mk, k, Hk, T, B, false) ||
       !make_tile_map(&mv, v, Hv, T, B, false) ||
@@ -1153,10 +1242,17 @@ gdn_status launch(const void* q, const void* k, const void* v, const float* la, 
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC) !=
       cudaSuccess)
     return GDN_ERR_CUDA;
+  if (cudaFuncSetAttribute(tb_prepass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           PP_SMEM) != cudaSuccess)
+    return GDN_ERR_CUDA;
   const long grid = (long)B * Hv;
-  if (grid > 0x7fffffffL) return GDN_ERR_UNSUPPORTED;
-  kern<<<(unsigned)grid, kThreads, SMEM_ALLOC, st>>>(mq, mk, mv, mo, la, be, S0, S_T, T, Hk, Hv,
-                                                     scale);
+  const int nC = (T + C - 1) / C;
+  if (grid > 0x7fffffffL || Hv > 65535 || B > 65535) return GDN_ERR_UNSUPPORTED;
+  tb_prepass_kernel<<<dim3(nC, Hv, B), PP_THREADS, PP_SMEM, st>>>(
+      static_cast<const __nv_bfloat16*>(k), la, be, tb, T, Hk, Hv);
+  if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+  kern<<<(unsigned)grid, kThreads, SMEM_ALLOC, st>>>(mq, mk, mv, mo, la, be, tb, S0, S_T, T, Hk,
+                                                     Hv, scale);
   return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -1172,18 +1268,23 @@ inline bool tc_chunk_supported(int dk, int dv, int chunk, bool bf16) {
   return bf16 && dk == 128 && dv == 128 && chunk == tcf::C;
 }
 
+// Scratch bytes of the tensor-core forward (the T_b hand-over buffer), 256-byte aligned.
+inline size_t tc_chunk_scratch_bytes(int B, int T, int Hv) { return tcf::scratch_bytes(B, T, Hv); }
+
 inline gdn_status tc_chunk_launch(const void* q, const void* k, const void* v, const float* la,
                                   const float* be, const float* S0, void* o, float* S_T, int B,
-                                  int T, int Hk, int Hv, float scale, cudaStream_t st) {
+                                  int T, int Hk, int Hv, float scale, void* scratch,
+                                  cudaStream_t st) {
   return tcf::launch<__nv_bfloat16>(q, k, v, la, be, S0, static_cast<__nv_bfloat16*>(o), S_T, B,
-                                    T, Hk, Hv, scale, st);
+                                    T, Hk, Hv, scale, static_cast<float*>(scratch), st);
 }
 
 inline gdn_status tc_chunk_launch_f32out(const void* q, const void* k, const void* v,
                                          const float* la, const float* be, const float* S0,
                                          float* o, float* S_T, int B, int T, int Hk, int Hv,
-                                         float scale, cudaStream_t st) {
-  return tcf::launch<float>(q, k, v, la, be, S0, o, S_T, B, T, Hk, Hv, scale, st);
+                                         float scale, void* scratch, cudaStream_t st) {
+  return tcf::launch<float>(q, k, v, la, be, S0, o, S_T, B, T, Hk, Hv, scale,
+                            static_cast<float*>(scratch), st);
 }
 
 }  // namespace gdn
