@@ -3,41 +3,37 @@
 //
 // Per value head and chunk, with the chunk-start state M = S^T (128 x 128, fp32), the chunk form of
 // the recurrence ("Chapitre 16 - Assembler un système de type Kimi K3", 16.2: matrix operations
-// inside each block, state handed from block to block) is computed as
-//   state-independent part:
-//     G = cumsum(log alpha), gamma = exp(G), S = [Q; K] K^T                (bf16 MMA, 128x64x128)
+// inside each block, state handed from block to block) splits into
+//   a state-independent part, for every chunk at once in a pre-pass (many small CTAs):
+//     G = cumsum(log alpha), gamma = exp(G), ktil_t = exp(G_last - G_t)
 //     P = lower_incl(exp(G_i - G_j) q_i.k_j) * scale,  A = strict_lower(beta_i exp(G_i - G_j) k_i.k_j)
-//     T = (I + A)^-1 (fp32, blocked by 16),  T_b = T diag(beta)
-//     A2 = [P T_b; T_b]                     (P T_b: tf32 MMA, 64x64x64)
-//   state-dependent chain (all 128 value columns at once):
-//     X = [Q; K] M                           (bf16 MMA, 128x128x128, M as a two-term bf16 split)
+//     T_b = (I + A)^-1 diag(beta)                     (fp32, blocked by 16)
+//     PT = P T_b,  W = (diag(ktil) K)^T T_b           (64 x 64 and 128 x 64)
+//   and the state-dependent chain, one CTA per (batch, value head), all 128 value columns at once:
+//     X = [Q; K] M                           (bf16 MMA, 128x128x128, M as one bf16 copy or a pair)
 //     R' = V - diag(gamma) (K M)             (rows 64..127 of X)
-//     Y = A2 R' = [P Delta; Delta]           (bf16 MMA, 128x128x64, three-term split of both
-//                                             operands), Delta = T_b (V - diag(gamma) K M)
-//     o = diag(gamma) scale (Q M) + P Delta  (rows 0..63 of X and Y)
-//     M <- gamma_last M + K^T (ktil Delta),  ktil = exp(G_last - G)
-//                                            (bf16 MMA on a two-term bf16 split of ktil Delta,
-//                                             accumulated onto gamma_last M kept in TMEM)
-// which is the token recurrence reorganised exactly (Delta's rows are beta_t (v_t - alpha_t
-// S_{t-1} k_t)).  Accumulations and the master state are fp32.  The operands that carry the state
-// through the chain (M, A2, R', ktil Delta) are split into bf16 pairs hi + lo (|x - hi - lo| <
-// 2^-14 |x|) and multiplied term by term (hi.hi + lo.hi + hi.lo where both sides are split): with
-// plain bf16, or even tf32, there the state's largest entries drift by a few percent (about one
-// percent for tf32) of its RMS.  The splits are integer mask / byte-permute operations (the
-// conversion instructions run at a quarter of the ALU rate).
+//     o = diag(gamma) scale (Q M) + PT R'    (rows 0..63 of X;  Y = PT R', bf16 MMA 128x128x64)
+//     M <- gamma_last M + W R'               (bf16 MMA accumulating onto gamma_last M in TMEM)
+// which is the token recurrence reorganised exactly: Delta = T_b R' has rows beta_t (v_t - alpha_t
+// S_{t-1} k_t), and M's update K^T diag(ktil) Delta is W R'.  Accumulations and the master state are
+// fp32.  The operands that carry the state through the chain (PT, W, R') are bf16 pairs hi + lo
+// (|x - hi - lo| < 2^-14 |x|) multiplied term by term (hi.hi + lo.hi + hi.lo): with plain bf16, or
+// even tf32, the state's largest entries drift by a few percent (about one percent for tf32) of its
+// RMS.  The splits are integer mask / byte-permute operations (the conversion instructions run at a
+// quarter of the ALU rate).
 //
-// One CTA per (batch, value head), 512 threads in specialised warps:
-//   warp 0        TMA producer (Q, K tiles double-buffered; V single-buffered)
-//   warp 1        TMEM owner; issues the state-independent MMAs (S and P T_b)
-//   warp 2        issues the chain MMAs (X, Y and the state update)
-//   warps 4-7     "pre" warpgroup: gates (one chunk ahead), A, P, the triangular solve, T_b
-//                 (A2's rows P T_b are written by the chain's O warps once their MMA is done)
-//   warps 8-11    chain warpgroup of value columns 0..63; warps 12-15 of columns 64..127
-// so the state-independent work of chunk c+1 overlaps the chain of chunk c.  The fp32 master state
-// lives in TMEM (the update MMA accumulates onto it); o leaves through shared memory and TMA
-// stores.  Every wait is bounded (about 2 s): on expiry the CTA records the library's timeout bit,
-// every role leaves its loop at the next uniform check point, in-flight TMA copies and MMAs are
-// drained, TMEM is released and the kernel returns.
+// The pre-pass hands each chunk to the recurrence as its MMA operands themselves (48 KB of
+// swizzled tiles plus gamma), so the recurrence's critical path holds only X, R', the state
+// update and the state's bf16 copy.  Recurrence CTA, 384 threads in specialised warps:
+//   warp 0        TMA producer (Q, K tiles and the chunk's operand tiles, double-buffered)
+//   warp 1        TMEM owner; issues every MMA (X, the state update, then Y)
+//   warps 4-7     value columns 0..63; warps 8-11 columns 64..127.  Lanes 0..63 of each group
+//                 make o, lanes 64..127 make R' (V comes straight into registers one chunk
+//                 ahead); all four warps copy the updated state out of TMEM.
+// The fp32 master state lives in TMEM (the update MMA accumulates onto it); o leaves through
+// shared memory and TMA stores.  Every wait is bounded (about 2 s): on expiry the CTA records the
+// library's timeout bit, every role leaves its loop at the next uniform check point, in-flight TMA
+// copies and MMAs are drained, TMEM is released and the kernel returns.
 #pragma once
 
 #include <cuda.h>
@@ -50,49 +46,39 @@ namespace gdn {
 namespace tcf {
 
 constexpr int C = 64;
-constexpr int kThreads = 512;
+constexpr int kThreads = 384;
 constexpr uint64_t kBudget = 4000000000ull;   // wait budget in SM cycles (about 2 s)
 
 // shared memory map (bytes from a 1024-aligned base); every MMA tile is 128-byte swizzled
 constexpr uint32_t OFF_QK = 0;          // 2 stages x 32 KB: kb0 [Q 64 rows | K 64 rows], kb1 [...]
 constexpr uint32_t QK_STAGE = 32768;
-constexpr uint32_t OFF_V = 65536;       // 16 KB: V[t][64 dv] bf16, one 8 KB tile per column half
-constexpr uint32_t OFF_RD = 81920;      // 32 KB, per column half 16 KB: the bf16 low part of M
-                                        // [128 dk][128 B] for X, then R' bf16 hi [64 t][128 B] +
-                                        // lo, then ktil Delta bf16 hi [64 t][128 B] + lo
-constexpr uint32_t OFF_A2 = 114688;     // 32 KB: A2 bf16 hi [128 rows][128 B] + lo; between the
-                                        // Y MMA and the next chunk's A2 it stages the o tile
-constexpr uint32_t OFF_MB = 147456;     // 32 KB, per column half 16 KB: bf16 M [128 dk][128 B]
-constexpr uint32_t OFF_W = 180224;      // 32 KB: solve scratch, then P (tf32) and T_b (tf32)
-constexpr uint32_t OFF_WT = OFF_W + 16384;   // T_b, [dv block][64 rows][128 B]
-constexpr uint32_t SOLVE_T = 12800;     // byte offset of T inside the solve scratch
-constexpr uint32_t OFF_GB = 212992;     // 3 slots x 2 KB: G log2(e)[64], gamma[64], ktil[64],
-                                        // beta[64], E[4][64] (E[b][j] = exp(G_16b - G_j), j < 16b)
-constexpr uint32_t GB_SLOT = 2048;
-constexpr uint32_t OFF_BAR = OFF_GB + 3 * GB_SLOT;
-constexpr int NBAR = 26;
+constexpr uint32_t OFF_RD = 65536;      // 32 KB, per column half 16 KB: R' bf16 hi [64 t][128 B] +
+                                        // lo; with a split X first the bf16 low part of M
+constexpr uint32_t OFF_MB = 98304;      // 32 KB, per column half 16 KB: bf16 M [128 dk][128 B]
+constexpr uint32_t OFF_PW = 131072;     // 2 slots x 48 KB: a chunk's PT hi, PT lo, W hi, W lo;
+constexpr uint32_t PW_SLOT = 49152;     // after Y (and the update) the o tile is staged there
+constexpr uint32_t OFF_BAR = OFF_PW + 2 * PW_SLOT;
+constexpr int NBAR = 20;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;   // +0 TMEM base, +4 abort flag
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
-static_assert(2 * SOLVE_T <= 32768, "solve scratch");
 
-// TMEM columns (512 allocated, 128 lanes x 32 bit)
-constexpr uint32_t TM_S = 0, TM_PT = 64, TM_X = 128, TM_Y = 256, TM_M = 384;
+// TMEM columns (512 allocated, 128 lanes x 32 bit): X double-buffered by chunk parity
+constexpr uint32_t TM_X = 0, TM_Y = 256, TM_M = 384;
 
 // mbarriers
+// The chunk's operand slot arrives in two parts with their own barriers: W (for the state update,
+// on the critical path) is reloaded as soon as the update has read it; PT (for o) once o has
+// left the slot.
 enum : int {
-  B_QK_FULL = 0, B_IN_EMPTY = 2, B_S_FULL = 4, B_S_EMPTY, B_PT_READY, B_PT_FULL, B_PT_EMPTY,
-  B_PRE_FULL, B_A2_EMPTY, B_GATE, B_X_FULL = B_GATE + 3, B_R_FULL, B_Y_FULL, B_D_FULL, B_D3_FULL,
-  B_M_READY, B_V_FULL, B_V_EMPTY, B_O_DONE, B_M_SCALED, B_DRAIN, B_END = B_DRAIN + 2
+  B_QK_FULL = 0, B_QK_EMPTY = 2, B_W_FULL = 4, B_W_EMPTY = 6, B_P_FULL = 8, B_P_EMPTY = 10,
+  B_X_FULL = 12, B_R_FULL, B_D3_FULL, B_Y_FULL, B_Y_EMPTY, B_M_READY, B_M_SCALED, B_DRAIN, B_END
 };
 static_assert(B_END <= NBAR, "barrier map");
 
-constexpr uint32_t ID_S = tc::idesc_bf16(128, 64, false, false);
-constexpr uint32_t ID_PT = tc::idesc_tf32(128, 64, false, true);   // rows 64..127 unused
 constexpr uint32_t ID_X = tc::idesc_bf16(128, 128, false, true);
 constexpr uint32_t ID_Y = tc::idesc_bf16(128, 128, false, true);
-constexpr uint32_t ID_U = tc::idesc_bf16(128, 128, true, true);
 
 // Optional per-chunk timestamps for studying the pipeline (compiled only with GDN_TC_TRACE):
 // slot (block, chunk, event) of a caller-provided buffer receives clock64().
@@ -107,7 +93,13 @@ __device__ unsigned long long* g_tc_trace = nullptr;
   do {                                                                                \
     if (g_tc_trace) g_tc_trace[((size_t)blockIdx.x * nC + (c)) * 64 + (ev)] = tc::globaltimer_ns(); \
   } while (0)
+#define GDN_TRACE_PP(ev)                                                               \
+  do {                                                                                 \
+    if (g_tc_trace && threadIdx.x == 0)                                                \
+      g_tc_trace[(((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * 64 + (ev)] = clock64(); \
+  } while (0)
 #else
+#define GDN_TRACE_PP(ev) do {} while (0)
 #define GDN_TRACE(c, ev) do {} while (0)
 #define GDN_TRACE_G(c, ev) do {} while (0)
 #endif
@@ -198,8 +190,7 @@ __device__ __forceinline__ void st_frag(uint32_t B, int n0, int g, int t, const 
 // as warp MMAs on 16 x 8 half blocks.  On return the off-diagonal blocks of T are in `tv`: item m
 // of warp w is half block hp = w + 4 m (block bi = hp / 2, columns 8 (hp % 2) ..) as a C fragment;
 // the diagonal blocks D_b are in sT.  sA's blocks are overwritten.
-__device__ __forceinline__ void solve_unit_lower(uint32_t sA, uint32_t sT, int ptid, float (&tv)[3][4],
-                                                 [[maybe_unused]] int c, [[maybe_unused]] int nC) {
+__device__ __forceinline__ void solve_unit_lower(uint32_t sA, uint32_t sT, int ptid, float (&tv)[3][4]) {
   if (ptid < 64) {                                    // D_b, column `col` of block b
     const int b = ptid >> 4, col = ptid & 15;
     const uint32_t Ab = blk(sA, b, b);
@@ -225,7 +216,6 @@ __device__ __forceinline__ void solve_unit_lower(uint32_t sA, uint32_t sT, int p
     for (int i = 0; i < 16; ++i) tc::sts1(at(Tb, i, col), x[i]);
   }
   tc::named_bar(1, 128);
-  if (ptid == 0) GDN_TRACE(c, 9);
   const int w = ptid >> 5, lane = ptid & 31, g = lane >> 2, t = lane & 3;
   {                                                   // At_ik = D_i A_ik, into T's off-diagonal
     Tile tl[3];
@@ -245,7 +235,6 @@ __device__ __forceinline__ void solve_unit_lower(uint32_t sA, uint32_t sT, int p
     }
   }
   tc::named_bar(1, 128);
-  if (ptid == 0) GDN_TRACE(c, 23);
   // U_20 = -At_20 + At_21 At_10;  U_31 = -At_31 + At_32 At_21;  V_30 = -At_30 + At_31 At_10
   // (into sA's blocks (2,0), (3,1), (3,0); A itself is no longer needed).  Half blocks w, w + 4.
   {
@@ -272,7 +261,6 @@ __device__ __forceinline__ void solve_unit_lower(uint32_t sA, uint32_t sT, int p
       }
   }
   tc::named_bar(1, 128);
-  if (ptid == 0) GDN_TRACE(c, 24);
   if (w < 2) {                                        // U_30 = V_30 - At_32 U_20
     const int n0 = 8 * w;
     const Tile tl[1] = {Tile{blk(sT, 3, 2), blk(sA, 2, 0), n0}};
@@ -284,7 +272,6 @@ __device__ __forceinline__ void solve_unit_lower(uint32_t sA, uint32_t sT, int p
     st_frag(blk(sA, 3, 0), n0, g, t, v);
   }
   tc::named_bar(1, 128);
-  if (ptid == 0) GDN_TRACE(c, 25);
   {                                                   // T_ik = U_ik D_k (U = -At next to diag)
     Tile tl[3];
     float acc[3][4] = {};
@@ -304,7 +291,6 @@ __device__ __forceinline__ void solve_unit_lower(uint32_t sA, uint32_t sT, int p
       for (int e = 0; e < 4; ++e) tv[m][e] = sg * acc[m][e];
     }
   }
-  if (ptid == 0) GDN_TRACE(c, 26);
 }
 
 __device__ __forceinline__ bool vote_abort(uint32_t id, uint32_t n, volatile int* abort) {
@@ -357,18 +343,7 @@ __device__ __forceinline__ void tmem_st64(uint32_t taddr, const float (&v)[64]) 
   tc::tmem_st32(taddr + 32, b);
 }
 
-// Four fp32 values rounded to tf32, stored as one 16-byte chunk.
-__device__ __forceinline__ void st_tf32x4(uint32_t addr, float a, float b, float c, float d) {
-  tc::st_shared_v4(addr, tc::to_tf32(a), tc::to_tf32(b), tc::to_tf32(c), tc::to_tf32(d));
-}
-__device__ __forceinline__ void st_tf32x4(uint32_t addr, float4 v) {
-  st_tf32x4(addr, v.x, v.y, v.z, v.w);
-}
-// Non-finite guard for the tf32 operands.  The tensor cores' tf32 path does not carry a NaN operand
-// into the product, while it does carry an infinity; a thread whose tf32 values sum to a non-finite
-// value (any NaN or infinity among them; finite values near FLT_MAX can also trip it) rewrites them
-// as +infinity, so that a non-finite input still reaches o and the state as a non-finite value.
-__device__ __forceinline__ bool nonfinite(float sum) { return !(fabsf(sum) <= 3.402823466e38f); }
+// +infinity, written over the operands of a chunk whose P or A is not finite.
 constexpr float kInf = __builtin_huge_valf();
 
 // x = hi + lo + e with hi = x truncated to bf16 and lo = (x - hi) truncated to bf16, |e| < 2^-14 |x|;
@@ -390,84 +365,101 @@ __device__ __forceinline__ void st_split8(uint32_t hi_addr, uint32_t lo_addr, co
   tc::st_shared_v4(lo_addr, l[0], l[1], l[2], l[3]);
 }
 
-// Row `kr` (0..63), columns n..n+3 (n % 4 == 0) of T_b into its two operand layouts: rows 64..127
-// of the K-major bf16 hi / lo A2 (8 bytes of a 16-byte chunk each) and the MN-major tf32 B operand
-// of P T_b (32-byte chunks).
-__device__ __forceinline__ void store_tb(uint32_t sb, int kr, int n, float4 v) {
-  uint32_t h0, h1, l0, l1;
-  split2(v.x, v.y, h0, l0);
-  split2(v.z, v.w, h1, l1);
-  const uint32_t a2 = sb + OFF_A2 + (64 + kr) * 128 + (((n >> 3) ^ (kr & 7)) << 4) + (n & 7) * 2;
-  asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(a2), "r"(h0), "r"(h1) : "memory");
-  asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(a2 + 16384), "r"(l0), "r"(l1) : "memory");
-  st_tf32x4(sb + OFF_WT + (n >> 5) * 8192 + kr * 128 + ((((n & 31) >> 3) ^ (kr & 3)) << 5) +
-                ((n >> 2) & 1) * 16,
-            v);
-}
-
-// Same for two values (columns n, n + 1, n even).
-__device__ __forceinline__ void store_tb2(uint32_t sb, int kr, int n, float a, float b) {
-  uint32_t h, l;
-  split2(a, b, h, l);
-  const uint32_t a2 = sb + OFF_A2 + (64 + kr) * 128 + (((n >> 3) ^ (kr & 7)) << 4) + (n & 7) * 2;
-  asm volatile("st.shared.b32 [%0], %1;" ::"r"(a2), "r"(h) : "memory");
-  asm volatile("st.shared.b32 [%0], %1;" ::"r"(a2 + 16384), "r"(l) : "memory");
-  const uint32_t wt = sb + OFF_WT + (n >> 5) * 8192 + kr * 128 +
-                      ((((n & 31) >> 3) ^ (kr & 3)) << 5) + (n & 7) * 4;
-  asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(wt), "r"(tc::to_tf32(a)), "r"(tc::to_tf32(b))
-               : "memory");
-}
-
 // ------------------------------------------------------------------------------------------
-// pre-pass: T_b = (I + A)^-1 diag(beta) of every (batch, value head, chunk), independently
+// pre-pass: the state-independent operands of every (batch, value head, chunk), independently
 // ------------------------------------------------------------------------------------------
-// T_b depends on nothing across chunks, so it is computed ahead of the recurrence by many small
-// CTAs at once and handed over through HBM as 10 packed 16 x 16 blocks (block (i, k), i >= k, at
-// index i(i+1)/2 + k, rows of 16 floats): 10 KB per chunk.  A = strict_lower(beta_i exp(G_i - G_j)
-// k_i . k_j) with k_i . k_j from bf16 warp MMAs (exact products, fp32 sums) and the blocked solve
-// above.  A chunk whose A holds a NaN or an infinity gets T_b = +inf everywhere (the solve's
-// warp MMAs may drop a NaN operand), so the recurrence still sees a non-finite value.
-constexpr int kTbFloats = 10 * 256;                 // floats per chunk
+// With T_b = (I + A)^-1 diag(beta), P = lower_incl(exp(G_i - G_j) q_i.k_j) scale and
+// ktil_t = exp(G_last - G_t), the chunk needs from outside the state only
+//   PT = P T_b      (64 x 64: o = gamma scale Q M + PT R')
+//   W  = K^T diag(ktil) T_b   (128 x 64: M <- gamma_last M + W R')
+// since Delta = T_b R'.  Neither depends on the state, so one small CTA per chunk computes them
+// ahead of the recurrence, on the tensor cores: S = [Q; K] K^T (bf16 MMA into TMEM), P and A from
+// S with the gates (one TMEM row per thread), the blocked solve, then PT = P T_b and
+// W = K^T (ktil T_b) as bf16 MMAs on hi + lo splits (hi.hi + lo.hi + hi.lo for PT; K is exact, so
+// two terms for W).  The result goes to HBM as the recurrence's MMA operands themselves: per
+// chunk 48 KB of 128-byte-swizzled K-major bf16 tiles, PT hi [64 rows][128 B], PT lo, W hi [128
+// rows][128 B], W lo, followed by gamma_t = exp(G_t) (64 fp32).  A chunk whose P or A holds a NaN
+// or an infinity gets +inf in every tile, so the recurrence still sees a non-finite value.
+constexpr int kPwTiles = 49152;              // the four operand tiles of a chunk
+constexpr int kPwBytes = kPwTiles + 256;     // + gamma_t = exp(G_t), 64 fp32
 constexpr int PP_THREADS = 128;
-constexpr int PP_KROW = 136;                        // K tile row stride in bf16 (272 bytes)
-constexpr uint32_t PP_OFF_G = 64 * PP_KROW * 2;     // 17408: G log2(e)[64], beta[64], flag
-constexpr uint32_t PP_OFF_A = PP_OFF_G + 1024;      // 18432: solve scratch, A then T
-constexpr uint32_t PP_SMEM = PP_OFF_A + 2 * SOLVE_T;   // 44032
-static_assert(PP_OFF_A % 16 == 0, "solve scratch alignment");
+constexpr uint32_t PP_QK = 0;        // 32 KB: Q cols 0..63 | K cols 0..63 | Q 64..127 | K 64..127;
+                                     // P hi over the first Q box, P lo over the second
+constexpr uint32_t PP_TB = 32768;    // solve scratch, then 4 x 8 KB MN-major B tiles [64 rows][128 B]:
+                                     // T_b hi, T_b lo, ktil T_b hi, ktil T_b lo
+constexpr uint32_t PP_G = 65536;     // G'[64], beta[64], ktil[64], flag, abort, then at float 256
+                                     // E[4][64]; barriers at +3072
+constexpr uint32_t PP_BAR = PP_G + 3072;
+constexpr uint32_t PP_SMEM = PP_BAR + 64 + 1024;   // + alignment slack (three CTAs per SM)
+constexpr uint32_t SOLVE_T = 12800;  // byte offset of T inside the solve scratch
+static_assert(2 * SOLVE_T <= 32768, "solve scratch fits the B tiles' space");
+constexpr uint32_t ID_S = tc::idesc_bf16(128, 64, false, false);   // [Q; K] K^T
+constexpr uint32_t ID_PT = tc::idesc_bf16(128, 64, false, true);   // P T_b (rows 64..127 unused)
+constexpr uint32_t ID_W = tc::idesc_bf16(128, 64, true, true);     // K^T (ktil T_b)
 
-__device__ __forceinline__ void mma_m16n8k16_bf16(float (&d)[4], const uint32_t (&a)[4],
-                                                  uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-      "{%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+// Byte offset of element (r, j), j < 64, of a [rows][128 B] bf16 tile, 128-byte swizzle.
+__device__ __forceinline__ uint32_t sw_elem(int r, int j) {
+  return (uint32_t)(r * 128 + ((((j >> 3) ^ (r & 7))) << 4) + (j & 7) * 2);
+}
+// T_b values (row, n), (row, n + 1) (n even) into the four B tiles.
+__device__ __forceinline__ void store_tb_pair(uint32_t tb, int row, int n, float a, float b,
+                                              float kt) {
+  uint32_t h, l, kh, kl;
+  split2(a, b, h, l);
+  split2(kt * a, kt * b, kh, kl);
+  const uint32_t o = tb + sw_elem(row, n);
+  tc::sts1(o, __uint_as_float(h));
+  tc::sts1(o + 8192, __uint_as_float(l));
+  tc::sts1(o + 16384, __uint_as_float(kh));
+  tc::sts1(o + 24576, __uint_as_float(kl));
 }
 
-// grid (nC, Hv, B), 128 threads.
-__global__ void __launch_bounds__(PP_THREADS)
-tb_prepass_kernel(const __nv_bfloat16* __restrict__ k, const float* __restrict__ log_alpha,
-                  const float* __restrict__ beta, float* __restrict__ Tb, int T, int Hk, int Hv) {
-  extern __shared__ __align__(16) uint8_t pp_smem[];
-  const uint32_t sb = tc::smem_u32(pp_smem);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
+// grid (nC, Hv, B), 128 threads; thread r owns TMEM lane r.
+__global__ void __launch_bounds__(PP_THREADS, 3)
+pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                  const float* __restrict__ log_alpha, const float* __restrict__ beta,
+                  uint8_t* __restrict__ pw, int T, int Hk, int Hv, float scale) {
+  extern __shared__ __align__(1024) uint8_t pp_raw[];
+  uint8_t* smem = pp_raw + ((1024u - (tc::smem_u32(pp_raw) & 1023u)) & 1023u);
+  const uint32_t sb = tc::smem_u32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x, h = blockIdx.y, bq = blockIdx.z, nC = gridDim.x;
   const int hk = h / (Hv / Hk);
   const long t0 = (long)c * C;
-  float* gG = reinterpret_cast<float*>(pp_smem + PP_OFF_G);
+  float* gG = reinterpret_cast<float*>(smem + PP_G);
   float* gB = gG + 64;
-  volatile int* flag = reinterpret_cast<volatile int*>(gG + 128);
-  const uint32_t sA = sb + PP_OFF_A, sT = sA + SOLVE_T;
+  float* gKt = gG + 128;
+  volatile int* flag = reinterpret_cast<volatile int*>(gG + 192);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gG + 193);
+  const uint32_t tma_bar = sb + PP_BAR, mma_bar = sb + PP_BAR + 8;
+  const uint32_t qk = sb + PP_QK, tb = sb + PP_TB;
+  uint8_t* rec = pw + (((long)bq * Hv + h) * nC + c) * (long)kPwBytes;
 
-  // K tile, rows past T zero
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int idx = tid + PP_THREADS * i, row = idx >> 4, ch = idx & 15;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (t0 + row < T)
-      v = *reinterpret_cast<const uint4*>(k + (((long)bq * T + t0 + row) * Hk + hk) * 128 + ch * 8);
-    *reinterpret_cast<uint4*>(pp_smem + row * PP_KROW * 2 + ch * 16) = v;
+  if (tid == 0) {
+    tc::mbar_init(tma_bar, 1);
+    tc::mbar_init(mma_bar, 1);
+    *flag = 0;
+    *abort_flag = 0;
+    tc::fence_barrier_init();
   }
-  // gates: G = cumsum(log alpha) over the chunk (log2-scaled), beta; zero past T
+  if (warp == 0) {
+    tc::tmem_alloc(sb + PP_BAR + 16, 128);
+    tc::tmem_relinquish();
+    tc::tc_fence_before();
+  }
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + PP_BAR + 16);
+  const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
+  GDN_TRACE_PP(1);
+  if (tid == 0) {
+    tc::mbar_arrive_expect_tx(tma_bar, 32768);
+    tc::tma_load_4d(qk, &tmq, tma_bar, 0, hk, (int)t0, bq);
+    tc::tma_load_4d(qk + 8192, &tmk, tma_bar, 0, hk, (int)t0, bq);
+    tc::tma_load_4d(qk + 16384, &tmq, tma_bar, 64, hk, (int)t0, bq);
+    tc::tma_load_4d(qk + 24576, &tmk, tma_bar, 64, hk, (int)t0, bq);
+  }
+  // gates: G' = cumsum(log alpha) log2(e) over the chunk, beta, ktil, gamma (zero / flat past T)
   if (tid < 64) {
     const long tt = t0 + tid;
     const float la = tt < T ? log_alpha[((long)bq * T + tt) * Hv + h] : 0.f;
@@ -480,91 +472,226 @@ tb_prepass_kernel(const __nv_bfloat16* __restrict__ k, const float* __restrict__
     }
     gG[tid] = incl;
   }
-  if (tid == 0) *flag = 0;
   __syncthreads();
   if (tid >= 32 && tid < 64) gG[tid] += gG[31];       // carry of the first 32 tokens
   __syncthreads();
   if (tid < 64) gG[tid] *= 1.4426950408889634f;
   __syncthreads();
-
-  // k_t . k_j for the 20 16 x 8 tiles of the lower block triangle (tile (mi, ni) with
-  // 8 ni < 16 (mi + 1)), five per warp, then A = strict_lower(beta_t 2^(G'_t - G'_j) k_t . k_j)
-  // into the packed solve blocks
-  bool bad = false;
-#pragma unroll 1
-  for (int m = 0; m < 5; ++m) {
-    const int tile = warp + 4 * m;
-    // tile -> (mi, ni): mi = 0 holds tiles 0..1, mi = 1 tiles 2..5, mi = 2 tiles 6..11, mi = 3 12..19
-    const int mi = tile < 2 ? 0 : (tile < 6 ? 1 : (tile < 12 ? 2 : 3));
-    const int ni = tile - (mi == 0 ? 0 : (mi == 1 ? 2 : (mi == 2 ? 6 : 12)));
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const uint8_t* ra0 = pp_smem + (16 * mi + g) * PP_KROW * 2;
-    const uint8_t* ra1 = ra0 + 8 * PP_KROW * 2;
-    const uint8_t* rb = pp_smem + (8 * ni + g) * PP_KROW * 2;
+  float* gE = gG + 256;
+  if (tid < 64) {
+    gKt[tid] = tc::ex2(gG[63] - gG[tid]);
+    reinterpret_cast<float*>(rec + kPwTiles)[tid] = tc::ex2(gG[tid]);
+    // block factors E[b][j] = exp(G_16b - G_j) for j < 16b (each <= 1: G never increases)
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const int kc = 16 * ks + 2 * t4;             // bf16 column of this lane's pair
-      const uint32_t a[4] = {*reinterpret_cast<const uint32_t*>(ra0 + kc * 2),
-                             *reinterpret_cast<const uint32_t*>(ra1 + kc * 2),
-                             *reinterpret_cast<const uint32_t*>(ra0 + (kc + 8) * 2),
-                             *reinterpret_cast<const uint32_t*>(ra1 + (kc + 8) * 2)};
-      mma_m16n8k16_bf16(acc, a, *reinterpret_cast<const uint32_t*>(rb + kc * 2),
-                        *reinterpret_cast<const uint32_t*>(rb + (kc + 8) * 2));
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int t = 16 * mi + g + 8 * (e >> 1), j = 8 * ni + 2 * t4 + (e & 1);
-      const float a = j < t ? gB[t] * tc::ex2(gG[t] - gG[j]) * acc[e] : 0.f;
-      bad |= !(fabsf(a) <= 3.402823466e38f);
-      tc::sts1(at(blk(sA, t >> 4, j >> 4), t & 15, j & 15), a);
-    }
+    for (int b = 1; b < 4; ++b) gE[64 * b + tid] = tid < 16 * b ? tc::ex2(gG[16 * b] - gG[tid]) : 0.f;
   }
-  if (bad) *flag = 1;
-  tc::named_bar(1, PP_THREADS);
 
+  // S = [Q; K] K^T into TMEM columns 0..63
+  if (tid == 0) {
+    if (tc::mbar_wait(tma_bar, 0, abort_flag, kBudget)) {
+      GDN_TRACE_PP(2);
+      tc::tc_fence_after();
+      const uint64_t dq = tc::sdesc_sw128(qk, 16, 1024);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+        tc::mma_bf16(tmem, tc::desc_adv(dq, off), tc::desc_adv(dq, off + 8192), ID_S, ks > 0);
+      }
+    }
+    tc::mma_commit(mma_bar);
+  }
+  __syncthreads();                                    // gates visible
+  tc::mbar_wait(mma_bar, 0, abort_flag, kBudget);
+  GDN_TRACE_PP(3);
+  tc::tc_fence_after();
+  {
+    // row r of S: r < 64 is (q_t . k_j), r >= 64 is (k_t . k_j), t = r mod 64
+    float s[64];
+    tc::tmem_ld32(tmem + lane_off, *reinterpret_cast<float(*)[32]>(&s[0]));
+    tc::tmem_ld32(tmem + lane_off + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
+    tc::tmem_wait_ld();
+    // exp(G_t - G_j) = 2^(G'_t - G'_j) inside t's 16-token block directly, across blocks as
+    // 2^(G'_t - G'_16ti) E[ti][j] (both factors <= 1, so strong decay underflows to 0 instead of
+    // overflowing); P takes scale and j <= t, A takes beta_t and j < t
+    const int t = tid & 63, ti = t >> 4;
+    const bool isP = tid < 64;
+    const float gt = gG[t];
+    const float rowf = (isP ? scale : gB[t]) * tc::ex2(gt - gG[16 * ti]);
+    const float diagf = isP ? scale : gB[t];
+    const int jmax = isP ? t : t - 1;                 // last j kept
+    float sum = 0.f;
+#pragma unroll
+    for (int kb = 0; kb < 4; ++kb) {
+      float f[16];
+      if (kb < ti) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4 e = *reinterpret_cast<const float4*>(gE + 64 * ti + 16 * kb + 4 * i);
+          f[4 * i] = rowf * e.x; f[4 * i + 1] = rowf * e.y;
+          f[4 * i + 2] = rowf * e.z; f[4 * i + 3] = rowf * e.w;
+        }
+      } else if (kb == ti) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int j = 16 * kb + e;
+          f[e] = j <= jmax ? diagf * tc::ex2(gt - gG[j]) : 0.f;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) f[e] = 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        f[e] *= s[16 * kb + e];
+        sum += f[e];
+      }
+      if (isP) {                // P row t: K-major bf16 hi over the first Q box, lo over the second
+#pragma unroll
+        for (int h8 = 0; h8 < 2; ++h8) {
+          const int j8 = 2 * kb + h8;
+          const uint32_t o = qk + (uint32_t)(t * 128 + ((j8 ^ (t & 7)) << 4));
+          st_split8(o, o + 16384, f + 8 * h8);
+        }
+      } else if (kb <= ti) {    // A row t into the solve's packed 16 x 16 blocks
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          tc::sts4(at(blk(tb, ti, kb), t & 15, 4 * i),
+                   make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]));
+      }
+    }
+    if (!(fabsf(sum) <= 3.402823466e38f)) *flag = 1;
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+
+  GDN_TRACE_PP(4);
   float tv[3][4];
-  solve_unit_lower(sA, sT, tid, tv, c, nC);
-  const bool poison = *flag != 0;
-
-  // T_b = T diag(beta): off-diagonal half blocks (C fragments of the solve), diagonal blocks
-  float* out = Tb + (((long)bq * Hv + h) * nC + c) * kTbFloats;
-#pragma unroll
-  for (int m = 0; m < 3; ++m) {
-    const int hp = warp + 4 * m, bi = hp >> 1, n0 = (hp & 1) * 8;
-    const int i = blk_i(bi), kk = blk_k(bi, i);
-    const int col = n0 + 2 * t4;
-    const float b0 = gB[16 * kk + col], b1 = gB[16 * kk + col + 1];
-    float* ob = out + (i * (i + 1) / 2 + kk) * 256;
-    const float2 r0 = poison ? make_float2(kInf, kInf) : make_float2(tv[m][0] * b0, tv[m][1] * b1);
-    const float2 r1 = poison ? make_float2(kInf, kInf) : make_float2(tv[m][2] * b0, tv[m][3] * b1);
-    *reinterpret_cast<float2*>(ob + g * 16 + col) = r0;
-    *reinterpret_cast<float2*>(ob + (g + 8) * 16 + col) = r1;
-  }
+  solve_unit_lower(tb, tb + SOLVE_T, tid, tv);
+  GDN_TRACE_PP(5);
+  float4 dg[2];
 #pragma unroll
   for (int m = 0; m < 2; ++m) {
     const int id = tid + PP_THREADS * m, b = id >> 6, r = (id >> 2) & 15, cs = id & 3;
-    const float4 d = tc::lds4(at(blk(sT, b, b), r, 4 * cs));
-    const float4 be = *reinterpret_cast<const float4*>(gB + 16 * b + 4 * cs);
-    const float4 v = poison ? make_float4(kInf, kInf, kInf, kInf)
-                            : make_float4(d.x * be.x, d.y * be.y, d.z * be.z, d.w * be.w);
-    *reinterpret_cast<float4*>(out + (b * (b + 1) / 2 + b) * 256 + r * 16 + 4 * cs) = v;
+    dg[m] = tc::lds4(at(blk(tb + SOLVE_T, b, b), r, 4 * cs));
+  }
+  __syncthreads();                                    // the solve scratch is dead
+  {
+    const int g = lane >> 2, t4 = lane & 3;
+#pragma unroll
+    for (int m = 0; m < 3; ++m) {                     // off-diagonal blocks and their zero mirrors
+      const int hp = warp + 4 * m, bi = hp >> 1, n0 = (hp & 1) * 8;
+      const int i = blk_i(bi), kk = blk_k(bi, i);
+      const int col = 16 * kk + n0 + 2 * t4, row = 16 * i + g;
+      store_tb_pair(tb, row, col, tv[m][0] * gB[col], tv[m][1] * gB[col + 1], gKt[row]);
+      store_tb_pair(tb, row + 8, col, tv[m][2] * gB[col], tv[m][3] * gB[col + 1], gKt[row + 8]);
+      const int urow = 16 * kk + g, ucol = 16 * i + n0 + 2 * t4;
+      store_tb_pair(tb, urow, ucol, 0.f, 0.f, 0.f);
+      store_tb_pair(tb, urow + 8, ucol, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {                     // diagonal blocks (zero above the diagonal)
+      const int id = tid + PP_THREADS * m, b = id >> 6, r = (id >> 2) & 15, cs = id & 3;
+      const int row = 16 * b + r, col = 16 * b + 4 * cs;
+      store_tb_pair(tb, row, col, dg[m].x * gB[col], dg[m].y * gB[col + 1], gKt[row]);
+      store_tb_pair(tb, row, col + 2, dg[m].z * gB[col + 2], dg[m].w * gB[col + 3], gKt[row]);
+    }
+  }
+  tc::fence_proxy_async_smem();
+  tc::tc_fence_before();
+  __syncthreads();
+
+  // PT = P T_b (columns 64..127) and W = K^T (ktil T_b) (columns 0..63; S is consumed)
+  GDN_TRACE_PP(6);
+  if (tid == 0) {
+    tc::tc_fence_after();
+    const uint64_t dp = tc::sdesc_sw128(qk, 16, 1024);
+    const uint64_t dt = tc::sdesc_sw128(tb, 8192, 1024);
+    const uint64_t dk = tc::sdesc_sw128(qk + 8192, 16384, 1024);
+#pragma unroll
+    for (int i = 0; i < 12; ++i) {
+      const int ks = i / 3, term = i - 3 * ks;
+      tc::mma_bf16(tmem + 64, tc::desc_adv(dp, (term == 1 ? 16384 : 0) + ks * 32),
+                   tc::desc_adv(dt, (term == 2 ? 8192 : 0) + ks * 2048), ID_PT, i > 0);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int ks = i >> 1, term = i & 1;
+      tc::mma_bf16(tmem, tc::desc_adv(dk, ks * 2048), tc::desc_adv(dt, 16384 + term * 8192 + ks * 2048),
+                   ID_W, i > 0);
+    }
+    tc::mma_commit(mma_bar);
+  }
+  tc::mbar_wait(mma_bar, 1, abort_flag, kBudget);
+  GDN_TRACE_PP(7);
+  tc::tc_fence_after();
+  const bool poison = *flag != 0;
+  {
+    // staging in the record's order: PT hi [64][128 B], PT lo, W hi [128][128 B], W lo (every
+    // operand read by the MMAs above is dead)
+    float w[64];
+    tc::tmem_ld32(tmem + lane_off, *reinterpret_cast<float(*)[32]>(&w[0]));
+    tc::tmem_ld32(tmem + lane_off + 32, *reinterpret_cast<float(*)[32]>(&w[32]));
+    tc::tmem_wait_ld();
+    if (poison) {
+#pragma unroll
+      for (int j = 0; j < 64; ++j) w[j] = kInf;
+    }
+    __syncthreads();                                  // every thread is past its MMA-operand reads
+#pragma unroll
+    for (int j8 = 0; j8 < 8; ++j8) {
+      const uint32_t o = sb + 16384 + (uint32_t)(tid * 128 + ((j8 ^ (tid & 7)) << 4));
+      st_split8(o, o + 16384, w + 8 * j8);
+    }
+    if (tid < 64) {
+      tc::tmem_ld32(tmem + lane_off + 64, *reinterpret_cast<float(*)[32]>(&w[0]));
+      tc::tmem_ld32(tmem + lane_off + 96, *reinterpret_cast<float(*)[32]>(&w[32]));
+      tc::tmem_wait_ld();
+      if (poison) {
+#pragma unroll
+        for (int j = 0; j < 64; ++j) w[j] = kInf;
+      }
+#pragma unroll
+      for (int j8 = 0; j8 < 8; ++j8) {
+        const uint32_t o = sb + (uint32_t)(tid * 128 + ((j8 ^ (tid & 7)) << 4));
+        st_split8(o, o + 8192, w + 8 * j8);
+      }
+    }
+  }
+  tc::fence_proxy_async_smem();
+  tc::tc_fence_before();
+  __syncthreads();
+  GDN_TRACE_PP(8);
+  if (tid == 0) {
+    tc::bulk_store(rec, sb, kPwTiles);
+    tc::bulk_commit();
+    tc::bulk_wait_read_all();                         // the source may be released; the write
+                                                      // completes on its own
+    GDN_TRACE_PP(9);
+    if (*abort_flag) record_error(kErrTimeout);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 128);
   }
 }
 
 // ------------------------------------------------------------------------------------------
-// the kernel
+// the recurrence
 // ------------------------------------------------------------------------------------------
 template <typename Tout>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                    const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
-                    const float* __restrict__ log_alpha, const float* __restrict__ beta,
-                    const float* __restrict__ Tb, const float* __restrict__ S0,
+                    const __grid_constant__ CUtensorMap tmo, const __nv_bfloat16* __restrict__ v,
+                    const uint8_t* __restrict__ pw, const float* __restrict__ S0,
                     float* __restrict__ S_T, int T, int Hk, int Hv, float scale) {
   constexpr bool kF32 = sizeof(Tout) == 4;
   // X takes M as a hi + lo bf16 pair when o is fp32 (the layer, whose gated norm magnifies o's
   // error); a bf16 o carries its own rounding, and one round-to-nearest bf16 copy of M suffices.
   constexpr bool kSplitX = kF32;
+  // The low half of a split M shares the R' buffer, so there Y (which reads R') runs before the
+  // state update; otherwise the update, which the next chunk waits for, goes first.
+  constexpr bool kYFirst = kSplitX;
   // Offsetting the __shared__ array itself (not a round trip through an integer) keeps every
   // access below a shared-memory access (ld/st.shared), not a generic one.
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -576,24 +703,22 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   const int bq = blockIdx.x / Hv;
   const int hk = h / (Hv / Hk);
   const int nC = (T + C - 1) / C;
+  const long head = (long)bq * Hv + h;
+  const uint8_t* pw_head = pw + head * nC * (long)kPwBytes;
   auto bar = [&](int i) -> uint32_t { return sb + OFF_BAR + 8u * i; };
-  auto gslot = [&](int c) -> float* {
-    return reinterpret_cast<float*>(smem + OFF_GB + (c % 3) * GB_SLOT);
-  };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(bar(B_QK_FULL + s), 1);
-      tc::mbar_init(bar(B_IN_EMPTY + s), 3);     // S, X and state-update MMAs read the tile
-    }
-    const int ones[] = {B_S_FULL, B_S_EMPTY, B_PT_READY, B_PT_FULL, B_A2_EMPTY, B_GATE,
-                        B_GATE + 1, B_GATE + 2, B_X_FULL, B_Y_FULL, B_D3_FULL, B_V_FULL, B_DRAIN,
-                        B_DRAIN + 1};
+    const int ones[] = {B_QK_FULL, B_QK_FULL + 1, B_QK_EMPTY, B_QK_EMPTY + 1, B_W_FULL,
+                        B_W_FULL + 1, B_P_FULL, B_P_FULL + 1, B_X_FULL, B_D3_FULL, B_Y_FULL, B_DRAIN};
     for (int i : ones) tc::mbar_init(bar(i), 1);
-    const int twos[] = {B_R_FULL, B_D_FULL, B_M_READY, B_V_EMPTY, B_O_DONE, B_M_SCALED,
-                        B_PT_EMPTY};
+    const int twos[] = {B_R_FULL, B_Y_EMPTY, B_M_READY, B_M_SCALED};
     for (int i : twos) tc::mbar_init(bar(i), 2);   // one arrive per column half
-    tc::mbar_init(bar(B_PRE_FULL), 3);             // T_b rows (pre) + P T_b rows (each half)
+    // the MMAs that read a part, and the o stores of both halves staged in it (an fp32 o tile
+    // spills into W's part)
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(bar(B_P_EMPTY + s), 3);
+      tc::mbar_init(bar(B_W_EMPTY + s), kF32 ? 3 : 1);
+    }
     *abort_flag = 0;
     tc::fence_barrier_init();
   }
@@ -605,7 +730,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   if (warp == 0 && lane == 0) {
     tc::tma_prefetch_desc(&tmq);
     tc::tma_prefetch_desc(&tmk);
-    tc::tma_prefetch_desc(&tmv);
     tc::tma_prefetch_desc(&tmo);
   }
   __syncthreads();
@@ -614,13 +738,13 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   if (threadIdx.x == 0) GDN_TRACE_G(0, 10);
 
   if (warp == 0) {
-    // ------------------------------- TMA producer -------------------------------------------
+    // ------------------------------- loads ----------------------------------------------------
     if (lane == 0) {
-      int armed_qk[2] = {-1, -1}, armed_v = -1;
+      int armed_qk[2] = {-1, -1}, armed_w[2] = {-1, -1}, armed_p[2] = {-1, -1};
       bool ok = true;
       for (int c = 0; c < nC && ok; ++c) {
         const int s = c & 1, t0 = c * C;
-        if (c >= 2) ok = tc::mbar_wait(bar(B_IN_EMPTY + s), ((c >> 1) - 1) & 1, abort_flag, kBudget);
+        if (c >= 2) ok = tc::mbar_wait(bar(B_QK_EMPTY + s), ((c >> 1) - 1) & 1, abort_flag, kBudget);
         if (!ok) break;
         const uint32_t dst = sb + OFF_QK + s * QK_STAGE;
         tc::mbar_arrive_expect_tx(bar(B_QK_FULL + s), 32768);
@@ -629,316 +753,116 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         tc::tma_load_4d(dst + 16384, &tmq, bar(B_QK_FULL + s), 64, hk, t0, bq);
         tc::tma_load_4d(dst + 24576, &tmk, bar(B_QK_FULL + s), 64, hk, t0, bq);
         armed_qk[s] = c;
-        if (c >= 1) ok = tc::mbar_wait(bar(B_V_EMPTY), (c - 1) & 1, abort_flag, kBudget);
+        const uint8_t* src = pw_head + (long)c * kPwBytes;
+        const uint32_t slot = sb + OFF_PW + s * PW_SLOT;
+        if (c >= 2) ok = tc::mbar_wait(bar(B_W_EMPTY + s), ((c >> 1) - 1) & 1, abort_flag, kBudget);
         if (!ok) break;
-        tc::mbar_arrive_expect_tx(bar(B_V_FULL), 16384);
-        tc::tma_load_4d(sb + OFF_V, &tmv, bar(B_V_FULL), 0, h, t0, bq);
-        tc::tma_load_4d(sb + OFF_V + 8192, &tmv, bar(B_V_FULL), 64, h, t0, bq);
-        armed_v = c;
+        tc::mbar_arrive_expect_tx(bar(B_W_FULL + s), 32768);
+        tc::bulk_load(slot + 16384, src + 16384, 32768, bar(B_W_FULL + s));
+        armed_w[s] = c;
+        if (c >= 2) ok = tc::mbar_wait(bar(B_P_EMPTY + s), ((c >> 1) - 1) & 1, abort_flag, kBudget);
+        if (!ok) break;
+        tc::mbar_arrive_expect_tx(bar(B_P_FULL + s), 16384);
+        tc::bulk_load(slot, src, 16384, bar(B_P_FULL + s));
+        armed_p[s] = c;
       }
-      if (!ok) {   // let every load already issued land before the CTA can leave
-        volatile int never = 0;
-        for (int s = 0; s < 2; ++s)
-          if (armed_qk[s] >= 0)
-            tc::mbar_wait(bar(B_QK_FULL + s), (armed_qk[s] >> 1) & 1, &never, kBudget / 4);
-        if (armed_v >= 0) tc::mbar_wait(bar(B_V_FULL), armed_v & 1, &never, kBudget / 4);
+      // every load issued lands before the CTA can leave (at once unless a consumer gave up)
+      volatile int never = 0;
+      for (int s = 0; s < 2; ++s) {
+        if (armed_qk[s] >= 0)
+          tc::mbar_wait(bar(B_QK_FULL + s), (armed_qk[s] >> 1) & 1, &never, kBudget / 4);
+        if (armed_w[s] >= 0)
+          tc::mbar_wait(bar(B_W_FULL + s), (armed_w[s] >> 1) & 1, &never, kBudget / 4);
+        if (armed_p[s] >= 0)
+          tc::mbar_wait(bar(B_P_FULL + s), (armed_p[s] >> 1) & 1, &never, kBudget / 4);
       }
     }
   } else if (warp == 1) {
-    // -------------------- state-independent MMAs: S = [Q;K] K^T and P T_b --------------------
-    if (lane == 0) {
-      auto issue_S = [&](int c) -> bool {
-        const int s = c & 1;
-        if (!tc::mbar_wait(bar(B_QK_FULL + s), (c >> 1) & 1, abort_flag, kBudget)) return false;
-        if (c >= 1 && !tc::mbar_wait(bar(B_S_EMPTY), (c - 1) & 1, abort_flag, kBudget))
-          return false;
-        tc::tc_fence_after();
-        const uint32_t qk = sb + OFF_QK + s * QK_STAGE;
-#pragma unroll 1
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-          tc::mma_bf16(tmem + TM_S, tc::sdesc_sw128(qk + off, 16, 1024),
-                       tc::sdesc_sw128(qk + off + 8192, 16, 1024), ID_S, ks > 0);
-        }
-        tc::mma_commit(bar(B_S_FULL));
-        tc::mma_commit(bar(B_IN_EMPTY + s));
-        return true;
-      };
-      bool ok = issue_S(0);
-      for (int c = 0; c < nC && ok; ++c) {
-        ok = tc::mbar_wait(bar(B_PT_READY), c & 1, abort_flag, kBudget) &&
-             (c == 0 || tc::mbar_wait(bar(B_PT_EMPTY), (c - 1) & 1, abort_flag, kBudget));
-        if (!ok) break;
-        tc::tc_fence_after();
-#pragma unroll 1
-        for (int ks = 0; ks < 8; ++ks)   // P (64 x 64, K-major) x T_b (64 x 64, MN-major), tf32
-          tc::mma_tf32(tmem + TM_PT,
-                       tc::sdesc_sw128(sb + OFF_W + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024),
-                       tc::sdesc_sw128_b32(sb + OFF_WT + ks * 1024, 8192), ID_PT, ks > 0);
-        tc::mma_commit(bar(B_PT_FULL));
-        if (c + 1 < nC) ok = issue_S(c + 1);
-      }
-      tc::mma_commit(bar(B_DRAIN + 0));
-      volatile int never = 0;
-      tc::mbar_wait(bar(B_DRAIN + 0), 0, &never, kBudget / 4);
-    }
-  } else if (warp == 2) {
-    // -------------------------------- chain MMAs ---------------------------------------------
+    // -------------------------------- MMAs -----------------------------------------------------
     if (lane == 0) {
       bool ok = true;
       for (int c = 0; c < nC && ok; ++c) {
         const int s = c & 1;
         const uint32_t qk = sb + OFF_QK + s * QK_STAGE;
-        // X = [Q; K] M_hi + [Q; K] M_lo  (M = M_hi + M_lo, two bf16 terms)      (bf16)
+        const uint32_t pws = sb + OFF_PW + s * PW_SLOT;
+        // X = [Q; K] M  (M as one bf16 copy, or a hi + lo pair)                     (bf16)
         ok = tc::mbar_wait(bar(B_QK_FULL + s), (c >> 1) & 1, abort_flag, kBudget) &&
              tc::mbar_wait(bar(B_M_READY), c & 1, abort_flag, kBudget);
         if (!ok) break;
+        GDN_TRACE(c, 12);
         tc::tc_fence_after();
-#pragma unroll 1
-        for (int ks = 0; ks < (kSplitX ? 16 : 8); ++ks)
-          tc::mma_bf16(tmem + TM_X,
-                       tc::sdesc_sw128(qk + ((ks >> 2) & 1) * 16384 + (ks & 3) * 32, 16, 1024),
-                       tc::sdesc_sw128(sb + (ks < 8 ? OFF_MB : OFF_RD) + (ks & 7) * 2048, 16384, 1024),
-                       ID_X, ks > 0);
+        {
+          const uint64_t dq = tc::sdesc_sw128(qk, 16, 1024);
+          const uint64_t dm = tc::sdesc_sw128(sb + OFF_MB, 16384, 1024);
+          const uint64_t dml = tc::sdesc_sw128(sb + OFF_RD, 16384, 1024);
+#pragma unroll
+          for (int ks = 0; ks < (kSplitX ? 16 : 8); ++ks)
+            tc::mma_bf16(tmem + TM_X + 128 * s, tc::desc_adv(dq, ((ks >> 2) & 1) * 16384 + (ks & 3) * 32),
+                         tc::desc_adv(ks < 8 ? dm : dml, (ks & 7) * 2048), ID_X, ks > 0);
+        }
         tc::mma_commit(bar(B_X_FULL));
-        tc::mma_commit(bar(B_IN_EMPTY + s));
+        tc::mma_commit(bar(B_QK_EMPTY + s));
         GDN_TRACE(c, 20);
-        // Y = A2_hi R'_hi + A2_lo R'_hi + A2_hi R'_lo                           (bf16)
-        ok = tc::mbar_wait(bar(B_R_FULL), c & 1, abort_flag, kBudget) &&
-             tc::mbar_wait(bar(B_PRE_FULL), c & 1, abort_flag, kBudget);
+        ok = tc::mbar_wait(bar(B_R_FULL), c & 1, abort_flag, kBudget);
         if (!ok) break;
-        tc::tc_fence_after();
-#pragma unroll 1
-        for (int i = 0; i < 12; ++i) {
-          const int ks = i / 3, term = i - 3 * ks;
-          tc::mma_bf16(tmem + TM_Y,
-                       tc::sdesc_sw128(sb + OFF_A2 + (term == 1 ? 16384 : 0) + ks * 32, 16, 1024),
-                       tc::sdesc_sw128(sb + OFF_RD + (term == 2 ? 8192 : 0) + ks * 2048, 16384, 1024),
-                       ID_Y, i > 0);
-        }
-        tc::mma_commit(bar(B_Y_FULL));
-        tc::mma_commit(bar(B_A2_EMPTY));
-        GDN_TRACE(c, 21);
-        // M += K^T (ktil Delta)_hi + K^T (ktil Delta)_lo  (TMEM holds gamma_last M)  (bf16)
-        ok = tc::mbar_wait(bar(B_D_FULL), c & 1, abort_flag, kBudget) &&
-             tc::mbar_wait(bar(B_M_SCALED), c & 1, abort_flag, kBudget);
+        GDN_TRACE(c, 13);
+        // Y = PT R' (rows 0..63 used) and M += W R' (TMEM holds gamma_last M), each as
+        // hi.hi + lo.hi + hi.lo bf16 products                                        (bf16)
+        const uint64_t dpw = tc::sdesc_sw128(pws, 16, 1024);
+        const uint64_t drd = tc::sdesc_sw128(sb + OFF_RD, 16384, 1024);
+        auto issue_Y = [&]() -> bool {
+          if (c >= 1 && !tc::mbar_wait(bar(B_Y_EMPTY), (c - 1) & 1, abort_flag, kBudget)) return false;
+          if (!tc::mbar_wait(bar(B_P_FULL + s), (c >> 1) & 1, abort_flag, kBudget)) return false;
+          GDN_TRACE(c, 16);
+          tc::tc_fence_after();
+#pragma unroll
+          for (int i = 0; i < 12; ++i) {
+            const int ks = i / 3, term = i - 3 * ks;
+            tc::mma_bf16(tmem + TM_Y, tc::desc_adv(dpw, (term == 1 ? 8192 : 0) + ks * 32),
+                         tc::desc_adv(drd, (term == 2 ? 8192 : 0) + ks * 2048), ID_Y, i > 0);
+          }
+          tc::mma_commit(bar(B_Y_FULL));
+          tc::mma_commit(bar(B_P_EMPTY + s));
+          GDN_TRACE(c, 22);
+          return true;
+        };
+        auto issue_D3 = [&]() -> bool {
+          if (!tc::mbar_wait(bar(B_M_SCALED), c & 1, abort_flag, kBudget)) return false;
+          if (!tc::mbar_wait(bar(B_W_FULL + s), (c >> 1) & 1, abort_flag, kBudget)) return false;
+          GDN_TRACE(c, 15);
+          tc::tc_fence_after();
+#pragma unroll
+          for (int i = 0; i < 12; ++i) {
+            const int ks = i / 3, term = i - 3 * ks;
+            tc::mma_bf16(tmem + TM_M, tc::desc_adv(dpw, 16384 + (term == 1 ? 16384 : 0) + ks * 32),
+                         tc::desc_adv(drd, (term == 2 ? 8192 : 0) + ks * 2048), ID_Y, 1);
+          }
+          tc::mma_commit(bar(B_D3_FULL));
+          tc::mma_commit(bar(B_W_EMPTY + s));
+          GDN_TRACE(c, 21);
+          return true;
+        };
+        ok = kYFirst ? (issue_Y() && issue_D3()) : (issue_D3() && issue_Y());
         if (!ok) break;
-        tc::tc_fence_after();
-#pragma unroll 1
-        for (int ks = 0; ks < 8; ++ks)
-          tc::mma_bf16(tmem + TM_M, tc::sdesc_sw128(qk + 8192 + (ks & 3) * 2048, 16384, 1024),
-                       tc::sdesc_sw128(sb + OFF_RD + (ks >> 2) * 8192 + (ks & 3) * 2048, 16384, 1024),
-                       ID_U, 1);
-        tc::mma_commit(bar(B_D3_FULL));
-        tc::mma_commit(bar(B_IN_EMPTY + s));
-        GDN_TRACE(c, 22);
       }
-      tc::mma_commit(bar(B_DRAIN + 1));
+      tc::mma_commit(bar(B_DRAIN));
       volatile int never = 0;
-      tc::mbar_wait(bar(B_DRAIN + 1), 0, &never, kBudget / 4);
+      tc::mbar_wait(bar(B_DRAIN), 0, &never, kBudget / 4);
     }
-  } else if (warp == 3) {
-    // idle
-  } else if (warp < 8) {
-    // ------------------------------- pre warpgroup -------------------------------------------
-    const int ptid = threadIdx.x - 128;                 // = TMEM lane of this thread
-    const int q = warp & 3;
-    const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
-    // gates, computed by warp 4 one chunk ahead: lane l holds tokens 2l, 2l+1 of the next chunk
-    float pla0 = 0.f, pla1 = 0.f, pbe0 = 0.f, pbe1 = 0.f;
-    auto load_gates = [&](int c) {
-      const long ta = (long)c * C + 2 * lane, tb = ta + 1;
-      pla0 = pla1 = pbe0 = pbe1 = 0.f;
-      if (ta < T) { pla0 = log_alpha[((long)bq * T + ta) * Hv + h]; pbe0 = beta[((long)bq * T + ta) * Hv + h]; }
-      if (tb < T) { pla1 = log_alpha[((long)bq * T + tb) * Hv + h]; pbe1 = beta[((long)bq * T + tb) * Hv + h]; }
-    };
-    auto publish_gates = [&](int c) {
-      float* gG = gslot(c);
-      float* gGam = gG + 64;
-      float* gKt = gG + 128;
-      float* gBeta = gG + 192;
-      float* gE = gG + 256;
-      const float la0 = pla0, la1 = pla1, be0 = pbe0, be1 = pbe1;
-      float incl = la0 + la1;
-#pragma unroll
-      for (int d = 1; d < 32; d <<= 1) {
-        const float n = __shfl_up_sync(0xffffffffu, incl, d);
-        if (lane >= d) incl += n;
-      }
-      const float g1 = incl, g0 = incl - la1;
-      const float gl = __shfl_sync(0xffffffffu, incl, 31);
-      constexpr float kLog2e = 1.4426950408889634f;
-      gG[2 * lane] = g0 * kLog2e;    gG[2 * lane + 1] = g1 * kLog2e;
-      gGam[2 * lane] = tc::ex2(g0 * kLog2e);     gGam[2 * lane + 1] = tc::ex2(g1 * kLog2e);
-      gKt[2 * lane] = tc::ex2((gl - g0) * kLog2e); gKt[2 * lane + 1] = tc::ex2((gl - g1) * kLog2e);
-      gBeta[2 * lane] = be0;         gBeta[2 * lane + 1] = be1;
-      // block factors E[b][j] = exp(G_16b - G_j) for j < 16b (each <= 1: G never increases)
-#pragma unroll
-      for (int b = 1; b < 4; ++b) {
-        const float gb = __shfl_sync(0xffffffffu, g0, 8 * b) * kLog2e;   // G at token 16b
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int j = 2 * lane + e;
-          const float gj = (e ? g1 : g0) * kLog2e;
-          gE[64 * b + j] = (j < 16 * b) ? tc::ex2(gb - gj) : 0.f;
-        }
-      }
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(bar(B_GATE + c % 3));   // release: orders the stores above
-      if (c + 1 < nC) load_gates(c + 1);                      // after the arrive, never before it
-    };
-    // T_b of a chunk from the pre-pass: this thread's items id = ptid + 128 m (m < 5) of the 640
-    // float4 of the 10 packed blocks (block id / 64, row (id / 4) % 16, columns 4 (id % 4) ..),
-    // loaded one chunk ahead
-    float4 tbv[5];
-    auto load_tb = [&](int cc) {
-      const float4* src =
-          reinterpret_cast<const float4*>(Tb + (((long)bq * Hv + h) * nC + cc) * kTbFloats);
-#pragma unroll
-      for (int m = 0; m < 5; ++m) tbv[m] = src[ptid + 128 * m];
-    };
-    load_tb(0);
-    if (ptid < 32) {
-      load_gates(0);
-      publish_gates(0);
-    }
-    bool stop = false;
-    for (int c = 0; c < nC && !stop; ++c) {
-      if (ptid == 0) GDN_TRACE(c, 0);
-      const float* gG = gslot(c);
-      const float* gE = gG + 256;
-      tc::mbar_wait(bar(B_GATE + c % 3), (c / 3) & 1, abort_flag, kBudget);
-      tc::mbar_wait(bar(B_S_FULL), c & 1, abort_flag, kBudget);
-      if (ptid == 0) GDN_TRACE(c, 1);
-      tc::tc_fence_after();
-      // Rows 0..63 of S hold (q_t . k_j): P[t][j] = exp(G_t - G_j) (q_t . k_j) scale for j <= t,
-      // kept in the same TMEM row as fp32 until it goes out as the tf32 A operand of P T_b;
-      // exp(G_t - G_j) = 2^(G'_t - G'_j), G' = G log2 e, inside t's 16-token block directly and
-      // across blocks as 2^(G'_t - G'_16ti) E[ti][j] (both factors <= 1)
-      if (ptid < 64) {
-        const int t = ptid, ti = t >> 4;
-        const float gt = gG[t];
-        const float rowf = scale * tc::ex2(gt - gG[16 * ti]);
-        const float4* g4 = reinterpret_cast<const float4*>(gG);
-        const float4* e4p = reinterpret_cast<const float4*>(gE + 64 * ti);
-#pragma unroll 1
-        for (int p = 0; p < 2; ++p) {                // columns 32p .. 32p+31
-          float sv[32];
-          tc::tmem_ld32(tmem + lane_off + TM_S + 32 * p, sv);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int kb2 = 0; kb2 < 2; ++kb2) {
-            const int kb = 2 * p + kb2;
-            float* v = sv + 16 * kb2;
-            if (kb < ti) {
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const float4 e = e4p[4 * kb + i];
-                v[4 * i] *= rowf * e.x;     v[4 * i + 1] *= rowf * e.y;
-                v[4 * i + 2] *= rowf * e.z; v[4 * i + 3] *= rowf * e.w;
-              }
-            } else if (kb == ti) {
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const float4 g = g4[4 * kb + i];
-                const float gj[4] = {g.x, g.y, g.z, g.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const int j = 16 * kb + 4 * i + e;
-                  v[4 * i + e] = (j <= t) ? scale * tc::ex2(gt - gj[e]) * v[4 * i + e] : 0.f;
-                }
-              }
-            } else {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) v[e] = 0.f;
-            }
-          }
-          tc::tmem_st32(tmem + lane_off + TM_S + 32 * p, sv);
-        }
-        tc::tmem_wait_st();
-      }
-      if (ptid == 0) GDN_TRACE(c, 2);
-      float4 cur[5];
-#pragma unroll
-      for (int m = 0; m < 5; ++m) cur[m] = tbv[m];
-      if (c + 1 < nC) load_tb(c + 1);
-      if (c >= 1) {   // A2 (and the o tile staged in it) is free once Y and the o stores are done
-        tc::mbar_wait(bar(B_A2_EMPTY), (c - 1) & 1, abort_flag, kBudget);
-        tc::mbar_wait(bar(B_O_DONE), (c - 1) & 1, abort_flag, kBudget);
-      }
-      if (ptid == 0) GDN_TRACE(c, 4);
-      // T_b into A2's rows 64..127 (bf16 hi / lo) and into the B operand of P T_b (tf32), zero
-      // above the diagonal; the P T_b operands of the previous chunk are free (S of this chunk
-      // was issued after, and completed after, that MMA)
-      {
-        float sum = 0.f;
-#pragma unroll
-        for (int m = 0; m < 5; ++m) sum += (cur[m].x + cur[m].y) + (cur[m].z + cur[m].w);
-        const bool bad = nonfinite(sum);
-        const float4 inf4 = make_float4(kInf, kInf, kInf, kInf);
-#pragma unroll
-        for (int m = 0; m < 5; ++m) {
-          const int id = ptid + 128 * m, bb = id >> 6, r = (id >> 2) & 15, cs = id & 3;
-          const int i = bb >= 6 ? 3 : (bb >= 3 ? 2 : (bb >= 1 ? 1 : 0));
-          const int k = bb - i * (i + 1) / 2;
-          store_tb(sb, 16 * i + r, 16 * k + 4 * cs, bad ? inf4 : cur[m]);
-          if (i > k) store_tb(sb, 16 * k + r, 16 * i + 4 * cs, make_float4(0.f, 0.f, 0.f, 0.f));
-        }
-      }
-      if (ptid == 0) GDN_TRACE(c, 5);
-      // P rows (threads 0..63, warps 4 and 5): back from TMEM, rounded to tf32, into the K-major
-      // A operand of P T_b
-      if (ptid < 64) {
-        const int t = ptid;
-        float sum = 0.f;
-#pragma unroll 1
-        for (int p = 0; p < 2; ++p) {
-          float pv[32];
-          tc::tmem_ld32(tmem + lane_off + TM_S + 32 * p, pv);
-          tc::tmem_wait_ld();
-          const uint32_t prow = sb + OFF_W + p * 8192 + t * 128;
-#pragma unroll
-          for (int cc = 0; cc < 8; ++cc) {
-            const float* v = pv + 4 * cc;
-            sum += (v[0] + v[1]) + (v[2] + v[3]);
-            st_tf32x4(prow + ((cc ^ (t & 7)) << 4), v[0], v[1], v[2], v[3]);
-          }
-        }
-        if (nonfinite(sum)) {
-#pragma unroll 1
-          for (int p = 0; p < 2; ++p)
-#pragma unroll
-            for (int cc = 0; cc < 8; ++cc)
-              st_tf32x4(sb + OFF_W + p * 8192 + t * 128 + ((cc ^ (t & 7)) << 4), kInf, kInf, kInf, kInf);
-        }
-      }
-      tc::tc_fence_before();
-      tc::fence_proxy_async_smem();
-      tc::named_bar(1, 128);
-      if (ptid == 0) {
-        tc::mbar_arrive(bar(B_S_EMPTY));
-        tc::mbar_arrive(bar(B_PT_READY));
-        GDN_TRACE(c, 6);
-      }
-      if (ptid < 32 && c + 1 < nC) publish_gates(c + 1);
-      // A2 rows 0..63 = P T_b are written by the chain's O warps once the MMA is done
-      stop = vote_abort(1, 128, abort_flag);
-      if (ptid == 0) {
-        tc::mbar_arrive(bar(B_PRE_FULL));
-        GDN_TRACE(c, 8);
-      }
-    }
-  } else {
+  } else if (warp >= 4) {
     // ------------------------------- chain warpgroups ----------------------------------------
-    const int hh = (warp - 8) >> 2, q = warp & 3, r = 32 * q + lane;
+    // warps 4-7: value columns 0..63, warps 8-11: 64..127.  Lanes 0..63 (q < 2) make o of token
+    // t = r, lanes 64..127 make R' of token t = r - 64; all take M's row r.
+    const int hh = (warp - 4) >> 2, q = warp & 3, r = 32 * q + lane, t = r & 63;
     const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
     const uint32_t tcol = 64 * hh;                       // this half's TMEM / value columns
     const uint32_t mb = sb + OFF_MB + hh * 16384, rd = sb + OFF_RD + hh * 16384;
-    const uint32_t vb = sb + OFF_V + hh * 8192;
-    const uint32_t id_wg = 2 + 3 * hh, id_lo = 3 + 3 * hh, id_hi = 4 + 3 * hh;
-    const long head = (long)bq * Hv + h;
+    const uint32_t id_wg = 1 + 3 * hh, id_lo = 2 + 3 * hh, id_hi = 3 + 3 * hh;
     const bool leader = (q == 0 && lane == 0);
     [[maybe_unused]] const int ev = 10 * hh;
+    auto gam_at = [&](int c, int i) -> float {
+      return reinterpret_cast<const float*>(pw_head + (long)c * kPwBytes + kPwTiles)[i];
+    };
     // 32 columns (32p ..) of M row r (this half) for the X MMA: one round-to-nearest bf16 copy in Mb,
     // or (kSplitX) a hi + lo pair, hi into Mb and lo into the R' buffer
     auto store_m32 = [&](const float (&m)[32], int p) {
@@ -948,37 +872,27 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         if constexpr (kSplitX) {
           st_split8(mb + sw, rd + sw, m + 8 * j);
         } else {
-          const float* v = m + 8 * j;
-          tc::st_shared_v4(mb + sw, tc::pack_bf16(v[0], v[1]), tc::pack_bf16(v[2], v[3]),
-                           tc::pack_bf16(v[4], v[5]), tc::pack_bf16(v[6], v[7]));
+          const float* w = m + 8 * j;
+          tc::st_shared_v4(mb + sw, tc::pack_bf16(w[0], w[1]), tc::pack_bf16(w[2], w[3]),
+                           tc::pack_bf16(w[4], w[5]), tc::pack_bf16(w[6], w[7]));
         }
       }
     };
-    // A2 rows 0..63 = P T_b of chunk cn (O warps, q < 2): row r = TMEM lane r, this half takes
-    // columns 32 hh .. 32 hh + 31 of the 64
-    auto a2_top = [&](int cn) {
-      tc::mbar_wait(bar(B_PT_FULL), cn & 1, abort_flag, kBudget);
-      if (cn >= 1) tc::mbar_wait(bar(B_O_DONE), (cn - 1) & 1, abort_flag, kBudget);
-      if (leader && hh == 0) GDN_TRACE(cn, 16);
-      tc::tc_fence_after();
-      float pv[32];
-      tc::tmem_ld32(tmem + lane_off + TM_PT + 32 * hh, pv);
-      tc::tmem_wait_ld();
-      const uint32_t a2_row = sb + OFF_A2 + r * 128;
+    // row t of V for this half's columns (R' lanes), loaded one chunk ahead into registers
+    uint4 vr[8];
+    auto load_v = [&](int c) {
+      const long tok = (long)c * C + t;
+      if (tok < T) {
+        const uint4* src = reinterpret_cast<const uint4*>(v + (((long)bq * T + tok) * Hv + h) * 128 + tcol);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint32_t sw = ((4 * hh + j) ^ (r & 7)) << 4;
-        st_split8(a2_row + sw, a2_row + 16384 + sw, pv + 8 * j);
-      }
-      tc::fence_proxy_async_smem();
-      tc::tc_fence_before();
-      tc::named_bar(id_lo, 64);
-      if (leader) {
-        if (hh == 0) GDN_TRACE(cn, 17);
-        tc::mbar_arrive(bar(B_PT_EMPTY));
-        tc::mbar_arrive(bar(B_PRE_FULL));
+        for (int i = 0; i < 8; ++i) vr[i] = src[i];
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) vr[i] = make_uint4(0u, 0u, 0u, 0u);
       }
     };
+    if (q >= 2) load_v(0);
+    float g_t = gam_at(0, t);
     bool stop = false;
     {
       float m[64];
@@ -986,8 +900,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         const float4* src = reinterpret_cast<const float4*>(S0 + (head * 128 + r) * 128 + tcol);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float4 v = src[i];
-          m[4 * i] = v.x; m[4 * i + 1] = v.y; m[4 * i + 2] = v.z; m[4 * i + 3] = v.w;
+          const float4 w = src[i];
+          m[4 * i] = w.x; m[4 * i + 1] = w.y; m[4 * i + 2] = w.z; m[4 * i + 3] = w.w;
         }
       } else {
 #pragma unroll
@@ -995,8 +909,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       }
       store_m32(*reinterpret_cast<const float(*)[32]>(&m[0]), 0);
       store_m32(*reinterpret_cast<const float(*)[32]>(&m[32]), 1);
-      tc::mbar_wait(bar(B_GATE + 0), 0, abort_flag, kBudget);
-      const float gl = gslot(0)[64 + 63];
+      const float gl = gam_at(0, 63);
 #pragma unroll
       for (int i = 0; i < 64; ++i) m[i] *= gl;
       tmem_st64(tmem + lane_off + TM_M + tcol, m);
@@ -1008,97 +921,105 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         tc::mbar_arrive(bar(B_M_READY));
         tc::mbar_arrive(bar(B_M_SCALED));
       }
-      if (!stop && q < 2) a2_top(0);
     }
 
     for (int c = 0; c < nC && !stop; ++c) {
-      const float* gGam = gslot(c) + 64;
-      const float* gKt = gGam + 64;
+      const int s = c & 1;
+      const uint32_t tx = tmem + lane_off + TM_X + 128 * s + tcol;
+      // the next chunk's gates: gamma_last for the state below, gamma_t for the next chunk
+      float g_nt = 0.f, g_nl = 0.f;
+      if (c + 1 < nC) {
+        g_nt = gam_at(c + 1, t);
+        g_nl = gam_at(c + 1, 63);
+      }
       if (q >= 2) {
-        // R' = V - gamma (K M) for token t (tf32), then ktil Delta as bf16 hi + lo
-        const int t = r - 64;
+        // R' = V - gamma (K M) for token t, as a bf16 hi + lo pair (the B operand of Y and of
+        // the state update)
         tc::mbar_wait(bar(B_X_FULL), c & 1, abort_flag, kBudget);
-        tc::mbar_wait(bar(B_GATE + c % 3), (c / 3) & 1, abort_flag, kBudget);
-        tc::mbar_wait(bar(B_V_FULL), c & 1, abort_flag, kBudget);
         if (q == 2 && lane == 0) GDN_TRACE(c, 30 + ev);
         tc::tc_fence_after();
-        const float g = gGam[t];
 #pragma unroll 1
         for (int p = 0; p < 2; ++p) {            // value columns 32p .. 32p+31 of this half
           float x[32];
-          tc::tmem_ld32(tmem + lane_off + TM_X + tcol + 32 * p, x);
-          uint4 u[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) u[j] = tc::ld_shared_v4(vb + tc::sw128(t, 4 * p + j));
+          tc::tmem_ld32(tx + 32 * p, x);
           tc::tmem_wait_ld();
-          if (p == 0 && hh == 0 && q == 2 && lane == 0) GDN_TRACE(c, 55);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const float* xx = x + 8 * j;
-            const uint32_t w4[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
+            const uint4 u = p ? vr[4 + j] : vr[j];   // (no dynamic register indexing)
+            const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
             float rv[8];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              rv[2 * e] = fmaf(-g, xx[2 * e], tc::bf16lo(w4[e]));
-              rv[2 * e + 1] = fmaf(-g, xx[2 * e + 1], tc::bf16hi(w4[e]));
+              rv[2 * e] = fmaf(-g_t, xx[2 * e], tc::bf16lo(w4[e]));
+              rv[2 * e + 1] = fmaf(-g_t, xx[2 * e + 1], tc::bf16hi(w4[e]));
             }
-            // MN-major bf16 B operand of Y: row t (K), 16-byte chunk 4p + j of this half's columns
+            // MN-major bf16 B operand: row t (K), 16-byte chunk 4p + j of this half's columns
             const uint32_t sw = tc::sw128(t, 4 * p + j);
             st_split8(rd + sw, rd + 8192 + sw, rv);
           }
-          if (hh == 0 && q == 2 && lane == 0) GDN_TRACE(c, 56 + p);
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
-        if (hh == 0 && q == 2 && lane == 0) GDN_TRACE(c, 58);
         tc::named_bar(id_hi, 64);
         if (q == 2 && lane == 0) {
           GDN_TRACE(c, 31 + ev);
           tc::mbar_arrive(bar(B_R_FULL));
-          tc::mbar_arrive(bar(B_V_EMPTY));
         }
-        tc::mbar_wait(bar(B_Y_FULL), c & 1, abort_flag, kBudget);
-        if (q == 2 && lane == 0) GDN_TRACE(c, 32 + ev);
-        tc::tc_fence_after();
-        const float kt = gKt[t];
-#pragma unroll 1
-        for (int p = 0; p < 2; ++p) {
-          float y[32];
-          tc::tmem_ld32(tmem + lane_off + TM_Y + tcol + 32 * p, y);
-          tc::tmem_wait_ld();
-          if (p == 0 && hh == 0 && q == 2 && lane == 0) GDN_TRACE(c, 59);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) y[i] *= kt;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t sw = tc::sw128(t, 4 * p + j);
-            st_split8(rd + sw, rd + 8192 + sw, y + 8 * j);
-          }
-        }
-        if (hh == 0 && q == 2 && lane == 0) GDN_TRACE(c, 60);
+        if (c + 1 < nC) load_v(c + 1);
+      }
+      // M <- gamma_last M + W R' is now in TMEM (row r of this half).  Its bf16 copy goes out
+      // first (the next X needs it); then TMEM is scaled by the next chunk's gamma_last for the
+      // next update, which waits for that separately.
+      tc::mbar_wait(bar(B_D3_FULL), c & 1, abort_flag, kBudget);
+      if (leader) GDN_TRACE(c, 37 + ev);
+      tc::tc_fence_after();
+      if (c + 1 < nC) {
+        float m[64];
+        tmem_ld64(tmem + lane_off + TM_M + tcol, m);
+        tc::tmem_wait_ld();
+        store_m32(*reinterpret_cast<const float(*)[32]>(&m[0]), 0);
+        store_m32(*reinterpret_cast<const float(*)[32]>(&m[32]), 1);
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
-        if (hh == 0 && q == 2 && lane == 0) GDN_TRACE(c, 61);
-        tc::named_bar(id_hi, 64);
-        if (q == 2 && lane == 0) {
-          GDN_TRACE(c, 33 + ev);
-          tc::mbar_arrive(bar(B_D_FULL));
+        tc::named_bar(id_wg, 128);
+        if (leader) {
+          GDN_TRACE(c, 38 + ev);
+          tc::mbar_arrive(bar(B_M_READY));
         }
-      } else {
-        // o_t = gamma_t scale (Q M)_t + (P Delta)_t, staged in shared memory for a TMA store
-        const int t = r;
-        tc::mbar_wait(bar(B_X_FULL), c & 1, abort_flag, kBudget);
-        tc::mbar_wait(bar(B_GATE + c % 3), (c / 3) & 1, abort_flag, kBudget);
+#pragma unroll
+        for (int i = 0; i < 64; ++i) m[i] *= g_nl;
+        tmem_st64(tmem + lane_off + TM_M + tcol, m);
+        tc::tmem_wait_st();
+      } else if (S_T && !*abort_flag) {
+        float m[64];
+        tmem_ld64(tmem + lane_off + TM_M + tcol, m);
+        tc::tmem_wait_ld();
+        float4* dst = reinterpret_cast<float4*>(S_T + (head * 128 + r) * 128 + tcol);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          dst[i] = make_float4(m[4 * i], m[4 * i + 1], m[4 * i + 2], m[4 * i + 3]);
+      }
+      tc::tc_fence_before();
+      stop = vote_abort(id_wg, 128, abort_flag);
+      if (leader) {
+        if (hh == 0) GDN_TRACE(c, 52);
+        tc::mbar_arrive(bar(B_M_SCALED));
+      }
+      if (q < 2 && !stop) {
+        // o_t = gamma_t scale (Q M)_t + (PT R')_t, staged in the chunk's operand slot (the PT
+        // tiles, which Y has finished reading; fp32 also takes W's, after the update) for a TMA
+        // store
         tc::mbar_wait(bar(B_Y_FULL), c & 1, abort_flag, kBudget);
         if (leader) GDN_TRACE(c, 34 + ev);
         tc::tc_fence_after();
-        const float g = gGam[t] * scale;
+        const float g = g_t * scale;
         // bf16: one [64 t][64 dv] tile per half; fp32: two [64 t][32 dv] tiles per half
-        const uint32_t stage = sb + OFF_A2 + hh * (kF32 ? 16384 : 8192);
+        const uint32_t stage = sb + OFF_PW + s * PW_SLOT + hh * (kF32 ? 16384 : 8192);
 #pragma unroll 1
         for (int p = 0; p < 4; ++p) {            // value columns 16p .. 16p+15 of this half
           float x[16], y[16];
-          tmem_ld16(tmem + lane_off + TM_X + tcol + 16 * p, x);
+          tmem_ld16(tx + 16 * p, x);
           tmem_ld16(tmem + lane_off + TM_Y + tcol + 16 * p, y);
           tc::tmem_wait_ld();
 #pragma unroll
@@ -1122,6 +1043,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         tc::tc_fence_before();
         tc::named_bar(id_lo, 64);
         if (leader) {
+          tc::mbar_arrive(bar(B_Y_EMPTY));
           GDN_TRACE(c, 35 + ev);
           if constexpr (kF32) {
             tc::tma_store_4d(&tmo, stage, 64 * hh, h, c * C, bq);
@@ -1131,52 +1053,12 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
           }
           tc::bulk_commit();
           tc::bulk_wait_read_all();
-          tc::mbar_arrive(bar(B_O_DONE));
+          tc::mbar_arrive(bar(B_P_EMPTY + s));
+          if constexpr (kF32) tc::mbar_arrive(bar(B_W_EMPTY + s));
           GDN_TRACE(c, 36 + ev);
         }
       }
-      // M <- gamma_last M + K^T (ktil Delta) is now in TMEM (row r of this half).  Its bf16 pair
-      // goes out first (the next X needs it); then TMEM is scaled by the next chunk's
-      // gamma_last for the next update, which waits for that separately.
-      tc::mbar_wait(bar(B_D3_FULL), c & 1, abort_flag, kBudget);
-      if (leader) GDN_TRACE(c, 37 + ev);
-      tc::tc_fence_after();
-      if (c + 1 < nC) {
-        float m[64];
-        tmem_ld64(tmem + lane_off + TM_M + tcol, m);
-        tc::mbar_wait(bar(B_GATE + (c + 1) % 3), ((c + 1) / 3) & 1, abort_flag, kBudget);
-        const float gl = gslot(c + 1)[64 + 63];
-        tc::tmem_wait_ld();
-        if (leader && hh == 0) GDN_TRACE(c, 50);
-        store_m32(*reinterpret_cast<const float(*)[32]>(&m[0]), 0);
-        store_m32(*reinterpret_cast<const float(*)[32]>(&m[32]), 1);
-        tc::fence_proxy_async_smem();
-        tc::named_bar(id_wg, 128);
-        if (leader) {
-          GDN_TRACE(c, 38 + ev);
-          tc::mbar_arrive(bar(B_M_READY));
-        }
-#pragma unroll
-        for (int i = 0; i < 64; ++i) m[i] *= gl;
-        tmem_st64(tmem + lane_off + TM_M + tcol, m);
-        tc::tmem_wait_st();
-        if (leader && hh == 0) GDN_TRACE(c, 51);
-      } else if (S_T && !*abort_flag) {
-        float m[64];
-        tmem_ld64(tmem + lane_off + TM_M + tcol, m);
-        tc::tmem_wait_ld();
-        float4* dst = reinterpret_cast<float4*>(S_T + (head * 128 + r) * 128 + tcol);
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          dst[i] = make_float4(m[4 * i], m[4 * i + 1], m[4 * i + 2], m[4 * i + 3]);
-      }
-      tc::tc_fence_before();
-      stop = vote_abort(id_wg, 128, abort_flag);
-      if (leader) {
-        if (hh == 0) GDN_TRACE(c, 52);
-        tc::mbar_arrive(bar(B_M_SCALED));
-      }
-      if (!stop && q < 2 && c + 1 < nC) a2_top(c + 1);
+      g_t = g_nt;
     }
     if (leader) tc::bulk_wait_all();               // every o tile has reached global memory
   }
@@ -1223,36 +1105,35 @@ inline bool make_tile_map(CUtensorMap* m, const void* base, int H, int T, int B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Bytes of the T_b hand-over buffer between the pre-pass and the recurrence.
+// Bytes of the operand hand-over buffer between the pre-pass and the recurrence.
 inline size_t scratch_bytes(int B, int T, int Hv) {
   const size_t nC = (size_t)(T + C - 1) / C;
-  return (size_t)B * Hv * nC * kTbFloats * sizeof(float);
+  return (size_t)B * Hv * nC * kPwBytes;
 }
 
 template <typename Tout>
 gdn_status launch(const void* q, const void* k, const void* v, const float* la, const float* be,
                   const float* S0, Tout* o, float* S_T, int B, int T, int Hk, int Hv, float scale,
-                  float* tb, cudaStream_t st) {
-  CUtensorMap mq, mk, mv, mo;
+                  uint8_t* pw, cudaStream_t st) {
+  CUtensorMap mq, mk, mo;
   if (!make_tile_map(&mq, q, Hk, T, B, false) || !make_tile_map(&mk, k, Hk, T, B, false) ||
-      !make_tile_map(&mv, v, Hv, T, B, false) ||
       !make_tile_map(&mo, o, Hv, T, B, sizeof(Tout) == 4))
     return GDN_ERR_CUDA;
   auto kern = chunk_fwd_tc_kernel<Tout>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC) !=
       cudaSuccess)
     return GDN_ERR_CUDA;
-  if (cudaFuncSetAttribute(tb_prepass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(pw_prepass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            PP_SMEM) != cudaSuccess)
     return GDN_ERR_CUDA;
   const long grid = (long)B * Hv;
   const int nC = (T + C - 1) / C;
   if (grid > 0x7fffffffL || Hv > 65535 || B > 65535) return GDN_ERR_UNSUPPORTED;
-  tb_prepass_kernel<<<dim3(nC, Hv, B), PP_THREADS, PP_SMEM, st>>>(
-      static_cast<const __nv_bfloat16*>(k), la, be, tb, T, Hk, Hv);
+  pw_prepass_kernel<<<dim3(nC, Hv, B), PP_THREADS, PP_SMEM, st>>>(mq, mk, la, be, pw, T, Hk, Hv,
+                                                                   scale);
   if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
-  kern<<<(unsigned)grid, kThreads, SMEM_ALLOC, st>>>(mq, mk, mv, mo, la, be, tb, S0, S_T, T, Hk,
-                                                     Hv, scale);
+  kern<<<(unsigned)grid, kThreads, SMEM_ALLOC, st>>>(
+      mq, mk, mo, static_cast<const __nv_bfloat16*>(v), pw, S0, S_T, T, Hk, Hv, scale);
   return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -1268,7 +1149,7 @@ inline bool tc_chunk_supported(int dk, int dv, int chunk, bool bf16) {
   return bf16 && dk == 128 && dv == 128 && chunk == tcf::C;
 }
 
-// Scratch bytes of the tensor-core forward (the T_b hand-over buffer), 256-byte aligned.
+// Scratch bytes of the tensor-core forward (the pre-pass's operand hand-over buffer).
 inline size_t tc_chunk_scratch_bytes(int B, int T, int Hv) { return tcf::scratch_bytes(B, T, Hv); }
 
 inline gdn_status tc_chunk_launch(const void* q, const void* k, const void* v, const float* la,
@@ -1276,7 +1157,7 @@ inline gdn_status tc_chunk_launch(const void* q, const void* k, const void* v, c
                                   int T, int Hk, int Hv, float scale, void* scratch,
                                   cudaStream_t st) {
   return tcf::launch<__nv_bfloat16>(q, k, v, la, be, S0, static_cast<__nv_bfloat16*>(o), S_T, B,
-                                    T, Hk, Hv, scale, static_cast<float*>(scratch), st);
+                                    T, Hk, Hv, scale, static_cast<uint8_t*>(scratch), st);
 }
 
 inline gdn_status tc_chunk_launch_f32out(const void* q, const void* k, const void* v,
@@ -1284,7 +1165,7 @@ inline gdn_status tc_chunk_launch_f32out(const void* q, const void* k, const voi
                                          float* o, float* S_T, int B, int T, int Hk, int Hv,
                                          float scale, void* scratch, cudaStream_t st) {
   return tcf::launch<float>(q, k, v, la, be, S0, o, S_T, B, T, Hk, Hv, scale,
-                            static_cast<float*>(scratch), st);
+                            static_cast<uint8_t*>(scratch), st);
 }
 
 }  // namespace gdn

@@ -48,20 +48,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Same, but the thread may be suspended in hardware until the phase completes or `hint_ns`
-// passes, so waiting warps take no issue slots from the warps doing the work.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
-                                                    uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
@@ -72,14 +58,15 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 // Bounded wait: returns false if `abort` was raised by another thread or once `budget_cycles`
-// SM clock cycles passed (it then raises `abort` itself).  Never spins forever: each poll
-// suspends the thread for up to 50 us unless the phase completes first.
+// SM clock cycles passed (it then raises `abort` itself).  Never spins forever.  Each poll is a
+// try_wait with the hardware's own short suspend limit: a long suspend hint wakes the thread
+// hundreds of cycles after the phase completes, which the recurrence's hand-offs cannot afford.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           uint64_t budget_cycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (;;) {
-    if (mbar_try_wait_sleep(bar, parity, 50000u)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
     if ((uint64_t)(clock64() - t0) > budget_cycles) {
       *abort = 1;
@@ -111,6 +98,24 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, uint
       " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
       : "memory");
+}
+
+// Untiled bulk copy of `bytes` contiguous bytes, global -> shared, completing on an mbarrier
+// (both addresses 16-byte aligned, `bytes` a multiple of 16).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// Untiled bulk copy shared -> global (bulk-group completion, same alignment rules).
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
+                   reinterpret_cast<uint64_t>(dst)),
+               "r"(src), "r"(bytes)
+               : "memory");
 }
 
 // Tiled 4-D store of a shared-memory box to global memory (bulk-group completion); rows past
@@ -239,6 +244,11 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
   d |= (uint64_t)layout << 61;
   return d;
 }
+// The same descriptor moved `bytes` further (a multiple of 16; the address field stays below
+// 256 KB, so the add never carries into the other fields).  Issue loops unrolled over such
+// constant steps from one base keep the tensor pipe fed: a loop that rebuilds each descriptor
+// from scratch issues at about half the MMA rate.
+__device__ __forceinline__ uint64_t desc_adv(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
 // 128-byte swizzle, 16-byte chunks (bf16 operands, K-major tf32 operands)
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return sdesc(saddr, lbo, sbo, 2);

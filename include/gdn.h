@@ -96,8 +96,10 @@ GDN_API gdn_status gdn_check_error(gdn_stream_t stream);
  *   T    need not be a multiple of `chunk`; the ragged last block is masked.
  *   scale multiplies q (o = scale * S q).
  * Exact in real arithmetic for any chunk size; the chunk size only reorders rounding.
- * The tensor-core family (bf16, d_k = d_v = 128, chunk 64) first computes every chunk's T_b in a
- * pre-pass and hands it to the recurrence through a device buffer of B * Hv * ceil(T/64) * 10 KB;
+ * The tensor-core family (bf16, d_k = d_v = 128, chunk 64) first computes every chunk's
+ * state-independent operands (P T_b and (diag(ktil) K)^T T_b as bf16 hi/lo tiles, and gamma) in a
+ * pre-pass and hands them to the recurrence through a device buffer of
+ * B * Hv * ceil(T/64) * 49408 bytes;
  * that buffer is taken from a memory pool of the library (one per device, stream-ordered, kept
  * between calls) and given back at the end of the call on `stream`.
  */
@@ -189,7 +191,7 @@ GDN_API size_t gdn_layer_workspace_bytes(int B, int T, int Hk, int Hv, int dk, i
  *   Arguments, layouts, results and errors are those of gdn_layer_fwd without `workspace` and
  *   `workspace_bytes`.  The scratch is GDN_LAYER_STATIC_SCRATCH_BYTES of device memory built into
  *   the library (one per device); sizes for which gdn_layer_workspace_bytes(...) exceeds it return
- *   GDN_ERR_UNSUPPORTED before any work (about 630 tokens at Hk=16, Hv=48, d=128, bf16).
+ *   GDN_ERR_UNSUPPORTED before any work (about 380 tokens at Hk=16, Hv=48, d=128, bf16).
  *   The first call on a device looks the scratch's device address up (cudaGetSymbolAddress on
  *   the current device, which must be the device of every pointer and of `stream`) and keeps it;
  *   that lookup allocates nothing, but make the first call on each device before any stream
