@@ -84,21 +84,24 @@ constexpr uint32_t ID_Y = tc::idesc_bf16(128, 128, false, true);
 // slot (block, chunk, event) of a caller-provided buffer receives clock64().
 #ifdef GDN_TC_TRACE
 __device__ unsigned long long* g_tc_trace = nullptr;
+// the buffer pointer is read once per kernel (GDN_TRACE_INIT), so a timestamp costs one store
+#define GDN_TRACE_INIT unsigned long long* const tr_buf_ = g_tc_trace
 #define GDN_TRACE(c, ev)                                                              \
   do {                                                                                \
-    if (g_tc_trace) g_tc_trace[((size_t)blockIdx.x * nC + (c)) * 64 + (ev)] = clock64(); \
+    if (tr_buf_) tr_buf_[((size_t)blockIdx.x * nC + (c)) * 64 + (ev)] = clock64();    \
   } while (0)
 // same with the global nanosecond timer (comparable across SMs)
 #define GDN_TRACE_G(c, ev)                                                            \
   do {                                                                                \
-    if (g_tc_trace) g_tc_trace[((size_t)blockIdx.x * nC + (c)) * 64 + (ev)] = tc::globaltimer_ns(); \
+    if (tr_buf_) tr_buf_[((size_t)blockIdx.x * nC + (c)) * 64 + (ev)] = tc::globaltimer_ns(); \
   } while (0)
 #define GDN_TRACE_PP(ev)                                                               \
   do {                                                                                 \
-    if (g_tc_trace && threadIdx.x == 0)                                                \
-      g_tc_trace[(((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * 64 + (ev)] = clock64(); \
+    if (tr_buf_ && threadIdx.x == 0)                                                   \
+      tr_buf_[(((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * 64 + (ev)] = clock64(); \
   } while (0)
 #else
+#define GDN_TRACE_INIT do {} while (0)
 #define GDN_TRACE_PP(ev) do {} while (0)
 #define GDN_TRACE(c, ev) do {} while (0)
 #define GDN_TRACE_G(c, ev) do {} while (0)
@@ -419,6 +422,7 @@ __global__ void __launch_bounds__(PP_THREADS, 3)
 pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const float* __restrict__ log_alpha, const float* __restrict__ beta,
                   uint8_t* __restrict__ pw, int T, int Hk, int Hv, float scale) {
+  GDN_TRACE_INIT;
   extern __shared__ __align__(1024) uint8_t pp_raw[];
   uint8_t* smem = pp_raw + ((1024u - (tc::smem_u32(pp_raw) & 1023u)) & 1023u);
   const uint32_t sb = tc::smem_u32(smem);
@@ -431,13 +435,14 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
   float* gKt = gG + 128;
   volatile int* flag = reinterpret_cast<volatile int*>(gG + 192);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gG + 193);
-  const uint32_t tma_bar = sb + PP_BAR, mma_bar = sb + PP_BAR + 8;
+  const uint32_t tma_bar = sb + PP_BAR, mma_bar = sb + PP_BAR + 8, pt_bar = sb + PP_BAR + 24;
   const uint32_t qk = sb + PP_QK, tb = sb + PP_TB;
   uint8_t* rec = pw + (((long)bq * Hv + h) * nC + c) * (long)kPwBytes;
 
   if (tid == 0) {
     tc::mbar_init(tma_bar, 1);
     tc::mbar_init(mma_bar, 1);
+    tc::mbar_init(pt_bar, 1);
     *flag = 0;
     *abort_flag = 0;
     tc::fence_barrier_init();
@@ -600,7 +605,8 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
   tc::tc_fence_before();
   __syncthreads();
 
-  // PT = P T_b (columns 64..127) and W = K^T (ktil T_b) (columns 0..63; S is consumed)
+  // W = K^T (ktil T_b) (columns 0..63; S is consumed), then PT = P T_b (columns 64..127), each
+  // with its own completion so W's rows go out while PT is still being multiplied
   GDN_TRACE_PP(6);
   if (tid == 0) {
     tc::tc_fence_after();
@@ -608,26 +614,36 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     const uint64_t dt = tc::sdesc_sw128(tb, 8192, 1024);
     const uint64_t dk = tc::sdesc_sw128(qk + 8192, 16384, 1024);
 #pragma unroll
-    for (int i = 0; i < 12; ++i) {
-      const int ks = i / 3, term = i - 3 * ks;
-      tc::mma_bf16(tmem + 64, tc::desc_adv(dp, (term == 1 ? 16384 : 0) + ks * 32),
-                   tc::desc_adv(dt, (term == 2 ? 8192 : 0) + ks * 2048), ID_PT, i > 0);
-    }
-#pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int ks = i >> 1, term = i & 1;
       tc::mma_bf16(tmem, tc::desc_adv(dk, ks * 2048), tc::desc_adv(dt, 16384 + term * 8192 + ks * 2048),
                    ID_W, i > 0);
     }
     tc::mma_commit(mma_bar);
+#pragma unroll
+    for (int i = 0; i < 12; ++i) {
+      const int ks = i / 3, term = i - 3 * ks;
+      tc::mma_bf16(tmem + 64, tc::desc_adv(dp, (term == 1 ? 16384 : 0) + ks * 32),
+                   tc::desc_adv(dt, (term == 2 ? 8192 : 0) + ks * 2048), ID_PT, i > 0);
+    }
+    tc::mma_commit(pt_bar);
   }
   tc::mbar_wait(mma_bar, 1, abort_flag, kBudget);
   GDN_TRACE_PP(7);
   tc::tc_fence_after();
   const bool poison = *flag != 0;
+  // Rows from TMEM are split and staged (swizzled, in the record's tile layout) in shared memory
+  // the pending MMAs no longer read, then leave by bulk copies: W's while PT is still being
+  // multiplied (W hi over the ktil T_b tiles, W lo rows 0..63 / 64..127 over the two K boxes),
+  // PT's once it is done (hi over P hi, lo over P lo).
+  auto stage_row = [&](uint32_t hi_base, uint32_t lo_base, int r, const float* w) {
+#pragma unroll
+    for (int j8 = 0; j8 < 8; ++j8) {
+      const uint32_t o = (uint32_t)(r * 128 + ((j8 ^ (r & 7)) << 4));
+      st_split8(hi_base + o, lo_base + o, w + 8 * j8);
+    }
+  };
   {
-    // staging in the record's order: PT hi [64][128 B], PT lo, W hi [128][128 B], W lo (every
-    // operand read by the MMAs above is dead)
     float w[64];
     tc::tmem_ld32(tmem + lane_off, *reinterpret_cast<float(*)[32]>(&w[0]));
     tc::tmem_ld32(tmem + lane_off + 32, *reinterpret_cast<float(*)[32]>(&w[32]));
@@ -636,13 +652,19 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 #pragma unroll
       for (int j = 0; j < 64; ++j) w[j] = kInf;
     }
-    __syncthreads();                                  // every thread is past its MMA-operand reads
-#pragma unroll
-    for (int j8 = 0; j8 < 8; ++j8) {
-      const uint32_t o = sb + 16384 + (uint32_t)(tid * 128 + ((j8 ^ (tid & 7)) << 4));
-      st_split8(o, o + 16384, w + 8 * j8);
+    // W row r: hi at tb + 16384 + r * 128, lo at qk + 8192 (r < 64) or qk + 24576 (r >= 64)
+    stage_row(tb + 16384, qk + (tid < 64 ? 8192 : 24576 - 64 * 128), tid, w);
+    tc::fence_proxy_async_smem();
+    tc::named_bar(1, 128);
+    if (tid == 0) {
+      tc::bulk_store(rec + 16384, tb + 16384, 16384);
+      tc::bulk_store(rec + 32768, qk + 8192, 8192);
+      tc::bulk_store(rec + 40960, qk + 24576, 8192);
+      tc::bulk_commit();
     }
     if (tid < 64) {
+      tc::mbar_wait(pt_bar, 0, abort_flag, kBudget);
+      tc::tc_fence_after();
       tc::tmem_ld32(tmem + lane_off + 64, *reinterpret_cast<float(*)[32]>(&w[0]));
       tc::tmem_ld32(tmem + lane_off + 96, *reinterpret_cast<float(*)[32]>(&w[32]));
       tc::tmem_wait_ld();
@@ -650,25 +672,21 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 #pragma unroll
         for (int j = 0; j < 64; ++j) w[j] = kInf;
       }
-#pragma unroll
-      for (int j8 = 0; j8 < 8; ++j8) {
-        const uint32_t o = sb + (uint32_t)(tid * 128 + ((j8 ^ (tid & 7)) << 4));
-        st_split8(o, o + 8192, w + 8 * j8);
-      }
+      stage_row(qk, qk + 16384, tid, w);
+      tc::fence_proxy_async_smem();
+      tc::named_bar(2, 64);
+      if (tid == 0) {
+        tc::bulk_store(rec, qk, 8192);
+        tc::bulk_store(rec + 8192, qk + 16384, 8192);
+        tc::bulk_commit();
+        tc::bulk_wait_read_all();                     // every source read; the writes complete
+      }                                               // on their own
     }
   }
-  tc::fence_proxy_async_smem();
-  tc::tc_fence_before();
-  __syncthreads();
   GDN_TRACE_PP(8);
-  if (tid == 0) {
-    tc::bulk_store(rec, sb, kPwTiles);
-    tc::bulk_commit();
-    tc::bulk_wait_read_all();                         // the source may be released; the write
-                                                      // completes on its own
-    GDN_TRACE_PP(9);
-    if (*abort_flag) record_error(kErrTimeout);
-  }
+  GDN_TRACE_PP(9);
+  if (tid == 0 && *abort_flag) record_error(kErrTimeout);
+  tc::tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc::tc_fence_after();
@@ -692,6 +710,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   // The low half of a split M shares the R' buffer, so there Y (which reads R') runs before the
   // state update; otherwise the update, which the next chunk waits for, goes first.
   constexpr bool kYFirst = kSplitX;
+  GDN_TRACE_INIT;
   // Offsetting the __shared__ array itself (not a round trip through an integer) keeps every
   // access below a shared-memory access (ld/st.shared), not a generic one.
   extern __shared__ __align__(1024) uint8_t smem_raw[];
