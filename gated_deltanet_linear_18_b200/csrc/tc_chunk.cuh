@@ -25,15 +25,18 @@
 // The pre-pass hands each chunk to the recurrence as its MMA operands themselves (48 KB of
 // swizzled tiles plus gamma), so the recurrence's critical path holds only X, R', the state
 // update and the state's bf16 copy.  Recurrence CTA, 384 threads in specialised warps:
-//   warp 0        TMA producer (Q, K tiles and the chunk's operand tiles, double-buffered)
-//   warp 1        TMEM owner; issues every MMA (X, the state update, then Y)
+//   warp 0        TMA producer (the Q, K tile of the next chunk as soon as X has read the last;
+//                 the chunks' operand tiles double-buffered)
+//   warp 1        TMEM owner; issues every MMA: X of chunk c, Y of chunk c - 1 (from the other
+//                 of two R' buffers, while R' of chunk c is formed), the state update of c
 //   warps 4-7     value columns 0..63; warps 8-11 columns 64..127.  Lanes 0..63 of each group
 //                 make o, lanes 64..127 make R' (V comes straight into registers one chunk
 //                 ahead); all four warps copy the updated state out of TMEM.
 // The fp32 master state lives in TMEM (the update MMA accumulates onto it); o leaves through
-// shared memory and TMA stores.  Every wait is bounded (about 2 s): on expiry the CTA records the
-// library's timeout bit, every role leaves its loop at the next uniform check point, in-flight TMA
-// copies and MMAs are drained, TMEM is released and the kernel returns.
+// shared memory (staged in the chunk's PT tiles once Y has read them) and TMA stores.  Every
+// wait is bounded (about 2 s): on expiry the CTA records the library's timeout bit, every role
+// leaves its loop at the next uniform check point, in-flight TMA copies and MMAs are drained,
+// TMEM is released and the kernel returns.
 #pragma once
 
 #include <cuda.h>
@@ -50,12 +53,12 @@ constexpr int kThreads = 384;
 constexpr uint64_t kBudget = 4000000000ull;   // wait budget in SM cycles (about 2 s)
 
 // shared memory map (bytes from a 1024-aligned base); every MMA tile is 128-byte swizzled
-constexpr uint32_t OFF_QK = 0;          // 2 stages x 32 KB: kb0 [Q 64 rows | K 64 rows], kb1 [...]
-constexpr uint32_t QK_STAGE = 32768;
-constexpr uint32_t OFF_RD = 65536;      // 32 KB, per column half 16 KB: R' bf16 hi [64 t][128 B] +
-                                        // lo; with a split X first the bf16 low part of M
+constexpr uint32_t OFF_QK = 0;          // 32 KB: kb0 [Q 64 rows | K 64 rows], kb1 [...]
+constexpr uint32_t OFF_RD = 32768;      // 2 buffers (chunk parity) x 32 KB, per column half 16 KB:
+constexpr uint32_t RD_BUF = 32768;      // R' bf16 hi [64 t][128 B] + lo; with a split X, before
+                                        // R' of a chunk, the bf16 low part of M for its X
 constexpr uint32_t OFF_MB = 98304;      // 32 KB, per column half 16 KB: bf16 M [128 dk][128 B]
-constexpr uint32_t OFF_PW = 131072;     // 2 slots x 48 KB: a chunk's PT hi, PT lo, W hi, W lo;
+constexpr uint32_t OFF_PW = 131072;     // 2 slots x 48 KB: a chunk's PT hi, PT lo, W hi, W lo
 constexpr uint32_t PW_SLOT = 49152;     // after Y (and the update) the o tile is staged there
 constexpr uint32_t OFF_BAR = OFF_PW + 2 * PW_SLOT;
 constexpr int NBAR = 20;
@@ -72,8 +75,8 @@ constexpr uint32_t TM_X = 0, TM_Y = 256, TM_M = 384;
 // on the critical path) is reloaded as soon as the update has read it; PT (for o) once o has
 // left the slot.
 enum : int {
-  B_QK_FULL = 0, B_QK_EMPTY = 2, B_W_FULL = 4, B_W_EMPTY = 6, B_P_FULL = 8, B_P_EMPTY = 10,
-  B_X_FULL = 12, B_R_FULL, B_D3_FULL, B_Y_FULL, B_Y_EMPTY, B_M_READY, B_M_SCALED, B_DRAIN, B_END
+  B_QK_FULL = 0, B_QK_EMPTY, B_W_FULL = 2, B_W_EMPTY = 4, B_P_FULL = 6, B_P_EMPTY = 8,
+  B_X_FULL = 10, B_R_FULL, B_D3_FULL, B_Y_FULL, B_Y_EMPTY, B_M_READY, B_M_SCALED, B_DRAIN, B_END
 };
 static_assert(B_END <= NBAR, "barrier map");
 
@@ -707,9 +710,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   // X takes M as a hi + lo bf16 pair when o is fp32 (the layer, whose gated norm magnifies o's
   // error); a bf16 o carries its own rounding, and one round-to-nearest bf16 copy of M suffices.
   constexpr bool kSplitX = kF32;
-  // The low half of a split M shares the R' buffer, so there Y (which reads R') runs before the
-  // state update; otherwise the update, which the next chunk waits for, goes first.
-  constexpr bool kYFirst = kSplitX;
   GDN_TRACE_INIT;
   // Offsetting the __shared__ array itself (not a round trip through an integer) keeps every
   // access below a shared-memory access (ld/st.shared), not a generic one.
@@ -727,8 +727,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   auto bar = [&](int i) -> uint32_t { return sb + OFF_BAR + 8u * i; };
 
   if (threadIdx.x == 0) {
-    const int ones[] = {B_QK_FULL, B_QK_FULL + 1, B_QK_EMPTY, B_QK_EMPTY + 1, B_W_FULL,
-                        B_W_FULL + 1, B_P_FULL, B_P_FULL + 1, B_X_FULL, B_D3_FULL, B_Y_FULL, B_DRAIN};
+    const int ones[] = {B_QK_FULL, B_QK_EMPTY, B_W_FULL, B_W_FULL + 1, B_P_FULL, B_P_FULL + 1,
+                        B_X_FULL, B_D3_FULL, B_Y_FULL, B_DRAIN};
     for (int i : ones) tc::mbar_init(bar(i), 1);
     const int twos[] = {B_R_FULL, B_Y_EMPTY, B_M_READY, B_M_SCALED};
     for (int i : twos) tc::mbar_init(bar(i), 2);   // one arrive per column half
@@ -759,19 +759,20 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   if (warp == 0) {
     // ------------------------------- loads ----------------------------------------------------
     if (lane == 0) {
-      int armed_qk[2] = {-1, -1}, armed_w[2] = {-1, -1}, armed_p[2] = {-1, -1};
+      int armed_qk = -1, armed_w[2] = {-1, -1}, armed_p[2] = {-1, -1};
       bool ok = true;
       for (int c = 0; c < nC && ok; ++c) {
         const int s = c & 1, t0 = c * C;
-        if (c >= 2) ok = tc::mbar_wait(bar(B_QK_EMPTY + s), ((c >> 1) - 1) & 1, abort_flag, kBudget);
+        // one Q/K stage: chunk c's tile is loaded as soon as X of chunk c - 1 has read the last
+        if (c >= 1) ok = tc::mbar_wait(bar(B_QK_EMPTY), (c - 1) & 1, abort_flag, kBudget);
         if (!ok) break;
-        const uint32_t dst = sb + OFF_QK + s * QK_STAGE;
-        tc::mbar_arrive_expect_tx(bar(B_QK_FULL + s), 32768);
-        tc::tma_load_4d(dst, &tmq, bar(B_QK_FULL + s), 0, hk, t0, bq);
-        tc::tma_load_4d(dst + 8192, &tmk, bar(B_QK_FULL + s), 0, hk, t0, bq);
-        tc::tma_load_4d(dst + 16384, &tmq, bar(B_QK_FULL + s), 64, hk, t0, bq);
-        tc::tma_load_4d(dst + 24576, &tmk, bar(B_QK_FULL + s), 64, hk, t0, bq);
-        armed_qk[s] = c;
+        const uint32_t dst = sb + OFF_QK;
+        tc::mbar_arrive_expect_tx(bar(B_QK_FULL), 32768);
+        tc::tma_load_4d(dst, &tmq, bar(B_QK_FULL), 0, hk, t0, bq);
+        tc::tma_load_4d(dst + 8192, &tmk, bar(B_QK_FULL), 0, hk, t0, bq);
+        tc::tma_load_4d(dst + 16384, &tmq, bar(B_QK_FULL), 64, hk, t0, bq);
+        tc::tma_load_4d(dst + 24576, &tmk, bar(B_QK_FULL), 64, hk, t0, bq);
+        armed_qk = c;
         const uint8_t* src = pw_head + (long)c * kPwBytes;
         const uint32_t slot = sb + OFF_PW + s * PW_SLOT;
         if (c >= 2) ok = tc::mbar_wait(bar(B_W_EMPTY + s), ((c >> 1) - 1) & 1, abort_flag, kBudget);
@@ -787,9 +788,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       }
       // every load issued lands before the CTA can leave (at once unless a consumer gave up)
       volatile int never = 0;
+      if (armed_qk >= 0) tc::mbar_wait(bar(B_QK_FULL), armed_qk & 1, &never, kBudget / 4);
       for (int s = 0; s < 2; ++s) {
-        if (armed_qk[s] >= 0)
-          tc::mbar_wait(bar(B_QK_FULL + s), (armed_qk[s] >> 1) & 1, &never, kBudget / 4);
         if (armed_w[s] >= 0)
           tc::mbar_wait(bar(B_W_FULL + s), (armed_w[s] >> 1) & 1, &never, kBudget / 4);
         if (armed_p[s] >= 0)
@@ -798,72 +798,73 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     }
   } else if (warp == 1) {
     // -------------------------------- MMAs -----------------------------------------------------
+    // Per chunk c: X(c), then Y(c - 1) (it reads the other R' buffer and runs while R'(c) is
+    // being formed, off the state chain), then the state update of chunk c; Y of the last chunk
+    // follows the loop.
     if (lane == 0) {
+      const uint64_t dq = tc::sdesc_sw128(sb + OFF_QK, 16, 1024);
+      const uint64_t dm = tc::sdesc_sw128(sb + OFF_MB, 16384, 1024);
+      // Y = PT R' (rows 0..63 used), as hi.hi + lo.hi + hi.lo bf16 products             (bf16)
+      auto issue_Y = [&](int cy) -> bool {
+        const int sy = cy & 1;
+        if (cy >= 1 && !tc::mbar_wait(bar(B_Y_EMPTY), (cy - 1) & 1, abort_flag, kBudget)) return false;
+        if (!tc::mbar_wait(bar(B_P_FULL + sy), (cy >> 1) & 1, abort_flag, kBudget)) return false;
+        tc::tc_fence_after();
+        const uint64_t dpw = tc::sdesc_sw128(sb + OFF_PW + sy * PW_SLOT, 16, 1024);
+        const uint64_t drd = tc::sdesc_sw128(sb + OFF_RD + sy * RD_BUF, 16384, 1024);
+#pragma unroll
+        for (int i = 0; i < 12; ++i) {
+          const int ks = i / 3, term = i - 3 * ks;
+          tc::mma_bf16(tmem + TM_Y, tc::desc_adv(dpw, (term == 1 ? 8192 : 0) + ks * 32),
+                       tc::desc_adv(drd, (term == 2 ? 8192 : 0) + ks * 2048), ID_Y, i > 0);
+        }
+        tc::mma_commit(bar(B_Y_FULL));
+        tc::mma_commit(bar(B_P_EMPTY + sy));
+        GDN_TRACE(cy, 22);
+        return true;
+      };
       bool ok = true;
       for (int c = 0; c < nC && ok; ++c) {
         const int s = c & 1;
-        const uint32_t qk = sb + OFF_QK + s * QK_STAGE;
-        const uint32_t pws = sb + OFF_PW + s * PW_SLOT;
         // X = [Q; K] M  (M as one bf16 copy, or a hi + lo pair)                     (bf16)
-        ok = tc::mbar_wait(bar(B_QK_FULL + s), (c >> 1) & 1, abort_flag, kBudget) &&
+        ok = tc::mbar_wait(bar(B_QK_FULL), c & 1, abort_flag, kBudget) &&
              tc::mbar_wait(bar(B_M_READY), c & 1, abort_flag, kBudget);
         if (!ok) break;
         GDN_TRACE(c, 12);
         tc::tc_fence_after();
         {
-          const uint64_t dq = tc::sdesc_sw128(qk, 16, 1024);
-          const uint64_t dm = tc::sdesc_sw128(sb + OFF_MB, 16384, 1024);
-          const uint64_t dml = tc::sdesc_sw128(sb + OFF_RD, 16384, 1024);
+          const uint64_t dml = tc::sdesc_sw128(sb + OFF_RD + s * RD_BUF, 16384, 1024);
 #pragma unroll
           for (int ks = 0; ks < (kSplitX ? 16 : 8); ++ks)
             tc::mma_bf16(tmem + TM_X + 128 * s, tc::desc_adv(dq, ((ks >> 2) & 1) * 16384 + (ks & 3) * 32),
                          tc::desc_adv(ks < 8 ? dm : dml, (ks & 7) * 2048), ID_X, ks > 0);
         }
         tc::mma_commit(bar(B_X_FULL));
-        tc::mma_commit(bar(B_QK_EMPTY + s));
+        tc::mma_commit(bar(B_QK_EMPTY));
         GDN_TRACE(c, 20);
-        ok = tc::mbar_wait(bar(B_R_FULL), c & 1, abort_flag, kBudget);
+        if (c >= 1 && !(ok = issue_Y(c - 1))) break;
+        // M += W R' (TMEM holds gamma_last M), hi.hi + lo.hi + hi.lo bf16 products     (bf16)
+        ok = tc::mbar_wait(bar(B_R_FULL), c & 1, abort_flag, kBudget) &&
+             tc::mbar_wait(bar(B_M_SCALED), c & 1, abort_flag, kBudget) &&
+             tc::mbar_wait(bar(B_W_FULL + s), (c >> 1) & 1, abort_flag, kBudget);
         if (!ok) break;
         GDN_TRACE(c, 13);
-        // Y = PT R' (rows 0..63 used) and M += W R' (TMEM holds gamma_last M), each as
-        // hi.hi + lo.hi + hi.lo bf16 products                                        (bf16)
-        const uint64_t dpw = tc::sdesc_sw128(pws, 16, 1024);
-        const uint64_t drd = tc::sdesc_sw128(sb + OFF_RD, 16384, 1024);
-        auto issue_Y = [&]() -> bool {
-          if (c >= 1 && !tc::mbar_wait(bar(B_Y_EMPTY), (c - 1) & 1, abort_flag, kBudget)) return false;
-          if (!tc::mbar_wait(bar(B_P_FULL + s), (c >> 1) & 1, abort_flag, kBudget)) return false;
-          GDN_TRACE(c, 16);
-          tc::tc_fence_after();
-#pragma unroll
-          for (int i = 0; i < 12; ++i) {
-            const int ks = i / 3, term = i - 3 * ks;
-            tc::mma_bf16(tmem + TM_Y, tc::desc_adv(dpw, (term == 1 ? 8192 : 0) + ks * 32),
-                         tc::desc_adv(drd, (term == 2 ? 8192 : 0) + ks * 2048), ID_Y, i > 0);
-          }
-          tc::mma_commit(bar(B_Y_FULL));
-          tc::mma_commit(bar(B_P_EMPTY + s));
-          GDN_TRACE(c, 22);
-          return true;
-        };
-        auto issue_D3 = [&]() -> bool {
-          if (!tc::mbar_wait(bar(B_M_SCALED), c & 1, abort_flag, kBudget)) return false;
-          if (!tc::mbar_wait(bar(B_W_FULL + s), (c >> 1) & 1, abort_flag, kBudget)) return false;
-          GDN_TRACE(c, 15);
-          tc::tc_fence_after();
+        tc::tc_fence_after();
+        {
+          const uint64_t dpw = tc::sdesc_sw128(sb + OFF_PW + s * PW_SLOT, 16, 1024);
+          const uint64_t drd = tc::sdesc_sw128(sb + OFF_RD + s * RD_BUF, 16384, 1024);
 #pragma unroll
           for (int i = 0; i < 12; ++i) {
             const int ks = i / 3, term = i - 3 * ks;
             tc::mma_bf16(tmem + TM_M, tc::desc_adv(dpw, 16384 + (term == 1 ? 16384 : 0) + ks * 32),
                          tc::desc_adv(drd, (term == 2 ? 8192 : 0) + ks * 2048), ID_Y, 1);
           }
-          tc::mma_commit(bar(B_D3_FULL));
-          tc::mma_commit(bar(B_W_EMPTY + s));
-          GDN_TRACE(c, 21);
-          return true;
-        };
-        ok = kYFirst ? (issue_Y() && issue_D3()) : (issue_D3() && issue_Y());
-        if (!ok) break;
+        }
+        tc::mma_commit(bar(B_D3_FULL));
+        tc::mma_commit(bar(B_W_EMPTY + s));
+        GDN_TRACE(c, 21);
       }
+      if (ok && nC >= 1) issue_Y(nC - 1);
       tc::mma_commit(bar(B_DRAIN));
       volatile int never = 0;
       tc::mbar_wait(bar(B_DRAIN), 0, &never, kBudget / 4);
@@ -875,7 +876,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     const int hh = (warp - 4) >> 2, q = warp & 3, r = 32 * q + lane, t = r & 63;
     const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
     const uint32_t tcol = 64 * hh;                       // this half's TMEM / value columns
-    const uint32_t mb = sb + OFF_MB + hh * 16384, rd = sb + OFF_RD + hh * 16384;
+    const uint32_t mb = sb + OFF_MB + hh * 16384, rd0 = sb + OFF_RD + hh * 16384;
     const uint32_t id_wg = 1 + 3 * hh, id_lo = 2 + 3 * hh, id_hi = 3 + 3 * hh;
     const bool leader = (q == 0 && lane == 0);
     [[maybe_unused]] const int ev = 10 * hh;
@@ -884,7 +885,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     };
     // 32 columns (32p ..) of M row r (this half) for the X MMA: one round-to-nearest bf16 copy in Mb,
     // or (kSplitX) a hi + lo pair, hi into Mb and lo into the R' buffer
-    auto store_m32 = [&](const float (&m)[32], int p) {
+    auto store_m32 = [&](const float (&m)[32], int p, uint32_t rd) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const uint32_t sw = tc::sw128(r, 4 * p + j);
@@ -926,8 +927,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
 #pragma unroll
         for (int i = 0; i < 64; ++i) m[i] = 0.f;
       }
-      store_m32(*reinterpret_cast<const float(*)[32]>(&m[0]), 0);
-      store_m32(*reinterpret_cast<const float(*)[32]>(&m[32]), 1);
+      store_m32(*reinterpret_cast<const float(*)[32]>(&m[0]), 0, rd0);
+      store_m32(*reinterpret_cast<const float(*)[32]>(&m[32]), 1, rd0);
       const float gl = gam_at(0, 63);
 #pragma unroll
       for (int i = 0; i < 64; ++i) m[i] *= gl;
@@ -975,7 +976,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
             }
             // MN-major bf16 B operand: row t (K), 16-byte chunk 4p + j of this half's columns
             const uint32_t sw = tc::sw128(t, 4 * p + j);
-            st_split8(rd + sw, rd + 8192 + sw, rv);
+            st_split8(rd0 + s * RD_BUF + sw, rd0 + s * RD_BUF + 8192 + sw, rv);
           }
         }
         tc::fence_proxy_async_smem();
@@ -997,8 +998,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         float m[64];
         tmem_ld64(tmem + lane_off + TM_M + tcol, m);
         tc::tmem_wait_ld();
-        store_m32(*reinterpret_cast<const float(*)[32]>(&m[0]), 0);
-        store_m32(*reinterpret_cast<const float(*)[32]>(&m[32]), 1);
+        // the next chunk's X reads the low part from the other R' buffer (whose Y is done:
+        // this update was issued after it)
+        store_m32(*reinterpret_cast<const float(*)[32]>(&m[0]), 0, rd0 + ((c + 1) & 1) * RD_BUF);
+        store_m32(*reinterpret_cast<const float(*)[32]>(&m[32]), 1, rd0 + ((c + 1) & 1) * RD_BUF);
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
         tc::named_bar(id_wg, 128);
