@@ -429,7 +429,9 @@ def profile_case(args):
         step()
     torch.cuda.synchronize()
     gdn.check_error(dev)
-    print(json.dumps({"profile_case": workload_name(w), "launches": args.steps}), flush=True)
+    variant = gdn.chunk_fwd_variant(w.dk, w.dv, w.chunk, w.torch_dtype)
+    print(json.dumps({"profile_case": workload_name(w), "calls": args.steps,
+                      "launches": args.steps * (2 if variant == "tcgen05" else 1)}), flush=True)
 
 
 def main():
@@ -515,7 +517,10 @@ def main():
                        "seq_len": w.T, "parallelism": f"replicas x{world} (no exchange)",
                        "kernel_variant": variant,
                        "l2": "256 MiB write between timed steps (outside the events)"},
-            "roofline": roof, "gpu_launches": args.steps * 1,
+            "roofline": roof,
+            # the tensor-core forward is two kernels per call (the operand pre-pass, then the
+            # recurrence); the SIMT forward one
+            "gpu_launches": args.steps * (2 if variant == "tcgen05" else 1),
             "clocks": clocks.summary()}
 
     e2e = e2e_prefill(gdn, x, w, dev, steps=max(3, min(args.steps, 10)))
