@@ -30,7 +30,8 @@ from typing import Dict, Optional
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_decode_inputs", "make_layer_inputs"]
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_decode_inputs", "make_layer_inputs",
+           "make_decode_layer_inputs"]
 
 
 @dataclass(frozen=True)
@@ -80,6 +81,11 @@ WORKLOADS: Dict[str, Workload] = {
     # full layer, 8:1 value/key variant: conv k=4 + SiLU + L2 prologue, gated RMSNorm epilogue
     "layer_8to1": Workload("layer_8to1", B=2, T=8192, Hk=16, Hv=128, dk=128, dv=128, chunk=64,
                            dtype="bf16", gate="wide", seed=4, layer=True),
+    # full-layer decode: 256 sequences x 1 token per step, the decode shapes with the layer's
+    # raw projections, a carried 3-token conv history and the gated norm, 100 steps
+    "decode_layer": Workload("decode_layer", B=256, T=1, Hk=16, Hv=48, dk=128, dv=128, chunk=64,
+                             dtype="bf16", gate="wide", s0_std=0.02, seed=5, steps=100,
+                             layer=True),
 }
 
 
@@ -167,6 +173,41 @@ def make_layer_inputs(w: Workload) -> Dict[str, Optional[torch.Tensor]]:
     norm_w = torch.ones(w.dv)
     return {"q_raw": q_raw.contiguous(), "k_raw": k_raw.contiguous(), "v_raw": v_raw.contiguous(),
             "log_alpha": log_alpha, "beta": beta, "S0": S0, "z": z.contiguous(),
+            "conv_wq": conv_wq.contiguous(), "conv_wk": conv_wk.contiguous(),
+            "conv_wv": conv_wv.contiguous(), "norm_w": norm_w}
+
+
+def make_decode_layer_inputs(w: Workload) -> Dict[str, torch.Tensor]:
+    """Inputs of ``w.steps`` consecutive full-layer decode steps over ``w.B`` sequences.
+
+    Per step: raw q, k [steps, N, Hk*dk], raw v, z [steps, N, Hv*dv] (N(0,1), storage dtype) and
+    the gates [steps, N, Hv]; once: S0 [N, Hv, dk, dv] ~ N(0, s0_std), the conv history of the
+    three tokens before the first step [N, 3, channels] (N(0,1), storage dtype, oldest first: as if
+    the request had already run three tokens), conv taps [channels, 4] ~ N(0, conv_w_std) and the
+    d_v gain of ones.
+    """
+    if not (w.layer and w.steps):
+        raise ValueError("not a decode-layer workload")
+    g = _gen(w.seed)
+    dt = w.torch_dtype
+    s, n = w.steps, w.B
+    cq, cv = w.Hk * w.dk, w.Hv * w.dv
+    q_raw = torch.randn(s, n, cq, generator=g).to(dt)
+    k_raw = torch.randn(s, n, cq, generator=g).to(dt)
+    v_raw = torch.randn(s, n, cv, generator=g).to(dt)
+    log_alpha, beta = _gates(g, (s, n, w.Hv), w.gate)
+    S0 = torch.randn(n, w.Hv, w.dk, w.dv, generator=g) * w.s0_std
+    z = torch.randn(s, n, cv, generator=g).to(dt)
+    hq = torch.randn(n, 3, cq, generator=g).to(dt)
+    hk = torch.randn(n, 3, cq, generator=g).to(dt)
+    hv = torch.randn(n, 3, cv, generator=g).to(dt)
+    conv_wq = torch.randn(cq, 4, generator=g) * w.conv_w_std
+    conv_wk = torch.randn(cq, 4, generator=g) * w.conv_w_std
+    conv_wv = torch.randn(cv, 4, generator=g) * w.conv_w_std
+    norm_w = torch.ones(w.dv)
+    return {"q_raw": q_raw.contiguous(), "k_raw": k_raw.contiguous(), "v_raw": v_raw.contiguous(),
+            "log_alpha": log_alpha, "beta": beta, "S0": S0.contiguous(), "z": z.contiguous(),
+            "hq": hq.contiguous(), "hk": hk.contiguous(), "hv": hv.contiguous(),
             "conv_wq": conv_wq.contiguous(), "conv_wk": conv_wk.contiguous(),
             "conv_wv": conv_wv.contiguous(), "norm_w": norm_w}
 

@@ -23,6 +23,10 @@ Functions and the passages they follow (page titles; the C file's header has the
                             activation of the model but the state is BF16 ("L'attention
                             hybride", "Le float32 n'est pas un détail").
   * ``round_bf16``        — that rounding, written from the bf16 format (8 significant bits).
+  * ``decode_layer_steps`` — the layer one token at a time ("Chapitre 16 ... Kimi K3", 16.3) with
+                            the conv's three-token history carried between steps: the composition
+                            above on [history; token].  Pinned by equality with ``layer_forward``
+                            over the whole sequence.
 """
 from __future__ import annotations
 
@@ -210,6 +214,42 @@ class OracleLib:
         return y, sT
 
 
+def _decode_layer_steps(lib: "OracleLib", q_raw, k_raw, v_raw, z, hq, hk, hv, wq, wk, wv,
+                        log_alpha, beta, S0, norm_w, Hk: int, Hv: int, dk: int, dv: int,
+                        l2_eps: float = 1e-6, norm_eps: float = 1e-5, scale: float = 1.0,
+                        threads: Optional[int] = None):
+    """Consecutive full-layer decode steps.  Per step s: raw q, k [steps,N,Hk*dk], raw v, z
+    [steps,N,Hv*dv], gates [steps,N,Hv]; hq, hk [N,3,Hk*dk] and hv [N,3,Hv*dv] are the raw inputs
+    of the three tokens before the first step (oldest first); S0 [N,Hv,dk,dv] holds S^T.
+
+    A step is the layer on one more token of each sequence: the conv sees the carried history,
+    which is the conv of the concatenated sequence [history; token] at its last position (the
+    zero-history conv over four tokens, read at the fourth), then L2, one recurrence step and the
+    gated norm.  Returns (y [steps,N,Hv,dv], final state, final hq, hk, hv), fp64."""
+    q_raw, k_raw, v_raw, z = _f64(q_raw), _f64(k_raw), _f64(v_raw), _f64(z)
+    hq, hk, hv, S = _f64(hq).copy(), _f64(hk).copy(), _f64(hv).copy(), _f64(S0)
+    la, be = _f64(log_alpha), _f64(beta)
+    steps, N = q_raw.shape[:2]
+    ys = []
+    for s in range(steps):
+        xq = np.concatenate([hq, q_raw[s][:, None]], axis=1)            # [N, 4, C]
+        xk = np.concatenate([hk, k_raw[s][:, None]], axis=1)
+        xv = np.concatenate([hv, v_raw[s][:, None]], axis=1)
+        qc = lib.causal_conv_silu(xq, wq)[:, 3]
+        kc = lib.causal_conv_silu(xk, wk)[:, 3]
+        vc = lib.causal_conv_silu(xv, wv)[:, 3]
+        q = lib.l2_normalize(qc.reshape(N, 1, Hk, dk), l2_eps)
+        k = lib.l2_normalize(kc.reshape(N, 1, Hk, dk), l2_eps)
+        o, S = lib.gated_delta(q, k, vc.reshape(N, 1, Hv, dv), la[s][:, None], be[s][:, None], S,
+                               scale=scale, threads=threads)
+        ys.append(lib.gated_rmsnorm(o[:, 0], z[s].reshape(N, Hv, dv), norm_w, norm_eps))
+        hq, hk, hv = xq[:, 1:], xk[:, 1:], xv[:, 1:]
+    return np.stack(ys), S, hq, hk, hv
+
+
+OracleLib.decode_layer_steps = _decode_layer_steps
+
+
 def get() -> OracleLib:
     """The default oracle (compiled on first use)."""
     global _default
@@ -245,3 +285,7 @@ def prologue(*a, **kw):
 
 def layer_forward(*a, **kw):
     return get().layer_forward(*a, **kw)
+
+
+def decode_layer_steps(*a, **kw):
+    return get().decode_layer_steps(*a, **kw)

@@ -287,4 +287,61 @@ def pin_round_bf16_matches_library(orc):
     assert np.array_equal(oracle.round_bf16(x), ref)
 
 
+# ---------------------------------------------------------------------------------------------
+# the layer one token at a time, conv history carried ([KIMI] 16.3)
+# ---------------------------------------------------------------------------------------------
+def _layer_rand(seed, N=2, T=6, Hk=1, Hv=2, dk=4, dv=4):
+    rng = np.random.default_rng(seed)
+    cq, cv = Hk * dk, Hv * dv
+    d = {"q_raw": rng.standard_normal((N, T, cq)), "k_raw": rng.standard_normal((N, T, cq)),
+         "v_raw": rng.standard_normal((N, T, cv)), "z": rng.standard_normal((N, T, cv)),
+         "wq": rng.standard_normal((cq, 4)) * 0.5, "wk": rng.standard_normal((cq, 4)) * 0.5,
+         "wv": rng.standard_normal((cv, 4)) * 0.5,
+         "la": -np.log1p(np.exp(rng.standard_normal((N, T, Hv)))) * 0.3,
+         "be": expit(rng.standard_normal((N, T, Hv))),
+         "S0": rng.standard_normal((N, Hv, dk, dv)) * 0.3,
+         "w": 0.5 + rng.random(dv)}
+    return d
+
+
+def pin_decode_layer_steps_equal_layer_forward(orc):
+    """T single-token layer steps from a zero conv history equal the layer over the T-token
+    sequence (a fresh request run token by token): same outputs, same final state."""
+    Hk, Hv, dk, dv, T = 1, 2, 4, 4, 6
+    d = _layer_rand(31, T=T, Hk=Hk, Hv=Hv, dk=dk, dv=dv)
+    y, sT = orc.layer_forward(d["q_raw"], d["k_raw"], d["v_raw"], d["z"], d["wq"], d["wk"],
+                              d["wv"], d["la"], d["be"], d["S0"], d["w"], Hk, Hv, dk, dv,
+                              scale=0.7)
+    N = d["q_raw"].shape[0]
+    zq = np.zeros((N, 3, Hk * dk))
+    zv = np.zeros((N, 3, Hv * dv))
+    tm = lambda a: np.swapaxes(a, 0, 1)                     # [N, T, ...] -> [T, N, ...]
+    ys, sS, hq, hk, hv = orc.decode_layer_steps(
+        tm(d["q_raw"]), tm(d["k_raw"]), tm(d["v_raw"]), tm(d["z"]), zq, zq, zv, d["wq"], d["wk"],
+        d["wv"], tm(d["la"]), tm(d["be"]), d["S0"], d["w"], Hk, Hv, dk, dv, scale=0.7)
+    assert np.allclose(tm(ys), y, rtol=1e-12, atol=1e-12)
+    assert np.allclose(sS, sT, rtol=1e-12, atol=1e-12)
+    assert np.array_equal(hv, d["v_raw"][:, -3:])
+
+
+def pin_decode_layer_history_is_the_three_previous_tokens(orc):
+    """A carried history acts as three earlier tokens: the steps equal the layer over
+    [history; tokens] in which the three history tokens change no state (alpha = 1, beta = 0),
+    read from the fourth position on.  Catches a reversed or shifted history."""
+    Hk, Hv, dk, dv, T = 1, 2, 4, 4, 4
+    d = _layer_rand(32, T=T + 3, Hk=Hk, Hv=Hv, dk=dk, dv=dv)
+    la, be = d["la"].copy(), d["be"].copy()
+    la[:, :3] = 0.0
+    be[:, :3] = 0.0
+    y, sT = orc.layer_forward(d["q_raw"], d["k_raw"], d["v_raw"], d["z"], d["wq"], d["wk"],
+                              d["wv"], la, be, d["S0"], d["w"], Hk, Hv, dk, dv)
+    tm = lambda a: np.swapaxes(a, 0, 1)
+    ys, sS, _, _, _ = orc.decode_layer_steps(
+        tm(d["q_raw"][:, 3:]), tm(d["k_raw"][:, 3:]), tm(d["v_raw"][:, 3:]), tm(d["z"][:, 3:]),
+        d["q_raw"][:, :3], d["k_raw"][:, :3], d["v_raw"][:, :3], d["wq"], d["wk"], d["wv"],
+        tm(la[:, 3:]), tm(be[:, 3:]), d["S0"], d["w"], Hk, Hv, dk, dv)
+    assert np.allclose(tm(ys), y[:, 3:], rtol=1e-12, atol=1e-12)
+    assert np.allclose(sS, sT, rtol=1e-12, atol=1e-12)
+
+
 ALL_PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]

@@ -43,3 +43,14 @@ def test_decode_and_layer_recipes():
     L = gi.make_layer_inputs(lw)
     assert L["q_raw"].shape == (2, 16, 2048) and L["v_raw"].shape == (2, 16, 16384)
     assert L["conv_wv"].shape == (16384, 4) and torch.equal(L["norm_w"], torch.ones(128))
+
+
+def test_decode_layer_inputs_shapes_and_determinism():
+    w = gi.WORKLOADS["decode_layer"].with_sizes(B=3, Hk=2, Hv=6, steps=2)
+    a, b = gi.make_decode_layer_inputs(w), gi.make_decode_layer_inputs(w)
+    assert a["q_raw"].shape == (2, 3, 2 * 128) and a["v_raw"].shape == (2, 3, 6 * 128)
+    assert a["hq"].shape == (3, 3, 2 * 128) and a["hv"].shape == (3, 3, 6 * 128)
+    assert a["log_alpha"].shape == (2, 3, 6) and a["S0"].shape == (3, 6, 128, 128)
+    assert a["q_raw"].dtype == torch.bfloat16 and a["conv_wv"].shape == (6 * 128, 4)
+    for k in a:
+        assert torch.equal(a[k], b[k]), k
