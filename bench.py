@@ -69,6 +69,16 @@ def decode_bytes(w: gi.Workload) -> int:
                                                  + 8 * w.Hv)
 
 
+def decode_layer_bytes(w: gi.Workload) -> int:
+    """One full-layer decode step: the state read and written, the raw q, k, v, z of the token,
+    the conv history read and written (3 tokens of every channel), the gates and the output y.
+    (Conv taps and the norm gain are per-layer constants, read from L2.)"""
+    s = 2 if w.dtype == "bf16" else 4
+    N, cq, cv = w.B, w.Hk * w.dk, w.Hv * w.dv
+    return (2 * N * w.Hv * w.dk * w.dv * 4 + N * (2 * cq + 2 * cv) * s
+            + 2 * N * 3 * (2 * cq + cv) * s + N * 8 * w.Hv + N * cv * s)
+
+
 # ------------------------------------------------------------------------------------------------
 # helpers
 # ------------------------------------------------------------------------------------------------
@@ -260,6 +270,43 @@ def bench_decode(gdn, dev, warmup, flush, peaks):
     torch.cuda.synchronize()
     t = a.elapsed_time(b) / 1e3 / w.steps
     by = decode_bytes(w)
+    return {"value": by / t / 1e9, "unit": "GB/s", "us_per_step": t * 1e6,
+            "tokens_per_s": w.B / t, "roofline_frac": by / t / 1e9 / peaks["hbm_gbs"],
+            "bytes_per_step": by, "workload": workload_name(w)}
+
+
+def bench_decode_layer(gdn, dev, warmup, flush, peaks):
+    """The fused full-layer decode step on the decode shapes (256 sequences, Hk16 Hv48 d128)."""
+    w = gi.WORKLOADS["decode_layer"]
+    x = gi.make_decode_layer_inputs(w)
+    d = to_dev(x, dev)
+    S = d["S0"].clone()
+    hist = [[d["hq"].clone(), d["hk"].clone(), d["hv"].clone()]]
+    hist.append([torch.empty_like(t) for t in hist[0]])
+    y = torch.empty(w.B, w.Hv, w.dv, device=dev, dtype=w.torch_dtype)
+    state = {"s": 0}
+
+    def step():
+        s = state["s"] % w.steps
+        hin, hout = hist[state["s"] & 1], hist[(state["s"] + 1) & 1]
+        gdn.decode_layer_step(d["q_raw"][s], d["k_raw"][s], d["v_raw"][s], d["z"][s], *hin, *hout,
+                              d["conv_wq"], d["conv_wk"], d["conv_wv"], d["log_alpha"][s],
+                              d["beta"][s], S, d["norm_w"], Hk=w.Hk, Hv=w.Hv, dk=w.dk, dv=w.dv,
+                              out=y)
+        state["s"] += 1
+    # the state (805 MB) is far larger than L2: consecutive steps need no flush
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(w.steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    gdn.check_error(dev)
+    t = a.elapsed_time(b) / 1e3 / w.steps
+    by = decode_layer_bytes(w)
     return {"value": by / t / 1e9, "unit": "GB/s", "us_per_step": t * 1e6,
             "tokens_per_s": w.B / t, "roofline_frac": by / t / 1e9 / peaks["hbm_gbs"],
             "bytes_per_step": by, "workload": workload_name(w)}
@@ -534,6 +581,7 @@ def main():
         if not args.no_secondary:
             sec = {}
             sec["decode"] = bench_decode(gdn, dev, args.warmup, flush, peaks)
+            sec["decode_layer"] = bench_decode_layer(gdn, dev, args.warmup, flush, peaks)
             del d
             torch.cuda.empty_cache()
             _, xl, dl, _, sec["long_context"] = bench_prefill_like(

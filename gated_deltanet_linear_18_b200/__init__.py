@@ -62,6 +62,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_chunk_fwd_variant.restype = I
         L.gdn_decode_step.argtypes = [P] * 7 + [I] * 5 + [F, I, P]
         L.gdn_decode_step.restype = I
+        L.gdn_decode_layer_step.argtypes = [P] * 18 + [I] * 5 + [F, F, F, I, P]
+        L.gdn_decode_layer_step.restype = I
         L.gdn_prologue.argtypes = [P] * 9 + [I] * 6 + [F, I, P]
         L.gdn_prologue.restype = I
         L.gdn_out_norm.argtypes = [P, P, P, P, LL, I, F, I, P]
@@ -165,6 +167,35 @@ def decode_step(q, k, v, log_alpha, beta, S, *, scale: float = 1.0,
                                    N, Hk, Hv, dk, dv, float(scale), _io_dtype(q), _stream(dev))
     _check("gdn_decode_step", st)
     return o
+
+
+def decode_layer_step(q_raw, k_raw, v_raw, z, hq_in, hk_in, hv_in, hq_out, hk_out, hv_out,
+                      wq, wk, wv, log_alpha, beta, S, norm_w, *, Hk: int, Hv: int, dk: int,
+                      dv: int, scale: float = 1.0, l2_eps: float = 1e-6, norm_eps: float = 1e-5,
+                      out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One full-layer decode step (conv over the carried history + SiLU + L2, recurrence step
+    with S updated in place, gated RMSNorm) in one kernel.  q_raw, k_raw [N,Hk*dk]; v_raw, z
+    [N,Hv*dv]; histories [N,3,channels] (the _out set receives the moved-on history); conv taps
+    [channels,4]; gates [N,Hv]; S [N,Hv,dk,dv]; norm_w [dv].  Returns y [N,Hv,dv]."""
+    N = q_raw.shape[0]
+    if (k_raw.shape != q_raw.shape or q_raw.shape[1] != Hk * dk or v_raw.shape != (N, Hv * dv)
+            or z.shape != v_raw.shape or hq_in.shape != (N, 3, Hk * dk)
+            or hk_in.shape != hq_in.shape or hv_in.shape != (N, 3, Hv * dv)
+            or hq_out.shape != hq_in.shape or hk_out.shape != hk_in.shape
+            or hv_out.shape != hv_in.shape or S.shape != (N, Hv, dk, dv)):
+        raise ValueError("decode-layer shapes disagree")
+    _f32(wq, wk, wv, log_alpha, beta, S, norm_w)
+    y = torch.empty(N, Hv, dv, device=q_raw.device, dtype=q_raw.dtype) if out is None else out
+    dev = _dev(q_raw, k_raw, v_raw, z, hq_in, hk_in, hv_in, hq_out, hk_out, hv_out, wq, wk, wv,
+               log_alpha, beta, S, norm_w, y)
+    with torch.cuda.device(dev):
+        st = lib().gdn_decode_layer_step(
+            _p(q_raw), _p(k_raw), _p(v_raw), _p(z), _p(hq_in), _p(hk_in), _p(hv_in), _p(hq_out),
+            _p(hk_out), _p(hv_out), _p(wq), _p(wk), _p(wv), _p(log_alpha), _p(beta), _p(S),
+            _p(norm_w), _p(y), N, Hk, Hv, dk, dv, float(scale), float(l2_eps), float(norm_eps),
+            _io_dtype(q_raw), _stream(dev))
+    _check("gdn_decode_layer_step", st)
+    return y
 
 
 def prologue(q_raw, k_raw, v_raw, wq, wk, wv, Hk: int, Hv: int, dk: int, dv: int,

@@ -8,6 +8,7 @@
 #include "gdn.h"
 #include "common.cuh"
 #include "decode.cuh"
+#include "decode_layer.cuh"
 #include "elementwise.cuh"
 #include "simt_chunk.cuh"
 #include "tc_chunk.cuh"
@@ -103,6 +104,55 @@ gdn_status decode_dispatch(int dk, int dv, const void* q, const void* k, const v
     case 64: return decode_dispatch_dv<Tio, 64>(dv, q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
     case 128:
       return decode_dispatch_dv<Tio, 128>(dv, q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
+  }
+  return GDN_ERR_UNSUPPORTED;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Full-layer decode step dispatch over (dk, dv)
+// ---------------------------------------------------------------------------------------------
+struct DecodeLayerArgs {
+  const void *q_raw, *k_raw, *v_raw, *z, *hq_in, *hk_in, *hv_in;
+  void *hq_out, *hk_out, *hv_out;
+  const float *wq, *wk, *wv, *la, *be;
+  float* S;
+  const float* norm_w;
+  void* y;
+  int N, Hk, Hv;
+  float scale, l2_eps, norm_eps;
+};
+
+template <int DK, int DV, typename Tio>
+gdn_status decode_layer_launch(const DecodeLayerArgs& a, cudaStream_t st) {
+  using Sh = DecodeShape<DK, DV>;
+  decode_layer_step_kernel<DK, DV, Tio><<<(unsigned)((long)a.N * a.Hv), Sh::NT, 0, st>>>(
+      static_cast<const Tio*>(a.q_raw), static_cast<const Tio*>(a.k_raw),
+      static_cast<const Tio*>(a.v_raw), static_cast<const Tio*>(a.z),
+      static_cast<const Tio*>(a.hq_in), static_cast<const Tio*>(a.hk_in),
+      static_cast<const Tio*>(a.hv_in), static_cast<Tio*>(a.hq_out), static_cast<Tio*>(a.hk_out),
+      static_cast<Tio*>(a.hv_out), a.wq, a.wk, a.wv, a.la, a.be, a.S, a.norm_w,
+      static_cast<Tio*>(a.y), a.Hk, a.Hv, a.scale, a.l2_eps, a.norm_eps);
+  return launch_status();
+}
+
+template <typename Tio, int DK>
+gdn_status decode_layer_dispatch_dv(int dv, const DecodeLayerArgs& a, cudaStream_t st) {
+  switch (dv) {
+    case 16: return decode_layer_launch<DK, 16, Tio>(a, st);
+    case 32: return decode_layer_launch<DK, 32, Tio>(a, st);
+    case 64: return decode_layer_launch<DK, 64, Tio>(a, st);
+    case 128: return decode_layer_launch<DK, 128, Tio>(a, st);
+  }
+  return GDN_ERR_UNSUPPORTED;
+}
+
+template <typename Tio>
+gdn_status decode_layer_dispatch(int dk, int dv, const DecodeLayerArgs& a, cudaStream_t st) {
+  switch (dk) {
+    case 16: return decode_layer_dispatch_dv<Tio, 16>(dv, a, st);
+    case 32: return decode_layer_dispatch_dv<Tio, 32>(dv, a, st);
+    case 64: return decode_layer_dispatch_dv<Tio, 64>(dv, a, st);
+    case 128: return decode_layer_dispatch_dv<Tio, 128>(dv, a, st);
   }
   return GDN_ERR_UNSUPPORTED;
 }
@@ -243,6 +293,35 @@ gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const floa
                          gdn_dtype dtype, gdn_stream_t stream) {
   return gdn_chunk_fwd_ex(q, k, v, log_alpha, beta, S0, o, S_T, B, T, Hk, Hv, dk, dv, chunk,
                           scale, dtype, GDN_VARIANT_AUTO, stream);
+}
+
+gdn_status gdn_decode_layer_step(const void* q_raw, const void* k_raw, const void* v_raw,
+                                 const void* z, const void* hq_in, const void* hk_in,
+                                 const void* hv_in, void* hq_out, void* hk_out, void* hv_out,
+                                 const float* wq, const float* wk, const float* wv,
+                                 const float* log_alpha, const float* beta, float* S,
+                                 const float* norm_w, void* y, int N, int Hk, int Hv, int dk,
+                                 int dv, float scale, float l2_eps, float norm_eps,
+                                 gdn_dtype dtype, gdn_stream_t stream) {
+  if (N < 0 || !valid_dtype(dtype)) return GDN_ERR_INVALID_ARG;
+  gdn_status s = validate_heads(Hk, Hv, dk, dv);
+  if (s != GDN_OK) return s;
+  if (!(l2_eps >= 0.f) || !(norm_eps >= 0.f)) return GDN_ERR_INVALID_ARG;
+  if (N == 0) return GDN_OK;
+  const void* tensors[] = {q_raw, k_raw, v_raw, z, hq_in, hk_in, hv_in, hq_out, hk_out, hv_out,
+                           S, y};
+  for (const void* p : tensors)
+    if (!p || !aligned16(p)) return GDN_ERR_INVALID_ARG;
+  const float* weights[] = {wq, wk, wv, log_alpha, beta, norm_w};
+  for (const float* p : weights)
+    if (!p || !aligned4(p)) return GDN_ERR_INVALID_ARG;
+  if ((long)N * Hv > 0x7fffffffL) return GDN_ERR_UNSUPPORTED;
+  const DecodeLayerArgs a{q_raw, k_raw, v_raw, z, hq_in, hk_in, hv_in, hq_out, hk_out, hv_out,
+                          wq, wk, wv, log_alpha, beta, S, norm_w, y, N, Hk, Hv, scale,
+                          l2_eps, norm_eps};
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == GDN_F32) return decode_layer_dispatch<float>(dk, dv, a, st);
+  return decode_layer_dispatch<__nv_bfloat16>(dk, dv, a, st);
 }
 
 gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const float* log_alpha,

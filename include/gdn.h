@@ -133,6 +133,35 @@ GDN_API gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
                            gdn_dtype dtype, gdn_stream_t stream);
 
 /*
+ * One decode step of the whole layer for N sequences, in one kernel: the prologue (causal conv of
+ * 4 taps over a carried three-token history, SiLU, L2 normalisation of each q and k head), the
+ * recurrence step (state in place) and the gated RMSNorm.  ("Chapitre 16 - Assembler un système
+ * de type Kimi K3", 16.3: read the fixed state, compute the output, update the state; "L'attention
+ * hybride", "Le décompte": conv kernel 4, swish output gate, one dv-wide norm gain; "Les briques
+ * d'un réseau de neurones", 2. SiLU and 4. RMSNorm.)  It equals gdn_layer_fwd run one token at a
+ * time with the conv history carried, except that q, k, v stay in fp32 between the prologue and
+ * the recurrence (they never leave the chip).
+ *   q_raw, k_raw [N, Hk*dk]; v_raw, z [N, Hv*dv]                        (dtype)
+ *   hq_in, hk_in [N, 3, Hk*dk]; hv_in [N, 3, Hv*dv]                     (dtype) raw inputs of
+ *        the three previous tokens, oldest first (zeros for a fresh request)
+ *   hq_out, hk_out, hv_out: same shapes, written with the history after this token.  They must
+ *        not overlap the _in buffers (swap the two sets between steps).
+ *   wq, wk [Hk*dk, 4]; wv [Hv*dv, 4] float: conv taps, tap 3 on the current token
+ *   log_alpha, beta [N, Hv] float; S [N, Hv, dk, dv] float (S transposed per head), in place
+ *   norm_w [dv] float; y [N, Hv, dv] (dtype, output)
+ *   scale multiplies q; l2_eps is added under the L2 square root, norm_eps under the RMS one.
+ * dk, dv in {16, 32, 64, 128}.
+ */
+GDN_API gdn_status gdn_decode_layer_step(const void *q_raw, const void *k_raw, const void *v_raw,
+                                 const void *z, const void *hq_in, const void *hk_in,
+                                 const void *hv_in, void *hq_out, void *hk_out, void *hv_out,
+                                 const float *wq, const float *wk, const float *wv,
+                                 const float *log_alpha, const float *beta, float *S,
+                                 const float *norm_w, void *y, int N, int Hk, int Hv, int dk,
+                                 int dv, float scale, float l2_eps, float norm_eps,
+                                 gdn_dtype dtype, gdn_stream_t stream);
+
+/*
  * Layer prologue: causal depthwise convolution with 4 taps and no bias, then SiLU, on the q, k
  * and v channels; then each q and k head is divided by sqrt(sum of squares + l2_eps).
  * ("L'attention hybride", "Le décompte": conv kernel 4 over the q, k, v channels, 4 weights per

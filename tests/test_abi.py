@@ -27,8 +27,8 @@ def declared_functions():
 
 def test_header_declares_the_calls():
     names = declared_functions()
-    for must in ("gdn_prologue", "gdn_chunk_fwd", "gdn_decode_step", "gdn_out_norm",
-                 "gdn_layer_fwd", "gdn_status_string", "gdn_check_error"):
+    for must in ("gdn_prologue", "gdn_chunk_fwd", "gdn_decode_step", "gdn_decode_layer_step",
+                 "gdn_out_norm", "gdn_layer_fwd", "gdn_status_string", "gdn_check_error"):
         assert must in names
 
 
@@ -87,6 +87,20 @@ def test_decode_validation(L):
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 4, 2, 2, 16, 16, 1.0, 0, None) == 1
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 2, 24, 16, 1.0, 0, None) == 2
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, 2, 16, 16, 1.0, 0, None) == 0
+
+
+def test_decode_layer_validation(L):
+    f = L.gdn_decode_layer_step
+    t = [FAKE] * 18
+    assert f(*t, -1, 2, 2, 16, 16, 1.0, 1e-6, 1e-5, 1, None) == 1          # N < 0
+    assert f(*t, 4, 2, 3, 16, 16, 1.0, 1e-6, 1e-5, 1, None) == 1            # Hv % Hk
+    assert f(*t, 4, 2, 2, 24, 16, 1.0, 1e-6, 1e-5, 1, None) == 2            # unsupported dk
+    assert f(*t, 4, 2, 2, 16, 16, 1.0, -1e-6, 1e-5, 1, None) == 1           # eps < 0
+    for i in range(18):                                                     # each pointer
+        u = list(t)
+        u[i] = None
+        assert f(*u, 4, 2, 2, 16, 16, 1.0, 1e-6, 1e-5, 1, None) == 1, i
+    assert f(*t, 0, 2, 2, 16, 16, 1.0, 1e-6, 1e-5, 1, None) == 0            # nothing to do
 
 
 def test_prologue_and_out_norm_validation(L):

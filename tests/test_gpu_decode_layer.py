@@ -1,0 +1,93 @@
+"""The fused full-layer decode step (gdn_decode_layer_step) against the fp64 oracle's layer run
+one token at a time with the conv history carried, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import gdn_inputs as gi
+import gated_deltanet_linear_18_b200 as gdn
+from gpu_util import (TOL_BF16_OUT, TOL_BF16_STATE, TOL_F32_ABS, max_abs, np64, out_err,
+                      rel_rms, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(dtype, N=5, Hk=2, Hv=6, dk=128, dv=128, steps=3, seed=5):
+    w = gi.WORKLOADS["decode_layer"].with_sizes(B=N, Hk=Hk, Hv=Hv, dk=dk, dv=dv, steps=steps,
+                                                dtype=dtype, seed=seed)
+    return w, gi.make_decode_layer_inputs(w)
+
+
+def _run_gpu(w, x, steps=None, scale=1.0):
+    """Steps on the GPU with the two history sets swapped between steps.  Returns the outputs
+    [steps, N, Hv, dv], the final state and the final histories (host tensors)."""
+    d = to_dev(x)
+    S = d["S0"].clone()
+    hin = [d["hq"].clone(), d["hk"].clone(), d["hv"].clone()]
+    hout = [torch.empty_like(t) for t in hin]
+    ys = []
+    for s in range(steps or w.steps):
+        y = gdn.decode_layer_step(d["q_raw"][s], d["k_raw"][s], d["v_raw"][s], d["z"][s], *hin,
+                                  *hout, d["conv_wq"], d["conv_wk"], d["conv_wv"],
+                                  d["log_alpha"][s], d["beta"][s], S, d["norm_w"], Hk=w.Hk,
+                                  Hv=w.Hv, dk=w.dk, dv=w.dv, scale=scale)
+        ys.append(y)
+        hin, hout = hout, hin
+    torch.cuda.synchronize()
+    gdn.check_error()
+    return torch.stack(ys).cpu(), S.cpu(), [t.cpu() for t in hin]
+
+
+def _run_oracle(orc, w, x, steps=None, seqs=slice(None), scale=1.0):
+    s = slice(0, steps or w.steps)
+    return orc.decode_layer_steps(
+        x["q_raw"][s, seqs], x["k_raw"][s, seqs], x["v_raw"][s, seqs], x["z"][s, seqs],
+        x["hq"][seqs], x["hk"][seqs], x["hv"][seqs], x["conv_wq"], x["conv_wk"], x["conv_wv"],
+        x["log_alpha"][s, seqs], x["beta"][s, seqs], x["S0"][seqs], x["norm_w"], w.Hk, w.Hv,
+        w.dk, w.dv, l2_eps=w.l2_eps, norm_eps=w.norm_eps, scale=scale)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 32), (16, 16)])
+def test_decode_layer_steps_match_oracle(orc, dtype, dk, dv):
+    """Three steps, GQA 3:1, nonzero state and history: outputs of every step, the final state,
+    and the carried history (bit for bit)."""
+    w, x = _inputs(dtype, dk=dk, dv=dv)
+    y, S, h = _run_gpu(w, x, scale=0.7)
+    y_ref, S_ref, hq, hk, hv = _run_oracle(orc, w, x, scale=0.7)
+    for got, ref in zip(h, (hq, hk, hv)):
+        assert np.array_equal(np64(got), ref)
+    if dtype == "bf16":
+        assert out_err(y, y_ref) <= TOL_BF16_OUT, out_err(y, y_ref)
+        assert rel_rms(S, S_ref) <= TOL_BF16_STATE, rel_rms(S, S_ref)
+    else:
+        assert max_abs(y, y_ref) <= TOL_F32_ABS, max_abs(y, y_ref)
+        assert max_abs(S, S_ref) <= TOL_F32_ABS, max_abs(S, S_ref)
+
+
+def test_decode_layer_fresh_request_equals_layer_forward(orc):
+    """From a zero history and a zero state, T decode steps give the layer's outputs over the
+    T-token request (the full-layer oracle, fp32 activations)."""
+    w, x = _inputs("f32", N=3, Hk=2, Hv=6, dk=64, dv=64, steps=5, seed=9)
+    for key in ("hq", "hk", "hv"):
+        x[key] = torch.zeros_like(x[key])
+    x["S0"] = torch.zeros_like(x["S0"])
+    y, S, _ = _run_gpu(w, x)
+    tm = lambda a: np.swapaxes(np64(a), 0, 1)
+    y_ref, S_ref = orc.layer_forward(tm(x["q_raw"]), tm(x["k_raw"]), tm(x["v_raw"]), tm(x["z"]),
+                                     x["conv_wq"], x["conv_wk"], x["conv_wv"],
+                                     tm(x["log_alpha"]), tm(x["beta"]), None, x["norm_w"],
+                                     w.Hk, w.Hv, w.dk, w.dv)
+    assert max_abs(torch.from_numpy(tm(y)), y_ref) <= TOL_F32_ABS
+    assert max_abs(S, S_ref) <= TOL_F32_ABS
+
+
+def test_decode_layer_full_size_sampled(orc):
+    """The decode-layer workload's sizes (256 sequences, Hk16 Hv48 d128, bf16), two steps, the
+    oracle on a sample of sequences (the sequences are independent)."""
+    w, x = _inputs("bf16", N=256, Hk=16, Hv=48, steps=2, seed=5)
+    y, S, _ = _run_gpu(w, x)
+    seqs = [0, 77, 255]
+    y_ref, S_ref, _, _, _ = _run_oracle(orc, w, x, seqs=seqs)
+    assert out_err(y[:, seqs], y_ref) <= TOL_BF16_OUT
+    assert rel_rms(S[seqs], S_ref) <= TOL_BF16_STATE
