@@ -64,6 +64,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_decode_step.restype = I
         L.gdn_decode_layer_step.argtypes = [P] * 18 + [I] * 5 + [F, F, F, I, P]
         L.gdn_decode_layer_step.restype = I
+        L.gdn_wait_timeout_selftest.argtypes = [LL, P]
+        L.gdn_wait_timeout_selftest.restype = I
         L.gdn_prologue.argtypes = [P] * 9 + [I] * 6 + [F, I, P]
         L.gdn_prologue.restype = I
         L.gdn_out_norm.argtypes = [P, P, P, P, LL, I, F, I, P]

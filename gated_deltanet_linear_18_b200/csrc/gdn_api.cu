@@ -109,6 +109,22 @@ gdn_status decode_dispatch(int dk, int dv, const void* q, const void* k, const v
 }
 
 // ---------------------------------------------------------------------------------------------
+// Failure-detection self-test: one thread waits on a barrier that nothing completes
+// ---------------------------------------------------------------------------------------------
+__global__ void wait_timeout_selftest_kernel(unsigned long long budget) {
+  __shared__ __align__(8) unsigned long long bar;
+  __shared__ int abort_word;
+  if (threadIdx.x == 0) {
+    const uint32_t b = tc::smem_u32(&bar);
+    tc::mbar_init(b, 1);                  // phase 0 needs one arrive; none comes
+    tc::fence_barrier_init();
+    abort_word = 0;
+    volatile int* abort_flag = &abort_word;
+    if (!tc::mbar_wait(b, 0, abort_flag, budget)) record_error(kErrTimeout);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
 // Full-layer decode step dispatch over (dk, dv)
 // ---------------------------------------------------------------------------------------------
 struct DecodeLayerArgs {
@@ -231,6 +247,13 @@ gdn_status gdn_check_error(gdn_stream_t stream) {
   if (word != 0 && cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess)
     return GDN_ERR_CUDA;
   return (word & kErrTimeout) ? GDN_ERR_TIMEOUT : GDN_OK;
+}
+
+gdn_status gdn_wait_timeout_selftest(long long budget_cycles, gdn_stream_t stream) {
+  if (budget_cycles < 1 || budget_cycles > 4000000000LL) return GDN_ERR_INVALID_ARG;
+  wait_timeout_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      (unsigned long long)budget_cycles);
+  return launch_status();
 }
 
 gdn_variant gdn_chunk_fwd_variant(int dk, int dv, int chunk, gdn_dtype dtype) {

@@ -86,6 +86,17 @@ GDN_API int gdn_version(void);
 GDN_API gdn_status gdn_check_error(gdn_stream_t stream);
 
 /*
+ * Failure-detection self-test (no fault, no hang): enqueues one single-thread kernel that waits,
+ * with the same bounded wait the kernels use, on a barrier that nothing completes.  After
+ * `budget_cycles` SM clock cycles (1 .. 4e9, about 2 s at most) the wait gives up, the kernel
+ * records the timeout bit and returns, so the next gdn_check_error on the stream reports
+ * GDN_ERR_TIMEOUT (once: the call clears the bit) and the context stays usable.  This library's
+ * own check that a wait which runs out is reported; the pages have no counterpart.
+ *   GDN_ERR_INVALID_ARG for a budget out of range (nothing enqueued).
+ */
+GDN_API gdn_status gdn_wait_timeout_selftest(long long budget_cycles, gdn_stream_t stream);
+
+/*
  * Chunked prefill forward ("Chapitre 16 - Assembler un système de type Kimi K3", 16.2: each block
  * of `chunk` tokens is processed with matrix operations and the state is handed to the next
  * block).  Computes o for all T tokens and the state after token T-1.

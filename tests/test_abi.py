@@ -103,6 +103,12 @@ def test_decode_layer_validation(L):
     assert f(*t, 0, 2, 2, 16, 16, 1.0, 1e-6, 1e-5, 1, None) == 0            # nothing to do
 
 
+def test_wait_selftest_validation(L):
+    assert L.gdn_wait_timeout_selftest(0, None) == 1
+    assert L.gdn_wait_timeout_selftest(-5, None) == 1
+    assert L.gdn_wait_timeout_selftest(5_000_000_000, None) == 1
+
+
 def test_prologue_and_out_norm_validation(L):
     assert L.gdn_prologue(*([FAKE] * 9), 1, 8, 2, 4, 16, 16, -1.0, 1, None) == 1   # eps < 0
     assert L.gdn_prologue(*([FAKE] * 8), None, 1, 8, 2, 4, 16, 16, 1e-6, 1, None) == 1
