@@ -312,6 +312,22 @@ def bench_decode_layer(gdn, dev, warmup, flush, peaks):
             "bytes_per_step": by, "workload": workload_name(w)}
 
 
+def bench_gates(gdn, dev, warmup, flush, peaks, steps=20):
+    """Gates from the in_proj_ba outputs on the prefill shape (B4 T2048, 48 value heads, bf16)."""
+    w = gi.WORKLOADS["prefill"]
+    g = torch.Generator().manual_seed(11)
+    ba = (torch.randn(w.B, w.T, 2 * w.Hv, generator=g) * 2.0).to(w.torch_dtype).to(dev)
+
+    def step():
+        gdn.gates(ba, w.Hv)
+    ms = time_steps(step, steps, warmup, flush, 1)
+    t = sum(ms) / len(ms) / 1e3
+    by = w.B * w.T * w.Hv * (2 * ba.element_size() + 2 * 4)
+    return {"value": by / t / 1e9, "unit": "GB/s", "us_per_call": t * 1e6,
+            "roofline_frac": by / t / 1e9 / peaks["hbm_gbs"], "bytes_per_call": by,
+            "workload": f"gates B{w.B} T{w.T} Hv{w.Hv} {w.dtype}"}
+
+
 def bench_layer(gdn, dev, warmup, flush, peaks, steps=3):
     w = gi.WORKLOADS["layer_8to1"]
     x = gi.make_layer_inputs(w)
@@ -582,6 +598,7 @@ def main():
             sec = {}
             sec["decode"] = bench_decode(gdn, dev, args.warmup, flush, peaks)
             sec["decode_layer"] = bench_decode_layer(gdn, dev, args.warmup, flush, peaks)
+            sec["gates"] = bench_gates(gdn, dev, args.warmup, flush, peaks)
             del d
             torch.cuda.empty_cache()
             _, xl, dl, _, sec["long_context"] = bench_prefill_like(

@@ -64,6 +64,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_decode_step.restype = I
         L.gdn_decode_layer_step.argtypes = [P] * 18 + [I] * 5 + [F, F, F, I, P]
         L.gdn_decode_layer_step.restype = I
+        L.gdn_gates.argtypes = [P, P, P, LL, I, I, P]
+        L.gdn_gates.restype = I
         L.gdn_wait_timeout_selftest.argtypes = [LL, P]
         L.gdn_wait_timeout_selftest.restype = I
         L.gdn_prologue.argtypes = [P] * 9 + [I] * 6 + [F, I, P]
@@ -198,6 +200,22 @@ def decode_layer_step(q_raw, k_raw, v_raw, z, hq_in, hk_in, hv_in, hq_out, hk_ou
             _io_dtype(q_raw), _stream(dev))
     _check("gdn_decode_layer_step", st)
     return y
+
+
+def gates(ba, Hv: int) -> Tuple[torch.Tensor, torch.Tensor]:
+    """in_proj_ba outputs [..., 2*Hv] (b then a) -> (log_alpha, beta) [..., Hv] fp32:
+    beta = sigmoid(b), log alpha = -softplus(-a)."""
+    if ba.shape[-1] != 2 * Hv:
+        raise ValueError("ba must end in 2*Hv values")
+    rows = ba.numel() // (2 * Hv)
+    log_alpha = torch.empty(ba.shape[:-1] + (Hv,), device=ba.device, dtype=torch.float32)
+    beta = torch.empty_like(log_alpha)
+    dev = _dev(ba, log_alpha, beta)
+    with torch.cuda.device(dev):
+        st = lib().gdn_gates(_p(ba), _p(log_alpha), _p(beta), rows, Hv, _io_dtype(ba),
+                             _stream(dev))
+    _check("gdn_gates", st)
+    return log_alpha, beta
 
 
 def prologue(q_raw, k_raw, v_raw, wq, wk, wv, Hk: int, Hv: int, dk: int, dv: int,

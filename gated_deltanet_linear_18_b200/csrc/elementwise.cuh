@@ -172,4 +172,20 @@ out_norm_kernel(const To* __restrict__ o, const Tio* __restrict__ z, const float
   }
 }
 
+// Gates from the in_proj_ba outputs: beta = sigmoid(b), log alpha = -softplus(-a), one thread per
+// (token, value head); rows of 2 Hv inputs and Hv outputs, so both sides are read and written
+// contiguously across the threads of a warp.
+template <typename Tin>
+__global__ void gates_kernel(const Tin* __restrict__ ba, float* __restrict__ log_alpha,
+                             float* __restrict__ beta, long long rows, int Hv) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= rows * Hv) return;
+  const long long r = i / Hv;
+  const int h = (int)(i - r * Hv);
+  const float b = to_f(ba[r * 2 * Hv + h]), a = to_f(ba[r * 2 * Hv + Hv + h]);
+  beta[i] = 1.0f / (1.0f + expf(-b));
+  // -softplus(-a), written so that neither branch overflows
+  log_alpha[i] = a >= 0.f ? -log1pf(expf(-a)) : a - log1pf(expf(a));
+}
+
 }  // namespace gdn

@@ -249,6 +249,25 @@ gdn_status gdn_check_error(gdn_stream_t stream) {
   return (word & kErrTimeout) ? GDN_ERR_TIMEOUT : GDN_OK;
 }
 
+gdn_status gdn_gates(const void* ba, float* log_alpha, float* beta, long long rows, int Hv,
+                     gdn_dtype dtype, gdn_stream_t stream) {
+  if (rows < 0 || Hv <= 0 || !valid_dtype(dtype)) return GDN_ERR_INVALID_ARG;
+  if (rows == 0) return GDN_OK;
+  if (!ba || !log_alpha || !beta || !aligned16(ba) || !aligned4(log_alpha) || !aligned4(beta))
+    return GDN_ERR_INVALID_ARG;
+  const long long n = rows * Hv;
+  if (n / Hv != rows || (n + 255) / 256 > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const unsigned grid = (unsigned)((n + 255) / 256);
+  if (dtype == GDN_F32)
+    gates_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(ba), log_alpha, beta,
+                                              rows, Hv);
+  else
+    gates_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(ba),
+                                                      log_alpha, beta, rows, Hv);
+  return launch_status();
+}
+
 gdn_status gdn_wait_timeout_selftest(long long budget_cycles, gdn_stream_t stream) {
   if (budget_cycles < 1 || budget_cycles > 4000000000LL) return GDN_ERR_INVALID_ARG;
   wait_timeout_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(

@@ -173,6 +173,19 @@ GDN_API gdn_status gdn_decode_layer_step(const void *q_raw, const void *k_raw, c
                                  gdn_dtype dtype, gdn_stream_t stream);
 
 /*
+ * Gates from the in_proj_ba outputs, per (token, value head): beta = sigmoid(b) and
+ * log_alpha = log sigmoid(a) = -softplus(-a).  ("L'attention hybride", "Le décompte": in_proj_ba
+ * makes one beta and one alpha per value head and the layer counts no other gate parameter;
+ * "La récurrence": alpha, beta in ]0,1[; "Les briques d'un réseau de neurones", 2.: the sigmoid
+ * is the gate, softplus is log(1 + e^x).  The pages give no other parameterisation of alpha;
+ * this is the plainest one that fits them.)
+ *   ba [rows, 2*Hv] (dtype): the Hv b values, then the Hv a values, of each token
+ *   log_alpha, beta [rows, Hv] float (outputs, the gates gdn_chunk_fwd and gdn_layer_fwd take)
+ */
+GDN_API gdn_status gdn_gates(const void *ba, float *log_alpha, float *beta, long long rows, int Hv,
+                     gdn_dtype dtype, gdn_stream_t stream);
+
+/*
  * Layer prologue: causal depthwise convolution with 4 taps and no bias, then SiLU, on the q, k
  * and v channels; then each q and k head is divided by sqrt(sum of squares + l2_eps).
  * ("L'attention hybride", "Le décompte": conv kernel 4 over the q, k, v channels, 4 weights per

@@ -23,6 +23,10 @@ Functions and the passages they follow (page titles; the C file's header has the
                             activation of the model but the state is BF16 ("L'attention
                             hybride", "Le float32 n'est pas un détail").
   * ``round_bf16``        — that rounding, written from the bf16 format (8 significant bits).
+  * ``gates``             — (log alpha, beta) from the in_proj_ba outputs: beta = sigmoid(b),
+                            alpha = sigmoid(a) ("L'attention hybride", "Le décompte": one beta
+                            and one alpha per value head and no other gate parameter; "Les
+                            briques d'un réseau de neurones", 2.: sigmoid as the gate, softplus).
   * ``decode_layer_steps`` — the layer one token at a time ("Chapitre 16 ... Kimi K3", 16.3) with
                             the conv's three-token history carried between steps: the composition
                             above on [history; token].  Pinned by equality with ``layer_forward``
@@ -115,6 +119,8 @@ class OracleLib:
         lib.oracle_l2_normalize.restype = None
         lib.oracle_gated_rmsnorm.argtypes = [P, P, P, P, L, I, D]
         lib.oracle_gated_rmsnorm.restype = None
+        lib.oracle_gates.argtypes = [P, P, P, L, I]
+        lib.oracle_gates.restype = None
         self.lib = lib
         self.path = path
 
@@ -184,6 +190,17 @@ class OracleLib:
         self.lib.oracle_gated_rmsnorm(_ptr(o), _ptr(z), _ptr(w), _ptr(y), o.size // d, d,
                                       float(eps))
         return y
+
+    def gates(self, ba, Hv: int) -> Tuple[np.ndarray, np.ndarray]:
+        """in_proj_ba outputs [..., 2*Hv] (b then a) -> (log_alpha, beta) [..., Hv]:
+        beta = sigmoid(b), log alpha = -softplus(-a) (alpha = sigmoid(a))."""
+        ba = _f64(ba)
+        assert ba.shape[-1] == 2 * Hv
+        rows = ba.size // (2 * Hv)
+        la = np.zeros(ba.shape[:-1] + (Hv,))
+        be = np.zeros_like(la)
+        self.lib.oracle_gates(_ptr(ba), _ptr(la), _ptr(be), rows, Hv)
+        return la, be
 
     def prologue(self, q_raw, k_raw, v_raw, wq, wk, wv, Hk: int, Hv: int, dk: int, dv: int,
                  l2_eps: float):
@@ -289,3 +306,7 @@ def layer_forward(*a, **kw):
 
 def decode_layer_steps(*a, **kw):
     return get().decode_layer_steps(*a, **kw)
+
+
+def gates(*a, **kw):
+    return get().gates(*a, **kw)

@@ -199,3 +199,22 @@ void oracle_gated_rmsnorm(const double *o, const double *z, const double *w, dou
         }
     }
 }
+
+/*
+ * Gates of one (token, value head) from the in_proj_ba outputs ([HYB] Le décompte: in_proj_ba
+ * makes one beta and one alpha per value head, 2 x 48 outputs, and no other gate parameter is
+ * counted; [BRK] 2.: the sigmoid is the gate that squashes into (0, 1), softplus is
+ * log(1 + e^x)).  Reading: beta = sigmoid(b), alpha = sigmoid(a), so log alpha = -softplus(-a).
+ * ba: [rows, 2 * Hv], the Hv b values then the Hv a values; log_alpha, beta: [rows, Hv].
+ */
+static double softplus(double x) { return x > 0.0 ? x + log1p(exp(-x)) : log1p(exp(x)); }
+
+void oracle_gates(const double *ba, double *log_alpha, double *beta, long rows, int Hv)
+{
+    for (long r = 0; r < rows; ++r)
+        for (int h = 0; h < Hv; ++h) {
+            const double b = ba[r * 2 * Hv + h], a = ba[r * 2 * Hv + Hv + h];
+            beta[r * Hv + h] = sigmoid(b);
+            log_alpha[r * Hv + h] = -softplus(-a);
+        }
+}

@@ -344,4 +344,31 @@ def pin_decode_layer_history_is_the_three_previous_tokens(orc):
     assert np.allclose(sS, sT, rtol=1e-12, atol=1e-12)
 
 
+# ---------------------------------------------------------------------------------------------
+# gates from the in_proj_ba outputs
+# ---------------------------------------------------------------------------------------------
+def pin_gates_match_library_sigmoid(orc):
+    """beta = sigmoid(b) and log alpha = log sigmoid(a) equal scipy's expit and log_expit, over
+    a wide range (|x| up to 60, where the naive forms lose everything), with b first in the row."""
+    from scipy.special import log_expit
+    rng = np.random.default_rng(21)
+    Hv = 5
+    ba = rng.standard_normal((7, 3, 2 * Hv)) * np.exp2(rng.integers(-4, 6, (7, 3, 2 * Hv)))
+    la, be = orc.gates(ba, Hv)
+    assert np.allclose(be, expit(ba[..., :Hv]), rtol=1e-13, atol=0)
+    assert np.allclose(la, log_expit(ba[..., Hv:]), rtol=1e-13, atol=1e-300)
+
+
+def pin_gates_closed_forms(orc):
+    """alpha in (0, 1) and alpha(a) + alpha(-a) = 1; a = 0 gives alpha = beta = 1/2."""
+    x = np.linspace(-30, 30, 121)
+    ba = np.stack([np.zeros_like(x), x], axis=-1)               # Hv = 1: b = 0, a = x
+    la, be = orc.gates(ba, 1)
+    lam, _ = orc.gates(np.stack([np.zeros_like(x), -x], axis=-1), 1)
+    a = np.exp(la[:, 0])
+    assert np.all((a > 0) & (a < 1)) and np.allclose(be, 0.5)
+    assert np.allclose(a + np.exp(lam[:, 0]), 1.0, rtol=0, atol=1e-15)
+    assert np.isclose(np.exp(la[60, 0]), 0.5)
+
+
 ALL_PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]

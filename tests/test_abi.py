@@ -103,6 +103,15 @@ def test_decode_layer_validation(L):
     assert f(*t, 0, 2, 2, 16, 16, 1.0, 1e-6, 1e-5, 1, None) == 0            # nothing to do
 
 
+def test_gates_validation(L):
+    assert L.gdn_gates(FAKE, FAKE, FAKE, -1, 48, 1, None) == 1
+    assert L.gdn_gates(FAKE, FAKE, FAKE, 10, 0, 1, None) == 1
+    assert L.gdn_gates(None, FAKE, FAKE, 10, 48, 1, None) == 1
+    assert L.gdn_gates(FAKE, FAKE, None, 10, 48, 1, None) == 1
+    assert L.gdn_gates(FAKE, FAKE, FAKE, 10, 48, 7, None) == 1         # dtype
+    assert L.gdn_gates(FAKE, FAKE, FAKE, 0, 48, 1, None) == 0
+
+
 def test_wait_selftest_validation(L):
     assert L.gdn_wait_timeout_selftest(0, None) == 1
     assert L.gdn_wait_timeout_selftest(-5, None) == 1
