@@ -312,6 +312,34 @@ def bench_decode_layer(gdn, dev, warmup, flush, peaks):
             "bytes_per_step": by, "workload": workload_name(w)}
 
 
+def bench_varlen(gdn, dev, warmup, flush, peaks, steps=10):
+    """Packed prefill of 32 requests of seeded lengths U[64, 1024] (the prefill heads, bf16),
+    each from a nonzero state: the serving form of the chunked forward."""
+    w = gi.WORKLOADS["prefill"]
+    g = torch.Generator().manual_seed(12)
+    lengths = torch.randint(64, 1025, (32,), generator=g)
+    total = int(lengths.sum())
+    unit = lambda x: x / torch.linalg.vector_norm(x, dim=-1, keepdim=True)
+    q = unit(torch.randn(total, w.Hk, w.dk, generator=g)).to(w.torch_dtype).to(dev)
+    k = unit(torch.randn(total, w.Hk, w.dk, generator=g)).to(w.torch_dtype).to(dev)
+    v = torch.randn(total, w.Hv, w.dv, generator=g).to(w.torch_dtype).to(dev)
+    la = (-torch.nn.functional.softplus(torch.randn(total, w.Hv, generator=g))
+          * torch.exp(torch.rand(total, w.Hv, generator=g) * 4.0 - 5.0)).to(dev)
+    be = torch.sigmoid(torch.randn(total, w.Hv, generator=g)).to(dev)
+    S0 = (torch.randn(32, w.Hv, w.dk, w.dv, generator=g) * 0.02).to(dev)
+    cu = torch.cat([torch.zeros(1, dtype=torch.int64), lengths.cumsum(0)]).to(torch.int32).to(dev)
+    o = torch.empty_like(v)
+
+    def step():
+        gdn.chunk_fwd_varlen(q, k, v, la, be, cu, int(lengths.max()), S0, out=o)
+    ms = time_steps(step, steps, warmup, flush, 2)
+    gdn.check_error(dev)
+    t = sum(ms) / len(ms) / 1e3
+    return {"value": total / t, "unit": "tokens/s", "ms_per_call": t * 1e3, "tokens": total,
+            "requests": 32, "workload": f"varlen 32 requests U[64,1024] ({total} tokens) "
+            f"Hk{w.Hk} Hv{w.Hv} dk{w.dk} dv{w.dv} chunk{w.chunk} {w.dtype} S0~N(0,0.02)"}
+
+
 def bench_gates(gdn, dev, warmup, flush, peaks, steps=20):
     """Gates from the in_proj_ba outputs on the prefill shape (B4 T2048, 48 value heads, bf16)."""
     w = gi.WORKLOADS["prefill"]
@@ -599,6 +627,7 @@ def main():
             sec["decode"] = bench_decode(gdn, dev, args.warmup, flush, peaks)
             sec["decode_layer"] = bench_decode_layer(gdn, dev, args.warmup, flush, peaks)
             sec["gates"] = bench_gates(gdn, dev, args.warmup, flush, peaks)
+            sec["varlen"] = bench_varlen(gdn, dev, args.warmup, flush, peaks)
             del d
             torch.cuda.empty_cache()
             _, xl, dl, _, sec["long_context"] = bench_prefill_like(

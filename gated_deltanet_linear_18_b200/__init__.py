@@ -64,6 +64,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_decode_step.restype = I
         L.gdn_decode_layer_step.argtypes = [P] * 18 + [I] * 5 + [F, F, F, I, P]
         L.gdn_decode_layer_step.restype = I
+        L.gdn_chunk_fwd_varlen.argtypes = [P] * 6 + [I, I] + [P] * 3 + [I] * 6 + [F, I, P]
+        L.gdn_chunk_fwd_varlen.restype = I
         L.gdn_gates.argtypes = [P, P, P, LL, I, I, P]
         L.gdn_gates.restype = I
         L.gdn_wait_timeout_selftest.argtypes = [LL, P]
@@ -200,6 +202,32 @@ def decode_layer_step(q_raw, k_raw, v_raw, z, hq_in, hk_in, hv_in, hq_out, hk_ou
             _io_dtype(q_raw), _stream(dev))
     _check("gdn_decode_layer_step", st)
     return y
+
+
+def chunk_fwd_varlen(q, k, v, log_alpha, beta, cu_seqlens, max_seqlen: int, S0=None, *,
+                     chunk: int = 64, scale: float = 1.0, out: Optional[torch.Tensor] = None,
+                     want_state: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Packed sequences: q,k [total,Hk,dk]; v [total,Hv,dv]; gates [total,Hv]; cu_seqlens
+    [nseq+1] int32 on the device; S0 [nseq,Hv,dk,dv] or None.  Returns (o [total,Hv,dv],
+    S_T [nseq,Hv,dk,dv] or None)."""
+    total, Hk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    nseq = cu_seqlens.numel() - 1
+    if (k.shape != q.shape or v.shape[0] != total or log_alpha.shape != (total, Hv)
+            or beta.shape != log_alpha.shape or cu_seqlens.dtype != torch.int32 or nseq < 0):
+        raise ValueError("packed shapes disagree")
+    _f32(log_alpha, beta)
+    o = torch.empty_like(v) if out is None else out
+    sT = (torch.empty(nseq, Hv, dk, dv, device=q.device, dtype=torch.float32)
+          if want_state else None)
+    dev = _dev(q, k, v, log_alpha, beta, cu_seqlens, o)
+    with torch.cuda.device(dev):
+        st = lib().gdn_chunk_fwd_varlen(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta),
+                                        _p(cu_seqlens), nseq, int(max_seqlen), _p(S0), _p(o),
+                                        _p(sT), total, Hk, Hv, dk, dv, chunk, float(scale),
+                                        _io_dtype(q), _stream(dev))
+    _check("gdn_chunk_fwd_varlen", st)
+    return o, sT
 
 
 def gates(ba, Hv: int) -> Tuple[torch.Tensor, torch.Tensor]:

@@ -249,6 +249,46 @@ gdn_status gdn_check_error(gdn_stream_t stream) {
   return (word & kErrTimeout) ? GDN_ERR_TIMEOUT : GDN_OK;
 }
 
+gdn_status gdn_chunk_fwd_varlen(const void* q, const void* k, const void* v,
+                                const float* log_alpha, const float* beta, const int* cu_seqlens,
+                                int nseq, int max_seqlen, const float* S0, void* o, float* S_T,
+                                int total_T, int Hk, int Hv, int dk, int dv, int chunk,
+                                float scale, gdn_dtype dtype, gdn_stream_t stream) {
+  if (nseq < 0 || max_seqlen < 0 || total_T < 0 || !valid_dtype(dtype))
+    return GDN_ERR_INVALID_ARG;
+  gdn_status s = validate_heads(Hk, Hv, dk, dv);
+  if (s != GDN_OK) return s;
+  if (chunk <= 0) return GDN_ERR_INVALID_ARG;
+  if (!tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16)) return GDN_ERR_UNSUPPORTED;
+  if (nseq > 65535) return GDN_ERR_UNSUPPORTED;
+  if (nseq == 0) return GDN_OK;
+  if (!cu_seqlens || !aligned4(cu_seqlens) || !opt_aligned16(S0) || !opt_aligned16(S_T))
+    return GDN_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (total_T == 0 || max_seqlen == 0) {   // every sequence is empty: the states pass through
+    if (!S_T) return GDN_OK;
+    const size_t bytes = (size_t)nseq * Hv * dk * dv * sizeof(float);
+    cudaError_t e = S0 ? cudaMemcpyAsync(S_T, S0, bytes, cudaMemcpyDeviceToDevice, st)
+                       : cudaMemsetAsync(S_T, 0, bytes, st);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+  }
+  if (!q || !k || !v || !log_alpha || !beta || !o) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(log_alpha) ||
+      !aligned4(beta))
+    return GDN_ERR_INVALID_ARG;
+  cudaMemPool_t pool = nullptr;
+  s = scratch_pool(&pool);
+  if (s != GDN_OK) return s;
+  void* scratch = nullptr;
+  if (cudaMallocFromPoolAsync(&scratch, tc_chunk_varlen_scratch_bytes(nseq, max_seqlen, Hv), pool,
+                              st) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  s = tc_chunk_launch_varlen(q, k, v, log_alpha, beta, cu_seqlens, nseq, max_seqlen, S0, o, S_T,
+                             total_T, Hk, Hv, scale, scratch, st);
+  const cudaError_t e = cudaFreeAsync(scratch, st);   // ordered after the kernels
+  return s != GDN_OK ? s : (e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA);
+}
+
 gdn_status gdn_gates(const void* ba, float* log_alpha, float* beta, long long rows, int Hv,
                      gdn_dtype dtype, gdn_stream_t stream) {
   if (rows < 0 || Hv <= 0 || !valid_dtype(dtype)) return GDN_ERR_INVALID_ARG;

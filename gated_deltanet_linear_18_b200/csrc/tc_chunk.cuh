@@ -372,6 +372,25 @@ __device__ __forceinline__ void st_split8(uint32_t hi_addr, uint32_t lo_addr, co
 }
 
 // ------------------------------------------------------------------------------------------
+// Where sequence s lives.  Fixed length (cu == nullptr): batch s of [B, T, ...] tensors.  Packed
+// (cu != nullptr): tokens cu[s] .. cu[s + 1] - 1 of [1, T, ...] tensors (T = total tokens); the
+// offsets come from device memory, so they are clamped to the tensor and the length to max_len,
+// which keeps every access in bounds whatever they hold.
+// ------------------------------------------------------------------------------------------
+struct SeqSpan {
+  int tok0;      // first token in the tensor map's token dimension
+  int len;       // tokens of the sequence
+  int bcoord;    // tensor map batch coordinate
+  long row0;     // row of the first token in [rows, heads, d] tensors and [rows, heads] gates
+};
+__device__ __forceinline__ SeqSpan seq_span(const int* __restrict__ cu, int s, int T, int max_len) {
+  if (!cu) return SeqSpan{0, T, s, (long)s * T};
+  const int a = min(max(cu[s], 0), T);
+  const int b = min(max(cu[s + 1], a), min(T, a + max_len));
+  return SeqSpan{a, b - a, 0, (long)a};
+}
+
+// ------------------------------------------------------------------------------------------
 // pre-pass: the state-independent operands of every (batch, value head, chunk), independently
 // ------------------------------------------------------------------------------------------
 // With T_b = (I + A)^-1 diag(beta), P = lower_incl(exp(G_i - G_j) q_i.k_j) scale and
@@ -420,17 +439,22 @@ __device__ __forceinline__ void store_tb_pair(uint32_t tb, int row, int n, float
   tc::sts1(o + 24576, __uint_as_float(kl));
 }
 
-// grid (nC, Hv, B), 128 threads; thread r owns TMEM lane r.
+// grid (nCmax, Hv, sequences), 128 threads; thread r owns TMEM lane r.  CTAs past the end of
+// their sequence return at once.
 __global__ void __launch_bounds__(PP_THREADS, 3)
 pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const float* __restrict__ log_alpha, const float* __restrict__ beta,
-                  uint8_t* __restrict__ pw, int T, int Hk, int Hv, float scale) {
+                  uint8_t* __restrict__ pw, int T, int Hk, int Hv, float scale,
+                  const int* __restrict__ cu, int max_len) {
   GDN_TRACE_INIT;
   extern __shared__ __align__(1024) uint8_t pp_raw[];
   uint8_t* smem = pp_raw + ((1024u - (tc::smem_u32(pp_raw) & 1023u)) & 1023u);
   const uint32_t sb = tc::smem_u32(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int c = blockIdx.x, h = blockIdx.y, bq = blockIdx.z, nC = gridDim.x;
+  const int c = blockIdx.x, h = blockIdx.y, sq = blockIdx.z, nC = gridDim.x;
+  const SeqSpan sp = seq_span(cu, sq, T, max_len);
+  if (c * C >= sp.len) return;                        // (uniform: before any barrier)
+  const int vrows = min(C, sp.len - c * C);           // tokens of this chunk in the sequence
   const int hk = h / (Hv / Hk);
   const long t0 = (long)c * C;
   float* gG = reinterpret_cast<float*>(smem + PP_G);
@@ -440,7 +464,7 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gG + 193);
   const uint32_t tma_bar = sb + PP_BAR, mma_bar = sb + PP_BAR + 8, pt_bar = sb + PP_BAR + 24;
   const uint32_t qk = sb + PP_QK, tb = sb + PP_TB;
-  uint8_t* rec = pw + (((long)bq * Hv + h) * nC + c) * (long)kPwBytes;
+  uint8_t* rec = pw + (((long)sq * Hv + h) * nC + c) * (long)kPwBytes;
 
   if (tid == 0) {
     tc::mbar_init(tma_bar, 1);
@@ -462,16 +486,17 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
   GDN_TRACE_PP(1);
   if (tid == 0) {
     tc::mbar_arrive_expect_tx(tma_bar, 32768);
-    tc::tma_load_4d(qk, &tmq, tma_bar, 0, hk, (int)t0, bq);
-    tc::tma_load_4d(qk + 8192, &tmk, tma_bar, 0, hk, (int)t0, bq);
-    tc::tma_load_4d(qk + 16384, &tmq, tma_bar, 64, hk, (int)t0, bq);
-    tc::tma_load_4d(qk + 24576, &tmk, tma_bar, 64, hk, (int)t0, bq);
+    const int tc0 = sp.tok0 + (int)t0;
+    tc::tma_load_4d(qk, &tmq, tma_bar, 0, hk, tc0, sp.bcoord);
+    tc::tma_load_4d(qk + 8192, &tmk, tma_bar, 0, hk, tc0, sp.bcoord);
+    tc::tma_load_4d(qk + 16384, &tmq, tma_bar, 64, hk, tc0, sp.bcoord);
+    tc::tma_load_4d(qk + 24576, &tmk, tma_bar, 64, hk, tc0, sp.bcoord);
   }
   // gates: G' = cumsum(log alpha) log2(e) over the chunk, beta, ktil, gamma (zero / flat past T)
   if (tid < 64) {
     const long tt = t0 + tid;
-    const float la = tt < T ? log_alpha[((long)bq * T + tt) * Hv + h] : 0.f;
-    gB[tid] = tt < T ? beta[((long)bq * T + tt) * Hv + h] : 0.f;
+    const float la = tt < sp.len ? log_alpha[(sp.row0 + tt) * Hv + h] : 0.f;
+    gB[tid] = tt < sp.len ? beta[(sp.row0 + tt) * Hv + h] : 0.f;
     float incl = la;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
@@ -494,9 +519,20 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     for (int b = 1; b < 4; ++b) gE[64 * b + tid] = tid < 16 * b ? tc::ex2(gG[16 * b] - gG[tid]) : 0.f;
   }
 
-  // S = [Q; K] K^T into TMEM columns 0..63
+  // S = [Q; K] K^T into TMEM columns 0..63.  Rows of the tile past the sequence's end (the next
+  // packed sequence's tokens) are zeroed first, so they reach no product.
+  const bool tile_ok = tc::mbar_wait(tma_bar, 0, abort_flag, kBudget);
+  if (vrows < C) {
+    for (int i = tid; i < 4 * (C - vrows) * 8; i += PP_THREADS) {
+      const int box = i / ((C - vrows) * 8), rem = i - box * (C - vrows) * 8;
+      tc::st_shared_v4(qk + box * 8192 + (vrows + (rem >> 3)) * 128 + (rem & 7) * 16, 0u, 0u, 0u,
+                       0u);
+    }
+    tc::fence_proxy_async_smem();
+  }
+  __syncthreads();                                    // gates visible, tile complete
   if (tid == 0) {
-    if (tc::mbar_wait(tma_bar, 0, abort_flag, kBudget)) {
+    if (tile_ok) {
       GDN_TRACE_PP(2);
       tc::tc_fence_after();
       const uint64_t dq = tc::sdesc_sw128(qk, 16, 1024);
@@ -508,7 +544,6 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     }
     tc::mma_commit(mma_bar);
   }
-  __syncthreads();                                    // gates visible
   tc::mbar_wait(mma_bar, 0, abort_flag, kBudget);
   GDN_TRACE_PP(3);
   tc::tc_fence_after();
@@ -705,7 +740,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmo, const __nv_bfloat16* __restrict__ v,
                     const uint8_t* __restrict__ pw, const float* __restrict__ S0,
-                    float* __restrict__ S_T, int T, int Hk, int Hv, float scale) {
+                    float* __restrict__ S_T, int T, int Hk, int Hv, float scale,
+                    const int* __restrict__ cu, int max_len, int nCmax, Tout* __restrict__ o) {
   constexpr bool kF32 = sizeof(Tout) == 4;
   // X takes M as a hi + lo bf16 pair when o is fp32 (the layer, whose gated norm magnifies o's
   // error); a bf16 o carries its own rounding, and one round-to-nearest bf16 copy of M suffices.
@@ -719,11 +755,21 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.x % Hv;
-  const int bq = blockIdx.x / Hv;
+  const int bq = blockIdx.x / Hv;                    // the sequence
   const int hk = h / (Hv / Hk);
-  const int nC = (T + C - 1) / C;
+  const SeqSpan sp = seq_span(cu, bq, T, max_len);
+  const int nC = (sp.len + C - 1) / C;
+  const bool packed = cu != nullptr;
   const long head = (long)bq * Hv + h;
-  const uint8_t* pw_head = pw + head * nC * (long)kPwBytes;
+  const uint8_t* pw_head = pw + head * nCmax * (long)kPwBytes;
+  if (nC == 0) {   // an empty sequence: the state passes through (uniform, before any barrier)
+    if (S_T)
+      for (int i = threadIdx.x; i < 128 * 128 / 4; i += blockDim.x)
+        reinterpret_cast<float4*>(S_T + head * 128 * 128)[i] =
+            S0 ? reinterpret_cast<const float4*>(S0 + head * 128 * 128)[i]
+               : make_float4(0.f, 0.f, 0.f, 0.f);
+    return;
+  }
   auto bar = [&](int i) -> uint32_t { return sb + OFF_BAR + 8u * i; };
 
   if (threadIdx.x == 0) {
@@ -762,16 +808,16 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       int armed_qk = -1, armed_w[2] = {-1, -1}, armed_p[2] = {-1, -1};
       bool ok = true;
       for (int c = 0; c < nC && ok; ++c) {
-        const int s = c & 1, t0 = c * C;
+        const int s = c & 1, t0 = sp.tok0 + c * C;
         // one Q/K stage: chunk c's tile is loaded as soon as X of chunk c - 1 has read the last
         if (c >= 1) ok = tc::mbar_wait(bar(B_QK_EMPTY), (c - 1) & 1, abort_flag, kBudget);
         if (!ok) break;
         const uint32_t dst = sb + OFF_QK;
         tc::mbar_arrive_expect_tx(bar(B_QK_FULL), 32768);
-        tc::tma_load_4d(dst, &tmq, bar(B_QK_FULL), 0, hk, t0, bq);
-        tc::tma_load_4d(dst + 8192, &tmk, bar(B_QK_FULL), 0, hk, t0, bq);
-        tc::tma_load_4d(dst + 16384, &tmq, bar(B_QK_FULL), 64, hk, t0, bq);
-        tc::tma_load_4d(dst + 24576, &tmk, bar(B_QK_FULL), 64, hk, t0, bq);
+        tc::tma_load_4d(dst, &tmq, bar(B_QK_FULL), 0, hk, t0, sp.bcoord);
+        tc::tma_load_4d(dst + 8192, &tmk, bar(B_QK_FULL), 0, hk, t0, sp.bcoord);
+        tc::tma_load_4d(dst + 16384, &tmq, bar(B_QK_FULL), 64, hk, t0, sp.bcoord);
+        tc::tma_load_4d(dst + 24576, &tmk, bar(B_QK_FULL), 64, hk, t0, sp.bcoord);
         armed_qk = c;
         const uint8_t* src = pw_head + (long)c * kPwBytes;
         const uint32_t slot = sb + OFF_PW + s * PW_SLOT;
@@ -902,8 +948,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     uint4 vr[8];
     auto load_v = [&](int c) {
       const long tok = (long)c * C + t;
-      if (tok < T) {
-        const uint4* src = reinterpret_cast<const uint4*>(v + (((long)bq * T + tok) * Hv + h) * 128 + tcol);
+      if (tok < sp.len) {
+        const uint4* src = reinterpret_cast<const uint4*>(v + ((sp.row0 + tok) * Hv + h) * 128 + tcol);
 #pragma unroll
         for (int i = 0; i < 8; ++i) vr[i] = src[i];
       } else {
@@ -958,6 +1004,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         tc::mbar_wait(bar(B_X_FULL), c & 1, abort_flag, kBudget);
         if (q == 2 && lane == 0) GDN_TRACE(c, 30 + ev);
         tc::tc_fence_after();
+        const bool t_out = (long)c * C + t >= sp.len;
 #pragma unroll 1
         for (int p = 0; p < 2; ++p) {            // value columns 32p .. 32p+31 of this half
           float x[32];
@@ -973,6 +1020,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
             for (int e = 0; e < 4; ++e) {
               rv[2 * e] = fmaf(-g_t, xx[2 * e], tc::bf16lo(w4[e]));
               rv[2 * e + 1] = fmaf(-g_t, xx[2 * e + 1], tc::bf16hi(w4[e]));
+            }
+            if (t_out) {                         // past the sequence's end: no contribution
+#pragma unroll
+              for (int e = 0; e < 8; ++e) rv[e] = 0.f;
             }
             // MN-major bf16 B operand: row t (K), 16-byte chunk 4p + j of this half's columns
             const uint32_t sw = tc::sw128(t, 4 * p + j);
@@ -1038,6 +1089,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         const float g = g_t * scale;
         // bf16: one [64 t][64 dv] tile per half; fp32: two [64 t][32 dv] tiles per half
         const uint32_t stage = sb + OFF_PW + s * PW_SLOT + hh * (kF32 ? 16384 : 8192);
+        // the last chunk of a packed sequence ends inside the tile: its valid rows go straight to
+        // global memory (a box store would write into the next sequence)
+        const bool ragged = packed && (c + 1) * C > sp.len;
+        const bool t_valid = (long)c * C + t < sp.len;
+        Tout* orow = o + ((sp.row0 + (long)c * C + t) * Hv + h) * 128 + tcol;
 #pragma unroll 1
         for (int p = 0; p < 4; ++p) {            // value columns 16p .. 16p+15 of this half
           float x[16], y[16];
@@ -1046,7 +1102,24 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
           tc::tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 16; ++i) y[i] = fmaf(g, x[i], y[i]);
-          if constexpr (kF32) {                  // tile p / 2, 16-byte chunks 4 (p % 2) ..
+          if (ragged) {
+            if (t_valid) {
+              if constexpr (kF32) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                  reinterpret_cast<float4*>(orow + 16 * p)[j] =
+                      make_float4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]);
+              } else {
+#pragma unroll
+                for (int j = 0; j < 2; ++j)
+                  reinterpret_cast<uint4*>(orow + 16 * p)[j] =
+                      make_uint4(tc::pack_bf16(y[8 * j], y[8 * j + 1]),
+                                 tc::pack_bf16(y[8 * j + 2], y[8 * j + 3]),
+                                 tc::pack_bf16(y[8 * j + 4], y[8 * j + 5]),
+                                 tc::pack_bf16(y[8 * j + 6], y[8 * j + 7]));
+              }
+            }
+          } else if constexpr (kF32) {           // tile p / 2, 16-byte chunks 4 (p % 2) ..
 #pragma unroll
             for (int j = 0; j < 4; ++j)
               tc::st_shared_v4(stage + (p >> 1) * 8192 + tc::sw128(t, 4 * (p & 1) + j),
@@ -1067,14 +1140,17 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         if (leader) {
           tc::mbar_arrive(bar(B_Y_EMPTY));
           GDN_TRACE(c, 35 + ev);
-          if constexpr (kF32) {
-            tc::tma_store_4d(&tmo, stage, 64 * hh, h, c * C, bq);
-            tc::tma_store_4d(&tmo, stage + 8192, 64 * hh + 32, h, c * C, bq);
-          } else {
-            tc::tma_store_4d(&tmo, stage, 64 * hh, h, c * C, bq);
+          if (!ragged) {
+            const int oc = sp.tok0 + c * C;
+            if constexpr (kF32) {
+              tc::tma_store_4d(&tmo, stage, 64 * hh, h, oc, sp.bcoord);
+              tc::tma_store_4d(&tmo, stage + 8192, 64 * hh + 32, h, oc, sp.bcoord);
+            } else {
+              tc::tma_store_4d(&tmo, stage, 64 * hh, h, oc, sp.bcoord);
+            }
+            tc::bulk_commit();
+            tc::bulk_wait_read_all();
           }
-          tc::bulk_commit();
-          tc::bulk_wait_read_all();
           tc::mbar_arrive(bar(B_P_EMPTY + s));
           if constexpr (kF32) tc::mbar_arrive(bar(B_W_EMPTY + s));
           GDN_TRACE(c, 36 + ev);
@@ -1133,13 +1209,17 @@ inline size_t scratch_bytes(int B, int T, int Hv) {
   return (size_t)B * Hv * nC * kPwBytes;
 }
 
+// `nseq` sequences.  Fixed length (cu == nullptr): [nseq, T, ...] tensors, max_len = T.  Packed:
+// [T, ...] tensors of T tokens in all, sequence s at cu[s] .. cu[s + 1] - 1 (device offsets),
+// none longer than max_len.  `pw`: nseq * Hv * ceil(max_len / 64) records.
 template <typename Tout>
 gdn_status launch(const void* q, const void* k, const void* v, const float* la, const float* be,
-                  const float* S0, Tout* o, float* S_T, int B, int T, int Hk, int Hv, float scale,
-                  uint8_t* pw, cudaStream_t st) {
+                  const float* S0, Tout* o, float* S_T, int nseq, int T, int Hk, int Hv,
+                  float scale, uint8_t* pw, const int* cu, int max_len, cudaStream_t st) {
+  const int mapB = cu ? 1 : nseq;
   CUtensorMap mq, mk, mo;
-  if (!make_tile_map(&mq, q, Hk, T, B, false) || !make_tile_map(&mk, k, Hk, T, B, false) ||
-      !make_tile_map(&mo, o, Hv, T, B, sizeof(Tout) == 4))
+  if (!make_tile_map(&mq, q, Hk, T, mapB, false) || !make_tile_map(&mk, k, Hk, T, mapB, false) ||
+      !make_tile_map(&mo, o, Hv, T, mapB, sizeof(Tout) == 4))
     return GDN_ERR_CUDA;
   auto kern = chunk_fwd_tc_kernel<Tout>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC) !=
@@ -1148,14 +1228,16 @@ gdn_status launch(const void* q, const void* k, const void* v, const float* la, 
   if (cudaFuncSetAttribute(pw_prepass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            PP_SMEM) != cudaSuccess)
     return GDN_ERR_CUDA;
-  const long grid = (long)B * Hv;
-  const int nC = (T + C - 1) / C;
-  if (grid > 0x7fffffffL || Hv > 65535 || B > 65535) return GDN_ERR_UNSUPPORTED;
-  pw_prepass_kernel<<<dim3(nC, Hv, B), PP_THREADS, PP_SMEM, st>>>(mq, mk, la, be, pw, T, Hk, Hv,
-                                                                   scale);
+  const long grid = (long)nseq * Hv;
+  const int nCmax = (max_len + C - 1) / C;
+  if (grid > 0x7fffffffL || Hv > 65535 || nseq > 65535) return GDN_ERR_UNSUPPORTED;
+  if (nCmax == 0) return GDN_OK;
+  pw_prepass_kernel<<<dim3(nCmax, Hv, nseq), PP_THREADS, PP_SMEM, st>>>(
+      mq, mk, la, be, pw, T, Hk, Hv, scale, cu, max_len);
   if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
-  kern<<<(unsigned)grid, kThreads, SMEM_ALLOC, st>>>(
-      mq, mk, mo, static_cast<const __nv_bfloat16*>(v), pw, S0, S_T, T, Hk, Hv, scale);
+  kern<<<(unsigned)grid, kThreads, SMEM_ALLOC, st>>>(mq, mk, mo,
+                                                     static_cast<const __nv_bfloat16*>(v), pw, S0,
+                                                     S_T, T, Hk, Hv, scale, cu, max_len, nCmax, o);
   return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -1179,7 +1261,24 @@ inline gdn_status tc_chunk_launch(const void* q, const void* k, const void* v, c
                                   int T, int Hk, int Hv, float scale, void* scratch,
                                   cudaStream_t st) {
   return tcf::launch<__nv_bfloat16>(q, k, v, la, be, S0, static_cast<__nv_bfloat16*>(o), S_T, B,
-                                    T, Hk, Hv, scale, static_cast<uint8_t*>(scratch), st);
+                                    T, Hk, Hv, scale, static_cast<uint8_t*>(scratch), nullptr, T,
+                                    st);
+}
+
+// Packed sequences: q, k [total, Hk, 128], v, o [total, Hv, 128], gates [total, Hv]; sequence s is
+// tokens cu[s] .. cu[s + 1] - 1 (device int32 offsets), none longer than max_len; S0, S_T
+// [nseq, Hv, 128, 128].  `scratch`: tc_chunk_varlen_scratch_bytes(nseq, max_len, Hv).
+inline size_t tc_chunk_varlen_scratch_bytes(int nseq, int max_len, int Hv) {
+  return tcf::scratch_bytes(nseq, max_len, Hv);
+}
+inline gdn_status tc_chunk_launch_varlen(const void* q, const void* k, const void* v,
+                                         const float* la, const float* be, const int* cu,
+                                         int nseq, int max_len, const float* S0, void* o,
+                                         float* S_T, int total, int Hk, int Hv, float scale,
+                                         void* scratch, cudaStream_t st) {
+  return tcf::launch<__nv_bfloat16>(q, k, v, la, be, S0, static_cast<__nv_bfloat16*>(o), S_T,
+                                    nseq, total, Hk, Hv, scale, static_cast<uint8_t*>(scratch), cu,
+                                    max_len, st);
 }
 
 inline gdn_status tc_chunk_launch_f32out(const void* q, const void* k, const void* v,
@@ -1187,7 +1286,7 @@ inline gdn_status tc_chunk_launch_f32out(const void* q, const void* k, const voi
                                          float* o, float* S_T, int B, int T, int Hk, int Hv,
                                          float scale, void* scratch, cudaStream_t st) {
   return tcf::launch<float>(q, k, v, la, be, S0, o, S_T, B, T, Hk, Hv, scale,
-                            static_cast<uint8_t*>(scratch), st);
+                            static_cast<uint8_t*>(scratch), nullptr, T, st);
 }
 
 }  // namespace gdn

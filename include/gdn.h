@@ -173,6 +173,29 @@ GDN_API gdn_status gdn_decode_layer_step(const void *q_raw, const void *k_raw, c
                                  gdn_dtype dtype, gdn_stream_t stream);
 
 /*
+ * Chunked prefill over packed sequences of different lengths: the serving form of gdn_chunk_fwd,
+ * many requests in one call, each with its own state ("Chapitre 16 - Assembler un système de type
+ * Kimi K3", 16.2: a prompt in blocks with the state handed on; 16.1: the working state belongs to
+ * the request).
+ *   q, k [total_T, Hk, dk]; v, o [total_T, Hv, dv]                 (dtype)
+ *   log_alpha, beta [total_T, Hv] float
+ *   cu_seqlens [nseq + 1] int32 in device memory: sequence s is tokens cu[s] .. cu[s+1] - 1
+ *        (cu[0] = 0, non-decreasing, cu[nseq] <= total_T); empty sequences are allowed.  Offsets
+ *        outside [0, total_T] are clamped and a sequence longer than max_seqlen is cut there
+ *        (tokens outside every sequence keep their o untouched).
+ *   max_seqlen: a host-side upper bound of the lengths (it sizes the launch)
+ *   S0 [nseq, Hv, dk, dv] float or NULL (zero states); S_T [nseq, Hv, dk, dv] float or NULL
+ * Supported: the tensor-core family (bf16, dk = dv = 128, chunk 64); other sizes return
+ * GDN_ERR_UNSUPPORTED.  Scratch as gdn_chunk_fwd, nseq * Hv * ceil(max_seqlen / 64) * 49408
+ * bytes from the library's pool.
+ */
+GDN_API gdn_status gdn_chunk_fwd_varlen(const void *q, const void *k, const void *v,
+                                const float *log_alpha, const float *beta, const int *cu_seqlens,
+                                int nseq, int max_seqlen, const float *S0, void *o, float *S_T,
+                                int total_T, int Hk, int Hv, int dk, int dv, int chunk,
+                                float scale, gdn_dtype dtype, gdn_stream_t stream);
+
+/*
  * Gates from the in_proj_ba outputs, per (token, value head): beta = sigmoid(b) and
  * log_alpha = log sigmoid(a) = -softplus(-a).  ("L'attention hybride", "Le décompte": in_proj_ba
  * makes one beta and one alpha per value head and the layer counts no other gate parameter;

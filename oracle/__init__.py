@@ -27,6 +27,9 @@ Functions and the passages they follow (page titles; the C file's header has the
                             alpha = sigmoid(a) ("L'attention hybride", "Le décompte": one beta
                             and one alpha per value head and no other gate parameter; "Les
                             briques d'un réseau de neurones", 2.: sigmoid as the gate, softplus).
+  * ``gated_delta_varlen`` — packed requests of different lengths, each its own recurrence
+                            from its own state ("Chapitre 16 ... Kimi K3", 16.1-16.2).  Pinned
+                            by equality with the batched call when the lengths are equal.
   * ``decode_layer_steps`` — the layer one token at a time ("Chapitre 16 ... Kimi K3", 16.3) with
                             the conv's three-token history carried between steps: the composition
                             above on [history; token].  Pinned by equality with ``layer_forward``
@@ -231,6 +234,34 @@ class OracleLib:
         return y, sT
 
 
+def _gated_delta_varlen(lib: "OracleLib", q, k, v, log_alpha, beta, cu_seqlens, S0=None,
+                        scale: float = 1.0, threads: Optional[int] = None):
+    """Packed sequences: q,k [total,Hk,dk]; v [total,Hv,dv]; gates [total,Hv]; sequence s is
+    tokens cu[s] .. cu[s+1]-1, each an independent request from S0[s] (or zero).  Returns
+    (o [total,Hv,dv] with zeros outside every sequence, S_T [nseq,Hv,dk,dv])."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    la, be, s0 = _f64(log_alpha), _f64(beta), _f64(S0)
+    cu = [int(c) for c in np.asarray(cu_seqlens).reshape(-1)]
+    nseq = len(cu) - 1
+    Hv, dk, dv = v.shape[1], q.shape[2], v.shape[2]
+    o = np.zeros(v.shape)
+    sT = np.zeros((nseq, Hv, dk, dv))
+    for s in range(nseq):
+        a, b = cu[s], cu[s + 1]
+        init = None if s0 is None else s0[s:s + 1]
+        if b == a:
+            sT[s] = 0.0 if s0 is None else s0[s]
+            continue
+        os_, ss = lib.gated_delta(q[None, a:b], k[None, a:b], v[None, a:b], la[None, a:b],
+                                  be[None, a:b], init, scale=scale, threads=threads)
+        o[a:b] = os_[0]
+        sT[s] = ss[0]
+    return o, sT
+
+
+OracleLib.gated_delta_varlen = _gated_delta_varlen
+
+
 def _decode_layer_steps(lib: "OracleLib", q_raw, k_raw, v_raw, z, hq, hk, hv, wq, wk, wv,
                         log_alpha, beta, S0, norm_w, Hk: int, Hv: int, dk: int, dv: int,
                         l2_eps: float = 1e-6, norm_eps: float = 1e-5, scale: float = 1.0,
@@ -310,3 +341,7 @@ def decode_layer_steps(*a, **kw):
 
 def gates(*a, **kw):
     return get().gates(*a, **kw)
+
+
+def gated_delta_varlen(*a, **kw):
+    return get().gated_delta_varlen(*a, **kw)

@@ -345,6 +345,23 @@ def pin_decode_layer_history_is_the_three_previous_tokens(orc):
 
 
 # ---------------------------------------------------------------------------------------------
+# packed requests
+# ---------------------------------------------------------------------------------------------
+def pin_varlen_equal_lengths_equals_batched_call(orc):
+    """Packing B equal-length requests back to back equals the batched call on [B, T, ...], and
+    an empty request hands its state through unchanged."""
+    q, k, v, la, be, S0 = _rand(41, B=3, T=5, Hk=1, Hv=2)
+    o, sT = orc.gated_delta(q, k, v, la, be, S0)
+    flat = lambda a: a.reshape((-1,) + a.shape[2:])
+    cu = np.array([0, 5, 5, 10, 15])                 # the second request is empty
+    S0p = np.concatenate([S0[:1], S0[1:2] * 0.5, S0[1:]])
+    op, sTp = orc.gated_delta_varlen(flat(q), flat(k), flat(v), flat(la), flat(be), cu, S0p)
+    assert np.allclose(op, flat(o), rtol=1e-13, atol=1e-13)
+    assert np.allclose(sTp[[0, 2, 3]], sT, rtol=1e-13, atol=1e-13)
+    assert np.array_equal(sTp[1], S0p[1])
+
+
+# ---------------------------------------------------------------------------------------------
 # gates from the in_proj_ba outputs
 # ---------------------------------------------------------------------------------------------
 def pin_gates_match_library_sigmoid(orc):

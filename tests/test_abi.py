@@ -103,6 +103,19 @@ def test_decode_layer_validation(L):
     assert f(*t, 0, 2, 2, 16, 16, 1.0, 1e-6, 1e-5, 1, None) == 0            # nothing to do
 
 
+def test_varlen_validation(L):
+    f = L.gdn_chunk_fwd_varlen
+    t6 = [FAKE] * 6
+    # only the tensor-core family (bf16, 128, 128, chunk 64) is supported
+    assert f(*t6, 2, 64, FAKE, FAKE, FAKE, 128, 2, 6, 64, 64, 64, 1.0, 1, None) == 2
+    assert f(*t6, 2, 64, FAKE, FAKE, FAKE, 128, 2, 6, 128, 128, 64, 1.0, 0, None) == 2
+    assert f(*t6, -1, 64, FAKE, FAKE, FAKE, 128, 2, 6, 128, 128, 64, 1.0, 1, None) == 1
+    u = list(t6)
+    u[5] = None                                                   # cu_seqlens
+    assert f(*u, 2, 64, FAKE, FAKE, FAKE, 128, 2, 6, 128, 128, 64, 1.0, 1, None) == 1
+    assert f(*t6, 0, 64, FAKE, FAKE, FAKE, 128, 2, 6, 128, 128, 64, 1.0, 1, None) == 0
+
+
 def test_gates_validation(L):
     assert L.gdn_gates(FAKE, FAKE, FAKE, -1, 48, 1, None) == 1
     assert L.gdn_gates(FAKE, FAKE, FAKE, 10, 0, 1, None) == 1
