@@ -466,6 +466,20 @@ def dist_setup(n_gpus):
     return world, rank, local
 
 
+def max_over_ranks(value: float, device) -> float:
+    """The slowest rank sets a whole-job time: one all-reduce (MAX), outside any timed region."""
+    import torch.distributed as dist
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, t_max: float, world: int) -> float:
+    """Weak scaling: every rank ran its own replica, so the job did world x the units in the
+    slowest rank's time."""
+    return units_per_rank * world / t_max
+
+
 def run_reference(args, world, rank):
     """Reference arm: the fp64 oracle on the host cores (rank 0 only)."""
     if rank != 0:
@@ -577,9 +591,7 @@ def main():
     t_step = sum(ms) / len(ms) / 1e3
     if world > 1:
         import torch.distributed as dist
-        tt = torch.tensor([t_step], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_step = float(tt.item())
+        t_step = max_over_ranks(t_step, dev)
         dist.barrier()
     gdn.check_error(dev)
 
@@ -600,7 +612,7 @@ def main():
             "other_bound_frac": (t_ten / t_step) if hbm_bound else (t_hbm / t_step)}
     roof["frac"] = roof["achieved"] / roof["peak"]
 
-    line = {"metric": METRIC, "value": w.B * w.T * world / t_step, "unit": "tokens/s",
+    line = {"metric": METRIC, "value": whole_job_rate(w.B * w.T, t_step, world), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -616,10 +628,8 @@ def main():
 
     e2e = e2e_prefill(gdn, x, w, dev, steps=max(3, min(args.steps, 10)))
     if world > 1:   # whole-job e2e: every rank ran its replica; the slowest one sets the time
-        import torch.distributed as dist
-        tt = torch.tensor([w.B * w.T / e2e["value"]], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e["value"] = w.B * w.T * world / float(tt.item())
+        e2e["value"] = whole_job_rate(w.B * w.T, max_over_ranks(w.B * w.T / e2e["value"], dev),
+                                      world)
     line["e2e"] = e2e
     if rank == 0:
         if not args.no_secondary:
