@@ -466,6 +466,18 @@ def dist_setup(n_gpus):
     return world, rank, local
 
 
+def tc_launches_per_call(w: gi.Workload, dev, variant: str) -> int:
+    """Kernels one forward call launches: the SIMT forward one; the tensor-core forward two (the
+    operand pre-pass, then the recurrence), or four when the library splits a batched call whose
+    B * Hv recurrences exceed the SM count into tail and leading batches."""
+    if variant != "tcgen05":
+        return 1
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    head_b = sms // w.Hv
+    split = w.B >= 2 and w.B * w.Hv > sms and 1 <= head_b < w.B
+    return 4 if split else 2
+
+
 def max_over_ranks(value: float, device) -> float:
     """The slowest rank sets a whole-job time: one all-reduce (MAX), outside any timed region."""
     import torch.distributed as dist
@@ -536,7 +548,8 @@ def profile_case(args):
     gdn.check_error(dev)
     variant = gdn.chunk_fwd_variant(w.dk, w.dv, w.chunk, w.torch_dtype)
     print(json.dumps({"profile_case": workload_name(w), "calls": args.steps,
-                      "launches": args.steps * (2 if variant == "tcgen05" else 1)}), flush=True)
+                      "launches": args.steps * tc_launches_per_call(w, dev, variant)}),
+          flush=True)
 
 
 def main():
@@ -621,9 +634,7 @@ def main():
                        "kernel_variant": variant,
                        "l2": "256 MiB write between timed steps (outside the events)"},
             "roofline": roof,
-            # the tensor-core forward is two kernels per call (the operand pre-pass, then the
-            # recurrence); the SIMT forward one
-            "gpu_launches": args.steps * (2 if variant == "tcgen05" else 1),
+            "gpu_launches": args.steps * tc_launches_per_call(w, dev, variant),
             "clocks": clocks.summary()}
 
     e2e = e2e_prefill(gdn, x, w, dev, steps=max(3, min(args.steps, 10)))

@@ -42,6 +42,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "tc_ptx.cuh"
 
@@ -1209,13 +1211,46 @@ inline size_t scratch_bytes(int B, int T, int Hv) {
   return (size_t)B * Hv * nC * kPwBytes;
 }
 
-// `nseq` sequences.  Fixed length (cu == nullptr): [nseq, T, ...] tensors, max_len = T.  Packed:
-// [T, ...] tensors of T tokens in all, sequence s at cu[s] .. cu[s + 1] - 1 (device offsets),
-// none longer than max_len.  `pw`: nseq * Hv * ceil(max_len / 64) records.
+// Per device: a high- and a low-priority stream and two events for the split launch below, and
+// the SM count; calls enqueue under the mutex, so they never share the events.
+struct Split {
+  cudaStream_t s_hi = nullptr, s_lo = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_pre = nullptr, ev_hi = nullptr, ev_lo = nullptr;
+  int sms = 0;
+  bool ready = false;
+};
+inline std::mutex& split_mutex() {
+  static std::mutex mu;
+  return mu;
+}
+inline Split* split_for_device() {   // call with split_mutex() held
+  static Split splits[64];
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  Split& p = splits[dev];
+  if (!p.ready) {
+    int least = 0, greatest = 0;
+    if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
+        cudaDeviceGetAttribute(&p.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&p.s_hi, cudaStreamNonBlocking, greatest) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&p.s_lo, cudaStreamNonBlocking, least) != cudaSuccess)
+      return nullptr;
+    for (cudaEvent_t* e : {&p.ev_fork, &p.ev_pre, &p.ev_hi, &p.ev_lo})
+      if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+    p.ready = true;
+  }
+  return &p;
+}
+
+// The two kernels of one call on `st`.  `nseq` sequences.  Fixed length (cu == nullptr): [nseq, T,
+// ...] tensors, max_len = T.  Packed: [T, ...] tensors of T tokens in all, sequence s at cu[s] ..
+// cu[s + 1] - 1 (device offsets), none longer than max_len.  `pw`: nseq * Hv * ceil(max_len / 64)
+// records.
 template <typename Tout>
-gdn_status launch(const void* q, const void* k, const void* v, const float* la, const float* be,
-                  const float* S0, Tout* o, float* S_T, int nseq, int T, int Hk, int Hv,
-                  float scale, uint8_t* pw, const int* cu, int max_len, cudaStream_t st) {
+gdn_status launch_one(const void* q, const void* k, const void* v, const float* la,
+                      const float* be, const float* S0, Tout* o, float* S_T, int nseq, int T,
+                      int Hk, int Hv, float scale, uint8_t* pw, const int* cu, int max_len,
+                      cudaStream_t st, cudaEvent_t ev_after_pre) {
   const int mapB = cu ? 1 : nseq;
   CUtensorMap mq, mk, mo;
   if (!make_tile_map(&mq, q, Hk, T, mapB, false) || !make_tile_map(&mk, k, Hk, T, mapB, false) ||
@@ -1235,10 +1270,68 @@ gdn_status launch(const void* q, const void* k, const void* v, const float* la, 
   pw_prepass_kernel<<<dim3(nCmax, Hv, nseq), PP_THREADS, PP_SMEM, st>>>(
       mq, mk, la, be, pw, T, Hk, Hv, scale, cu, max_len);
   if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+  if (ev_after_pre && cudaEventRecord(ev_after_pre, st) != cudaSuccess) return GDN_ERR_CUDA;
   kern<<<(unsigned)grid, kThreads, SMEM_ALLOC, st>>>(mq, mk, mo,
-                                                     static_cast<const __nv_bfloat16*>(v), pw, S0,
-                                                     S_T, T, Hk, Hv, scale, cu, max_len, nCmax, o);
+                                                          static_cast<const __nv_bfloat16*>(v), pw,
+                                                          S0, S_T, T, Hk, Hv, scale, cu, max_len,
+                                                          nCmax, o);
   return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+// One call.  When a batched call has more (batch, head) recurrences than SMs, its recurrence would
+// run in two waves with most SMs idle in the second.  The call is then split by batches: the tail
+// batches go first (their pre-pass, then their recurrence on a high-priority stream), and the
+// pre-pass of the leading batches runs on the SMs the tail's recurrence leaves free, after which
+// their recurrence fills the GPU in one wave.  Results are those of one launch (the recurrences
+// are independent); the caller's stream waits for both parts.
+template <typename Tout>
+gdn_status launch(const void* q, const void* k, const void* v, const float* la, const float* be,
+                  const float* S0, Tout* o, float* S_T, int nseq, int T, int Hk, int Hv,
+                  float scale, uint8_t* pw, const int* cu, int max_len, cudaStream_t st) {
+  std::unique_lock<std::mutex> lock(split_mutex());
+  Split* sp = split_for_device();
+  if (!sp) return GDN_ERR_CUDA;
+  const int head_b = sp->sms / (Hv > 0 ? Hv : 1);        // batches that fill at most one wave
+  if (cu || nseq < 2 || (long)nseq * Hv <= sp->sms || head_b < 1 || head_b >= nseq) {
+    lock.unlock();
+    return launch_one<Tout>(q, k, v, la, be, S0, o, S_T, nseq, T, Hk, Hv, scale, pw, cu, max_len,
+                            st, nullptr);
+  }
+  const int tail_b = nseq - head_b;
+  const size_t tq = (size_t)T * Hk * 128, tv = (size_t)T * Hv * 128, tg = (size_t)T * Hv;
+  const size_t ts = (size_t)Hv * 128 * 128;
+  const size_t tpw = (size_t)Hv * ((T + C - 1) / C) * kPwBytes;
+  auto at_b = [&](const void* p, size_t per_batch, int b, size_t esize) -> const void* {
+    return p ? static_cast<const char*>(p) + (size_t)b * per_batch * esize : nullptr;
+  };
+  const void* qt = at_b(q, tq, head_b, 2);
+  const void* kt = at_b(k, tq, head_b, 2);
+  const void* vt = at_b(v, tv, head_b, 2);
+  const float* lat = static_cast<const float*>(at_b(la, tg, head_b, 4));
+  const float* bet = static_cast<const float*>(at_b(be, tg, head_b, 4));
+  const float* S0t = static_cast<const float*>(at_b(S0, ts, head_b, 4));
+  Tout* ot = const_cast<Tout*>(static_cast<const Tout*>(at_b(o, tv, head_b, sizeof(Tout))));
+  float* STt = const_cast<float*>(static_cast<const float*>(at_b(S_T, ts, head_b, 4)));
+  uint8_t* pwt = pw + (size_t)head_b * tpw;
+  bool ok = cudaEventRecord(sp->ev_fork, st) == cudaSuccess &&
+            cudaStreamWaitEvent(sp->s_hi, sp->ev_fork, 0) == cudaSuccess &&
+            cudaStreamWaitEvent(sp->s_lo, sp->ev_fork, 0) == cudaSuccess;
+  gdn_status s = ok ? GDN_OK : GDN_ERR_CUDA;
+  if (s == GDN_OK)   // the tail: pre-pass, then its recurrence, both on the high-priority stream
+    s = launch_one<Tout>(qt, kt, vt, lat, bet, S0t, ot, STt, tail_b, T, Hk, Hv, scale, pwt,
+                         nullptr, T, sp->s_hi, sp->ev_pre);
+  // the leading batches start once the tail's pre-pass is done
+  if (s == GDN_OK && cudaStreamWaitEvent(sp->s_lo, sp->ev_pre, 0) != cudaSuccess)
+    s = GDN_ERR_CUDA;
+  if (s == GDN_OK)
+    s = launch_one<Tout>(q, k, v, la, be, S0, o, S_T, head_b, T, Hk, Hv, scale, pw, nullptr, T,
+                         sp->s_lo, nullptr);
+  // the caller's stream waits for both parts, also after a failure, so no work outlives it
+  const bool joined = cudaEventRecord(sp->ev_hi, sp->s_hi) == cudaSuccess &&
+                      cudaEventRecord(sp->ev_lo, sp->s_lo) == cudaSuccess &&
+                      cudaStreamWaitEvent(st, sp->ev_hi, 0) == cudaSuccess &&
+                      cudaStreamWaitEvent(st, sp->ev_lo, 0) == cudaSuccess;
+  return s != GDN_OK ? s : (joined ? GDN_OK : GDN_ERR_CUDA);
 }
 
 }  // namespace tcf
