@@ -112,7 +112,10 @@ GDN_API gdn_status gdn_wait_timeout_selftest(long long budget_cycles, gdn_stream
  * pre-pass and hands them to the recurrence through a device buffer of
  * B * Hv * ceil(T/64) * 49408 bytes;
  * that buffer is taken from a memory pool of the library (one per device, stream-ordered, kept
- * between calls) and given back at the end of the call on `stream`.
+ * between calls) and given back at the end of the call on `stream`.  When B * Hv exceeds the
+ * device's SM count the call runs in two parts (the last batches first) on two internal streams
+ * of the library that fork from and join back into `stream`, so that the recurrence runs in one
+ * wave; the results are those of one launch.
  */
 GDN_API gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v,
                          const float *log_alpha, const float *beta, const float *S0,
