@@ -123,6 +123,13 @@ __device__ __forceinline__ uint32_t blk(uint32_t base, int i, int k) {
 __device__ __forceinline__ uint32_t at(uint32_t blk_base, int r, int c) {
   return blk_base + (uint32_t)((r * BLD + c) * 4);
 }
+// The solve's scratch: A's ten blocks, then the six off-diagonal blocks of T; T's diagonal blocks
+// take the place of A's.
+constexpr uint32_t SOLVE_BYTES = 16 * BSZ * 4;
+__device__ __forceinline__ uint32_t blkT(uint32_t base, int i, int k) {
+  return i == k ? blk(base, i, i)
+                : base + (uint32_t)((10 + i * (i - 1) / 2 + k) * BSZ * 4);
+}
 
 // block index bi = 0..5 -> (i, k) = (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
 __device__ __forceinline__ int blk_i(int bi) { return bi < 1 ? 1 : (bi < 3 ? 2 : 3); }
@@ -191,14 +198,15 @@ __device__ __forceinline__ void st_frag(uint32_t B, int n0, int g, int t, const 
   sts2(at(B, g + 8, n0 + 2 * t), c[2], c[3]);
 }
 
-// T = (I + A)^-1 for a 64 x 64 strictly lower A (128 threads = 4 warps, named barrier 1), blocked
+// T = (I + A)^-1 for a 64 x 64 strictly lower A (128 threads = 4 warps, named barriers 1 and 3), blocked
 // by 16:  D_b = (I + A_bb)^-1 by forward substitution (one column per thread);  At_ik = D_i A_ik;
 // U = (I + At)^-1 (U_ii = I; At is block-nilpotent, so U is closed-form in At's blocks);
 // T_ik = U_ik D_k.   (I + A = blockdiag(I + A_bb) (I + At), so T = U D.)  The block products run
 // as warp MMAs on 16 x 8 half blocks.  On return the off-diagonal blocks of T are in `tv`: item m
 // of warp w is half block hp = w + 4 m (block bi = hp / 2, columns 8 (hp % 2) ..) as a C fragment;
-// the diagonal blocks D_b are in sT.  sA's blocks are overwritten.
-__device__ __forceinline__ void solve_unit_lower(uint32_t sA, uint32_t sT, int ptid, float (&tv)[3][4]) {
+// the diagonal blocks D_b are in blkT(s, b, b), over A_bb.  A's other blocks are overwritten.
+__device__ __forceinline__ void solve_unit_lower(uint32_t s, int ptid, float (&tv)[3][4]) {
+  const uint32_t sA = s;
   if (ptid < 64) {                                    // D_b, column `col` of block b
     const int b = ptid >> 4, col = ptid & 15;
     const uint32_t Ab = blk(sA, b, b);
@@ -219,7 +227,8 @@ __device__ __forceinline__ void solve_unit_lower(uint32_t sA, uint32_t sT, int p
       }
       x[i] = a0 + a1;
     }
-    const uint32_t Tb = blk(sT, b, b);
+    tc::named_bar(3, 64);                             // every row of A_bb read: D_b replaces it
+    const uint32_t Tb = blkT(s, b, b);
 #pragma unroll
     for (int i = 0; i < 16; ++i) tc::sts1(at(Tb, i, col), x[i]);
   }
@@ -232,14 +241,14 @@ __device__ __forceinline__ void solve_unit_lower(uint32_t sA, uint32_t sT, int p
     for (int m = 0; m < 3; ++m) {
       const int hp = w + 4 * m, bi = hp >> 1, n0 = (hp & 1) * 8;
       const int i = blk_i(bi), k = blk_k(bi, i);
-      tl[m] = Tile{blk(sT, i, i), blk(sA, i, k), n0};
+      tl[m] = Tile{blkT(s, i, i), blk(sA, i, k), n0};
     }
     mma_tiles(tl, g, t, acc);
 #pragma unroll
     for (int m = 0; m < 3; ++m) {
       const int bi = (w + 4 * m) >> 1;
       const int i = blk_i(bi), k = blk_k(bi, i);
-      st_frag(blk(sT, i, k), tl[m].n0, g, t, acc[m]);
+      st_frag(blkT(s, i, k), tl[m].n0, g, t, acc[m]);
     }
   }
   tc::named_bar(1, 128);
@@ -254,10 +263,10 @@ __device__ __forceinline__ void solve_unit_lower(uint32_t sA, uint32_t sT, int p
       const int hp = m < nt ? w + 4 * m : w, bi = hp >> 1, n0 = (hp & 1) * 8;
       const int oi = bi == 0 ? 2 : 3, ok = bi == 1 ? 1 : 0;    // output block (oi, ok)
       const int xk = bi == 1 ? 2 : 1;                           // X = At_(oi, xk), Y = At_(xk, ok)
-      ld_frag(blk(sT, oi, ok), n0, g, t, acc[m]);
+      ld_frag(blkT(s, oi, ok), n0, g, t, acc[m]);
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[m][e] = -acc[m][e];
-      tl[m] = Tile{blk(sT, oi, xk), blk(sT, xk, ok), n0};
+      tl[m] = Tile{blkT(s, oi, xk), blkT(s, xk, ok), n0};
     }
     mma_tiles(tl, g, t, acc);
 #pragma unroll
@@ -271,7 +280,7 @@ __device__ __forceinline__ void solve_unit_lower(uint32_t sA, uint32_t sT, int p
   tc::named_bar(1, 128);
   if (w < 2) {                                        // U_30 = V_30 - At_32 U_20
     const int n0 = 8 * w;
-    const Tile tl[1] = {Tile{blk(sT, 3, 2), blk(sA, 2, 0), n0}};
+    const Tile tl[1] = {Tile{blkT(s, 3, 2), blk(sA, 2, 0), n0}};
     float acc[1][4] = {}, v[4];
     ld_frag(blk(sA, 3, 0), n0, g, t, v);
     mma_tiles(tl, g, t, acc);
@@ -287,7 +296,7 @@ __device__ __forceinline__ void solve_unit_lower(uint32_t sA, uint32_t sT, int p
     for (int m = 0; m < 3; ++m) {
       const int hp = w + 4 * m, bi = hp >> 1, n0 = (hp & 1) * 8;
       const int i = blk_i(bi), k = blk_k(bi, i);
-      tl[m] = Tile{(i == k + 1) ? blk(sT, i, k) : blk(sA, i, k), blk(sT, k, k), n0};
+      tl[m] = Tile{(i == k + 1) ? blkT(s, i, k) : blk(sA, i, k), blkT(s, k, k), n0};
     }
     mma_tiles(tl, g, t, acc);
 #pragma unroll
@@ -401,9 +410,9 @@ __device__ __forceinline__ SeqSpan seq_span(const int* __restrict__ cu, int s, i
 //   W  = K^T diag(ktil) T_b   (128 x 64: M <- gamma_last M + W R')
 // since Delta = T_b R'.  Neither depends on the state, so one small CTA per chunk computes them
 // ahead of the recurrence, on the tensor cores: S = [Q; K] K^T (bf16 MMA into TMEM), P and A from
-// S with the gates (one TMEM row per thread), the blocked solve, then PT = P T_b and
-// W = K^T (ktil T_b) as bf16 MMAs on hi + lo splits (hi.hi + lo.hi + hi.lo for PT; K is exact, so
-// two terms for W).  The result goes to HBM as the recurrence's MMA operands themselves: per
+// S with the gates (one TMEM row per thread), the blocked solve, then PT = P T_b and, through the
+// same pair of operand tiles once PT has read them, W = K^T (ktil T_b), as bf16 MMAs on hi + lo
+// splits (hi.hi + lo.hi + hi.lo for PT; K is exact, so two terms for W).  The result goes to HBM as the recurrence's MMA operands themselves: per
 // chunk 48 KB of 128-byte-swizzled K-major bf16 tiles, PT hi [64 rows][128 B], PT lo, W hi [128
 // rows][128 B], W lo, followed by gamma_t = exp(G_t) (64 fp32).  A chunk whose P or A holds a NaN
 // or an infinity gets +inf in every tile, so the recurrence still sees a non-finite value.
@@ -412,14 +421,14 @@ constexpr int kPwBytes = kPwTiles + 256;     // + gamma_t = exp(G_t), 64 fp32
 constexpr int PP_THREADS = 128;
 constexpr uint32_t PP_QK = 0;        // 32 KB: Q cols 0..63 | K cols 0..63 | Q 64..127 | K 64..127;
                                      // P hi over the first Q box, P lo over the second
-constexpr uint32_t PP_TB = 32768;    // solve scratch, then 4 x 8 KB MN-major B tiles [64 rows][128 B]:
-                                     // T_b hi, T_b lo, ktil T_b hi, ktil T_b lo
-constexpr uint32_t PP_G = 65536;     // G'[64], beta[64], ktil[64], flag, abort, then at float 256
-                                     // E[4][64]; barriers at +3072
-constexpr uint32_t PP_BAR = PP_G + 3072;
-constexpr uint32_t PP_SMEM = PP_BAR + 64 + 1024;   // + alignment slack (three CTAs per SM)
-constexpr uint32_t SOLVE_T = 12800;  // byte offset of T inside the solve scratch
-static_assert(2 * SOLVE_T <= 32768, "solve scratch fits the B tiles' space");
+constexpr uint32_t PP_TB = 32768;    // solve scratch, then 2 x 8 KB MN-major B tiles [64 rows][128 B]:
+                                     // T_b hi, T_b lo, later ktil T_b hi, ktil T_b lo
+constexpr uint32_t PP_G = PP_TB + SOLVE_BYTES;   // G'[64], beta[64], ktil[64], flag, abort, then
+                                                 // at float 256 E[4][64]; barriers at +2048
+constexpr uint32_t PP_BAR = PP_G + 2048;
+constexpr uint32_t PP_SMEM = PP_BAR + 64 + 1024;   // + alignment slack (four CTAs per SM)
+static_assert(SOLVE_BYTES >= 16384, "the B tile pair fits the solve scratch's space");
+static_assert(4 * (PP_SMEM + 1024) <= 233472, "four pre-pass CTAs per SM");
 constexpr uint32_t ID_S = tc::idesc_bf16(128, 64, false, false);   // [Q; K] K^T
 constexpr uint32_t ID_PT = tc::idesc_bf16(128, 64, false, true);   // P T_b (rows 64..127 unused)
 constexpr uint32_t ID_W = tc::idesc_bf16(128, 64, true, true);     // K^T (ktil T_b)
@@ -428,22 +437,18 @@ constexpr uint32_t ID_W = tc::idesc_bf16(128, 64, true, true);     // K^T (ktil 
 __device__ __forceinline__ uint32_t sw_elem(int r, int j) {
   return (uint32_t)(r * 128 + ((((j >> 3) ^ (r & 7))) << 4) + (j & 7) * 2);
 }
-// T_b values (row, n), (row, n + 1) (n even) into the four B tiles.
-__device__ __forceinline__ void store_tb_pair(uint32_t tb, int row, int n, float a, float b,
-                                              float kt) {
-  uint32_t h, l, kh, kl;
+// Values (row, n), (row, n + 1) (n even) into the B tile pair (hi at tb, lo at tb + 8192).
+__device__ __forceinline__ void store_b_pair(uint32_t tb, int row, int n, float a, float b) {
+  uint32_t h, l;
   split2(a, b, h, l);
-  split2(kt * a, kt * b, kh, kl);
   const uint32_t o = tb + sw_elem(row, n);
   tc::sts1(o, __uint_as_float(h));
   tc::sts1(o + 8192, __uint_as_float(l));
-  tc::sts1(o + 16384, __uint_as_float(kh));
-  tc::sts1(o + 24576, __uint_as_float(kl));
 }
 
 // grid (nCmax, Hv, sequences), 128 threads; thread r owns TMEM lane r.  CTAs past the end of
 // their sequence return at once.
-__global__ void __launch_bounds__(PP_THREADS, 3)
+__global__ void __launch_bounds__(PP_THREADS, 4)
 pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const float* __restrict__ log_alpha, const float* __restrict__ beta,
                   uint8_t* __restrict__ pw, int T, int Hk, int Hv, float scale,
@@ -611,55 +616,52 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 
   GDN_TRACE_PP(4);
   float tv[3][4];
-  solve_unit_lower(tb, tb + SOLVE_T, tid, tv);
+  solve_unit_lower(tb, tid, tv);
   GDN_TRACE_PP(5);
   float4 dg[2];
 #pragma unroll
   for (int m = 0; m < 2; ++m) {
     const int id = tid + PP_THREADS * m, b = id >> 6, r = (id >> 2) & 15, cs = id & 3;
-    dg[m] = tc::lds4(at(blk(tb + SOLVE_T, b, b), r, 4 * cs));
+    dg[m] = tc::lds4(at(blkT(tb, b, b), r, 4 * cs));
   }
   __syncthreads();                                    // the solve scratch is dead
-  {
+  // T_b (kt false) or ktil T_b (kt true) into the B tile pair; the zeros above the diagonal
+  // blocks are written once and serve both
+  auto put_b = [&](bool kt) {
     const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
     for (int m = 0; m < 3; ++m) {                     // off-diagonal blocks and their zero mirrors
       const int hp = warp + 4 * m, bi = hp >> 1, n0 = (hp & 1) * 8;
       const int i = blk_i(bi), kk = blk_k(bi, i);
       const int col = 16 * kk + n0 + 2 * t4, row = 16 * i + g;
-      store_tb_pair(tb, row, col, tv[m][0] * gB[col], tv[m][1] * gB[col + 1], gKt[row]);
-      store_tb_pair(tb, row + 8, col, tv[m][2] * gB[col], tv[m][3] * gB[col + 1], gKt[row + 8]);
-      const int urow = 16 * kk + g, ucol = 16 * i + n0 + 2 * t4;
-      store_tb_pair(tb, urow, ucol, 0.f, 0.f, 0.f);
-      store_tb_pair(tb, urow + 8, ucol, 0.f, 0.f, 0.f);
+      const float f0 = kt ? gKt[row] : 1.f, f1 = kt ? gKt[row + 8] : 1.f;
+      store_b_pair(tb, row, col, f0 * (tv[m][0] * gB[col]), f0 * (tv[m][1] * gB[col + 1]));
+      store_b_pair(tb, row + 8, col, f1 * (tv[m][2] * gB[col]), f1 * (tv[m][3] * gB[col + 1]));
+      if (!kt) {
+        const int urow = 16 * kk + g, ucol = 16 * i + n0 + 2 * t4;
+        store_b_pair(tb, urow, ucol, 0.f, 0.f);
+        store_b_pair(tb, urow + 8, ucol, 0.f, 0.f);
+      }
     }
 #pragma unroll
     for (int m = 0; m < 2; ++m) {                     // diagonal blocks (zero above the diagonal)
       const int id = tid + PP_THREADS * m, b = id >> 6, r = (id >> 2) & 15, cs = id & 3;
       const int row = 16 * b + r, col = 16 * b + 4 * cs;
-      store_tb_pair(tb, row, col, dg[m].x * gB[col], dg[m].y * gB[col + 1], gKt[row]);
-      store_tb_pair(tb, row, col + 2, dg[m].z * gB[col + 2], dg[m].w * gB[col + 3], gKt[row]);
+      const float f = kt ? gKt[row] : 1.f;
+      store_b_pair(tb, row, col, f * (dg[m].x * gB[col]), f * (dg[m].y * gB[col + 1]));
+      store_b_pair(tb, row, col + 2, f * (dg[m].z * gB[col + 2]), f * (dg[m].w * gB[col + 3]));
     }
-  }
-  tc::fence_proxy_async_smem();
-  tc::tc_fence_before();
-  __syncthreads();
-
-  // W = K^T (ktil T_b) (columns 0..63; S is consumed), then PT = P T_b (columns 64..127), each
-  // with its own completion so W's rows go out while PT is still being multiplied
+    tc::fence_proxy_async_smem();
+    tc::tc_fence_before();
+    __syncthreads();
+  };
+  const uint64_t dt = tc::sdesc_sw128(tb, 8192, 1024);
+  put_b(false);
+  // PT = P T_b into columns 64..127
   GDN_TRACE_PP(6);
   if (tid == 0) {
     tc::tc_fence_after();
     const uint64_t dp = tc::sdesc_sw128(qk, 16, 1024);
-    const uint64_t dt = tc::sdesc_sw128(tb, 8192, 1024);
-    const uint64_t dk = tc::sdesc_sw128(qk + 8192, 16384, 1024);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int ks = i >> 1, term = i & 1;
-      tc::mma_bf16(tmem, tc::desc_adv(dk, ks * 2048), tc::desc_adv(dt, 16384 + term * 8192 + ks * 2048),
-                   ID_W, i > 0);
-    }
-    tc::mma_commit(mma_bar);
 #pragma unroll
     for (int i = 0; i < 12; ++i) {
       const int ks = i / 3, term = i - 3 * ks;
@@ -668,14 +670,27 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     }
     tc::mma_commit(pt_bar);
   }
-  tc::mbar_wait(mma_bar, 1, abort_flag, kBudget);
-  GDN_TRACE_PP(7);
+  tc::mbar_wait(pt_bar, 0, abort_flag, kBudget);
   tc::tc_fence_after();
+  // W = K^T (ktil T_b) into columns 0..63 (S is consumed) from the same tiles, now free
+  put_b(true);
+  if (tid == 0) {
+    tc::tc_fence_after();
+    const uint64_t dk = tc::sdesc_sw128(qk + 8192, 16384, 1024);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int ks = i >> 1, term = i & 1;
+      tc::mma_bf16(tmem, tc::desc_adv(dk, ks * 2048), tc::desc_adv(dt, term * 8192 + ks * 2048),
+                   ID_W, i > 0);
+    }
+    tc::mma_commit(mma_bar);
+  }
+  GDN_TRACE_PP(7);
   const bool poison = *flag != 0;
   // Rows from TMEM are split and staged (swizzled, in the record's tile layout) in shared memory
-  // the pending MMAs no longer read, then leave by bulk copies: W's while PT is still being
-  // multiplied (W hi over the ktil T_b tiles, W lo rows 0..63 / 64..127 over the two K boxes),
-  // PT's once it is done (hi over P hi, lo over P lo).
+  // the MMAs no longer read, then leave by bulk copies: PT's while W is still being multiplied
+  // (hi over P hi, lo over P lo), W's once it is done (hi over the B tile pair, lo rows 0..63 /
+  // 64..127 over the two K boxes).
   auto stage_row = [&](uint32_t hi_base, uint32_t lo_base, int r, const float* w) {
 #pragma unroll
     for (int j8 = 0; j8 < 8; ++j8) {
@@ -685,26 +700,7 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
   };
   {
     float w[64];
-    tc::tmem_ld32(tmem + lane_off, *reinterpret_cast<float(*)[32]>(&w[0]));
-    tc::tmem_ld32(tmem + lane_off + 32, *reinterpret_cast<float(*)[32]>(&w[32]));
-    tc::tmem_wait_ld();
-    if (poison) {
-#pragma unroll
-      for (int j = 0; j < 64; ++j) w[j] = kInf;
-    }
-    // W row r: hi at tb + 16384 + r * 128, lo at qk + 8192 (r < 64) or qk + 24576 (r >= 64)
-    stage_row(tb + 16384, qk + (tid < 64 ? 8192 : 24576 - 64 * 128), tid, w);
-    tc::fence_proxy_async_smem();
-    tc::named_bar(1, 128);
-    if (tid == 0) {
-      tc::bulk_store(rec + 16384, tb + 16384, 16384);
-      tc::bulk_store(rec + 32768, qk + 8192, 8192);
-      tc::bulk_store(rec + 40960, qk + 24576, 8192);
-      tc::bulk_commit();
-    }
     if (tid < 64) {
-      tc::mbar_wait(pt_bar, 0, abort_flag, kBudget);
-      tc::tc_fence_after();
       tc::tmem_ld32(tmem + lane_off + 64, *reinterpret_cast<float(*)[32]>(&w[0]));
       tc::tmem_ld32(tmem + lane_off + 96, *reinterpret_cast<float(*)[32]>(&w[32]));
       tc::tmem_wait_ld();
@@ -719,9 +715,28 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         tc::bulk_store(rec, qk, 8192);
         tc::bulk_store(rec + 8192, qk + 16384, 8192);
         tc::bulk_commit();
-        tc::bulk_wait_read_all();                     // every source read; the writes complete
-      }                                               // on their own
+      }
     }
+    tc::mbar_wait(mma_bar, 1, abort_flag, kBudget);
+    tc::tc_fence_after();
+    tc::tmem_ld32(tmem + lane_off, *reinterpret_cast<float(*)[32]>(&w[0]));
+    tc::tmem_ld32(tmem + lane_off + 32, *reinterpret_cast<float(*)[32]>(&w[32]));
+    tc::tmem_wait_ld();
+    if (poison) {
+#pragma unroll
+      for (int j = 0; j < 64; ++j) w[j] = kInf;
+    }
+    // W row r: hi at tb + r * 128, lo at qk + 8192 (r < 64) or qk + 24576 (r >= 64)
+    stage_row(tb, qk + (tid < 64 ? 8192 : 24576 - 64 * 128), tid, w);
+    tc::fence_proxy_async_smem();
+    tc::named_bar(1, 128);
+    if (tid == 0) {
+      tc::bulk_store(rec + 16384, tb, 16384);
+      tc::bulk_store(rec + 32768, qk + 8192, 8192);
+      tc::bulk_store(rec + 40960, qk + 24576, 8192);
+      tc::bulk_commit();
+      tc::bulk_wait_read_all();                       // every source read; the writes complete
+    }                                                 // on their own
   }
   GDN_TRACE_PP(8);
   GDN_TRACE_PP(9);
