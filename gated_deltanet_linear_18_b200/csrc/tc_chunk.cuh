@@ -368,8 +368,9 @@ constexpr float kInf = __builtin_huge_valf();
 // non-finite in hi or lo.
 __device__ __forceinline__ void split2(float a, float b, uint32_t& hi2, uint32_t& lo2) {
   const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(b);
-  const float la = a - __uint_as_float(ua & 0xFFFF0000u);
-  const float lb = b - __uint_as_float(ub & 0xFFFF0000u);
+  float la, lb;
+  tc::f2_get(tc::sub2(tc::f2(a, b), tc::f2(__uint_as_float(ua & 0xFFFF0000u),
+                                           __uint_as_float(ub & 0xFFFF0000u))), la, lb);
   hi2 = __byte_perm(ua, ub, 0x7632);
   lo2 = __byte_perm(__float_as_uint(la), __float_as_uint(lb), 0x7632);
 }
@@ -577,8 +578,8 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float4 e = *reinterpret_cast<const float4*>(gE + 64 * ti + 16 * kb + 4 * i);
-          f[4 * i] = rowf * e.x; f[4 * i + 1] = rowf * e.y;
-          f[4 * i + 2] = rowf * e.z; f[4 * i + 3] = rowf * e.w;
+          tc::f2_get(tc::mul2(tc::f2(rowf, rowf), tc::f2(e.x, e.y)), f[4 * i], f[4 * i + 1]);
+          tc::f2_get(tc::mul2(tc::f2(rowf, rowf), tc::f2(e.z, e.w)), f[4 * i + 2], f[4 * i + 3]);
         }
       } else if (kb == ti) {
 #pragma unroll
@@ -591,10 +592,11 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         for (int e = 0; e < 16; ++e) f[e] = 0.f;
       }
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        f[e] *= s[16 * kb + e];
-        sum += f[e];
-      }
+      for (int e = 0; e < 16; e += 2)
+        tc::f2_get(tc::mul2(tc::f2(f[e], f[e + 1]), tc::f2(s[16 * kb + e], s[16 * kb + e + 1])),
+                   f[e], f[e + 1]);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) sum += f[e];
       if (isP) {                // P row t: K-major bf16 hi over the first Q box, lo over the second
 #pragma unroll
         for (int h8 = 0; h8 < 2; ++h8) {
@@ -1034,10 +1036,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
             const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
             float rv[8];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              rv[2 * e] = fmaf(-g_t, xx[2 * e], tc::bf16lo(w4[e]));
-              rv[2 * e + 1] = fmaf(-g_t, xx[2 * e + 1], tc::bf16hi(w4[e]));
-            }
+            for (int e = 0; e < 4; ++e)
+              tc::f2_get(tc::fma2(tc::f2(-g_t, -g_t), tc::f2(xx[2 * e], xx[2 * e + 1]),
+                                  tc::f2(tc::bf16lo(w4[e]), tc::bf16hi(w4[e]))),
+                         rv[2 * e], rv[2 * e + 1]);
             if (t_out) {                         // past the sequence's end: no contribution
 #pragma unroll
               for (int e = 0; e < 8; ++e) rv[e] = 0.f;
@@ -1078,7 +1080,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
           tc::mbar_arrive(bar(B_M_READY));
         }
 #pragma unroll
-        for (int i = 0; i < 64; ++i) m[i] *= g_nl;
+        for (int i = 0; i < 64; i += 2)
+          tc::f2_get(tc::mul2(tc::f2(m[i], m[i + 1]), tc::f2(g_nl, g_nl)), m[i], m[i + 1]);
         tmem_st64(tmem + lane_off + TM_M + tcol, m);
         tc::tmem_wait_st();
       } else if (S_T && !*abort_flag) {
@@ -1118,7 +1121,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
           tmem_ld16(tmem + lane_off + TM_Y + tcol + 16 * p, y);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) y[i] = fmaf(g, x[i], y[i]);
+          for (int i = 0; i < 16; i += 2)
+            tc::f2_get(tc::fma2(tc::f2(g, g), tc::f2(x[i], x[i + 1]), tc::f2(y[i], y[i + 1])),
+                       y[i], y[i + 1]);
           if (ragged) {
             if (t_valid) {
               if constexpr (kF32) {
