@@ -63,9 +63,10 @@ constexpr uint32_t OFF_MB = 98304;      // 32 KB, per column half 16 KB: bf16 M 
 constexpr uint32_t OFF_PW = 131072;     // 2 slots x 48 KB: a chunk's PT hi, PT lo, W hi, W lo
 constexpr uint32_t PW_SLOT = 49152;     // after Y (and the update) the o tile is staged there
 constexpr uint32_t OFF_BAR = OFF_PW + 2 * PW_SLOT;
-constexpr int NBAR = 20;
+constexpr int NBAR = 22;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;   // +0 TMEM base, +4 abort flag
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 16;
+constexpr uint32_t OFF_GAM = OFF_MISC + 16;         // 2 slots (chunk parity) x gamma_t, 64 fp32
+constexpr uint32_t SMEM_BYTES = OFF_GAM + 2 * 256;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 
@@ -78,7 +79,8 @@ constexpr uint32_t TM_X = 0, TM_Y = 256, TM_M = 384;
 // left the slot.
 enum : int {
   B_QK_FULL = 0, B_QK_EMPTY, B_W_FULL = 2, B_W_EMPTY = 4, B_P_FULL = 6, B_P_EMPTY = 8,
-  B_X_FULL = 10, B_R_FULL, B_D3_FULL, B_Y_FULL, B_Y_EMPTY, B_M_READY, B_M_SCALED, B_DRAIN, B_END
+  B_X_FULL = 10, B_R_FULL, B_D3_FULL, B_Y_FULL, B_Y_EMPTY, B_M_READY, B_M_SCALED, B_DRAIN,
+  B_G_FULL = 18, B_G_EMPTY = 20, B_END = 22
 };
 static_assert(B_END <= NBAR, "barrier map");
 
@@ -447,19 +449,20 @@ __device__ __forceinline__ void store_b_pair(uint32_t tb, int row, int n, float 
   tc::sts1(o + 8192, __uint_as_float(l));
 }
 
-// grid (nCmax, Hv, sequences), 128 threads; thread r owns TMEM lane r.  CTAs past the end of
-// their sequence return at once.
+// grid (Hv, nCmax, sequences), 128 threads; thread r owns TMEM lane r.  CTAs past the end of
+// their sequence return at once.  With `ready`, each CTA sets ready[(s * Hv + h) * nCmax + c] to 1
+// (release) once its record is in global memory, for a recurrence that runs alongside.
 __global__ void __launch_bounds__(PP_THREADS, 4)
 pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const float* __restrict__ log_alpha, const float* __restrict__ beta,
                   uint8_t* __restrict__ pw, int T, int Hk, int Hv, float scale,
-                  const int* __restrict__ cu, int max_len) {
+                  const int* __restrict__ cu, int max_len, int* __restrict__ ready) {
   GDN_TRACE_INIT;
   extern __shared__ __align__(1024) uint8_t pp_raw[];
   uint8_t* smem = pp_raw + ((1024u - (tc::smem_u32(pp_raw) & 1023u)) & 1023u);
   const uint32_t sb = tc::smem_u32(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int c = blockIdx.x, h = blockIdx.y, sq = blockIdx.z, nC = gridDim.x;
+  const int h = blockIdx.x, c = blockIdx.y, sq = blockIdx.z, nC = gridDim.y;
   const SeqSpan sp = seq_span(cu, sq, T, max_len);
   if (c * C >= sp.len) return;                        // (uniform: before any barrier)
   const int vrows = min(C, sp.len - c * C);           // tokens of this chunk in the sequence
@@ -737,8 +740,14 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
       tc::bulk_store(rec + 32768, qk + 8192, 8192);
       tc::bulk_store(rec + 40960, qk + 24576, 8192);
       tc::bulk_commit();
-      tc::bulk_wait_read_all();                       // every source read; the writes complete
-    }                                                 // on their own
+      if (ready) {                                    // the record is complete, then published
+        tc::bulk_wait_all();
+        tc::fence_proxy_async_global();
+        tc::st_release_gpu(ready + ((long)sq * Hv + h) * nC + c, 1);
+      } else {
+        tc::bulk_wait_read_all();                     // every source read; the writes complete
+      }                                               // on their own
+    }
   }
   GDN_TRACE_PP(8);
   GDN_TRACE_PP(9);
@@ -760,7 +769,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
                     const __grid_constant__ CUtensorMap tmo, const __nv_bfloat16* __restrict__ v,
                     const uint8_t* __restrict__ pw, const float* __restrict__ S0,
                     float* __restrict__ S_T, int T, int Hk, int Hv, float scale,
-                    const int* __restrict__ cu, int max_len, int nCmax, Tout* __restrict__ o) {
+                    const int* __restrict__ cu, int max_len, int nCmax, Tout* __restrict__ o,
+                    const int* __restrict__ ready) {
   constexpr bool kF32 = sizeof(Tout) == 4;
   // X takes M as a hi + lo bf16 pair when o is fp32 (the layer, whose gated norm magnifies o's
   // error); a bf16 o carries its own rounding, and one round-to-nearest bf16 copy of M suffices.
@@ -781,6 +791,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   const bool packed = cu != nullptr;
   const long head = (long)bq * Hv + h;
   const uint8_t* pw_head = pw + head * nCmax * (long)kPwBytes;
+  // with `ready`, record c of this head may still be being written by a pre-pass that runs
+  // alongside: every reader of it first waits for its flag (acquire)
+  const int* ready_head = ready ? ready + head * nCmax : nullptr;
   if (nC == 0) {   // an empty sequence: the state passes through (uniform, before any barrier)
     if (S_T)
       for (int i = threadIdx.x; i < 128 * 128 / 4; i += blockDim.x)
@@ -802,6 +815,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(bar(B_P_EMPTY + s), 3);
       tc::mbar_init(bar(B_W_EMPTY + s), kF32 ? 3 : 1);
+      tc::mbar_init(bar(B_G_FULL + s), 1);
+      tc::mbar_init(bar(B_G_EMPTY + s), 8);           // one arrive per chain warp
     }
     *abort_flag = 0;
     tc::fence_barrier_init();
@@ -840,6 +855,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         armed_qk = c;
         const uint8_t* src = pw_head + (long)c * kPwBytes;
         const uint32_t slot = sb + OFF_PW + s * PW_SLOT;
+        if (ready_head) {
+          if (!(ok = tc::flag_wait(ready_head + c, abort_flag, kBudget))) break;
+          tc::fence_proxy_async_global();
+        }
         if (c >= 2) ok = tc::mbar_wait(bar(B_W_EMPTY + s), ((c >> 1) - 1) & 1, abort_flag, kBudget);
         if (!ok) break;
         tc::mbar_arrive_expect_tx(bar(B_W_FULL + s), 32768);
@@ -934,6 +953,25 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       volatile int never = 0;
       tc::mbar_wait(bar(B_DRAIN), 0, &never, kBudget / 4);
     }
+  } else if (warp == 2) {
+    // ------------------------------- gamma ---------------------------------------------------
+    // gamma_t of chunk c into ring slot c & 1 (after the record's ready flag, when there is one),
+    // so that the chain reads it from shared memory
+    const float* gsrc = reinterpret_cast<const float*>(pw_head + kPwTiles);
+    for (int c = 0; c < nC; ++c) {
+      const int s = c & 1;
+      int ok = 1;
+      if (lane == 0 && c >= 2)
+        ok = tc::mbar_wait(bar(B_G_EMPTY + s), ((c >> 1) - 1) & 1, abort_flag, kBudget);
+      __syncwarp();                                    // the slot's readers before its writers
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (ok && ready_head) ok = tc::flag_wait(ready_head + c, abort_flag, kBudget);  // each lane
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const float2 g = reinterpret_cast<const float2*>(gsrc + (long)c * (kPwBytes / 4))[lane];
+      *reinterpret_cast<float2*>(smem + OFF_GAM + s * 256 + 8 * lane) = g;
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar(B_G_FULL + s));
+    }
   } else if (warp >= 4) {
     // ------------------------------- chain warpgroups ----------------------------------------
     // warps 4-7: value columns 0..63, warps 8-11: 64..127.  Lanes 0..63 (q < 2) make o of token
@@ -945,8 +983,14 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     const uint32_t id_wg = 1 + 3 * hh, id_lo = 2 + 3 * hh, id_hi = 3 + 3 * hh;
     const bool leader = (q == 0 && lane == 0);
     [[maybe_unused]] const int ev = 10 * hh;
-    auto gam_at = [&](int c, int i) -> float {
-      return reinterpret_cast<const float*>(pw_head + (long)c * kPwBytes + kPwTiles)[i];
+    // gamma_t (t) and gamma_last of chunk c from the ring; the slot is handed back at once
+    auto gam_get = [&](int c, float& gt, float& gl) {
+      tc::mbar_wait(bar(B_G_FULL + (c & 1)), (c >> 1) & 1, abort_flag, kBudget);
+      const float* g = reinterpret_cast<const float*>(smem + OFF_GAM + (c & 1) * 256);
+      gt = g[t];
+      gl = g[63];
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar(B_G_EMPTY + (c & 1)));
     };
     // 32 columns (32p ..) of M row r (this half) for the X MMA: one round-to-nearest bf16 copy in Mb,
     // or (kSplitX) a hi + lo pair, hi into Mb and lo into the R' buffer
@@ -977,7 +1021,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       }
     };
     if (q >= 2) load_v(0);
-    float g_t = gam_at(0, t);
+    float g_t, g_l0;
+    gam_get(0, g_t, g_l0);
     bool stop = false;
     {
       float m[64];
@@ -994,9 +1039,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       }
       store_m32(*reinterpret_cast<const float(*)[32]>(&m[0]), 0, rd0);
       store_m32(*reinterpret_cast<const float(*)[32]>(&m[32]), 1, rd0);
-      const float gl = gam_at(0, 63);
 #pragma unroll
-      for (int i = 0; i < 64; ++i) m[i] *= gl;
+      for (int i = 0; i < 64; ++i) m[i] *= g_l0;
       tmem_st64(tmem + lane_off + TM_M + tcol, m);
       tc::tmem_wait_st();
       tc::fence_proxy_async_smem();
@@ -1013,10 +1057,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       const uint32_t tx = tmem + lane_off + TM_X + 128 * s + tcol;
       // the next chunk's gates: gamma_last for the state below, gamma_t for the next chunk
       float g_nt = 0.f, g_nl = 0.f;
-      if (c + 1 < nC) {
-        g_nt = gam_at(c + 1, t);
-        g_nl = gam_at(c + 1, 63);
-      }
+      if (c + 1 < nC) gam_get(c + 1, g_nt, g_nl);
       if (q >= 2) {
         // R' = V - gamma (K M) for token t, as a bf16 hi + lo pair (the B operand of Y and of
         // the state update)
@@ -1225,10 +1266,11 @@ inline bool make_tile_map(CUtensorMap* m, const void* base, int H, int T, int B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Bytes of the operand hand-over buffer between the pre-pass and the recurrence.
+// Bytes of the operand hand-over buffer between the pre-pass and the recurrence: the records,
+// then one int32 ready flag per record (used when a recurrence runs alongside its pre-pass).
+inline size_t records(int B, int T, int Hv) { return (size_t)B * Hv * ((T + C - 1) / C); }
 inline size_t scratch_bytes(int B, int T, int Hv) {
-  const size_t nC = (size_t)(T + C - 1) / C;
-  return (size_t)B * Hv * nC * kPwBytes;
+  return records(B, T, Hv) * kPwBytes + ((records(B, T, Hv) * 4 + 255) & ~(size_t)255);
 }
 
 // Per device: a high- and a low-priority stream and two events for the split launch below, and
@@ -1262,15 +1304,18 @@ inline Split* split_for_device() {   // call with split_mutex() held
   return &p;
 }
 
-// The two kernels of one call on `st`.  `nseq` sequences.  Fixed length (cu == nullptr): [nseq, T,
-// ...] tensors, max_len = T.  Packed: [T, ...] tensors of T tokens in all, sequence s at cu[s] ..
-// cu[s + 1] - 1 (device offsets), none longer than max_len.  `pw`: nseq * Hv * ceil(max_len / 64)
-// records.
+// The two kernels of one call on `st` (`parts`: kPre, kRec or both).  `nseq` sequences.  Fixed
+// length (cu == nullptr): [nseq, T, ...] tensors, max_len = T.  Packed: [T, ...] tensors of T
+// tokens in all, sequence s at cu[s] .. cu[s + 1] - 1 (device offsets), none longer than max_len.
+// `pw`: nseq * Hv * ceil(max_len / 64) records.  `ready` (or nullptr): one zeroed flag per record,
+// through which a recurrence launched before its pre-pass (on another stream) follows it.
+constexpr int kPre = 1, kRec = 2;
 template <typename Tout>
 gdn_status launch_one(const void* q, const void* k, const void* v, const float* la,
                       const float* be, const float* S0, Tout* o, float* S_T, int nseq, int T,
                       int Hk, int Hv, float scale, uint8_t* pw, const int* cu, int max_len,
-                      cudaStream_t st, cudaEvent_t ev_after_pre) {
+                      cudaStream_t st, cudaEvent_t ev_after_pre, int* ready = nullptr,
+                      int parts = kPre | kRec) {
   const int mapB = cu ? 1 : nseq;
   CUtensorMap mq, mk, mo;
   if (!make_tile_map(&mq, q, Hk, T, mapB, false) || !make_tile_map(&mk, k, Hk, T, mapB, false) ||
@@ -1285,25 +1330,32 @@ gdn_status launch_one(const void* q, const void* k, const void* v, const float* 
     return GDN_ERR_CUDA;
   const long grid = (long)nseq * Hv;
   const int nCmax = (max_len + C - 1) / C;
-  if (grid > 0x7fffffffL || Hv > 65535 || nseq > 65535) return GDN_ERR_UNSUPPORTED;
+  if (grid > 0x7fffffffL || nCmax > 65535 || nseq > 65535) return GDN_ERR_UNSUPPORTED;
   if (nCmax == 0) return GDN_OK;
-  pw_prepass_kernel<<<dim3(nCmax, Hv, nseq), PP_THREADS, PP_SMEM, st>>>(
-      mq, mk, la, be, pw, T, Hk, Hv, scale, cu, max_len);
-  if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+  if (parts & kPre) {   // head-fastest: every head's chunk c before any head's chunk c + 1
+    pw_prepass_kernel<<<dim3(Hv, nCmax, nseq), PP_THREADS, PP_SMEM, st>>>(
+        mq, mk, la, be, pw, T, Hk, Hv, scale, cu, max_len, ready);
+    if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+  }
   if (ev_after_pre && cudaEventRecord(ev_after_pre, st) != cudaSuccess) return GDN_ERR_CUDA;
-  kern<<<(unsigned)grid, kThreads, SMEM_ALLOC, st>>>(mq, mk, mo,
-                                                          static_cast<const __nv_bfloat16*>(v), pw,
-                                                          S0, S_T, T, Hk, Hv, scale, cu, max_len,
-                                                          nCmax, o);
-  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+  if (parts & kRec) {
+    kern<<<(unsigned)grid, kThreads, SMEM_ALLOC, st>>>(
+        mq, mk, mo, static_cast<const __nv_bfloat16*>(v), pw, S0, S_T, T, Hk, Hv, scale, cu,
+        max_len, nCmax, o, ready);
+    if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+  }
+  return GDN_OK;
 }
 
 // One call.  When a batched call has more (batch, head) recurrences than SMs, its recurrence would
 // run in two waves with most SMs idle in the second.  The call is then split by batches: the tail
-// batches go first (their pre-pass, then their recurrence on a high-priority stream), and the
-// pre-pass of the leading batches runs on the SMs the tail's recurrence leaves free, after which
-// their recurrence fills the GPU in one wave.  Results are those of one launch (the recurrences
-// are independent); the caller's stream waits for both parts.
+// batches go first, and the pre-pass of the leading batches runs on the SMs the tail's recurrence
+// leaves free, after which their recurrence fills the GPU in one wave.  When the tail's
+// recurrences take at most a third of the SMs, the tail's recurrence is launched first (on the
+// high-priority stream) and follows its own pre-pass record by record through ready flags, so it
+// does not wait for the whole pre-pass; otherwise the tail runs its pre-pass, then its recurrence.
+// Results are those of one launch (the recurrences are independent, and the flags only order
+// reads after writes); the caller's stream waits for both parts.
 template <typename Tout>
 gdn_status launch(const void* q, const void* k, const void* v, const float* la, const float* be,
                   const float* S0, Tout* o, float* S_T, int nseq, int T, int Hk, int Hv,
@@ -1337,12 +1389,29 @@ gdn_status launch(const void* q, const void* k, const void* v, const float* la, 
             cudaStreamWaitEvent(sp->s_hi, sp->ev_fork, 0) == cudaSuccess &&
             cudaStreamWaitEvent(sp->s_lo, sp->ev_fork, 0) == cudaSuccess;
   gdn_status s = ok ? GDN_OK : GDN_ERR_CUDA;
-  if (s == GDN_OK)   // the tail: pre-pass, then its recurrence, both on the high-priority stream
-    s = launch_one<Tout>(qt, kt, vt, lat, bet, S0t, ot, STt, tail_b, T, Hk, Hv, scale, pwt,
-                         nullptr, T, sp->s_hi, sp->ev_pre);
-  // the leading batches start once the tail's pre-pass is done
-  if (s == GDN_OK && cudaStreamWaitEvent(sp->s_lo, sp->ev_pre, 0) != cudaSuccess)
-    s = GDN_ERR_CUDA;
+  if ((long)tail_b * Hv * 3 <= sp->sms) {
+    // the tail's flags (after all records) are cleared, then its recurrence starts on the
+    // high-priority stream and its pre-pass, followed by the leading batches', on the other
+    int* ready = reinterpret_cast<int*>(pw + records(nseq, T, Hv) * kPwBytes);
+    if (s == GDN_OK &&
+        (cudaMemsetAsync(ready, 0, records(tail_b, T, Hv) * 4, sp->s_hi) != cudaSuccess ||
+         cudaEventRecord(sp->ev_pre, sp->s_hi) != cudaSuccess ||
+         cudaStreamWaitEvent(sp->s_lo, sp->ev_pre, 0) != cudaSuccess))
+      s = GDN_ERR_CUDA;
+    if (s == GDN_OK)
+      s = launch_one<Tout>(qt, kt, vt, lat, bet, S0t, ot, STt, tail_b, T, Hk, Hv, scale, pwt,
+                           nullptr, T, sp->s_hi, nullptr, ready, kRec);
+    if (s == GDN_OK)
+      s = launch_one<Tout>(qt, kt, vt, lat, bet, S0t, ot, STt, tail_b, T, Hk, Hv, scale, pwt,
+                           nullptr, T, sp->s_lo, nullptr, ready, kPre);
+  } else {
+    if (s == GDN_OK)   // the tail: pre-pass, then its recurrence, both on the high-priority stream
+      s = launch_one<Tout>(qt, kt, vt, lat, bet, S0t, ot, STt, tail_b, T, Hk, Hv, scale, pwt,
+                           nullptr, T, sp->s_hi, sp->ev_pre);
+    // the leading batches start once the tail's pre-pass is done
+    if (s == GDN_OK && cudaStreamWaitEvent(sp->s_lo, sp->ev_pre, 0) != cudaSuccess)
+      s = GDN_ERR_CUDA;
+  }
   if (s == GDN_OK)
     s = launch_one<Tout>(q, k, v, la, be, S0, o, S_T, head_b, T, Hk, Hv, scale, pw, nullptr, T,
                          sp->s_lo, nullptr);
