@@ -276,6 +276,7 @@ gdn_status gdn_chunk_fwd_varlen(const void* q, const void* k, const void* v,
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(log_alpha) ||
       !aligned4(beta))
     return GDN_ERR_INVALID_ARG;
+  if (!tc_chunk_length_ok(max_seqlen)) return GDN_ERR_UNSUPPORTED;
   cudaMemPool_t pool = nullptr;
   s = scratch_pool(&pool);
   if (s != GDN_OK) return s;
@@ -351,6 +352,7 @@ gdn_status gdn_chunk_fwd_ex(const void* q, const void* k, const void* v, const f
   const bool tc_ok = tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16);
   if (variant == GDN_VARIANT_TCGEN05 && !tc_ok) return GDN_ERR_UNSUPPORTED;
   if (tc_ok && variant != GDN_VARIANT_SIMT) {
+    if (!tc_chunk_length_ok(T)) return GDN_ERR_UNSUPPORTED;
     cudaMemPool_t pool = nullptr;
     s = scratch_pool(&pool);
     if (s != GDN_OK) return s;

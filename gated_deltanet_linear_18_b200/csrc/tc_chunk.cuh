@@ -450,13 +450,12 @@ __device__ __forceinline__ void store_b_pair(uint32_t tb, int row, int n, float 
 }
 
 // grid (Hv, nCmax, sequences), 128 threads; thread r owns TMEM lane r.  CTAs past the end of
-// their sequence return at once.  With `ready`, each CTA sets ready[(s * Hv + h) * nCmax + c] to 1
-// (release) once its record is in global memory, for a recurrence that runs alongside.
+// their sequence return at once.
 __global__ void __launch_bounds__(PP_THREADS, 4)
 pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const float* __restrict__ log_alpha, const float* __restrict__ beta,
                   uint8_t* __restrict__ pw, int T, int Hk, int Hv, float scale,
-                  const int* __restrict__ cu, int max_len, int* __restrict__ ready) {
+                  const int* __restrict__ cu, int max_len) {
   GDN_TRACE_INIT;
   extern __shared__ __align__(1024) uint8_t pp_raw[];
   uint8_t* smem = pp_raw + ((1024u - (tc::smem_u32(pp_raw) & 1023u)) & 1023u);
@@ -740,14 +739,8 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
       tc::bulk_store(rec + 32768, qk + 8192, 8192);
       tc::bulk_store(rec + 40960, qk + 24576, 8192);
       tc::bulk_commit();
-      if (ready) {                                    // the record is complete, then published
-        tc::bulk_wait_all();
-        tc::fence_proxy_async_global();
-        tc::st_release_gpu(ready + ((long)sq * Hv + h) * nC + c, 1);
-      } else {
-        tc::bulk_wait_read_all();                     // every source read; the writes complete
-      }                                               // on their own
-    }
+      tc::bulk_wait_read_all();                       // every source read; the writes complete
+    }                                                 // on their own
   }
   GDN_TRACE_PP(8);
   GDN_TRACE_PP(9);
@@ -769,8 +762,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
                     const __grid_constant__ CUtensorMap tmo, const __nv_bfloat16* __restrict__ v,
                     const uint8_t* __restrict__ pw, const float* __restrict__ S0,
                     float* __restrict__ S_T, int T, int Hk, int Hv, float scale,
-                    const int* __restrict__ cu, int max_len, int nCmax, Tout* __restrict__ o,
-                    const int* __restrict__ ready) {
+                    const int* __restrict__ cu, int max_len, int nCmax, Tout* __restrict__ o) {
   constexpr bool kF32 = sizeof(Tout) == 4;
   // X takes M as a hi + lo bf16 pair when o is fp32 (the layer, whose gated norm magnifies o's
   // error); a bf16 o carries its own rounding, and one round-to-nearest bf16 copy of M suffices.
@@ -791,9 +783,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   const bool packed = cu != nullptr;
   const long head = (long)bq * Hv + h;
   const uint8_t* pw_head = pw + head * nCmax * (long)kPwBytes;
-  // with `ready`, record c of this head may still be being written by a pre-pass that runs
-  // alongside: every reader of it first waits for its flag (acquire)
-  const int* ready_head = ready ? ready + head * nCmax : nullptr;
   if (nC == 0) {   // an empty sequence: the state passes through (uniform, before any barrier)
     if (S_T)
       for (int i = threadIdx.x; i < 128 * 128 / 4; i += blockDim.x)
@@ -855,10 +844,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         armed_qk = c;
         const uint8_t* src = pw_head + (long)c * kPwBytes;
         const uint32_t slot = sb + OFF_PW + s * PW_SLOT;
-        if (ready_head) {
-          if (!(ok = tc::flag_wait(ready_head + c, abort_flag, kBudget))) break;
-          tc::fence_proxy_async_global();
-        }
         if (c >= 2) ok = tc::mbar_wait(bar(B_W_EMPTY + s), ((c >> 1) - 1) & 1, abort_flag, kBudget);
         if (!ok) break;
         tc::mbar_arrive_expect_tx(bar(B_W_FULL + s), 32768);
@@ -955,8 +940,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     }
   } else if (warp == 2) {
     // ------------------------------- gamma ---------------------------------------------------
-    // gamma_t of chunk c into ring slot c & 1 (after the record's ready flag, when there is one),
-    // so that the chain reads it from shared memory
+    // gamma_t of chunk c into ring slot c & 1, so that the chain reads it from shared memory
+    // (off the chain's critical path) instead of global memory
     const float* gsrc = reinterpret_cast<const float*>(pw_head + kPwTiles);
     for (int c = 0; c < nC; ++c) {
       const int s = c & 1;
@@ -964,9 +949,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       if (lane == 0 && c >= 2)
         ok = tc::mbar_wait(bar(B_G_EMPTY + s), ((c >> 1) - 1) & 1, abort_flag, kBudget);
       __syncwarp();                                    // the slot's readers before its writers
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (ok && ready_head) ok = tc::flag_wait(ready_head + c, abort_flag, kBudget);  // each lane
-      if (!__all_sync(0xffffffffu, ok)) break;
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       const float2 g = reinterpret_cast<const float2*>(gsrc + (long)c * (kPwBytes / 4))[lane];
       *reinterpret_cast<float2*>(smem + OFF_GAM + s * 256 + 8 * lane) = g;
       __syncwarp();
@@ -1266,11 +1249,10 @@ inline bool make_tile_map(CUtensorMap* m, const void* base, int H, int T, int B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Bytes of the operand hand-over buffer between the pre-pass and the recurrence: the records,
-// then one int32 ready flag per record (used when a recurrence runs alongside its pre-pass).
-inline size_t records(int B, int T, int Hv) { return (size_t)B * Hv * ((T + C - 1) / C); }
+// Bytes of the operand hand-over buffer between the pre-pass and the recurrence.
 inline size_t scratch_bytes(int B, int T, int Hv) {
-  return records(B, T, Hv) * kPwBytes + ((records(B, T, Hv) * 4 + 255) & ~(size_t)255);
+  const size_t nC = (size_t)(T + C - 1) / C;
+  return (size_t)B * Hv * nC * kPwBytes;
 }
 
 // Per device: a high- and a low-priority stream and two events for the split launch below, and
@@ -1304,18 +1286,15 @@ inline Split* split_for_device() {   // call with split_mutex() held
   return &p;
 }
 
-// The two kernels of one call on `st` (`parts`: kPre, kRec or both).  `nseq` sequences.  Fixed
-// length (cu == nullptr): [nseq, T, ...] tensors, max_len = T.  Packed: [T, ...] tensors of T
-// tokens in all, sequence s at cu[s] .. cu[s + 1] - 1 (device offsets), none longer than max_len.
-// `pw`: nseq * Hv * ceil(max_len / 64) records.  `ready` (or nullptr): one zeroed flag per record,
-// through which a recurrence launched before its pre-pass (on another stream) follows it.
-constexpr int kPre = 1, kRec = 2;
+// The two kernels of one call on `st`.  `nseq` sequences.  Fixed length (cu == nullptr): [nseq, T,
+// ...] tensors, max_len = T.  Packed: [T, ...] tensors of T tokens in all, sequence s at cu[s] ..
+// cu[s + 1] - 1 (device offsets), none longer than max_len.  `pw`: nseq * Hv * ceil(max_len / 64)
+// records.  The recurrence reads the pre-pass's records only after it in stream order.
 template <typename Tout>
 gdn_status launch_one(const void* q, const void* k, const void* v, const float* la,
                       const float* be, const float* S0, Tout* o, float* S_T, int nseq, int T,
                       int Hk, int Hv, float scale, uint8_t* pw, const int* cu, int max_len,
-                      cudaStream_t st, cudaEvent_t ev_after_pre, int* ready = nullptr,
-                      int parts = kPre | kRec) {
+                      cudaStream_t st, cudaEvent_t ev_after_pre) {
   const int mapB = cu ? 1 : nseq;
   CUtensorMap mq, mk, mo;
   if (!make_tile_map(&mq, q, Hk, T, mapB, false) || !make_tile_map(&mk, k, Hk, T, mapB, false) ||
@@ -1332,34 +1311,28 @@ gdn_status launch_one(const void* q, const void* k, const void* v, const float* 
   const int nCmax = (max_len + C - 1) / C;
   if (grid > 0x7fffffffL || nCmax > 65535 || nseq > 65535) return GDN_ERR_UNSUPPORTED;
   if (nCmax == 0) return GDN_OK;
-  if (parts & kPre) {   // head-fastest: every head's chunk c before any head's chunk c + 1
-    pw_prepass_kernel<<<dim3(Hv, nCmax, nseq), PP_THREADS, PP_SMEM, st>>>(
-        mq, mk, la, be, pw, T, Hk, Hv, scale, cu, max_len, ready);
-    if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
-  }
+  // head-fastest: the value heads that share a key head's Q/K tiles run side by side
+  pw_prepass_kernel<<<dim3(Hv, nCmax, nseq), PP_THREADS, PP_SMEM, st>>>(
+      mq, mk, la, be, pw, T, Hk, Hv, scale, cu, max_len);
+  if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
   if (ev_after_pre && cudaEventRecord(ev_after_pre, st) != cudaSuccess) return GDN_ERR_CUDA;
-  if (parts & kRec) {
-    kern<<<(unsigned)grid, kThreads, SMEM_ALLOC, st>>>(
-        mq, mk, mo, static_cast<const __nv_bfloat16*>(v), pw, S0, S_T, T, Hk, Hv, scale, cu,
-        max_len, nCmax, o, ready);
-    if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
-  }
-  return GDN_OK;
+  kern<<<(unsigned)grid, kThreads, SMEM_ALLOC, st>>>(
+      mq, mk, mo, static_cast<const __nv_bfloat16*>(v), pw, S0, S_T, T, Hk, Hv, scale, cu,
+      max_len, nCmax, o);
+  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 // One call.  When a batched call has more (batch, head) recurrences than SMs, its recurrence would
 // run in two waves with most SMs idle in the second.  The call is then split by batches: the tail
-// batches go first, and the pre-pass of the leading batches runs on the SMs the tail's recurrence
-// leaves free, after which their recurrence fills the GPU in one wave.  When the tail's
-// recurrences take at most a third of the SMs, the tail's recurrence is launched first (on the
-// high-priority stream) and follows its own pre-pass record by record through ready flags, so it
-// does not wait for the whole pre-pass; otherwise the tail runs its pre-pass, then its recurrence.
-// Results are those of one launch (the recurrences are independent, and the flags only order
-// reads after writes); the caller's stream waits for both parts.
+// batches go first (their pre-pass, then their recurrence on a high-priority stream), and the
+// pre-pass of the leading batches runs on the SMs the tail's recurrence leaves free, after which
+// their recurrence fills the GPU in one wave.  Results are those of one launch (the recurrences
+// are independent); the caller's stream waits for both parts.
 template <typename Tout>
 gdn_status launch(const void* q, const void* k, const void* v, const float* la, const float* be,
                   const float* S0, Tout* o, float* S_T, int nseq, int T, int Hk, int Hv,
                   float scale, uint8_t* pw, const int* cu, int max_len, cudaStream_t st) {
+  if ((max_len + C - 1) / C > 65535) return GDN_ERR_UNSUPPORTED;   // chunks index a grid's y
   std::unique_lock<std::mutex> lock(split_mutex());
   Split* sp = split_for_device();
   if (!sp) return GDN_ERR_CUDA;
@@ -1389,29 +1362,12 @@ gdn_status launch(const void* q, const void* k, const void* v, const float* la, 
             cudaStreamWaitEvent(sp->s_hi, sp->ev_fork, 0) == cudaSuccess &&
             cudaStreamWaitEvent(sp->s_lo, sp->ev_fork, 0) == cudaSuccess;
   gdn_status s = ok ? GDN_OK : GDN_ERR_CUDA;
-  if ((long)tail_b * Hv * 3 <= sp->sms) {
-    // the tail's flags (after all records) are cleared, then its recurrence starts on the
-    // high-priority stream and its pre-pass, followed by the leading batches', on the other
-    int* ready = reinterpret_cast<int*>(pw + records(nseq, T, Hv) * kPwBytes);
-    if (s == GDN_OK &&
-        (cudaMemsetAsync(ready, 0, records(tail_b, T, Hv) * 4, sp->s_hi) != cudaSuccess ||
-         cudaEventRecord(sp->ev_pre, sp->s_hi) != cudaSuccess ||
-         cudaStreamWaitEvent(sp->s_lo, sp->ev_pre, 0) != cudaSuccess))
-      s = GDN_ERR_CUDA;
-    if (s == GDN_OK)
-      s = launch_one<Tout>(qt, kt, vt, lat, bet, S0t, ot, STt, tail_b, T, Hk, Hv, scale, pwt,
-                           nullptr, T, sp->s_hi, nullptr, ready, kRec);
-    if (s == GDN_OK)
-      s = launch_one<Tout>(qt, kt, vt, lat, bet, S0t, ot, STt, tail_b, T, Hk, Hv, scale, pwt,
-                           nullptr, T, sp->s_lo, nullptr, ready, kPre);
-  } else {
-    if (s == GDN_OK)   // the tail: pre-pass, then its recurrence, both on the high-priority stream
-      s = launch_one<Tout>(qt, kt, vt, lat, bet, S0t, ot, STt, tail_b, T, Hk, Hv, scale, pwt,
-                           nullptr, T, sp->s_hi, sp->ev_pre);
-    // the leading batches start once the tail's pre-pass is done
-    if (s == GDN_OK && cudaStreamWaitEvent(sp->s_lo, sp->ev_pre, 0) != cudaSuccess)
-      s = GDN_ERR_CUDA;
-  }
+  if (s == GDN_OK)   // the tail: pre-pass, then its recurrence, both on the high-priority stream
+    s = launch_one<Tout>(qt, kt, vt, lat, bet, S0t, ot, STt, tail_b, T, Hk, Hv, scale, pwt,
+                         nullptr, T, sp->s_hi, sp->ev_pre);
+  // the leading batches start once the tail's pre-pass is done
+  if (s == GDN_OK && cudaStreamWaitEvent(sp->s_lo, sp->ev_pre, 0) != cudaSuccess)
+    s = GDN_ERR_CUDA;
   if (s == GDN_OK)
     s = launch_one<Tout>(q, k, v, la, be, S0, o, S_T, head_b, T, Hk, Hv, scale, pw, nullptr, T,
                          sp->s_lo, nullptr);
@@ -1434,6 +1390,9 @@ extern "C" GDN_API void gdn_debug_set_trace(void* p) {
 inline bool tc_chunk_supported(int dk, int dv, int chunk, bool bf16) {
   return bf16 && dk == 128 && dv == 128 && chunk == tcf::C;
 }
+
+// Sequences of up to 65535 chunks (the pre-pass's grid holds the chunk index in y).
+inline bool tc_chunk_length_ok(long max_len) { return (max_len + tcf::C - 1) / tcf::C <= 65535; }
 
 // Scratch bytes of the tensor-core forward (the pre-pass's operand hand-over buffer).
 inline size_t tc_chunk_scratch_bytes(int B, int T, int Hv) { return tcf::scratch_bytes(B, T, Hv); }

@@ -81,33 +81,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-// Orders this thread's global-memory accesses of the async proxy (bulk copies) against its
-// generic-proxy accesses.
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release_gpu(int* p, int v) {
-  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-// Bounded wait for a nonzero global flag (acquire), with mbar_wait's abort and budget rules.
-__device__ __forceinline__ bool flag_wait(const int* flag, volatile int* abort,
-                                          uint64_t budget_cycles) {
-  if (ld_acquire_gpu(flag)) return true;
-  const long long t0 = clock64();
-  for (;;) {
-    if (ld_acquire_gpu(flag)) return true;
-    if (*abort) return false;
-    if ((uint64_t)(clock64() - t0) > budget_cycles) {
-      *abort = 1;
-      return false;
-    }
-  }
-}
 __device__ __forceinline__ void named_bar(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

@@ -110,7 +110,8 @@ GDN_API gdn_status gdn_wait_timeout_selftest(long long budget_cycles, gdn_stream
  * The tensor-core family (bf16, d_k = d_v = 128, chunk 64) first computes every chunk's
  * state-independent operands (P T_b and (diag(ktil) K)^T T_b as bf16 hi/lo tiles, and gamma) in a
  * pre-pass and hands them to the recurrence through a device buffer of
- * B * Hv * ceil(T/64) * 49408 bytes;
+ * B * Hv * ceil(T/64) * 49408 bytes (T up to 65535 chunks, 4,194,240 tokens, else
+ * GDN_ERR_UNSUPPORTED before any work);
  * that buffer is taken from a memory pool of the library (one per device, stream-ordered, kept
  * between calls) and given back at the end of the call on `stream`.  When B * Hv exceeds the
  * device's SM count the call runs in two parts (the last batches first) on two internal streams
