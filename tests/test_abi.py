@@ -148,3 +148,16 @@ def test_layer_validation(L):
     # misaligned workspace
     assert L.gdn_layer_fwd(*args, P(0x1010), 1 << 30, 1, 8, 2, 4, 16, 16, 16, 1.0, 1e-6, 1e-5,
                            1, None) == 1
+
+
+def test_tensor_core_forward_rejects_more_than_65535_chunks(L):
+    """The tensor-core family takes sequences of up to 65535 chunks of 64 tokens; a longer one
+    returns GDN_ERR_UNSUPPORTED (2) before any allocation or launch (the pointers are fakes)."""
+    longest = 65535 * 64
+    t8 = [FAKE] * 8
+    for variant in (0, 2):                                         # auto, tcgen05
+        assert L.gdn_chunk_fwd_ex(*t8, 1, longest + 1, 16, 48, 128, 128, 64, 1.0, 1, variant,
+                                  None) == 2
+    t6 = [FAKE] * 6
+    assert L.gdn_chunk_fwd_varlen(*t6, 1, longest + 1, FAKE, FAKE, FAKE, longest + 1, 16, 48,
+                                  128, 128, 64, 1.0, 1, None) == 2
