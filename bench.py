@@ -468,11 +468,16 @@ def dist_setup(n_gpus):
 
 def tc_launches_per_call(w: gi.Workload, dev, variant: str) -> int:
     """Kernels one forward call launches: the SIMT forward one; the tensor-core forward two (the
-    operand pre-pass, then the recurrence), or four when the library splits a batched call whose
-    B * Hv recurrences exceed the SM count into tail and leading batches."""
+    operand pre-pass, then the recurrence), four when the library splits a batched call whose
+    B * Hv recurrences exceed the SM count into tail and leading batches, or two per range of 128
+    chunks when it runs a single long sequence (B = 1, at least 256 chunks, 2 Hv <= SMs) in
+    ranges."""
     if variant != "tcgen05":
         return 1
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    n_chunks = (w.T + 63) // 64
+    if w.B == 1 and 2 * w.Hv <= sms and n_chunks >= 256:
+        return 2 * ((n_chunks + 127) // 128)
     head_b = sms // w.Hv
     split = w.B >= 2 and w.B * w.Hv > sms and 1 <= head_b < w.B
     return 4 if split else 2

@@ -42,6 +42,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -200,8 +201,8 @@ __device__ __forceinline__ void st_frag(uint32_t B, int n0, int g, int t, const 
   sts2(at(B, g + 8, n0 + 2 * t), c[2], c[3]);
 }
 
-// T = (I + A)^-1 for a 64 x 64 strictly lower A (128 threads = 4 warps, named barriers 1 and 3), blocked
-// by 16:  D_b = (I + A_bb)^-1 by forward substitution (one column per thread);  At_ik = D_i A_ik;
+// T = (I + A)^-1 for a 64 x 64 strictly lower A (128 threads = 4 warps, named barriers 1 and 3),
+// blocked by 16:  D_b = (I + A_bb)^-1 by forward substitution (one column per thread);  At_ik = D_i A_ik;
 // U = (I + At)^-1 (U_ii = I; At is block-nilpotent, so U is closed-form in At's blocks);
 // T_ik = U_ik D_k.   (I + A = blockdiag(I + A_bb) (I + At), so T = U D.)  The block products run
 // as warp MMAs on 16 x 8 half blocks.  On return the off-diagonal blocks of T are in `tv`: item m
@@ -415,10 +416,11 @@ __device__ __forceinline__ SeqSpan seq_span(const int* __restrict__ cu, int s, i
 // ahead of the recurrence, on the tensor cores: S = [Q; K] K^T (bf16 MMA into TMEM), P and A from
 // S with the gates (one TMEM row per thread), the blocked solve, then PT = P T_b and, through the
 // same pair of operand tiles once PT has read them, W = K^T (ktil T_b), as bf16 MMAs on hi + lo
-// splits (hi.hi + lo.hi + hi.lo for PT; K is exact, so two terms for W).  The result goes to HBM as the recurrence's MMA operands themselves: per
-// chunk 48 KB of 128-byte-swizzled K-major bf16 tiles, PT hi [64 rows][128 B], PT lo, W hi [128
-// rows][128 B], W lo, followed by gamma_t = exp(G_t) (64 fp32).  A chunk whose P or A holds a NaN
-// or an infinity gets +inf in every tile, so the recurrence still sees a non-finite value.
+// splits (hi.hi + lo.hi + hi.lo for PT; K is exact, so two terms for W).  The result goes to HBM
+// as the recurrence's MMA operands themselves: per chunk 48 KB of 128-byte-swizzled K-major bf16
+// tiles, PT hi [64 rows][128 B], PT lo, W hi [128 rows][128 B], W lo, followed by
+// gamma_t = exp(G_t) (64 fp32).  A chunk whose P or A holds a NaN or an infinity gets +inf in
+// every tile, so the recurrence still sees a non-finite value.
 constexpr int kPwTiles = 49152;              // the four operand tiles of a chunk
 constexpr int kPwBytes = kPwTiles + 256;     // + gamma_t = exp(G_t), 64 fp32
 constexpr int PP_THREADS = 128;
@@ -1249,10 +1251,18 @@ inline bool make_tile_map(CUtensorMap* m, const void* base, int H, int T, int B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Bytes of the operand hand-over buffer between the pre-pass and the recurrence.
+// A single sequence of at least 2 * kRangeChunks chunks whose recurrences leave at least half of
+// the SMs idle runs in ranges of kRangeChunks chunks (see launch()).
+constexpr int kRangeChunks = 128;
+inline bool ranged(int nseq, int T, int Hv, int sms) {
+  return nseq == 1 && 2L * Hv <= sms && (T + C - 1) / C >= 2 * kRangeChunks;
+}
+// Bytes of the operand hand-over buffer between the pre-pass and the recurrence; for sequences
+// long enough to run in ranges, two fp32 states follow the records (the state between ranges).
 inline size_t scratch_bytes(int B, int T, int Hv) {
   const size_t nC = (size_t)(T + C - 1) / C;
-  return (size_t)B * Hv * nC * kPwBytes;
+  const size_t states = nC >= 2 * (size_t)kRangeChunks ? 2 * (size_t)B * Hv * 128 * 128 * 4 : 0;
+  return (size_t)B * Hv * nC * kPwBytes + states;
 }
 
 // Per device: a high- and a low-priority stream and two events for the split launch below, and
@@ -1289,12 +1299,14 @@ inline Split* split_for_device() {   // call with split_mutex() held
 // The two kernels of one call on `st`.  `nseq` sequences.  Fixed length (cu == nullptr): [nseq, T,
 // ...] tensors, max_len = T.  Packed: [T, ...] tensors of T tokens in all, sequence s at cu[s] ..
 // cu[s + 1] - 1 (device offsets), none longer than max_len.  `pw`: nseq * Hv * ceil(max_len / 64)
-// records.  The recurrence reads the pre-pass's records only after it in stream order.
+// records.  The recurrence reads the pre-pass's records only after it in stream order.  `parts`:
+// kPre, kRec or both; a recurrence launched alone must follow its pre-pass on `st` by an event.
+constexpr int kPre = 1, kRec = 2;
 template <typename Tout>
 gdn_status launch_one(const void* q, const void* k, const void* v, const float* la,
                       const float* be, const float* S0, Tout* o, float* S_T, int nseq, int T,
                       int Hk, int Hv, float scale, uint8_t* pw, const int* cu, int max_len,
-                      cudaStream_t st, cudaEvent_t ev_after_pre) {
+                      cudaStream_t st, cudaEvent_t ev_after_pre, int parts = kPre | kRec) {
   const int mapB = cu ? 1 : nseq;
   CUtensorMap mq, mk, mo;
   if (!make_tile_map(&mq, q, Hk, T, mapB, false) || !make_tile_map(&mk, k, Hk, T, mapB, false) ||
@@ -1311,15 +1323,20 @@ gdn_status launch_one(const void* q, const void* k, const void* v, const float* 
   const int nCmax = (max_len + C - 1) / C;
   if (grid > 0x7fffffffL || nCmax > 65535 || nseq > 65535) return GDN_ERR_UNSUPPORTED;
   if (nCmax == 0) return GDN_OK;
-  // head-fastest: the value heads that share a key head's Q/K tiles run side by side
-  pw_prepass_kernel<<<dim3(Hv, nCmax, nseq), PP_THREADS, PP_SMEM, st>>>(
-      mq, mk, la, be, pw, T, Hk, Hv, scale, cu, max_len);
-  if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+  if (parts & kPre) {
+    // head-fastest: the value heads that share a key head's Q/K tiles run side by side
+    pw_prepass_kernel<<<dim3(Hv, nCmax, nseq), PP_THREADS, PP_SMEM, st>>>(
+        mq, mk, la, be, pw, T, Hk, Hv, scale, cu, max_len);
+    if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+  }
   if (ev_after_pre && cudaEventRecord(ev_after_pre, st) != cudaSuccess) return GDN_ERR_CUDA;
-  kern<<<(unsigned)grid, kThreads, SMEM_ALLOC, st>>>(
-      mq, mk, mo, static_cast<const __nv_bfloat16*>(v), pw, S0, S_T, T, Hk, Hv, scale, cu,
-      max_len, nCmax, o);
-  return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+  if (parts & kRec) {
+    kern<<<(unsigned)grid, kThreads, SMEM_ALLOC, st>>>(
+        mq, mk, mo, static_cast<const __nv_bfloat16*>(v), pw, S0, S_T, T, Hk, Hv, scale, cu,
+        max_len, nCmax, o);
+    if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+  }
+  return GDN_OK;
 }
 
 // One call.  When a batched call has more (batch, head) recurrences than SMs, its recurrence would
@@ -1336,6 +1353,42 @@ gdn_status launch(const void* q, const void* k, const void* v, const float* la, 
   std::unique_lock<std::mutex> lock(split_mutex());
   Split* sp = split_for_device();
   if (!sp) return GDN_ERR_CUDA;
+  if (!cu && ranged(nseq, T, Hv, sp->sms)) {
+    // Ranges of kRangeChunks chunks: every pre-pass on the low-priority stream, one after the
+    // other; the recurrence of range r on the high-priority stream once pre-pass r is done and
+    // after recurrence r - 1, starting from its final state.  Pre-pass r + 1 thus runs on the
+    // SMs recurrence r leaves idle.  Splitting at chunk boundaries gives the one-launch result.
+    const int nC = (T + C - 1) / C, nR = (nC + kRangeChunks - 1) / kRangeChunks;
+    float* mid[2];
+    mid[0] = reinterpret_cast<float*>(pw + (size_t)Hv * nC * kPwBytes);
+    mid[1] = mid[0] + (size_t)Hv * 128 * 128;
+    bool ok = cudaEventRecord(sp->ev_fork, st) == cudaSuccess &&
+              cudaStreamWaitEvent(sp->s_hi, sp->ev_fork, 0) == cudaSuccess &&
+              cudaStreamWaitEvent(sp->s_lo, sp->ev_fork, 0) == cudaSuccess;
+    gdn_status s = ok ? GDN_OK : GDN_ERR_CUDA;
+    for (int r = 0; r < nR && s == GDN_OK; ++r) {
+      const long t0 = (long)r * kRangeChunks * C;
+      const int Tr = (int)std::min<long>(T - t0, (long)kRangeChunks * C);
+      const auto* bq = static_cast<const __nv_bfloat16*>(q) + t0 * Hk * 128;
+      const auto* bk = static_cast<const __nv_bfloat16*>(k) + t0 * Hk * 128;
+      const auto* bv = static_cast<const __nv_bfloat16*>(v) + t0 * Hv * 128;
+      const float* S0r = r == 0 ? S0 : mid[(r - 1) & 1];
+      float* STr = r == nR - 1 ? S_T : mid[r & 1];
+      uint8_t* pwr = pw + (size_t)Hv * r * kRangeChunks * kPwBytes;
+      s = launch_one<Tout>(bq, bk, bv, la + t0 * Hv, be + t0 * Hv, S0r, o + t0 * Hv * 128, STr, 1,
+                           Tr, Hk, Hv, scale, pwr, nullptr, Tr, sp->s_lo, sp->ev_pre, kPre);
+      if (s == GDN_OK && cudaStreamWaitEvent(sp->s_hi, sp->ev_pre, 0) != cudaSuccess)
+        s = GDN_ERR_CUDA;
+      if (s == GDN_OK)
+        s = launch_one<Tout>(bq, bk, bv, la + t0 * Hv, be + t0 * Hv, S0r, o + t0 * Hv * 128, STr,
+                             1, Tr, Hk, Hv, scale, pwr, nullptr, Tr, sp->s_hi, nullptr, kRec);
+    }
+    const bool joined = cudaEventRecord(sp->ev_hi, sp->s_hi) == cudaSuccess &&
+                        cudaEventRecord(sp->ev_lo, sp->s_lo) == cudaSuccess &&
+                        cudaStreamWaitEvent(st, sp->ev_hi, 0) == cudaSuccess &&
+                        cudaStreamWaitEvent(st, sp->ev_lo, 0) == cudaSuccess;
+    return s != GDN_OK ? s : (joined ? GDN_OK : GDN_ERR_CUDA);
+  }
   const int head_b = sp->sms / (Hv > 0 ? Hv : 1);        // batches that fill at most one wave
   if (cu || nseq < 2 || (long)nseq * Hv <= sp->sms || head_b < 1 || head_b >= nseq) {
     lock.unlock();

@@ -116,7 +116,11 @@ GDN_API gdn_status gdn_wait_timeout_selftest(long long budget_cycles, gdn_stream
  * between calls) and given back at the end of the call on `stream`.  When B * Hv exceeds the
  * device's SM count the call runs in two parts (the last batches first) on two internal streams
  * of the library that fork from and join back into `stream`, so that the recurrence runs in one
- * wave; the results are those of one launch.
+ * wave; the results are those of one launch.  A single sequence (B = 1) of at least 256 chunks
+ * whose Hv recurrences take at most half of the SMs runs in ranges of 128 chunks on the same two
+ * streams (the pre-pass of the next range beside the recurrence of the current one, the state
+ * handed on through two fp32 states after the records, 2 * Hv * 64 KiB more scratch); the
+ * results are again those of one launch.
  */
 GDN_API gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v,
                          const float *log_alpha, const float *beta, const float *S0,
