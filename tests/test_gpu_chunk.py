@@ -95,6 +95,27 @@ def test_split_run_equals_one_run():
     assert rel_rms(S, np64(sT)) <= 1e-3
 
 
+def test_long_sequence_in_ranges_equals_chained_calls():
+    """A single sequence of 259 chunks runs in ranges of 128 chunks (three, the last ragged); it
+    gives bit for bit what three calls give that each run in one launch, chained by S_T -> S0."""
+    w = gi.WORKLOADS["prefill"].with_sizes(B=1, T=128 * 64 * 2 + 3 * 64 - 20, Hk=4, Hv=12,
+                                           s0_std=0.02, seed=13)
+    d = to_dev(gi.make_inputs(w))
+    o, sT = gdn.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"], chunk=64)
+    S, parts = d["S0"], []
+    for t0 in range(0, w.T, 128 * 64):
+        sl = slice(t0, min(w.T, t0 + 128 * 64))
+        oc, S = gdn.chunk_fwd(d["q"][:, sl].contiguous(), d["k"][:, sl].contiguous(),
+                              d["v"][:, sl].contiguous(), d["log_alpha"][:, sl].contiguous(),
+                              d["beta"][:, sl].contiguous(), S, chunk=64)
+        parts.append(oc)
+    torch.cuda.synchronize()
+    gdn.check_error()
+    assert len(parts) == 3
+    assert torch.equal(torch.cat(parts, dim=1), o)
+    assert torch.equal(S, sT)
+
+
 def test_chunk_size_invariance_fp32():
     w = gi.WORKLOADS["tiny_fp32"].with_sizes(B=1, T=150, Hk=1, Hv=2, dk=64, dv=64, s0_std=0.1,
                                              seed=5)
