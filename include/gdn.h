@@ -119,8 +119,8 @@ GDN_API gdn_status gdn_wait_timeout_selftest(long long budget_cycles, gdn_stream
  * wave; the results are those of one launch.  A single sequence (B = 1) of at least 256 chunks
  * whose Hv recurrences take at most half of the SMs runs in ranges of 128 chunks on the same two
  * streams (the pre-pass of the next range beside the recurrence of the current one, the state
- * handed on through two fp32 states after the records, 2 * Hv * 64 KiB more scratch); the
- * results are again those of one launch.
+ * handed on through two fp32 states after the records); the results are again those of one
+ * launch.  The buffer holds those 2 * B * Hv * 64 KiB whenever T reaches 256 chunks.
  */
 GDN_API gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v,
                          const float *log_alpha, const float *beta, const float *S0,
