@@ -206,18 +206,44 @@ def time_steps(fn, steps: int, warmup: int, flush: Flusher, launches_per_step: i
 # workloads
 # ------------------------------------------------------------------------------------------------
 
-def prefill_fn(gdn, d, w):
-    o = torch.empty_like(d["v"])
-    sT = torch.empty(w.B, w.Hv, w.dk, w.dv, device=d["v"].device, dtype=torch.float32)
+def workspace_for(gdn, w, dev):
+    """The caller-owned scratch of the chunked forward, allocated once (outside any timing)."""
+    need = gdn.chunk_fwd_workspace_bytes(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv, w.chunk,
+                                         w.torch_dtype)
+    return torch.empty(need, device=dev, dtype=torch.uint8) if need else None
+
+
+def prefill_fn(gdn, d, w, out_dtype=None):
+    dev = d["v"].device
+    o = torch.empty(d["v"].shape, device=dev, dtype=out_dtype or d["v"].dtype)
+    sT = torch.empty(w.B, w.Hv, w.dk, w.dv, device=dev, dtype=torch.float32)
+    ws = workspace_for(gdn, w, dev)
 
     def step():
         gdn.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
-                      chunk=w.chunk, out=o, state_out=sT)
+                      chunk=w.chunk, out=o, state_out=sT, workspace=ws)
     return step
 
 
 def to_dev(x, dev):
     return {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+
+
+def roofline_block(B, F, t, peaks, kernel, traffic=None, peak_key="hbm_gbs"):
+    """Achieved work per second of one call against the measured peaks; the bound is the larger
+    of the HBM time and the dense bf16 time of the algorithmic bytes and FLOPs."""
+    t_hbm = B / (peaks[peak_key] * 1e9)
+    t_ten = F / (peaks["bf16_tflops"] * 1e12) if F else 0.0
+    hbm_bound = t_hbm >= t_ten
+    r = {"bound": "hbm" if hbm_bound else "tensor",
+         "achieved": (B / t / 1e9) if hbm_bound else (F / t / 1e12),
+         "peak": peaks[peak_key] if hbm_bound else peaks["bf16_tflops"],
+         "unit": "GB/s" if hbm_bound else "TFLOP/s", "traffic": traffic, "kernel": kernel,
+         "algorithmic_bytes": B, "algorithmic_flops": F,
+         "peak_source": peaks.get("source", "measured") + " burst",
+         "other_bound_frac": (t_ten / t) if hbm_bound else (t_hbm / t)}
+    r["frac"] = r["achieved"] / r["peak"]
+    return r
 
 
 def bench_prefill_like(gdn, name, dev, steps, warmup, flush, peaks):
@@ -228,10 +254,14 @@ def bench_prefill_like(gdn, name, dev, steps, warmup, flush, peaks):
     t = statistics.mean(ms) / 1e3
     B = fwd_bytes(w, x["S0"] is not None, True)
     F = fwd_flops(w)
-    t_roof = max(B / (peaks["hbm_gbs"] * 1e9), F / (peaks["bf16_tflops"] * 1e12))
+    roof = roofline_block(B, F, t, peaks, "gdn_chunk_fwd_tc",
+                          recorded_traffic("gdn_chunk_fwd_tc", name))
     return w, x, d, ms, {
-        "value": w.B * w.T / t, "unit": "tokens/s", "ms_per_step": t * 1e3,
-        "hbm_gbs": B / t / 1e9, "tflops": F / t / 1e12, "roofline_frac": t_roof / t,
+        "value": w.B * w.T / t, "unit": "tokens/s", "ms_per_step": t * 1e3, "steps": steps,
+        "hbm_gbs": B / t / 1e9, "tflops": F / t / 1e12, "roofline_frac": roof["frac"],
+        "roofline": roof,
+        "gpu_launches_per_call": gdn.chunk_fwd_launches(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv,
+                                                        w.chunk, w.torch_dtype),
         "variant": gdn.chunk_fwd_variant(w.dk, w.dv, w.chunk, w.torch_dtype),
         "workload": workload_name(w)}
 
@@ -329,9 +359,12 @@ def bench_varlen(gdn, dev, warmup, flush, peaks, steps=10):
     S0 = (torch.randn(32, w.Hv, w.dk, w.dv, generator=g) * 0.02).to(dev)
     cu = torch.cat([torch.zeros(1, dtype=torch.int64), lengths.cumsum(0)]).to(torch.int32).to(dev)
     o = torch.empty_like(v)
+    need = gdn.lib().gdn_chunk_fwd_varlen_workspace_bytes(32, int(lengths.max()), w.Hk, w.Hv,
+                                                          w.dk, w.dv, w.chunk, 1)
+    ws = torch.empty(need, device=dev, dtype=torch.uint8)
 
     def step():
-        gdn.chunk_fwd_varlen(q, k, v, la, be, cu, int(lengths.max()), S0, out=o)
+        gdn.chunk_fwd_varlen(q, k, v, la, be, cu, int(lengths.max()), S0, out=o, workspace=ws)
     ms = time_steps(step, steps, warmup, flush, 2)
     gdn.check_error(dev)
     t = sum(ms) / len(ms) / 1e3
@@ -356,7 +389,7 @@ def bench_gates(gdn, dev, warmup, flush, peaks, steps=20):
             "workload": f"gates B{w.B} T{w.T} Hv{w.Hv} {w.dtype}"}
 
 
-def bench_layer(gdn, dev, warmup, flush, peaks, steps=3):
+def bench_layer(gdn, dev, warmup, flush, peaks, steps=10):
     w = gi.WORKLOADS["layer_8to1"]
     x = gi.make_layer_inputs(w)
     d = to_dev(x, dev)
@@ -373,10 +406,11 @@ def bench_layer(gdn, dev, warmup, flush, peaks, steps=3):
     t = statistics.mean(ms) / 1e3
     B = fwd_bytes(w, False, True, layer=True)
     F = fwd_flops(w)
-    t_roof = max(B / (peaks["hbm_gbs"] * 1e9), F / (peaks["bf16_tflops"] * 1e12))
-    return {"value": w.B * w.T / t, "unit": "tokens/s", "ms_per_step": t * 1e3,
-            "hbm_gbs": B / t / 1e9, "roofline_frac": t_roof / t, "workspace_bytes": ws_bytes,
-            "workload": workload_name(w)}
+    roof = roofline_block(B, F, t, peaks, "gdn_layer_fwd",
+                          recorded_traffic("gdn_layer_fwd", "layer_8to1"))
+    return {"value": w.B * w.T / t, "unit": "tokens/s", "ms_per_step": t * 1e3, "steps": steps,
+            "hbm_gbs": B / t / 1e9, "roofline_frac": roof["frac"], "roofline": roof,
+            "workspace_bytes": ws_bytes, "workload": workload_name(w)}
 
 
 def e2e_prefill(gdn, x, w, dev, steps):
@@ -385,23 +419,37 @@ def e2e_prefill(gdn, x, w, dev, steps):
     serving loop would run them: pipelined over an upload, a compute and a download stream with
     two device buffer sets, so step i's upload overlaps step i - 1's call and step i - 2's
     download (PCIe carries both directions at once); events order every reuse of a buffer set.
-    The timed region includes the pipeline's fill and drain."""
+    The timed region includes the pipeline's fill and drain.  Consecutive steps take different
+    inputs (three pinned input sets whose v differ, in rotation) and every buffer set downloads
+    into its own host outputs, so that the last two steps' downloads, checked afterwards against
+    plain calls on their own inputs, would show a step that read stale or overwritten buffers."""
     names = ["q", "k", "v", "log_alpha", "beta"]
-    host = {n: x[n].pin_memory() for n in names}
-    o_h = torch.empty(w.B, w.T, w.Hv, w.dv, dtype=w.torch_dtype).pin_memory()
-    s_h = torch.empty(w.B, w.Hv, w.dk, w.dv, dtype=torch.float32).pin_memory()
+    n_in = 3
+    inputs = []
+    for i in range(n_in):
+        h = {n: x[n].pin_memory() for n in names}
+        if i:
+            h["v"] = (x["v"].float() * (1.0 + 0.25 * i)).to(x["v"].dtype).pin_memory()
+        inputs.append(h)
     nbuf = 2
+    o_h = [torch.empty(w.B, w.T, w.Hv, w.dv, dtype=w.torch_dtype).pin_memory()
+           for _ in range(nbuf)]
+    s_h = [torch.empty(w.B, w.Hv, w.dk, w.dv, dtype=torch.float32).pin_memory()
+           for _ in range(nbuf)]
     dbuf = [{n: torch.empty_like(x[n], device=dev) for n in names} for _ in range(nbuf)]
-    o_d = [torch.empty(o_h.shape, dtype=o_h.dtype, device=dev) for _ in range(nbuf)]
-    s_d = [torch.empty(s_h.shape, dtype=s_h.dtype, device=dev) for _ in range(nbuf)]
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = o_h.numel() * o_h.element_size() + s_h.numel() * s_h.element_size()
+    o_d = [torch.empty(o_h[0].shape, dtype=o_h[0].dtype, device=dev) for _ in range(nbuf)]
+    s_d = [torch.empty(s_h[0].shape, dtype=s_h[0].dtype, device=dev) for _ in range(nbuf)]
+    ws = [workspace_for(gdn, w, dev) for _ in range(nbuf)]
+    h2d = sum(t.numel() * t.element_size() for t in inputs[0].values())
+    d2h = o_h[0].numel() * o_h[0].element_size() + s_h[0].numel() * s_h[0].element_size()
     s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
     ev_in, ev_comp, ev_out = ([torch.cuda.Event() for _ in range(nbuf)] for _ in range(3))
     used = [False] * nbuf
+    last_input = [None] * nbuf
 
     def step(i):
         j = i % nbuf
+        host = inputs[i % n_in]
         with torch.cuda.stream(s_in):
             if used[j]:
                 s_in.wait_event(ev_comp[j])          # the call that read buffer set j is done
@@ -413,14 +461,16 @@ def e2e_prefill(gdn, x, w, dev, steps):
             if used[j]:
                 s_comp.wait_event(ev_out[j])         # its previous o and S_T are downloaded
             gdn.chunk_fwd(dbuf[j]["q"], dbuf[j]["k"], dbuf[j]["v"], dbuf[j]["log_alpha"],
-                          dbuf[j]["beta"], None, chunk=w.chunk, out=o_d[j], state_out=s_d[j])
+                          dbuf[j]["beta"], None, chunk=w.chunk, out=o_d[j], state_out=s_d[j],
+                          workspace=ws[j])
             ev_comp[j].record(s_comp)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_comp[j])
-            o_h.copy_(o_d[j], non_blocking=True)
-            s_h.copy_(s_d[j], non_blocking=True)
+            o_h[j].copy_(o_d[j], non_blocking=True)
+            s_h[j].copy_(s_d[j], non_blocking=True)
             ev_out[j].record(s_out)
         used[j] = True
+        last_input[j] = i % n_in
 
     for i in range(nbuf):                            # warm-up: both buffer sets once
         step(i)
@@ -437,14 +487,18 @@ def e2e_prefill(gdn, x, w, dev, steps):
     b.record(cur)
     torch.cuda.synchronize()
     t = a.elapsed_time(b) / 1e3 / steps
-    # the last step's downloads against one plain call on the same inputs (outside the timing)
-    o_ref, s_ref = gdn.chunk_fwd(dbuf[0]["q"], dbuf[0]["k"], dbuf[0]["v"], dbuf[0]["log_alpha"],
-                                 dbuf[0]["beta"], None, chunk=w.chunk)
-    same = bool(torch.equal(o_ref.cpu(), o_h) and torch.equal(s_ref.cpu(), s_h))
+    # the last two steps' downloads against plain calls on their own inputs (outside the timing)
+    same = True
+    for j in range(nbuf):
+        hin = inputs[last_input[j]]
+        dd = {n: hin[n].to(dev) for n in names}
+        o_ref, s_ref = gdn.chunk_fwd(dd["q"], dd["k"], dd["v"], dd["log_alpha"], dd["beta"], None,
+                                     chunk=w.chunk)
+        same = same and bool(torch.equal(o_ref.cpu(), o_h[j]) and torch.equal(s_ref.cpu(), s_h[j]))
     return {"value": w.B * w.T / t, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h,
-            "pipelined": "upload / call / download streams, 2 buffer sets",
-            "downloads_match_plain_call": same}
+            "pipelined": "upload / call / download streams, 2 buffer sets, 3 input sets in rotation",
+            "last_two_steps_match_plain_calls": same}
 
 
 # ------------------------------------------------------------------------------------------------
@@ -501,21 +555,10 @@ def dist_setup(n_gpus):
     return world, rank, local
 
 
-def tc_launches_per_call(w: gi.Workload, dev, variant: str) -> int:
-    """Kernels one forward call launches: the SIMT forward one; the tensor-core forward two (the
-    operand pre-pass, then the recurrence), four when the library splits a batched call whose
-    B * Hv recurrences exceed the SM count into tail and leading batches, or two per range of 128
-    chunks when it runs a single long sequence (B = 1, at least 256 chunks, 2 Hv <= SMs) in
-    ranges."""
-    if variant != "tcgen05":
-        return 1
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    n_chunks = (w.T + 63) // 64
-    if w.B == 1 and 2 * w.Hv <= sms and n_chunks >= 256:
-        return 2 * ((n_chunks + 127) // 128)
-    head_b = sms // w.Hv
-    split = w.B >= 2 and w.B * w.Hv > sms and 1 <= head_b < w.B
-    return 4 if split else 2
+def launches_per_call(gdn, w: gi.Workload) -> int:
+    """Kernels one forward call launches on this device, as the library itself schedules them
+    (gdn_chunk_fwd_launches)."""
+    return gdn.chunk_fwd_launches(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv, w.chunk, w.torch_dtype)
 
 
 def max_over_ranks(value: float, device) -> float:
@@ -586,10 +629,8 @@ def profile_case(args):
         step()
     torch.cuda.synchronize()
     gdn.check_error(dev)
-    variant = gdn.chunk_fwd_variant(w.dk, w.dv, w.chunk, w.torch_dtype)
     print(json.dumps({"profile_case": workload_name(w), "calls": args.steps,
-                      "launches": args.steps * tc_launches_per_call(w, dev, variant)}),
-          flush=True)
+                      "launches": args.steps * launches_per_call(gdn, w)}), flush=True)
 
 
 def main():
@@ -650,20 +691,9 @@ def main():
 
     B = fwd_bytes(w, False, True)
     F = fwd_flops(w)
-    t_hbm = B / (peaks["hbm_gbs"] * 1e9)
-    t_ten = F / (peaks["bf16_tflops"] * 1e12)
-    hbm_bound = t_hbm >= t_ten
     variant = gdn.chunk_fwd_variant(w.dk, w.dv, w.chunk, w.torch_dtype)
     kname = "gdn_chunk_fwd_tc" if variant == "tcgen05" else "chunk_fwd_simt_kernel"
-    roof = {"bound": "hbm" if hbm_bound else "tensor",
-            "achieved": (B / t_step / 1e9) if hbm_bound else (F / t_step / 1e12),
-            "peak": peaks["hbm_gbs"] if hbm_bound else peaks["bf16_tflops"],
-            "unit": "GB/s" if hbm_bound else "TFLOP/s",
-            "traffic": recorded_traffic(kname, "prefill"),
-            "kernel": kname, "algorithmic_bytes": B, "algorithmic_flops": F,
-            "peak_source": peaks.get("source", "measured") + (" burst" if not hbm_bound else ""),
-            "other_bound_frac": (t_ten / t_step) if hbm_bound else (t_hbm / t_step)}
-    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof = roofline_block(B, F, t_step, peaks, kname, recorded_traffic(kname, "prefill"))
 
     line = {"metric": METRIC, "value": whole_job_rate(w.B * w.T, t_step, world), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -674,7 +704,7 @@ def main():
                        "kernel_variant": variant,
                        "l2": "256 MiB write between timed steps (outside the events)"},
             "roofline": roof,
-            "gpu_launches": args.steps * tc_launches_per_call(w, dev, variant),
+            "gpu_launches": args.steps * launches_per_call(gdn, w),
             "clocks": clocks.summary()}
 
     e2e = e2e_prefill(gdn, x, w, dev, steps=max(3, min(args.steps, 10)))
@@ -692,10 +722,10 @@ def main():
             del d
             torch.cuda.empty_cache()
             _, xl, dl, _, sec["long_context"] = bench_prefill_like(
-                gdn, "long_context", dev, 3, 3, flush, peaks)
+                gdn, "long_context", dev, 10, 3, flush, peaks)
             del xl, dl
             torch.cuda.empty_cache()
-            sec["layer_8to1"] = bench_layer(gdn, dev, 3, flush, peaks)
+            sec["layer_8to1"] = bench_layer(gdn, dev, 3, flush, peaks, steps=10)
             line["secondary"] = sec
         if not args.no_cpu_baseline and world == 1:
             cb = oracle_sample_rate(x, w, target_s=10.0)

@@ -15,7 +15,8 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["GdnError", "lib", "library_path", "chunk_fwd", "chunk_fwd_variant", "decode_step",
+__all__ = ["GdnError", "lib", "library_path", "chunk_fwd", "chunk_fwd_variant",
+           "chunk_fwd_workspace_bytes", "chunk_fwd_launches", "chunk_fwd_ba", "decode_step",
            "prologue", "out_norm", "layer_fwd", "layer_workspace_bytes", "check_error",
            "STATUS", "VARIANTS"]
 
@@ -54,17 +55,26 @@ def lib() -> ctypes.CDLL:
         L.gdn_version.restype = I
         L.gdn_check_error.argtypes = [P]
         L.gdn_check_error.restype = I
-        L.gdn_chunk_fwd.argtypes = [P] * 8 + [I] * 7 + [F, I, P]
+        L.gdn_chunk_fwd.argtypes = [P] * 9 + [SZ] + [I] * 7 + [F, I, I, P]
         L.gdn_chunk_fwd.restype = I
-        L.gdn_chunk_fwd_ex.argtypes = [P] * 8 + [I] * 7 + [F, I, I, P]
+        L.gdn_chunk_fwd_ex.argtypes = [P] * 9 + [SZ] + [I] * 7 + [F, I, I, I, P]
         L.gdn_chunk_fwd_ex.restype = I
+        L.gdn_chunk_fwd_ba.argtypes = [P] * 8 + [SZ] + [I] * 7 + [F, I, I, P]
+        L.gdn_chunk_fwd_ba.restype = I
+        L.gdn_chunk_fwd_workspace_bytes.argtypes = [I] * 8
+        L.gdn_chunk_fwd_workspace_bytes.restype = SZ
+        L.gdn_chunk_fwd_launches.argtypes = [I] * 10
+        L.gdn_chunk_fwd_launches.restype = I
+        L.gdn_chunk_fwd_varlen_workspace_bytes.argtypes = [I] * 8
+        L.gdn_chunk_fwd_varlen_workspace_bytes.restype = SZ
         L.gdn_chunk_fwd_variant.argtypes = [I, I, I, I]
         L.gdn_chunk_fwd_variant.restype = I
-        L.gdn_decode_step.argtypes = [P] * 7 + [I] * 5 + [F, I, P]
+        L.gdn_decode_step.argtypes = [P] * 7 + [I] * 5 + [F, I, I, P]
         L.gdn_decode_step.restype = I
         L.gdn_decode_layer_step.argtypes = [P] * 18 + [I] * 5 + [F, F, F, I, P]
         L.gdn_decode_layer_step.restype = I
-        L.gdn_chunk_fwd_varlen.argtypes = [P] * 6 + [I, I] + [P] * 3 + [I] * 6 + [F, I, P]
+        L.gdn_chunk_fwd_varlen.argtypes = [P] * 6 + [I, I] + [P] * 4 + [SZ] + [I] * 6 + \
+            [F, I, I, P]
         L.gdn_chunk_fwd_varlen.restype = I
         L.gdn_gates.argtypes = [P, P, P, LL, I, I, P]
         L.gdn_gates.restype = I
@@ -74,10 +84,10 @@ def lib() -> ctypes.CDLL:
         L.gdn_prologue.restype = I
         L.gdn_out_norm.argtypes = [P, P, P, P, LL, I, F, I, P]
         L.gdn_out_norm.restype = I
-        L.gdn_layer_fwd.argtypes = [P] * 14 + [SZ] + [I] * 7 + [F, F, F, I, P]
+        L.gdn_layer_fwd.argtypes = [P] * 14 + [SZ] + [I] * 7 + [F, F, F, I, I, P]
         L.gdn_layer_fwd.restype = I
         L.gdn_layer_workspace_bytes.argtypes = [I] * 7 + [I]
-        L.gdn_layer_fwd_static.argtypes = [P] * 13 + [I] * 7 + [F, F, F, I, P]
+        L.gdn_layer_fwd_static.argtypes = [P] * 13 + [I] * 7 + [F, F, F, I, I, P]
         L.gdn_layer_fwd_static.restype = I
         L.gdn_layer_workspace_bytes.restype = SZ
         _lib = L
@@ -131,11 +141,41 @@ def chunk_fwd_variant(dk: int, dv: int, chunk: int, dtype: torch.dtype) -> str:
     return {1: "simt", 2: "tcgen05"}[v]
 
 
+def chunk_fwd_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, dtype) -> int:
+    """Device scratch bytes ``chunk_fwd`` needs (0 for the CUDA-core family)."""
+    return int(lib().gdn_chunk_fwd_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, _DTYPES[dtype]))
+
+
+def chunk_fwd_launches(B, T, Hk, Hv, dk, dv, chunk, dtype, variant: str = "auto",
+                       sms: int = 0) -> int:
+    """Kernel launches of one ``chunk_fwd`` call (the library's own schedule decision) on a
+    device of ``sms`` SMs, or on the current device when ``sms`` is 0."""
+    n = lib().gdn_chunk_fwd_launches(B, T, Hk, Hv, dk, dv, chunk, _DTYPES[dtype],
+                                     VARIANTS[variant], sms)
+    if n < 0:
+        raise ValueError("gdn_chunk_fwd_launches rejected the arguments")
+    return n
+
+
+def _workspace(need: int, dev, workspace: Optional[torch.Tensor]):
+    """The caller-owned scratch of a call: the given tensor, or a fresh uint8 tensor from torch's
+    allocator when none is given (torch's tensors are 256-byte aligned)."""
+    if need == 0:
+        return None, 0
+    if workspace is None:
+        workspace = torch.empty(need, device=dev, dtype=torch.uint8)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
 def chunk_fwd(q, k, v, log_alpha, beta, S0=None, *, chunk: int = 64, scale: float = 1.0,
               out: Optional[torch.Tensor] = None, state_out: Optional[torch.Tensor] = None,
-              want_state: bool = True, variant: str = "auto"
+              want_state: bool = True, variant: str = "auto",
+              out_dtype: Optional[torch.dtype] = None,
+              workspace: Optional[torch.Tensor] = None
               ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-    """Chunked prefill forward: returns (o [B,T,Hv,dv], S_T [B,Hv,dk,dv] or None)."""
+    """Chunked prefill forward: returns (o [B,T,Hv,dv], S_T [B,Hv,dk,dv] or None).  ``out_dtype``
+    (default: q's dtype) may be float32 for bf16 inputs.  ``workspace``: a device uint8 tensor of
+    at least ``chunk_fwd_workspace_bytes(...)`` bytes, else one is allocated for the call."""
     B, T, Hk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
     if k.shape != q.shape or v.shape[:2] != (B, T) or k.dtype != q.dtype or v.dtype != q.dtype:
@@ -143,34 +183,72 @@ def chunk_fwd(q, k, v, log_alpha, beta, S0=None, *, chunk: int = 64, scale: floa
     if log_alpha.shape != (B, T, Hv) or beta.shape != (B, T, Hv):
         raise ValueError("gates must be [B, T, Hv]")
     _f32(log_alpha, beta, S0)
-    o = torch.empty_like(v) if out is None else out
+    odt = q.dtype if out_dtype is None else out_dtype
+    o = torch.empty(v.shape, device=v.device, dtype=odt) if out is None else out
     sT = None
     if want_state:
         sT = torch.empty(B, Hv, dk, dv, device=q.device, dtype=torch.float32) \
             if state_out is None else state_out
-    dev = _dev(q, k, v, log_alpha, beta, S0, o, sT)
+    dev = _dev(q, k, v, log_alpha, beta, S0, o, sT, workspace)
+    need = 0 if variant == "simt" else chunk_fwd_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk,
+                                                                q.dtype)
+    ws, wbytes = _workspace(need, dev, workspace)
     with torch.cuda.device(dev):
         st = lib().gdn_chunk_fwd_ex(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(S0), _p(o),
-                                    _p(sT), B, T, Hk, Hv, dk, dv, chunk, float(scale),
-                                    _io_dtype(q), VARIANTS[variant], _stream(dev))
+                                    _p(sT), _p(ws), wbytes, B, T, Hk, Hv, dk, dv, chunk,
+                                    float(scale), _io_dtype(q), _io_dtype(o), VARIANTS[variant],
+                                    _stream(dev))
     _check("gdn_chunk_fwd", st)
     return o, sT
 
 
+def chunk_fwd_ba(q, k, v, ba, S0=None, *, chunk: int = 64, scale: float = 1.0,
+                 out: Optional[torch.Tensor] = None, state_out: Optional[torch.Tensor] = None,
+                 want_state: bool = True, out_dtype: Optional[torch.dtype] = None,
+                 workspace: Optional[torch.Tensor] = None
+                 ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """``chunk_fwd`` with the gates computed from the in_proj_ba outputs ``ba`` [B,T,2*Hv] bf16
+    (b then a): beta = sigmoid(b), log alpha = log sigmoid(a), inside the tensor-core pre-pass."""
+    B, T, Hk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    if (k.shape != q.shape or v.shape[:2] != (B, T) or ba.shape != (B, T, 2 * Hv)
+            or ba.dtype != torch.bfloat16):
+        raise ValueError("q, k, v, ba shapes/dtypes disagree")
+    _f32(S0)
+    odt = q.dtype if out_dtype is None else out_dtype
+    o = torch.empty(v.shape, device=v.device, dtype=odt) if out is None else out
+    sT = None
+    if want_state:
+        sT = torch.empty(B, Hv, dk, dv, device=q.device, dtype=torch.float32) \
+            if state_out is None else state_out
+    dev = _dev(q, k, v, ba, S0, o, sT, workspace)
+    need = chunk_fwd_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, q.dtype)
+    ws, wbytes = _workspace(need, dev, workspace)
+    with torch.cuda.device(dev):
+        st = lib().gdn_chunk_fwd_ba(_p(q), _p(k), _p(v), _p(ba), _p(S0), _p(o), _p(sT), _p(ws),
+                                    wbytes, B, T, Hk, Hv, dk, dv, chunk, float(scale),
+                                    _io_dtype(q), _io_dtype(o), _stream(dev))
+    _check("gdn_chunk_fwd_ba", st)
+    return o, sT
+
+
 def decode_step(q, k, v, log_alpha, beta, S, *, scale: float = 1.0,
-                out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                out: Optional[torch.Tensor] = None,
+                out_dtype: Optional[torch.dtype] = None) -> torch.Tensor:
     """One decode step: q,k [N,Hk,dk]; v [N,Hv,dv]; gates [N,Hv]; S [N,Hv,dk,dv] updated in
-    place.  Returns o [N,Hv,dv]."""
+    place.  Returns o [N,Hv,dv] (``out_dtype``, default v's dtype; float32 for bf16 inputs)."""
     N, Hk, dk = q.shape
     Hv, dv = v.shape[1], v.shape[2]
     if k.shape != q.shape or v.shape[0] != N or S.shape != (N, Hv, dk, dv):
         raise ValueError("decode shapes disagree")
     _f32(log_alpha, beta, S)
-    o = torch.empty_like(v) if out is None else out
+    odt = v.dtype if out_dtype is None else out_dtype
+    o = torch.empty(v.shape, device=v.device, dtype=odt) if out is None else out
     dev = _dev(q, k, v, log_alpha, beta, S, o)
     with torch.cuda.device(dev):
         st = lib().gdn_decode_step(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(S), _p(o),
-                                   N, Hk, Hv, dk, dv, float(scale), _io_dtype(q), _stream(dev))
+                                   N, Hk, Hv, dk, dv, float(scale), _io_dtype(q), _io_dtype(o),
+                                   _stream(dev))
     _check("gdn_decode_step", st)
     return o
 
@@ -206,7 +284,9 @@ def decode_layer_step(q_raw, k_raw, v_raw, z, hq_in, hk_in, hv_in, hq_out, hk_ou
 
 def chunk_fwd_varlen(q, k, v, log_alpha, beta, cu_seqlens, max_seqlen: int, S0=None, *,
                      chunk: int = 64, scale: float = 1.0, out: Optional[torch.Tensor] = None,
-                     want_state: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+                     want_state: bool = True, out_dtype: Optional[torch.dtype] = None,
+                     workspace: Optional[torch.Tensor] = None
+                     ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Packed sequences: q,k [total,Hk,dk]; v [total,Hv,dv]; gates [total,Hv]; cu_seqlens
     [nseq+1] int32 on the device; S0 [nseq,Hv,dk,dv] or None.  Returns (o [total,Hv,dv],
     S_T [nseq,Hv,dk,dv] or None)."""
@@ -217,15 +297,19 @@ def chunk_fwd_varlen(q, k, v, log_alpha, beta, cu_seqlens, max_seqlen: int, S0=N
             or beta.shape != log_alpha.shape or cu_seqlens.dtype != torch.int32 or nseq < 0):
         raise ValueError("packed shapes disagree")
     _f32(log_alpha, beta)
-    o = torch.empty_like(v) if out is None else out
+    odt = q.dtype if out_dtype is None else out_dtype
+    o = torch.empty(v.shape, device=v.device, dtype=odt) if out is None else out
     sT = (torch.empty(nseq, Hv, dk, dv, device=q.device, dtype=torch.float32)
           if want_state else None)
-    dev = _dev(q, k, v, log_alpha, beta, cu_seqlens, o)
+    dev = _dev(q, k, v, log_alpha, beta, cu_seqlens, o, workspace)
+    need = int(lib().gdn_chunk_fwd_varlen_workspace_bytes(nseq, int(max_seqlen), Hk, Hv, dk, dv,
+                                                          chunk, _DTYPES[q.dtype]))
+    ws, wbytes = _workspace(need, dev, workspace)
     with torch.cuda.device(dev):
         st = lib().gdn_chunk_fwd_varlen(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta),
                                         _p(cu_seqlens), nseq, int(max_seqlen), _p(S0), _p(o),
-                                        _p(sT), total, Hk, Hv, dk, dv, chunk, float(scale),
-                                        _io_dtype(q), _stream(dev))
+                                        _p(sT), _p(ws), wbytes, total, Hk, Hv, dk, dv, chunk,
+                                        float(scale), _io_dtype(q), _io_dtype(o), _stream(dev))
     _check("gdn_chunk_fwd_varlen", st)
     return o, sT
 
@@ -286,11 +370,13 @@ def layer_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, dtype) -> int:
 def layer_fwd(q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, *, Hk: int,
               Hv: int, dk: int, dv: int, chunk: int = 64, scale: float = 1.0,
               l2_eps: float = 1e-6, norm_eps: float = 1e-5, want_state: bool = True,
-              workspace: Optional[torch.Tensor] = None):
-    """Whole layer between the projections: returns (y [B,T,Hv,dv], S_T or None)."""
+              workspace: Optional[torch.Tensor] = None,
+              out_dtype: Optional[torch.dtype] = None):
+    """Whole layer between the projections: returns (y [B,T,Hv,dv], S_T or None); y in
+    ``out_dtype`` (default the inputs' dtype; float32 for bf16 inputs)."""
     B, T = q_raw.shape[:2]
     _f32(wq, wk, wv, log_alpha, beta, S0, norm_w)
-    y = torch.empty(B, T, Hv, dv, device=q_raw.device, dtype=q_raw.dtype)
+    y = torch.empty(B, T, Hv, dv, device=q_raw.device, dtype=out_dtype or q_raw.dtype)
     sT = torch.empty(B, Hv, dk, dv, device=q_raw.device, dtype=torch.float32) \
         if want_state else None
     need = layer_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, q_raw.dtype)
@@ -303,20 +389,21 @@ def layer_fwd(q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, *
                                  _p(log_alpha), _p(beta), _p(S0), _p(norm_w), _p(y), _p(sT),
                                  _p(workspace), wbytes, B, T, Hk, Hv, dk, dv, chunk,
                                  float(scale), float(l2_eps), float(norm_eps),
-                                 _io_dtype(q_raw), _stream(dev))
+                                 _io_dtype(q_raw), _io_dtype(y), _stream(dev))
     _check("gdn_layer_fwd", st)
     return y, sT
 
 
 def layer_fwd_static(q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, *,
                      Hk: int, Hv: int, dk: int, dv: int, chunk: int = 64, scale: float = 1.0,
-                     l2_eps: float = 1e-6, norm_eps: float = 1e-5, want_state: bool = True):
+                     l2_eps: float = 1e-6, norm_eps: float = 1e-5, want_state: bool = True,
+                     out_dtype: Optional[torch.dtype] = None):
     """layer_fwd with the library's built-in device scratch instead of a workspace (see
     gdn_layer_fwd_static in gdn.h: at most GDN_LAYER_STATIC_SCRATCH_BYTES of scratch, and calls
     on one device must not overlap on the GPU)."""
     B, T = q_raw.shape[:2]
     _f32(wq, wk, wv, log_alpha, beta, S0, norm_w)
-    y = torch.empty(B, T, Hv, dv, device=q_raw.device, dtype=q_raw.dtype)
+    y = torch.empty(B, T, Hv, dv, device=q_raw.device, dtype=out_dtype or q_raw.dtype)
     sT = torch.empty(B, Hv, dk, dv, device=q_raw.device, dtype=torch.float32) \
         if want_state else None
     dev = _dev(q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, y, sT)
@@ -325,7 +412,7 @@ def layer_fwd_static(q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, no
                                         _p(wv), _p(log_alpha), _p(beta), _p(S0), _p(norm_w),
                                         _p(y), _p(sT), B, T, Hk, Hv, dk, dv, chunk, float(scale),
                                         float(l2_eps), float(norm_eps), _io_dtype(q_raw),
-                                        _stream(dev))
+                                        _io_dtype(y), _stream(dev))
     _check("gdn_layer_fwd_static", st)
     return y, sT
 

@@ -26,11 +26,11 @@ struct DecodeShape {
   static_assert(NT % 32 == 0 && DK % RG == 0 && NT >= DV, "decode shape");
 };
 
-template <int DK, int DV, typename Tio>
+template <int DK, int DV, typename Tio, typename Tout = Tio>
 __global__ void __launch_bounds__(DecodeShape<DK, DV>::NT)
 decode_step_kernel(const Tio* __restrict__ q, const Tio* __restrict__ k,
                    const Tio* __restrict__ v, const float* __restrict__ log_alpha,
-                   const float* __restrict__ beta, float* __restrict__ S, Tio* __restrict__ o,
+                   const float* __restrict__ beta, float* __restrict__ S, Tout* __restrict__ o,
                    int Hk, int Hv, float scale) {
   using Sh = DecodeShape<DK, DV>;
   constexpr int CG = Sh::CG, NT = Sh::NT, RG = Sh::RG, RPT = Sh::RPT;
@@ -86,7 +86,7 @@ decode_step_kernel(const Tio* __restrict__ q, const Tio* __restrict__ k,
     const float vj = to_f(v[nh * (long)DV + j]);
     const float u = bt * (vj - a * rr);
     su[j] = u;
-    o[nh * (long)DV + j] = from_f<Tio>(a * ss + s_qk * u);
+    o[nh * (long)DV + j] = from_f<Tout>(a * ss + s_qk * u);
   }
   __syncthreads();
   const float4 u4 = *reinterpret_cast<const float4*>(&su[cg * 4]);

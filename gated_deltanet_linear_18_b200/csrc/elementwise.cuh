@@ -12,7 +12,7 @@
 
 namespace gdn {
 
-constexpr int kPrologueTokens = 256;    // tokens per CTA
+constexpr int kPrologueTokens = 64;     // tokens per CTA
 
 // Vectors of 16 bytes: 8 bf16 or 4 fp32 values.
 template <typename T> struct Vec16;
@@ -50,10 +50,13 @@ template <> struct Vec16<__nv_bfloat16> {
 
 __device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 
-// grid: (ceil(T / 256), 2*Hk + Hv, B); block: 128 threads.  A head row of d channels is held by
-// L = d / N threads (N channels each, one 16-byte load per token); the 128 / L row groups of the
-// CTA take consecutive spans of 256 L / 128 tokens, each span starting from its own 3-token conv
-// history.  The L2 norm of a q or k row is a shuffle reduction over its L threads.
+// grid: (ceil(T / kPrologueTokens), 2*Hk + Hv, B); block: 128 threads.  One CTA takes one head
+// (d channels) of kPrologueTokens tokens: the raw rows of those tokens and of the three before
+// them (zeros before t = 0) come into shared memory by 16-byte asynchronous copies, all issued at
+// once (so each SM keeps many tiles' worth of loads in flight), then every token is convolved from
+// shared memory.  A head row of d channels is held by L = d / N threads (N channels of one 16-byte
+// vector each); the 128 / L row groups of the CTA take every (128 / L)-th token.  The L2 norm of a
+// q or k row is a shuffle reduction over its L threads (one warp).
 template <typename Tio>
 __global__ void __launch_bounds__(128)
 prologue_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
@@ -62,6 +65,9 @@ prologue_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
                 Tio* __restrict__ yq, Tio* __restrict__ yk, Tio* __restrict__ yv, int T, int Hk,
                 int Hv, int dk, int dv, float eps) {
   constexpr int N = Vec16<Tio>::N;
+  constexpr int R = kPrologueTokens + 3;      // staged rows: 3 history tokens, then the tile
+  extern __shared__ __align__(16) uint8_t pro_smem[];
+  Tio* tile = reinterpret_cast<Tio*>(pro_smem);
   const int slot = blockIdx.y;
   const long b = blockIdx.z;
   const Tio* x;
@@ -77,37 +83,39 @@ prologue_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
     x = xv; w = wv; y = yv; d = dv; head = slot - 2 * Hk; width = Hv * dv; l2 = false;
   }
   const int L = d / N;                        // 2 .. 32, a power of two
-  const int grp = threadIdx.x / L, lc = threadIdx.x % L;
-  const int span = kPrologueTokens * L / 128;
+  const long t0 = (long)blockIdx.x * kPrologueTokens;
+  const Tio* xh = x + b * T * (long)width + (long)head * d;
+  // stage rows t0 - 3 .. t0 + kPrologueTokens - 1 (row r holds token t0 - 3 + r)
+  for (int i = threadIdx.x; i < R * L; i += 128) {
+    const int r = i / L, c = i - r * L;
+    const long t = t0 - 3 + r;
+    const bool in = t >= 0 && t < T;
+    const Tio* src = in ? xh + t * width + c * N : xh;
+    const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(tile + (long)r * d + c * N));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(in ? 16 : 0) : "memory");
+  }
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+  const int grp = threadIdx.x / L, lc = threadIdx.x % L, ngrp = 128 / L;
   const long c0 = (long)head * d + lc * N;    // first channel of this thread
   float wt[N][4];
 #pragma unroll
   for (int i = 0; i < N; ++i)                 // weights need only 4-byte alignment
 #pragma unroll
     for (int j = 0; j < 4; ++j) wt[i][j] = w[(c0 + i) * 4 + j];
-  const long ts = (long)blockIdx.x * kPrologueTokens + (long)grp * span;
-  auto load = [&](long t, float (&v)[N]) {
-    if (t >= 0 && t < T) {
-      Vec16<Tio>::load(x + (b * T + t) * width + c0, v);
-    } else {
+  __syncthreads();
+  const long rem = T - t0;
+  const int nt = rem < kPrologueTokens ? (int)rem : kPrologueTokens;
+  for (int i = grp; i < kPrologueTokens; i += ngrp) {   // same trip count within a warp
+    float h[4][N];
 #pragma unroll
-      for (int i = 0; i < N; ++i) v[i] = 0.f;
-    }
-  };
-  float h3[N], h2[N], h1[N];                  // x[t-3], x[t-2], x[t-1]
-  load(ts - 3, h3);
-  load(ts - 2, h2);
-  load(ts - 1, h1);
-#pragma unroll 4
-  for (int i = 0; i < span; ++i) {            // same trip count for every thread of the warp
-    const long t = ts + i;
-    float xt[N], yv_[N];
-    load(t, xt);
+    for (int j = 0; j < 4; ++j) Vec16<Tio>::load(tile + (long)(i + j) * d + lc * N, h[j]);
+    float yv_[N];
     float ss = 0.f;
 #pragma unroll
     for (int j = 0; j < N; ++j) {
-      const float pre = wt[j][0] * h3[j] + wt[j][1] * h2[j] + wt[j][2] * h1[j] + wt[j][3] * xt[j];
-      h3[j] = h2[j]; h2[j] = h1[j]; h1[j] = xt[j];
+      const float pre = wt[j][0] * h[0][j] + wt[j][1] * h[1][j] + wt[j][2] * h[2][j] +
+                        wt[j][3] * h[3][j];
       yv_[j] = silu_fast(pre);
       ss += yv_[j] * yv_[j];
     }
@@ -117,8 +125,13 @@ prologue_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
 #pragma unroll
       for (int j = 0; j < N; ++j) yv_[j] *= inv;
     }
-    if (t < T) Vec16<Tio>::store(y + (b * T + t) * width + c0, yv_);
+    if (i < nt) Vec16<Tio>::store(y + (b * T + t0 + i) * width + c0, yv_);
   }
+}
+
+// Shared memory of one prologue CTA for heads of d channels.
+inline size_t prologue_smem_bytes(int d, size_t elem) {
+  return (size_t)(kPrologueTokens + 3) * d * elem;
 }
 
 // One warp per row of dv <= 128 values, 4 consecutive channels per lane.  `o` may be wider than
@@ -146,10 +159,10 @@ template <> struct Vec4<__nv_bfloat16> {
   }
 };
 
-template <typename To, typename Tio>
+template <typename To, typename Tz, typename Ty = Tz>
 __global__ void __launch_bounds__(256)
-out_norm_kernel(const To* __restrict__ o, const Tio* __restrict__ z, const float* __restrict__ w,
-                Tio* __restrict__ y, long long rows, int dv, float eps) {
+out_norm_kernel(const To* __restrict__ o, const Tz* __restrict__ z, const float* __restrict__ w,
+                Ty* __restrict__ y, long long rows, int dv, float eps) {
   const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -158,7 +171,7 @@ out_norm_kernel(const To* __restrict__ o, const Tio* __restrict__ z, const float
   float ov[4] = {0.f, 0.f, 0.f, 0.f}, zv[4] = {0.f, 0.f, 0.f, 0.f};
   if (active) {
     Vec4<To>::load(o + row * dv + c, ov);
-    Vec4<Tio>::load(z + row * dv + c, zv);
+    Vec4<Tz>::load(z + row * dv + c, zv);
   }
   float ss = (ov[0] * ov[0] + ov[1] * ov[1]) + (ov[2] * ov[2] + ov[3] * ov[3]);
   ss = warp_sum(ss);
@@ -168,7 +181,7 @@ out_norm_kernel(const To* __restrict__ o, const Tio* __restrict__ z, const float
     float yv[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) yv[e] = ov[e] * inv * ww[e] * silu_fast(zv[e]);
-    Vec4<Tio>::store(y + row * dv + c, yv);
+    Vec4<Ty>::store(y + row * dv + c, yv);
   }
 }
 

@@ -70,40 +70,44 @@ gdn_status simt_dispatch(int dk, int chunk, const void* q, const void* k, const 
 // ---------------------------------------------------------------------------------------------
 // Decode dispatch over (dk, dv)
 // ---------------------------------------------------------------------------------------------
-template <int DK, int DV, typename Tio>
+template <int DK, int DV, typename Tio, typename Tout>
 gdn_status decode_launch(const void* q, const void* k, const void* v, const float* la,
                          const float* be, float* S, void* o, int N, int Hk, int Hv, float scale,
                          cudaStream_t st) {
   using Sh = DecodeShape<DK, DV>;
-  decode_step_kernel<DK, DV, Tio><<<(unsigned)((long)N * Hv), Sh::NT, 0, st>>>(
+  decode_step_kernel<DK, DV, Tio, Tout><<<(unsigned)((long)N * Hv), Sh::NT, 0, st>>>(
       static_cast<const Tio*>(q), static_cast<const Tio*>(k), static_cast<const Tio*>(v), la,
-      be, S, static_cast<Tio*>(o), Hk, Hv, scale);
+      be, S, static_cast<Tout*>(o), Hk, Hv, scale);
   return launch_status();
 }
 
-template <typename Tio, int DK>
+template <typename Tio, typename Tout, int DK>
 gdn_status decode_dispatch_dv(int dv, const void* q, const void* k, const void* v,
                               const float* la, const float* be, float* S, void* o, int N, int Hk,
                               int Hv, float scale, cudaStream_t st) {
   switch (dv) {
-    case 16: return decode_launch<DK, 16, Tio>(q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
-    case 32: return decode_launch<DK, 32, Tio>(q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
-    case 64: return decode_launch<DK, 64, Tio>(q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
-    case 128: return decode_launch<DK, 128, Tio>(q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
+    case 16: return decode_launch<DK, 16, Tio, Tout>(q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
+    case 32: return decode_launch<DK, 32, Tio, Tout>(q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
+    case 64: return decode_launch<DK, 64, Tio, Tout>(q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
+    case 128:
+      return decode_launch<DK, 128, Tio, Tout>(q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
   }
   return GDN_ERR_UNSUPPORTED;
 }
 
-template <typename Tio>
+template <typename Tio, typename Tout>
 gdn_status decode_dispatch(int dk, int dv, const void* q, const void* k, const void* v,
                            const float* la, const float* be, float* S, void* o, int N, int Hk,
                            int Hv, float scale, cudaStream_t st) {
   switch (dk) {
-    case 16: return decode_dispatch_dv<Tio, 16>(dv, q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
-    case 32: return decode_dispatch_dv<Tio, 32>(dv, q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
-    case 64: return decode_dispatch_dv<Tio, 64>(dv, q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
+    case 16:
+      return decode_dispatch_dv<Tio, Tout, 16>(dv, q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
+    case 32:
+      return decode_dispatch_dv<Tio, Tout, 32>(dv, q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
+    case 64:
+      return decode_dispatch_dv<Tio, Tout, 64>(dv, q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
     case 128:
-      return decode_dispatch_dv<Tio, 128>(dv, q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
+      return decode_dispatch_dv<Tio, Tout, 128>(dv, q, k, v, la, be, S, o, N, Hk, Hv, scale, st);
   }
   return GDN_ERR_UNSUPPORTED;
 }
@@ -173,14 +177,13 @@ gdn_status decode_layer_dispatch(int dk, int dv, const DecodeLayerArgs& a, cudaS
   return GDN_ERR_UNSUPPORTED;
 }
 
-// The recurrence inside gdn_layer_fwd: inputs in `dtype`, output o in fp32; `scratch` is the
-// tensor-core forward's hand-over buffer (part of the layer workspace).
+// The CUDA-core recurrence inside gdn_layer_fwd (sizes the tensor-core family does not take):
+// inputs in `dtype`, output o in fp32 for the separate gated norm.
 gdn_status layer_chunk_fwd(const void* q, const void* k, const void* v, const float* la,
                            const float* be, const float* S0, float* o, float* S_T, int B, int T,
                            int Hk, int Hv, int dk, int dv, int chunk, float scale,
                            gdn_dtype dtype, void* scratch, cudaStream_t st) {
-  if (tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16))
-    return tc_chunk_launch_f32out(q, k, v, la, be, S0, o, S_T, B, T, Hk, Hv, scale, scratch, st);
+  (void)scratch;
   if (dtype == GDN_F32)
     return simt_dispatch<float, float>(dk, chunk, q, k, v, la, be, S0, o, S_T, B, T, Hk, Hv, dv,
                                        scale, st);
@@ -188,32 +191,14 @@ gdn_status layer_chunk_fwd(const void* q, const void* k, const void* v, const fl
                                              Hv, dv, scale, st);
 }
 
-// The tensor-core forward's scratch comes from a library-private stream-ordered memory pool per
-// device that keeps its memory between calls (so a repeated call reuses it without a new
-// device allocation).
-std::mutex g_pool_mu;
-cudaMemPool_t g_pools[64] = {};
-
-gdn_status scratch_pool(cudaMemPool_t* out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GDN_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_pool_mu);
-  if (!g_pools[dev]) {
-    cudaMemPoolProps props = {};
-    props.allocType = cudaMemAllocationTypePinned;
-    props.handleTypes = cudaMemHandleTypeNone;
-    props.location.type = cudaMemLocationTypeDevice;
-    props.location.id = dev;
-    cudaMemPool_t p = nullptr;
-    if (cudaMemPoolCreate(&p, &props) != cudaSuccess) return GDN_ERR_CUDA;
-    uint64_t keep = ~0ull;
-    if (cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess)
-      return GDN_ERR_CUDA;
-    g_pools[dev] = p;
-  }
-  *out = g_pools[dev];
-  return GDN_OK;
+// A caller workspace: present, 256-byte aligned and large enough for `need` bytes.
+bool workspace_ok(const void* ws, size_t bytes, size_t need) {
+  if (need == 0) return true;
+  return ws != nullptr && bytes >= need && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0;
 }
+
+// Input/output dtype pairs with a kernel: fp32 -> fp32, bf16 -> bf16, bf16 -> fp32.
+bool io_pair_ok(gdn_dtype in, gdn_dtype out) { return !(in == GDN_F32 && out == GDN_BF16); }
 
 gdn_status validate_heads(int Hk, int Hv, int dk, int dv) {
   if (Hk <= 0 || Hv <= 0 || dk <= 0 || dv <= 0 || Hv % Hk != 0) return GDN_ERR_INVALID_ARG;
@@ -249,12 +234,21 @@ gdn_status gdn_check_error(gdn_stream_t stream) {
   return (word & kErrTimeout) ? GDN_ERR_TIMEOUT : GDN_OK;
 }
 
+size_t gdn_chunk_fwd_varlen_workspace_bytes(int nseq, int max_seqlen, int Hk, int Hv, int dk,
+                                            int dv, int chunk, gdn_dtype dtype) {
+  (void)Hk;
+  if (nseq <= 0 || max_seqlen <= 0 || Hv <= 0) return 0;
+  if (!tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16)) return 0;
+  return tc_chunk_varlen_scratch_bytes(nseq, max_seqlen, Hv);
+}
+
 gdn_status gdn_chunk_fwd_varlen(const void* q, const void* k, const void* v,
                                 const float* log_alpha, const float* beta, const int* cu_seqlens,
                                 int nseq, int max_seqlen, const float* S0, void* o, float* S_T,
-                                int total_T, int Hk, int Hv, int dk, int dv, int chunk,
-                                float scale, gdn_dtype dtype, gdn_stream_t stream) {
-  if (nseq < 0 || max_seqlen < 0 || total_T < 0 || !valid_dtype(dtype))
+                                void* workspace, size_t workspace_bytes, int total_T, int Hk,
+                                int Hv, int dk, int dv, int chunk, float scale, gdn_dtype dtype,
+                                gdn_dtype o_dtype, gdn_stream_t stream) {
+  if (nseq < 0 || max_seqlen < 0 || total_T < 0 || !valid_dtype(dtype) || !valid_dtype(o_dtype))
     return GDN_ERR_INVALID_ARG;
   gdn_status s = validate_heads(Hk, Hv, dk, dv);
   if (s != GDN_OK) return s;
@@ -277,17 +271,10 @@ gdn_status gdn_chunk_fwd_varlen(const void* q, const void* k, const void* v,
       !aligned4(beta))
     return GDN_ERR_INVALID_ARG;
   if (!tc_chunk_length_ok(max_seqlen)) return GDN_ERR_UNSUPPORTED;
-  cudaMemPool_t pool = nullptr;
-  s = scratch_pool(&pool);
-  if (s != GDN_OK) return s;
-  void* scratch = nullptr;
-  if (cudaMallocFromPoolAsync(&scratch, tc_chunk_varlen_scratch_bytes(nseq, max_seqlen, Hv), pool,
-                              st) != cudaSuccess)
-    return GDN_ERR_CUDA;
-  s = tc_chunk_launch_varlen(q, k, v, log_alpha, beta, cu_seqlens, nseq, max_seqlen, S0, o, S_T,
-                             total_T, Hk, Hv, scale, scratch, st);
-  const cudaError_t e = cudaFreeAsync(scratch, st);   // ordered after the kernels
-  return s != GDN_OK ? s : (e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA);
+  const size_t need = tc_chunk_varlen_scratch_bytes(nseq, max_seqlen, Hv);
+  if (!workspace_ok(workspace, workspace_bytes, need)) return GDN_ERR_INVALID_ARG;
+  return tc_chunk_launch_varlen(q, k, v, log_alpha, beta, cu_seqlens, nseq, max_seqlen, S0, o,
+                                S_T, total_T, Hk, Hv, scale, o_dtype == GDN_F32, workspace, st);
 }
 
 gdn_status gdn_gates(const void* ba, float* log_alpha, float* beta, long long rows, int Hv,
@@ -321,11 +308,20 @@ gdn_variant gdn_chunk_fwd_variant(int dk, int dv, int chunk, gdn_dtype dtype) {
   return GDN_VARIANT_SIMT;
 }
 
-gdn_status gdn_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* log_alpha,
-                            const float* beta, const float* S0, void* o, float* S_T, int B,
-                            int T, int Hk, int Hv, int dk, int dv, int chunk, float scale,
-                            gdn_dtype dtype, gdn_variant variant, gdn_stream_t stream) {
-  if (B < 0 || T < 0 || !valid_dtype(dtype)) return GDN_ERR_INVALID_ARG;
+size_t gdn_chunk_fwd_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, int chunk,
+                                     gdn_dtype dtype) {
+  (void)Hk;
+  if (B <= 0 || T <= 0 || Hv <= 0) return 0;
+  if (!tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16)) return 0;
+  return tc_chunk_scratch_bytes(B, T, Hv);
+}
+
+// Arguments of gdn_chunk_fwd_ex that decide the kernel family, checked without any CUDA call.
+// On success *tc says whether the tensor-core family runs.
+static gdn_status chunk_fwd_check(int B, int T, int Hk, int Hv, int dk, int dv, int chunk,
+                                  gdn_dtype dtype, gdn_dtype o_dtype, gdn_variant variant,
+                                  bool* tc) {
+  if (B < 0 || T < 0 || !valid_dtype(dtype) || !valid_dtype(o_dtype)) return GDN_ERR_INVALID_ARG;
   if (variant != GDN_VARIANT_AUTO && variant != GDN_VARIANT_SIMT &&
       variant != GDN_VARIANT_TCGEN05)
     return GDN_ERR_INVALID_ARG;
@@ -333,12 +329,41 @@ gdn_status gdn_chunk_fwd_ex(const void* q, const void* k, const void* v, const f
   if (s != GDN_OK) return s;
   if (chunk <= 0) return GDN_ERR_INVALID_ARG;
   if (!supported_chunk(chunk)) return GDN_ERR_UNSUPPORTED;
+  if (!io_pair_ok(dtype, o_dtype)) return GDN_ERR_UNSUPPORTED;
   if (B > 65535) return GDN_ERR_UNSUPPORTED;
+  const bool tc_ok = tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16);
+  if (variant == GDN_VARIANT_TCGEN05 && !tc_ok) return GDN_ERR_UNSUPPORTED;
+  *tc = tc_ok && variant != GDN_VARIANT_SIMT;
+  if (*tc && !tc_chunk_length_ok(T)) return GDN_ERR_UNSUPPORTED;
+  return GDN_OK;
+}
+
+int gdn_chunk_fwd_launches(int B, int T, int Hk, int Hv, int dk, int dv, int chunk,
+                           gdn_dtype dtype, gdn_variant variant, int sms) {
+  bool tc = false;
+  if (chunk_fwd_check(B, T, Hk, Hv, dk, dv, chunk, dtype, dtype == GDN_BF16 ? GDN_BF16 : GDN_F32,
+                      variant, &tc) != GDN_OK)
+    return -1;
+  if ((long)B * T == 0) return 0;
+  if (sms < 0) return -1;
+  return tc ? tc_chunk_launches(B, T, Hv, false, sms) : 1;
+}
+
+gdn_status gdn_chunk_fwd_ex(const void* q, const void* k, const void* v, const float* log_alpha,
+                            const float* beta, const float* S0, void* o, float* S_T,
+                            void* workspace, size_t workspace_bytes, int B, int T, int Hk,
+                            int Hv, int dk, int dv, int chunk, float scale, gdn_dtype dtype,
+                            gdn_dtype o_dtype, gdn_variant variant, gdn_stream_t stream) {
+  bool tc = false;
+  gdn_status s = chunk_fwd_check(B, T, Hk, Hv, dk, dv, chunk, dtype, o_dtype, variant, &tc);
+  if (s != GDN_OK) return s;
   const bool work = (long)B * T > 0;
   if (work && (!q || !k || !v || !log_alpha || !beta || !o)) return GDN_ERR_INVALID_ARG;
   if (!opt_aligned16(q) || !opt_aligned16(k) || !opt_aligned16(v) || !opt_aligned16(o) ||
       !opt_aligned4(log_alpha) || !opt_aligned4(beta) || !opt_aligned16(S0) ||
       !opt_aligned16(S_T))
+    return GDN_ERR_INVALID_ARG;
+  if (work && tc && !workspace_ok(workspace, workspace_bytes, tc_chunk_scratch_bytes(B, T, Hv)))
     return GDN_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (B == 0) return GDN_OK;
@@ -349,34 +374,52 @@ gdn_status gdn_chunk_fwd_ex(const void* q, const void* k, const void* v, const f
                        : cudaMemsetAsync(S_T, 0, bytes, st);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
   }
-  const bool tc_ok = tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16);
-  if (variant == GDN_VARIANT_TCGEN05 && !tc_ok) return GDN_ERR_UNSUPPORTED;
-  if (tc_ok && variant != GDN_VARIANT_SIMT) {
-    if (!tc_chunk_length_ok(T)) return GDN_ERR_UNSUPPORTED;
-    cudaMemPool_t pool = nullptr;
-    s = scratch_pool(&pool);
-    if (s != GDN_OK) return s;
-    void* scratch = nullptr;
-    if (cudaMallocFromPoolAsync(&scratch, tc_chunk_scratch_bytes(B, T, Hv), pool, st) !=
-        cudaSuccess)
-      return GDN_ERR_CUDA;
-    s = tc_chunk_launch(q, k, v, log_alpha, beta, S0, o, S_T, B, T, Hk, Hv, scale, scratch, st);
-    const cudaError_t e = cudaFreeAsync(scratch, st);   // ordered after the kernels
-    return s != GDN_OK ? s : (e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA);
-  }
+  if (tc)
+    return tc_chunk_launch(q, k, v, log_alpha, beta, S0, o, S_T, B, T, Hk, Hv, scale,
+                           o_dtype == GDN_F32, workspace, st);
   if (dtype == GDN_F32)
     return simt_dispatch<float>(dk, chunk, q, k, v, log_alpha, beta, S0, o, S_T, B, T, Hk, Hv,
                                 dv, scale, st);
+  if (o_dtype == GDN_F32)
+    return simt_dispatch<__nv_bfloat16, float>(dk, chunk, q, k, v, log_alpha, beta, S0, o, S_T, B,
+                                                T, Hk, Hv, dv, scale, st);
   return simt_dispatch<__nv_bfloat16>(dk, chunk, q, k, v, log_alpha, beta, S0, o, S_T, B, T, Hk,
                                       Hv, dv, scale, st);
 }
 
+gdn_status gdn_chunk_fwd_ba(const void* q, const void* k, const void* v, const void* ba,
+                            const float* S0, void* o, float* S_T, void* workspace,
+                            size_t workspace_bytes, int B, int T, int Hk, int Hv, int dk, int dv,
+                            int chunk, float scale, gdn_dtype dtype, gdn_dtype o_dtype,
+                            gdn_stream_t stream) {
+  bool tc = false;
+  gdn_status s = chunk_fwd_check(B, T, Hk, Hv, dk, dv, chunk, dtype, o_dtype,
+                                 GDN_VARIANT_AUTO, &tc);
+  if (s != GDN_OK) return s;
+  if (!tc) return GDN_ERR_UNSUPPORTED;
+  const bool work = (long)B * T > 0;
+  if (work && (!q || !k || !v || !ba || !o)) return GDN_ERR_INVALID_ARG;
+  if (!opt_aligned16(q) || !opt_aligned16(k) || !opt_aligned16(v) || !opt_aligned16(o) ||
+      !opt_aligned4(ba) || !opt_aligned16(S0) || !opt_aligned16(S_T))
+    return GDN_ERR_INVALID_ARG;
+  if (work && !workspace_ok(workspace, workspace_bytes, tc_chunk_scratch_bytes(B, T, Hv)))
+    return GDN_ERR_INVALID_ARG;
+  if (!work)
+    return gdn_chunk_fwd(nullptr, nullptr, nullptr, nullptr, nullptr, S0, nullptr, S_T, nullptr, 0,
+                         B, T, Hk, Hv, dk, dv, chunk, scale, dtype, o_dtype, stream);
+  return tc_chunk_launch(q, k, v, nullptr, nullptr, S0, o, S_T, B, T, Hk, Hv, scale,
+                         o_dtype == GDN_F32, workspace, reinterpret_cast<cudaStream_t>(stream),
+                         ba);
+}
+
 gdn_status gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* log_alpha,
-                         const float* beta, const float* S0, void* o, float* S_T, int B, int T,
-                         int Hk, int Hv, int dk, int dv, int chunk, float scale,
-                         gdn_dtype dtype, gdn_stream_t stream) {
-  return gdn_chunk_fwd_ex(q, k, v, log_alpha, beta, S0, o, S_T, B, T, Hk, Hv, dk, dv, chunk,
-                          scale, dtype, GDN_VARIANT_AUTO, stream);
+                         const float* beta, const float* S0, void* o, float* S_T, void* workspace,
+                         size_t workspace_bytes, int B, int T, int Hk, int Hv, int dk, int dv,
+                         int chunk, float scale, gdn_dtype dtype, gdn_dtype o_dtype,
+                         gdn_stream_t stream) {
+  return gdn_chunk_fwd_ex(q, k, v, log_alpha, beta, S0, o, S_T, workspace, workspace_bytes, B, T,
+                          Hk, Hv, dk, dv, chunk, scale, dtype, o_dtype, GDN_VARIANT_AUTO,
+                          stream);
 }
 
 gdn_status gdn_decode_layer_step(const void* q_raw, const void* k_raw, const void* v_raw,
@@ -410,10 +453,12 @@ gdn_status gdn_decode_layer_step(const void* q_raw, const void* k_raw, const voi
 
 gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const float* log_alpha,
                            const float* beta, float* S, void* o, int N, int Hk, int Hv, int dk,
-                           int dv, float scale, gdn_dtype dtype, gdn_stream_t stream) {
-  if (N < 0 || !valid_dtype(dtype)) return GDN_ERR_INVALID_ARG;
+                           int dv, float scale, gdn_dtype dtype, gdn_dtype o_dtype,
+                           gdn_stream_t stream) {
+  if (N < 0 || !valid_dtype(dtype) || !valid_dtype(o_dtype)) return GDN_ERR_INVALID_ARG;
   gdn_status s = validate_heads(Hk, Hv, dk, dv);
   if (s != GDN_OK) return s;
+  if (!io_pair_ok(dtype, o_dtype)) return GDN_ERR_UNSUPPORTED;
   if (N == 0) return GDN_OK;
   if (!q || !k || !v || !log_alpha || !beta || !S || !o) return GDN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned4(log_alpha) ||
@@ -422,9 +467,13 @@ gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const fl
   if ((long)N * Hv > 0x7fffffffL) return GDN_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == GDN_F32)
-    return decode_dispatch<float>(dk, dv, q, k, v, log_alpha, beta, S, o, N, Hk, Hv, scale, st);
-  return decode_dispatch<__nv_bfloat16>(dk, dv, q, k, v, log_alpha, beta, S, o, N, Hk, Hv, scale,
-                                        st);
+    return decode_dispatch<float, float>(dk, dv, q, k, v, log_alpha, beta, S, o, N, Hk, Hv, scale,
+                                         st);
+  if (o_dtype == GDN_F32)
+    return decode_dispatch<__nv_bfloat16, float>(dk, dv, q, k, v, log_alpha, beta, S, o, N, Hk,
+                                                 Hv, scale, st);
+  return decode_dispatch<__nv_bfloat16, __nv_bfloat16>(dk, dv, q, k, v, log_alpha, beta, S, o, N,
+                                                       Hk, Hv, scale, st);
 }
 
 gdn_status gdn_prologue(const void* q_raw, const void* k_raw, const void* v_raw, const float* wq,
@@ -443,12 +492,13 @@ gdn_status gdn_prologue(const void* q_raw, const void* k_raw, const void* v_raw,
     return GDN_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   dim3 grid((T + kPrologueTokens - 1) / kPrologueTokens, 2 * Hk + Hv, B);
+  const int dmax = dk > dv ? dk : dv;
   if (dtype == GDN_F32)
-    prologue_kernel<float><<<grid, 128, 0, st>>>(
+    prologue_kernel<float><<<grid, 128, prologue_smem_bytes(dmax, 4), st>>>(
         (const float*)q_raw, (const float*)k_raw, (const float*)v_raw, wq, wk, wv, (float*)q,
         (float*)k, (float*)v, T, Hk, Hv, dk, dv, l2_eps);
   else
-    prologue_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(
+    prologue_kernel<__nv_bfloat16><<<grid, 128, prologue_smem_bytes(dmax, 2), st>>>(
         (const __nv_bfloat16*)q_raw, (const __nv_bfloat16*)k_raw, (const __nv_bfloat16*)v_raw,
         wq, wk, wv, (__nv_bfloat16*)q, (__nv_bfloat16*)k, (__nv_bfloat16*)v, T, Hk, Hv, dk, dv,
         l2_eps);
@@ -476,16 +526,16 @@ gdn_status gdn_out_norm(const void* o, const void* z, const float* w, void* y, l
 
 size_t gdn_layer_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, int chunk,
                                  gdn_dtype dtype) {
-  (void)chunk;
   if (B <= 0 || T <= 0 || Hk <= 0 || Hv <= 0 || dk <= 0 || dv <= 0) return 0;
   const size_t el = dtype == GDN_F32 ? 4 : 2;
   const size_t tok = (size_t)B * T;
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-  // normalised q, k and convolved v in the storage dtype; the pre-norm output o in fp32; the
-  // tensor-core forward's hand-over buffer when that forward runs
-  const size_t tc = tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16)
-                        ? up(tc_chunk_scratch_bytes(B, T, Hv)) : 0;
-  return 2 * up(tok * Hk * dk * el) + up(tok * Hv * dv * el) + up(tok * Hv * dv * 4) + tc;
+  // normalised q, k and convolved v in the storage dtype; then either the tensor-core forward's
+  // hand-over buffer (the gated norm runs in its epilogue) or the pre-norm output o in fp32
+  const size_t qkv = 2 * up(tok * Hk * dk * el) + up(tok * Hv * dv * el);
+  if (tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16))
+    return qkv + up(tc_chunk_scratch_bytes(B, T, Hv));
+  return qkv + up(tok * Hv * dv * 4);
 }
 
 gdn_status gdn_layer_fwd(const void* q_raw, const void* k_raw, const void* v_raw, const void* z,
@@ -494,23 +544,24 @@ gdn_status gdn_layer_fwd(const void* q_raw, const void* k_raw, const void* v_raw
                          const float* norm_w, void* y, float* S_T, void* workspace,
                          size_t workspace_bytes, int B, int T, int Hk, int Hv, int dk, int dv,
                          int chunk, float scale, float l2_eps, float norm_eps, gdn_dtype dtype,
-                         gdn_stream_t stream) {
-  if (B < 0 || T < 0 || !valid_dtype(dtype)) return GDN_ERR_INVALID_ARG;
+                         gdn_dtype y_dtype, gdn_stream_t stream) {
+  if (B < 0 || T < 0 || !valid_dtype(dtype) || !valid_dtype(y_dtype)) return GDN_ERR_INVALID_ARG;
+  if (!io_pair_ok(dtype, y_dtype)) return GDN_ERR_UNSUPPORTED;
   gdn_status s = validate_heads(Hk, Hv, dk, dv);
   if (s != GDN_OK) return s;
-  if (chunk <= 0) return GDN_ERR_INVALID_ARG;
+  if (chunk <= 0 || !(norm_eps >= 0.f)) return GDN_ERR_INVALID_ARG;
   if (!supported_chunk(chunk)) return GDN_ERR_UNSUPPORTED;
+  const bool tc = tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16);
+  if (tc && !tc_chunk_length_ok(T)) return GDN_ERR_UNSUPPORTED;
   const size_t need = gdn_layer_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, dtype);
   if ((long)B * T > 0) {
     if (!z || !norm_w || !y || !aligned16(z) || !aligned4(norm_w) || !aligned16(y))
       return GDN_ERR_INVALID_ARG;
-    if (need > 0 && (!workspace || workspace_bytes < need ||
-                     (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0))
-      return GDN_ERR_INVALID_ARG;
+    if (!workspace_ok(workspace, workspace_bytes, need)) return GDN_ERR_INVALID_ARG;
   }
   if ((long)B * T == 0)
-    return gdn_chunk_fwd(nullptr, nullptr, nullptr, nullptr, nullptr, S0, nullptr, S_T, B, T, Hk,
-                         Hv, dk, dv, chunk, scale, dtype, stream);
+    return gdn_chunk_fwd(nullptr, nullptr, nullptr, nullptr, nullptr, S0, nullptr, S_T, nullptr, 0,
+                         B, T, Hk, Hv, dk, dv, chunk, scale, dtype, dtype, stream);
   const size_t el = dtype == GDN_F32 ? 4 : 2;
   const size_t tok = (size_t)B * T;
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
@@ -518,23 +569,28 @@ gdn_status gdn_layer_fwd(const void* q_raw, const void* k_raw, const void* v_raw
   void* qn = ws;
   void* kn = ws + up(tok * Hk * dk * el);
   void* vc = ws + 2 * up(tok * Hk * dk * el);
-  void* o = ws + 2 * up(tok * Hk * dk * el) + up(tok * Hv * dv * el);
-  void* tc_scratch = static_cast<char*>(o) + up(tok * Hv * dv * 4);
+  char* rest = ws + 2 * up(tok * Hk * dk * el) + up(tok * Hv * dv * el);
   s = gdn_prologue(q_raw, k_raw, v_raw, wq, wk, wv, qn, kn, vc, B, T, Hk, Hv, dk, dv, l2_eps,
                    dtype, stream);
   if (s != GDN_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (tc)   // the recurrence applies the gated norm in its epilogue and writes y itself
+    return tc_layer_launch(qn, kn, vc, log_alpha, beta, S0, y, S_T, B, T, Hk, Hv, scale, z,
+                           norm_w, norm_eps, y_dtype == GDN_F32, rest, st);
   // the recurrence writes o in fp32 so that the gated norm reads it unrounded
-  s = layer_chunk_fwd(qn, kn, vc, log_alpha, beta, S0, static_cast<float*>(o), S_T, B, T, Hk, Hv,
-                      dk, dv, chunk, scale, dtype, tc_scratch,
-                      reinterpret_cast<cudaStream_t>(stream));
+  float* o = reinterpret_cast<float*>(rest);
+  s = layer_chunk_fwd(qn, kn, vc, log_alpha, beta, S0, o, S_T, B, T, Hk, Hv, dk, dv, chunk, scale,
+                      dtype, nullptr, st);
   if (s != GDN_OK) return s;
   const long long rows = (long long)tok * Hv;
   const long long blocks = (rows + 7) / 8;
   if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == GDN_F32)
     out_norm_kernel<float, float><<<(unsigned)blocks, 256, 0, st>>>(
         (const float*)o, (const float*)z, norm_w, (float*)y, rows, dv, norm_eps);
+  else if (y_dtype == GDN_F32)
+    out_norm_kernel<float, __nv_bfloat16, float><<<(unsigned)blocks, 256, 0, st>>>(
+        (const float*)o, (const __nv_bfloat16*)z, norm_w, (float*)y, rows, dv, norm_eps);
   else
     out_norm_kernel<float, __nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
         (const float*)o, (const __nv_bfloat16*)z, norm_w, (__nv_bfloat16*)y, rows, dv, norm_eps);
@@ -578,7 +634,8 @@ extern "C" gdn_status gdn_layer_fwd_static(
     const void* q_raw, const void* k_raw, const void* v_raw, const void* z, const float* wq,
     const float* wk, const float* wv, const float* log_alpha, const float* beta, const float* S0,
     const float* norm_w, void* y, float* S_T, int B, int T, int Hk, int Hv, int dk, int dv,
-    int chunk, float scale, float l2_eps, float norm_eps, gdn_dtype dtype, gdn_stream_t stream) {
+    int chunk, float scale, float l2_eps, float norm_eps, gdn_dtype dtype, gdn_dtype y_dtype,
+    gdn_stream_t stream) {
   if (B < 0 || T < 0 || !valid_dtype(dtype)) return GDN_ERR_INVALID_ARG;
   const size_t need = gdn_layer_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, dtype);
   if (need > (size_t)GDN_LAYER_STATIC_SCRATCH_BYTES) return GDN_ERR_UNSUPPORTED;
@@ -589,5 +646,5 @@ extern "C" gdn_status gdn_layer_fwd_static(
   }
   return gdn_layer_fwd(q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, y, S_T,
                        scratch, need > 0 ? (size_t)GDN_LAYER_STATIC_SCRATCH_BYTES : 0, B, T, Hk,
-                       Hv, dk, dv, chunk, scale, l2_eps, norm_eps, dtype, stream);
+                       Hv, dk, dv, chunk, scale, l2_eps, norm_eps, dtype, y_dtype, stream);
 }

@@ -64,10 +64,15 @@ constexpr uint32_t OFF_MB = 98304;      // 32 KB, per column half 16 KB: bf16 M 
 constexpr uint32_t OFF_PW = 131072;     // 2 slots x 48 KB: a chunk's PT hi, PT lo, W hi, W lo
 constexpr uint32_t PW_SLOT = 49152;     // after Y (and the update) the o tile is staged there
 constexpr uint32_t OFF_BAR = OFF_PW + 2 * PW_SLOT;
-constexpr int NBAR = 22;
+constexpr int NBAR = 24;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;   // +0 TMEM base, +4 abort flag
 constexpr uint32_t OFF_GAM = OFF_MISC + 16;         // 2 slots (chunk parity) x gamma_t, 64 fp32
-constexpr uint32_t SMEM_BYTES = OFF_GAM + 2 * 256;
+constexpr uint32_t OFF_NW = OFF_GAM + 2 * 256;      // the gated norm's gain, 128 fp32
+constexpr uint32_t SMEM_BYTES = OFF_NW + 512;
+// With the gated norm fused into the o epilogue, the two column halves of a token's row exchange
+// their sums of squares in the chunk's slot, past the staged o tiles (the W lo part, free once
+// the update has read it): 2 halves x 64 tokens fp32.
+constexpr uint32_t RED_OFF = 32768;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 
@@ -81,7 +86,7 @@ constexpr uint32_t TM_X = 0, TM_Y = 256, TM_M = 384;
 enum : int {
   B_QK_FULL = 0, B_QK_EMPTY, B_W_FULL = 2, B_W_EMPTY = 4, B_P_FULL = 6, B_P_EMPTY = 8,
   B_X_FULL = 10, B_R_FULL, B_D3_FULL, B_Y_FULL, B_Y_EMPTY, B_M_READY, B_M_SCALED, B_DRAIN,
-  B_G_FULL = 18, B_G_EMPTY = 20, B_END = 22
+  B_G_FULL = 18, B_G_EMPTY = 20, B_RED = 22, B_END = 24
 };
 static_assert(B_END <= NBAR, "barrier map");
 
@@ -457,7 +462,7 @@ __global__ void __launch_bounds__(PP_THREADS, 4)
 pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const float* __restrict__ log_alpha, const float* __restrict__ beta,
                   uint8_t* __restrict__ pw, int T, int Hk, int Hv, float scale,
-                  const int* __restrict__ cu, int max_len) {
+                  const int* __restrict__ cu, int max_len, const __nv_bfloat16* __restrict__ ba) {
   GDN_TRACE_INIT;
   extern __shared__ __align__(1024) uint8_t pp_raw[];
   uint8_t* smem = pp_raw + ((1024u - (tc::smem_u32(pp_raw) & 1023u)) & 1023u);
@@ -507,8 +512,19 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
   // gates: G' = cumsum(log alpha) log2(e) over the chunk, beta, ktil, gamma (zero / flat past T)
   if (tid < 64) {
     const long tt = t0 + tid;
-    const float la = tt < sp.len ? log_alpha[(sp.row0 + tt) * Hv + h] : 0.f;
-    gB[tid] = tt < sp.len ? beta[(sp.row0 + tt) * Hv + h] : 0.f;
+    float la = 0.f, bt = 0.f;
+    if (tt < sp.len) {
+      if (ba) {   // from the in_proj_ba outputs: beta = sigmoid(b), log alpha = -softplus(-a)
+        const __nv_bfloat16* row = ba + (sp.row0 + tt) * 2 * Hv;
+        const float b = __bfloat162float(row[h]), a = __bfloat162float(row[Hv + h]);
+        bt = 1.0f / (1.0f + expf(-b));
+        la = a >= 0.f ? -log1pf(expf(-a)) : a - log1pf(expf(a));
+      } else {
+        la = log_alpha[(sp.row0 + tt) * Hv + h];
+        bt = beta[(sp.row0 + tt) * Hv + h];
+      }
+    }
+    gB[tid] = bt;
     float incl = la;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
@@ -758,17 +774,25 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 // ------------------------------------------------------------------------------------------
 // the recurrence
 // ------------------------------------------------------------------------------------------
-template <typename Tout>
+// kNorm: the layer's gated RMSNorm is applied to o in the epilogue, y = o / sqrt(mean(o^2) + eps)
+// * w (.) SiLU(z) per (token, head), and y (in Tout) is stored instead of o.
+template <typename Tout, bool kNorm>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmo, const __nv_bfloat16* __restrict__ v,
                     const uint8_t* __restrict__ pw, const float* __restrict__ S0,
                     float* __restrict__ S_T, int T, int Hk, int Hv, float scale,
-                    const int* __restrict__ cu, int max_len, int nCmax, Tout* __restrict__ o) {
+                    const int* __restrict__ cu, int max_len, int nCmax, Tout* __restrict__ o,
+                    const __nv_bfloat16* __restrict__ z, const float* __restrict__ norm_w,
+                    float norm_eps) {
   constexpr bool kF32 = sizeof(Tout) == 4;
-  // X takes M as a hi + lo bf16 pair when o is fp32 (the layer, whose gated norm magnifies o's
-  // error); a bf16 o carries its own rounding, and one round-to-nearest bf16 copy of M suffices.
-  constexpr bool kSplitX = kF32;
+  // X takes M as a hi + lo bf16 pair when o is fp32 or goes through the gated norm (whose
+  // per-row normalisation magnifies o's error); a bf16 o carries its own rounding, and one
+  // round-to-nearest bf16 copy of M suffices.
+  constexpr bool kSplitX = kF32 || kNorm;
+  // the o leaders also hand back W's part of the slot when the o tile spills into it or the norm
+  // exchange uses it
+  constexpr bool kOutUsesW = kF32 || kNorm;
   GDN_TRACE_INIT;
   // Offsetting the __shared__ array itself (not a round trip through an integer) keeps every
   // access below a shared-memory access (ld/st.shared), not a generic one.
@@ -805,9 +829,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     // spills into W's part)
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(bar(B_P_EMPTY + s), 3);
-      tc::mbar_init(bar(B_W_EMPTY + s), kF32 ? 3 : 1);
+      tc::mbar_init(bar(B_W_EMPTY + s), kOutUsesW ? 3 : 1);
       tc::mbar_init(bar(B_G_FULL + s), 1);
       tc::mbar_init(bar(B_G_EMPTY + s), 8);           // one arrive per chain warp
+      tc::mbar_init(bar(B_RED + s), 2);               // one arrive per column half
     }
     *abort_flag = 0;
     tc::fence_barrier_init();
@@ -816,6 +841,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     tc::tmem_alloc(sb + OFF_MISC, 512);
     tc::tmem_relinquish();
     tc::tc_fence_before();
+  }
+  if constexpr (kNorm) {
+    if (threadIdx.x < 128) reinterpret_cast<float*>(smem + OFF_NW)[threadIdx.x] = norm_w[threadIdx.x];
   }
   if (warp == 0 && lane == 0) {
     tc::tma_prefetch_desc(&tmq);
@@ -878,8 +906,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       // Y = PT R' (rows 0..63 used), as hi.hi + lo.hi + hi.lo bf16 products             (bf16)
       auto issue_Y = [&](int cy) -> bool {
         const int sy = cy & 1;
-        if (cy >= 1 && !tc::mbar_wait(bar(B_Y_EMPTY), (cy - 1) & 1, abort_flag, kBudget)) return false;
-        if (!tc::mbar_wait(bar(B_P_FULL + sy), (cy >> 1) & 1, abort_flag, kBudget)) return false;
+        if (cy >= 1 && !tc::mbar_wait_spin(bar(B_Y_EMPTY), (cy - 1) & 1, abort_flag, kBudget)) return false;
+        if (!tc::mbar_wait_spin(bar(B_P_FULL + sy), (cy >> 1) & 1, abort_flag, kBudget)) return false;
         tc::tc_fence_after();
         const uint64_t dpw = tc::sdesc_sw128(sb + OFF_PW + sy * PW_SLOT, 16, 1024);
         const uint64_t drd = tc::sdesc_sw128(sb + OFF_RD + sy * RD_BUF, 16384, 1024);
@@ -898,8 +926,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       for (int c = 0; c < nC && ok; ++c) {
         const int s = c & 1;
         // X = [Q; K] M  (M as one bf16 copy, or a hi + lo pair)                     (bf16)
-        ok = tc::mbar_wait(bar(B_QK_FULL), c & 1, abort_flag, kBudget) &&
-             tc::mbar_wait(bar(B_M_READY), c & 1, abort_flag, kBudget);
+        ok = tc::mbar_wait_spin(bar(B_QK_FULL), c & 1, abort_flag, kBudget) &&
+             tc::mbar_wait_spin(bar(B_M_READY), c & 1, abort_flag, kBudget);
         if (!ok) break;
         GDN_TRACE(c, 12);
         tc::tc_fence_after();
@@ -915,9 +943,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         GDN_TRACE(c, 20);
         if (c >= 1 && !(ok = issue_Y(c - 1))) break;
         // M += W R' (TMEM holds gamma_last M), hi.hi + lo.hi + hi.lo bf16 products     (bf16)
-        ok = tc::mbar_wait(bar(B_R_FULL), c & 1, abort_flag, kBudget) &&
-             tc::mbar_wait(bar(B_M_SCALED), c & 1, abort_flag, kBudget) &&
-             tc::mbar_wait(bar(B_W_FULL + s), (c >> 1) & 1, abort_flag, kBudget);
+        ok = tc::mbar_wait_spin(bar(B_R_FULL), c & 1, abort_flag, kBudget) &&
+             tc::mbar_wait_spin(bar(B_M_SCALED), c & 1, abort_flag, kBudget) &&
+             tc::mbar_wait_spin(bar(B_W_FULL + s), (c >> 1) & 1, abort_flag, kBudget);
         if (!ok) break;
         GDN_TRACE(c, 13);
         tc::tc_fence_after();
@@ -1128,7 +1156,20 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       if (q < 2 && !stop) {
         // o_t = gamma_t scale (Q M)_t + (PT R')_t, staged in the chunk's operand slot (the PT
         // tiles, which Y has finished reading; fp32 also takes W's, after the update) for a TMA
-        // store
+        // store.  With kNorm, y_t (the gated norm of o_t) takes o's place.
+        const bool t_valid = (long)c * C + t < sp.len;
+        [[maybe_unused]] uint4 zr[8];
+        if constexpr (kNorm) {                   // z row t of this half, before the wait
+          if (t_valid) {
+            const uint4* src = reinterpret_cast<const uint4*>(
+                z + ((sp.row0 + (long)c * C + t) * Hv + h) * 128 + tcol);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) zr[i] = src[i];
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) zr[i] = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
         tc::mbar_wait(bar(B_Y_FULL), c & 1, abort_flag, kBudget);
         if (leader) GDN_TRACE(c, 34 + ev);
         tc::tc_fence_after();
@@ -1138,18 +1179,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         // the last chunk of a packed sequence ends inside the tile: its valid rows go straight to
         // global memory (a box store would write into the next sequence)
         const bool ragged = packed && (c + 1) * C > sp.len;
-        const bool t_valid = (long)c * C + t < sp.len;
         Tout* orow = o + ((sp.row0 + (long)c * C + t) * Hv + h) * 128 + tcol;
-#pragma unroll 1
-        for (int p = 0; p < 4; ++p) {            // value columns 16p .. 16p+15 of this half
-          float x[16], y[16];
-          tmem_ld16(tx + 16 * p, x);
-          tmem_ld16(tmem + lane_off + TM_Y + tcol + 16 * p, y);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 16; i += 2)
-            tc::f2_get(tc::fma2(tc::f2(g, g), tc::f2(x[i], x[i + 1]), tc::f2(y[i], y[i + 1])),
-                       y[i], y[i + 1]);
+        // value columns 16p .. 16p+15 of this half (y[16]) to global memory or the staged tile
+        auto put16 = [&](int p, const float* y) {
           if (ragged) {
             if (t_valid) {
               if constexpr (kF32) {
@@ -1181,6 +1213,57 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
                                tc::pack_bf16(y[8 * j + 4], y[8 * j + 5]),
                                tc::pack_bf16(y[8 * j + 6], y[8 * j + 7]));
           }
+        };
+        if constexpr (kNorm) {
+          float ov[64];
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            float x[16], y[16];
+            tmem_ld16(tx + 16 * p, x);
+            tmem_ld16(tmem + lane_off + TM_Y + tcol + 16 * p, y);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; i += 2)
+              tc::f2_get(tc::fma2(tc::f2(g, g), tc::f2(x[i], x[i + 1]), tc::f2(y[i], y[i + 1])),
+                         ov[16 * p + i], ov[16 * p + i + 1]);
+          }
+          float ss = 0.f;
+#pragma unroll
+          for (int i = 0; i < 64; ++i) ss = fmaf(ov[i], ov[i], ss);
+          // the row's other half is held by the same lane of the other column group
+          float* red = reinterpret_cast<float*>(smem + OFF_PW + s * PW_SLOT + RED_OFF);
+          red[hh * 64 + t] = ss;
+          tc::named_bar(id_lo, 64);
+          if (leader) tc::mbar_arrive(bar(B_RED + s));
+          tc::mbar_wait(bar(B_RED + s), (c >> 1) & 1, abort_flag, kBudget);
+          const float inv = rsqrtf((red[t] + red[64 + t]) * (1.0f / 128.0f) + norm_eps);
+          const float* nw = reinterpret_cast<const float*>(smem + OFF_NW) + tcol;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t w4[4] = {zr[j].x, zr[j].y, zr[j].z, zr[j].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float za = tc::bf16lo(w4[e]), zb = tc::bf16hi(w4[e]);
+              const int i = 8 * j + 2 * e;
+              ov[i] = ov[i] * inv * nw[i] * __fdividef(za, 1.0f + __expf(-za));
+              ov[i + 1] = ov[i + 1] * inv * nw[i + 1] * __fdividef(zb, 1.0f + __expf(-zb));
+            }
+          }
+#pragma unroll
+          for (int p = 0; p < 4; ++p) put16(p, ov + 16 * p);
+        } else {
+#pragma unroll 1
+          for (int p = 0; p < 4; ++p) {            // value columns 16p .. 16p+15 of this half
+            float x[16], y[16];
+            tmem_ld16(tx + 16 * p, x);
+            tmem_ld16(tmem + lane_off + TM_Y + tcol + 16 * p, y);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; i += 2)
+              tc::f2_get(tc::fma2(tc::f2(g, g), tc::f2(x[i], x[i + 1]), tc::f2(y[i], y[i + 1])),
+                         y[i], y[i + 1]);
+            put16(p, y);
+          }
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
@@ -1200,7 +1283,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
             tc::bulk_wait_read_all();
           }
           tc::mbar_arrive(bar(B_P_EMPTY + s));
-          if constexpr (kF32) tc::mbar_arrive(bar(B_W_EMPTY + s));
+          if constexpr (kOutUsesW) tc::mbar_arrive(bar(B_W_EMPTY + s));
           GDN_TRACE(c, 36 + ev);
         }
       }
@@ -1257,6 +1340,29 @@ constexpr int kRangeChunks = 128;
 inline bool ranged(int nseq, int T, int Hv, int sms) {
   return nseq == 1 && 2L * Hv <= sms && (T + C - 1) / C >= 2 * kRangeChunks;
 }
+
+// How launch() runs a call: in one part (pre-pass + recurrence), in ranges of a long single
+// sequence, or split into leading and tail batches.  launch() and launch_count() both decide here.
+enum class Plan { kOne, kRanges, kSplit };
+inline Plan plan(int nseq, int T, int Hv, int sms, bool packed) {
+  if (!packed && ranged(nseq, T, Hv, sms)) return Plan::kRanges;
+  const int head_b = sms / (Hv > 0 ? Hv : 1);        // batches that fill at most one wave
+  if (packed || nseq < 2 || (long)nseq * Hv <= sms || head_b < 1 || head_b >= nseq)
+    return Plan::kOne;
+  return Plan::kSplit;
+}
+// Kernel launches of one call (two per part: pre-pass and recurrence).
+inline int launch_count(int nseq, int T, int Hv, int sms, bool packed) {
+  if (nseq <= 0 || T <= 0) return 0;
+  switch (plan(nseq, T, Hv, sms, packed)) {
+    case Plan::kRanges: {
+      const int nC = (T + C - 1) / C;
+      return 2 * ((nC + kRangeChunks - 1) / kRangeChunks);
+    }
+    case Plan::kSplit: return 4;
+    default: return 2;
+  }
+}
 // Bytes of the operand hand-over buffer between the pre-pass and the recurrence; for sequences
 // long enough to run in ranges, two fp32 states follow the records (the state between ranges).
 inline size_t scratch_bytes(int B, int T, int Hv) {
@@ -1302,17 +1408,32 @@ inline Split* split_for_device() {   // call with split_mutex() held
 // records.  The recurrence reads the pre-pass's records only after it in stream order.  `parts`:
 // kPre, kRec or both; a recurrence launched alone must follow its pre-pass on `st` by an event.
 constexpr int kPre = 1, kRec = 2;
+// Optional parts of a call: the gated norm fused into the o epilogue (z == nullptr: plain o; z has
+// o's layout, bf16), and gates taken from the in_proj_ba outputs (ba [tokens, 2 Hv] bf16) instead
+// of log_alpha / beta.  at(): the same for the part of the call starting `tokens` tokens in.
+struct NormArgs {
+  const __nv_bfloat16* z = nullptr;
+  const float* w = nullptr;
+  float eps = 0.f;
+  const __nv_bfloat16* ba = nullptr;
+  int Hv = 0;
+  NormArgs at(size_t tokens) const {
+    return NormArgs{z ? z + tokens * Hv * 128 : nullptr, w, eps,
+                    ba ? ba + tokens * 2 * Hv : nullptr, Hv};
+  }
+};
 template <typename Tout>
 gdn_status launch_one(const void* q, const void* k, const void* v, const float* la,
                       const float* be, const float* S0, Tout* o, float* S_T, int nseq, int T,
                       int Hk, int Hv, float scale, uint8_t* pw, const int* cu, int max_len,
-                      cudaStream_t st, cudaEvent_t ev_after_pre, int parts = kPre | kRec) {
+                      const NormArgs& nrm, cudaStream_t st, cudaEvent_t ev_after_pre,
+                      int parts = kPre | kRec) {
   const int mapB = cu ? 1 : nseq;
   CUtensorMap mq, mk, mo;
   if (!make_tile_map(&mq, q, Hk, T, mapB, false) || !make_tile_map(&mk, k, Hk, T, mapB, false) ||
       !make_tile_map(&mo, o, Hv, T, mapB, sizeof(Tout) == 4))
     return GDN_ERR_CUDA;
-  auto kern = chunk_fwd_tc_kernel<Tout>;
+  auto kern = nrm.z ? chunk_fwd_tc_kernel<Tout, true> : chunk_fwd_tc_kernel<Tout, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC) !=
       cudaSuccess)
     return GDN_ERR_CUDA;
@@ -1326,14 +1447,14 @@ gdn_status launch_one(const void* q, const void* k, const void* v, const float* 
   if (parts & kPre) {
     // head-fastest: the value heads that share a key head's Q/K tiles run side by side
     pw_prepass_kernel<<<dim3(Hv, nCmax, nseq), PP_THREADS, PP_SMEM, st>>>(
-        mq, mk, la, be, pw, T, Hk, Hv, scale, cu, max_len);
+        mq, mk, la, be, pw, T, Hk, Hv, scale, cu, max_len, nrm.ba);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
   }
   if (ev_after_pre && cudaEventRecord(ev_after_pre, st) != cudaSuccess) return GDN_ERR_CUDA;
   if (parts & kRec) {
     kern<<<(unsigned)grid, kThreads, SMEM_ALLOC, st>>>(
         mq, mk, mo, static_cast<const __nv_bfloat16*>(v), pw, S0, S_T, T, Hk, Hv, scale, cu,
-        max_len, nCmax, o);
+        max_len, nCmax, o, nrm.z, nrm.w, nrm.eps);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
   }
   return GDN_OK;
@@ -1348,12 +1469,14 @@ gdn_status launch_one(const void* q, const void* k, const void* v, const float* 
 template <typename Tout>
 gdn_status launch(const void* q, const void* k, const void* v, const float* la, const float* be,
                   const float* S0, Tout* o, float* S_T, int nseq, int T, int Hk, int Hv,
-                  float scale, uint8_t* pw, const int* cu, int max_len, cudaStream_t st) {
+                  float scale, uint8_t* pw, const int* cu, int max_len, cudaStream_t st,
+                  const NormArgs& nrm = NormArgs{}) {
   if ((max_len + C - 1) / C > 65535) return GDN_ERR_UNSUPPORTED;   // chunks index a grid's y
   std::unique_lock<std::mutex> lock(split_mutex());
   Split* sp = split_for_device();
   if (!sp) return GDN_ERR_CUDA;
-  if (!cu && ranged(nseq, T, Hv, sp->sms)) {
+  const Plan pl = plan(nseq, T, Hv, sp->sms, cu != nullptr);
+  if (pl == Plan::kRanges) {
     // Ranges of kRangeChunks chunks: every pre-pass on the low-priority stream, one after the
     // other; the recurrence of range r on the high-priority stream once pre-pass r is done and
     // after recurrence r - 1, starting from its final state.  Pre-pass r + 1 thus runs on the
@@ -1375,13 +1498,16 @@ gdn_status launch(const void* q, const void* k, const void* v, const float* la, 
       const float* S0r = r == 0 ? S0 : mid[(r - 1) & 1];
       float* STr = r == nR - 1 ? S_T : mid[r & 1];
       uint8_t* pwr = pw + (size_t)Hv * r * kRangeChunks * kPwBytes;
-      s = launch_one<Tout>(bq, bk, bv, la + t0 * Hv, be + t0 * Hv, S0r, o + t0 * Hv * 128, STr, 1,
-                           Tr, Hk, Hv, scale, pwr, nullptr, Tr, sp->s_lo, sp->ev_pre, kPre);
+      const NormArgs nr = nrm.at((size_t)t0);
+      const float* lar = la ? la + t0 * Hv : nullptr;
+      const float* ber = be ? be + t0 * Hv : nullptr;
+      s = launch_one<Tout>(bq, bk, bv, lar, ber, S0r, o + t0 * Hv * 128, STr, 1,
+                           Tr, Hk, Hv, scale, pwr, nullptr, Tr, nr, sp->s_lo, sp->ev_pre, kPre);
       if (s == GDN_OK && cudaStreamWaitEvent(sp->s_hi, sp->ev_pre, 0) != cudaSuccess)
         s = GDN_ERR_CUDA;
       if (s == GDN_OK)
-        s = launch_one<Tout>(bq, bk, bv, la + t0 * Hv, be + t0 * Hv, S0r, o + t0 * Hv * 128, STr,
-                             1, Tr, Hk, Hv, scale, pwr, nullptr, Tr, sp->s_hi, nullptr, kRec);
+        s = launch_one<Tout>(bq, bk, bv, lar, ber, S0r, o + t0 * Hv * 128, STr,
+                             1, Tr, Hk, Hv, scale, pwr, nullptr, Tr, nr, sp->s_hi, nullptr, kRec);
     }
     const bool joined = cudaEventRecord(sp->ev_hi, sp->s_hi) == cudaSuccess &&
                         cudaEventRecord(sp->ev_lo, sp->s_lo) == cudaSuccess &&
@@ -1390,10 +1516,10 @@ gdn_status launch(const void* q, const void* k, const void* v, const float* la, 
     return s != GDN_OK ? s : (joined ? GDN_OK : GDN_ERR_CUDA);
   }
   const int head_b = sp->sms / (Hv > 0 ? Hv : 1);        // batches that fill at most one wave
-  if (cu || nseq < 2 || (long)nseq * Hv <= sp->sms || head_b < 1 || head_b >= nseq) {
+  if (pl == Plan::kOne) {
     lock.unlock();
     return launch_one<Tout>(q, k, v, la, be, S0, o, S_T, nseq, T, Hk, Hv, scale, pw, cu, max_len,
-                            st, nullptr);
+                            nrm, st, nullptr);
   }
   const int tail_b = nseq - head_b;
   const size_t tq = (size_t)T * Hk * 128, tv = (size_t)T * Hv * 128, tg = (size_t)T * Hv;
@@ -1417,13 +1543,13 @@ gdn_status launch(const void* q, const void* k, const void* v, const float* la, 
   gdn_status s = ok ? GDN_OK : GDN_ERR_CUDA;
   if (s == GDN_OK)   // the tail: pre-pass, then its recurrence, both on the high-priority stream
     s = launch_one<Tout>(qt, kt, vt, lat, bet, S0t, ot, STt, tail_b, T, Hk, Hv, scale, pwt,
-                         nullptr, T, sp->s_hi, sp->ev_pre);
+                         nullptr, T, nrm.at((size_t)head_b * T), sp->s_hi, sp->ev_pre);
   // the leading batches start once the tail's pre-pass is done
   if (s == GDN_OK && cudaStreamWaitEvent(sp->s_lo, sp->ev_pre, 0) != cudaSuccess)
     s = GDN_ERR_CUDA;
   if (s == GDN_OK)
     s = launch_one<Tout>(q, k, v, la, be, S0, o, S_T, head_b, T, Hk, Hv, scale, pw, nullptr, T,
-                         sp->s_lo, nullptr);
+                         nrm, sp->s_lo, nullptr);
   // the caller's stream waits for both parts, also after a failure, so no work outlives it
   const bool joined = cudaEventRecord(sp->ev_hi, sp->s_hi) == cudaSuccess &&
                       cudaEventRecord(sp->ev_lo, sp->s_lo) == cudaSuccess &&
@@ -1440,6 +1566,18 @@ extern "C" GDN_API void gdn_debug_set_trace(void* p) {
 }
 #endif
 
+// Kernel launches of one tensor-core call on a device of `sms` SMs, or on the current device when
+// sms is 0 (-1 if that query fails).
+inline int tc_chunk_launches(int nseq, int T, int Hv, bool packed, int sms) {
+  if (sms == 0) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return -1;
+  }
+  return tcf::launch_count(nseq, T, Hv, sms, packed);
+}
+
 inline bool tc_chunk_supported(int dk, int dv, int chunk, bool bf16) {
   return bf16 && dk == 128 && dv == 128 && chunk == tcf::C;
 }
@@ -1450,13 +1588,39 @@ inline bool tc_chunk_length_ok(long max_len) { return (max_len + tcf::C - 1) / t
 // Scratch bytes of the tensor-core forward (the pre-pass's operand hand-over buffer).
 inline size_t tc_chunk_scratch_bytes(int B, int T, int Hv) { return tcf::scratch_bytes(B, T, Hv); }
 
+// o in bf16, or in fp32 when f32out (o's box stores then carry fp32 and the X product takes the
+// state as a hi + lo pair).
+// `ba` (optional, [B, T, 2 Hv] bf16): gates from the in_proj_ba outputs instead of la / be.
 inline gdn_status tc_chunk_launch(const void* q, const void* k, const void* v, const float* la,
                                   const float* be, const float* S0, void* o, float* S_T, int B,
-                                  int T, int Hk, int Hv, float scale, void* scratch,
-                                  cudaStream_t st) {
+                                  int T, int Hk, int Hv, float scale, bool f32out, void* scratch,
+                                  cudaStream_t st, const void* ba = nullptr) {
+  uint8_t* pw = static_cast<uint8_t*>(scratch);
+  tcf::NormArgs ex;
+  ex.ba = static_cast<const __nv_bfloat16*>(ba);
+  ex.Hv = Hv;
+  if (f32out)
+    return tcf::launch<float>(q, k, v, la, be, S0, static_cast<float*>(o), S_T, B, T, Hk, Hv,
+                              scale, pw, nullptr, T, st, ex);
   return tcf::launch<__nv_bfloat16>(q, k, v, la, be, S0, static_cast<__nv_bfloat16*>(o), S_T, B,
-                                    T, Hk, Hv, scale, static_cast<uint8_t*>(scratch), nullptr, T,
-                                    st);
+                                    T, Hk, Hv, scale, pw, nullptr, T, st, ex);
+}
+
+// The recurrence with the layer's gated norm in its epilogue: y = o / sqrt(mean(o^2) + eps) * w
+// (.) SiLU(z) per (token, head) instead of o; z [B, T, Hv, 128] bf16, w [128] fp32; y in bf16, or
+// fp32 when f32y.
+inline gdn_status tc_layer_launch(const void* q, const void* k, const void* v, const float* la,
+                                  const float* be, const float* S0, void* y, float* S_T, int B,
+                                  int T, int Hk, int Hv, float scale, const void* z,
+                                  const float* norm_w, float norm_eps, bool f32y, void* scratch,
+                                  cudaStream_t st) {
+  uint8_t* pw = static_cast<uint8_t*>(scratch);
+  const tcf::NormArgs nrm{static_cast<const __nv_bfloat16*>(z), norm_w, norm_eps, nullptr, Hv};
+  if (f32y)
+    return tcf::launch<float>(q, k, v, la, be, S0, static_cast<float*>(y), S_T, B, T, Hk, Hv,
+                              scale, pw, nullptr, T, st, nrm);
+  return tcf::launch<__nv_bfloat16>(q, k, v, la, be, S0, static_cast<__nv_bfloat16*>(y), S_T, B,
+                                    T, Hk, Hv, scale, pw, nullptr, T, st, nrm);
 }
 
 // Packed sequences: q, k [total, Hk, 128], v, o [total, Hv, 128], gates [total, Hv]; sequence s is
@@ -1469,18 +1633,13 @@ inline gdn_status tc_chunk_launch_varlen(const void* q, const void* k, const voi
                                          const float* la, const float* be, const int* cu,
                                          int nseq, int max_len, const float* S0, void* o,
                                          float* S_T, int total, int Hk, int Hv, float scale,
-                                         void* scratch, cudaStream_t st) {
+                                         bool f32out, void* scratch, cudaStream_t st) {
+  uint8_t* pw = static_cast<uint8_t*>(scratch);
+  if (f32out)
+    return tcf::launch<float>(q, k, v, la, be, S0, static_cast<float*>(o), S_T, nseq, total, Hk,
+                              Hv, scale, pw, cu, max_len, st);
   return tcf::launch<__nv_bfloat16>(q, k, v, la, be, S0, static_cast<__nv_bfloat16*>(o), S_T,
-                                    nseq, total, Hk, Hv, scale, static_cast<uint8_t*>(scratch), cu,
-                                    max_len, st);
-}
-
-inline gdn_status tc_chunk_launch_f32out(const void* q, const void* k, const void* v,
-                                         const float* la, const float* be, const float* S0,
-                                         float* o, float* S_T, int B, int T, int Hk, int Hv,
-                                         float scale, void* scratch, cudaStream_t st) {
-  return tcf::launch<float>(q, k, v, la, be, S0, o, S_T, B, T, Hk, Hv, scale,
-                            static_cast<uint8_t*>(scratch), nullptr, T, st);
+                                    nseq, total, Hk, Hv, scale, pw, cu, max_len, st);
 }
 
 }  // namespace gdn

@@ -75,6 +75,34 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// The same bounded wait without suspension: mbarrier.test_wait never parks the thread, so a
+// single-thread role (the MMA issuer) resumes within a poll of the phase completing instead of
+// after try_wait's suspend interval.  It keeps its warp's issue slot busy while it polls.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity,
+                                               volatile int* abort, uint64_t budget_cycles) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (;;) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if ((uint64_t)(clock64() - t0) > budget_cycles) {
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------------------------
 // fences and named barriers
 // ---------------------------------------------------------------------------------------------

@@ -15,19 +15,27 @@
  *
  * Layouts (row-major, last index contiguous, no padding, no strides):
  *   q, k        [B, T, Hk, dk]        dtype given by `dtype`
- *   v, o        [B, T, Hv, dv]        dtype given by `dtype`
+ *   v           [B, T, Hv, dv]        dtype given by `dtype`
+ *   o           [B, T, Hv, dv]        dtype given by `o_dtype` (chunked forward) or `dtype`
  *   log_alpha   [B, T, Hv]  float     alpha = exp(log_alpha), expected in ]0, 1]
  *   beta        [B, T, Hv]  float     expected in [0, 1]
  *   S0, S_T, S  [B, Hv, dk, dv] float, holding S transposed: S_store[b][h][i][j] = S[j][i]
  *               (i over d_k, j over d_v; d_v contiguous)
  *
- * Pointers.  Every tensor pointer is a DEVICE pointer (cudaMalloc'd or equivalent) on the device
- * current for the calling thread, unless a comment says otherwise.  The caller owns every
- * buffer; the library keeps no pointer after a call returns and allocates no device memory,
- * except one 4-byte device error word per device, created statically with the library.
+ * Pointers and ownership.  Every tensor pointer is a DEVICE pointer (cudaMalloc'd or equivalent)
+ * on the device current for the calling thread, unless a comment says otherwise.  The caller owns
+ * every buffer, including the device scratch ("workspace") that the chunked forward and the layer
+ * need: size it with gdn_chunk_fwd_workspace_bytes / gdn_chunk_fwd_varlen_workspace_bytes /
+ * gdn_layer_workspace_bytes and pass it in.  No call allocates or frees device memory.  The
+ * library keeps no pointer after a call returns.  Its own device memory is part of its device
+ * image, loaded with it: a 4-byte error word, and the 32 MiB scratch of gdn_layer_fwd_static.
+ * Host-side state: on first use per device the tensor-core chunked forward creates two CUDA
+ * streams (high and low priority) and four events and keeps them for the life of the process
+ * (see gdn_chunk_fwd).
  * Outputs must not overlap inputs, except S in gdn_decode_step, which is read and written in
- * place.  Tensor pointers (q, k, v, o, z, y, states, raw projections, workspace) must be 16-byte
- * aligned; gate and weight pointers (log_alpha, beta, conv taps, norm gain) 4-byte aligned.
+ * place.  Tensor pointers (q, k, v, o, z, y, states, raw projections) must be 16-byte aligned,
+ * workspaces 256-byte aligned, gate and weight pointers (log_alpha, beta, conv taps, norm gain)
+ * 4-byte aligned.
  *
  * Streams.  `stream` is a cudaStream_t (NULL = the legacy default stream).  Each compute call
  * validates its arguments synchronously, enqueues its kernels on `stream` and returns without
@@ -35,8 +43,9 @@
  *
  * Errors.  Calls return gdn_status and never abort, throw or trap.  GDN_ERR_INVALID_ARG: a null
  * required pointer, a non-positive size, Hv not a multiple of Hk, misalignment, or an
- * unsupported enum value; nothing is enqueued.  GDN_ERR_UNSUPPORTED: valid sizes this build has
- * no kernel for (dk, dv not in {16, 32, 64, 128}, chunk not in {16, 32, 64}); nothing enqueued.
+ * unsupported enum value, or a missing, misaligned or too small workspace; nothing is enqueued.
+ * GDN_ERR_UNSUPPORTED: valid sizes or dtypes this build has no kernel for (dk, dv not in {16, 32,
+ * 64, 128}, chunk not in {16, 32, 64}, fp32 inputs with a bf16 output); nothing enqueued.
  * GDN_ERR_CUDA: a CUDA call failed (e.g. the launch); the CUDA error is left for
  * cudaGetLastError.  GDN_ERR_TIMEOUT is reported by gdn_check_error when a kernel gave up on a
  * bounded wait (it then skipped the rest of its work; its outputs are undefined).
@@ -103,53 +112,86 @@ GDN_API gdn_status gdn_wait_timeout_selftest(long long budget_cycles, gdn_stream
  *   S0   may be NULL: the zero state of a fresh request (16.1: the working state is reset for
  *        the next request).  Otherwise the state after the previous call, so that splitting a
  *        sequence over calls gives the same result as one call.
+ *   o    [B, T, Hv, dv] in `o_dtype`: GDN_BF16 or GDN_F32 for bf16 inputs, GDN_F32 for fp32
+ *        inputs (fp32 inputs with a bf16 o return GDN_ERR_UNSUPPORTED).
  *   S_T  may be NULL when the final state is not wanted.
+ *   workspace, workspace_bytes: device scratch of at least
+ *        gdn_chunk_fwd_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, dtype) bytes, 256-byte
+ *        aligned (NULL and 0 when that size is 0).  Its contents are undefined after the call; it
+ *        must not be used by other work until the call's kernels are done on `stream`.
  *   T    need not be a multiple of `chunk`; the ragged last block is masked.
  *   scale multiplies q (o = scale * S q).
  * Exact in real arithmetic for any chunk size; the chunk size only reorders rounding.
  * The tensor-core family (bf16, d_k = d_v = 128, chunk 64) first computes every chunk's
- * state-independent operands (P T_b and (diag(ktil) K)^T T_b as bf16 hi/lo tiles, and gamma) in a
- * pre-pass and hands them to the recurrence through a device buffer of
- * B * Hv * ceil(T/64) * 49408 bytes (T up to 65535 chunks, 4,194,240 tokens, else
- * GDN_ERR_UNSUPPORTED before any work);
- * that buffer is taken from a memory pool of the library (one per device, stream-ordered, kept
- * between calls) and given back at the end of the call on `stream`.  When B * Hv exceeds the
- * device's SM count the call runs in two parts (the last batches first) on two internal streams
- * of the library that fork from and join back into `stream`, so that the recurrence runs in one
- * wave; the results are those of one launch.  A single sequence (B = 1) of at least 256 chunks
- * whose Hv recurrences take at most half of the SMs runs in ranges of 128 chunks on the same two
- * streams (the pre-pass of the next range beside the recurrence of the current one, the state
- * handed on through two fp32 states after the records); the results are again those of one
- * launch.  The buffer holds those 2 * B * Hv * 64 KiB whenever T reaches 256 chunks.
+ * state-independent operands in a pre-pass and hands them to the recurrence through the
+ * workspace (one record per (batch, value head, chunk); T up to 65535 chunks, 4,194,240 tokens,
+ * else GDN_ERR_UNSUPPORTED before any work).  When B * Hv exceeds the device's SM count the
+ * call runs in two parts (the last batches first) on two internal streams of the library that
+ * fork from and join back into `stream`, so that the recurrence runs in one wave; the results
+ * are those of one launch.  A single sequence (B = 1) of at least 256 chunks whose Hv
+ * recurrences take at most half of the SMs runs in ranges of 128 chunks on the same two streams
+ * (the pre-pass of the next range beside the recurrence of the current one, the state handed on
+ * through two fp32 states kept in the workspace); the results are again those of one launch.
  */
 GDN_API gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v,
                          const float *log_alpha, const float *beta, const float *S0,
-                         void *o, float *S_T,
+                         void *o, float *S_T, void *workspace, size_t workspace_bytes,
                          int B, int T, int Hk, int Hv, int dk, int dv, int chunk,
-                         float scale, gdn_dtype dtype, gdn_stream_t stream);
+                         float scale, gdn_dtype dtype, gdn_dtype o_dtype,
+                         gdn_stream_t stream);
+
+/* Device scratch bytes gdn_chunk_fwd needs for these sizes (host only, no CUDA call): the
+ * tensor-core family's operand hand-over, 0 for the CUDA-core family and for empty calls. */
+GDN_API size_t gdn_chunk_fwd_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv,
+                                     int chunk, gdn_dtype dtype);
 
 /* gdn_chunk_fwd with an explicit kernel family.  GDN_ERR_UNSUPPORTED if the requested family has
- * no kernel for these sizes/dtype. */
+ * no kernel for these sizes/dtype.  With GDN_VARIANT_SIMT no workspace is needed. */
 GDN_API gdn_status gdn_chunk_fwd_ex(const void *q, const void *k, const void *v,
                             const float *log_alpha, const float *beta, const float *S0,
-                            void *o, float *S_T,
+                            void *o, float *S_T, void *workspace, size_t workspace_bytes,
                             int B, int T, int Hk, int Hv, int dk, int dv, int chunk,
-                            float scale, gdn_dtype dtype, gdn_variant variant,
-                            gdn_stream_t stream);
+                            float scale, gdn_dtype dtype, gdn_dtype o_dtype,
+                            gdn_variant variant, gdn_stream_t stream);
+
+/*
+ * gdn_chunk_fwd with the gates taken from the in_proj_ba outputs, computed where the pre-pass
+ * loads each chunk's gates (so serving from the projections costs no extra pass over HBM):
+ * beta = sigmoid(b), log_alpha = log sigmoid(a), the same definitions as gdn_gates ("L'attention
+ * hybride", "Le décompte": in_proj_ba makes one beta and one alpha per value head).
+ *   ba [B, T, 2*Hv] bf16: the Hv b values, then the Hv a values, of each token (2-byte aligned)
+ * Other arguments as gdn_chunk_fwd (same workspace size).  Supported: the tensor-core family
+ * (bf16, dk = dv = 128, chunk 64); other sizes return GDN_ERR_UNSUPPORTED.
+ */
+GDN_API gdn_status gdn_chunk_fwd_ba(const void *q, const void *k, const void *v, const void *ba,
+                            const float *S0, void *o, float *S_T, void *workspace,
+                            size_t workspace_bytes, int B, int T, int Hk, int Hv, int dk,
+                            int dv, int chunk, float scale, gdn_dtype dtype,
+                            gdn_dtype o_dtype, gdn_stream_t stream);
 
 /* The family gdn_chunk_fwd would run for these sizes (host only, no CUDA call). */
 GDN_API gdn_variant gdn_chunk_fwd_variant(int dk, int dv, int chunk, gdn_dtype dtype);
 
+/* How many kernels one gdn_chunk_fwd_ex call with these arguments launches (the schedule above,
+ * decided by the same code the call runs: one for the CUDA-core family; two for the tensor-core
+ * family, four when a batched call is split, two per range of a long single sequence; 0 when
+ * there is no token).  `sms`: the device's SM count, or 0 to read it from the current device (a
+ * CUDA attribute query, nothing enqueued; with sms > 0 no CUDA call is made).  Returns -1 for
+ * arguments the call would reject or if the query fails. */
+GDN_API int gdn_chunk_fwd_launches(int B, int T, int Hk, int Hv, int dk, int dv, int chunk,
+                           gdn_dtype dtype, gdn_variant variant, int sms);
+
 /*
  * One decode step for N independent sequences ("Chapitre 16 ...", 16.3: read the fixed state,
- * compute the output, update the state).  q, k [N, Hk, dk]; v, o [N, Hv, dv]; log_alpha, beta
+ * compute the output, update the state).  q, k [N, Hk, dk]; v [N, Hv, dv] (dtype); o [N, Hv,
+ * dv] (o_dtype: GDN_BF16 or GDN_F32 for bf16 inputs, GDN_F32 for fp32 inputs); log_alpha, beta
  * [N, Hv]; S [N, Hv, dk, dv] (S transposed, fp32) is read and overwritten in place with the
  * state after the token.  o_t reads the updated state.
  */
 GDN_API gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
                            const float *log_alpha, const float *beta, float *S, void *o,
                            int N, int Hk, int Hv, int dk, int dv, float scale,
-                           gdn_dtype dtype, gdn_stream_t stream);
+                           gdn_dtype dtype, gdn_dtype o_dtype, gdn_stream_t stream);
 
 /*
  * One decode step of the whole layer for N sequences, in one kernel: the prologue (causal conv of
@@ -185,23 +227,30 @@ GDN_API gdn_status gdn_decode_layer_step(const void *q_raw, const void *k_raw, c
  * many requests in one call, each with its own state ("Chapitre 16 - Assembler un système de type
  * Kimi K3", 16.2: a prompt in blocks with the state handed on; 16.1: the working state belongs to
  * the request).
- *   q, k [total_T, Hk, dk]; v, o [total_T, Hv, dv]                 (dtype)
+ *   q, k [total_T, Hk, dk]; v [total_T, Hv, dv] (dtype); o [total_T, Hv, dv] (o_dtype)
  *   log_alpha, beta [total_T, Hv] float
  *   cu_seqlens [nseq + 1] int32 in device memory: sequence s is tokens cu[s] .. cu[s+1] - 1
  *        (cu[0] = 0, non-decreasing, cu[nseq] <= total_T); empty sequences are allowed.  Offsets
  *        outside [0, total_T] are clamped and a sequence longer than max_seqlen is cut there
  *        (tokens outside every sequence keep their o untouched).
- *   max_seqlen: a host-side upper bound of the lengths (it sizes the launch)
+ *   max_seqlen: a host-side upper bound of the lengths (it sizes the launch and the workspace)
  *   S0 [nseq, Hv, dk, dv] float or NULL (zero states); S_T [nseq, Hv, dk, dv] float or NULL
- * Supported: the tensor-core family (bf16, dk = dv = 128, chunk 64); other sizes return
- * GDN_ERR_UNSUPPORTED.  Scratch as gdn_chunk_fwd, nseq * Hv * ceil(max_seqlen / 64) * 49408
- * bytes from the library's pool.
+ *   workspace, workspace_bytes: at least gdn_chunk_fwd_varlen_workspace_bytes(nseq, max_seqlen,
+ *        Hk, Hv, dk, dv, chunk, dtype) bytes, 256-byte aligned, as for gdn_chunk_fwd.
+ * Supported: the tensor-core family (bf16 inputs, dk = dv = 128, chunk 64; o bf16 or fp32);
+ * other sizes return GDN_ERR_UNSUPPORTED.
  */
 GDN_API gdn_status gdn_chunk_fwd_varlen(const void *q, const void *k, const void *v,
                                 const float *log_alpha, const float *beta, const int *cu_seqlens,
                                 int nseq, int max_seqlen, const float *S0, void *o, float *S_T,
+                                void *workspace, size_t workspace_bytes,
                                 int total_T, int Hk, int Hv, int dk, int dv, int chunk,
-                                float scale, gdn_dtype dtype, gdn_stream_t stream);
+                                float scale, gdn_dtype dtype, gdn_dtype o_dtype,
+                                gdn_stream_t stream);
+
+/* Device scratch bytes gdn_chunk_fwd_varlen needs (host only, no CUDA call). */
+GDN_API size_t gdn_chunk_fwd_varlen_workspace_bytes(int nseq, int max_seqlen, int Hk, int Hv,
+                                            int dk, int dv, int chunk, gdn_dtype dtype);
 
 /*
  * Gates from the in_proj_ba outputs, per (token, value head): beta = sigmoid(b) and
@@ -246,7 +295,8 @@ GDN_API gdn_status gdn_out_norm(const void *o, const void *z, const float *w, vo
  * Whole layer between the projections: gdn_prologue -> gdn_chunk_fwd -> gdn_out_norm.
  *   q_raw, k_raw [B, T, Hk*dk]; v_raw, z [B, T, Hv*dv] (dtype); wq, wk, wv conv taps as in
  *   gdn_prologue; log_alpha, beta [B, T, Hv]; S0 nullable; norm_w [dv];
- *   y [B, T, Hv, dv] (dtype, output); S_T nullable (output).
+ *   y [B, T, Hv, dv] (y_dtype, output: GDN_BF16 or GDN_F32 for bf16 inputs, GDN_F32 for fp32
+ *   inputs); S_T nullable (output).
  *   workspace: device scratch of at least gdn_layer_workspace_bytes(...) bytes, 256-byte
  *   aligned, or NULL when that size is 0.  Its contents are undefined after the call.
  */
@@ -257,7 +307,7 @@ GDN_API gdn_status gdn_layer_fwd(const void *q_raw, const void *k_raw, const voi
                          void *workspace, size_t workspace_bytes,
                          int B, int T, int Hk, int Hv, int dk, int dv, int chunk,
                          float scale, float l2_eps, float norm_eps,
-                         gdn_dtype dtype, gdn_stream_t stream);
+                         gdn_dtype dtype, gdn_dtype y_dtype, gdn_stream_t stream);
 
 /* Scratch bytes gdn_layer_fwd needs for these sizes (host only, no CUDA call); 0 if none. */
 GDN_API size_t gdn_layer_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, int chunk,
@@ -289,7 +339,7 @@ GDN_API gdn_status gdn_layer_fwd_static(const void *q_raw, const void *k_raw, co
                          const float *norm_w, void *y, float *S_T,
                          int B, int T, int Hk, int Hv, int dk, int dv, int chunk,
                          float scale, float l2_eps, float norm_eps,
-                         gdn_dtype dtype, gdn_stream_t stream);
+                         gdn_dtype dtype, gdn_dtype y_dtype, gdn_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -3,16 +3,20 @@
 Tolerances (from the target statement of this library, applied to every workload):
   * fp32 workloads: max |x - x_ref| <= 1e-4 for the output o and the final state.
   * bf16-input / fp32-state workloads: max |o - o_ref| / rms(o_ref) <= 2e-2 and
-    max |S - S_ref| / rms(S_ref) <= 1e-2 for the final state.
+    max |S - S_ref| / rms(S_ref) <= 1e-2 for the final state, the RMS taken over the whole
+    output (or state) of the workload.  These plain bounds are checked on fp32 outputs: every
+    bf16-input entry point can write o (or the layer's y) in fp32.
 
-The output o of the bf16 workloads is stored in bf16 ("L'attention hybride", "Le float32 n'est pas
-un détail": the state is float32 while the rest of the model is BF16).  Rounding a value r to bf16
-moves it by up to half a bf16 ulp, 2^(floor(log2|r|) - 8), which alone reaches 2.5-2.9% of the RMS
-on the long-context workload (max |o| / rms(o) is 8-10 there).  So for bf16 outputs the 2e-2 bound
-applies to the error beyond that rounding:
-    max_i max(0, |o_i - r_i| - halfulp_bf16(r_i)) / rms(r)        (``rel_rms_bf16``)
-and the tests also report the plain max/rms and Frobenius-relative errors.
+A bf16-stored output cannot meet the plain bound whatever the kernel does: rounding a value r to
+bf16 moves it by up to half a bf16 ulp, 2^(floor(log2|r|) - 8), and max |o| / rms(o) is about 10.7
+on the prefill and decode workloads (2.1 % of the RMS from the rounding alone) and 49 for the
+layer's y.  For bf16 outputs the tests therefore also check the error beyond that rounding,
+    max_i max(0, |o_i - r_i| - halfulp_bf16(r_i)) / rms(r)        (``rel_rms_bf16``),
+an extra report next to the plain check of the fp32 leg.
 """
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -64,3 +68,23 @@ def frob_rel(got, ref) -> float:
 
 def to_dev(d, device="cuda"):
     return {k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+
+
+def global_rel_rms(got_parts, ref_parts) -> float:
+    """max |got - ref| over several parts of one output, over the RMS of the whole reference."""
+    num, ss, n = 0.0, 0.0, 0
+    for g, r in zip(got_parts, ref_parts):
+        if r.size == 0:
+            continue
+        num = max(num, float(np.max(np.abs(np64(g) - r))))
+        ss += float(np.sum(r ** 2))
+        n += r.size
+    return num / max(np.sqrt(ss / max(n, 1)), 1e-30)
+
+
+def report(name: str, **errors):
+    """Append measured errors to the file named by GDN_PARITY_LOG (if set), one JSON line each."""
+    path = os.environ.get("GDN_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"test": name, **{k: float(v) for k, v in errors.items()}}) + "\n")

@@ -63,30 +63,88 @@ P = ctypes.c_void_p
 FAKE = P(0x1000)          # never dereferenced: validation fails or returns before any CUDA call
 
 
-def chunk(L, B=1, T=64, Hk=2, Hv=2, dk=16, dv=16, C=16, dtype=0, q=FAKE, o=FAKE, variant=0):
-    return L.gdn_chunk_fwd_ex(q, FAKE, FAKE, FAKE, FAKE, None, o, None, B, T, Hk, Hv, dk, dv, C,
-                              1.0, dtype, variant, None)
+def chunk(L, B=1, T=64, Hk=2, Hv=2, dk=16, dv=16, C=16, dtype=0, q=FAKE, o=FAKE, variant=0,
+          odtype=None, ws=None, ws_bytes=0):
+    odt = dtype if odtype is None else odtype
+    return L.gdn_chunk_fwd_ex(q, FAKE, FAKE, FAKE, FAKE, None, o, None, ws, ws_bytes, B, T, Hk, Hv,
+                              dk, dv, C, 1.0, dtype, odt, variant, None)
 
 
 @pytest.mark.parametrize("kw,expect", [
     (dict(B=-1), 1), (dict(T=-5), 1), (dict(Hk=0), 1), (dict(Hv=3), 1),   # Hv % Hk != 0
     (dict(dk=0), 1), (dict(C=0), 1), (dict(dtype=7), 1), (dict(variant=9), 1),
+    (dict(odtype=5), 1),                                                  # bad output dtype
     (dict(q=None), 1), (dict(o=None), 1), (dict(q=P(0x1004)), 1),        # null / misaligned
     (dict(dk=48), 2), (dict(dv=256), 2), (dict(C=128), 2), (dict(C=8), 2),
     (dict(variant=2, dtype=0), 2),                                        # no tcgen05 fp32 kernel
+    (dict(dtype=0, odtype=1), 2),                                         # fp32 in, bf16 out
     (dict(B=0), 0),                                                       # empty batch: no work
 ])
 def test_chunk_fwd_validation(L, kw, expect):
     assert chunk(L, **kw) == expect
 
 
+TC = dict(B=2, T=130, Hk=2, Hv=6, dk=128, dv=128, C=64, dtype=1)
+
+
+def test_chunk_fwd_workspace_bytes(L):
+    """The tensor-core family needs one operand record per (batch, value head, chunk); the CUDA-core
+    family and empty calls need none."""
+    need = L.gdn_chunk_fwd_workspace_bytes(2, 130, 2, 6, 128, 128, 64, 1)
+    assert need > 0 and need == 2 * 6 * 3 * (need // 36)
+    assert L.gdn_chunk_fwd_workspace_bytes(2, 130, 2, 6, 128, 128, 64, 0) == 0    # fp32: SIMT
+    assert L.gdn_chunk_fwd_workspace_bytes(2, 130, 2, 6, 64, 64, 64, 1) == 0      # d64: SIMT
+    assert L.gdn_chunk_fwd_workspace_bytes(0, 130, 2, 6, 128, 128, 64, 1) == 0
+    # a single sequence of 256 chunks or more also keeps the two states between ranges
+    n255 = L.gdn_chunk_fwd_workspace_bytes(1, 255 * 64, 16, 48, 128, 128, 64, 1)
+    n256 = L.gdn_chunk_fwd_workspace_bytes(1, 256 * 64, 16, 48, 128, 128, 64, 1)
+    assert n256 - n255 * 256 // 255 == 2 * 48 * 128 * 128 * 4
+    assert L.gdn_chunk_fwd_varlen_workspace_bytes(3, 130, 2, 6, 128, 128, 64, 1) == \
+        L.gdn_chunk_fwd_workspace_bytes(3, 130, 2, 6, 128, 128, 64, 1)
+
+
+def test_chunk_fwd_rejects_missing_or_small_workspace(L):
+    """A tensor-core call whose workspace is missing, too small or not 256-byte aligned returns
+    GDN_ERR_INVALID_ARG (1) before any work (the pointers are fakes, never dereferenced)."""
+    need = L.gdn_chunk_fwd_workspace_bytes(2, 130, 2, 6, 128, 128, 64, 1)
+    assert chunk(L, **TC) == 1                                           # none
+    assert chunk(L, **TC, ws=P(0x10000), ws_bytes=need - 1) == 1         # one byte short
+    assert chunk(L, **TC, ws=P(0x10010), ws_bytes=need) == 1             # misaligned
+    t6 = [FAKE] * 6
+    assert L.gdn_chunk_fwd_varlen(*t6, 2, 64, FAKE, FAKE, FAKE, None, 0, 128, 2, 6, 128, 128, 64,
+                                  1.0, 1, 1, None) == 1
+
+
+def test_chunk_fwd_ba_validation(L):
+    """Gates from in_proj_ba: only the tensor-core family; missing ba or workspace rejected."""
+    f = L.gdn_chunk_fwd_ba
+    t3 = [FAKE] * 3
+    big = [P(0x100000), 1 << 40]
+    assert f(*t3, FAKE, None, FAKE, None, *big, 1, 64, 2, 6, 64, 64, 64, 1.0, 1, 1, None) == 2
+    assert f(*t3, None, None, FAKE, None, *big, 1, 64, 2, 6, 128, 128, 64, 1.0, 1, 1, None) == 1
+    assert f(*t3, FAKE, None, FAKE, None, None, 0, 1, 64, 2, 6, 128, 128, 64, 1.0, 1, 1,
+             None) == 1
+    assert f(*t3, FAKE, None, FAKE, None, *big, 0, 64, 2, 6, 128, 128, 64, 1.0, 1, 1, None) == 0
+
+
+def test_launch_count_rejects_what_the_call_rejects(L):
+    assert L.gdn_chunk_fwd_launches(1, 64, 2, 3, 16, 16, 16, 0, 0, 148) == -1   # Hv % Hk
+    assert L.gdn_chunk_fwd_launches(1, 64, 2, 2, 48, 16, 16, 0, 0, 148) == -1   # dk
+    assert L.gdn_chunk_fwd_launches(1, 64, 2, 2, 16, 16, 16, 0, 2, 148) == -1   # no fp32 tcgen05
+    assert L.gdn_chunk_fwd_launches(1, 64, 2, 2, 16, 16, 16, 0, 0, -1) == -1    # bad SM count
+    assert L.gdn_chunk_fwd_launches(1, 64, 2, 2, 16, 16, 16, 0, 0, 148) == 1    # SIMT: one
+    assert L.gdn_chunk_fwd_launches(0, 64, 2, 2, 16, 16, 16, 0, 0, 148) == 0    # nothing to do
+
+
 def test_decode_validation(L):
     f = L.gdn_decode_step
-    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, -1, 2, 2, 16, 16, 1.0, 0, None) == 1
-    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 3, 16, 16, 1.0, 0, None) == 1
-    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 4, 2, 2, 16, 16, 1.0, 0, None) == 1
-    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 2, 24, 16, 1.0, 0, None) == 2
-    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, 2, 16, 16, 1.0, 0, None) == 0
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, -1, 2, 2, 16, 16, 1.0, 0, 0, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 3, 16, 16, 1.0, 0, 0, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 4, 2, 2, 16, 16, 1.0, 0, 0, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 2, 24, 16, 1.0, 0, 0, None) == 2
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 2, 16, 16, 1.0, 0, 1, None) == 2
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 2, 16, 16, 1.0, 1, 6, None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, 2, 16, 16, 1.0, 0, 0, None) == 0
 
 
 def test_decode_layer_validation(L):
@@ -106,14 +164,16 @@ def test_decode_layer_validation(L):
 def test_varlen_validation(L):
     f = L.gdn_chunk_fwd_varlen
     t6 = [FAKE] * 6
+    ws = [FAKE, FAKE, FAKE, P(0x100000), 1 << 40]                 # S0, o, S_T, workspace, bytes
     # only the tensor-core family (bf16, 128, 128, chunk 64) is supported
-    assert f(*t6, 2, 64, FAKE, FAKE, FAKE, 128, 2, 6, 64, 64, 64, 1.0, 1, None) == 2
-    assert f(*t6, 2, 64, FAKE, FAKE, FAKE, 128, 2, 6, 128, 128, 64, 1.0, 0, None) == 2
-    assert f(*t6, -1, 64, FAKE, FAKE, FAKE, 128, 2, 6, 128, 128, 64, 1.0, 1, None) == 1
+    assert f(*t6, 2, 64, *ws, 128, 2, 6, 64, 64, 64, 1.0, 1, 1, None) == 2
+    assert f(*t6, 2, 64, *ws, 128, 2, 6, 128, 128, 64, 1.0, 0, 0, None) == 2
+    assert f(*t6, -1, 64, *ws, 128, 2, 6, 128, 128, 64, 1.0, 1, 1, None) == 1
+    assert f(*t6, 2, 64, *ws, 128, 2, 6, 128, 128, 64, 1.0, 1, 9, None) == 1   # o dtype
     u = list(t6)
     u[5] = None                                                   # cu_seqlens
-    assert f(*u, 2, 64, FAKE, FAKE, FAKE, 128, 2, 6, 128, 128, 64, 1.0, 1, None) == 1
-    assert f(*t6, 0, 64, FAKE, FAKE, FAKE, 128, 2, 6, 128, 128, 64, 1.0, 1, None) == 0
+    assert f(*u, 2, 64, *ws, 128, 2, 6, 128, 128, 64, 1.0, 1, 1, None) == 1
+    assert f(*t6, 0, 64, *ws, 128, 2, 6, 128, 128, 64, 1.0, 1, 1, None) == 0
 
 
 def test_gates_validation(L):
@@ -143,21 +203,26 @@ def test_prologue_and_out_norm_validation(L):
 def test_layer_validation(L):
     args = [FAKE] * 13
     # workspace missing although one is needed
-    assert L.gdn_layer_fwd(*args, None, 0, 1, 8, 2, 4, 16, 16, 16, 1.0, 1e-6, 1e-5, 1,
+    assert L.gdn_layer_fwd(*args, None, 0, 1, 8, 2, 4, 16, 16, 16, 1.0, 1e-6, 1e-5, 1, 1,
                            None) == 1
     # misaligned workspace
     assert L.gdn_layer_fwd(*args, P(0x1010), 1 << 30, 1, 8, 2, 4, 16, 16, 16, 1.0, 1e-6, 1e-5,
-                           1, None) == 1
+                           1, 1, None) == 1
+    # fp32 inputs with a bf16 y
+    assert L.gdn_layer_fwd(*args, P(0x1000), 1 << 30, 1, 8, 2, 4, 16, 16, 16, 1.0, 1e-6, 1e-5,
+                           0, 1, None) == 2
 
 
 def test_tensor_core_forward_rejects_more_than_65535_chunks(L):
     """The tensor-core family takes sequences of up to 65535 chunks of 64 tokens; a longer one
-    returns GDN_ERR_UNSUPPORTED (2) before any allocation or launch (the pointers are fakes)."""
+    returns GDN_ERR_UNSUPPORTED (2) before any launch (the pointers are fakes)."""
     longest = 65535 * 64
     t8 = [FAKE] * 8
+    big = [P(0x100000), 1 << 50]
     for variant in (0, 2):                                         # auto, tcgen05
-        assert L.gdn_chunk_fwd_ex(*t8, 1, longest + 1, 16, 48, 128, 128, 64, 1.0, 1, variant,
-                                  None) == 2
+        assert L.gdn_chunk_fwd_ex(*t8, *big, 1, longest + 1, 16, 48, 128, 128, 64, 1.0, 1, 1,
+                                  variant, None) == 2
+    assert L.gdn_chunk_fwd_launches(1, longest + 1, 16, 48, 128, 128, 64, 1, 0, 148) == -1
     t6 = [FAKE] * 6
-    assert L.gdn_chunk_fwd_varlen(*t6, 1, longest + 1, FAKE, FAKE, FAKE, longest + 1, 16, 48,
-                                  128, 128, 64, 1.0, 1, None) == 2
+    assert L.gdn_chunk_fwd_varlen(*t6, 1, longest + 1, FAKE, FAKE, FAKE, *big, longest + 1, 16,
+                                  48, 128, 128, 64, 1.0, 1, 1, None) == 2

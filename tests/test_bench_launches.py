@@ -1,24 +1,18 @@
-"""bench.py's count of the kernels one tensor-core forward call launches (its `gpu_launches`
-claim), for the library's three launch schedules, on a 148-SM device (no GPU: the device query
-is replaced)."""
-import os
-import sys
-import types
-
+"""The count of kernels one chunked-forward call launches (bench.py's `gpu_launches` claim) comes
+from the library itself (gdn_chunk_fwd_launches, decided by the same code as the launch); here it
+is checked, without a GPU, against the three launch schedules on a 148-SM device."""
 import pytest
 import torch
 
-ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-sys.path.insert(0, ROOT)
-
-import bench  # noqa: E402
-import gdn_inputs as gi  # noqa: E402
+import gdn_inputs as gi
 
 
-@pytest.fixture
-def b200(monkeypatch):
-    monkeypatch.setattr(torch.cuda, "get_device_properties",
-                        lambda dev: types.SimpleNamespace(multi_processor_count=148))
+@pytest.fixture(scope="module")
+def gdn():
+    from gated_deltanet_linear_18_b200 import _build
+    _build.build()
+    import gated_deltanet_linear_18_b200 as g
+    return g
 
 
 @pytest.mark.parametrize("name, sizes, expected", [
@@ -36,10 +30,16 @@ def b200(monkeypatch):
     ("prefill", dict(B=1, T=259 * 64, Hk=4, Hv=12), 6),
     ("prefill", dict(B=1, T=300 * 64, Hk=16, Hv=80), 2),  # 2 Hv > 148 SMs: no ranges
 ])
-def test_tensor_core_launches_per_call(b200, name, sizes, expected):
+def test_tensor_core_launches_per_call(gdn, name, sizes, expected):
     w = gi.WORKLOADS[name].with_sizes(**sizes) if sizes else gi.WORKLOADS[name]
-    assert bench.tc_launches_per_call(w, None, "tcgen05") == expected
+    assert gdn.chunk_fwd_launches(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv, w.chunk, torch.bfloat16,
+                                  sms=148) == expected
 
 
-def test_simt_forward_is_one_launch(b200):
-    assert bench.tc_launches_per_call(gi.WORKLOADS["tiny_fp32"], None, "simt") == 1
+def test_simt_forward_is_one_launch(gdn):
+    w = gi.WORKLOADS["tiny_fp32"]
+    assert gdn.chunk_fwd_launches(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv, w.chunk, torch.float32,
+                                  sms=148) == 1
+    w = gi.WORKLOADS["prefill"]
+    assert gdn.chunk_fwd_launches(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv, w.chunk, torch.bfloat16,
+                                  variant="simt", sms=148) == 1

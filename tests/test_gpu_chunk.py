@@ -5,16 +5,16 @@ import torch
 
 import gdn_inputs as gi
 import gated_deltanet_linear_18_b200 as gdn
-from gpu_util import (TOL_BF16_OUT, TOL_BF16_STATE, TOL_F32_ABS, frob_rel, max_abs, np64,
-                      out_err, rel_rms, to_dev)
+from gpu_util import (TOL_BF16_OUT, TOL_BF16_STATE, TOL_F32_ABS, frob_rel, halfulp_bf16,
+                      max_abs, np64, out_err, rel_rms, report, to_dev)
 
 pytestmark = pytest.mark.gpu
 
 
-def run(x, chunk, variant="auto", scale=1.0):
+def run(x, chunk, variant="auto", scale=1.0, out_dtype=None):
     d = to_dev(x)
     o, sT = gdn.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
-                          chunk=chunk, scale=scale, variant=variant)
+                          chunk=chunk, scale=scale, variant=variant, out_dtype=out_dtype)
     torch.cuda.synchronize()
     gdn.check_error()
     return o, sT
@@ -171,33 +171,183 @@ def test_nonfinite_propagates(variant, what, idx, val):
     assert torch.isfinite(o[1].float()).all() and torch.isfinite(sT[1]).all()
 
 
-def _sampled_heads(orc, x, o, sT, heads, Hk, Hv):
-    G = Hv // Hk
-    for b, h in heads:
-        hk = h // G
-        sl = lambda t, hh: t[b:b + 1, :, hh:hh + 1]
-        s0 = None if x["S0"] is None else x["S0"][b:b + 1, h:h + 1]
-        o_ref, s_ref = orc.gated_delta(sl(x["q"], hk), sl(x["k"], hk), sl(x["v"], h),
-                                       x["log_alpha"][b:b + 1, :, h:h + 1],
-                                       x["beta"][b:b + 1, :, h:h + 1], s0)
-        go, gs = o[b:b + 1, :, h:h + 1], sT[b:b + 1, h:h + 1]
-        e_o, e_s = out_err(go, o_ref), rel_rms(gs, s_ref)
-        assert e_o <= TOL_BF16_OUT, (b, h, e_o, rel_rms(go, o_ref), frob_rel(go, o_ref))
-        assert e_s <= TOL_BF16_STATE, (b, h, e_s, frob_rel(gs, s_ref))
+class AllHeads:
+    """Errors of several GPU results of one workload against one oracle run over every (batch,
+    value head) pair, the oracle taken a few key heads at a time (bounded host memory).  Plain
+    errors are max |x - x_ref| over the RMS of the whole reference output (or final state); the
+    worst single head, normalised by its own RMS, and the Frobenius error are reported too."""
+
+    def __init__(self, names):
+        self.acc = {n: dict(num_o=0.0, num_s=0.0, ex_o=0.0, head_o=0.0, head_s=0.0, d2=0.0)
+                    for n in names}
+        self.ss_o = self.ss_s = 0.0
+        self.n_o = self.n_s = 0
+
+    def add(self, outs, o_ref, s_ref):
+        """outs: name -> (o, S_T) slices [B, T, h, dv] / [B, h, dk, dv] matching the refs."""
+        self.ss_o += float(np.sum(o_ref ** 2))
+        self.ss_s += float(np.sum(s_ref ** 2))
+        self.n_o += o_ref.size
+        self.n_s += s_ref.size
+        nh = o_ref.shape[2]
+        for name, (o, sT) in outs.items():
+            a = self.acc[name]
+            do = np.abs(np64(o) - o_ref)
+            ds = np.abs(np64(sT) - s_ref)
+            a["num_o"] = max(a["num_o"], float(do.max()))
+            a["num_s"] = max(a["num_s"], float(ds.max()))
+            a["d2"] += float(np.sum(do ** 2))
+            if o.dtype == torch.bfloat16:
+                a["ex_o"] = max(a["ex_o"], float(np.max(np.maximum(do - halfulp_bf16(o_ref), 0))))
+            for j in range(nh):
+                r = o_ref[:, :, j]
+                a["head_o"] = max(a["head_o"], float(do[:, :, j].max()) /
+                                  max(float(np.sqrt(np.mean(r ** 2))), 1e-30))
+                rs = s_ref[:, j]
+                a["head_s"] = max(a["head_s"], float(ds[:, j].max()) /
+                                  max(float(np.sqrt(np.mean(rs ** 2))), 1e-30))
+
+    def errors(self, name):
+        a = self.acc[name]
+        rms_o = np.sqrt(self.ss_o / self.n_o)
+        rms_s = np.sqrt(self.ss_s / self.n_s)
+        return dict(o_plain=a["num_o"] / rms_o, o_beyond_halfulp=a["ex_o"] / rms_o,
+                    o_worst_head=a["head_o"], o_frob=np.sqrt(a["d2"] / self.ss_o),
+                    state=a["num_s"] / rms_s, state_worst_head=a["head_s"])
 
 
-def test_prefill_full_size_sampled(orc):
-    """Prefill workload at full size (B4 T2048 Hk16 Hv48 d128 chunk 64), launched exactly as the
-    bench launches it; the oracle checks sampled heads, each one computed whole."""
+def all_heads_check(orc, name, x, w, outs, key_heads_per_oracle_call):
+    """Runs the oracle over every head and checks: fp32 outputs at the plain bound, bf16 outputs
+    beyond their storage rounding, every final state at the plain state bound."""
+    G = w.Hv // w.Hk
+    chk = AllHeads(outs.keys())
+    for k0 in range(0, w.Hk, key_heads_per_oracle_call):
+        k1 = min(w.Hk, k0 + key_heads_per_oracle_call)
+        h0, h1 = k0 * G, k1 * G
+        s0 = None if x["S0"] is None else x["S0"][:, h0:h1]
+        o_ref, s_ref = orc.gated_delta(x["q"][:, :, k0:k1], x["k"][:, :, k0:k1],
+                                       x["v"][:, :, h0:h1], x["log_alpha"][:, :, h0:h1],
+                                       x["beta"][:, :, h0:h1], s0)
+        chk.add({n: (o[:, :, h0:h1], sT[:, h0:h1]) for n, (o, sT) in outs.items()}, o_ref, s_ref)
+    for n, (o, _) in outs.items():
+        e = chk.errors(n)
+        report(f"{name}[{n}]", **e)
+        assert e["state"] <= TOL_BF16_STATE, (n, e)
+        if o.dtype == torch.float32:
+            assert e["o_plain"] <= TOL_BF16_OUT, (n, e)
+        else:
+            assert e["o_beyond_halfulp"] <= TOL_BF16_OUT, (n, e)
+
+
+def test_prefill_full_size_all_heads(orc):
+    """Prefill workload at full size (B4 T2048 Hk16 Hv48 d128 chunk 64), launched as the bench
+    launches it (bf16 o) and with an fp32 o; the oracle checks every (batch, value head): the
+    fp32 o at max |o - o_ref| / rms(o_ref) <= 2e-2, the final state at <= 1e-2."""
     w = gi.WORKLOADS["prefill"]
     x = gi.make_inputs(w)
-    o, sT = run(x, w.chunk)
-    _sampled_heads(orc, x, o.cpu(), sT.cpu(), [(0, 0), (1, 17), (2, 46), (3, 47)], w.Hk, w.Hv)
+    ob, sb = run(x, w.chunk)
+    of, sf = run(x, w.chunk, out_dtype=torch.float32)
+    all_heads_check(orc, "prefill", x, w, {"bf16_o": (ob.cpu(), sb.cpu()),
+                                           "fp32_o": (of.cpu(), sf.cpu())}, 16)
 
 
-def test_long_context_full_size_sampled(orc):
-    """Long context (B1 T65536, S0 ~ N(0, 0.02)): output and final state of sampled heads."""
+def test_long_context_full_size_all_heads(orc):
+    """Long context (B1 T65536, S0 ~ N(0, 0.02), run in ranges of 128 chunks): every value head's
+    output and final state, bf16 and fp32 o."""
     w = gi.WORKLOADS["long_context"]
     x = gi.make_inputs(w)
-    o, sT = run(x, w.chunk)
-    _sampled_heads(orc, x, o.cpu(), sT.cpu(), [(0, 0), (0, 29), (0, 47)], w.Hk, w.Hv)
+    ob, sb = run(x, w.chunk)
+    ob, sb = ob.cpu(), sb.cpu()
+    of, sf = run(x, w.chunk, out_dtype=torch.float32)
+    of, sf = of.cpu(), sf.cpu()
+    all_heads_check(orc, "long_context", x, w, {"bf16_o": (ob, sb), "fp32_o": (of, sf)}, 4)
+
+
+@pytest.mark.parametrize("variant", ["tcgen05", "simt"])
+def test_strong_decay(orc, variant):
+    """log alpha = -softplus(N(0,1)) exp(U(0, 3)): decay of up to e^-60 per token, so the
+    cumulative gates underflow to zero inside a chunk (the pre-pass's block-factored gates must
+    give zeros, not inf * 0)."""
+    w = gi.WORKLOADS["prefill"].with_sizes(B=2, T=300, Hk=2, Hv=6, s0_std=0.02, seed=77)
+    x = gi.make_inputs(w)
+    g = torch.Generator().manual_seed(78)
+    x["log_alpha"] = (-torch.nn.functional.softplus(torch.randn(w.B, w.T, w.Hv, generator=g))
+                      * torch.exp(torch.rand(w.B, w.T, w.Hv, generator=g) * 3.0)).contiguous()
+    assert float(x["log_alpha"].min()) < -20.0
+    of, sf = run(x, 64, variant=variant, out_dtype=torch.float32)
+    ob, _ = run(x, 64, variant=variant)
+    o_ref, s_ref = ref(orc, x)
+    assert torch.isfinite(of).all() and torch.isfinite(sf).all()
+    report(f"strong_decay[{variant}]", o_plain=rel_rms(of, o_ref), state=rel_rms(sf, s_ref),
+           o_beyond_halfulp=out_err(ob, o_ref))
+    assert rel_rms(of, o_ref) <= TOL_BF16_OUT
+    assert rel_rms(sf, s_ref) <= TOL_BF16_STATE
+    assert out_err(ob, o_ref) <= TOL_BF16_OUT
+
+
+def _orthonormal_keys(T, Hk, d, g):
+    """k_t = e_{pi(t)} for a random permutation pi (T <= d): orthonormal and exact in bf16."""
+    k = torch.zeros(1, T, Hk, d)
+    for hk in range(Hk):
+        perm = torch.randperm(d, generator=g)[:T]
+        k[0, torch.arange(T), hk, perm] = 1.0
+    return k
+
+
+@pytest.mark.parametrize("variant", ["tcgen05", "simt"])
+def test_retrieval_alpha1_beta1_orthonormal_keys(orc, variant):
+    """alpha = 1, beta = 1 and orthonormal keys ("L'attention hybride", "La récurrence": beta
+    replaces the association bound to k_t): every written pair is retrieved, S_T k_i = v_i, and
+    with q_t = k_t the output is o_t = v_t exactly in real arithmetic, whatever S0 held."""
+    T, Hk, Hv, d = 128, 2, 6, 128
+    g = torch.Generator().manual_seed(5)
+    k = _orthonormal_keys(T, Hk, d, g)
+    x = {"q": k.clone().to(torch.bfloat16), "k": k.to(torch.bfloat16),
+         "v": torch.randn(1, T, Hv, d, generator=g).to(torch.bfloat16),
+         "log_alpha": torch.zeros(1, T, Hv), "beta": torch.ones(1, T, Hv),
+         "S0": torch.randn(1, Hv, d, d, generator=g) * 0.02}
+    of, sf = run(x, 64, variant=variant, out_dtype=torch.float32)
+    of, sf = of.cpu().double(), sf.cpu().double()
+    v = x["v"].double()
+    assert float((of - v).abs().max()) <= 1e-3 * float(v.abs().max())
+    kk = k.double()
+    for h in range(Hv):
+        hk = h // (Hv // Hk)
+        got = torch.einsum("td,de->te", kk[0, :, hk], sf[0, h])     # (S_T k_t) as rows
+        assert float((got - v[0, :, h]).abs().max()) <= 1e-3 * float(v.abs().max())
+    o_ref, s_ref = ref(orc, x)
+    assert rel_rms(sf, s_ref) <= TOL_BF16_STATE
+
+
+@pytest.mark.parametrize("variant", ["tcgen05", "simt"])
+def test_same_key_written_twice_keeps_the_second_value(variant):
+    """The same key written twice with beta = 1, alpha = 1 (tokens 3 and 40, in one chunk, and
+    tokens 70 and 130, across chunks); every other token writes a basis key orthogonal to both.
+    Reading with that key returns the second value ("Chapitre 16 - Assembler un système de type
+    Kimi K3", 16.4: the linear memory is correctable)."""
+    T, Hk, Hv, d = 160, 1, 3, 128
+    g = torch.Generator().manual_seed(9)
+    a, b = 17, 93                                  # the two repeated keys e_a, e_b
+    others = [i for i in range(d) if i not in (a, b)]
+    perm = torch.randperm(len(others), generator=g)
+    k = torch.zeros(1, T, Hk, d)
+    for t in range(T):
+        k[0, t, 0, others[int(perm[t % len(others)])]] = 1.0
+    for t in (3, 40):
+        k[0, t, 0].zero_()
+        k[0, t, 0, a] = 1.0
+    for t in (70, 130):
+        k[0, t, 0].zero_()
+        k[0, t, 0, b] = 1.0
+    q = torch.zeros_like(k)
+    q[0, T - 1, 0, a] = 1.0
+    q[0, T - 2, 0, b] = 1.0
+    x = {"q": q.to(torch.bfloat16), "k": k.to(torch.bfloat16),
+         "v": torch.randn(1, T, Hv, d, generator=g).to(torch.bfloat16),
+         "log_alpha": torch.zeros(1, T, Hv), "beta": torch.ones(1, T, Hv), "S0": None}
+    of, _ = run(x, 64, variant=variant, out_dtype=torch.float32)
+    of, v = of.cpu().double(), x["v"].double()
+    tol = 1e-3 * float(v.abs().max())
+    assert float((of[0, T - 1] - v[0, 40]).abs().max()) <= tol
+    assert float((of[0, T - 2] - v[0, 130]).abs().max()) <= tol
+    assert float((of[0, T - 1] - v[0, 3]).abs().max()) > 100 * tol     # the first value is gone

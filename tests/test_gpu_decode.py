@@ -5,19 +5,19 @@ import torch
 
 import gdn_inputs as gi
 import gated_deltanet_linear_18_b200 as gdn
-from gpu_util import (TOL_BF16_OUT, TOL_BF16_STATE, TOL_F32_ABS, halfulp_bf16, max_abs, np64,
-                      out_err, rel_rms)
+from gpu_util import (TOL_BF16_OUT, TOL_BF16_STATE, TOL_F32_ABS, frob_rel, halfulp_bf16,
+                      max_abs, np64, out_err, rel_rms, report)
 
 pytestmark = pytest.mark.gpu
 
 
-def run_steps(x, scale=1.0):
+def run_steps(x, scale=1.0, out_dtype=None):
     d = {k: v.cuda() for k, v in x.items()}
     S = d["S0"].clone()
     outs = []
     for s in range(d["q"].shape[0]):
         outs.append(gdn.decode_step(d["q"][s], d["k"][s], d["v"][s], d["log_alpha"][s],
-                                    d["beta"][s], S, scale=scale))
+                                    d["beta"][s], S, scale=scale, out_dtype=out_dtype))
     torch.cuda.synchronize()
     return torch.stack(outs), S
 
@@ -34,19 +34,26 @@ def test_fp32_shapes(orc, dk, dv):
     assert max_abs(S, S_ref) <= TOL_F32_ABS
 
 
-def test_decode_full_size_sampled(orc):
-    """The decode workload at full size (256 sequences, Hk16 Hv48 d128, 100 steps, S0 != 0); the
-    oracle follows sampled sequences over all 100 steps (o at every step, S after step 100)."""
+def test_decode_full_size_all_sequences(orc):
+    """The decode workload at full size (256 sequences, Hk16 Hv48 d128, 100 steps, S0 != 0): the
+    oracle follows every sequence over all 100 steps.  With an fp32 o: max |o - o_ref| /
+    rms(o_ref) <= 2e-2 over all steps and max |S - S_ref| / rms(S_ref) <= 1e-2 after step 100;
+    with the bf16 o the bench times, the error beyond the bf16 rounding."""
     w = gi.WORKLOADS["decode"]
     x = gi.make_decode_inputs(w)
-    o, S = run_steps(x)
-    o, S = o.cpu(), S.cpu()
-    for n in (0, 101, 255):
-        sl = lambda t: t[:, n:n + 1]
-        o_ref, S_ref = orc.decode_steps(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["log_alpha"]),
-                                        sl(x["beta"]), x["S0"][n:n + 1])
-        assert out_err(o[:, n:n + 1], o_ref) <= TOL_BF16_OUT
-        assert rel_rms(S[n:n + 1], S_ref) <= TOL_BF16_STATE
+    of, Sf = run_steps(x, out_dtype=torch.float32)
+    of, Sf = of.cpu(), Sf.cpu()
+    ob, Sb = run_steps(x)
+    ob, Sb = ob.cpu(), Sb.cpu()
+    o_ref, S_ref = orc.decode_steps(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"])
+    e = dict(o_plain=rel_rms(of, o_ref), o_frob=frob_rel(of, o_ref), state=rel_rms(Sf, S_ref),
+             bf16_o_beyond_halfulp=out_err(ob, o_ref), bf16_o_plain=rel_rms(ob, o_ref),
+             bf16_state=rel_rms(Sb, S_ref))
+    report("decode_all", **e)
+    assert e["o_plain"] <= TOL_BF16_OUT, e
+    assert e["state"] <= TOL_BF16_STATE, e
+    assert e["bf16_o_beyond_halfulp"] <= TOL_BF16_OUT, e
+    assert e["bf16_state"] <= TOL_BF16_STATE, e
 
 
 def test_decode_equals_chunk_fwd(orc):

@@ -5,8 +5,8 @@ import torch
 
 import gdn_inputs as gi
 import gated_deltanet_linear_18_b200 as gdn
-from gpu_util import (TOL_BF16_OUT, TOL_BF16_STATE, TOL_F32_ABS, max_abs, np64, out_err,
-                      rel_rms, to_dev)
+from gpu_util import (TOL_BF16_OUT, TOL_BF16_STATE, TOL_F32_ABS, frob_rel, halfulp_bf16,
+                      max_abs, np64, out_err, rel_rms, report, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -50,27 +50,29 @@ def test_out_norm(orc, dtype, dv):
         assert np.all(np.abs(np64(y) - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-6)
 
 
-def _layer(x, w):
+def _layer(x, w, out_dtype=None):
     d = to_dev(x)
     y, sT = gdn.layer_fwd(d["q_raw"], d["k_raw"], d["v_raw"], d["z"], d["conv_wq"], d["conv_wk"],
                           d["conv_wv"], d["log_alpha"], d["beta"], d["S0"], d["norm_w"],
                           Hk=w.Hk, Hv=w.Hv, dk=w.dk, dv=w.dv, chunk=w.chunk,
-                          l2_eps=w.l2_eps, norm_eps=w.norm_eps)
+                          l2_eps=w.l2_eps, norm_eps=w.norm_eps, out_dtype=out_dtype)
     torch.cuda.synchronize()
     gdn.check_error()
     return y, sT
 
 
-def _ref_layer(orc, x, w, b=None, h=None):
+def _ref_layer(orc, x, w, b=None, h=None, act_dtype="model"):
     """Oracle of the whole layer, optionally for one (batch, value head) only (channel slices).
     For bf16 workloads the recurrence's q, k, v are the prologue's outputs rounded to bf16: the
     model keeps every activation but the state in BF16 ("L'attention hybride", "Le float32 n'est
-    pas un détail"), so a bf16 layer hands bf16 q, k, v to the recurrence."""
+    pas un détail"), so a bf16 layer hands bf16 q, k, v to the recurrence.  act_dtype="f64" keeps
+    them in fp64 (reported, not asserted)."""
+    act = w.dtype if act_dtype == "model" else act_dtype
     if h is None:
         return orc.layer_forward(x["q_raw"], x["k_raw"], x["v_raw"], x["z"], x["conv_wq"],
                                  x["conv_wk"], x["conv_wv"], x["log_alpha"], x["beta"], x["S0"],
                                  x["norm_w"], w.Hk, w.Hv, w.dk, w.dv, w.l2_eps, w.norm_eps,
-                                 act_dtype=w.dtype)
+                                 act_dtype=act)
     hk = h // (w.Hv // w.Hk)
     qs, vs = slice(hk * w.dk, (hk + 1) * w.dk), slice(h * w.dv, (h + 1) * w.dv)
     bb = slice(b, b + 1)
@@ -79,27 +81,43 @@ def _ref_layer(orc, x, w, b=None, h=None):
                              x["z"][bb, :, vs], x["conv_wq"][qs], x["conv_wk"][qs],
                              x["conv_wv"][vs], x["log_alpha"][bb, :, h:h + 1],
                              x["beta"][bb, :, h:h + 1], s0, x["norm_w"], 1, 1, w.dk, w.dv,
-                             w.l2_eps, w.norm_eps, act_dtype=w.dtype)
+                             w.l2_eps, w.norm_eps, act_dtype=act)
 
 
 def test_layer_small(orc):
     w = layer_w(B=2, T=150, Hk=2, Hv=16, seed=31, s0_std=0.02)
     x = gi.make_layer_inputs(w)
     y, sT = _layer(x, w)
+    yf, sf = _layer(x, w, out_dtype=torch.float32)
     y_ref, s_ref = _ref_layer(orc, x, w)
     assert out_err(y, y_ref) <= TOL_BF16_OUT, (out_err(y, y_ref), rel_rms(y, y_ref))
+    assert rel_rms(yf, y_ref) <= TOL_BF16_OUT, rel_rms(yf, y_ref)
     assert rel_rms(sT, s_ref) <= TOL_BF16_STATE, rel_rms(sT, s_ref)
+    y64, s64 = _ref_layer(orc, x, w, act_dtype="f64")
+    report("layer_small", y_plain=rel_rms(yf, y_ref), y_plain_vs_fp64_activations=rel_rms(yf, y64),
+           state_vs_fp64_activations=rel_rms(sf, s64))
 
 
-def test_layer_full_size_sampled(orc):
-    """The 8:1 full layer at full size (B2 T8192 Hk16 Hv128); sampled (batch, head) pairs."""
+def test_layer_full_size_all_pairs(orc):
+    """The 8:1 full layer at full size (B2 T8192 Hk16 Hv128), every (batch, value head) pair,
+    with the bf16 y the bench times and with an fp32 y (plain bound)."""
     w = gi.WORKLOADS["layer_8to1"]
     x = gi.make_layer_inputs(w)
-    y, sT = _layer(x, w)
-    y, sT = y.cpu(), sT.cpu()
-    for b, h in ((0, 0), (1, 77), (1, 127)):
-        y_ref, s_ref = _ref_layer(orc, x, w, b, h)
-        e_y = out_err(y[b:b + 1, :, h:h + 1], y_ref)
-        e_s = rel_rms(sT[b:b + 1, h:h + 1], s_ref)
-        assert e_y <= TOL_BF16_OUT, (b, h, e_y)
-        assert e_s <= TOL_BF16_STATE, (b, h, e_s)
+    yb, sb = _layer(x, w)
+    yb, sb = yb.cpu(), sb.cpu()
+    yf, sf = _layer(x, w, out_dtype=torch.float32)
+    yf, sf = yf.cpu(), sf.cpu()
+    y_ref, s_ref = _ref_layer(orc, x, w)
+    e = dict(y_plain=rel_rms(yf, y_ref), y_frob=frob_rel(yf, y_ref), state=rel_rms(sf, s_ref),
+             bf16_y_beyond_halfulp=out_err(yb, y_ref), bf16_y_plain=rel_rms(yb, y_ref),
+             bf16_state=rel_rms(sb, s_ref))
+    del y_ref
+    y64, s64 = _ref_layer(orc, x, w, act_dtype="f64")
+    e.update(y_plain_vs_fp64_activations=rel_rms(yf, y64),
+             y_frob_vs_fp64_activations=frob_rel(yf, y64),
+             state_vs_fp64_activations=rel_rms(sf, s64))
+    report("layer_8to1_all", **e)
+    assert e["y_plain"] <= TOL_BF16_OUT, e
+    assert e["state"] <= TOL_BF16_STATE, e
+    assert e["bf16_y_beyond_halfulp"] <= TOL_BF16_OUT, e
+    assert e["bf16_state"] <= TOL_BF16_STATE, e
