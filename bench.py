@@ -616,21 +616,54 @@ def run_reference(args, world, rank):
 
 
 def profile_case(args):
-    """A few launches of the chunked forward on one workload, nothing else (for profilers)."""
+    """A few calls of one workload's entry point, nothing else (a small, fixed command for
+    profilers): the chunked forward for prefill / long_context, the whole layer for layer_8to1,
+    decode steps for decode and decode_layer.  Sizes from --B / --T (and --B as N for decode)."""
     import gated_deltanet_linear_18_b200 as gdn
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    w = gi.WORKLOADS[args.profile_case]
+    name = args.profile_case
+    w = gi.WORKLOADS[name]
     kw = {k: v for k, v in (("B", args.B), ("T", args.T)) if v is not None}
     if kw:
         w = w.with_sizes(**kw)
-    step = prefill_fn(gdn, to_dev(gi.make_inputs(w), dev), w)
+    if name == "layer_8to1":
+        d = to_dev(gi.make_layer_inputs(w), dev)
+        ws = torch.empty(gdn.layer_workspace_bytes(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv, w.chunk,
+                                                   w.torch_dtype), device=dev, dtype=torch.uint8)
+
+        def step():
+            gdn.layer_fwd(d["q_raw"], d["k_raw"], d["v_raw"], d["z"], d["conv_wq"], d["conv_wk"],
+                          d["conv_wv"], d["log_alpha"], d["beta"], d["S0"], d["norm_w"],
+                          Hk=w.Hk, Hv=w.Hv, dk=w.dk, dv=w.dv, chunk=w.chunk, workspace=ws)
+        launches = 1 + launches_per_call(gdn, w)
+    elif name in ("decode", "decode_layer"):
+        mk = gi.make_decode_inputs if name == "decode" else gi.make_decode_layer_inputs
+        d = to_dev(mk(w.with_sizes(steps=1)), dev)
+        S = d["S0"].clone()
+        if name == "decode":
+            def step():
+                gdn.decode_step(d["q"][0], d["k"][0], d["v"][0], d["log_alpha"][0], d["beta"][0],
+                                S)
+        else:
+            hist = [d["hq"].clone(), d["hk"].clone(), d["hv"].clone()]
+            hout = [torch.empty_like(t) for t in hist]
+
+            def step():
+                gdn.decode_layer_step(d["q_raw"][0], d["k_raw"][0], d["v_raw"][0], d["z"][0],
+                                      *hist, *hout, d["conv_wq"], d["conv_wk"], d["conv_wv"],
+                                      d["log_alpha"][0], d["beta"][0], S, d["norm_w"], Hk=w.Hk,
+                                      Hv=w.Hv, dk=w.dk, dv=w.dv)
+        launches = 1
+    else:
+        step = prefill_fn(gdn, to_dev(gi.make_inputs(w), dev), w)
+        launches = launches_per_call(gdn, w)
     for _ in range(args.steps):
         step()
     torch.cuda.synchronize()
     gdn.check_error(dev)
     print(json.dumps({"profile_case": workload_name(w), "calls": args.steps,
-                      "launches": args.steps * launches_per_call(gdn, w)}), flush=True)
+                      "launches": args.steps * launches}), flush=True)
 
 
 def main():

@@ -177,13 +177,15 @@ gdn_status decode_layer_dispatch(int dk, int dv, const DecodeLayerArgs& a, cudaS
   return GDN_ERR_UNSUPPORTED;
 }
 
-// The CUDA-core recurrence inside gdn_layer_fwd (sizes the tensor-core family does not take):
-// inputs in `dtype`, output o in fp32 for the separate gated norm.
+// The recurrence inside gdn_layer_fwd: inputs in `dtype`, output o in fp32 (for the separate
+// gated norm); `scratch` is the tensor-core forward's hand-over buffer (part of the layer
+// workspace).
 gdn_status layer_chunk_fwd(const void* q, const void* k, const void* v, const float* la,
                            const float* be, const float* S0, float* o, float* S_T, int B, int T,
                            int Hk, int Hv, int dk, int dv, int chunk, float scale,
                            gdn_dtype dtype, void* scratch, cudaStream_t st) {
-  (void)scratch;
+  if (tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16))
+    return tc_chunk_launch(q, k, v, la, be, S0, o, S_T, B, T, Hk, Hv, scale, true, scratch, st);
   if (dtype == GDN_F32)
     return simt_dispatch<float, float>(dk, chunk, q, k, v, la, be, S0, o, S_T, B, T, Hk, Hv, dv,
                                        scale, st);
@@ -491,7 +493,8 @@ gdn_status gdn_prologue(const void* q_raw, const void* k_raw, const void* v_raw,
   if (!wq || !wk || !wv || !aligned4(wq) || !aligned4(wk) || !aligned4(wv))
     return GDN_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  dim3 grid((T + kPrologueTokens - 1) / kPrologueTokens, 2 * Hk + Hv, B);
+  if ((T + kPrologueTokens - 1) / kPrologueTokens > 65535) return GDN_ERR_UNSUPPORTED;
+  dim3 grid(2 * Hk + Hv, (T + kPrologueTokens - 1) / kPrologueTokens, B);
   const int dmax = dk > dv ? dk : dv;
   if (dtype == GDN_F32)
     prologue_kernel<float><<<grid, 128, prologue_smem_bytes(dmax, 4), st>>>(
@@ -530,12 +533,12 @@ size_t gdn_layer_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, i
   const size_t el = dtype == GDN_F32 ? 4 : 2;
   const size_t tok = (size_t)B * T;
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-  // normalised q, k and convolved v in the storage dtype; then either the tensor-core forward's
-  // hand-over buffer (the gated norm runs in its epilogue) or the pre-norm output o in fp32
+  // normalised q, k and convolved v in the storage dtype; the pre-norm output o in fp32; the
+  // tensor-core forward's hand-over buffer when that forward runs
   const size_t qkv = 2 * up(tok * Hk * dk * el) + up(tok * Hv * dv * el);
-  if (tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16))
-    return qkv + up(tc_chunk_scratch_bytes(B, T, Hv));
-  return qkv + up(tok * Hv * dv * 4);
+  const size_t tc = tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16)
+                        ? up(tc_chunk_scratch_bytes(B, T, Hv)) : 0;
+  return qkv + up(tok * Hv * dv * 4) + tc;
 }
 
 gdn_status gdn_layer_fwd(const void* q_raw, const void* k_raw, const void* v_raw, const void* z,
@@ -574,13 +577,11 @@ gdn_status gdn_layer_fwd(const void* q_raw, const void* k_raw, const void* v_raw
                    dtype, stream);
   if (s != GDN_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (tc)   // the recurrence applies the gated norm in its epilogue and writes y itself
-    return tc_layer_launch(qn, kn, vc, log_alpha, beta, S0, y, S_T, B, T, Hk, Hv, scale, z,
-                           norm_w, norm_eps, y_dtype == GDN_F32, rest, st);
   // the recurrence writes o in fp32 so that the gated norm reads it unrounded
   float* o = reinterpret_cast<float*>(rest);
+  void* tc_scratch = rest + up(tok * Hv * dv * 4);
   s = layer_chunk_fwd(qn, kn, vc, log_alpha, beta, S0, o, S_T, B, T, Hk, Hv, dk, dv, chunk, scale,
-                      dtype, nullptr, st);
+                      dtype, tc_scratch, st);
   if (s != GDN_OK) return s;
   const long long rows = (long long)tok * Hv;
   const long long blocks = (rows + 7) / 8;

@@ -64,15 +64,10 @@ constexpr uint32_t OFF_MB = 98304;      // 32 KB, per column half 16 KB: bf16 M 
 constexpr uint32_t OFF_PW = 131072;     // 2 slots x 48 KB: a chunk's PT hi, PT lo, W hi, W lo
 constexpr uint32_t PW_SLOT = 49152;     // after Y (and the update) the o tile is staged there
 constexpr uint32_t OFF_BAR = OFF_PW + 2 * PW_SLOT;
-constexpr int NBAR = 24;
+constexpr int NBAR = 22;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;   // +0 TMEM base, +4 abort flag
 constexpr uint32_t OFF_GAM = OFF_MISC + 16;         // 2 slots (chunk parity) x gamma_t, 64 fp32
-constexpr uint32_t OFF_NW = OFF_GAM + 2 * 256;      // the gated norm's gain, 128 fp32
-constexpr uint32_t SMEM_BYTES = OFF_NW + 512;
-// With the gated norm fused into the o epilogue, the two column halves of a token's row exchange
-// their sums of squares in the chunk's slot, past the staged o tiles (the W lo part, free once
-// the update has read it): 2 halves x 64 tokens fp32.
-constexpr uint32_t RED_OFF = 32768;
+constexpr uint32_t SMEM_BYTES = OFF_GAM + 2 * 256;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 
@@ -86,7 +81,7 @@ constexpr uint32_t TM_X = 0, TM_Y = 256, TM_M = 384;
 enum : int {
   B_QK_FULL = 0, B_QK_EMPTY, B_W_FULL = 2, B_W_EMPTY = 4, B_P_FULL = 6, B_P_EMPTY = 8,
   B_X_FULL = 10, B_R_FULL, B_D3_FULL, B_Y_FULL, B_Y_EMPTY, B_M_READY, B_M_SCALED, B_DRAIN,
-  B_G_FULL = 18, B_G_EMPTY = 20, B_RED = 22, B_END = 24
+  B_G_FULL = 18, B_G_EMPTY = 20, B_END = 22
 };
 static_assert(B_END <= NBAR, "barrier map");
 
@@ -428,7 +423,7 @@ __device__ __forceinline__ SeqSpan seq_span(const int* __restrict__ cu, int s, i
 // every tile, so the recurrence still sees a non-finite value.
 constexpr int kPwTiles = 49152;              // the four operand tiles of a chunk
 constexpr int kPwBytes = kPwTiles + 256;     // + gamma_t = exp(G_t), 64 fp32
-constexpr int PP_THREADS = 128;
+constexpr int PP_THREADS = 256;   // warps w and w + 4 share TMEM lane quadrant w, one column half each
 constexpr uint32_t PP_QK = 0;        // 32 KB: Q cols 0..63 | K cols 0..63 | Q 64..127 | K 64..127;
                                      // P hi over the first Q box, P lo over the second
 constexpr uint32_t PP_TB = 32768;    // solve scratch, then 2 x 8 KB MN-major B tiles [64 rows][128 B]:
@@ -456,8 +451,9 @@ __device__ __forceinline__ void store_b_pair(uint32_t tb, int row, int n, float 
   tc::sts1(o + 8192, __uint_as_float(l));
 }
 
-// grid (Hv, nCmax, sequences), 128 threads; thread r owns TMEM lane r.  CTAs past the end of
-// their sequence return at once.
+// grid (Hv, nCmax, sequences), 256 threads; thread r owns TMEM lane r % 128 and column half r / 128
+// of that lane's row (the solve runs on the first 128).  CTAs past the end of their sequence
+// return at once.
 __global__ void __launch_bounds__(PP_THREADS, 4)
 pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const float* __restrict__ log_alpha, const float* __restrict__ beta,
@@ -499,7 +495,8 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + PP_BAR + 16);
-  const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
+  const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+  const int row = tid & 127, half = tid >> 7;         // TMEM lane and column half of this thread
   GDN_TRACE_PP(1);
   if (tid == 0) {
     tc::mbar_arrive_expect_tx(tma_bar, 32768);
@@ -576,23 +573,24 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
   GDN_TRACE_PP(3);
   tc::tc_fence_after();
   {
-    // row r of S: r < 64 is (q_t . k_j), r >= 64 is (k_t . k_j), t = r mod 64
-    float s[64];
-    tc::tmem_ld32(tmem + lane_off, *reinterpret_cast<float(*)[32]>(&s[0]));
-    tc::tmem_ld32(tmem + lane_off + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
+    // row r of S: r < 64 is (q_t . k_j), r >= 64 is (k_t . k_j), t = r mod 64; this thread takes
+    // columns j = 32 half .. 32 half + 31
+    float s[32];
+    tc::tmem_ld32(tmem + lane_off + 32 * half, s);
     tc::tmem_wait_ld();
     // exp(G_t - G_j) = 2^(G'_t - G'_j) inside t's 16-token block directly, across blocks as
     // 2^(G'_t - G'_16ti) E[ti][j] (both factors <= 1, so strong decay underflows to 0 instead of
     // overflowing); P takes scale and j <= t, A takes beta_t and j < t
-    const int t = tid & 63, ti = t >> 4;
-    const bool isP = tid < 64;
+    const int t = row & 63, ti = t >> 4;
+    const bool isP = row < 64;
     const float gt = gG[t];
     const float rowf = (isP ? scale : gB[t]) * tc::ex2(gt - gG[16 * ti]);
     const float diagf = isP ? scale : gB[t];
     const int jmax = isP ? t : t - 1;                 // last j kept
     float sum = 0.f;
 #pragma unroll
-    for (int kb = 0; kb < 4; ++kb) {
+    for (int kk = 0; kk < 2; ++kk) {
+      const int kb = 2 * half + kk;                   // 16-column block of this thread
       float f[16];
       if (kb < ti) {
 #pragma unroll
@@ -613,7 +611,7 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
       }
 #pragma unroll
       for (int e = 0; e < 16; e += 2)
-        tc::f2_get(tc::mul2(tc::f2(f[e], f[e + 1]), tc::f2(s[16 * kb + e], s[16 * kb + e + 1])),
+        tc::f2_get(tc::mul2(tc::f2(f[e], f[e + 1]), tc::f2(s[16 * kk + e], s[16 * kk + e + 1])),
                    f[e], f[e + 1]);
 #pragma unroll
       for (int e = 0; e < 16; ++e) sum += f[e];
@@ -638,21 +636,19 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 
   GDN_TRACE_PP(4);
   float tv[3][4];
-  solve_unit_lower(tb, tid, tv);
+  if (tid < 128) solve_unit_lower(tb, tid, tv);       // (warps 0-3; named barriers of 128, 64)
+  __syncthreads();                                    // T's diagonal blocks are in place
   GDN_TRACE_PP(5);
-  float4 dg[2];
-#pragma unroll
-  for (int m = 0; m < 2; ++m) {
-    const int id = tid + PP_THREADS * m, b = id >> 6, r = (id >> 2) & 15, cs = id & 3;
-    dg[m] = tc::lds4(at(blkT(tb, b, b), r, 4 * cs));
-  }
+  // one (diagonal block, row, 4-column group) per thread: 4 x 16 x 4 = 256
+  const float4 dg = tc::lds4(at(blkT(tb, tid >> 6, tid >> 6), (tid >> 2) & 15, 4 * (tid & 3)));
   __syncthreads();                                    // the solve scratch is dead
   // T_b (kt false) or ktil T_b (kt true) into the B tile pair; the zeros above the diagonal
   // blocks are written once and serve both
   auto put_b = [&](bool kt) {
     const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
-    for (int m = 0; m < 3; ++m) {                     // off-diagonal blocks and their zero mirrors
+    for (int m = 0; m < 3 && tid < 128; ++m) {        // off-diagonal blocks and their zero mirrors
+                                                      // (from the solve's fragments, warps 0-3)
       const int hp = warp + 4 * m, bi = hp >> 1, n0 = (hp & 1) * 8;
       const int i = blk_i(bi), kk = blk_k(bi, i);
       const int col = 16 * kk + n0 + 2 * t4, row = 16 * i + g;
@@ -665,13 +661,12 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         store_b_pair(tb, urow + 8, ucol, 0.f, 0.f);
       }
     }
-#pragma unroll
-    for (int m = 0; m < 2; ++m) {                     // diagonal blocks (zero above the diagonal)
-      const int id = tid + PP_THREADS * m, b = id >> 6, r = (id >> 2) & 15, cs = id & 3;
-      const int row = 16 * b + r, col = 16 * b + 4 * cs;
-      const float f = kt ? gKt[row] : 1.f;
-      store_b_pair(tb, row, col, f * (dg[m].x * gB[col]), f * (dg[m].y * gB[col + 1]));
-      store_b_pair(tb, row, col + 2, f * (dg[m].z * gB[col + 2]), f * (dg[m].w * gB[col + 3]));
+    {                                                 // diagonal blocks (zero above the diagonal)
+      const int b = tid >> 6, r = (tid >> 2) & 15, cs = tid & 3;
+      const int brow = 16 * b + r, col = 16 * b + 4 * cs;
+      const float f = kt ? gKt[brow] : 1.f;
+      store_b_pair(tb, brow, col, f * (dg.x * gB[col]), f * (dg.y * gB[col + 1]));
+      store_b_pair(tb, brow, col + 2, f * (dg.z * gB[col + 2]), f * (dg.w * gB[col + 3]));
     }
     tc::fence_proxy_async_smem();
     tc::tc_fence_before();
@@ -713,26 +708,27 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
   // the MMAs no longer read, then leave by bulk copies: PT's while W is still being multiplied
   // (hi over P hi, lo over P lo), W's once it is done (hi over the B tile pair, lo rows 0..63 /
   // 64..127 over the two K boxes).
-  auto stage_row = [&](uint32_t hi_base, uint32_t lo_base, int r, const float* w) {
+  // 32 values (this thread's column half) of row r, split and staged in the record's tile layout
+  auto stage_half = [&](uint32_t hi_base, uint32_t lo_base, int r, const float* w) {
 #pragma unroll
-    for (int j8 = 0; j8 < 8; ++j8) {
+    for (int jj = 0; jj < 4; ++jj) {
+      const int j8 = 4 * half + jj;
       const uint32_t o = (uint32_t)(r * 128 + ((j8 ^ (r & 7)) << 4));
-      st_split8(hi_base + o, lo_base + o, w + 8 * j8);
+      st_split8(hi_base + o, lo_base + o, w + 8 * jj);
     }
   };
   {
-    float w[64];
-    if (tid < 64) {
-      tc::tmem_ld32(tmem + lane_off + 64, *reinterpret_cast<float(*)[32]>(&w[0]));
-      tc::tmem_ld32(tmem + lane_off + 96, *reinterpret_cast<float(*)[32]>(&w[32]));
+    float w[32];
+    if (row < 64) {             // PT rows: warps 0, 1 (columns 0..31) and 4, 5 (32..63)
+      tc::tmem_ld32(tmem + lane_off + 64 + 32 * half, w);
       tc::tmem_wait_ld();
       if (poison) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) w[j] = kInf;
+        for (int j = 0; j < 32; ++j) w[j] = kInf;
       }
-      stage_row(qk, qk + 16384, tid, w);
+      stage_half(qk, qk + 16384, row, w);
       tc::fence_proxy_async_smem();
-      tc::named_bar(2, 64);
+      tc::named_bar(2, 128);
       if (tid == 0) {
         tc::bulk_store(rec, qk, 8192);
         tc::bulk_store(rec + 8192, qk + 16384, 8192);
@@ -741,17 +737,16 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     }
     tc::mbar_wait(mma_bar, 1, abort_flag, kBudget);
     tc::tc_fence_after();
-    tc::tmem_ld32(tmem + lane_off, *reinterpret_cast<float(*)[32]>(&w[0]));
-    tc::tmem_ld32(tmem + lane_off + 32, *reinterpret_cast<float(*)[32]>(&w[32]));
+    tc::tmem_ld32(tmem + lane_off + 32 * half, w);
     tc::tmem_wait_ld();
     if (poison) {
 #pragma unroll
-      for (int j = 0; j < 64; ++j) w[j] = kInf;
+      for (int j = 0; j < 32; ++j) w[j] = kInf;
     }
     // W row r: hi at tb + r * 128, lo at qk + 8192 (r < 64) or qk + 24576 (r >= 64)
-    stage_row(tb, qk + (tid < 64 ? 8192 : 24576 - 64 * 128), tid, w);
+    stage_half(tb, qk + (row < 64 ? 8192 : 24576 - 64 * 128), row, w);
     tc::fence_proxy_async_smem();
-    tc::named_bar(1, 128);
+    tc::named_bar(4, PP_THREADS);
     if (tid == 0) {
       tc::bulk_store(rec + 16384, tb, 16384);
       tc::bulk_store(rec + 32768, qk + 8192, 8192);
@@ -774,25 +769,17 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 // ------------------------------------------------------------------------------------------
 // the recurrence
 // ------------------------------------------------------------------------------------------
-// kNorm: the layer's gated RMSNorm is applied to o in the epilogue, y = o / sqrt(mean(o^2) + eps)
-// * w (.) SiLU(z) per (token, head), and y (in Tout) is stored instead of o.
-template <typename Tout, bool kNorm>
+template <typename Tout>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmo, const __nv_bfloat16* __restrict__ v,
                     const uint8_t* __restrict__ pw, const float* __restrict__ S0,
                     float* __restrict__ S_T, int T, int Hk, int Hv, float scale,
-                    const int* __restrict__ cu, int max_len, int nCmax, Tout* __restrict__ o,
-                    const __nv_bfloat16* __restrict__ z, const float* __restrict__ norm_w,
-                    float norm_eps) {
+                    const int* __restrict__ cu, int max_len, int nCmax, Tout* __restrict__ o) {
   constexpr bool kF32 = sizeof(Tout) == 4;
-  // X takes M as a hi + lo bf16 pair when o is fp32 or goes through the gated norm (whose
-  // per-row normalisation magnifies o's error); a bf16 o carries its own rounding, and one
-  // round-to-nearest bf16 copy of M suffices.
-  constexpr bool kSplitX = kF32 || kNorm;
-  // the o leaders also hand back W's part of the slot when the o tile spills into it or the norm
-  // exchange uses it
-  constexpr bool kOutUsesW = kF32 || kNorm;
+  // X takes M as a hi + lo bf16 pair when o is fp32 (the layer, whose gated norm magnifies o's
+  // error); a bf16 o carries its own rounding, and one round-to-nearest bf16 copy of M suffices.
+  constexpr bool kSplitX = kF32;
   GDN_TRACE_INIT;
   // Offsetting the __shared__ array itself (not a round trip through an integer) keeps every
   // access below a shared-memory access (ld/st.shared), not a generic one.
@@ -829,10 +816,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     // spills into W's part)
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(bar(B_P_EMPTY + s), 3);
-      tc::mbar_init(bar(B_W_EMPTY + s), kOutUsesW ? 3 : 1);
+      tc::mbar_init(bar(B_W_EMPTY + s), kF32 ? 3 : 1);
       tc::mbar_init(bar(B_G_FULL + s), 1);
       tc::mbar_init(bar(B_G_EMPTY + s), 8);           // one arrive per chain warp
-      tc::mbar_init(bar(B_RED + s), 2);               // one arrive per column half
     }
     *abort_flag = 0;
     tc::fence_barrier_init();
@@ -841,9 +827,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     tc::tmem_alloc(sb + OFF_MISC, 512);
     tc::tmem_relinquish();
     tc::tc_fence_before();
-  }
-  if constexpr (kNorm) {
-    if (threadIdx.x < 128) reinterpret_cast<float*>(smem + OFF_NW)[threadIdx.x] = norm_w[threadIdx.x];
   }
   if (warp == 0 && lane == 0) {
     tc::tma_prefetch_desc(&tmq);
@@ -878,11 +861,13 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         if (!ok) break;
         tc::mbar_arrive_expect_tx(bar(B_W_FULL + s), 32768);
         tc::bulk_load(slot + 16384, src + 16384, 32768, bar(B_W_FULL + s));
+        GDN_TRACE(c, 17);
         armed_w[s] = c;
         if (c >= 2) ok = tc::mbar_wait(bar(B_P_EMPTY + s), ((c >> 1) - 1) & 1, abort_flag, kBudget);
         if (!ok) break;
         tc::mbar_arrive_expect_tx(bar(B_P_FULL + s), 16384);
         tc::bulk_load(slot, src, 16384, bar(B_P_FULL + s));
+        GDN_TRACE(c, 18);
         armed_p[s] = c;
       }
       // every load issued lands before the CTA can leave (at once unless a consumer gave up)
@@ -926,8 +911,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       for (int c = 0; c < nC && ok; ++c) {
         const int s = c & 1;
         // X = [Q; K] M  (M as one bf16 copy, or a hi + lo pair)                     (bf16)
+        // X(c) goes to the TMEM buffer of X(c - 2), whose o rows the o path of chunk c - 2 reads:
+        // it signals Y_EMPTY once its TMEM reads are done
         ok = tc::mbar_wait_spin(bar(B_QK_FULL), c & 1, abort_flag, kBudget) &&
-             tc::mbar_wait_spin(bar(B_M_READY), c & 1, abort_flag, kBudget);
+             tc::mbar_wait_spin(bar(B_M_READY), c & 1, abort_flag, kBudget) &&
+             (c < 2 || tc::mbar_wait_spin(bar(B_Y_EMPTY), c & 1, abort_flag, kBudget));
         if (!ok) break;
         GDN_TRACE(c, 12);
         tc::tc_fence_after();
@@ -943,9 +931,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         GDN_TRACE(c, 20);
         if (c >= 1 && !(ok = issue_Y(c - 1))) break;
         // M += W R' (TMEM holds gamma_last M), hi.hi + lo.hi + hi.lo bf16 products     (bf16)
-        ok = tc::mbar_wait_spin(bar(B_R_FULL), c & 1, abort_flag, kBudget) &&
-             tc::mbar_wait_spin(bar(B_M_SCALED), c & 1, abort_flag, kBudget) &&
-             tc::mbar_wait_spin(bar(B_W_FULL + s), (c >> 1) & 1, abort_flag, kBudget);
+        ok = tc::mbar_wait_spin(bar(B_R_FULL), c & 1, abort_flag, kBudget);
+        GDN_TRACE(c, 14);
+        ok = ok && tc::mbar_wait_spin(bar(B_M_SCALED), c & 1, abort_flag, kBudget);
+        GDN_TRACE(c, 15);
+        ok = ok && tc::mbar_wait_spin(bar(B_W_FULL + s), (c >> 1) & 1, abort_flag, kBudget);
         if (!ok) break;
         GDN_TRACE(c, 13);
         tc::tc_fence_after();
@@ -1156,20 +1146,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       if (q < 2 && !stop) {
         // o_t = gamma_t scale (Q M)_t + (PT R')_t, staged in the chunk's operand slot (the PT
         // tiles, which Y has finished reading; fp32 also takes W's, after the update) for a TMA
-        // store.  With kNorm, y_t (the gated norm of o_t) takes o's place.
+        // store
         const bool t_valid = (long)c * C + t < sp.len;
-        [[maybe_unused]] uint4 zr[8];
-        if constexpr (kNorm) {                   // z row t of this half, before the wait
-          if (t_valid) {
-            const uint4* src = reinterpret_cast<const uint4*>(
-                z + ((sp.row0 + (long)c * C + t) * Hv + h) * 128 + tcol);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) zr[i] = src[i];
-          } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) zr[i] = make_uint4(0u, 0u, 0u, 0u);
-          }
-        }
         tc::mbar_wait(bar(B_Y_FULL), c & 1, abort_flag, kBudget);
         if (leader) GDN_TRACE(c, 34 + ev);
         tc::tc_fence_after();
@@ -1214,56 +1192,17 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
                                tc::pack_bf16(y[8 * j + 6], y[8 * j + 7]));
           }
         };
-        if constexpr (kNorm) {
-          float ov[64];
-#pragma unroll
-          for (int p = 0; p < 4; ++p) {
-            float x[16], y[16];
-            tmem_ld16(tx + 16 * p, x);
-            tmem_ld16(tmem + lane_off + TM_Y + tcol + 16 * p, y);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; i += 2)
-              tc::f2_get(tc::fma2(tc::f2(g, g), tc::f2(x[i], x[i + 1]), tc::f2(y[i], y[i + 1])),
-                         ov[16 * p + i], ov[16 * p + i + 1]);
-          }
-          float ss = 0.f;
-#pragma unroll
-          for (int i = 0; i < 64; ++i) ss = fmaf(ov[i], ov[i], ss);
-          // the row's other half is held by the same lane of the other column group
-          float* red = reinterpret_cast<float*>(smem + OFF_PW + s * PW_SLOT + RED_OFF);
-          red[hh * 64 + t] = ss;
-          tc::named_bar(id_lo, 64);
-          if (leader) tc::mbar_arrive(bar(B_RED + s));
-          tc::mbar_wait(bar(B_RED + s), (c >> 1) & 1, abort_flag, kBudget);
-          const float inv = rsqrtf((red[t] + red[64 + t]) * (1.0f / 128.0f) + norm_eps);
-          const float* nw = reinterpret_cast<const float*>(smem + OFF_NW) + tcol;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint32_t w4[4] = {zr[j].x, zr[j].y, zr[j].z, zr[j].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float za = tc::bf16lo(w4[e]), zb = tc::bf16hi(w4[e]);
-              const int i = 8 * j + 2 * e;
-              ov[i] = ov[i] * inv * nw[i] * __fdividef(za, 1.0f + __expf(-za));
-              ov[i + 1] = ov[i + 1] * inv * nw[i + 1] * __fdividef(zb, 1.0f + __expf(-zb));
-            }
-          }
-#pragma unroll
-          for (int p = 0; p < 4; ++p) put16(p, ov + 16 * p);
-        } else {
 #pragma unroll 1
-          for (int p = 0; p < 4; ++p) {            // value columns 16p .. 16p+15 of this half
-            float x[16], y[16];
-            tmem_ld16(tx + 16 * p, x);
-            tmem_ld16(tmem + lane_off + TM_Y + tcol + 16 * p, y);
-            tc::tmem_wait_ld();
+        for (int p = 0; p < 4; ++p) {            // value columns 16p .. 16p+15 of this half
+          float x[16], y[16];
+          tmem_ld16(tx + 16 * p, x);
+          tmem_ld16(tmem + lane_off + TM_Y + tcol + 16 * p, y);
+          tc::tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 16; i += 2)
-              tc::f2_get(tc::fma2(tc::f2(g, g), tc::f2(x[i], x[i + 1]), tc::f2(y[i], y[i + 1])),
-                         y[i], y[i + 1]);
-            put16(p, y);
-          }
+          for (int i = 0; i < 16; i += 2)
+            tc::f2_get(tc::fma2(tc::f2(g, g), tc::f2(x[i], x[i + 1]), tc::f2(y[i], y[i + 1])),
+                       y[i], y[i + 1]);
+          put16(p, y);
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
@@ -1283,7 +1222,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
             tc::bulk_wait_read_all();
           }
           tc::mbar_arrive(bar(B_P_EMPTY + s));
-          if constexpr (kOutUsesW) tc::mbar_arrive(bar(B_W_EMPTY + s));
+          if constexpr (kF32) tc::mbar_arrive(bar(B_W_EMPTY + s));
           GDN_TRACE(c, 36 + ev);
         }
       }
@@ -1408,32 +1347,26 @@ inline Split* split_for_device() {   // call with split_mutex() held
 // records.  The recurrence reads the pre-pass's records only after it in stream order.  `parts`:
 // kPre, kRec or both; a recurrence launched alone must follow its pre-pass on `st` by an event.
 constexpr int kPre = 1, kRec = 2;
-// Optional parts of a call: the gated norm fused into the o epilogue (z == nullptr: plain o; z has
-// o's layout, bf16), and gates taken from the in_proj_ba outputs (ba [tokens, 2 Hv] bf16) instead
-// of log_alpha / beta.  at(): the same for the part of the call starting `tokens` tokens in.
-struct NormArgs {
-  const __nv_bfloat16* z = nullptr;
-  const float* w = nullptr;
-  float eps = 0.f;
+// Gates taken from the in_proj_ba outputs (ba [tokens, 2 Hv] bf16) instead of log_alpha / beta
+// (ba == nullptr: the gates are given).  at(): the same for the part of the call starting
+// `tokens` tokens in.
+struct GateSrc {
   const __nv_bfloat16* ba = nullptr;
   int Hv = 0;
-  NormArgs at(size_t tokens) const {
-    return NormArgs{z ? z + tokens * Hv * 128 : nullptr, w, eps,
-                    ba ? ba + tokens * 2 * Hv : nullptr, Hv};
-  }
+  GateSrc at(size_t tokens) const { return GateSrc{ba ? ba + tokens * 2 * Hv : nullptr, Hv}; }
 };
 template <typename Tout>
 gdn_status launch_one(const void* q, const void* k, const void* v, const float* la,
                       const float* be, const float* S0, Tout* o, float* S_T, int nseq, int T,
                       int Hk, int Hv, float scale, uint8_t* pw, const int* cu, int max_len,
-                      const NormArgs& nrm, cudaStream_t st, cudaEvent_t ev_after_pre,
+                      const GateSrc& nrm, cudaStream_t st, cudaEvent_t ev_after_pre,
                       int parts = kPre | kRec) {
   const int mapB = cu ? 1 : nseq;
   CUtensorMap mq, mk, mo;
   if (!make_tile_map(&mq, q, Hk, T, mapB, false) || !make_tile_map(&mk, k, Hk, T, mapB, false) ||
       !make_tile_map(&mo, o, Hv, T, mapB, sizeof(Tout) == 4))
     return GDN_ERR_CUDA;
-  auto kern = nrm.z ? chunk_fwd_tc_kernel<Tout, true> : chunk_fwd_tc_kernel<Tout, false>;
+  auto kern = chunk_fwd_tc_kernel<Tout>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC) !=
       cudaSuccess)
     return GDN_ERR_CUDA;
@@ -1454,7 +1387,7 @@ gdn_status launch_one(const void* q, const void* k, const void* v, const float* 
   if (parts & kRec) {
     kern<<<(unsigned)grid, kThreads, SMEM_ALLOC, st>>>(
         mq, mk, mo, static_cast<const __nv_bfloat16*>(v), pw, S0, S_T, T, Hk, Hv, scale, cu,
-        max_len, nCmax, o, nrm.z, nrm.w, nrm.eps);
+        max_len, nCmax, o);
     if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
   }
   return GDN_OK;
@@ -1470,7 +1403,7 @@ template <typename Tout>
 gdn_status launch(const void* q, const void* k, const void* v, const float* la, const float* be,
                   const float* S0, Tout* o, float* S_T, int nseq, int T, int Hk, int Hv,
                   float scale, uint8_t* pw, const int* cu, int max_len, cudaStream_t st,
-                  const NormArgs& nrm = NormArgs{}) {
+                  const GateSrc& nrm = GateSrc{}) {
   if ((max_len + C - 1) / C > 65535) return GDN_ERR_UNSUPPORTED;   // chunks index a grid's y
   std::unique_lock<std::mutex> lock(split_mutex());
   Split* sp = split_for_device();
@@ -1498,7 +1431,7 @@ gdn_status launch(const void* q, const void* k, const void* v, const float* la, 
       const float* S0r = r == 0 ? S0 : mid[(r - 1) & 1];
       float* STr = r == nR - 1 ? S_T : mid[r & 1];
       uint8_t* pwr = pw + (size_t)Hv * r * kRangeChunks * kPwBytes;
-      const NormArgs nr = nrm.at((size_t)t0);
+      const GateSrc nr = nrm.at((size_t)t0);
       const float* lar = la ? la + t0 * Hv : nullptr;
       const float* ber = be ? be + t0 * Hv : nullptr;
       s = launch_one<Tout>(bq, bk, bv, lar, ber, S0r, o + t0 * Hv * 128, STr, 1,
@@ -1596,31 +1529,12 @@ inline gdn_status tc_chunk_launch(const void* q, const void* k, const void* v, c
                                   int T, int Hk, int Hv, float scale, bool f32out, void* scratch,
                                   cudaStream_t st, const void* ba = nullptr) {
   uint8_t* pw = static_cast<uint8_t*>(scratch);
-  tcf::NormArgs ex;
-  ex.ba = static_cast<const __nv_bfloat16*>(ba);
-  ex.Hv = Hv;
+  const tcf::GateSrc ex{static_cast<const __nv_bfloat16*>(ba), Hv};
   if (f32out)
     return tcf::launch<float>(q, k, v, la, be, S0, static_cast<float*>(o), S_T, B, T, Hk, Hv,
                               scale, pw, nullptr, T, st, ex);
   return tcf::launch<__nv_bfloat16>(q, k, v, la, be, S0, static_cast<__nv_bfloat16*>(o), S_T, B,
                                     T, Hk, Hv, scale, pw, nullptr, T, st, ex);
-}
-
-// The recurrence with the layer's gated norm in its epilogue: y = o / sqrt(mean(o^2) + eps) * w
-// (.) SiLU(z) per (token, head) instead of o; z [B, T, Hv, 128] bf16, w [128] fp32; y in bf16, or
-// fp32 when f32y.
-inline gdn_status tc_layer_launch(const void* q, const void* k, const void* v, const float* la,
-                                  const float* be, const float* S0, void* y, float* S_T, int B,
-                                  int T, int Hk, int Hv, float scale, const void* z,
-                                  const float* norm_w, float norm_eps, bool f32y, void* scratch,
-                                  cudaStream_t st) {
-  uint8_t* pw = static_cast<uint8_t*>(scratch);
-  const tcf::NormArgs nrm{static_cast<const __nv_bfloat16*>(z), norm_w, norm_eps, nullptr, Hv};
-  if (f32y)
-    return tcf::launch<float>(q, k, v, la, be, S0, static_cast<float*>(y), S_T, B, T, Hk, Hv,
-                              scale, pw, nullptr, T, st, nrm);
-  return tcf::launch<__nv_bfloat16>(q, k, v, la, be, S0, static_cast<__nv_bfloat16*>(y), S_T, B,
-                                    T, Hk, Hv, scale, pw, nullptr, T, st, nrm);
 }
 
 // Packed sequences: q, k [total, Hk, 128], v, o [total, Hv, 128], gates [total, Hv]; sequence s is

@@ -274,6 +274,9 @@ GDN_API gdn_status gdn_gates(const void *ba, float *log_alpha, float *beta, long
  *   wq, wk [Hk*dk, 4]; wv [Hv*dv, 4] float: tap 3 multiplies the current token, tap 0 the token
  *        three steps back; positions before t = 0 are zeros (no carried conv state).
  *   q, k [B, T, Hk, dk]; v [B, T, Hv, dv]                    (dtype, outputs)
+ * bf16 outputs are the exact results rounded to the nearest bf16 (ties to even): a value whose
+ * rounding the fp32 computation cannot decide within its error bound is recomputed in fp64, so
+ * the rounding never depends on fp32 roundoff.
  */
 GDN_API gdn_status gdn_prologue(const void *q_raw, const void *k_raw, const void *v_raw,
                         const float *wq, const float *wk, const float *wv,
