@@ -64,20 +64,17 @@ __device__ __forceinline__ uint32_t bf16_pair_rn(double a, double b) {
          ((uint32_t)__bfloat16_as_ushort(__double2bfloat16(b)) << 16);
 }
 
-// bf16 round-to-nearest-even of an fp32 value, as the bit pattern (NaN and inf are not expected
-// here: the caller checks finiteness).
-__device__ __forceinline__ uint32_t bf16_bits_rn(float x) {
-  const uint32_t u = __float_as_uint(x);
-  return (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;
-}
-// Whether y and every value within e of it round to the same bf16 value.
+// Whether every value within e of y rounds to the same bf16 value as y: the rounding boundary of
+// y's bf16 cell (the midpoint, low 16 bits 0x8000) is farther than e, and e is below a quarter of
+// the cell (so no neighbouring cell's boundary is within reach either).  NaN is never decided.
 __device__ __forceinline__ bool bf16_decided(float y, float e) {
-  return fabsf(y) < 3.0e38f && bf16_bits_rn(y - e) == bf16_bits_rn(y + e);
+  const float mid = __uint_as_float((__float_as_uint(y) & 0xFFFF0000u) | 0x8000u);
+  return fabsf(y - mid) > e && e < fabsf(y) * 0.0009765625f;
 }
 
-// Fast approximations of 2^x, 1/x and 1/sqrt(x) (the SFU instructions).  The rounding decision
-// below budgets 8 units of fp32 roundoff (2^-21 relative) for each of them, more than the
-// maximum relative errors the PTX ISA documents for ex2.approx and rcp.approx.
+// Fast approximations of 2^x and 1/x (the SFU instructions).  The rounding decision below budgets
+// 8 units of fp32 roundoff (2^-21 relative) for each of them, more than the maximum relative
+// errors the PTX ISA documents for ex2.approx and rcp.approx.
 __device__ __forceinline__ float ex2_fast(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -89,63 +86,17 @@ __device__ __forceinline__ float rcp_fast(float x) {
   return y;
 }
 
-constexpr int kPrologueList = 1024;     // undecided v values one CTA redoes in fp64 afterwards
+constexpr int kPrologueList = 1024;     // undecided values one CTA redoes in fp64 afterwards
 
-// grid: (2*Hk + Hv, ceil(T / kPrologueTokens), B), head slots fastest, so that CTAs that run
-// together read neighbouring parts of the same token rows; block: 128 threads.  One CTA takes one
-// head (d channels) of kPrologueTokens tokens: the raw rows of those tokens and of the three
-// before them (zeros before t = 0) come into shared memory by 16-byte asynchronous copies, all
-// issued at once, then every token is convolved from shared memory.  A head row of d channels is
-// held by L = d / N threads (N channels of one 16-byte vector each); the 128 / L row groups of the
-// CTA take every (128 / L)-th token.  The L2 norm of a q or k row is a shuffle reduction over its
-// L threads (one warp).
-//
-// bf16 outputs: rounding to bf16 is a quantising decision, taken here as the exact result would
-// take it, i.e. as rounding the fp64 value does.  Each fp32 value y carries a bound E on its
-// distance from the exact value; values for which y - 2E and y + 2E round differently are redone
-// in fp64 after the tile is stored, from a list in shared memory (so the rare fp64 work does not
-// diverge the common path):
-//   v: the convolution's 4-term fp32 sum (at most about 4 units of roundoff of sum |w x|, carried
-//      through SiLU' <= 1.1), the rounding of the exponent's argument (|x| units, relative), the
-//      budgets of ex2.approx and rcp.approx and one unit per remaining operation;
-//   q, k: the convolution in fp64 (exact to fp32 precision), SiLU with expf (<= 2 ulp) and IEEE
-//      division, the row's sum of squares and norm in fp64; a row any of whose values is
-//      undecided is redone whole (they share the norm).
+// The staged tile of one prologue CTA: the raw rows of tokens t0 - 3 .. t0 + kPrologueTokens - 1
+// (zeros outside 0 .. T - 1) of one head of d channels, row r holding token t0 - 3 + r, brought in
+// by 16-byte asynchronous copies that are all issued at once (many tiles in flight per SM).
 template <typename Tio>
-__global__ void __launch_bounds__(128, 5)   // five tiles in flight per SM
-prologue_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
-                const Tio* __restrict__ xv, const float* __restrict__ wq,
-                const float* __restrict__ wk, const float* __restrict__ wv,
-                Tio* __restrict__ yq, Tio* __restrict__ yk, Tio* __restrict__ yv, int T, int Hk,
-                int Hv, int dk, int dv, float eps) {
+__device__ __forceinline__ void prologue_stage(Tio* tile, const Tio* xh, long t0, int T, int width,
+                                               int d) {
   constexpr int N = Vec16<Tio>::N;
-  constexpr bool kBf16 = sizeof(Tio) == 2;
-  constexpr float u = 5.9604645e-8f;          // 2^-24, the unit roundoff of fp32
-  constexpr int R = kPrologueTokens + 3;      // staged rows: 3 history tokens, then the tile
-  extern __shared__ __align__(16) uint8_t pro_smem[];
-  Tio* tile = reinterpret_cast<Tio*>(pro_smem);
-  __shared__ uint16_t list[kPrologueList];    // undecided (token << 8 | channel), or q/k rows
-  __shared__ int nlist;
-  const int slot = blockIdx.x;
-  const long b = blockIdx.z;
-  const Tio* x;
-  const float* w;
-  Tio* y;
-  int d, head, width;
-  bool l2;
-  if (slot < Hk) {
-    x = xq; w = wq; y = yq; d = dk; head = slot; width = Hk * dk; l2 = true;
-  } else if (slot < 2 * Hk) {
-    x = xk; w = wk; y = yk; d = dk; head = slot - Hk; width = Hk * dk; l2 = true;
-  } else {
-    x = xv; w = wv; y = yv; d = dv; head = slot - 2 * Hk; width = Hv * dv; l2 = false;
-  }
-  const int L = d / N;                        // 2 .. 32, a power of two
-  const long t0 = (long)blockIdx.y * kPrologueTokens;
-  const Tio* xh = x + b * T * (long)width + (long)head * d;
-  if (threadIdx.x == 0) nlist = 0;
-  // stage rows t0 - 3 .. t0 + kPrologueTokens - 1 (row r holds token t0 - 3 + r)
-  for (int i = threadIdx.x; i < R * L; i += 128) {
+  const int L = d / N;
+  for (int i = threadIdx.x; i < (kPrologueTokens + 3) * L; i += blockDim.x) {
     const int r = i / L, c = i - r * L;
     const long t = t0 - 3 + r;
     const bool in = t >= 0 && t < T;
@@ -155,7 +106,39 @@ prologue_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
                  "r"(in ? 16 : 0) : "memory");
   }
   asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
-  const int grp = threadIdx.x / L, lc = threadIdx.x % L, ngrp = 128 / L;
+}
+
+// Prologue of the v channels (no normalisation): grid (Hv, ceil(T / kPrologueTokens), B), head
+// slots fastest, so that CTAs that run together read neighbouring parts of the same token rows;
+// block: 128 threads.  One CTA takes one head of dv channels over kPrologueTokens tokens: a head
+// row is held by L = dv / N threads (N channels of one 16-byte vector each) and the 128 / L row
+// groups take consecutive spans of tokens, carrying the conv window in registers.
+//
+// bf16 outputs: rounding to bf16 is a quantising decision, taken here as the exact result would
+// take it, i.e. as rounding the fp64 value does.  Each fp32 value y carries a bound E on its
+// distance from the exact value: the convolution's 4-term fp32 sum (at most about 4 units of
+// roundoff of sum |w x|, carried through SiLU' <= 1.1), the rounding of the exponent's argument
+// (|x| units, relative), the budgets of ex2.approx and rcp.approx and one unit per remaining
+// operation.  Values with a rounding boundary within 2E are redone in fp64 after the tile is
+// stored, from a list in shared memory (so the rare fp64 work does not diverge the common path).
+template <typename Tio>
+__global__ void __launch_bounds__(128, 6)
+prologue_v_kernel(const Tio* __restrict__ x, const float* __restrict__ w, Tio* __restrict__ y,
+                  int T, int Hv, int dv) {
+  constexpr int N = Vec16<Tio>::N;
+  constexpr bool kBf16 = sizeof(Tio) == 2;
+  constexpr float u = 5.9604645e-8f;          // 2^-24, the unit roundoff of fp32
+  extern __shared__ __align__(16) uint8_t pro_smem[];
+  Tio* tile = reinterpret_cast<Tio*>(pro_smem);
+  __shared__ uint16_t list[kPrologueList];    // undecided (token << 8 | channel)
+  __shared__ int nlist;
+  const int head = blockIdx.x, d = dv, width = Hv * dv;
+  const long b = blockIdx.z;
+  const long t0 = (long)blockIdx.y * kPrologueTokens;
+  const int L = d / N, grp = threadIdx.x / L, lc = threadIdx.x % L, ngrp = 128 / L;
+  const int tpg = kPrologueTokens / ngrp, i0 = grp * tpg;  // this row group's tokens
+  if (threadIdx.x == 0) nlist = 0;
+  prologue_stage(tile, x + b * T * (long)width + (long)head * d, t0, T, width, d);
   const long c0 = (long)head * d + lc * N;    // first channel of this thread
   float wt[N][4];
 #pragma unroll
@@ -166,130 +149,206 @@ prologue_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
   const long rem = T - t0;
   const int nt = rem < kPrologueTokens ? (int)rem : kPrologueTokens;
   Tio* const yt = y + (b * T + t0) * width + c0;          // this thread's channels of token t0
-  for (int i = grp; i < kPrologueTokens; i += ngrp) {   // same trip count within a warp
-    float h[4][N];
+  float h0[N], h1[N], h2[N];                  // the window: rows i, i + 1, i + 2 of token i
+  Vec16<Tio>::load(tile + (long)i0 * d + lc * N, h0);
+  Vec16<Tio>::load(tile + (long)(i0 + 1) * d + lc * N, h1);
+  Vec16<Tio>::load(tile + (long)(i0 + 2) * d + lc * N, h2);
+#pragma unroll 4
+  for (int tt = 0; tt < tpg; ++tt) {
+    const int i = i0 + tt;
+    float h3[N], yv_[N];
+    Vec16<Tio>::load(tile + (long)(i + 3) * d + lc * N, h3);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) Vec16<Tio>::load(tile + (long)(i + j) * d + lc * N, h[j]);
-    float yv_[N];
-    if (!kBf16 || !l2) {
-      bool need = false;
-#pragma unroll
-      for (int j = 0; j < N; ++j) {
-        const float pre = fmaf(wt[j][3], h[3][j],
-                               fmaf(wt[j][2], h[2][j], fmaf(wt[j][1], h[1][j], wt[j][0] * h[0][j])));
-        // SiLU(pre) = pre / (1 + 2^(-pre log2 e))
-        const float s = pre * rcp_fast(1.0f + ex2_fast(pre * -1.4426950408889634f));
-        yv_[j] = s;
-        if constexpr (kBf16) {
-          const float A = fmaf(fabsf(wt[j][3]), fabsf(h[3][j]),
-                               fmaf(fabsf(wt[j][2]), fabsf(h[2][j]),
-                                    fmaf(fabsf(wt[j][1]), fabsf(h[1][j]),
-                                         fabsf(wt[j][0]) * fabsf(h[0][j]))));
-          const float e = 2.0f * u * fmaf(21.0f + fabsf(pre), fabsf(s), 6.0f * A);
-          if (!bf16_decided(s, e)) {
-            need = true;
-            const int k = atomicAdd(&nlist, 1);
-            if (k < kPrologueList) list[k] = (uint16_t)((i << 8) | (lc * N + j));
-          }
+    for (int j = 0; j < N; ++j) {
+      const float pre = fmaf(wt[j][3], h3[j], fmaf(wt[j][2], h2[j],
+                                                   fmaf(wt[j][1], h1[j], wt[j][0] * h0[j])));
+      // SiLU(pre) = pre / (1 + 2^(-pre log2 e))
+      const float s = pre * rcp_fast(1.0f + ex2_fast(pre * -1.4426950408889634f));
+      yv_[j] = s;
+      if constexpr (kBf16) {
+        const float A = fmaf(fabsf(wt[j][3]), fabsf(h3[j]),
+                             fmaf(fabsf(wt[j][2]), fabsf(h2[j]),
+                                  fmaf(fabsf(wt[j][1]), fabsf(h1[j]), fabsf(wt[j][0]) * fabsf(h0[j]))));
+        const float e = 2.0f * u * fmaf(21.0f + fabsf(pre), fabsf(s), 6.0f * A);
+        if (!bf16_decided(s, e)) {
+          const int k = atomicAdd(&nlist, 1);
+          if (k < kPrologueList) list[k] = (uint16_t)((i << 8) | (lc * N + j));
         }
       }
-      if (l2) {   // fp32 outputs: the row's norm in fp32
-        float ss = 0.f;
-#pragma unroll
-        for (int j = 0; j < N; ++j) ss = fmaf(yv_[j], yv_[j], ss);
-        for (int o = L >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        const float inv = rsqrtf(ss + eps);
-#pragma unroll
-        for (int j = 0; j < N; ++j) yv_[j] *= inv;
-      }
-      (void)need;
-    } else {
-      // q, k rows in bf16: convolution in fp64, SiLU in fp32 (expf, IEEE division), norm in fp64
-      float s[N], es[N];
-      double ssd = 0.0;
-#pragma unroll
-      for (int j = 0; j < N; ++j) {
-        double acc = 0.0;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) acc = fma((double)wt[j][k], (double)h[k][j], acc);
-        const float pre = (float)acc;         // within half a unit of the exact sum
-        s[j] = pre / (1.0f + expf(-pre));
-        es[j] = u * fmaf(fabsf(pre), 0.6f, 7.0f * fabsf(s[j]));   // expf, +, /, rounded pre
-        ssd = fma((double)s[j], (double)s[j], ssd);
-      }
-      float se = 0.f;                         // sum of 2 |s| es: the sum of squares' error
-#pragma unroll
-      for (int j = 0; j < N; ++j) se = fmaf(2.0f * fabsf(s[j]), es[j], se);
-      for (int o = L >> 1; o > 0; o >>= 1) {
-        ssd += __shfl_xor_sync(0xffffffffu, ssd, o);
-        se += __shfl_xor_sync(0xffffffffu, se, o);
-      }
-      const double invd = 1.0 / sqrt(ssd + (double)eps);
-      const float inv = (float)invd;
-      const float dinv = 0.5f * se * (float)(1.0 / (ssd + (double)eps)) * 1.01f + u;
-      bool need = false;
-#pragma unroll
-      for (int j = 0; j < N; ++j) {
-        yv_[j] = (float)((double)s[j] * invd);
-        const float e = 2.0f * (fabsf(yv_[j]) * (dinv + 2.0f * u) + es[j] * inv);
-        need = need || !bf16_decided(yv_[j], e);
-      }
-      for (int o = L >> 1; o > 0; o >>= 1) need |= __shfl_xor_sync(0xffffffffu, need, o) != 0;
-      if (need && lc == 0) {                  // the row, redone in fp64 below
-        const int k = atomicAdd(&nlist, 1);
-        if (k < kPrologueList) list[k] = (uint16_t)i;
-      }
+      h0[j] = h1[j]; h1[j] = h2[j]; h2[j] = h3[j];
     }
     if (i < nt) Vec16<Tio>::store(yt + (long)i * width, yv_);
   }
   if constexpr (kBf16) {
     __syncthreads();                          // the list is complete, the fast values stored
-    const int n = min(nlist, kPrologueList);
+    const int n = nlist;
     __nv_bfloat16* yb = reinterpret_cast<__nv_bfloat16*>(y) + (b * T + t0) * width + (long)head * d;
     const __nv_bfloat16* tb16 = reinterpret_cast<const __nv_bfloat16*>(tile);
     const float* wh = w + (long)head * d * 4;
-    if (!l2) {
+    if (n <= kPrologueList) {
       for (int e = threadIdx.x; e < n; e += 128) {
         const int i = list[e] >> 8, ch = list[e] & 255;
         if (i < nt)
           yb[(long)i * width + ch] = __double2bfloat16(
               silu_conv_fp64(tb16 + (long)i * d + ch, d, wh + ch * 4));
       }
-    } else {
-      // one row per group of L threads (the row's norm by shuffles over those lanes)
-      const unsigned rowmask = L == 32 ? 0xffffffffu
-                                       : (((1u << L) - 1u) << ((threadIdx.x & 31) & ~(L - 1)));
-      for (int e0 = 0; e0 < n; e0 += ngrp) {  // uniform trip count
-        const int e = e0 + grp;
-        if (e >= n) continue;                 // whole row groups skip together
-        const int i = list[e];
-        double yd[N], ss = 0.0;
-#pragma unroll
-        for (int j = 0; j < N; ++j) {
-          const int ch = lc * N + j;
-          yd[j] = silu_conv_fp64(tb16 + (long)i * d + ch, d, wh + ch * 4);
-          ss += yd[j] * yd[j];
-        }
-        for (int o = L >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(rowmask, ss, o);
-        const double invd = 1.0 / sqrt(ss + (double)eps);
-        if (i < nt) {
-          uint32_t pk[N / 2];
-#pragma unroll
-          for (int j = 0; j < N / 2; ++j) pk[j] = bf16_pair_rn(yd[2 * j] * invd, yd[2 * j + 1] * invd);
-          *reinterpret_cast<uint4*>(yb + (long)i * width + lc * N) =
-              make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        }
+    } else {                                  // an overfull list (not expected): redo the tile
+      for (int e = threadIdx.x; e < nt * d; e += 128) {
+        const int i = e / d, ch = e - i * d;
+        yb[(long)i * width + ch] = __double2bfloat16(
+            silu_conv_fp64(tb16 + (long)i * d + ch, d, wh + ch * 4));
       }
     }
-    if (nlist > kPrologueList) {              // an overfull list (not expected): redo in place
-      for (int i = grp; i < kPrologueTokens && !l2; i += ngrp) {
-        if (i >= nt) continue;
-#pragma unroll 1
-        for (int j = 0; j < N; ++j) {
-          const int ch = lc * N + j;
-          yb[(long)i * width + ch] = __double2bfloat16(
-              silu_conv_fp64(tb16 + (long)i * d + ch, d, wh + ch * 4));
-        }
+  }
+}
+
+// Prologue of the q and k channels (conv, SiLU, then each head row divided by its L2 norm): grid
+// (2 Hk, ceil(T / kPrologueTokens), B), q heads then k heads; the thread layout of the v kernel.
+// bf16 outputs: the convolution in fp64 (the weights widened once per thread, each input once, in
+// the window), SiLU in fp32 (expf, IEEE division: within 6 units of roundoff, plus the rounded
+// argument's 0.55 |x|), the row's sum of squares in fp32 with its roundoff bound, so that a value's
+// error is a few tens of units of roundoff at most; a row with any value whose bf16 rounding that
+// leaves open is redone whole in fp64 afterwards (the row's values share the norm).
+template <typename Tio>
+__global__ void __launch_bounds__(128, 3)
+prologue_qk_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
+                   const float* __restrict__ wq, const float* __restrict__ wk,
+                   Tio* __restrict__ yq, Tio* __restrict__ yk, int T, int Hk, int dk, float eps) {
+  constexpr int N = Vec16<Tio>::N;
+  constexpr bool kBf16 = sizeof(Tio) == 2;
+  constexpr float u = 5.9604645e-8f;
+  extern __shared__ __align__(16) uint8_t pro_smem[];
+  Tio* tile = reinterpret_cast<Tio*>(pro_smem);
+  __shared__ uint16_t list[kPrologueTokens];  // undecided rows (tokens)
+  __shared__ int nlist;
+  const bool isq = blockIdx.x < Hk;
+  const int head = isq ? blockIdx.x : blockIdx.x - Hk, d = dk, width = Hk * dk;
+  const Tio* x = isq ? xq : xk;
+  const float* w = isq ? wq : wk;
+  Tio* y = isq ? yq : yk;
+  const long b = blockIdx.z;
+  const long t0 = (long)blockIdx.y * kPrologueTokens;
+  const int L = d / N, grp = threadIdx.x / L, lc = threadIdx.x % L, ngrp = 128 / L;
+  const int tpg = kPrologueTokens / ngrp, i0 = grp * tpg;
+  if (threadIdx.x == 0) nlist = 0;
+  prologue_stage(tile, x + b * T * (long)width + (long)head * d, t0, T, width, d);
+  const long c0 = (long)head * d + lc * N;
+  float wt[N][4];
+#pragma unroll
+  for (int i = 0; i < N; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) wt[i][j] = w[(c0 + i) * 4 + j];
+  __syncthreads();
+  const long rem = T - t0;
+  const int nt = rem < kPrologueTokens ? (int)rem : kPrologueTokens;
+  Tio* const yt = y + (b * T + t0) * width + c0;
+  if constexpr (!kBf16) {                     // fp32 outputs: fp32 throughout
+    float h0[N], h1[N], h2[N];
+    Vec16<Tio>::load(tile + (long)i0 * d + lc * N, h0);
+    Vec16<Tio>::load(tile + (long)(i0 + 1) * d + lc * N, h1);
+    Vec16<Tio>::load(tile + (long)(i0 + 2) * d + lc * N, h2);
+#pragma unroll 2
+    for (int tt = 0; tt < tpg; ++tt) {
+      const int i = i0 + tt;
+      float h3[N], yv_[N], ss = 0.f;
+      Vec16<Tio>::load(tile + (long)(i + 3) * d + lc * N, h3);
+#pragma unroll
+      for (int j = 0; j < N; ++j) {
+        const float pre = fmaf(wt[j][3], h3[j], fmaf(wt[j][2], h2[j],
+                                                     fmaf(wt[j][1], h1[j], wt[j][0] * h0[j])));
+        yv_[j] = pre * rcp_fast(1.0f + ex2_fast(pre * -1.4426950408889634f));
+        ss = fmaf(yv_[j], yv_[j], ss);
+        h0[j] = h1[j]; h1[j] = h2[j]; h2[j] = h3[j];
+      }
+      for (int o = L >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float inv = rsqrtf(ss + eps);
+#pragma unroll
+      for (int j = 0; j < N; ++j) yv_[j] *= inv;
+      if (i < nt) Vec16<Tio>::store(yt + (long)i * width, yv_);
+    }
+  } else {
+    double wd[N][4];                          // the weights, widened once
+#pragma unroll
+    for (int j = 0; j < N; ++j)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) wd[j][k] = wt[j][k];
+    double d0[N], d1[N], d2[N];               // the window, widened once per input
+    {
+      float f[N];
+      Vec16<Tio>::load(tile + (long)i0 * d + lc * N, f);
+#pragma unroll
+      for (int j = 0; j < N; ++j) d0[j] = f[j];
+      Vec16<Tio>::load(tile + (long)(i0 + 1) * d + lc * N, f);
+#pragma unroll
+      for (int j = 0; j < N; ++j) d1[j] = f[j];
+      Vec16<Tio>::load(tile + (long)(i0 + 2) * d + lc * N, f);
+#pragma unroll
+      for (int j = 0; j < N; ++j) d2[j] = f[j];
+    }
+    for (int tt = 0; tt < tpg; ++tt) {
+      const int i = i0 + tt;
+      float f[N], s[N], es[N], yv_[N];
+      Vec16<Tio>::load(tile + (long)(i + 3) * d + lc * N, f);
+      float ss = 0.f, se = 0.f;
+#pragma unroll
+      for (int j = 0; j < N; ++j) {
+        const double d3 = f[j];
+        const double acc = fma(wd[j][3], d3, fma(wd[j][2], d2[j], fma(wd[j][1], d1[j],
+                                                                      wd[j][0] * d0[j])));
+        const float pre = (float)acc;         // within half a unit of the exact sum
+        s[j] = pre / (1.0f + expf(-pre));
+        es[j] = u * fmaf(fabsf(pre), 0.6f, 7.0f * fabsf(s[j]));   // expf, +, /, rounded pre
+        ss = fmaf(s[j], s[j], ss);
+        se = fmaf(2.0f * fabsf(s[j]), es[j], se);
+        d0[j] = d1[j]; d1[j] = d2[j]; d2[j] = d3;
+      }
+      for (int o = L >> 1; o > 0; o >>= 1) {
+        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        se += __shfl_xor_sync(0xffffffffu, se, o);
+      }
+      // sum of squares: at most (N + log2 L + 1) units of its own roundoff plus se from the
+      // values; 1/sqrt in fp32: sqrtf and the division, one unit each
+      const float den = ss + eps;
+      const float inv = 1.0f / sqrtf(den);
+      const float dinv = 0.5f * (se + (float)(N + 8) * u * ss) / den * 1.01f + 3.0f * u;
+      bool need = false;
+#pragma unroll
+      for (int j = 0; j < N; ++j) {
+        yv_[j] = s[j] * inv;                  // fp32 product: one more unit
+        const float e = 2.0f * (fabsf(yv_[j]) * (dinv + u) + es[j] * inv);
+        need = need || !bf16_decided(yv_[j], e);
+      }
+      for (int o = L >> 1; o > 0; o >>= 1) need |= __shfl_xor_sync(0xffffffffu, need, o) != 0;
+      if (need && lc == 0) list[atomicAdd(&nlist, 1)] = (uint16_t)i;   // at most one per token
+      if (i < nt) Vec16<Tio>::store(yt + (long)i * width, yv_);
+    }
+    __syncthreads();                          // the list is complete, the fast values stored
+    const int n = nlist;
+    __nv_bfloat16* yb = reinterpret_cast<__nv_bfloat16*>(y) + (b * T + t0) * width + (long)head * d;
+    const __nv_bfloat16* tb16 = reinterpret_cast<const __nv_bfloat16*>(tile);
+    const float* wh = w + (long)head * d * 4;
+    // one row per group of L threads (the row's norm by shuffles over those lanes)
+    const unsigned rowmask = L == 32 ? 0xffffffffu
+                                     : (((1u << L) - 1u) << ((threadIdx.x & 31) & ~(L - 1)));
+    for (int e0 = 0; e0 < n; e0 += ngrp) {    // uniform trip count
+      const int e = e0 + grp;
+      if (e >= n) continue;                   // whole row groups skip together
+      const int i = list[e];
+      double yd[N], ss = 0.0;
+#pragma unroll
+      for (int j = 0; j < N; ++j) {
+        const int ch = lc * N + j;
+        yd[j] = silu_conv_fp64(tb16 + (long)i * d + ch, d, wh + ch * 4);
+        ss += yd[j] * yd[j];
+      }
+      for (int o = L >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(rowmask, ss, o);
+      const double invd = 1.0 / sqrt(ss + (double)eps);
+      if (i < nt) {
+        uint32_t pk[N / 2];
+#pragma unroll
+        for (int j = 0; j < N / 2; ++j) pk[j] = bf16_pair_rn(yd[2 * j] * invd, yd[2 * j + 1] * invd);
+        *reinterpret_cast<uint4*>(yb + (long)i * width + lc * N) =
+            make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
     }
   }

@@ -494,17 +494,21 @@ gdn_status gdn_prologue(const void* q_raw, const void* k_raw, const void* v_raw,
     return GDN_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if ((T + kPrologueTokens - 1) / kPrologueTokens > 65535) return GDN_ERR_UNSUPPORTED;
-  dim3 grid(2 * Hk + Hv, (T + kPrologueTokens - 1) / kPrologueTokens, B);
-  const int dmax = dk > dv ? dk : dv;
-  if (dtype == GDN_F32)
-    prologue_kernel<float><<<grid, 128, prologue_smem_bytes(dmax, 4), st>>>(
-        (const float*)q_raw, (const float*)k_raw, (const float*)v_raw, wq, wk, wv, (float*)q,
-        (float*)k, (float*)v, T, Hk, Hv, dk, dv, l2_eps);
-  else
-    prologue_kernel<__nv_bfloat16><<<grid, 128, prologue_smem_bytes(dmax, 2), st>>>(
-        (const __nv_bfloat16*)q_raw, (const __nv_bfloat16*)k_raw, (const __nv_bfloat16*)v_raw,
-        wq, wk, wv, (__nv_bfloat16*)q, (__nv_bfloat16*)k, (__nv_bfloat16*)v, T, Hk, Hv, dk, dv,
-        l2_eps);
+  // q and k heads (normalised rows), then the v heads; head slots fastest in each grid
+  const unsigned tb = (unsigned)((T + kPrologueTokens - 1) / kPrologueTokens);
+  const dim3 gqk(2 * Hk, tb, B), gv(Hv, tb, B);
+  if (dtype == GDN_F32) {
+    prologue_qk_kernel<float><<<gqk, 128, prologue_smem_bytes(dk, 4), st>>>(
+        (const float*)q_raw, (const float*)k_raw, wq, wk, (float*)q, (float*)k, T, Hk, dk, l2_eps);
+    prologue_v_kernel<float><<<gv, 128, prologue_smem_bytes(dv, 4), st>>>(
+        (const float*)v_raw, wv, (float*)v, T, Hv, dv);
+  } else {
+    using bf = __nv_bfloat16;
+    prologue_qk_kernel<bf><<<gqk, 128, prologue_smem_bytes(dk, 2), st>>>(
+        (const bf*)q_raw, (const bf*)k_raw, wq, wk, (bf*)q, (bf*)k, T, Hk, dk, l2_eps);
+    prologue_v_kernel<bf><<<gv, 128, prologue_smem_bytes(dv, 2), st>>>(
+        (const bf*)v_raw, wv, (bf*)v, T, Hv, dv);
+  }
   return launch_status();
 }
 

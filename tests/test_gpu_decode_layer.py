@@ -7,7 +7,7 @@ import torch
 import gdn_inputs as gi
 import gated_deltanet_linear_18_b200 as gdn
 from gpu_util import (TOL_BF16_OUT, TOL_BF16_STATE, TOL_F32_ABS, max_abs, np64, out_err,
-                      rel_rms, to_dev)
+                      rel_rms, report, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -82,12 +82,16 @@ def test_decode_layer_fresh_request_equals_layer_forward(orc):
     assert max_abs(S, S_ref) <= TOL_F32_ABS
 
 
-def test_decode_layer_full_size_sampled(orc):
-    """The decode-layer workload's sizes (256 sequences, Hk16 Hv48 d128, bf16), two steps, the
-    oracle on a sample of sequences (the sequences are independent)."""
-    w, x = _inputs("bf16", N=256, Hk=16, Hv=48, steps=2, seed=5)
+def test_decode_layer_full_size_all_sequences(orc):
+    """The decode-layer workload's sizes (256 sequences, Hk16 Hv48 d128, bf16), three steps, every
+    sequence against the oracle: y beyond its bf16 rounding (y's max/rms of about 49 puts the plain
+    bound out of reach of any bf16-stored y, the rounding alone reaching 9.6 % of the RMS; the
+    kernel keeps q, k, v in fp32, so the oracle runs with fp64 activations), the state plain."""
+    w, x = _inputs("bf16", N=256, Hk=16, Hv=48, steps=3, seed=5)
     y, S, _ = _run_gpu(w, x)
-    seqs = [0, 77, 255]
-    y_ref, S_ref, _, _, _ = _run_oracle(orc, w, x, seqs=seqs)
-    assert out_err(y[:, seqs], y_ref) <= TOL_BF16_OUT
-    assert rel_rms(S[seqs], S_ref) <= TOL_BF16_STATE
+    y_ref, S_ref, _, _, _ = _run_oracle(orc, w, x)
+    e = dict(y_beyond_halfulp=out_err(y, y_ref), y_plain=rel_rms(y, y_ref),
+             state=rel_rms(S, S_ref))
+    report("decode_layer_all", **e)
+    assert e["y_beyond_halfulp"] <= TOL_BF16_OUT, e
+    assert e["state"] <= TOL_BF16_STATE, e
