@@ -108,8 +108,29 @@ __device__ unsigned long long* g_tc_trace = nullptr;
     if (tr_buf_ && threadIdx.x == 0)                                                   \
       tr_buf_[(((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * 64 + (ev)] = clock64(); \
   } while (0)
+// the pre-pass's slot receives a value (the SM, the global time) instead of clock64()
+#define GDN_TRACE_PPV(ev, val)                                                         \
+  do {                                                                                 \
+    if (tr_buf_ && threadIdx.x == 0)                                                   \
+      tr_buf_[(((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * 64 + (ev)] = (val); \
+  } while (0)
+// clock64() as seen by thread t
+#define GDN_TRACE_PPT(ev, t)                                                           \
+  do {                                                                                 \
+    if (tr_buf_ && threadIdx.x == (t))                                                 \
+      tr_buf_[(((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * 64 + (ev)] = clock64(); \
+  } while (0)
+// inside the solve (a device function: the buffer pointer is read where it is used)
+#define GDN_TRACE_SOLVE(ev)                                                            \
+  do {                                                                                 \
+    if (g_tc_trace && threadIdx.x == 0)                                                \
+      g_tc_trace[(((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) * 64 + (ev)] = clock64(); \
+  } while (0)
 #else
+#define GDN_TRACE_SOLVE(ev) do {} while (0)
 #define GDN_TRACE_INIT do {} while (0)
+#define GDN_TRACE_PPT(ev, t) do {} while (0)
+#define GDN_TRACE_PPV(ev, val) do {} while (0)
 #define GDN_TRACE_PP(ev) do {} while (0)
 #define GDN_TRACE(c, ev) do {} while (0)
 #define GDN_TRACE_G(c, ev) do {} while (0)
@@ -230,12 +251,14 @@ __device__ __forceinline__ void solve_unit_lower(uint32_t s, int ptid, float (&t
       }
       x[i] = a0 + a1;
     }
+    GDN_TRACE_SOLVE(23);
     tc::named_bar(3, 64);                             // every row of A_bb read: D_b replaces it
     const uint32_t Tb = blkT(s, b, b);
 #pragma unroll
     for (int i = 0; i < 16; ++i) tc::sts1(at(Tb, i, col), x[i]);
   }
   tc::named_bar(1, 128);
+  GDN_TRACE_SOLVE(24);
   const int w = ptid >> 5, lane = ptid & 31, g = lane >> 2, t = lane & 3;
   {                                                   // At_ik = D_i A_ik, into T's off-diagonal
     Tile tl[3];
@@ -255,6 +278,7 @@ __device__ __forceinline__ void solve_unit_lower(uint32_t s, int ptid, float (&t
     }
   }
   tc::named_bar(1, 128);
+  GDN_TRACE_SOLVE(25);
   // U_20 = -At_20 + At_21 At_10;  U_31 = -At_31 + At_32 At_21;  V_30 = -At_30 + At_31 At_10
   // (into sA's blocks (2,0), (3,1), (3,0); A itself is no longer needed).  Half blocks w, w + 4.
   {
@@ -281,6 +305,7 @@ __device__ __forceinline__ void solve_unit_lower(uint32_t s, int ptid, float (&t
       }
   }
   tc::named_bar(1, 128);
+  GDN_TRACE_SOLVE(26);
   if (w < 2) {                                        // U_30 = V_30 - At_32 U_20
     const int n0 = 8 * w;
     const Tile tl[1] = {Tile{blkT(s, 3, 2), blk(sA, 2, 0), n0}};
@@ -292,6 +317,7 @@ __device__ __forceinline__ void solve_unit_lower(uint32_t s, int ptid, float (&t
     st_frag(blk(sA, 3, 0), n0, g, t, v);
   }
   tc::named_bar(1, 128);
+  GDN_TRACE_SOLVE(27);
   {                                                   // T_ik = U_ik D_k (U = -At next to diag)
     Tile tl[3];
     float acc[3][4] = {};
@@ -460,6 +486,7 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                   uint8_t* __restrict__ pw, int T, int Hk, int Hv, float scale,
                   const int* __restrict__ cu, int max_len, const __nv_bfloat16* __restrict__ ba) {
   GDN_TRACE_INIT;
+  GDN_TRACE_PP(63);
   extern __shared__ __align__(1024) uint8_t pp_raw[];
   uint8_t* smem = pp_raw + ((1024u - (tc::smem_u32(pp_raw) & 1023u)) & 1023u);
   const uint32_t sb = tc::smem_u32(smem);
@@ -479,6 +506,22 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
   const uint32_t qk = sb + PP_QK, tb = sb + PP_TB;
   uint8_t* rec = pw + (((long)sq * Hv + h) * nC + c) * (long)kPwBytes;
 
+  // The chunk's gates are loaded first, by warps 2-3 (token t0 + gi), so that the loads are in
+  // flight during the setup and the tile load; thread 0 issues the tile load before the TMEM
+  // allocation and the S MMA as soon as the tile is in.
+  const int gi = tid - 64;
+  const bool gw = gi >= 0 && gi < 64;                 // a gate thread
+  float la = 0.f, bt = 0.f;
+  if (gw && t0 + gi < sp.len) {
+    const long r = sp.row0 + t0 + gi;
+    if (ba) {
+      bt = __bfloat162float(ba[r * 2 * Hv + h]);      // b, a: converted below
+      la = __bfloat162float(ba[r * 2 * Hv + Hv + h]);
+    } else {
+      la = log_alpha[r * Hv + h];
+      bt = beta[r * Hv + h];
+    }
+  }
   if (tid == 0) {
     tc::mbar_init(tma_bar, 1);
     tc::mbar_init(mma_bar, 1);
@@ -486,6 +529,13 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     *flag = 0;
     *abort_flag = 0;
     tc::fence_barrier_init();
+    tc::fence_proxy_async_smem();                     // the barriers, for the tile load below
+    tc::mbar_arrive_expect_tx(tma_bar, 32768);
+    const int tc0 = sp.tok0 + (int)t0;
+    tc::tma_load_4d(qk, &tmq, tma_bar, 0, hk, tc0, sp.bcoord);
+    tc::tma_load_4d(qk + 8192, &tmk, tma_bar, 0, hk, tc0, sp.bcoord);
+    tc::tma_load_4d(qk + 16384, &tmq, tma_bar, 64, hk, tc0, sp.bcoord);
+    tc::tma_load_4d(qk + 24576, &tmk, tma_bar, 64, hk, tc0, sp.bcoord);
   }
   if (warp == 0) {
     tc::tmem_alloc(sb + PP_BAR + 16, 128);
@@ -498,65 +548,24 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
   const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
   const int row = tid & 127, half = tid >> 7;         // TMEM lane and column half of this thread
   GDN_TRACE_PP(1);
-  if (tid == 0) {
-    tc::mbar_arrive_expect_tx(tma_bar, 32768);
-    const int tc0 = sp.tok0 + (int)t0;
-    tc::tma_load_4d(qk, &tmq, tma_bar, 0, hk, tc0, sp.bcoord);
-    tc::tma_load_4d(qk + 8192, &tmk, tma_bar, 0, hk, tc0, sp.bcoord);
-    tc::tma_load_4d(qk + 16384, &tmq, tma_bar, 64, hk, tc0, sp.bcoord);
-    tc::tma_load_4d(qk + 24576, &tmk, tma_bar, 64, hk, tc0, sp.bcoord);
-  }
-  // gates: G' = cumsum(log alpha) log2(e) over the chunk, beta, ktil, gamma (zero / flat past T)
-  if (tid < 64) {
-    const long tt = t0 + tid;
-    float la = 0.f, bt = 0.f;
-    if (tt < sp.len) {
-      if (ba) {   // from the in_proj_ba outputs: beta = sigmoid(b), log alpha = -softplus(-a)
-        const __nv_bfloat16* row = ba + (sp.row0 + tt) * 2 * Hv;
-        const float b = __bfloat162float(row[h]), a = __bfloat162float(row[Hv + h]);
-        bt = 1.0f / (1.0f + expf(-b));
-        la = a >= 0.f ? -log1pf(expf(-a)) : a - log1pf(expf(a));
-      } else {
-        la = log_alpha[(sp.row0 + tt) * Hv + h];
-        bt = beta[(sp.row0 + tt) * Hv + h];
-      }
-    }
-    gB[tid] = bt;
-    float incl = la;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const float n = __shfl_up_sync(0xffffffffu, incl, d);
-      if (lane >= d) incl += n;
-    }
-    gG[tid] = incl;
-  }
-  __syncthreads();
-  if (tid >= 32 && tid < 64) gG[tid] += gG[31];       // carry of the first 32 tokens
-  __syncthreads();
-  if (tid < 64) gG[tid] *= 1.4426950408889634f;
-  __syncthreads();
-  float* gE = gG + 256;
-  if (tid < 64) {
-    gKt[tid] = tc::ex2(gG[63] - gG[tid]);
-    reinterpret_cast<float*>(rec + kPwTiles)[tid] = tc::ex2(gG[tid]);
-    // block factors E[b][j] = exp(G_16b - G_j) for j < 16b (each <= 1: G never increases)
-#pragma unroll
-    for (int b = 1; b < 4; ++b) gE[64 * b + tid] = tid < 16 * b ? tc::ex2(gG[16 * b] - gG[tid]) : 0.f;
-  }
-
+  GDN_TRACE_PPV(55, tc::globaltimer_ns());
+  GDN_TRACE_PPV(57, tc::smid());
   // S = [Q; K] K^T into TMEM columns 0..63.  Rows of the tile past the sequence's end (the next
   // packed sequence's tokens) are zeroed first, so they reach no product.
-  const bool tile_ok = tc::mbar_wait(tma_bar, 0, abort_flag, kBudget);
-  if (vrows < C) {
+  bool tile_ok = true;
+  if (vrows < C) {                                    // (uniform)
+    tile_ok = tc::mbar_wait(tma_bar, 0, abort_flag, kBudget);
     for (int i = tid; i < 4 * (C - vrows) * 8; i += PP_THREADS) {
       const int box = i / ((C - vrows) * 8), rem = i - box * (C - vrows) * 8;
       tc::st_shared_v4(qk + box * 8192 + (vrows + (rem >> 3)) * 128 + (rem & 7) * 16, 0u, 0u, 0u,
                        0u);
     }
     tc::fence_proxy_async_smem();
+    __syncthreads();
   }
-  __syncthreads();                                    // gates visible, tile complete
   if (tid == 0) {
+    if (vrows == C) tile_ok = tc::mbar_wait(tma_bar, 0, abort_flag, kBudget);
+    GDN_TRACE_PP(62);
     if (tile_ok) {
       GDN_TRACE_PP(2);
       tc::tc_fence_after();
@@ -569,6 +578,37 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     }
     tc::mma_commit(mma_bar);
   }
+  // gates (warps 2-3, meanwhile): G' = cumsum(log alpha) log2(e) over the chunk, beta, ktil,
+  // gamma (zero / flat past the sequence's end)
+  float* gE = gG + 256;
+  if (gw) {
+    if (ba && t0 + gi < sp.len) {   // from the in_proj_ba outputs: beta = sigmoid(b),
+      const float b = bt, a = la;   // log alpha = -softplus(-a)
+      bt = 1.0f / (1.0f + expf(-b));
+      la = a >= 0.f ? -log1pf(expf(-a)) : a - log1pf(expf(a));
+    }
+    gB[gi] = bt;
+    float incl = la;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const float n = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += n;
+    }
+    if (gi == 31) gG[31] = incl;
+    tc::named_bar(5, 64);
+    if (gi >= 32) incl += gG[31];                     // carry of the first 32 tokens
+    const float g2 = incl * 1.4426950408889634f;
+    tc::named_bar(5, 64);                             // gG[31] read before it is rescaled
+    gG[gi] = g2;
+    tc::named_bar(5, 64);
+    gKt[gi] = tc::ex2(gG[63] - g2);
+    reinterpret_cast<float*>(rec + kPwTiles)[gi] = tc::ex2(g2);
+    // block factors E[b][j] = exp(G_16b - G_j) for j < 16b (each <= 1: G never increases)
+#pragma unroll
+    for (int b = 1; b < 4; ++b) gE[64 * b + gi] = gi < 16 * b ? tc::ex2(gG[16 * b] - g2) : 0.f;
+  }
+  GDN_TRACE_PPT(61, 64);
+  __syncthreads();                                    // gates visible
   tc::mbar_wait(mma_bar, 0, abort_flag, kBudget);
   GDN_TRACE_PP(3);
   tc::tc_fence_after();
@@ -735,7 +775,9 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         tc::bulk_commit();
       }
     }
+    GDN_TRACE_PP(58);
     tc::mbar_wait(mma_bar, 1, abort_flag, kBudget);
+    GDN_TRACE_PP(59);
     tc::tc_fence_after();
     tc::tmem_ld32(tmem + lane_off + 32 * half, w);
     tc::tmem_wait_ld();
@@ -756,7 +798,7 @@ pw_prepass_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     }                                                 // on their own
   }
   GDN_TRACE_PP(8);
-  GDN_TRACE_PP(9);
+  GDN_TRACE_PPV(56, tc::globaltimer_ns());
   if (tid == 0 && *abort_flag) record_error(kErrTimeout);
   tc::tc_fence_before();
   __syncthreads();
