@@ -636,7 +636,7 @@ def profile_case(args):
             gdn.layer_fwd(d["q_raw"], d["k_raw"], d["v_raw"], d["z"], d["conv_wq"], d["conv_wk"],
                           d["conv_wv"], d["log_alpha"], d["beta"], d["S0"], d["norm_w"],
                           Hk=w.Hk, Hv=w.Hv, dk=w.dk, dv=w.dv, chunk=w.chunk, workspace=ws)
-        launches = 1 + launches_per_call(gdn, w)
+        launches = 3 + launches_per_call(gdn, w)   # prologue (q/k, v), forward, gated norm
     elif name in ("decode", "decode_layer"):
         mk = gi.make_decode_inputs if name == "decode" else gi.make_decode_layer_inputs
         d = to_dev(mk(w.with_sizes(steps=1)), dev)
