@@ -494,22 +494,35 @@ gdn_status gdn_prologue(const void* q_raw, const void* k_raw, const void* v_raw,
     return GDN_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if ((T + kPrologueTokens - 1) / kPrologueTokens > 65535) return GDN_ERR_UNSUPPORTED;
-  // q and k heads (normalised rows), then the v heads; head slots fastest in each grid
+  // the q and k heads (normalised rows) on the library's high-priority stream, forked from and
+  // joined back into `stream`, beside the v heads on `stream`: the two kernels share the SMs (the
+  // q/k kernel is latency-bound at three CTAs per SM, the v kernel issue-bound); head slots
+  // fastest in each grid
   const unsigned tb = (unsigned)((T + kPrologueTokens - 1) / kPrologueTokens);
   const dim3 gqk(2 * Hk, tb, B), gv(Hv, tb, B);
+  std::lock_guard<std::mutex> lock(tcf::split_mutex());
+  tcf::Split* sp = tcf::split_for_device();
+  if (!sp || cudaEventRecord(sp->ev_fork, st) != cudaSuccess ||
+      cudaStreamWaitEvent(sp->s_hi, sp->ev_fork, 0) != cudaSuccess)
+    return GDN_ERR_CUDA;
   if (dtype == GDN_F32) {
-    prologue_qk_kernel<float><<<gqk, 128, prologue_smem_bytes(dk, 4), st>>>(
+    prologue_qk_kernel<float><<<gqk, 128, prologue_smem_bytes(dk, 4), sp->s_hi>>>(
         (const float*)q_raw, (const float*)k_raw, wq, wk, (float*)q, (float*)k, T, Hk, dk, l2_eps);
     prologue_v_kernel<float><<<gv, 128, prologue_smem_bytes(dv, 4), st>>>(
         (const float*)v_raw, wv, (float*)v, T, Hv, dv);
   } else {
     using bf = __nv_bfloat16;
-    prologue_qk_kernel<bf><<<gqk, 128, prologue_smem_bytes(dk, 2), st>>>(
+    prologue_qk_kernel<bf><<<gqk, 128, prologue_smem_bytes(dk, 2), sp->s_hi>>>(
         (const bf*)q_raw, (const bf*)k_raw, wq, wk, (bf*)q, (bf*)k, T, Hk, dk, l2_eps);
     prologue_v_kernel<bf><<<gv, 128, prologue_smem_bytes(dv, 2), st>>>(
         (const bf*)v_raw, wv, (bf*)v, T, Hv, dv);
   }
-  return launch_status();
+  const gdn_status ls = launch_status();
+  // the caller's stream waits for the q/k kernel, also after a failed launch
+  if (cudaEventRecord(sp->ev_hi, sp->s_hi) != cudaSuccess ||
+      cudaStreamWaitEvent(st, sp->ev_hi, 0) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  return ls;
 }
 
 gdn_status gdn_out_norm(const void* o, const void* z, const float* w, void* y, long long rows,

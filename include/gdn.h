@@ -276,7 +276,9 @@ GDN_API gdn_status gdn_gates(const void *ba, float *log_alpha, float *beta, long
  *   q, k [B, T, Hk, dk]; v [B, T, Hv, dv]                    (dtype, outputs)
  * bf16 outputs are the exact results rounded to the nearest bf16 (ties to even): a value whose
  * rounding the fp32 computation cannot decide within its error bound is recomputed in fp64, so
- * the rounding never depends on fp32 roundoff.
+ * the rounding never depends on fp32 roundoff.  Two kernels: the q and k heads run on the
+ * library's high-priority stream of the device (forked from and joined back into `stream`), the
+ * v heads on `stream`, so that both share the SMs; `stream` waits for both.
  */
 GDN_API gdn_status gdn_prologue(const void *q_raw, const void *k_raw, const void *v_raw,
                         const float *wq, const float *wk, const float *wv,
