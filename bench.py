@@ -93,24 +93,34 @@ def load_peaks():
     return dict(FALLBACK_PEAKS)
 
 
-def kernel_source_sha() -> str:
+# The source files whose kernels (and launch schedule) a recorded traffic figure depends on.
+TRAFFIC_SOURCES = {
+    "gdn_chunk_fwd_tc": ("common.cuh", "tc_chunk.cuh", "tc_ptx.cuh"),
+    "gdn_layer_fwd": None,                     # every file of csrc/
+}
+
+
+def kernel_source_sha(files=None) -> str:
+    """sha256 (16 hex digits) of the named files of csrc/, or of all of its .cu / .cuh files."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_deltanet_linear_18_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    names = sorted(files) if files else sorted(n for n in os.listdir(csrc)
+                                              if n.endswith((".cu", ".cuh")))
+    for name in names:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged."""
+    """DRAM bytes per call from the committed ncu summary, if the sources of its kernels are
+    unchanged since the capture (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         rec = json.load(f).get(kernel, {}).get(workload)
-    if not rec or rec.get("source_sha") != kernel_source_sha():
+    if not rec or rec.get("source_sha") != kernel_source_sha(TRAFFIC_SOURCES.get(kernel)):
         return None
     return rec.get("bytes_per_launch")
 
