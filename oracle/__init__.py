@@ -124,6 +124,8 @@ class OracleLib:
         lib.oracle_gated_rmsnorm.restype = None
         lib.oracle_gates.argtypes = [P, P, P, L, I]
         lib.oracle_gates.restype = None
+        lib.oracle_gated_delta_bwd.argtypes = [P] * 14 + [L, L, I, I, I, I, D, I]
+        lib.oracle_gated_delta_bwd.restype = I
         self.lib = lib
         self.path = path
 
@@ -150,6 +152,33 @@ class OracleLib:
         if rc != 0:
             raise ValueError("oracle_gated_delta rejected the sizes")
         return o, sT
+
+    def gated_delta_bwd(self, q, k, v, log_alpha, beta, S0, dO, dS_T=None, scale: float = 1.0,
+                        threads: Optional[int] = None) -> dict:
+        """Gradients of L = sum <dO, o> + <dS_T, S_T> (o, S_T of ``gated_delta`` on the same
+        inputs) by the chain rule through every token in reverse.  dO [B,T,Hv,dv]; dS_T
+        [B,Hv,dk,dv] holding S^T or None.  Returns fp64 dq, dk [B,T,Hk,dk] (summed over each
+        key head's value heads), dv [B,T,Hv,dv], dlog_alpha, dbeta [B,T,Hv], dS0 [B,Hv,dk,dv].
+        Each host thread keeps T + 1 states of one head."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        la, be, s0, do, dst = _f64(log_alpha), _f64(beta), _f64(S0), _f64(dO), _f64(dS_T)
+        B, T, Hk, dk = q.shape
+        Hv, dv = v.shape[2], v.shape[3]
+        assert k.shape == q.shape and v.shape[:2] == (B, T) and do.shape == v.shape
+        assert la.shape == (B, T, Hv) == be.shape
+        for s_ in (s0, dst):
+            assert s_ is None or s_.shape == (B, Hv, dk, dv)
+        out = {"dq": np.zeros((B, T, Hk, dk)), "dk": np.zeros((B, T, Hk, dk)),
+               "dv": np.zeros((B, T, Hv, dv)), "dlog_alpha": np.zeros((B, T, Hv)),
+               "dbeta": np.zeros((B, T, Hv)), "dS0": np.zeros((B, Hv, dk, dv))}
+        rc = self.lib.oracle_gated_delta_bwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(be), _ptr(s0), _ptr(do), _ptr(dst),
+            _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dlog_alpha"]),
+            _ptr(out["dbeta"]), _ptr(out["dS0"]), B, T, Hk, Hv, dk, dv, float(scale),
+            int(threads or default_threads()))
+        if rc != 0:
+            raise ValueError(f"oracle_gated_delta_bwd failed ({rc})")
+        return out
 
     def decode_steps(self, q, k, v, log_alpha, beta, S0, scale: float = 1.0,
                      threads: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray]:
@@ -309,6 +338,10 @@ def get() -> OracleLib:
 
 def gated_delta(*a, **kw):
     return get().gated_delta(*a, **kw)
+
+
+def gated_delta_bwd(*a, **kw):
+    return get().gated_delta_bwd(*a, **kw)
 
 
 def decode_steps(*a, **kw):

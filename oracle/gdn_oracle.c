@@ -218,3 +218,209 @@ void oracle_gates(const double *ba, double *log_alpha, double *beta, long rows, 
             log_alpha[r * Hv + h] = -softplus(-a);
         }
 }
+
+/* ------------------------------------------------------------------------------------------ */
+/* Backward pass of the recurrence: reverse-mode derivative of the loss through every token    */
+/* ------------------------------------------------------------------------------------------ */
+/*
+ * The pages train their models ([HYB], [KIMI]) but give the layer for inference only; the
+ * gradient here is the exact derivative of the recurrence above, taken by the chain rule one
+ * token at a time in reverse, in the equation's own order.  Per token, with P = S_{t-1}:
+ *
+ *      x = P k,   A = P - beta x k^T,   S_t = alpha A + beta v k^T,   o_t = scale S_t q_t.
+ *
+ * Given G = dL/dS_t (the state gradient from later tokens plus this token's output):
+ *      G     += scale do q^T                         (o_t = scale S_t q_t)
+ *      dq    += scale S_t^T do
+ *      dlog_alpha = alpha <G, A>,  dA = alpha G      (S_t = alpha A + ...)
+ *      dbeta += v^T G k,  dv = beta G k,  dk += beta G^T v        (... + beta v k^T)
+ *      dP = dA,  dbeta -= x^T dA k,  dx = -beta dA k,  dk -= beta dA^T x   (A = P - beta x k^T)
+ *      dP += dx k^T,  dk += P^T dx                    (x = P k)
+ *      dL/dS_{t-1} = dP.
+ * The states S_0 .. S_T of a (batch, value head) are recomputed forward first and kept (the
+ * tape).  The loss is L = sum <dO, o> + <dS_T, S_T>; dq and dk sum over the value heads that
+ * share a key head, so one worker owns all value heads of a (batch, key head).
+ */
+typedef struct {
+    const double *q, *k, *v, *log_alpha, *beta, *S0, *dO, *dST;
+    double *dq, *dk, *dv, *dla, *dbeta, *dS0;
+    long B, T;
+    int Hk, Hv, dk_, dv_;
+    double scale;
+    int nthreads, tid;
+} bwd_job;
+
+static void bwd_one_head(const bwd_job *J, long b, int h, double *tape, double *G, double *dP,
+                         double *x, double *dx, double *Gk, double *A)
+{
+    const int dk = J->dk_, dv = J->dv_, Hk = J->Hk, Hv = J->Hv;
+    const int group = Hv / Hk, hk = h / group;         /* GQA: contiguous groups */
+    const long T = J->T, SS = (long)dv * dk;
+    const long st0 = ((long)b * Hv + h) * dk * dv;      /* this head's [dk][dv] state slot */
+    /* forward: the tape of states, tape[t] = S_t (S_0 the initial state) */
+    for (int a = 0; a < dv; ++a)
+        for (int c = 0; c < dk; ++c)
+            tape[(long)a * dk + c] = J->S0 ? J->S0[st0 + (long)c * dv + a] : 0.0;
+    for (long t = 0; t < T; ++t) {
+        const double *P = tape + t * SS;
+        double *S = tape + (t + 1) * SS;
+        const double *k = J->k + ((b * T + t) * Hk + hk) * (long)dk;
+        const double *v = J->v + ((b * T + t) * Hv + h) * (long)dv;
+        const double alpha = exp(J->log_alpha[(b * T + t) * Hv + h]);
+        const double beta = J->beta[(b * T + t) * Hv + h];
+        for (int a = 0; a < dv; ++a) {
+            double acc = 0.0;
+            for (int c = 0; c < dk; ++c) acc += P[(long)a * dk + c] * k[c];
+            x[a] = acc;
+        }
+        for (int a = 0; a < dv; ++a)
+            for (int c = 0; c < dk; ++c)
+                S[(long)a * dk + c] = alpha * (P[(long)a * dk + c] - beta * x[a] * k[c]) +
+                                      beta * v[a] * k[c];
+    }
+    /* reverse */
+    for (int a = 0; a < dv; ++a)
+        for (int c = 0; c < dk; ++c)
+            G[(long)a * dk + c] = J->dST ? J->dST[st0 + (long)c * dv + a] : 0.0;
+    for (long t = T - 1; t >= 0; --t) {
+        const double *P = tape + t * SS, *S = tape + (t + 1) * SS;
+        const long row = (b * T + t) * Hv + h;
+        const double *q = J->q + ((b * T + t) * Hk + hk) * (long)dk;
+        const double *k = J->k + ((b * T + t) * Hk + hk) * (long)dk;
+        const double *v = J->v + row * (long)dv;
+        const double *dO = J->dO + row * (long)dv;
+        double *dq = J->dq + ((b * T + t) * Hk + hk) * (long)dk;
+        double *dkk = J->dk + ((b * T + t) * Hk + hk) * (long)dk;
+        double *dvv = J->dv + row * (long)dv;
+        const double alpha = exp(J->log_alpha[row]);
+        const double beta = J->beta[row];
+        /* o_t = scale S_t q_t */
+        for (int a = 0; a < dv; ++a)
+            for (int c = 0; c < dk; ++c) G[(long)a * dk + c] += J->scale * dO[a] * q[c];
+        for (int c = 0; c < dk; ++c) {
+            double acc = 0.0;
+            for (int a = 0; a < dv; ++a) acc += S[(long)a * dk + c] * dO[a];
+            dq[c] += J->scale * acc;
+        }
+        /* x = P k and A = P - beta x k^T, recomputed from the tape */
+        for (int a = 0; a < dv; ++a) {
+            double acc = 0.0;
+            for (int c = 0; c < dk; ++c) acc += P[(long)a * dk + c] * k[c];
+            x[a] = acc;
+        }
+        for (int a = 0; a < dv; ++a)
+            for (int c = 0; c < dk; ++c) A[(long)a * dk + c] = P[(long)a * dk + c] - beta * x[a] * k[c];
+        /* S_t = alpha A + beta v k^T */
+        double ga = 0.0;
+        for (long i = 0; i < SS; ++i) ga += G[i] * A[i];
+        J->dla[row] = alpha * ga;
+        for (int a = 0; a < dv; ++a) {
+            double acc = 0.0;
+            for (int c = 0; c < dk; ++c) acc += G[(long)a * dk + c] * k[c];
+            Gk[a] = acc;
+        }
+        double db = 0.0;
+        for (int a = 0; a < dv; ++a) db += v[a] * Gk[a];
+        for (int a = 0; a < dv; ++a) dvv[a] = beta * Gk[a];
+        for (int c = 0; c < dk; ++c) {
+            double acc = 0.0;
+            for (int a = 0; a < dv; ++a) acc += G[(long)a * dk + c] * v[a];
+            dkk[c] += beta * acc;
+        }
+        /* A = P - beta x k^T, with dA = alpha G */
+        for (long i = 0; i < SS; ++i) dP[i] = alpha * G[i];
+        for (int a = 0; a < dv; ++a) {
+            double acc = 0.0;
+            for (int c = 0; c < dk; ++c) acc += dP[(long)a * dk + c] * k[c];
+            db -= x[a] * acc;
+            dx[a] = -beta * acc;
+        }
+        for (int c = 0; c < dk; ++c) {
+            double acc = 0.0;
+            for (int a = 0; a < dv; ++a) acc += dP[(long)a * dk + c] * x[a];
+            dkk[c] -= beta * acc;
+        }
+        J->dbeta[row] = db;
+        /* x = P k */
+        for (int c = 0; c < dk; ++c) {
+            double acc = 0.0;
+            for (int a = 0; a < dv; ++a) acc += P[(long)a * dk + c] * dx[a];
+            dkk[c] += acc;
+        }
+        for (int a = 0; a < dv; ++a)
+            for (int c = 0; c < dk; ++c) dP[(long)a * dk + c] += dx[a] * k[c];
+        memcpy(G, dP, sizeof(double) * (size_t)SS);      /* dL/dS_{t-1} */
+    }
+    if (J->dS0)
+        for (int a = 0; a < dv; ++a)
+            for (int c = 0; c < dk; ++c)
+                J->dS0[st0 + (long)c * dv + a] = G[(long)a * dk + c];
+}
+
+static void *bwd_worker(void *arg)
+{
+    const bwd_job *J = (const bwd_job *)arg;
+    const long SS = (long)J->dk_ * J->dv_;
+    double *tape = (double *)malloc(sizeof(double) * (size_t)SS * (size_t)(J->T + 1));
+    double *G = (double *)malloc(sizeof(double) * (size_t)SS);
+    double *dP = (double *)malloc(sizeof(double) * (size_t)SS);
+    double *A = (double *)malloc(sizeof(double) * (size_t)SS);
+    double *x = (double *)malloc(sizeof(double) * (size_t)J->dv_ * 3);
+    if (!tape || !G || !dP || !A || !x) {
+        free(tape); free(G); free(dP); free(A); free(x);
+        return (void *)1;
+    }
+    const int G_ = J->Hv / J->Hk;
+    const long groups = J->B * J->Hk;
+    for (long p = J->tid; p < groups; p += J->nthreads) {
+        const long b = p / J->Hk;
+        const int hk = (int)(p % J->Hk);
+        for (long t = 0; t < J->T; ++t) {           /* this worker owns dq, dk of (b, hk) */
+            memset(J->dq + ((b * J->T + t) * J->Hk + hk) * (long)J->dk_, 0, sizeof(double) * J->dk_);
+            memset(J->dk + ((b * J->T + t) * J->Hk + hk) * (long)J->dk_, 0, sizeof(double) * J->dk_);
+        }
+        for (int g = 0; g < G_; ++g)
+            bwd_one_head(J, b, hk * G_ + g, tape, G, dP, x, x + J->dv_, x + 2 * J->dv_, A);
+    }
+    free(tape); free(G); free(dP); free(A); free(x);
+    return NULL;
+}
+
+/*
+ * Gradients of L = sum <dO, o> + <dS_T, S_T> with o, S_T from oracle_gated_delta on the same
+ * inputs.  Shapes as there; dO: [B, T, Hv, dv]; dS_T (nullable = zero): [B, Hv, dk, dv] (S^T).
+ * Outputs: dq, dk [B, T, Hk, dk] (summed over each key head's value heads), dv [B, T, Hv, dv],
+ * dlog_alpha, dbeta [B, T, Hv], dS0 (nullable) [B, Hv, dk, dv] (S^T).  Memory: one tape of T + 1
+ * states per host thread.  Returns 0, -1 on bad sizes, -2 if a tape could not be allocated.
+ */
+int oracle_gated_delta_bwd(const double *q, const double *k, const double *v,
+                           const double *log_alpha, const double *beta, const double *S0,
+                           const double *dO, const double *dS_T, double *dq, double *dk,
+                           double *dv, double *dlog_alpha, double *dbeta, double *dS0, long B,
+                           long T, int Hk, int Hv, int dk_, int dv_, double scale, int nthreads)
+{
+    if (B < 0 || T < 0 || Hk <= 0 || Hv <= 0 || dk_ <= 0 || dv_ <= 0 || Hv % Hk) return -1;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 1024) nthreads = 1024;
+    bwd_job *jobs = (bwd_job *)calloc((size_t)nthreads, sizeof(bwd_job));
+    pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    void **ret = (void **)calloc((size_t)nthreads, sizeof(void *));
+    for (int i = 0; i < nthreads; ++i) {
+        bwd_job J = {q, k, v, log_alpha, beta, S0, dO, dS_T, dq, dk, dv, dlog_alpha, dbeta, dS0,
+                     B, T, Hk, Hv, dk_, dv_, scale, nthreads, i};
+        jobs[i] = J;
+    }
+    char *started = (char *)calloc((size_t)nthreads, 1);
+    for (int i = 1; i < nthreads; ++i)
+        started[i] = pthread_create(&th[i], NULL, bwd_worker, &jobs[i]) == 0;
+    ret[0] = bwd_worker(&jobs[0]);
+    for (int i = 1; i < nthreads; ++i) {
+        if (started[i]) pthread_join(th[i], &ret[i]);
+        else ret[i] = bwd_worker(&jobs[i]);
+    }
+    int rc = 0;
+    for (int i = 0; i < nthreads; ++i)
+        if (ret[i]) rc = -2;
+    free(started); free(jobs); free(th); free(ret);
+    return rc;
+}

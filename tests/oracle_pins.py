@@ -388,4 +388,76 @@ def pin_gates_closed_forms(orc):
     assert np.isclose(np.exp(la[60, 0]), 0.5)
 
 
+# ---------------------------------------------------------------------------------------------
+# backward pass: the exact derivative of the recurrence
+# ---------------------------------------------------------------------------------------------
+
+def _loss(orc, q, k, v, la, be, S0, dO, dST, scale):
+    o, sT = orc.gated_delta(q, k, v, la, be, S0, scale=scale, threads=1)
+    return float(np.sum(dO * o) + np.sum(dST * sT))
+
+
+def pin_bwd_central_differences(orc):
+    """Every gradient entry equals the central difference (L(x + h) - L(x - h)) / 2h of the
+    forward oracle's loss L = <dO, o> + <dS_T, S_T>, for every input (q, k, v, log alpha, beta,
+    S0), with two value heads sharing a key head (dq, dk sum over them).  Central differences
+    are exact to O(h^2) for these smooth functions; h = 1e-5 gives about 1e-9 relative."""
+    q, k, v, la, be, S0 = _rand(41, T=5, Hk=1, Hv=2, dk=3, dv=2)
+    rng = np.random.default_rng(42)
+    dO = rng.standard_normal(v.shape)
+    dST = rng.standard_normal(S0.shape)
+    scale = 0.7
+    g = orc.gated_delta_bwd(q, k, v, la, be, S0, dO, dST, scale=scale, threads=1)
+    args = {"q": q, "k": k, "v": v, "la": la, "be": be, "S0": S0}
+    names = {"q": "dq", "k": "dk", "v": "dv", "la": "dlog_alpha", "be": "dbeta", "S0": "dS0"}
+    h = 1e-5
+    for name, x in args.items():
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            old = x[idx]
+            x[idx] = old + h
+            lp = _loss(orc, dO=dO, dST=dST, scale=scale, **args)
+            x[idx] = old - h
+            lm = _loss(orc, dO=dO, dST=dST, scale=scale, **args)
+            x[idx] = old
+            fd[idx] = (lp - lm) / (2 * h)
+        got = g[names[name]]
+        err = np.max(np.abs(got - fd)) / max(1.0, np.max(np.abs(fd)))
+        assert err < 1e-7, (name, err)
+
+
+def pin_bwd_closed_forms_alpha1_beta0(orc):
+    """alpha = 1, beta = 0: S_t = S0 for every t, so o_t = scale S0 q_t and
+    dq_t = sum_h scale S0_h^T dO_t,h;  dk = dv = 0;  dS0 = dS_T + sum_t scale dO_t q_t^T;
+    with G_t = dS_T + sum_{s >= t} scale dO_s q_s^T (the gradient reaching S_t):
+    dlog alpha_t = <G_t, S0>  and  dbeta_t = (v_t - S0 k_t)^T G_t k_t."""
+    B, T, Hk, Hv, dk, dv = 1, 6, 1, 2, 4, 3
+    q, k, v, _, _, S0 = _rand(43, B=B, T=T, Hk=Hk, Hv=Hv, dk=dk, dv=dv)
+    la = np.zeros((B, T, Hv))
+    be = np.zeros((B, T, Hv))
+    rng = np.random.default_rng(44)
+    dO = rng.standard_normal(v.shape)
+    dST = rng.standard_normal(S0.shape)
+    scale = 0.5
+    g = orc.gated_delta_bwd(q, k, v, la, be, S0, dO, dST, scale=scale, threads=1)
+    assert np.abs(g["dk"]).max() == 0.0 and np.abs(g["dv"]).max() == 0.0
+    dq = np.zeros((T, dk))
+    for h in range(Hv):
+        S = S0[0, h].T                                   # d_v x d_k, the equation's orientation
+        G = dST[0, h].T.copy()
+        Gs = [None] * T
+        for t in range(T - 1, -1, -1):
+            G = G + scale * np.outer(dO[0, t, h], q[0, t, 0])
+            Gs[t] = G.copy()
+        for t in range(T):
+            dq[t] += scale * S.T @ dO[0, t, h]
+            np.testing.assert_allclose(g["dlog_alpha"][0, t, h], np.sum(Gs[t] * S), rtol=1e-12,
+                                       atol=1e-12)
+            u = v[0, t, h] - S @ k[0, t, 0]
+            np.testing.assert_allclose(g["dbeta"][0, t, h], u @ Gs[t] @ k[0, t, 0], rtol=1e-12,
+                                       atol=1e-12)
+        np.testing.assert_allclose(g["dS0"][0, h], Gs[0].T, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(g["dq"][0, :, 0], dq, rtol=1e-12, atol=1e-12)
+
+
 ALL_PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]

@@ -49,6 +49,19 @@ MUTANTS = {
     "gate_sigmoid_not_silu": ("* (zz * sigmoid(zz));", "* sigmoid(zz);"),
     "gain_ignored": ("y[r * d + i] = (o[r * d + i] * inv) * w[i] * (zz * sigmoid(zz));",
                      "y[r * d + i] = (o[r * d + i] * inv) * (zz * sigmoid(zz));"),
+    # backward pass
+    "bwd_output_grad_ignores_scale": ("G[(long)a * dk + c] += J->scale * dO[a] * q[c];",
+                                      "G[(long)a * dk + c] += dO[a] * q[c];"),
+    "bwd_dq_reads_previous_state": ("for (int a = 0; a < dv; ++a) acc += S[(long)a * dk + c] * dO[a];",
+                                    "for (int a = 0; a < dv; ++a) acc += P[(long)a * dk + c] * dO[a];"),
+    "bwd_dlog_alpha_missing_alpha": ("J->dla[row] = alpha * ga;", "J->dla[row] = ga;"),
+    "bwd_dv_missing_beta": ("dvv[a] = beta * Gk[a];", "dvv[a] = Gk[a];"),
+    "bwd_state_grad_not_decayed": ("for (long i = 0; i < SS; ++i) dP[i] = alpha * G[i];",
+                                   "for (long i = 0; i < SS; ++i) dP[i] = G[i];"),
+    "bwd_dbeta_drops_erase_term": ("db -= x[a] * acc;", "db -= 0.0 * acc;"),
+    "bwd_dk_drops_state_term": ("dkk[c] += acc;", "dkk[c] += 0.0 * acc;"),
+    "bwd_state_grad_drops_rank1": ("dP[(long)a * dk + c] += dx[a] * k[c];",
+                                   "dP[(long)a * dk + c] += 0.0 * dx[a] * k[c];"),
 }
 
 
