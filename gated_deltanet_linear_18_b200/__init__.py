@@ -90,6 +90,10 @@ def lib() -> ctypes.CDLL:
         L.gdn_layer_fwd_static.argtypes = [P] * 13 + [I] * 7 + [F, F, F, I, I, P]
         L.gdn_layer_fwd_static.restype = I
         L.gdn_layer_workspace_bytes.restype = SZ
+        L.gdn_bwd.argtypes = [P] * 15 + [SZ] + [I] * 6 + [F, I, P]
+        L.gdn_bwd.restype = I
+        L.gdn_bwd_workspace_bytes.argtypes = [I] * 6
+        L.gdn_bwd_workspace_bytes.restype = SZ
         _lib = L
     return _lib
 
@@ -200,6 +204,41 @@ def chunk_fwd(q, k, v, log_alpha, beta, S0=None, *, chunk: int = 64, scale: floa
                                     _stream(dev))
     _check("gdn_chunk_fwd", st)
     return o, sT
+
+
+def bwd_workspace_bytes(B, T, Hk, Hv, dk, dv) -> int:
+    """Caller-owned device scratch one ``bwd`` call needs."""
+    return int(lib().gdn_bwd_workspace_bytes(B, T, Hk, Hv, dk, dv))
+
+
+def bwd(q, k, v, log_alpha, beta, S0, dO, dS_T=None, *, scale: float = 1.0,
+        workspace: Optional[torch.Tensor] = None, want_dS0: bool = True) -> dict:
+    """Gradients of sum <dO, o> + <dS_T, S_T> for the forward on the same inputs (gdn_bwd):
+    fp32 dq, dk [B,T,Hk,dk] (summed over each key head's value heads), dv [B,T,Hv,dv],
+    dlog_alpha, dbeta [B,T,Hv], dS0 [B,Hv,dk,dv] (None unless ``want_dS0``)."""
+    B, T, Hk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    if (k.shape != q.shape or v.shape[:2] != (B, T) or dO.shape != v.shape
+            or k.dtype != q.dtype or v.dtype != q.dtype or dO.dtype != q.dtype):
+        raise ValueError("q, k, v, dO shapes/dtypes disagree")
+    if log_alpha.shape != (B, T, Hv) or beta.shape != (B, T, Hv):
+        raise ValueError("gates must be [B, T, Hv]")
+    _f32(log_alpha, beta, S0, dS_T)
+    f = dict(device=q.device, dtype=torch.float32)
+    out = {"dq": torch.empty(B, T, Hk, dk, **f), "dk": torch.empty(B, T, Hk, dk, **f),
+           "dv": torch.empty(B, T, Hv, dv, **f), "dlog_alpha": torch.empty(B, T, Hv, **f),
+           "dbeta": torch.empty(B, T, Hv, **f),
+           "dS0": torch.empty(B, Hv, dk, dv, **f) if want_dS0 else None}
+    dev = _dev(q, k, v, log_alpha, beta, S0, dO, dS_T, workspace)
+    ws, wbytes = _workspace(bwd_workspace_bytes(B, T, Hk, Hv, dk, dv), dev, workspace)
+    with torch.cuda.device(dev):
+        st = lib().gdn_bwd(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(S0), _p(dO),
+                           _p(dS_T), _p(out["dq"]), _p(out["dk"]), _p(out["dv"]),
+                           _p(out["dlog_alpha"]), _p(out["dbeta"]), _p(out["dS0"]), _p(ws),
+                           wbytes, B, T, Hk, Hv, dk, dv, float(scale), _io_dtype(q),
+                           _stream(dev))
+    _check("gdn_bwd", st)
+    return out
 
 
 def chunk_fwd_ba(q, k, v, ba, S0=None, *, chunk: int = 64, scale: float = 1.0,

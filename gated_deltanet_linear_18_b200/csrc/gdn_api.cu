@@ -8,6 +8,7 @@
 #include "gdn.h"
 #include "common.cuh"
 #include "decode.cuh"
+#include "bwd.cuh"
 #include "decode_layer.cuh"
 #include "elementwise.cuh"
 #include "simt_chunk.cuh"
@@ -209,9 +210,112 @@ gdn_status validate_heads(int Hk, int Hv, int dk, int dv) {
   return GDN_OK;
 }
 
+// ---------------------------------------------------------------------------------------------
+// Backward pass: checkpoints every bwd::kSeg tokens, then (when key heads are shared) dq and dk
+// per value head, summed over each key head's group afterwards.  Workspace sections 256-aligned.
+// ---------------------------------------------------------------------------------------------
+size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
+struct BwdLayout {
+  size_t dqh = 0, dkh = 0, total = 0;   // offsets of the per-value-head dq, dk; total bytes
+};
+BwdLayout bwd_layout(int B, int T, int Hk, int Hv, int dk, int dv) {
+  BwdLayout L;
+  const size_t nseg = ((size_t)T + bwd::kSeg - 1) / bwd::kSeg;
+  const size_t ck = align256((size_t)B * Hv * nseg * dk * dv * sizeof(float));
+  const size_t per = Hv != Hk ? align256((size_t)B * T * Hv * dk * sizeof(float)) : 0;
+  L.dqh = ck;
+  L.dkh = ck + per;
+  L.total = ck + 2 * per;
+  return L;
+}
+
+template <int D, typename Tin>
+gdn_status bwd_launch(const void* q, const void* k, const void* v, const float* la,
+                      const float* be, const float* S0, const void* dO, const float* dST,
+                      float* dq, float* dk, float* dv, float* dla, float* dbeta, float* dS0,
+                      void* ws, int B, int T, int Hk, int Hv, float scale, cudaStream_t st) {
+  auto kern = bwd::bwd_kernel<D, D, Tin>;
+  const size_t smem = bwd::smem_bytes<D, D>();
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return GDN_ERR_CUDA;
+  const BwdLayout L = bwd_layout(B, T, Hk, Hv, D, D);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  const bool grouped = Hv != Hk;
+  float* dqo = grouped ? reinterpret_cast<float*>(w + L.dqh) : dq;
+  float* dko = grouped ? reinterpret_cast<float*>(w + L.dkh) : dk;
+  kern<<<(unsigned)((long)B * Hv), bwd::Shape<D, D>::NT, smem, st>>>(
+      static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v), la, be,
+      S0, static_cast<const Tin*>(dO), dST, dqo, dko, grouped ? Hv : Hk, dv, dla, dbeta, dS0,
+      reinterpret_cast<float*>(w), T, Hk, Hv, scale);
+  if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
+  if (grouped && T > 0) {
+    const long rows = (long)B * T * Hk;
+    const long n = 2 * rows * D;
+    const unsigned blocks = (unsigned)std::min<long>((n + 255) / 256, 148L * 16);
+    bwd::group_sum_kernel<<<blocks, 256, 0, st>>>(dqo, dq, dko, dk, rows, Hv / Hk, D);
+  }
+  return launch_status();
+}
+
+template <typename Tin>
+gdn_status bwd_dispatch(int d, const void* q, const void* k, const void* v, const float* la,
+                        const float* be, const float* S0, const void* dO, const float* dST,
+                        float* dq, float* dk, float* dv, float* dla, float* dbeta, float* dS0,
+                        void* ws, int B, int T, int Hk, int Hv, float scale, cudaStream_t st) {
+#define GDN_BWD(D)                                                                              \
+  case D:                                                                                       \
+    return bwd_launch<D, Tin>(q, k, v, la, be, S0, dO, dST, dq, dk, dv, dla, dbeta, dS0, ws, B, \
+                              T, Hk, Hv, scale, st);
+  switch (d) {
+    GDN_BWD(16)
+    GDN_BWD(32)
+    GDN_BWD(64)
+    GDN_BWD(128)
+    default: return GDN_ERR_UNSUPPORTED;
+  }
+#undef GDN_BWD
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t gdn_bwd_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv) {
+  if (B < 0 || T < 0 || validate_heads(Hk, Hv, dk, dv) != GDN_OK || dk != dv) return 0;
+  if ((long)B * T == 0) return 0;
+  return bwd_layout(B, T, Hk, Hv, dk, dv).total;
+}
+
+gdn_status gdn_bwd(const void* q, const void* k, const void* v, const float* log_alpha,
+                   const float* beta, const float* S0, const void* dO, const float* dS_T,
+                   float* dq, float* dk, float* dv, float* dlog_alpha, float* dbeta, float* dS0,
+                   void* workspace, size_t workspace_bytes, int B, int T, int Hk, int Hv,
+                   int dk_, int dv_, float scale, gdn_dtype dtype, gdn_stream_t stream) {
+  if (B < 0 || T < 0 || !valid_dtype(dtype)) return GDN_ERR_INVALID_ARG;
+  gdn_status s = validate_heads(Hk, Hv, dk_, dv_);
+  if (s != GDN_OK) return s;
+  if (dk_ != dv_) return GDN_ERR_UNSUPPORTED;
+  if ((long)B * Hv > 0x7fffffffL) return GDN_ERR_UNSUPPORTED;
+  const bool work = (long)B * T > 0;
+  if (work && (!q || !k || !v || !log_alpha || !beta || !dO || !dq || !dk || !dv ||
+               !dlog_alpha || !dbeta))
+    return GDN_ERR_INVALID_ARG;
+  if (!opt_aligned4(q) || !opt_aligned4(k) || !opt_aligned4(v) || !opt_aligned4(dO) ||
+      !opt_aligned4(log_alpha) || !opt_aligned4(beta) || !opt_aligned4(dq) ||
+      !opt_aligned4(dk) || !opt_aligned4(dlog_alpha) || !opt_aligned4(dbeta) ||
+      !opt_aligned16(dv) || !opt_aligned16(S0) || !opt_aligned16(dS_T) || !opt_aligned16(dS0))
+    return GDN_ERR_INVALID_ARG;
+  if (work && !workspace_ok(workspace, workspace_bytes, bwd_layout(B, T, Hk, Hv, dk_, dv_).total))
+    return GDN_ERR_INVALID_ARG;
+  if (B == 0) return GDN_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == GDN_F32)
+    return bwd_dispatch<float>(dk_, q, k, v, log_alpha, beta, S0, dO, dS_T, dq, dk, dv,
+                               dlog_alpha, dbeta, dS0, workspace, B, T, Hk, Hv, scale, st);
+  return bwd_dispatch<__nv_bfloat16>(dk_, q, k, v, log_alpha, beta, S0, dO, dS_T, dq, dk, dv,
+                                     dlog_alpha, dbeta, dS0, workspace, B, T, Hk, Hv, scale, st);
+}
 
 const char* gdn_status_string(gdn_status s) {
   switch (s) {

@@ -148,6 +148,16 @@ def make_decode_inputs(w: Workload) -> Dict[str, torch.Tensor]:
             "log_alpha": log_alpha, "beta": beta, "S0": S0.contiguous()}
 
 
+def make_output_grads(w: Workload, dst_std: float = 0.1) -> Dict[str, torch.Tensor]:
+    """The incoming gradients of a backward call on ``make_inputs(w)``: dO [B,T,Hv,dv] ~ N(0,1) in
+    the storage dtype and dS_T [B,Hv,dk,dv] ~ N(0, dst_std) fp32, from their own stream (seed + 1)
+    so that the forward inputs stay those of ``make_inputs``."""
+    g = _gen(w.seed + 1)
+    dO = torch.randn(w.B, w.T, w.Hv, w.dv, generator=g).to(w.torch_dtype)
+    dS_T = torch.randn(w.B, w.Hv, w.dk, w.dv, generator=g) * dst_std
+    return {"dO": dO.contiguous(), "dS_T": dS_T.contiguous()}
+
+
 def make_layer_inputs(w: Workload) -> Dict[str, Optional[torch.Tensor]]:
     """Inputs of one full-layer call: already-projected raw q, k, v, z, conv taps, gates, norm gain.
 

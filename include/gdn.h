@@ -248,6 +248,36 @@ GDN_API gdn_status gdn_chunk_fwd_varlen(const void *q, const void *k, const void
                                 float scale, gdn_dtype dtype, gdn_dtype o_dtype,
                                 gdn_stream_t stream);
 
+/*
+ * Backward pass: gradients of L = sum <dO, o> + <dS_T, S_T>, with o and S_T those of
+ * gdn_chunk_fwd on the same inputs, through the exact derivative of the token recurrence
+ * ("L'attention hybride", "La récurrence": S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T)
+ * + beta_t v_t k_t^T, o_t = scale S_t q_t; the pages give the layer for inference and train their
+ * models, so the backward is the chain rule through that recurrence, token by token).
+ *   q, k [B, T, Hk, dk]; v, dO [B, T, Hv, dv]            (dtype: GDN_F32 or GDN_BF16)
+ *   log_alpha, beta [B, T, Hv] float; S0, dS_T [B, Hv, dk, dv] float holding S^T (either may be
+ *        NULL: the zero state / no gradient on S_T)
+ *   dq, dk [B, T, Hk, dk] float: summed over the Hv / Hk value heads of each key head
+ *   dv [B, T, Hv, dv], dlog_alpha, dbeta [B, T, Hv] float; dS0 [B, Hv, dk, dv] float (nullable)
+ *   workspace: gdn_bwd_workspace_bytes(...) bytes, 256-byte aligned, owned by the caller (the
+ *        state every 8 tokens of every (batch, value head), and per-value-head dq, dk when key
+ *        heads are shared); NULL is accepted when that size is 0.
+ * dk == dv in {16, 32, 64, 128} (else GDN_ERR_UNSUPPORTED).  One CUDA-core kernel, one CTA per
+ * (batch, value head): a forward walk keeps the checkpoints, a reverse walk recomputes each
+ * state from the nearest of two kept states of its 8-token segment; a second launch sums dq, dk
+ * over each key head's value heads when Hv > Hk (a fixed order: the result is reproducible).
+ * Pointer alignment: 16 bytes for dv, S0, dS_T, dS0; 4 bytes for the rest.  Errors as
+ * gdn_chunk_fwd: GDN_ERR_INVALID_ARG (missing, misaligned, workspace too small) before any work.
+ */
+GDN_API gdn_status gdn_bwd(const void *q, const void *k, const void *v, const float *log_alpha,
+                   const float *beta, const float *S0, const void *dO, const float *dS_T,
+                   float *dq, float *dk, float *dv, float *dlog_alpha, float *dbeta, float *dS0,
+                   void *workspace, size_t workspace_bytes, int B, int T, int Hk, int Hv,
+                   int dk_, int dv_, float scale, gdn_dtype dtype, gdn_stream_t stream);
+
+/* Device scratch bytes gdn_bwd needs (host only, no CUDA call); 0 for invalid sizes. */
+GDN_API size_t gdn_bwd_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv);
+
 /* Device scratch bytes gdn_chunk_fwd_varlen needs (host only, no CUDA call). */
 GDN_API size_t gdn_chunk_fwd_varlen_workspace_bytes(int nseq, int max_seqlen, int Hk, int Hv,
                                             int dk, int dv, int chunk, gdn_dtype dtype);

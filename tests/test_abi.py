@@ -226,3 +226,33 @@ def test_tensor_core_forward_rejects_more_than_65535_chunks(L):
     t6 = [FAKE] * 6
     assert L.gdn_chunk_fwd_varlen(*t6, 1, longest + 1, FAKE, FAKE, FAKE, *big, longest + 1, 16,
                                   48, 128, 128, 64, 1.0, 1, 1, None) == 2
+
+
+def bwd(L, B=1, T=64, Hk=2, Hv=4, dk=64, dv=64, dtype=1, q=FAKE, dvo=FAKE, ws=None, ws_bytes=0):
+    return L.gdn_bwd(q, FAKE, FAKE, FAKE, FAKE, None, FAKE, None, FAKE, FAKE, dvo, FAKE, FAKE,
+                     None, ws, ws_bytes, B, T, Hk, Hv, dk, dv, 1.0, dtype, None)
+
+
+def test_bwd_workspace_bytes(L):
+    """A state every 8 tokens of every (batch, value head), then per-value-head dq and dk when
+    key heads are shared, each section 256-byte aligned; 0 for what the call rejects."""
+    ck = 2 * 6 * 17 * 128 * 128 * 4                  # T = 130: 17 segments of 8 tokens
+    per = 2 * 130 * 6 * 128 * 4
+    assert L.gdn_bwd_workspace_bytes(2, 130, 2, 6, 128, 128) == ck + 2 * per
+    assert L.gdn_bwd_workspace_bytes(2, 130, 2, 2, 128, 128) == 2 * 2 * 17 * 128 * 128 * 4
+    assert L.gdn_bwd_workspace_bytes(2, 130, 2, 6, 128, 64) == 0     # dk != dv
+    assert L.gdn_bwd_workspace_bytes(2, 130, 2, 6, 48, 48) == 0
+    assert L.gdn_bwd_workspace_bytes(0, 130, 2, 6, 128, 128) == 0
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(B=-1), 1), (dict(T=-1), 1), (dict(Hv=3), 1), (dict(dtype=7), 1),
+    (dict(dk=48, dv=48), 2), (dict(dk=64, dv=32), 2),
+    (dict(q=None), 1), (dict(dvo=P(0x1004)), 1),     # missing input, misaligned dv
+    (dict(), 1),                                      # no workspace
+    (dict(ws=P(0x10000), ws_bytes=100), 1),          # too small
+    (dict(B=0), 0),                                   # nothing to do
+])
+def test_bwd_validation(L, kw, expect):
+    """gdn_bwd rejects bad arguments before any work (the pointers are fakes, never read)."""
+    assert bwd(L, **kw) == expect
