@@ -46,6 +46,7 @@ struct Smem {
   float state0[DK * DV];      // the state before the segment's first token
   float statem[DK * DV];      // the state before the segment's token t0 + kHalf
   float red[2][2][Shape<DK, DV>::RG][DV];   // [parity][quantity][row group][column]
+  float col[2][2][DV];                       // [parity][quantity] the column sums
   float wsum[2][Shape<DK, DV>::NW];         // per-warp partials of <G, A>
 };
 
@@ -63,6 +64,38 @@ __device__ __forceinline__ float lane_sum(float x) {
 #pragma unroll
   for (int o = CG >> 1; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
   return x;
+}
+
+// Sums over the CG lanes of a row group of V values per lane, scattered by recursive halving:
+// at each step a lane keeps one half of its values (chosen by its lane bit), adds the partner's
+// copy of that half and passes the other half on, so V values cost V - 1 shuffles instead of
+// V log2(CG).  On return v[0] holds the total of value `idx` (every lane of the row group holds
+// the total of one value; lanes that differ only in the bits below `keep_mask` hold the same).
+template <int V, int CG>
+__device__ __forceinline__ void reduce_scatter(float (&v)[V], int lane, int& idx,
+                                               int& keep_mask) {
+  static_assert((V & (V - 1)) == 0 && V <= CG, "reduce_scatter");
+  idx = 0;
+  int n = V;
+#pragma unroll
+  for (int m = CG >> 1; m > 0; m >>= 1) {
+    if (n > 1) {
+      const bool up = (lane & m) != 0;
+#pragma unroll
+      for (int k = 0; k < V / 2; ++k) {
+        if (k < n / 2) {
+          const float lo = v[k], hi = v[k + n / 2];
+          const float keep = up ? hi : lo, send = up ? lo : hi;
+          v[k] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+      }
+      if (up) idx += n / 2;
+      n >>= 1;
+      keep_mask = m;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], m);
+    }
+  }
 }
 
 // The segment's token data (tokens t0 .. t0 + len - 1) into shared memory, as fp32.
@@ -117,18 +150,27 @@ struct Ctx {
   int par = 0;                  // reduction buffer in use (alternates, so one barrier suffices)
   __device__ Ctx(Smem<DK, DV>& s) : sm(s), cg(threadIdx.x % Sh::CG), rg(threadIdx.x / Sh::CG) {}
 
-  // Column sums over dk of two per-thread float4 partials (this thread's 4 columns).
-  __device__ __forceinline__ void colsum2(float4 a, float4 b, float4& sa, float4& sb) {
-    *reinterpret_cast<float4*>(&sm.red[par][0][rg][4 * cg]) = a;
-    *reinterpret_cast<float4*>(&sm.red[par][1][rg][4 * cg]) = b;
-    __syncthreads();
-    sa = f4(0.f);
-    sb = f4(0.f);
+  // Column sums over dk of NQ per-thread float4 partials (this thread's 4 columns): the row
+  // groups' partials go to shared memory, row group q sums quantity q's once, every thread reads
+  // the sums back.
+  template <int NQ>
+  __device__ __forceinline__ void colsum(const float4 (&a)[NQ], float4 (&s)[NQ]) {
+    static_assert(NQ <= 2 && NQ <= Sh::RG, "colsum");
 #pragma unroll
-    for (int g = 0; g < Sh::RG; ++g) {
-      sa = add4(sa, *reinterpret_cast<const float4*>(&sm.red[par][0][g][4 * cg]));
-      sb = add4(sb, *reinterpret_cast<const float4*>(&sm.red[par][1][g][4 * cg]));
+    for (int qn = 0; qn < NQ; ++qn)
+      *reinterpret_cast<float4*>(&sm.red[par][qn][rg][4 * cg]) = a[qn];
+    __syncthreads();
+    if (rg < NQ) {
+      float4 acc = f4(0.f);
+#pragma unroll
+      for (int g = 0; g < Sh::RG; ++g)
+        acc = add4(acc, *reinterpret_cast<const float4*>(&sm.red[par][rg][g][4 * cg]));
+      *reinterpret_cast<float4*>(&sm.col[par][rg][4 * cg]) = acc;
     }
+    __syncthreads();
+#pragma unroll
+    for (int qn = 0; qn < NQ; ++qn)
+      s[qn] = *reinterpret_cast<const float4*>(&sm.col[par][qn][4 * cg]);
     par ^= 1;
   }
 
@@ -142,8 +184,9 @@ struct Ctx {
       kk[r] = sm.k[j][rg + Sh::RG * r];
       x4 = fma4(M[r], f4(kk[r]), x4);
     }
-    float4 x, unused;
-    colsum2(x4, f4(0.f), x, unused);
+    float4 xa[1] = {x4}, xs[1];
+    colsum<1>(xa, xs);
+    const float4 x = xs[0];
     const float4 vv = *reinterpret_cast<const float4*>(&sm.v[j][4 * cg]);
     const float4 w = mul4(f4(be), fma4(f4(-a), x, vv));      // beta (v - alpha x)
 #pragma unroll
@@ -253,23 +296,28 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
       for (int o = 16; o > 0; o >>= 1) gp += __shfl_xor_sync(0xffffffffu, gp, o);
       if (lane == 0) sm.wsum[cx.par][warp] = gp;
       const int wpar = cx.par;
-      float4 x, Gk;
-      cx.colsum2(x4, g4, x, Gk);
+      float4 pa[2] = {x4, g4}, ps[2];
+      cx.colsum<2>(pa, ps);
+      const float4 x = ps[0], Gk = ps[1];
       const float4 u = fma4(f4(-a), x, vv);           // v - alpha x
       const float4 w = mul4(f4(be), u);                // S_t = alpha P + k w^T
       const float4 dx = mul4(f4(-a * be), Gk);
       // dq = scale S_t^T dO and dk = beta G^T (v - alpha x) + P^T dx, one value per row
       const float4 bu = mul4(f4(be), u);
+      float pv[2 * RPT];                              // dq rows, then dk rows, partial over 4 columns
 #pragma unroll
       for (int r = 0; r < RPT; ++r) {
-        float pq = dot4(fma4(f4(a), M[r], mul4(f4(kk[r]), w)), dd);
-        float pk = dot4(G[r], bu) + dot4(M[r], dx);
-        pq = lane_sum<CG>(pq);
-        pk = lane_sum<CG>(pk);
-        if (cg == 0) {
+        pv[r] = dot4(fma4(f4(a), M[r], mul4(f4(kk[r]), w)), dd);
+        pv[RPT + r] = dot4(G[r], bu) + dot4(M[r], dx);
+      }
+      {
+        int idx, keep_mask = CG;
+        reduce_scatter<2 * RPT, CG>(pv, lane, idx, keep_mask);
+        if ((lane & (keep_mask - 1)) == 0) {           // one lane per value
+          const int r = idx % RPT;
           const long o = ((b * T + t) * nqk + hq) * (long)DK + rg + RG * r;
-          dq_out[o] = scale * pq;
-          dk_out[o] = pk;
+          if (idx < RPT) dq_out[o] = scale * pv[0];
+          else dk_out[o] = pv[0];
         }
       }
       // dv, dbeta and dlog alpha from the row group 0 lanes (they hold every column once); the
