@@ -11,13 +11,15 @@
 //   dk = beta G^T (v - alpha x) + P^T dx,  and the gradient reaching S_{t-1} is alpha G + dx k^T.
 // The reverse walk needs every S_{t-1}: a forward pass first stores the state at the start of
 // every segment of kSeg tokens (checkpoints in the caller's workspace); the reverse pass then takes
-// the segments last to first, holding the segment's first state and its middle state in shared
+// the segments last to first, keeping the segment's first state and its middle state in shared
 // memory and recomputing each S_{t-1} from the nearer one (about two token steps per token).
 //
-// One CTA per (batch, value head), 512 threads.  The state and its gradient live in registers in
-// the decode kernel's layout: with M = S^T (dk x dv), thread t owns the 4 value columns of column
-// group t % (DV / 4) and the dk rows rg, rg + RG, ... (rg = t / (DV / 4)).  Reductions over dv stay
-// inside a warp (shuffles); reductions over dk cross warps (shared memory, one barrier each).
+// One CTA per (batch, value head).  Layout of the state M = S^T (dk x dv) and of its gradient:
+// the lanes of a warp take the dk rows (RL consecutive rows each), the warps the dv columns (CW
+// consecutive columns per thread).  So the sums over dk that the recurrence itself needs (S k and
+// G k) stay inside a warp (shuffles) and a token step needs no CTA barrier; the sums over dv
+// (dq, dk, dbeta, dlog alpha: outputs only) are written per column slice to shared memory and
+// added up once every kHalf tokens, in a fixed order.
 #pragma once
 
 #include "common.cuh"
@@ -28,96 +30,100 @@ namespace bwd {
 constexpr int kSeg = 8;          // tokens per checkpoint segment
 constexpr int kHalf = kSeg / 2;  // the segment's middle state is S before token t0 + kHalf
 
-template <int DK, int DV>
+template <int D>
 struct Shape {
-  static constexpr int CG = DV / 4;                                    // float4 column groups
-  static constexpr int NT = (CG * DK < 512) ? CG * DK : 512;           // threads per CTA
-  static constexpr int RG = NT / CG;                                   // row groups
-  static constexpr int RPT = DK / RG;                                  // rows per thread
-  static constexpr int NW = NT / 32;                                   // warps
-  static_assert(NT % 32 == 0 && DK % RG == 0 && 32 % CG == 0, "bwd shape");
+  static constexpr int LR = D < 32 ? D : 32;              // lanes along dk
+  static constexpr int RL = D / LR;                       // dk rows per lane
+  static constexpr int LC = 32 / LR;                      // column groups per warp
+  static constexpr int NT = D == 16 ? 128 : 512;          // threads per CTA
+  static constexpr int NW = NT / 32;
+  static constexpr int SL = NW * LC;                      // column slices
+  static constexpr int CW = D / SL;                       // dv columns per thread
+  static constexpr int VPT = RL * CW;                     // state values per thread
+  static_assert(CW >= 1 && SL * CW == D && 2 * CW <= LR && VPT % 2 == 0, "bwd shape");
 };
 
-// Shared memory of one CTA (floats): the segment's token data, two states, reduction buffers.
-template <int DK, int DV>
+template <int D>
 struct Smem {
-  float k[kSeg][DK], q[kSeg][DK], v[kSeg][DV], dO[kSeg][DV];
+  float k[kSeg][D], q[kSeg][D], v[kSeg][D], dO[kSeg][D];
   float alpha[kSeg], beta[kSeg];
-  float state0[DK * DV];      // the state before the segment's first token
-  float statem[DK * DV];      // the state before the segment's token t0 + kHalf
-  float red[2][2][Shape<DK, DV>::RG][DV];   // [parity][quantity][row group][column]
-  float col[2][2][DV];                       // [parity][quantity] the column sums
-  float wsum[2][Shape<DK, DV>::NW];         // per-warp partials of <G, A>
+  float state0[D * D];         // the state before the segment's first token (per-thread layout)
+  float statem[D * D];         // the state before the segment's token t0 + kHalf
+  float pdq[kHalf][Shape<D>::SL][D], pdk[kHalf][Shape<D>::SL][D];   // per-slice partials
+  float pa[kHalf][Shape<D>::SL], pb[kHalf][Shape<D>::SL];          // of <G, A>, dbeta
 };
 
-template <int DK, int DV>
-constexpr size_t smem_bytes() { return sizeof(Smem<DK, DV>); }
+template <int D>
+constexpr size_t smem_bytes() { return sizeof(Smem<D>); }
 
-template <int DK, int DV>
-struct Regs {
-  float4 m[Shape<DK, DV>::RPT];
-};
-
-// Sum over the CG lanes of a warp that share a row group (lanes xor 1 .. CG/2).
-template <int CG>
-__device__ __forceinline__ float lane_sum(float x) {
-#pragma unroll
-  for (int o = CG >> 1; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-  return x;
-}
-
-// Sums over the CG lanes of a row group of V values per lane, scattered by recursive halving:
-// at each step a lane keeps one half of its values (chosen by its lane bit), adds the partner's
-// copy of that half and passes the other half on, so V values cost V - 1 shuffles instead of
-// V log2(CG).  On return v[0] holds the total of value `idx` (every lane of the row group holds
-// the total of one value; lanes that differ only in the bits below `keep_mask` hold the same).
-template <int V, int CG>
-__device__ __forceinline__ void reduce_scatter(float (&v)[V], int lane, int& idx,
-                                               int& keep_mask) {
-  static_assert((V & (V - 1)) == 0 && V <= CG, "reduce_scatter");
-  idx = 0;
+// All-reduce over the LR lanes of a column group (lanes xor LR/2 .. 1) of V values per lane:
+// recursive halving (each step keeps one half, adds the partner's copy of it and passes the other
+// half on: V - 1 shuffles), then each total is fetched from the lane that holds it (V shuffles).
+template <int V, int LR>
+__device__ __forceinline__ void allreduce(float (&v)[V], int lane) {
+  static_assert((V & (V - 1)) == 0 && V <= LR, "allreduce");
   int n = V;
 #pragma unroll
-  for (int m = CG >> 1; m > 0; m >>= 1) {
+  for (int m = LR >> 1; m > 0; m >>= 1) {
     if (n > 1) {
       const bool up = (lane & m) != 0;
 #pragma unroll
-      for (int k = 0; k < V / 2; ++k) {
-        if (k < n / 2) {
-          const float lo = v[k], hi = v[k + n / 2];
-          const float keep = up ? hi : lo, send = up ? lo : hi;
-          v[k] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+      for (int kk = 0; kk < V / 2; ++kk) {
+        if (kk < n / 2) {
+          const float lo = v[kk], hi = v[kk + n / 2];
+          v[kk] = (up ? hi : lo) + __shfl_xor_sync(0xffffffffu, up ? lo : hi, m);
         }
       }
-      if (up) idx += n / 2;
       n >>= 1;
-      keep_mask = m;
     } else {
       v[0] += __shfl_xor_sync(0xffffffffu, v[0], m);
     }
   }
+  // value c sits in the lanes of this column group whose halving bits spell c
+  const float mine = v[0];
+  const int group = lane & ~(LR - 1);
+#pragma unroll
+  for (int c = 0; c < V; ++c) {
+    int src = group, half = V >> 1, m = LR >> 1;
+#pragma unroll
+    for (int s = 0; s < 5; ++s) {
+      if (half >= 1) {
+        if (c & half) src |= m;
+        half >>= 1;
+        m >>= 1;
+      }
+    }
+    v[c] = __shfl_sync(0xffffffffu, mine, src);
+  }
+}
+
+// Sum over the LR lanes of a column group.
+template <int LR>
+__device__ __forceinline__ float group_sum(float x) {
+#pragma unroll
+  for (int m = LR >> 1; m > 0; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
+  return x;
 }
 
 // The segment's token data (tokens t0 .. t0 + len - 1) into shared memory, as fp32.
-template <int DK, int DV, typename Tin>
-__device__ __forceinline__ void load_segment(Smem<DK, DV>& sm, const Tin* __restrict__ q,
+template <int D, typename Tin>
+__device__ __forceinline__ void load_segment(Smem<D>& sm, const Tin* __restrict__ q,
                                              const Tin* __restrict__ k, const Tin* __restrict__ v,
                                              const Tin* __restrict__ dO,
                                              const float* __restrict__ la,
                                              const float* __restrict__ be, long b, int h, int hk,
                                              int T, int Hk, int Hv, int t0, int len, bool with_q) {
-  constexpr int NT = Shape<DK, DV>::NT;
-  for (int e = threadIdx.x; e < len * DK; e += NT) {
-    const int j = e / DK, i = e - j * DK;
-    const long row = ((b * T + t0 + j) * Hk + hk) * (long)DK + i;
-    sm.k[j][i] = to_f(k[row]);
-    if (with_q) sm.q[j][i] = to_f(q[row]);
-  }
-  for (int e = threadIdx.x; e < len * DV; e += NT) {
-    const int j = e / DV, i = e - j * DV;
-    const long row = ((b * T + t0 + j) * Hv + h) * (long)DV + i;
-    sm.v[j][i] = to_f(v[row]);
-    if (with_q) sm.dO[j][i] = to_f(dO[row]);
+  constexpr int NT = Shape<D>::NT;
+  for (int e = threadIdx.x; e < len * D; e += NT) {
+    const int j = e / D, i = e - j * D;
+    const long rk = ((b * T + t0 + j) * Hk + hk) * (long)D + i;
+    const long rv = ((b * T + t0 + j) * Hv + h) * (long)D + i;
+    sm.k[j][i] = to_f(k[rk]);
+    sm.v[j][i] = to_f(v[rv]);
+    if (with_q) {
+      sm.q[j][i] = to_f(q[rk]);
+      sm.dO[j][i] = to_f(dO[rv]);
+    }
   }
   for (int j = threadIdx.x; j < len; j += NT) {
     const long g = (b * T + t0 + j) * Hv + h;
@@ -126,91 +132,19 @@ __device__ __forceinline__ void load_segment(Smem<DK, DV>& sm, const Tin* __rest
   }
 }
 
-__device__ __forceinline__ float4 f4(float a) { return make_float4(a, a, a, a); }
-__device__ __forceinline__ float4 add4(float4 a, float4 b) {
-  return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
-}
-__device__ __forceinline__ float4 fma4(float4 a, float4 b, float4 c) {   // a * b + c
-  return make_float4(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y), fmaf(a.z, b.z, c.z),
-                     fmaf(a.w, b.w, c.w));
-}
-__device__ __forceinline__ float4 mul4(float4 a, float4 b) {
-  return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w);
-}
-__device__ __forceinline__ float dot4(float4 a, float4 b) {
-  return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, a.w * b.w)));
-}
-
-// One CTA's state M (its RPT rows of 4 columns) and the shared-memory reductions over dk.
-template <int DK, int DV>
-struct Ctx {
-  using Sh = Shape<DK, DV>;
-  Smem<DK, DV>& sm;
-  int cg, rg;
-  int par = 0;                  // reduction buffer in use (alternates, so one barrier suffices)
-  __device__ Ctx(Smem<DK, DV>& s) : sm(s), cg(threadIdx.x % Sh::CG), rg(threadIdx.x / Sh::CG) {}
-
-  // Column sums over dk of NQ per-thread float4 partials (this thread's 4 columns): the row
-  // groups' partials go to shared memory, row group q sums quantity q's once, every thread reads
-  // the sums back.
-  template <int NQ>
-  __device__ __forceinline__ void colsum(const float4 (&a)[NQ], float4 (&s)[NQ]) {
-    static_assert(NQ <= 2 && NQ <= Sh::RG, "colsum");
-#pragma unroll
-    for (int qn = 0; qn < NQ; ++qn)
-      *reinterpret_cast<float4*>(&sm.red[par][qn][rg][4 * cg]) = a[qn];
-    __syncthreads();
-    if (rg < NQ) {
-      float4 acc = f4(0.f);
-#pragma unroll
-      for (int g = 0; g < Sh::RG; ++g)
-        acc = add4(acc, *reinterpret_cast<const float4*>(&sm.red[par][rg][g][4 * cg]));
-      *reinterpret_cast<float4*>(&sm.col[par][rg][4 * cg]) = acc;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int qn = 0; qn < NQ; ++qn)
-      s[qn] = *reinterpret_cast<const float4*>(&sm.col[par][qn][4 * cg]);
-    par ^= 1;
-  }
-
-  // One token of the recurrence on M = S^T: x = S k, S <- alpha S + beta (v - alpha x) k^T.
-  __device__ __forceinline__ void fwd_step(float4 (&M)[Sh::RPT], int j) {
-    const float a = sm.alpha[j], be = sm.beta[j];
-    float kk[Sh::RPT];
-    float4 x4 = f4(0.f);
-#pragma unroll
-    for (int r = 0; r < Sh::RPT; ++r) {
-      kk[r] = sm.k[j][rg + Sh::RG * r];
-      x4 = fma4(M[r], f4(kk[r]), x4);
-    }
-    float4 xa[1] = {x4}, xs[1];
-    colsum<1>(xa, xs);
-    const float4 x = xs[0];
-    const float4 vv = *reinterpret_cast<const float4*>(&sm.v[j][4 * cg]);
-    const float4 w = mul4(f4(be), fma4(f4(-a), x, vv));      // beta (v - alpha x)
-#pragma unroll
-    for (int r = 0; r < Sh::RPT; ++r) M[r] = fma4(f4(a), M[r], mul4(f4(kk[r]), w));
-  }
-
-  __device__ __forceinline__ void put(float* base, const float4 (&M)[Sh::RPT]) const {
-#pragma unroll
-    for (int r = 0; r < Sh::RPT; ++r)
-      *reinterpret_cast<float4*>(base + (long)(rg + Sh::RG * r) * DV + 4 * cg) = M[r];
-  }
-  __device__ __forceinline__ void get(const float* base, float4 (&M)[Sh::RPT]) const {
-#pragma unroll
-    for (int r = 0; r < Sh::RPT; ++r)
-      M[r] = *reinterpret_cast<const float4*>(base + (long)(rg + Sh::RG * r) * DV + 4 * cg);
-  }
+// One thread's share of a state: rows i0 .. i0 + RL - 1, columns j0 .. j0 + CW - 1.
+template <int D>
+struct Tile {
+  using Sh = Shape<D>;
+  float m[Sh::RL][Sh::CW];
 };
 
-// grid: B * Hv CTAs (b * Hv + h); block Shape::NT; dynamic shared memory smem_bytes<DK, DV>().
-// dq_out, dk_out: [B, T, nqk, DK] with nqk = Hv (one slice per value head, summed afterwards by
+// grid: B * Hv CTAs (b * Hv + h); block Shape<D>::NT; dynamic shared memory smem_bytes<D>().
+// dq_out, dk_out: [B, T, nqk, D] with nqk = Hv (one slice per value head, summed afterwards by
 // group_sum_kernel) or Hk when each key head has one value head.  ckpt: B * Hv * ceil(T / kSeg)
-// states of DK * DV floats.
-template <int DK, int DV, typename Tin>
-__global__ void __launch_bounds__(Shape<DK, DV>::NT, 1)
+// states of D * D floats, each in the CTA's own per-thread order.
+template <int D, typename Tin>
+__global__ void __launch_bounds__(Shape<D>::NT, 1)
 bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
            const float* __restrict__ log_alpha, const float* __restrict__ beta,
            const float* __restrict__ S0, const Tin* __restrict__ dO,
@@ -218,129 +152,196 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
            float* __restrict__ dk_out, int nqk, float* __restrict__ dv_out,
            float* __restrict__ dla_out, float* __restrict__ dbeta_out, float* __restrict__ dS0,
            float* __restrict__ ckpt, int T, int Hk, int Hv, float scale) {
-  using Sh = Shape<DK, DV>;
-  constexpr int RPT = Sh::RPT, RG = Sh::RG, CG = Sh::CG;
+  using Sh = Shape<D>;
+  constexpr int RL = Sh::RL, CW = Sh::CW, LR = Sh::LR, NT = Sh::NT, SL = Sh::SL, VPT = Sh::VPT;
   extern __shared__ __align__(16) unsigned char bwd_smem[];
-  Smem<DK, DV>& sm = *reinterpret_cast<Smem<DK, DV>*>(bwd_smem);
-  Ctx<DK, DV> cx(sm);
-  const int cg = cx.cg, rg = cx.rg, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  Smem<D>& sm = *reinterpret_cast<Smem<D>*>(bwd_smem);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int lr = lane % LR, sl = warp * Sh::LC + lane / LR;   // row lane, column slice
+  const int i0 = lr * RL, j0 = sl * CW;
   const long bh = blockIdx.x;
   const int h = (int)(bh % Hv);
   const long b = bh / Hv;
   const int hk = h / (Hv / Hk);
   const int hq = nqk == Hv ? h : hk;                 // this CTA's slice of dq, dk
   const int nseg = (T + kSeg - 1) / kSeg;
-  float* const ck = ckpt + bh * (long)nseg * DK * DV;
-  const long sbase = bh * (long)DK * DV;             // [dk][dv] slot of S0, dS_T, dS0
+  float* const ck = ckpt + bh * (long)nseg * D * D;
+  const long sbase = bh * (long)D * D;               // [dk][dv] slot of S0, dS_T, dS0
+
+  // a state in the [dk][dv] order of S0 / dS_T / dS0, and in the per-thread order of the
+  // checkpoints and the shared-memory copies (element e of thread t at e * NT + t)
+  auto get_sq = [&](const float* base, Tile<D>& M) {
+#pragma unroll
+    for (int r = 0; r < RL; ++r)
+#pragma unroll
+      for (int c = 0; c < CW; ++c) M.m[r][c] = base[(long)(i0 + r) * D + j0 + c];
+  };
+  auto put_sq = [&](float* base, const Tile<D>& M) {
+#pragma unroll
+    for (int r = 0; r < RL; ++r)
+#pragma unroll
+      for (int c = 0; c < CW; ++c) base[(long)(i0 + r) * D + j0 + c] = M.m[r][c];
+  };
+  auto get_pt = [&](const float* base, Tile<D>& M) {
+#pragma unroll
+    for (int e = 0; e < VPT; ++e) M.m[e / CW][e % CW] = base[(long)e * NT + tid];
+  };
+  auto put_pt = [&](float* base, const Tile<D>& M) {
+#pragma unroll
+    for (int e = 0; e < VPT; ++e) base[(long)e * NT + tid] = M.m[e / CW][e % CW];
+  };
+  // one token of the recurrence: x = S k (inside the warp), S <- alpha S + k (beta (v - alpha x))^T
+  auto fwd_step = [&](Tile<D>& M, int j) {
+    const float a = sm.alpha[j], be = sm.beta[j];
+    float kk[RL], x[CW];
+#pragma unroll
+    for (int r = 0; r < RL; ++r) kk[r] = sm.k[j][i0 + r];
+#pragma unroll
+    for (int c = 0; c < CW; ++c) {
+      float acc = 0.f;
+#pragma unroll
+      for (int r = 0; r < RL; ++r) acc = fmaf(M.m[r][c], kk[r], acc);
+      x[c] = acc;
+    }
+    allreduce<CW, LR>(x, lane);
+#pragma unroll
+    for (int c = 0; c < CW; ++c) {
+      const float w = be * fmaf(-a, x[c], sm.v[j][j0 + c]);
+#pragma unroll
+      for (int r = 0; r < RL; ++r) M.m[r][c] = fmaf(a, M.m[r][c], kk[r] * w);
+    }
+  };
 
   // pass 1: the recurrence forward, the state before every segment kept
-  float4 M[RPT], G[RPT];
-  if (S0) cx.get(S0 + sbase, M);
+  Tile<D> M, G;
+  if (S0) get_sq(S0 + sbase, M);
   else
 #pragma unroll
-    for (int r = 0; r < RPT; ++r) M[r] = f4(0.f);
+    for (int e = 0; e < VPT; ++e) M.m[e / CW][e % CW] = 0.f;
   for (int sg = 0; sg < nseg; ++sg) {
     const int t0 = sg * kSeg, len = min(kSeg, T - t0);
     __syncthreads();                                 // the previous segment's data is read
     load_segment(sm, q, k, v, dO, log_alpha, beta, b, h, hk, T, Hk, Hv, t0, len, false);
-    cx.put(ck + (long)sg * DK * DV, M);
+    put_pt(ck + (long)sg * D * D, M);
     __syncthreads();
-    for (int j = 0; j < len; ++j) cx.fwd_step(M, j);
+    for (int j = 0; j < len; ++j) fwd_step(M, j);
   }
 
   // pass 2: segments last to first, tokens last to first
-  if (dS_T) cx.get(dS_T + sbase, G);
+  if (dS_T) get_sq(dS_T + sbase, G);
   else
 #pragma unroll
-    for (int r = 0; r < RPT; ++r) G[r] = f4(0.f);
-  float* const st0 = sm.state0;
-  float* const stm = sm.statem;
+    for (int e = 0; e < VPT; ++e) G.m[e / CW][e % CW] = 0.f;
+  // the per-slice partials of tokens t0 + jb .. t0 + je - 1, summed into the outputs
+  auto flush = [&](int t0, int jb, int je) {
+    __syncthreads();
+    const int n = je - jb, per = 2 * D + 2;
+    for (int e = tid; e < n * per; e += NT) {
+      const int jj = e / per, f = e - jj * per, j = jb + jj, hj = j % kHalf;
+      const long t = t0 + j;
+      float acc = 0.f;
+      if (f < 2 * D) {
+        const int i = f % D;
+#pragma unroll 4
+        for (int s2 = 0; s2 < SL; ++s2) acc += f < D ? sm.pdq[hj][s2][i] : sm.pdk[hj][s2][i];
+        float* dst = f < D ? dq_out : dk_out;
+        dst[((b * T + t) * nqk + hq) * (long)D + i] = acc;
+      } else {
+        const bool isa = f == 2 * D;
+#pragma unroll 4
+        for (int s2 = 0; s2 < SL; ++s2) acc += isa ? sm.pa[hj][s2] : sm.pb[hj][s2];
+        const long g = (b * T + t) * Hv + h;
+        if (isa) dla_out[g] = sm.alpha[j] * acc;       // alpha <G, P - beta x k^T>
+        else dbeta_out[g] = acc;                       // (v - alpha x)^T Gk
+      }
+    }
+    __syncthreads();
+  };
   for (int sg = nseg - 1; sg >= 0; --sg) {
     const int t0 = sg * kSeg, len = min(kSeg, T - t0);
     __syncthreads();
     load_segment(sm, q, k, v, dO, log_alpha, beta, b, h, hk, T, Hk, Hv, t0, len, true);
-    cx.get(ck + (long)sg * DK * DV, M);              // this thread's own elements only
-    cx.put(st0, M);
+    get_pt(ck + (long)sg * D * D, M);                // this thread's own elements
+    put_pt(sm.state0, M);
     __syncthreads();
     if (len > kHalf) {
-      for (int j = 0; j < kHalf; ++j) cx.fwd_step(M, j);
-      cx.put(stm, M);
+      for (int j = 0; j < kHalf; ++j) fwd_step(M, j);
+      put_pt(sm.statem, M);
     }
     for (int j = len - 1; j >= 0; --j) {
       // P = S before token t0 + j, from the nearer kept state
-      int j0;
-      if (j >= kHalf) { cx.get(stm, M); j0 = kHalf; }
-      else { cx.get(st0, M); j0 = 0; }
-      for (int u = j0; u < j; ++u) cx.fwd_step(M, u);
-      const long t = t0 + j;
+      int j0s;
+      if (j >= kHalf) { get_pt(sm.statem, M); j0s = kHalf; }
+      else { get_pt(sm.state0, M); j0s = 0; }
+      for (int u = j0s; u < j; ++u) fwd_step(M, u);
       const float a = sm.alpha[j], be = sm.beta[j];
-      float kk[RPT], qs[RPT];
+      float kk[RL], qs[RL], vv[CW], dd[CW], xg[2 * CW];
 #pragma unroll
-      for (int r = 0; r < RPT; ++r) {
-        kk[r] = sm.k[j][rg + RG * r];
-        qs[r] = scale * sm.q[j][rg + RG * r];
+      for (int r = 0; r < RL; ++r) {
+        kk[r] = sm.k[j][i0 + r];
+        qs[r] = scale * sm.q[j][i0 + r];
       }
-      const float4 vv = *reinterpret_cast<const float4*>(&sm.v[j][4 * cg]);
-      const float4 dd = *reinterpret_cast<const float4*>(&sm.dO[j][4 * cg]);
-      // G += scale dO q^T; partials of x = P k, Gk = G k and <G, P>
-      float4 x4 = f4(0.f), g4 = f4(0.f);
+#pragma unroll
+      for (int c = 0; c < CW; ++c) {
+        vv[c] = sm.v[j][j0 + c];
+        dd[c] = sm.dO[j][j0 + c];
+      }
+      // G += scale dO q^T; x = P k and Gk = G k (sums over dk, in the warp); <G, P> partial
       float gp = 0.f;
 #pragma unroll
-      for (int r = 0; r < RPT; ++r) {
-        G[r] = fma4(f4(qs[r]), dd, G[r]);
-        x4 = fma4(M[r], f4(kk[r]), x4);
-        g4 = fma4(G[r], f4(kk[r]), g4);
-        gp += dot4(G[r], M[r]);
-      }
+      for (int c = 0; c < CW; ++c) {
+        float ax = 0.f, ag = 0.f;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) gp += __shfl_xor_sync(0xffffffffu, gp, o);
-      if (lane == 0) sm.wsum[cx.par][warp] = gp;
-      const int wpar = cx.par;
-      float4 pa[2] = {x4, g4}, ps[2];
-      cx.colsum<2>(pa, ps);
-      const float4 x = ps[0], Gk = ps[1];
-      const float4 u = fma4(f4(-a), x, vv);           // v - alpha x
-      const float4 w = mul4(f4(be), u);                // S_t = alpha P + k w^T
-      const float4 dx = mul4(f4(-a * be), Gk);
-      // dq = scale S_t^T dO and dk = beta G^T (v - alpha x) + P^T dx, one value per row
-      const float4 bu = mul4(f4(be), u);
-      float pv[2 * RPT];                              // dq rows, then dk rows, partial over 4 columns
-#pragma unroll
-      for (int r = 0; r < RPT; ++r) {
-        pv[r] = dot4(fma4(f4(a), M[r], mul4(f4(kk[r]), w)), dd);
-        pv[RPT + r] = dot4(G[r], bu) + dot4(M[r], dx);
-      }
-      {
-        int idx, keep_mask = CG;
-        reduce_scatter<2 * RPT, CG>(pv, lane, idx, keep_mask);
-        if ((lane & (keep_mask - 1)) == 0) {           // one lane per value
-          const int r = idx % RPT;
-          const long o = ((b * T + t) * nqk + hq) * (long)DK + rg + RG * r;
-          if (idx < RPT) dq_out[o] = scale * pv[0];
-          else dk_out[o] = pv[0];
+        for (int r = 0; r < RL; ++r) {
+          G.m[r][c] = fmaf(qs[r], dd[c], G.m[r][c]);
+          ax = fmaf(M.m[r][c], kk[r], ax);
+          ag = fmaf(G.m[r][c], kk[r], ag);
+          gp = fmaf(G.m[r][c], M.m[r][c], gp);
         }
+        xg[c] = ax;
+        xg[CW + c] = ag;
       }
-      // dv, dbeta and dlog alpha from the row group 0 lanes (they hold every column once); the
-      // sums over the columns run in every warp, so that all lanes take part in the shuffles
-      const float vg = lane_sum<CG>(dot4(u, Gk)), xg = lane_sum<CG>(dot4(x, Gk));
-      if (rg == 0) {
-        *reinterpret_cast<float4*>(dv_out + ((b * T + t) * Hv + h) * (long)DV + 4 * cg) =
-            mul4(f4(be), Gk);
-        if (tid == 0) {
-          float gsum = 0.f;
+      allreduce<2 * CW, LR>(xg, lane);
+      gp = group_sum<LR>(gp);
+      float u[CW], w[CW], dx[CW], ug = 0.f, xgk = 0.f;
 #pragma unroll
-          for (int w8 = 0; w8 < Sh::NW; ++w8) gsum += sm.wsum[wpar][w8];
-          const long g = (b * T + t) * Hv + h;
-          dbeta_out[g] = vg;                         // (v - alpha x)^T Gk
-          dla_out[g] = a * (gsum - be * xg);          // alpha <G, P - beta x k^T>
+      for (int c = 0; c < CW; ++c) {
+        u[c] = fmaf(-a, xg[c], vv[c]);                 // v - alpha x
+        w[c] = be * u[c];                              // S_t = alpha P + k w^T
+        dx[c] = -a * be * xg[CW + c];
+        ug = fmaf(u[c], xg[CW + c], ug);
+        xgk = fmaf(xg[c], xg[CW + c], xgk);
+      }
+      // per-slice partials: dq = scale S_t^T dO, dk = beta G^T (v - alpha x) + P^T dx
+      const int hj = j % kHalf;
+#pragma unroll
+      for (int r = 0; r < RL; ++r) {
+        float pq = 0.f, pk = 0.f;
+#pragma unroll
+        for (int c = 0; c < CW; ++c) {
+          pq = fmaf(fmaf(a, M.m[r][c], kk[r] * w[c]), dd[c], pq);
+          pk = fmaf(G.m[r][c], w[c], fmaf(M.m[r][c], dx[c], pk));   // beta G u = G w
         }
+        sm.pdq[hj][sl][i0 + r] = scale * pq;
+        sm.pdk[hj][sl][i0 + r] = pk;
+      }
+      if (lr == 0) {
+        sm.pa[hj][sl] = gp - be * xgk;                // this slice's <G, P - beta x k^T>
+        sm.pb[hj][sl] = ug;
+#pragma unroll
+        for (int c = 0; c < CW; ++c)
+          dv_out[((b * T + t0 + j) * Hv + h) * (long)D + j0 + c] = be * xg[CW + c];
       }
       // the gradient reaching S_{t-1}: alpha G + dx k^T
 #pragma unroll
-      for (int r = 0; r < RPT; ++r) G[r] = fma4(f4(a), G[r], mul4(f4(kk[r]), dx));
+      for (int c = 0; c < CW; ++c)
+#pragma unroll
+        for (int r = 0; r < RL; ++r) G.m[r][c] = fmaf(a, G.m[r][c], kk[r] * dx[c]);
+      if (j == kHalf) flush(t0, kHalf, len);
+      if (j == 0) flush(t0, 0, min(len, kHalf));
     }
   }
-  if (dS0) cx.put(dS0 + sbase, G);
+  if (dS0) put_sq(dS0 + sbase, G);
 }
 
 // dst [rows, D] = sum over g < G of src [rows * G + g, D] (the value heads of each key head).

@@ -234,8 +234,8 @@ gdn_status bwd_launch(const void* q, const void* k, const void* v, const float* 
                       const float* be, const float* S0, const void* dO, const float* dST,
                       float* dq, float* dk, float* dv, float* dla, float* dbeta, float* dS0,
                       void* ws, int B, int T, int Hk, int Hv, float scale, cudaStream_t st) {
-  auto kern = bwd::bwd_kernel<D, D, Tin>;
-  const size_t smem = bwd::smem_bytes<D, D>();
+  auto kern = bwd::bwd_kernel<D, Tin>;
+  const size_t smem = bwd::smem_bytes<D>();
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return GDN_ERR_CUDA;
@@ -244,7 +244,7 @@ gdn_status bwd_launch(const void* q, const void* k, const void* v, const float* 
   const bool grouped = Hv != Hk;
   float* dqo = grouped ? reinterpret_cast<float*>(w + L.dqh) : dq;
   float* dko = grouped ? reinterpret_cast<float*>(w + L.dkh) : dk;
-  kern<<<(unsigned)((long)B * Hv), bwd::Shape<D, D>::NT, smem, st>>>(
+  kern<<<(unsigned)((long)B * Hv), bwd::Shape<D>::NT, smem, st>>>(
       static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v), la, be,
       S0, static_cast<const Tin*>(dO), dST, dqo, dko, grouped ? Hv : Hk, dv, dla, dbeta, dS0,
       reinterpret_cast<float*>(w), T, Hk, Hv, scale);
