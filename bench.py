@@ -62,6 +62,19 @@ def fwd_flops(w: gi.Workload) -> float:
     return float(w.B * w.T * w.Hv * per)
 
 
+def bwd_flops(w: gi.Workload) -> float:
+    """Work of the backward per token and value head: 10 dk dv fused multiply-adds, i.e. the
+    reverse step's eight products with the state or its gradient (the output's rank-1 term, S k,
+    G k, <G, P>, dq, the two terms of dk, the decay of G) and one forward step (S k, the update)."""
+    return float(w.B * w.T * w.Hv * 20 * w.dk * w.dv)
+
+
+def fp32_peak_tflops(dev) -> float:
+    """fp32 FMA peak: SMs x 128 FP32 lanes x 2 flops x 1965 MHz (the part's maximum SM clock)."""
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    return sms * 128 * 2 * 1.965e9 / 1e12
+
+
 def decode_bytes(w: gi.Workload) -> int:
     s = 2 if w.dtype == "bf16" else 4
     N = w.B
@@ -399,6 +412,31 @@ def bench_gates(gdn, dev, warmup, flush, peaks, steps=20):
             "workload": f"gates B{w.B} T{w.T} Hv{w.Hv} {w.dtype}"}
 
 
+def bench_backward(gdn, dev, warmup, flush, steps=5):
+    """The backward pass (gdn_bwd) on the prefill workload, dO ~ N(0, 1), dS_T ~ N(0, 0.1)."""
+    w = gi.WORKLOADS["prefill"]
+    x, gr = gi.make_inputs(w), gi.make_output_grads(w)
+    d = to_dev({**x, **gr}, dev)
+    ws = torch.empty(max(gdn.bwd_workspace_bytes(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv), 1),
+                     device=dev, dtype=torch.uint8)
+
+    def step():
+        gdn.bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"], d["dO"], d["dS_T"],
+                workspace=ws)
+    launches = 1 + (1 if w.Hv != w.Hk else 0)
+    ms = time_steps(step, steps, warmup, flush, launches)
+    t = statistics.mean(ms) / 1e3
+    F = bwd_flops(w)
+    peak = fp32_peak_tflops(dev)
+    return {"value": w.B * w.T / t, "unit": "tokens/s", "ms_per_step": t * 1e3, "steps": steps,
+            "roofline": {"bound": "alu", "achieved": F / t / 1e12, "peak": peak,
+                         "unit": "TFLOP/s", "frac": F / t / 1e12 / peak, "traffic": None,
+                         "kernel": "bwd_kernel", "algorithmic_flops": F,
+                         "peak_source": "derived: SMs x 128 fp32 lanes x 2 x 1965 MHz"},
+            "workspace_bytes": ws.numel(), "gpu_launches_per_call": launches,
+            "workload": "backward " + workload_name(w)}
+
+
 def bench_layer(gdn, dev, warmup, flush, peaks, steps=10):
     w = gi.WORKLOADS["layer_8to1"]
     x = gi.make_layer_inputs(w)
@@ -633,7 +671,7 @@ def profile_case(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     name = args.profile_case
-    w = gi.WORKLOADS[name]
+    w = gi.WORKLOADS["prefill" if name == "backward" else name]
     kw = {k: v for k, v in (("B", args.B), ("T", args.T)) if v is not None}
     if kw:
         w = w.with_sizes(**kw)
@@ -647,6 +685,13 @@ def profile_case(args):
                           d["conv_wv"], d["log_alpha"], d["beta"], d["S0"], d["norm_w"],
                           Hk=w.Hk, Hv=w.Hv, dk=w.dk, dv=w.dv, chunk=w.chunk, workspace=ws)
         launches = 3 + launches_per_call(gdn, w)   # prologue (q/k, v), forward, gated norm
+    elif name == "backward":
+        d = to_dev({**gi.make_inputs(w), **gi.make_output_grads(w)}, dev)
+
+        def step():
+            gdn.bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"], d["dO"],
+                    d["dS_T"])
+        launches = 1 + (1 if w.Hv != w.Hk else 0)
     elif name in ("decode", "decode_layer"):
         mk = gi.make_decode_inputs if name == "decode" else gi.make_decode_layer_inputs
         d = to_dev(mk(w.with_sizes(steps=1)), dev)
@@ -769,6 +814,8 @@ def main():
             del xl, dl
             torch.cuda.empty_cache()
             sec["layer_8to1"] = bench_layer(gdn, dev, 3, flush, peaks, steps=10)
+            torch.cuda.empty_cache()
+            sec["backward"] = bench_backward(gdn, dev, 3, flush, steps=5)
             line["secondary"] = sec
         if not args.no_cpu_baseline and world == 1:
             cb = oracle_sample_rate(x, w, target_s=10.0)

@@ -169,7 +169,7 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
   const long sbase = bh * (long)D * D;               // [dk][dv] slot of S0, dS_T, dS0
 
   // a state in the [dk][dv] order of S0 / dS_T / dS0, and in the per-thread order of the
-  // checkpoints and the shared-memory copies (element e of thread t at e * NT + t)
+  // checkpoints and the shared-memory copies
   auto get_sq = [&](const float* base, Tile<D>& M) {
 #pragma unroll
     for (int r = 0; r < RL; ++r)
@@ -182,13 +182,20 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
 #pragma unroll
       for (int c = 0; c < CW; ++c) base[(long)(i0 + r) * D + j0 + c] = M.m[r][c];
   };
+  // (pairs of elements: element 2e, 2e + 1 of thread t at (e * NT + t) * 2, one 8-byte access)
   auto get_pt = [&](const float* base, Tile<D>& M) {
 #pragma unroll
-    for (int e = 0; e < VPT; ++e) M.m[e / CW][e % CW] = base[(long)e * NT + tid];
+    for (int e = 0; e < VPT / 2; ++e) {
+      const float2 p = *reinterpret_cast<const float2*>(base + ((long)e * NT + tid) * 2);
+      M.m[(2 * e) / CW][(2 * e) % CW] = p.x;
+      M.m[(2 * e + 1) / CW][(2 * e + 1) % CW] = p.y;
+    }
   };
   auto put_pt = [&](float* base, const Tile<D>& M) {
 #pragma unroll
-    for (int e = 0; e < VPT; ++e) base[(long)e * NT + tid] = M.m[e / CW][e % CW];
+    for (int e = 0; e < VPT / 2; ++e)
+      *reinterpret_cast<float2*>(base + ((long)e * NT + tid) * 2) =
+          make_float2(M.m[(2 * e) / CW][(2 * e) % CW], M.m[(2 * e + 1) / CW][(2 * e + 1) % CW]);
   };
   // one token of the recurrence: x = S k (inside the warp), S <- alpha S + k (beta (v - alpha x))^T
   auto fwd_step = [&](Tile<D>& M, int j) {
