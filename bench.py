@@ -109,7 +109,8 @@ def load_peaks():
 # The source files whose kernels (and launch schedule) a recorded traffic figure depends on.
 TRAFFIC_SOURCES = {
     "gdn_chunk_fwd_tc": ("common.cuh", "tc_chunk.cuh", "tc_ptx.cuh"),
-    "gdn_layer_fwd": None,                     # every file of csrc/
+    "gdn_layer_fwd": ("common.cuh", "elementwise.cuh", "gdn_api.cu", "tc_chunk.cuh",
+                      "tc_ptx.cuh"),
 }
 
 
