@@ -30,25 +30,34 @@ namespace bwd {
 constexpr int kSeg = 8;          // tokens per checkpoint segment
 constexpr int kHalf = kSeg / 2;  // the segment's middle state is S before token t0 + kHalf
 
+// A head's dv columns are split over NS CTAs (the recurrence never mixes columns: S k, G k and
+// every update act column by column; only the outputs sum over columns, and those partial sums
+// are added afterwards), so that small batches still fill the GPU and several CTAs share an SM.
+__host__ __device__ constexpr int head_slices(int D) { return D == 128 ? 4 : (D == 64 ? 2 : 1); }
+
 template <int D>
 struct Shape {
+  static constexpr int NS = head_slices(D);               // CTAs per head
+  static constexpr int DC = D / NS;                       // dv columns per CTA
   static constexpr int LR = D < 32 ? D : 32;              // lanes along dk
   static constexpr int RL = D / LR;                       // dk rows per lane
   static constexpr int LC = 32 / LR;                      // column groups per warp
-  static constexpr int NT = D == 16 ? 128 : 512;          // threads per CTA
+  static constexpr int NT = D == 128 ? 128 : (D == 64 ? 256 : (D == 32 ? 512 : 128));
   static constexpr int NW = NT / 32;
-  static constexpr int SL = NW * LC;                      // column slices
-  static constexpr int CW = D / SL;                       // dv columns per thread
+  static constexpr int SL = NW * LC;                      // column slices of the CTA
+  static constexpr int CW = DC / SL;                      // dv columns per thread
   static constexpr int VPT = RL * CW;                     // state values per thread
-  static_assert(CW >= 1 && SL * CW == D && 2 * CW <= LR && VPT % 2 == 0, "bwd shape");
+  static constexpr int MINB = D == 128 ? 3 : (D == 64 ? 2 : 1);   // CTAs per SM to fit
+  static_assert(CW >= 1 && SL * CW == DC && 2 * CW <= LR && VPT % 2 == 0, "bwd shape");
 };
 
 template <int D>
 struct Smem {
-  float k[kSeg][D], q[kSeg][D], v[kSeg][D], dO[kSeg][D];
+  static constexpr int DC = Shape<D>::DC;
+  float k[kSeg][D], q[kSeg][D], v[kSeg][DC], dO[kSeg][DC];
   float alpha[kSeg], beta[kSeg];
-  float state0[D * D];         // the state before the segment's first token (per-thread layout)
-  float statem[D * D];         // the state before the segment's token t0 + kHalf
+  float state0[D * DC];        // the state before the segment's first token (per-thread layout)
+  float statem[D * DC];        // the state before the segment's token t0 + kHalf
   float pdq[kHalf][Shape<D>::SL][D], pdk[kHalf][Shape<D>::SL][D];   // per-slice partials
   float pa[kHalf][Shape<D>::SL], pb[kHalf][Shape<D>::SL];          // of <G, A>, dbeta
 };
@@ -112,18 +121,20 @@ __device__ __forceinline__ void load_segment(Smem<D>& sm, const Tin* __restrict_
                                              const Tin* __restrict__ dO,
                                              const float* __restrict__ la,
                                              const float* __restrict__ be, long b, int h, int hk,
-                                             int T, int Hk, int Hv, int t0, int len, bool with_q) {
-  constexpr int NT = Shape<D>::NT;
+                                             int c0, int T, int Hk, int Hv, int t0, int len,
+                                             bool with_q) {
+  constexpr int NT = Shape<D>::NT, DC = Shape<D>::DC;
   for (int e = threadIdx.x; e < len * D; e += NT) {
     const int j = e / D, i = e - j * D;
     const long rk = ((b * T + t0 + j) * Hk + hk) * (long)D + i;
-    const long rv = ((b * T + t0 + j) * Hv + h) * (long)D + i;
     sm.k[j][i] = to_f(k[rk]);
+    if (with_q) sm.q[j][i] = to_f(q[rk]);
+  }
+  for (int e = threadIdx.x; e < len * DC; e += NT) {      // this CTA's columns c0 .. c0 + DC - 1
+    const int j = e / DC, i = e - j * DC;
+    const long rv = ((b * T + t0 + j) * Hv + h) * (long)D + c0 + i;
     sm.v[j][i] = to_f(v[rv]);
-    if (with_q) {
-      sm.q[j][i] = to_f(q[rk]);
-      sm.dO[j][i] = to_f(dO[rv]);
-    }
+    if (with_q) sm.dO[j][i] = to_f(dO[rv]);
   }
   for (int j = threadIdx.x; j < len; j += NT) {
     const long g = (b * T + t0 + j) * Hv + h;
@@ -139,33 +150,37 @@ struct Tile {
   float m[Sh::RL][Sh::CW];
 };
 
-// grid: B * Hv CTAs (b * Hv + h); block Shape<D>::NT; dynamic shared memory smem_bytes<D>().
-// dq_out, dk_out: [B, T, nqk, D] with nqk = Hv (one slice per value head, summed afterwards by
-// group_sum_kernel) or Hk when each key head has one value head.  ckpt: B * Hv * ceil(T / kSeg)
-// states of D * D floats, each in the CTA's own per-thread order.
+// grid: B * Hv * NS CTAs ((b * Hv + h) * NS + column slice); block Shape<D>::NT; dynamic shared
+// memory smem_bytes<D>().  direct (one value head per key head and one slice per head): dq_out,
+// dk_out are [B, T, Hk, D] and dla_out, dbeta_out [B, T, Hv]; otherwise they are the per-slice
+// partials [B, T, Hv * NS, D] and [B, T, Hv, NS], summed afterwards by group_sum_kernel.  ckpt:
+// B * Hv * NS * ceil(T / kSeg) slices of D * DC floats, each in the CTA's own per-thread order.
 template <int D, typename Tin>
-__global__ void __launch_bounds__(Shape<D>::NT, 1)
+__global__ void __launch_bounds__(Shape<D>::NT, Shape<D>::MINB)
 bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
            const float* __restrict__ log_alpha, const float* __restrict__ beta,
            const float* __restrict__ S0, const Tin* __restrict__ dO,
            const float* __restrict__ dS_T, float* __restrict__ dq_out,
-           float* __restrict__ dk_out, int nqk, float* __restrict__ dv_out,
+           float* __restrict__ dk_out, int direct, float* __restrict__ dv_out,
            float* __restrict__ dla_out, float* __restrict__ dbeta_out, float* __restrict__ dS0,
            float* __restrict__ ckpt, int T, int Hk, int Hv, float scale) {
   using Sh = Shape<D>;
   constexpr int RL = Sh::RL, CW = Sh::CW, LR = Sh::LR, NT = Sh::NT, SL = Sh::SL, VPT = Sh::VPT;
+  constexpr int NS = Sh::NS, DC = Sh::DC;
   extern __shared__ __align__(16) unsigned char bwd_smem[];
   Smem<D>& sm = *reinterpret_cast<Smem<D>*>(bwd_smem);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int lr = lane % LR, sl = warp * Sh::LC + lane / LR;   // row lane, column slice
-  const int i0 = lr * RL, j0 = sl * CW;
-  const long bh = blockIdx.x;
+  const long bh = blockIdx.x / NS;
+  const int ns = blockIdx.x % NS, c0 = ns * DC;      // this CTA's columns c0 .. c0 + DC - 1
+  const int i0 = lr * RL, jl = sl * CW, j0 = c0 + jl;   // rows; columns (local, of the head)
   const int h = (int)(bh % Hv);
   const long b = bh / Hv;
   const int hk = h / (Hv / Hk);
-  const int hq = nqk == Hv ? h : hk;                 // this CTA's slice of dq, dk
+  const int nqk = direct ? Hk : Hv * NS, hq = direct ? hk : h * NS + ns;   // dq, dk slot
+  const int nab = direct ? 1 : NS, hab = direct ? 0 : ns;                 // dla, dbeta slot
   const int nseg = (T + kSeg - 1) / kSeg;
-  float* const ck = ckpt + bh * (long)nseg * D * D;
+  float* const ck = ckpt + (long)blockIdx.x * nseg * D * DC;
   const long sbase = bh * (long)D * D;               // [dk][dv] slot of S0, dS_T, dS0
 
   // a state in the [dk][dv] order of S0 / dS_T / dS0, and in the per-thread order of the
@@ -213,7 +228,7 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
     allreduce<CW, LR>(x, lane);
 #pragma unroll
     for (int c = 0; c < CW; ++c) {
-      const float w = be * fmaf(-a, x[c], sm.v[j][j0 + c]);
+      const float w = be * fmaf(-a, x[c], sm.v[j][jl + c]);
 #pragma unroll
       for (int r = 0; r < RL; ++r) M.m[r][c] = fmaf(a, M.m[r][c], kk[r] * w);
     }
@@ -228,8 +243,8 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
   for (int sg = 0; sg < nseg; ++sg) {
     const int t0 = sg * kSeg, len = min(kSeg, T - t0);
     __syncthreads();                                 // the previous segment's data is read
-    load_segment(sm, q, k, v, dO, log_alpha, beta, b, h, hk, T, Hk, Hv, t0, len, false);
-    put_pt(ck + (long)sg * D * D, M);
+    load_segment(sm, q, k, v, dO, log_alpha, beta, b, h, hk, c0, T, Hk, Hv, t0, len, false);
+    put_pt(ck + (long)sg * D * DC, M);
     __syncthreads();
     for (int j = 0; j < len; ++j) fwd_step(M, j);
   }
@@ -257,7 +272,7 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
         const bool isa = f == 2 * D;
 #pragma unroll 4
         for (int s2 = 0; s2 < SL; ++s2) acc += isa ? sm.pa[hj][s2] : sm.pb[hj][s2];
-        const long g = (b * T + t) * Hv + h;
+        const long g = ((b * T + t) * Hv + h) * nab + hab;
         if (isa) dla_out[g] = sm.alpha[j] * acc;       // alpha <G, P - beta x k^T>
         else dbeta_out[g] = acc;                       // (v - alpha x)^T Gk
       }
@@ -267,8 +282,8 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
   for (int sg = nseg - 1; sg >= 0; --sg) {
     const int t0 = sg * kSeg, len = min(kSeg, T - t0);
     __syncthreads();
-    load_segment(sm, q, k, v, dO, log_alpha, beta, b, h, hk, T, Hk, Hv, t0, len, true);
-    get_pt(ck + (long)sg * D * D, M);                // this thread's own elements
+    load_segment(sm, q, k, v, dO, log_alpha, beta, b, h, hk, c0, T, Hk, Hv, t0, len, true);
+    get_pt(ck + (long)sg * D * DC, M);               // this thread's own elements
     put_pt(sm.state0, M);
     __syncthreads();
     if (len > kHalf) {
@@ -290,8 +305,8 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
       }
 #pragma unroll
       for (int c = 0; c < CW; ++c) {
-        vv[c] = sm.v[j][j0 + c];
-        dd[c] = sm.dO[j][j0 + c];
+        vv[c] = sm.v[j][jl + c];
+        dd[c] = sm.dO[j][jl + c];
       }
       // G += scale dO q^T; x = P k and Gk = G k (sums over dk, in the warp); <G, P> partial
       float gp = 0.f;

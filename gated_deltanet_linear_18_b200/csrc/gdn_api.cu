@@ -211,21 +211,27 @@ gdn_status validate_heads(int Hk, int Hv, int dk, int dv) {
 }
 
 // ---------------------------------------------------------------------------------------------
-// Backward pass: checkpoints every bwd::kSeg tokens, then (when key heads are shared) dq and dk
-// per value head, summed over each key head's group afterwards.  Workspace sections 256-aligned.
+// Backward pass: checkpoints every bwd::kSeg tokens; per-slice dq, dk (when key heads are shared
+// or heads are split over CTAs) and dlog alpha, dbeta (when heads are split), summed afterwards.
+// Workspace sections 256-aligned.
 // ---------------------------------------------------------------------------------------------
 size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
 struct BwdLayout {
-  size_t dqh = 0, dkh = 0, total = 0;   // offsets of the per-value-head dq, dk; total bytes
+  size_t dqh = 0, dkh = 0, dah = 0, dbh = 0, total = 0;   // section offsets; total bytes
 };
 BwdLayout bwd_layout(int B, int T, int Hk, int Hv, int dk, int dv) {
   BwdLayout L;
+  const size_t ns = (size_t)bwd::head_slices(dk);
   const size_t nseg = ((size_t)T + bwd::kSeg - 1) / bwd::kSeg;
   const size_t ck = align256((size_t)B * Hv * nseg * dk * dv * sizeof(float));
-  const size_t per = Hv != Hk ? align256((size_t)B * T * Hv * dk * sizeof(float)) : 0;
+  const bool direct = Hv == Hk && ns == 1;
+  const size_t per = direct ? 0 : align256((size_t)B * T * Hv * ns * dk * sizeof(float));
+  const size_t gate = ns > 1 ? align256((size_t)B * T * Hv * ns * sizeof(float)) : 0;
   L.dqh = ck;
   L.dkh = ck + per;
-  L.total = ck + 2 * per;
+  L.dah = ck + 2 * per;
+  L.dbh = ck + 2 * per + gate;
+  L.total = ck + 2 * per + 2 * gate;
   return L;
 }
 
@@ -234,6 +240,7 @@ gdn_status bwd_launch(const void* q, const void* k, const void* v, const float* 
                       const float* be, const float* S0, const void* dO, const float* dST,
                       float* dq, float* dk, float* dv, float* dla, float* dbeta, float* dS0,
                       void* ws, int B, int T, int Hk, int Hv, float scale, cudaStream_t st) {
+  constexpr int NS = bwd::Shape<D>::NS;
   auto kern = bwd::bwd_kernel<D, Tin>;
   const size_t smem = bwd::smem_bytes<D>();
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
@@ -241,20 +248,26 @@ gdn_status bwd_launch(const void* q, const void* k, const void* v, const float* 
     return GDN_ERR_CUDA;
   const BwdLayout L = bwd_layout(B, T, Hk, Hv, D, D);
   uint8_t* w = static_cast<uint8_t*>(ws);
-  const bool grouped = Hv != Hk;
-  float* dqo = grouped ? reinterpret_cast<float*>(w + L.dqh) : dq;
-  float* dko = grouped ? reinterpret_cast<float*>(w + L.dkh) : dk;
-  kern<<<(unsigned)((long)B * Hv), bwd::Shape<D>::NT, smem, st>>>(
+  const bool direct = Hv == Hk && NS == 1;
+  float* dqo = direct ? dq : reinterpret_cast<float*>(w + L.dqh);
+  float* dko = direct ? dk : reinterpret_cast<float*>(w + L.dkh);
+  float* dao = NS > 1 ? reinterpret_cast<float*>(w + L.dah) : dla;
+  float* dbo = NS > 1 ? reinterpret_cast<float*>(w + L.dbh) : dbeta;
+  const long ctas = (long)B * Hv * NS;
+  if (ctas > 0x7fffffffL) return GDN_ERR_UNSUPPORTED;
+  kern<<<(unsigned)ctas, bwd::Shape<D>::NT, smem, st>>>(
       static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v), la, be,
-      S0, static_cast<const Tin*>(dO), dST, dqo, dko, grouped ? Hv : Hk, dv, dla, dbeta, dS0,
+      S0, static_cast<const Tin*>(dO), dST, dqo, dko, direct ? 1 : 0, dv, dao, dbo, dS0,
       reinterpret_cast<float*>(w), T, Hk, Hv, scale);
   if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
-  if (grouped && T > 0) {
-    const long rows = (long)B * T * Hk;
-    const long n = 2 * rows * D;
+  auto sum = [&](const float* a_src, float* a_dst, const float* b_src, float* b_dst, long rows,
+                 int G, int Dd) {
+    const long n = 2 * rows * Dd;
     const unsigned blocks = (unsigned)std::min<long>((n + 255) / 256, 148L * 16);
-    bwd::group_sum_kernel<<<blocks, 256, 0, st>>>(dqo, dq, dko, dk, rows, Hv / Hk, D);
-  }
+    if (blocks > 0) bwd::group_sum_kernel<<<blocks, 256, 0, st>>>(a_src, a_dst, b_src, b_dst, rows, G, Dd);
+  };
+  if (!direct && T > 0) sum(dqo, dq, dko, dk, (long)B * T * Hk, (Hv / Hk) * NS, D);
+  if (NS > 1 && T > 0) sum(dao, dla, dbo, dbeta, (long)B * T * Hv, NS, 1);
   return launch_status();
 }
 

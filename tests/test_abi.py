@@ -234,12 +234,17 @@ def bwd(L, B=1, T=64, Hk=2, Hv=4, dk=64, dv=64, dtype=1, q=FAKE, dvo=FAKE, ws=No
 
 
 def test_bwd_workspace_bytes(L):
-    """A state every 8 tokens of every (batch, value head), then per-value-head dq and dk when
-    key heads are shared, each section 256-byte aligned; 0 for what the call rejects."""
+    """A state every 8 tokens of every (batch, value head); then, per head split over NS CTAs
+    (NS = 4 at d = 128, 2 at 64, 1 below) or key heads shared, per-slice dq and dk; and when
+    NS > 1 per-slice dlog alpha and dbeta; each section 256-byte aligned; 0 for what the call
+    rejects."""
+    al = lambda n: (n + 255) // 256 * 256
     ck = 2 * 6 * 17 * 128 * 128 * 4                  # T = 130: 17 segments of 8 tokens
-    per = 2 * 130 * 6 * 128 * 4
-    assert L.gdn_bwd_workspace_bytes(2, 130, 2, 6, 128, 128) == ck + 2 * per
-    assert L.gdn_bwd_workspace_bytes(2, 130, 2, 2, 128, 128) == 2 * 2 * 17 * 128 * 128 * 4
+    per = al(2 * 130 * 6 * 4 * 128 * 4)
+    gate = al(2 * 130 * 6 * 4 * 4)
+    assert L.gdn_bwd_workspace_bytes(2, 130, 2, 6, 128, 128) == ck + 2 * per + 2 * gate
+    # d = 32, one value head per key head, one CTA per head: checkpoints only
+    assert L.gdn_bwd_workspace_bytes(2, 130, 2, 2, 32, 32) == 2 * 2 * 17 * 32 * 32 * 4
     assert L.gdn_bwd_workspace_bytes(2, 130, 2, 6, 128, 64) == 0     # dk != dv
     assert L.gdn_bwd_workspace_bytes(2, 130, 2, 6, 48, 48) == 0
     assert L.gdn_bwd_workspace_bytes(0, 130, 2, 6, 128, 128) == 0
