@@ -260,12 +260,14 @@ GDN_API gdn_status gdn_chunk_fwd_varlen(const void *q, const void *k, const void
  *   dq, dk [B, T, Hk, dk] float: summed over the Hv / Hk value heads of each key head
  *   dv [B, T, Hv, dv], dlog_alpha, dbeta [B, T, Hv] float; dS0 [B, Hv, dk, dv] float (nullable)
  *   workspace: gdn_bwd_workspace_bytes(...) bytes, 256-byte aligned, owned by the caller (the
- *        state every 8 tokens of every (batch, value head), and per-value-head dq, dk when key
- *        heads are shared); NULL is accepted when that size is 0.
- * dk == dv in {16, 32, 64, 128} (else GDN_ERR_UNSUPPORTED).  One CUDA-core kernel, one CTA per
- * (batch, value head): a forward walk keeps the checkpoints, a reverse walk recomputes each
- * state from the nearest of two kept states of its 8-token segment; a second launch sums dq, dk
- * over each key head's value heads when Hv > Hk (a fixed order: the result is reproducible).
+ *        state every 8 tokens of every (batch, value head), and the per-slice partial outputs
+ *        summed at the end); NULL is accepted when that size is 0.
+ * dk == dv in {16, 32, 64, 128} (else GDN_ERR_UNSUPPORTED).  A CUDA-core kernel with a head's dv
+ * columns split over 4 CTAs (d = 128; 2 at d = 64, 1 below): a forward walk keeps the
+ * checkpoints, a reverse walk recomputes each state from the nearer of two kept states of its
+ * 8-token segment; up to two more launches add the partial dq, dk (over each key head's value
+ * heads and the slices) and dlog_alpha, dbeta (over the slices) in a fixed order, so the result
+ * is reproducible bit for bit.
  * Pointer alignment: 16 bytes for dv, S0, dS_T, dS0; 4 bytes for the rest.  Errors as
  * gdn_chunk_fwd: GDN_ERR_INVALID_ARG (missing, misaligned, workspace too small) before any work.
  */
