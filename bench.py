@@ -69,14 +69,6 @@ def bwd_flops(w: gi.Workload) -> float:
     return float(w.B * w.T * w.Hv * 20 * w.dk * w.dv)
 
 
-def bwd_launches(w: gi.Workload) -> int:
-    """Kernels one gdn_bwd call launches: the backward kernel, then the sum of the partial dq, dk
-    (when key heads are shared or heads split over CTAs) and of dlog alpha, dbeta (when heads are
-    split: 4 CTAs per head at d = 128, 2 at d = 64)."""
-    ns = 4 if w.dk == 128 else (2 if w.dk == 64 else 1)
-    return 1 + (0 if (w.Hv == w.Hk and ns == 1) else 1) + (1 if ns > 1 else 0)
-
-
 def fp32_peak_tflops(dev) -> float:
     """fp32 FMA peak: SMs x 128 FP32 lanes x 2 flops x 1965 MHz (the part's maximum SM clock)."""
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
@@ -432,7 +424,7 @@ def bench_backward(gdn, dev, warmup, flush, steps=5):
     def step():
         gdn.bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"], d["dO"], d["dS_T"],
                 workspace=ws)
-    launches = bwd_launches(w)
+    launches = gdn.bwd_launches(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv)
     ms = time_steps(step, steps, warmup, flush, launches)
     t = statistics.mean(ms) / 1e3
     F = bwd_flops(w)
@@ -700,7 +692,7 @@ def profile_case(args):
         def step():
             gdn.bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"], d["dO"],
                     d["dS_T"])
-        launches = bwd_launches(w)
+        launches = gdn.bwd_launches(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv)
     elif name in ("decode", "decode_layer"):
         mk = gi.make_decode_inputs if name == "decode" else gi.make_decode_layer_inputs
         d = to_dev(mk(w.with_sizes(steps=1)), dev)

@@ -94,6 +94,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_bwd.restype = I
         L.gdn_bwd_workspace_bytes.argtypes = [I] * 6
         L.gdn_bwd_workspace_bytes.restype = SZ
+        L.gdn_bwd_launches.argtypes = [I] * 6
+        L.gdn_bwd_launches.restype = I
         _lib = L
     return _lib
 
@@ -209,6 +211,14 @@ def chunk_fwd(q, k, v, log_alpha, beta, S0=None, *, chunk: int = 64, scale: floa
 def bwd_workspace_bytes(B, T, Hk, Hv, dk, dv) -> int:
     """Caller-owned device scratch one ``bwd`` call needs."""
     return int(lib().gdn_bwd_workspace_bytes(B, T, Hk, Hv, dk, dv))
+
+
+def bwd_launches(B, T, Hk, Hv, dk, dv) -> int:
+    """Kernels one ``bwd`` call launches (the library's own count)."""
+    n = lib().gdn_bwd_launches(B, T, Hk, Hv, dk, dv)
+    if n < 0:
+        raise ValueError("gdn_bwd_launches rejected the sizes")
+    return n
 
 
 def bwd(q, k, v, log_alpha, beta, S0, dO, dS_T=None, *, scale: float = 1.0,

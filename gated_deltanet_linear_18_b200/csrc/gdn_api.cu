@@ -294,6 +294,14 @@ gdn_status bwd_dispatch(int d, const void* q, const void* k, const void* v, cons
 
 extern "C" {
 
+int gdn_bwd_launches(int B, int T, int Hk, int Hv, int dk, int dv) {
+  if (B < 0 || T < 0 || validate_heads(Hk, Hv, dk, dv) != GDN_OK || dk != dv) return -1;
+  if (B == 0) return 0;
+  const int ns = bwd::head_slices(dk);
+  if (T == 0) return 1;                       // the kernel alone hands dS_T to dS0
+  return 1 + ((Hv == Hk && ns == 1) ? 0 : 1) + (ns > 1 ? 1 : 0);
+}
+
 size_t gdn_bwd_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv) {
   if (B < 0 || T < 0 || validate_heads(Hk, Hv, dk, dv) != GDN_OK || dk != dv) return 0;
   if ((long)B * T == 0) return 0;

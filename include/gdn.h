@@ -277,6 +277,11 @@ GDN_API gdn_status gdn_bwd(const void *q, const void *k, const void *v, const fl
                    void *workspace, size_t workspace_bytes, int B, int T, int Hk, int Hv,
                    int dk_, int dv_, float scale, gdn_dtype dtype, gdn_stream_t stream);
 
+/* Kernels one gdn_bwd call with these sizes launches (host only, no CUDA call): the backward
+ * kernel, plus the sums of the partial dq, dk and of dlog_alpha, dbeta where the call has them;
+ * -1 for sizes the call rejects. */
+GDN_API int gdn_bwd_launches(int B, int T, int Hk, int Hv, int dk, int dv);
+
 /* Device scratch bytes gdn_bwd needs (host only, no CUDA call); 0 for invalid sizes. */
 GDN_API size_t gdn_bwd_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv);
 

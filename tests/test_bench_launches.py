@@ -43,3 +43,15 @@ def test_simt_forward_is_one_launch(gdn):
     w = gi.WORKLOADS["prefill"]
     assert gdn.chunk_fwd_launches(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv, w.chunk, torch.bfloat16,
                                   variant="simt", sms=148) == 1
+
+
+@pytest.mark.parametrize("sizes, expected", [
+    (dict(B=4, T=2048, Hk=16, Hv=48, dk=128, dv=128), 3),   # 4 CTAs per head, shared key heads
+    (dict(B=1, T=64, Hk=2, Hv=2, dk=64, dv=64), 3),         # 2 CTAs per head
+    (dict(B=1, T=64, Hk=2, Hv=2, dk=32, dv=32), 1),         # nothing to add up
+    (dict(B=1, T=64, Hk=1, Hv=2, dk=32, dv=32), 2),         # dq, dk over the value heads
+    (dict(B=1, T=0, Hk=1, Hv=2, dk=128, dv=128), 1),
+    (dict(B=0, T=64, Hk=1, Hv=2, dk=128, dv=128), 0),
+])
+def test_backward_launches(gdn, sizes, expected):
+    assert gdn.bwd_launches(**sizes) == expected
