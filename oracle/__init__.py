@@ -126,6 +126,14 @@ class OracleLib:
         lib.oracle_gates.restype = None
         lib.oracle_gated_delta_bwd.argtypes = [P] * 14 + [L, L, I, I, I, I, D, I]
         lib.oracle_gated_delta_bwd.restype = I
+        lib.oracle_causal_conv_silu_bwd.argtypes = [P, P, P, P, P, L, L, L]
+        lib.oracle_causal_conv_silu_bwd.restype = None
+        lib.oracle_l2_normalize_bwd.argtypes = [P, P, P, L, I, D]
+        lib.oracle_l2_normalize_bwd.restype = None
+        lib.oracle_gated_rmsnorm_bwd.argtypes = [P, P, P, P, P, P, P, L, I, D]
+        lib.oracle_gated_rmsnorm_bwd.restype = None
+        lib.oracle_gates_bwd.argtypes = [P, P, P, P, L, I]
+        lib.oracle_gates_bwd.restype = None
         self.lib = lib
         self.path = path
 
@@ -179,6 +187,40 @@ class OracleLib:
         if rc != 0:
             raise ValueError(f"oracle_gated_delta_bwd failed ({rc})")
         return out
+
+    def causal_conv_silu_bwd(self, x, w, dy) -> Tuple[np.ndarray, np.ndarray]:
+        """Gradients (dx [B,T,C], dw [C,4]) of <dy, causal_conv_silu(x, w)>."""
+        x, w, dy = _f64(x), _f64(w), _f64(dy)
+        B, T, C = x.shape
+        dx, dw = np.zeros_like(x), np.zeros((C, 4))
+        self.lib.oracle_causal_conv_silu_bwd(_ptr(x), _ptr(w), _ptr(dy), _ptr(dx), _ptr(dw),
+                                             B, T, C)
+        return dx, dw
+
+    def l2_normalize_bwd(self, x, dy, eps: float = 0.0) -> np.ndarray:
+        """Gradient of <dy, l2_normalize(x)> over the last dimension."""
+        x, dy = _f64(x), _f64(dy)
+        dx = np.zeros_like(x)
+        d = x.shape[-1]
+        self.lib.oracle_l2_normalize_bwd(_ptr(x), _ptr(dy), _ptr(dx), x.size // d, d, float(eps))
+        return dx
+
+    def gated_rmsnorm_bwd(self, o, z, w, dy, eps: float = 1e-5):
+        """Gradients (do, dz, dw) of <dy, gated_rmsnorm(o, z, w)>; rows of d = w.size."""
+        o, z, w, dy = _f64(o), _f64(z), _f64(w), _f64(dy)
+        d = w.size
+        do_, dz, dw = np.zeros_like(o), np.zeros_like(z), np.zeros(d)
+        self.lib.oracle_gated_rmsnorm_bwd(_ptr(o), _ptr(z), _ptr(w), _ptr(dy), _ptr(do_),
+                                          _ptr(dz), _ptr(dw), o.size // d, d, float(eps))
+        return do_, dz, dw
+
+    def gates_bwd(self, ba, dlog_alpha, dbeta) -> np.ndarray:
+        """Gradient [rows, 2 Hv] of <dlog_alpha, log alpha> + <dbeta, beta> through gates(ba)."""
+        ba, dla, db = _f64(ba), _f64(dlog_alpha), _f64(dbeta)
+        Hv = ba.shape[-1] // 2
+        dba = np.zeros_like(ba)
+        self.lib.oracle_gates_bwd(_ptr(ba), _ptr(dla), _ptr(db), _ptr(dba), ba.size // (2 * Hv), Hv)
+        return dba
 
     def decode_steps(self, q, k, v, log_alpha, beta, S0, scale: float = 1.0,
                      threads: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray]:
@@ -378,3 +420,19 @@ def gates(*a, **kw):
 
 def gated_delta_varlen(*a, **kw):
     return get().gated_delta_varlen(*a, **kw)
+
+
+def causal_conv_silu_bwd(*a, **kw):
+    return get().causal_conv_silu_bwd(*a, **kw)
+
+
+def l2_normalize_bwd(*a, **kw):
+    return get().l2_normalize_bwd(*a, **kw)
+
+
+def gated_rmsnorm_bwd(*a, **kw):
+    return get().gated_rmsnorm_bwd(*a, **kw)
+
+
+def gates_bwd(*a, **kw):
+    return get().gates_bwd(*a, **kw)

@@ -424,3 +424,94 @@ int oracle_gated_delta_bwd(const double *q, const double *k, const double *v,
     free(started); free(jobs); free(th); free(ret);
     return rc;
 }
+
+/* ------------------------------------------------------------------------------------------ */
+/* Backward of the layer's other pieces: chain rule through each forward definition above      */
+/* ------------------------------------------------------------------------------------------ */
+
+/*
+ * y = SiLU(conv(x)) as oracle_causal_conv_silu; given dy, with pre the convolution and
+ * SiLU'(p) = sigmoid(p) (1 + p (1 - sigmoid(p))):
+ *   dpre = dy SiLU'(pre);  dx[s] = sum_j w[j] dpre[s + 3 - j];  dw[c][j] = sum_t dpre[t] x[t - 3 + j]
+ * (tokens outside 0 .. T - 1 contribute nothing).  dw is summed over every batch and token.
+ */
+void oracle_causal_conv_silu_bwd(const double *x, const double *w, const double *dy, double *dx,
+                                 double *dw, long B, long T, long C)
+{
+    for (long i = 0; i < B * T * C; ++i) dx[i] = 0.0;
+    for (long i = 0; i < C * 4; ++i) dw[i] = 0.0;
+    for (long b = 0; b < B; ++b)
+        for (long t = 0; t < T; ++t)
+            for (long c = 0; c < C; ++c) {
+                double pre = 0.0;
+                for (int j = 0; j < 4; ++j) {
+                    const long u = t - 3 + j;          /* the tap's token */
+                    if (u >= 0) pre += w[c * 4 + j] * x[(b * T + u) * C + c];
+                }
+                const double sg = sigmoid(pre);
+                const double dpre = dy[(b * T + t) * C + c] * sg * (1.0 + pre * (1.0 - sg));
+                for (int j = 0; j < 4; ++j) {
+                    const long u = t - 3 + j;          /* the tap's token */
+                    if (u < 0) continue;
+                    dx[(b * T + u) * C + c] += w[c * 4 + j] * dpre;
+                    dw[c * 4 + j] += x[(b * T + u) * C + c] * dpre;
+                }
+            }
+}
+
+/* y = x / sqrt(sum x^2 + eps) per row of d:  dx = dy / n - x (x . dy) / n^3,  n = sqrt(ss + eps). */
+void oracle_l2_normalize_bwd(const double *x, const double *dy, double *dx, long rows, int d,
+                             double eps)
+{
+    for (long r = 0; r < rows; ++r) {
+        double ss = 0.0, xd = 0.0;
+        for (int i = 0; i < d; ++i) {
+            ss += x[r * d + i] * x[r * d + i];
+            xd += x[r * d + i] * dy[r * d + i];
+        }
+        const double n = sqrt(ss + eps);
+        for (int i = 0; i < d; ++i) dx[r * d + i] = dy[r * d + i] / n - x[r * d + i] * xd / (n * n * n);
+    }
+}
+
+/*
+ * y_i = o_i inv w_i SiLU(z_i), inv = 1 / sqrt(mean(o^2) + eps), per row of d; given dy:
+ *   dz_i = dy_i o_i inv w_i SiLU'(z_i);  dw_i += dy_i o_i inv SiLU(z_i)  (summed over rows);
+ *   with g_i = dy_i w_i SiLU(z_i):  do_i = inv g_i - o_i inv^3 (sum_j g_j o_j) / d.
+ */
+void oracle_gated_rmsnorm_bwd(const double *o, const double *z, const double *w,
+                              const double *dy, double *dout, double *dz, double *dw, long rows,
+                              int d, double eps)
+{
+    for (int i = 0; i < d; ++i) dw[i] = 0.0;
+    for (long r = 0; r < rows; ++r) {
+        double ss = 0.0, go = 0.0;
+        for (int i = 0; i < d; ++i) ss += o[r * d + i] * o[r * d + i];
+        const double inv = 1.0 / sqrt(ss / (double)d + eps);   /* 1 / rms */
+        for (int i = 0; i < d; ++i) {
+            const double zz = z[r * d + i], sg = sigmoid(zz);
+            const double g = dy[r * d + i] * w[i] * (zz * sg);
+            go += g * o[r * d + i];
+            dz[r * d + i] = dy[r * d + i] * o[r * d + i] * inv * w[i] * sg * (1.0 + zz * (1.0 - sg));
+            dw[i] += dy[r * d + i] * o[r * d + i] * inv * (zz * sg);
+        }
+        for (int i = 0; i < d; ++i) {
+            const double g = dy[r * d + i] * w[i] * (z[r * d + i] * sigmoid(z[r * d + i]));
+            dout[r * d + i] = inv * g - o[r * d + i] * inv * inv * inv * go / d;
+        }
+    }
+}
+
+/* beta = sigmoid(b), log alpha = -softplus(-a):  db = dbeta beta (1 - beta),  da = dlog_alpha
+ * sigmoid(-a).  ba, dba: [rows, 2 Hv] (b values then a values). */
+void oracle_gates_bwd(const double *ba, const double *dlog_alpha, const double *dbeta, double *dba,
+                      long rows, int Hv)
+{
+    for (long r = 0; r < rows; ++r)
+        for (int h = 0; h < Hv; ++h) {
+            const double b = ba[r * 2 * Hv + h], a = ba[r * 2 * Hv + Hv + h];
+            const double sb = sigmoid(b);
+            dba[r * 2 * Hv + h] = dbeta[r * Hv + h] * sb * (1.0 - sb);
+            dba[r * 2 * Hv + Hv + h] = dlog_alpha[r * Hv + h] * sigmoid(-a);
+        }
+}

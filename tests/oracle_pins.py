@@ -460,4 +460,69 @@ def pin_bwd_closed_forms_alpha1_beta0(orc):
     np.testing.assert_allclose(g["dq"][0, :, 0], dq, rtol=1e-12, atol=1e-12)
 
 
+def _central(f, x, h=1e-6):
+    """Central differences of the scalar f at x, entry by entry."""
+    g = np.zeros_like(x)
+    for idx in np.ndindex(x.shape):
+        old = x[idx]
+        x[idx] = old + h
+        lp = f()
+        x[idx] = old - h
+        lm = f()
+        x[idx] = old
+        g[idx] = (lp - lm) / (2 * h)
+    return g
+
+
+def _close(got, fd, tol=1e-7):
+    err = np.max(np.abs(got - fd)) / max(1.0, np.max(np.abs(fd)))
+    assert err < tol, err
+
+
+def pin_bwd_conv_silu_central_differences(orc):
+    """dx and dw of <dy, SiLU(conv(x))> equal central differences (tokens before 0 are zeros)."""
+    rng = np.random.default_rng(51)
+    x = rng.standard_normal((2, 6, 3))
+    w = rng.standard_normal((3, 4)) * 0.5
+    dy = rng.standard_normal(x.shape)
+    dx, dw = orc.causal_conv_silu_bwd(x, w, dy)
+    f = lambda: float(np.sum(dy * orc.causal_conv_silu(x, w)))
+    _close(dx, _central(f, x))
+    _close(dw, _central(f, w))
+
+
+def pin_bwd_l2_normalize_central_differences(orc):
+    rng = np.random.default_rng(52)
+    x = rng.standard_normal((3, 5))
+    dy = rng.standard_normal(x.shape)
+    dx = orc.l2_normalize_bwd(x, dy, eps=1e-6)
+    _close(dx, _central(lambda: float(np.sum(dy * orc.l2_normalize(x, 1e-6))), x))
+
+
+def pin_bwd_gated_rmsnorm_central_differences(orc):
+    rng = np.random.default_rng(53)
+    o = rng.standard_normal((3, 4))
+    z = rng.standard_normal((3, 4))
+    w = rng.standard_normal(4)
+    dy = rng.standard_normal(o.shape)
+    do_, dz, dw = orc.gated_rmsnorm_bwd(o, z, w, dy, eps=1e-5)
+    f = lambda: float(np.sum(dy * orc.gated_rmsnorm(o, z, w, 1e-5)))
+    _close(do_, _central(f, o))
+    _close(dz, _central(f, z))
+    _close(dw, _central(f, w))
+
+
+def pin_bwd_gates_central_differences(orc):
+    rng = np.random.default_rng(54)
+    ba = rng.standard_normal((3, 4)) * 2.0             # Hv = 2
+    dla = rng.standard_normal((3, 2))
+    db = rng.standard_normal((3, 2))
+    dba = orc.gates_bwd(ba, dla, db)
+
+    def f():
+        la, be = orc.gates(ba, 2)
+        return float(np.sum(dla * la) + np.sum(db * be))
+    _close(dba, _central(f, ba))
+
+
 ALL_PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]

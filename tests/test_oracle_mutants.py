@@ -62,6 +62,17 @@ MUTANTS = {
     "bwd_dk_drops_state_term": ("dkk[c] += acc;", "dkk[c] += 0.0 * acc;"),
     "bwd_state_grad_drops_rank1": ("dP[(long)a * dk + c] += dx[a] * k[c];",
                                    "dP[(long)a * dk + c] += 0.0 * dx[a] * k[c];"),
+    "bwd_silu_derivative_is_sigmoid": (
+        "const double dpre = dy[(b * T + t) * C + c] * sg * (1.0 + pre * (1.0 - sg));",
+        "const double dpre = dy[(b * T + t) * C + c] * sg;"),
+    "bwd_conv_tap_reversed": ("dx[(b * T + u) * C + c] += w[c * 4 + j] * dpre;",
+                              "dx[(b * T + u) * C + c] += w[c * 4 + 3 - j] * dpre;"),
+    "bwd_l2_drops_projection": ("dx[r * d + i] = dy[r * d + i] / n - x[r * d + i] * xd / (n * n * n);",
+                                "dx[r * d + i] = dy[r * d + i] / n;"),
+    "bwd_rms_sum_not_mean": ("dout[r * d + i] = inv * g - o[r * d + i] * inv * inv * inv * go / d;",
+                             "dout[r * d + i] = inv * g - o[r * d + i] * inv * inv * inv * go;"),
+    "bwd_gate_a_sign": ("dba[r * 2 * Hv + Hv + h] = dlog_alpha[r * Hv + h] * sigmoid(-a);",
+                        "dba[r * 2 * Hv + Hv + h] = dlog_alpha[r * Hv + h] * sigmoid(a);"),
 }
 
 
