@@ -96,6 +96,12 @@ def lib() -> ctypes.CDLL:
         L.gdn_bwd_workspace_bytes.restype = SZ
         L.gdn_bwd_launches.argtypes = [I] * 6
         L.gdn_bwd_launches.restype = I
+        L.gdn_layer_bwd.argtypes = [P] * 25 + [SZ] + [I] * 7 + [F, F, F, I, I, P]
+        L.gdn_layer_bwd.restype = I
+        L.gdn_layer_bwd_workspace_bytes.argtypes = [I] * 8
+        L.gdn_layer_bwd_workspace_bytes.restype = SZ
+        L.gdn_gates_bwd.argtypes = [P, P, P, P, LL, I, I, P]
+        L.gdn_gates_bwd.restype = I
         _lib = L
     return _lib
 
@@ -441,6 +447,56 @@ def layer_fwd(q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, *
                                  _io_dtype(q_raw), _io_dtype(y), _stream(dev))
     _check("gdn_layer_fwd", st)
     return y, sT
+
+
+def layer_bwd_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, dtype) -> int:
+    return int(lib().gdn_layer_bwd_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, _DTYPES[dtype]))
+
+
+def layer_bwd(q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, dy, dS_T=None, *,
+              Hk: int, Hv: int, dk: int, dv: int, chunk: int = 64, scale: float = 1.0,
+              l2_eps: float = 1e-6, norm_eps: float = 1e-5, want_dS0: bool = True,
+              workspace: Optional[torch.Tensor] = None) -> dict:
+    """Gradients of <dy, y> + <dS_T, S_T> for layer_fwd's inputs and weights (gdn_layer_bwd):
+    fp32 dq_raw, dk_raw, dv_raw, dz, dwq, dwk, dwv, dlog_alpha, dbeta, dS0, dnorm_w."""
+    B, T = q_raw.shape[:2]
+    _f32(wq, wk, wv, log_alpha, beta, S0, norm_w, dS_T)
+    f = dict(device=q_raw.device, dtype=torch.float32)
+    out = {"dq_raw": torch.empty(q_raw.shape, **f), "dk_raw": torch.empty(k_raw.shape, **f),
+           "dv_raw": torch.empty(v_raw.shape, **f), "dz": torch.empty(z.shape, **f),
+           "dwq": torch.empty(wq.shape, **f), "dwk": torch.empty(wk.shape, **f),
+           "dwv": torch.empty(wv.shape, **f), "dlog_alpha": torch.empty(log_alpha.shape, **f),
+           "dbeta": torch.empty(beta.shape, **f),
+           "dS0": torch.empty(B, Hv, dk, dv, **f) if want_dS0 else None,
+           "dnorm_w": torch.empty(norm_w.shape, **f)}
+    dev = _dev(q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, dy, dS_T,
+               workspace)
+    ws, wbytes = _workspace(layer_bwd_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, q_raw.dtype),
+                            dev, workspace)
+    with torch.cuda.device(dev):
+        st = lib().gdn_layer_bwd(
+            _p(q_raw), _p(k_raw), _p(v_raw), _p(z), _p(wq), _p(wk), _p(wv), _p(log_alpha),
+            _p(beta), _p(S0), _p(norm_w), _p(dy), _p(dS_T), _p(out["dq_raw"]), _p(out["dk_raw"]),
+            _p(out["dv_raw"]), _p(out["dz"]), _p(out["dwq"]), _p(out["dwk"]), _p(out["dwv"]),
+            _p(out["dlog_alpha"]), _p(out["dbeta"]), _p(out["dS0"]), _p(out["dnorm_w"]), _p(ws),
+            wbytes, B, T, Hk, Hv, dk, dv, chunk, float(scale), float(l2_eps), float(norm_eps),
+            _io_dtype(q_raw), _io_dtype(dy), _stream(dev))
+    _check("gdn_layer_bwd", st)
+    return out
+
+
+def gates_bwd(ba, dlog_alpha, dbeta) -> torch.Tensor:
+    """Gradient [..., 2*Hv] fp32 of <dlog_alpha, log alpha> + <dbeta, beta> through gates(ba)."""
+    Hv = ba.shape[-1] // 2
+    rows = ba.numel() // (2 * Hv)
+    _f32(dlog_alpha, dbeta)
+    dba = torch.empty(ba.shape, device=ba.device, dtype=torch.float32)
+    dev = _dev(ba, dlog_alpha, dbeta, dba)
+    with torch.cuda.device(dev):
+        st = lib().gdn_gates_bwd(_p(ba), _p(dlog_alpha), _p(dbeta), _p(dba), rows, Hv,
+                                 _io_dtype(ba), _stream(dev))
+    _check("gdn_gates_bwd", st)
+    return dba
 
 
 def layer_fwd_static(q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, *,

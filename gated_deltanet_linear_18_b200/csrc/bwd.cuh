@@ -115,10 +115,10 @@ __device__ __forceinline__ float group_sum(float x) {
 }
 
 // The segment's token data (tokens t0 .. t0 + len - 1) into shared memory, as fp32.
-template <int D, typename Tin>
+template <int D, typename Tin, typename Tdo>
 __device__ __forceinline__ void load_segment(Smem<D>& sm, const Tin* __restrict__ q,
                                              const Tin* __restrict__ k, const Tin* __restrict__ v,
-                                             const Tin* __restrict__ dO,
+                                             const Tdo* __restrict__ dO,
                                              const float* __restrict__ la,
                                              const float* __restrict__ be, long b, int h, int hk,
                                              int c0, int T, int Hk, int Hv, int t0, int len,
@@ -155,11 +155,11 @@ struct Tile {
 // dk_out are [B, T, Hk, D] and dla_out, dbeta_out [B, T, Hv]; otherwise they are the per-slice
 // partials [B, T, Hv * NS, D] and [B, T, Hv, NS], summed afterwards by group_sum_kernel.  ckpt:
 // B * Hv * NS * ceil(T / kSeg) slices of D * DC floats, each in the CTA's own per-thread order.
-template <int D, typename Tin>
+template <int D, typename Tin, typename Tdo = Tin>
 __global__ void __launch_bounds__(Shape<D>::NT, Shape<D>::MINB)
 bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
            const float* __restrict__ log_alpha, const float* __restrict__ beta,
-           const float* __restrict__ S0, const Tin* __restrict__ dO,
+           const float* __restrict__ S0, const Tdo* __restrict__ dO,
            const float* __restrict__ dS_T, float* __restrict__ dq_out,
            float* __restrict__ dk_out, int direct, float* __restrict__ dv_out,
            float* __restrict__ dla_out, float* __restrict__ dbeta_out, float* __restrict__ dS0,

@@ -11,6 +11,7 @@
 #include "bwd.cuh"
 #include "decode_layer.cuh"
 #include "elementwise.cuh"
+#include "layer_bwd.cuh"
 #include "simt_chunk.cuh"
 #include "tc_chunk.cuh"
 
@@ -235,13 +236,13 @@ BwdLayout bwd_layout(int B, int T, int Hk, int Hv, int dk, int dv) {
   return L;
 }
 
-template <int D, typename Tin>
+template <int D, typename Tin, typename Tdo = Tin>
 gdn_status bwd_launch(const void* q, const void* k, const void* v, const float* la,
                       const float* be, const float* S0, const void* dO, const float* dST,
                       float* dq, float* dk, float* dv, float* dla, float* dbeta, float* dS0,
                       void* ws, int B, int T, int Hk, int Hv, float scale, cudaStream_t st) {
   constexpr int NS = bwd::Shape<D>::NS;
-  auto kern = bwd::bwd_kernel<D, Tin>;
+  auto kern = bwd::bwd_kernel<D, Tin, Tdo>;
   const size_t smem = bwd::smem_bytes<D>();
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
@@ -257,7 +258,7 @@ gdn_status bwd_launch(const void* q, const void* k, const void* v, const float* 
   if (ctas > 0x7fffffffL) return GDN_ERR_UNSUPPORTED;
   kern<<<(unsigned)ctas, bwd::Shape<D>::NT, smem, st>>>(
       static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v), la, be,
-      S0, static_cast<const Tin*>(dO), dST, dqo, dko, direct ? 1 : 0, dv, dao, dbo, dS0,
+      S0, static_cast<const Tdo*>(dO), dST, dqo, dko, direct ? 1 : 0, dv, dao, dbo, dS0,
       reinterpret_cast<float*>(w), T, Hk, Hv, scale);
   if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
   auto sum = [&](const float* a_src, float* a_dst, const float* b_src, float* b_dst, long rows,
@@ -271,15 +272,15 @@ gdn_status bwd_launch(const void* q, const void* k, const void* v, const float* 
   return launch_status();
 }
 
-template <typename Tin>
+template <typename Tin, typename Tdo = Tin>
 gdn_status bwd_dispatch(int d, const void* q, const void* k, const void* v, const float* la,
                         const float* be, const float* S0, const void* dO, const float* dST,
                         float* dq, float* dk, float* dv, float* dla, float* dbeta, float* dS0,
                         void* ws, int B, int T, int Hk, int Hv, float scale, cudaStream_t st) {
 #define GDN_BWD(D)                                                                              \
   case D:                                                                                       \
-    return bwd_launch<D, Tin>(q, k, v, la, be, S0, dO, dST, dq, dk, dv, dla, dbeta, dS0, ws, B, \
-                              T, Hk, Hv, scale, st);
+    return bwd_launch<D, Tin, Tdo>(q, k, v, la, be, S0, dO, dST, dq, dk, dv, dla, dbeta, dS0, ws, \
+                                   B, T, Hk, Hv, scale, st);
   switch (d) {
     GDN_BWD(16)
     GDN_BWD(32)
@@ -737,6 +738,180 @@ gdn_status gdn_layer_fwd(const void* q_raw, const void* k_raw, const void* v_raw
   else
     out_norm_kernel<float, __nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
         (const float*)o, (const __nv_bfloat16*)z, norm_w, (__nv_bfloat16*)y, rows, dv, norm_eps);
+  return launch_status();
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------------------
+// Layer backward: the forward recomputed (prologue, recurrence with fp32 o), then the gated norm's
+// backward (dO in fp32), the recurrence's (gdn_bwd with an fp32 dO), the prologue's.
+// ---------------------------------------------------------------------------------------------
+namespace {
+constexpr unsigned kNormBwdCtas = 592;   // fixed grid of the norm backward (its dw partial sums)
+struct LayerBwdLayout {
+  size_t fwd = 0, d_o = 0, dq = 0, dk = 0, dv = 0, bwd = 0, dpre = 0, nw = 0, cw = 0, total = 0;
+};
+LayerBwdLayout layer_bwd_layout(int B, int T, int Hk, int Hv, int dk, int dv, int chunk,
+                                gdn_dtype dtype) {
+  LayerBwdLayout L;
+  const size_t tok = (size_t)B * T;
+  const size_t C = std::max((size_t)Hk * dk, (size_t)Hv * dv);
+  const size_t tiles = (size_t)B * ((T + lbwd::kConvTok - 1) / lbwd::kConvTok);
+  size_t o = align256(gdn_layer_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, dtype));
+  L.fwd = 0;
+  L.d_o = o;  o += align256(tok * Hv * dv * 4);
+  L.dq = o;   o += align256(tok * Hk * dk * 4);
+  L.dk = o;   o += align256(tok * Hk * dk * 4);
+  L.dv = o;   o += align256(tok * Hv * dv * 4);
+  L.bwd = o;  o += align256(bwd_layout(B, T, Hk, Hv, dk, dv).total);
+  L.dpre = o; o += align256(tok * C * 4);
+  L.nw = o;   o += align256((size_t)kNormBwdCtas * dv * 4);
+  L.cw = o;   o += align256(tiles * C * 4 * 4);
+  L.total = o;
+  return L;
+}
+
+template <typename Tin>
+gdn_status prologue_bwd_one(const void* x_raw, const float* w, const float* dy, float* dx_raw,
+                            float* dw, float* dpre, float* dw_part, int B, int T, int heads,
+                            int d, bool normalize, float eps, cudaStream_t st) {
+  const long long rows = (long long)B * T * heads;
+  const long long blocks = (rows + 7) / 8;
+  lbwd::conv_dpre_kernel<Tin><<<(unsigned)blocks, 256, 0, st>>>(
+      static_cast<const Tin*>(x_raw), w, dy, dpre, rows, T, heads, d, normalize ? 1 : 0, eps);
+  const int C = heads * d;
+  const dim3 grid((C + 127) / 128, (T + lbwd::kConvTok - 1) / lbwd::kConvTok, B);
+  lbwd::conv_bwd_kernel<Tin><<<grid, 128, 0, st>>>(static_cast<const Tin*>(x_raw), w, dpre,
+                                                   dx_raw, dw_part, T, C);
+  lbwd::col_sum_kernel<<<(C * 4 + 255) / 256, 256, 0, st>>>(dw_part, dw, (int)(grid.y * grid.z),
+                                                            C * 4);
+  return launch_status();
+}
+
+template <typename Tin, typename Tdy>
+gdn_status layer_bwd_run(const void* q_raw, const void* k_raw, const void* v_raw, const void* z,
+                         const float* wq, const float* wk, const float* wv, const float* la,
+                         const float* be, const float* S0, const float* norm_w, const void* dy,
+                         const float* dS_T, float* dq_raw, float* dk_raw, float* dv_raw,
+                         float* dz, float* dwq, float* dwk, float* dwv, float* dla, float* dbeta,
+                         float* dS0, float* dnorm_w, char* ws, const LayerBwdLayout& L, int B,
+                         int T, int Hk, int Hv, int dk, int dv, int chunk, float scale,
+                         float l2_eps, float norm_eps, gdn_dtype dtype, gdn_stream_t stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t el = dtype == GDN_F32 ? 4 : 2;
+  const size_t tok = (size_t)B * T;
+  void* qn = ws;
+  void* kn = ws + align256(tok * Hk * dk * el);
+  void* vc = ws + 2 * align256(tok * Hk * dk * el);
+  char* rest = ws + 2 * align256(tok * Hk * dk * el) + align256(tok * Hv * dv * el);
+  float* o = reinterpret_cast<float*>(rest);
+  void* tc_scratch = rest + align256(tok * Hv * dv * 4);
+  gdn_status s = gdn_prologue(q_raw, k_raw, v_raw, wq, wk, wv, qn, kn, vc, B, T, Hk, Hv, dk, dv,
+                              l2_eps, dtype, stream);
+  if (s != GDN_OK) return s;
+  s = layer_chunk_fwd(qn, kn, vc, la, be, S0, o, nullptr, B, T, Hk, Hv, dk, dv, chunk, scale,
+                      dtype, tc_scratch, st);
+  if (s != GDN_OK) return s;
+  float* d_o = reinterpret_cast<float*>(ws + L.d_o);
+  float* nw = reinterpret_cast<float*>(ws + L.nw);
+  const long long rows = (long long)tok * Hv;
+  lbwd::out_norm_bwd_kernel<Tin, Tdy><<<kNormBwdCtas, 32 * lbwd::kNormWarps, 0, st>>>(
+      o, static_cast<const Tin*>(z), norm_w, static_cast<const Tdy*>(dy), d_o, dz, nw, rows, dv,
+      norm_eps);
+  lbwd::col_sum_kernel<<<(dv + 255) / 256, 256, 0, st>>>(nw, dnorm_w, (int)kNormBwdCtas, dv);
+  if (launch_status() != GDN_OK) return GDN_ERR_CUDA;
+  float* dqg = reinterpret_cast<float*>(ws + L.dq);
+  float* dkg = reinterpret_cast<float*>(ws + L.dk);
+  float* dvg = reinterpret_cast<float*>(ws + L.dv);
+  s = bwd_dispatch<Tin, float>(dk, qn, kn, vc, la, be, S0, d_o, dS_T, dqg, dkg, dvg, dla, dbeta,
+                               dS0, ws + L.bwd, B, T, Hk, Hv, scale, st);
+  if (s != GDN_OK) return s;
+  float* dpre = reinterpret_cast<float*>(ws + L.dpre);
+  float* cw = reinterpret_cast<float*>(ws + L.cw);
+  s = prologue_bwd_one<Tin>(q_raw, wq, dqg, dq_raw, dwq, dpre, cw, B, T, Hk, dk, true, l2_eps, st);
+  if (s == GDN_OK)
+    s = prologue_bwd_one<Tin>(k_raw, wk, dkg, dk_raw, dwk, dpre, cw, B, T, Hk, dk, true, l2_eps,
+                              st);
+  if (s == GDN_OK)
+    s = prologue_bwd_one<Tin>(v_raw, wv, dvg, dv_raw, dwv, dpre, cw, B, T, Hv, dv, false, 0.f, st);
+  return s;
+}
+}  // namespace
+
+extern "C" {
+
+size_t gdn_layer_bwd_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, int chunk,
+                                     gdn_dtype dtype) {
+  if (B <= 0 || T <= 0 || validate_heads(Hk, Hv, dk, dv) != GDN_OK || dk != dv ||
+      !valid_dtype(dtype) || !supported_chunk(chunk))
+    return 0;
+  return layer_bwd_layout(B, T, Hk, Hv, dk, dv, chunk, dtype).total;
+}
+
+gdn_status gdn_layer_bwd(const void* q_raw, const void* k_raw, const void* v_raw, const void* z,
+                         const float* wq, const float* wk, const float* wv,
+                         const float* log_alpha, const float* beta, const float* S0,
+                         const float* norm_w, const void* dy, const float* dS_T, float* dq_raw,
+                         float* dk_raw, float* dv_raw, float* dz, float* dwq, float* dwk,
+                         float* dwv, float* dlog_alpha, float* dbeta, float* dS0, float* dnorm_w,
+                         void* workspace, size_t workspace_bytes, int B, int T, int Hk, int Hv,
+                         int dk, int dv, int chunk, float scale, float l2_eps, float norm_eps,
+                         gdn_dtype dtype, gdn_dtype dy_dtype, gdn_stream_t stream) {
+  if (B < 0 || T < 0 || !valid_dtype(dtype) || !valid_dtype(dy_dtype)) return GDN_ERR_INVALID_ARG;
+  if (!io_pair_ok(dtype, dy_dtype)) return GDN_ERR_UNSUPPORTED;
+  gdn_status s = validate_heads(Hk, Hv, dk, dv);
+  if (s != GDN_OK) return s;
+  if (dk != dv) return GDN_ERR_UNSUPPORTED;
+  if (chunk <= 0 || !(norm_eps >= 0.f) || !(l2_eps >= 0.f)) return GDN_ERR_INVALID_ARG;
+  if (!supported_chunk(chunk)) return GDN_ERR_UNSUPPORTED;
+  const bool tc = tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16);
+  if (tc && !tc_chunk_length_ok(T)) return GDN_ERR_UNSUPPORTED;
+  if ((long)B * T == 0) return GDN_OK;
+  if (B > 65535 || (long)B * T * Hv > 0x7fffffffL * 8L) return GDN_ERR_UNSUPPORTED;
+  const void* in16[] = {q_raw, k_raw, v_raw, z, dy};
+  for (const void* p : in16)
+    if (!p || !aligned16(p)) return GDN_ERR_INVALID_ARG;
+  const void* in4[] = {wq, wk, wv, log_alpha, beta, norm_w, dq_raw, dk_raw, dv_raw, dz, dwq, dwk,
+                       dwv, dlog_alpha, dbeta, dnorm_w};
+  for (const void* p : in4)
+    if (!p || !aligned4(p)) return GDN_ERR_INVALID_ARG;
+  if (!opt_aligned16(S0) || !opt_aligned16(dS_T) || !opt_aligned16(dS0)) return GDN_ERR_INVALID_ARG;
+  const LayerBwdLayout L = layer_bwd_layout(B, T, Hk, Hv, dk, dv, chunk, dtype);
+  if (!workspace_ok(workspace, workspace_bytes, L.total)) return GDN_ERR_INVALID_ARG;
+  char* ws = static_cast<char*>(workspace);
+  if (dtype == GDN_F32)
+    return layer_bwd_run<float, float>(q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0,
+                                       norm_w, dy, dS_T, dq_raw, dk_raw, dv_raw, dz, dwq, dwk, dwv,
+                                       dlog_alpha, dbeta, dS0, dnorm_w, ws, L, B, T, Hk, Hv, dk,
+                                       dv, chunk, scale, l2_eps, norm_eps, dtype, stream);
+  if (dy_dtype == GDN_F32)
+    return layer_bwd_run<__nv_bfloat16, float>(
+        q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, dy, dS_T, dq_raw, dk_raw,
+        dv_raw, dz, dwq, dwk, dwv, dlog_alpha, dbeta, dS0, dnorm_w, ws, L, B, T, Hk, Hv, dk, dv,
+        chunk, scale, l2_eps, norm_eps, dtype, stream);
+  return layer_bwd_run<__nv_bfloat16, __nv_bfloat16>(
+      q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, dy, dS_T, dq_raw, dk_raw,
+      dv_raw, dz, dwq, dwk, dwv, dlog_alpha, dbeta, dS0, dnorm_w, ws, L, B, T, Hk, Hv, dk, dv,
+      chunk, scale, l2_eps, norm_eps, dtype, stream);
+}
+
+gdn_status gdn_gates_bwd(const void* ba, const float* dlog_alpha, const float* dbeta, float* dba,
+                         long long rows, int Hv, gdn_dtype dtype, gdn_stream_t stream) {
+  if (rows < 0 || Hv <= 0 || !valid_dtype(dtype)) return GDN_ERR_INVALID_ARG;
+  if (rows == 0) return GDN_OK;
+  if (!ba || !dlog_alpha || !dbeta || !dba || !aligned4(ba) || !aligned4(dlog_alpha) ||
+      !aligned4(dbeta) || !aligned4(dba))
+    return GDN_ERR_INVALID_ARG;
+  const long long n = rows * Hv, blocks = (n + 255) / 256;
+  if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == GDN_F32)
+    lbwd::gates_bwd_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(
+        (const float*)ba, dlog_alpha, dbeta, dba, rows, Hv);
+  else
+    lbwd::gates_bwd_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
+        (const __nv_bfloat16*)ba, dlog_alpha, dbeta, dba, rows, Hv);
   return launch_status();
 }
 

@@ -285,6 +285,44 @@ GDN_API int gdn_bwd_launches(int B, int T, int Hk, int Hv, int dk, int dv);
 /* Device scratch bytes gdn_bwd needs (host only, no CUDA call); 0 for invalid sizes. */
 GDN_API size_t gdn_bwd_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv);
 
+/*
+ * Backward of the whole layer of gdn_layer_fwd: gradients of <dy, y> + <dS_T, S_T> for every input
+ * and weight, by the chain rule through each piece ("L'attention hybride", "Les 48 couches Gated
+ * DeltaNet" and "Le décompte": conv kernel 4, swish output gate, one norm gain; "Les briques d'un
+ * réseau de neurones", 2. and 4.: SiLU, RMSNorm).  The forward is recomputed inside the call
+ * (prologue, then the recurrence with o in fp32); the bf16 rounding of the prologue's q, k, v
+ * passes the gradient unchanged.  Then the gated norm's backward (dO in fp32), gdn_bwd's work,
+ * and the prologue's: L2 norm (q, k), SiLU, the 4-tap convolution.
+ *   inputs as gdn_layer_fwd; dy [B, T, Hv * dv] (dy_dtype: dtype, or GDN_F32 for bf16 inputs);
+ *   dS_T [B, Hv, dk, dv] float or NULL
+ *   dq_raw, dk_raw [B, T, Hk * dk]; dv_raw, dz [B, T, Hv * dv]; dwq, dwk [Hk * dk, 4];
+ *   dwv [Hv * dv, 4]; dlog_alpha, dbeta [B, T, Hv]; dS0 [B, Hv, dk, dv] (nullable); dnorm_w [dv]
+ *   (all float outputs)
+ *   workspace: gdn_layer_bwd_workspace_bytes(...) bytes, 256-byte aligned, owned by the caller.
+ * dk == dv (else GDN_ERR_UNSUPPORTED); other limits as gdn_layer_fwd and gdn_bwd.  Weight
+ * gradients are sums of per-CTA partial sums taken in a fixed order (reproducible bit for bit).
+ */
+GDN_API gdn_status gdn_layer_bwd(const void *q_raw, const void *k_raw, const void *v_raw,
+                         const void *z, const float *wq, const float *wk, const float *wv,
+                         const float *log_alpha, const float *beta, const float *S0,
+                         const float *norm_w, const void *dy, const float *dS_T, float *dq_raw,
+                         float *dk_raw, float *dv_raw, float *dz, float *dwq, float *dwk,
+                         float *dwv, float *dlog_alpha, float *dbeta, float *dS0, float *dnorm_w,
+                         void *workspace, size_t workspace_bytes, int B, int T, int Hk, int Hv,
+                         int dk, int dv, int chunk, float scale, float l2_eps, float norm_eps,
+                         gdn_dtype dtype, gdn_dtype dy_dtype, gdn_stream_t stream);
+
+/* Device scratch bytes gdn_layer_bwd needs (host only, no CUDA call); 0 for invalid sizes. */
+GDN_API size_t gdn_layer_bwd_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv,
+                                             int chunk, gdn_dtype dtype);
+
+/*
+ * Backward of gdn_gates: dba [rows, 2*Hv] float, the b gradients dbeta beta (1 - beta) then the a
+ * gradients dlog_alpha sigmoid(-a) (d/da of log sigmoid(a)).  ba as gdn_gates (dtype).
+ */
+GDN_API gdn_status gdn_gates_bwd(const void *ba, const float *dlog_alpha, const float *dbeta,
+                         float *dba, long long rows, int Hv, gdn_dtype dtype, gdn_stream_t stream);
+
 /* Device scratch bytes gdn_chunk_fwd_varlen needs (host only, no CUDA call). */
 GDN_API size_t gdn_chunk_fwd_varlen_workspace_bytes(int nseq, int max_seqlen, int Hk, int Hv,
                                             int dk, int dv, int chunk, gdn_dtype dtype);

@@ -305,6 +305,43 @@ class OracleLib:
         return y, sT
 
 
+def _layer_backward(lib: "OracleLib", q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0,
+                    norm_w, dy, dS_T, Hk: int, Hv: int, dk: int, dv: int, l2_eps: float = 1e-6,
+                    norm_eps: float = 1e-5, scale: float = 1.0, threads: Optional[int] = None,
+                    act_dtype: str = "f64") -> dict:
+    """Gradients of <dy, y> + <dS_T, S_T> through layer_forward, composed from the pinned
+    backward pieces in reverse order: gated RMSNorm, recurrence, L2 normalisation (q, k), conv +
+    SiLU.  act_dtype "bf16": the recurrence runs on the bf16-rounded q, k, v and the gradient
+    passes the rounding unchanged."""
+    qc = lib.causal_conv_silu(q_raw, wq)
+    kc = lib.causal_conv_silu(k_raw, wk)
+    vc = lib.causal_conv_silu(v_raw, wv)
+    B, T = qc.shape[:2]
+    q = lib.l2_normalize(qc.reshape(B, T, Hk, dk), l2_eps)
+    k = lib.l2_normalize(kc.reshape(B, T, Hk, dk), l2_eps)
+    v = vc.reshape(B, T, Hv, dv)
+    if act_dtype == "bf16":
+        q, k, v = round_bf16(q), round_bf16(k), round_bf16(v)
+    elif act_dtype != "f64":
+        raise ValueError(act_dtype)
+    o, _ = lib.gated_delta(q, k, v, log_alpha, beta, S0, scale=scale, threads=threads)
+    do_, dz, dnw = lib.gated_rmsnorm_bwd(o, _f64(z).reshape(B, T, Hv, dv), norm_w,
+                                         _f64(dy).reshape(B, T, Hv, dv), norm_eps)
+    g = lib.gated_delta_bwd(q, k, v, log_alpha, beta, S0, do_, dS_T, scale=scale,
+                            threads=threads)
+    dqc = lib.l2_normalize_bwd(qc.reshape(B, T, Hk, dk), g["dq"], l2_eps).reshape(qc.shape)
+    dkc = lib.l2_normalize_bwd(kc.reshape(B, T, Hk, dk), g["dk"], l2_eps).reshape(kc.shape)
+    dq_raw, dwq = lib.causal_conv_silu_bwd(q_raw, wq, dqc)
+    dk_raw, dwk = lib.causal_conv_silu_bwd(k_raw, wk, dkc)
+    dv_raw, dwv = lib.causal_conv_silu_bwd(v_raw, wv, g["dv"].reshape(vc.shape))
+    return {"dq_raw": dq_raw, "dk_raw": dk_raw, "dv_raw": dv_raw, "dz": dz.reshape(_f64(z).shape),
+            "dwq": dwq, "dwk": dwk, "dwv": dwv, "dlog_alpha": g["dlog_alpha"],
+            "dbeta": g["dbeta"], "dS0": g["dS0"], "dnorm_w": dnw}
+
+
+OracleLib.layer_backward = _layer_backward
+
+
 def _gated_delta_varlen(lib: "OracleLib", q, k, v, log_alpha, beta, cu_seqlens, S0=None,
                         scale: float = 1.0, threads: Optional[int] = None):
     """Packed sequences: q,k [total,Hk,dk]; v [total,Hv,dv]; gates [total,Hv]; sequence s is
@@ -436,3 +473,7 @@ def gated_rmsnorm_bwd(*a, **kw):
 
 def gates_bwd(*a, **kw):
     return get().gates_bwd(*a, **kw)
+
+
+def layer_backward(*a, **kw):
+    return get().layer_backward(*a, **kw)

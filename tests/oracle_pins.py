@@ -525,4 +525,33 @@ def pin_bwd_gates_central_differences(orc):
     _close(dba, _central(f, ba))
 
 
+def pin_bwd_layer_central_differences(orc):
+    """The composed layer backward equals central differences of the composed layer forward on a
+    tiny layer (two value heads per key head), for the raw inputs, the conv taps, the gates and
+    the norm gain (fp64 activations: the composition itself, not the bf16 rounding)."""
+    rng = np.random.default_rng(55)
+    B, T, Hk, Hv, d = 1, 5, 1, 2, 3
+    q_raw = rng.standard_normal((B, T, Hk * d))
+    k_raw = rng.standard_normal((B, T, Hk * d))
+    v_raw = rng.standard_normal((B, T, Hv * d))
+    z = rng.standard_normal((B, T, Hv * d))
+    wq, wk, wv = (rng.standard_normal((c, 4)) * 0.5 for c in (Hk * d, Hk * d, Hv * d))
+    la = -np.log1p(np.exp(rng.standard_normal((B, T, Hv)))) * 0.3
+    be = expit(rng.standard_normal((B, T, Hv)))
+    S0 = rng.standard_normal((B, Hv, d, d)) * 0.3
+    nw = 1.0 + 0.1 * rng.standard_normal(d)
+    dy = rng.standard_normal((B, T, Hv, d))
+    dST = rng.standard_normal((B, Hv, d, d)) * 0.1
+    kw = dict(Hk=Hk, Hv=Hv, dk=d, dv=d, l2_eps=1e-6, norm_eps=1e-5, scale=0.7, threads=1)
+    g = orc.layer_backward(q_raw, k_raw, v_raw, z, wq, wk, wv, la, be, S0, nw, dy, dST, **kw)
+
+    def f():
+        y, sT = orc.layer_forward(q_raw, k_raw, v_raw, z, wq, wk, wv, la, be, S0, nw, **kw)
+        return float(np.sum(dy * y) + np.sum(dST * sT))
+    for name, x in (("dq_raw", q_raw), ("dk_raw", k_raw), ("dv_raw", v_raw), ("dz", z),
+                    ("dwq", wq), ("dwv", wv), ("dlog_alpha", la), ("dbeta", be), ("dS0", S0),
+                    ("dnorm_w", nw)):
+        _close(g[name], _central(f, x), tol=1e-6)
+
+
 ALL_PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]
