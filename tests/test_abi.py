@@ -261,3 +261,35 @@ def test_bwd_workspace_bytes(L):
 def test_bwd_validation(L, kw, expect):
     """gdn_bwd rejects bad arguments before any work (the pointers are fakes, never read)."""
     assert bwd(L, **kw) == expect
+
+
+def layer_bwd(L, B=1, T=64, Hk=2, Hv=4, dk=64, dv=64, dtype=1, dyt=1, ws=None, ws_bytes=0,
+              q_raw=FAKE):
+    p = [q_raw] + [FAKE] * 23           # 13 inputs, then 11 outputs
+    p[12] = None          # dS_T
+    p[22] = None          # dS0
+    return L.gdn_layer_bwd(*p, ws, ws_bytes, B, T, Hk, Hv, dk, dv, 64, 1.0, 1e-6, 1e-5, dtype,
+                           dyt, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(B=-1), 1), (dict(Hv=3), 1), (dict(dtype=7), 1), (dict(dyt=7), 1),
+    (dict(dtype=0, dyt=1), 2),                       # fp32 inputs, bf16 dy
+    (dict(dk=64, dv=32), 2), (dict(dk=48, dv=48), 2),
+    (dict(q_raw=None), 1), (dict(q_raw=P(0x1004)), 1),
+    (dict(), 1),                                     # no workspace
+    (dict(B=0), 0), (dict(T=0), 0),
+])
+def test_layer_bwd_validation(L, kw, expect):
+    """gdn_layer_bwd rejects bad arguments before any work (fake pointers, never read)."""
+    assert layer_bwd(L, **kw) == expect
+
+
+def test_layer_bwd_workspace_and_gates_bwd_validation(L):
+    assert L.gdn_layer_bwd_workspace_bytes(1, 64, 2, 4, 64, 64, 64, 1) > \
+        L.gdn_layer_workspace_bytes(1, 64, 2, 4, 64, 64, 64, 1)
+    assert L.gdn_layer_bwd_workspace_bytes(1, 64, 2, 4, 64, 32, 64, 1) == 0
+    assert L.gdn_layer_bwd_workspace_bytes(0, 64, 2, 4, 64, 64, 64, 1) == 0
+    assert L.gdn_gates_bwd(FAKE, FAKE, FAKE, FAKE, -1, 4, 1, None) == 1
+    assert L.gdn_gates_bwd(None, FAKE, FAKE, FAKE, 10, 4, 1, None) == 1
+    assert L.gdn_gates_bwd(FAKE, FAKE, FAKE, FAKE, 0, 4, 1, None) == 0
