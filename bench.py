@@ -438,6 +438,35 @@ def bench_backward(gdn, dev, warmup, flush, steps=5):
             "workload": "backward " + workload_name(w)}
 
 
+def bench_layer_backward(gdn, dev, warmup, flush, steps=3):
+    """The whole layer's backward (gdn_layer_bwd, forward recomputed inside) on the 8:1 layer
+    workload, dy ~ N(0, 1) bf16, dS_T ~ N(0, 0.1).  Work counted: the recurrence backward's
+    (bwd_flops); the recomputed forward and the elementwise pieces ride on top."""
+    w = gi.WORKLOADS["layer_8to1"]
+    x = gi.make_layer_inputs(w)
+    d = to_dev(x, dev)
+    g = torch.Generator().manual_seed(w.seed + 3)
+    dy = torch.randn(w.B, w.T, w.Hv, w.dv, generator=g).to(w.torch_dtype).to(dev)
+    dST = (torch.randn(w.B, w.Hv, w.dk, w.dv, generator=g) * 0.1).to(dev)
+    ws = torch.empty(gdn.layer_bwd_workspace_bytes(w.B, w.T, w.Hk, w.Hv, w.dk, w.dv, w.chunk,
+                                                   w.torch_dtype), device=dev, dtype=torch.uint8)
+
+    def step():
+        gdn.layer_bwd(d["q_raw"], d["k_raw"], d["v_raw"], d["z"], d["conv_wq"], d["conv_wk"],
+                      d["conv_wv"], d["log_alpha"], d["beta"], d["S0"], d["norm_w"], dy, dST,
+                      Hk=w.Hk, Hv=w.Hv, dk=w.dk, dv=w.dv, chunk=w.chunk, workspace=ws)
+    ms = time_steps(step, steps, warmup, flush, 1)
+    t = statistics.mean(ms) / 1e3
+    F = bwd_flops(w)
+    peak = fp32_peak_tflops(dev)
+    return {"value": w.B * w.T / t, "unit": "tokens/s", "ms_per_step": t * 1e3, "steps": steps,
+            "roofline": {"bound": "alu", "achieved": F / t / 1e12, "peak": peak,
+                         "unit": "TFLOP/s", "frac": F / t / 1e12 / peak, "traffic": None,
+                         "kernel": "bwd_kernel", "algorithmic_flops": F,
+                         "peak_source": "derived: SMs x 128 fp32 lanes x 2 x 1965 MHz"},
+            "workspace_bytes": ws.numel(), "workload": "layer backward " + workload_name(w)}
+
+
 def bench_layer(gdn, dev, warmup, flush, peaks, steps=10):
     w = gi.WORKLOADS["layer_8to1"]
     x = gi.make_layer_inputs(w)
@@ -817,6 +846,8 @@ def main():
             sec["layer_8to1"] = bench_layer(gdn, dev, 3, flush, peaks, steps=10)
             torch.cuda.empty_cache()
             sec["backward"] = bench_backward(gdn, dev, 3, flush, steps=5)
+            torch.cuda.empty_cache()
+            sec["layer_backward"] = bench_layer_backward(gdn, dev, 3, flush, steps=3)
             line["secondary"] = sec
         if not args.no_cpu_baseline and world == 1:
             cb = oracle_sample_rate(x, w, target_s=10.0)
