@@ -83,3 +83,15 @@ def test_gates_bwd(orc):
     torch.cuda.synchronize()
     r = orc.gates_bwd(ba, dla, db)
     assert rel_rms(out, r) <= 1e-5
+
+
+def test_layer_bwd_8to1_heads(orc):
+    """The 8:1 layer's heads (Hk16 Hv128 d128, bf16) at B1 T256: dq, dk sum 8 value heads x 4
+    column slices per key head."""
+    w, x, dy, dST = layer_case(1, 256, 16, 128, 128, "bf16", 9)
+    out = run(w, x, dy, dST)
+    r = ref(orc, w, x, dy, dST, "bf16")
+    e = {n: rel_rms(out[n], r[n]) for n in NAMES}
+    report("layer_bwd_8to1_B1_T256", **e)
+    for n in NAMES:
+        assert e[n] <= TOL_BF16_OUT, (n, e[n])
