@@ -143,11 +143,41 @@ __device__ __forceinline__ void load_segment(Smem<D>& sm, const Tin* __restrict_
   }
 }
 
-// One thread's share of a state: rows i0 .. i0 + RL - 1, columns j0 .. j0 + CW - 1.
+// Two fp32 lanes in one 64-bit register pair for the paired fp32 instructions of sm_100 (each lane
+// is the IEEE round-to-nearest operation of its scalar counterpart).
+using f2_t = unsigned long long;
+__device__ __forceinline__ f2_t pk2(float a, float b) {
+  f2_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void up2(f2_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ f2_t fma2(f2_t a, f2_t b, f2_t c) {   // a b + c
+  f2_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ f2_t mul2(f2_t a, f2_t b) {
+  f2_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ f2_t splat2(float a) { return pk2(a, a); }
+__device__ __forceinline__ float hsum2(f2_t r) {
+  float a, b;
+  up2(r, a, b);
+  return a + b;
+}
+
+// One thread's share of a state: rows i0 .. i0 + RL - 1, columns j0 .. j0 + CW - 1, held as
+// column pairs (c, c + 1).
 template <int D>
 struct Tile {
   using Sh = Shape<D>;
-  float m[Sh::RL][Sh::CW];
+  static_assert(Sh::CW % 2 == 0, "column pairs");
+  f2_t m[Sh::RL][Sh::CW / 2];
 };
 
 // grid: B * Hv * NS CTAs ((b * Hv + h) * NS + column slice); block Shape<D>::NT; dynamic shared
@@ -165,8 +195,8 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
            float* __restrict__ dla_out, float* __restrict__ dbeta_out, float* __restrict__ dS0,
            float* __restrict__ ckpt, int T, int Hk, int Hv, float scale) {
   using Sh = Shape<D>;
-  constexpr int RL = Sh::RL, CW = Sh::CW, LR = Sh::LR, NT = Sh::NT, SL = Sh::SL, VPT = Sh::VPT;
-  constexpr int NS = Sh::NS, DC = Sh::DC;
+  constexpr int RL = Sh::RL, CW = Sh::CW, CP = CW / 2, LR = Sh::LR, NT = Sh::NT, SL = Sh::SL;
+  constexpr int NS = Sh::NS, DC = Sh::DC, PPT = RL * CP;   // column pairs per thread
   extern __shared__ __align__(16) unsigned char bwd_smem[];
   Smem<D>& sm = *reinterpret_cast<Smem<D>*>(bwd_smem);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -183,63 +213,68 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
   float* const ck = ckpt + (long)blockIdx.x * nseg * D * DC;
   const long sbase = bh * (long)D * D;               // [dk][dv] slot of S0, dS_T, dS0
 
-  // a state in the [dk][dv] order of S0 / dS_T / dS0, and in the per-thread order of the
-  // checkpoints and the shared-memory copies
+  // a state in the [dk][dv] order of S0 / dS_T / dS0 (8-byte pairs: j0 and CW are even), and in
+  // the per-thread order of the checkpoints and the shared-memory copies (pair p of thread t at
+  // (p * NT + t) * 2)
   auto get_sq = [&](const float* base, Tile<D>& M) {
 #pragma unroll
     for (int r = 0; r < RL; ++r)
 #pragma unroll
-      for (int c = 0; c < CW; ++c) M.m[r][c] = base[(long)(i0 + r) * D + j0 + c];
+      for (int c = 0; c < CP; ++c)
+        M.m[r][c] = *reinterpret_cast<const f2_t*>(base + (long)(i0 + r) * D + j0 + 2 * c);
   };
   auto put_sq = [&](float* base, const Tile<D>& M) {
 #pragma unroll
     for (int r = 0; r < RL; ++r)
 #pragma unroll
-      for (int c = 0; c < CW; ++c) base[(long)(i0 + r) * D + j0 + c] = M.m[r][c];
+      for (int c = 0; c < CP; ++c)
+        *reinterpret_cast<f2_t*>(base + (long)(i0 + r) * D + j0 + 2 * c) = M.m[r][c];
   };
-  // (pairs of elements: element 2e, 2e + 1 of thread t at (e * NT + t) * 2, one 8-byte access)
   auto get_pt = [&](const float* base, Tile<D>& M) {
 #pragma unroll
-    for (int e = 0; e < VPT / 2; ++e) {
-      const float2 p = *reinterpret_cast<const float2*>(base + ((long)e * NT + tid) * 2);
-      M.m[(2 * e) / CW][(2 * e) % CW] = p.x;
-      M.m[(2 * e + 1) / CW][(2 * e + 1) % CW] = p.y;
-    }
+    for (int e = 0; e < PPT; ++e)
+      M.m[e / CP][e % CP] = *reinterpret_cast<const f2_t*>(base + ((long)e * NT + tid) * 2);
   };
   auto put_pt = [&](float* base, const Tile<D>& M) {
 #pragma unroll
-    for (int e = 0; e < VPT / 2; ++e)
-      *reinterpret_cast<float2*>(base + ((long)e * NT + tid) * 2) =
-          make_float2(M.m[(2 * e) / CW][(2 * e) % CW], M.m[(2 * e + 1) / CW][(2 * e + 1) % CW]);
+    for (int e = 0; e < PPT; ++e)
+      *reinterpret_cast<f2_t*>(base + ((long)e * NT + tid) * 2) = M.m[e / CP][e % CP];
+  };
+  auto zero = [&](Tile<D>& M) {
+#pragma unroll
+    for (int e = 0; e < PPT; ++e) M.m[e / CP][e % CP] = 0ull;
   };
   // one token of the recurrence: x = S k (inside the warp), S <- alpha S + k (beta (v - alpha x))^T
   auto fwd_step = [&](Tile<D>& M, int j) {
     const float a = sm.alpha[j], be = sm.beta[j];
-    float kk[RL], x[CW];
+    f2_t kk[RL], xp[CP];
 #pragma unroll
-    for (int r = 0; r < RL; ++r) kk[r] = sm.k[j][i0 + r];
+    for (int r = 0; r < RL; ++r) kk[r] = splat2(sm.k[j][i0 + r]);
 #pragma unroll
-    for (int c = 0; c < CW; ++c) {
-      float acc = 0.f;
+    for (int c = 0; c < CP; ++c) {
+      f2_t acc = 0ull;
 #pragma unroll
-      for (int r = 0; r < RL; ++r) acc = fmaf(M.m[r][c], kk[r], acc);
-      x[c] = acc;
+      for (int r = 0; r < RL; ++r) acc = fma2(M.m[r][c], kk[r], acc);
+      xp[c] = acc;
     }
+    float x[CW];
+#pragma unroll
+    for (int c = 0; c < CP; ++c) up2(xp[c], x[2 * c], x[2 * c + 1]);
     allreduce<CW, LR>(x, lane);
+    const f2_t a2 = splat2(a);
 #pragma unroll
-    for (int c = 0; c < CW; ++c) {
-      const float w = be * fmaf(-a, x[c], sm.v[j][jl + c]);
+    for (int c = 0; c < CP; ++c) {
+      const f2_t w = pk2(be * fmaf(-a, x[2 * c], sm.v[j][jl + 2 * c]),
+                         be * fmaf(-a, x[2 * c + 1], sm.v[j][jl + 2 * c + 1]));
 #pragma unroll
-      for (int r = 0; r < RL; ++r) M.m[r][c] = fmaf(a, M.m[r][c], kk[r] * w);
+      for (int r = 0; r < RL; ++r) M.m[r][c] = fma2(a2, M.m[r][c], mul2(kk[r], w));
     }
   };
 
   // pass 1: the recurrence forward, the state before every segment kept
   Tile<D> M, G;
   if (S0) get_sq(S0 + sbase, M);
-  else
-#pragma unroll
-    for (int e = 0; e < VPT; ++e) M.m[e / CW][e % CW] = 0.f;
+  else zero(M);
   for (int sg = 0; sg < nseg; ++sg) {
     const int t0 = sg * kSeg, len = min(kSeg, T - t0);
     __syncthreads();                                 // the previous segment's data is read
@@ -251,9 +286,7 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
 
   // pass 2: segments last to first, tokens last to first
   if (dS_T) get_sq(dS_T + sbase, G);
-  else
-#pragma unroll
-    for (int e = 0; e < VPT; ++e) G.m[e / CW][e % CW] = 0.f;
+  else zero(G);
   // the per-slice partials of tokens t0 + jb .. t0 + je - 1, summed into the outputs
   auto flush = [&](int t0, int jb, int je) {
     __syncthreads();
@@ -297,68 +330,74 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
       else { get_pt(sm.state0, M); j0s = 0; }
       for (int u = j0s; u < j; ++u) fwd_step(M, u);
       const float a = sm.alpha[j], be = sm.beta[j];
-      float kk[RL], qs[RL], vv[CW], dd[CW], xg[2 * CW];
+      f2_t kk[RL], qs[RL], dd[CP];
 #pragma unroll
       for (int r = 0; r < RL; ++r) {
-        kk[r] = sm.k[j][i0 + r];
-        qs[r] = scale * sm.q[j][i0 + r];
+        kk[r] = splat2(sm.k[j][i0 + r]);
+        qs[r] = splat2(scale * sm.q[j][i0 + r]);
       }
 #pragma unroll
-      for (int c = 0; c < CW; ++c) {
-        vv[c] = sm.v[j][jl + c];
-        dd[c] = sm.dO[j][jl + c];
-      }
+      for (int c = 0; c < CP; ++c) dd[c] = pk2(sm.dO[j][jl + 2 * c], sm.dO[j][jl + 2 * c + 1]);
       // G += scale dO q^T; x = P k and Gk = G k (sums over dk, in the warp); <G, P> partial
-      float gp = 0.f;
+      f2_t gp2 = 0ull;
+      float xg[2 * CW];
 #pragma unroll
-      for (int c = 0; c < CW; ++c) {
-        float ax = 0.f, ag = 0.f;
+      for (int c = 0; c < CP; ++c) {
+        f2_t ax = 0ull, ag = 0ull;
 #pragma unroll
         for (int r = 0; r < RL; ++r) {
-          G.m[r][c] = fmaf(qs[r], dd[c], G.m[r][c]);
-          ax = fmaf(M.m[r][c], kk[r], ax);
-          ag = fmaf(G.m[r][c], kk[r], ag);
-          gp = fmaf(G.m[r][c], M.m[r][c], gp);
+          G.m[r][c] = fma2(qs[r], dd[c], G.m[r][c]);
+          ax = fma2(M.m[r][c], kk[r], ax);
+          ag = fma2(G.m[r][c], kk[r], ag);
+          gp2 = fma2(G.m[r][c], M.m[r][c], gp2);
         }
-        xg[c] = ax;
-        xg[CW + c] = ag;
+        up2(ax, xg[2 * c], xg[2 * c + 1]);
+        up2(ag, xg[CW + 2 * c], xg[CW + 2 * c + 1]);
       }
       allreduce<2 * CW, LR>(xg, lane);
-      gp = group_sum<LR>(gp);
-      float u[CW], w[CW], dx[CW], ug = 0.f, xgk = 0.f;
+      const float gp = group_sum<LR>(hsum2(gp2));
+      f2_t w2[CP], dx2[CP];
+      float ug = 0.f, xgk = 0.f, gk[CW];
 #pragma unroll
       for (int c = 0; c < CW; ++c) {
-        u[c] = fmaf(-a, xg[c], vv[c]);                 // v - alpha x
-        w[c] = be * u[c];                              // S_t = alpha P + k w^T
-        dx[c] = -a * be * xg[CW + c];
-        ug = fmaf(u[c], xg[CW + c], ug);
-        xgk = fmaf(xg[c], xg[CW + c], xgk);
+        gk[c] = xg[CW + c];
+        const float uc = fmaf(-a, xg[c], sm.v[j][jl + c]);     // v - alpha x
+        ug = fmaf(uc, gk[c], ug);
+        xgk = fmaf(xg[c], gk[c], xgk);
+      }
+#pragma unroll
+      for (int c = 0; c < CP; ++c) {
+        const float u0 = fmaf(-a, xg[2 * c], sm.v[j][jl + 2 * c]);
+        const float u1 = fmaf(-a, xg[2 * c + 1], sm.v[j][jl + 2 * c + 1]);
+        w2[c] = pk2(be * u0, be * u1);                  // S_t = alpha P + k w^T
+        dx2[c] = pk2(-a * be * gk[2 * c], -a * be * gk[2 * c + 1]);
       }
       // per-slice partials: dq = scale S_t^T dO, dk = beta G^T (v - alpha x) + P^T dx
       const int hj = j % kHalf;
+      const f2_t a2 = splat2(a);
 #pragma unroll
       for (int r = 0; r < RL; ++r) {
-        float pq = 0.f, pk = 0.f;
+        f2_t pq = 0ull, pkk = 0ull;
 #pragma unroll
-        for (int c = 0; c < CW; ++c) {
-          pq = fmaf(fmaf(a, M.m[r][c], kk[r] * w[c]), dd[c], pq);
-          pk = fmaf(G.m[r][c], w[c], fmaf(M.m[r][c], dx[c], pk));   // beta G u = G w
+        for (int c = 0; c < CP; ++c) {
+          pq = fma2(fma2(a2, M.m[r][c], mul2(kk[r], w2[c])), dd[c], pq);
+          pkk = fma2(G.m[r][c], w2[c], fma2(M.m[r][c], dx2[c], pkk));   // beta G u = G w
         }
-        sm.pdq[hj][sl][i0 + r] = scale * pq;
-        sm.pdk[hj][sl][i0 + r] = pk;
+        sm.pdq[hj][sl][i0 + r] = scale * hsum2(pq);
+        sm.pdk[hj][sl][i0 + r] = hsum2(pkk);
       }
       if (lr == 0) {
         sm.pa[hj][sl] = gp - be * xgk;                // this slice's <G, P - beta x k^T>
         sm.pb[hj][sl] = ug;
 #pragma unroll
         for (int c = 0; c < CW; ++c)
-          dv_out[((b * T + t0 + j) * Hv + h) * (long)D + j0 + c] = be * xg[CW + c];
+          dv_out[((b * T + t0 + j) * Hv + h) * (long)D + j0 + c] = be * gk[c];
       }
       // the gradient reaching S_{t-1}: alpha G + dx k^T
 #pragma unroll
-      for (int c = 0; c < CW; ++c)
+      for (int c = 0; c < CP; ++c)
 #pragma unroll
-        for (int r = 0; r < RL; ++r) G.m[r][c] = fmaf(a, G.m[r][c], kk[r] * dx[c]);
+        for (int r = 0; r < RL; ++r) G.m[r][c] = fma2(a2, G.m[r][c], mul2(kk[r], dx2[c]));
       if (j == kHalf) flush(t0, kHalf, len);
       if (j == 0) flush(t0, 0, min(len, kHalf));
     }
