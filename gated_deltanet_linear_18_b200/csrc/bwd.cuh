@@ -143,34 +143,6 @@ __device__ __forceinline__ void load_segment(Smem<D>& sm, const Tin* __restrict_
   }
 }
 
-// Two fp32 lanes in one 64-bit register pair for the paired fp32 instructions of sm_100 (each lane
-// is the IEEE round-to-nearest operation of its scalar counterpart).
-using f2_t = unsigned long long;
-__device__ __forceinline__ f2_t pk2(float a, float b) {
-  f2_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ void up2(f2_t r, float& a, float& b) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
-}
-__device__ __forceinline__ f2_t fma2(f2_t a, f2_t b, f2_t c) {   // a b + c
-  f2_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ f2_t mul2(f2_t a, f2_t b) {
-  f2_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ f2_t splat2(float a) { return pk2(a, a); }
-__device__ __forceinline__ float hsum2(f2_t r) {
-  float a, b;
-  up2(r, a, b);
-  return a + b;
-}
-
 // One thread's share of a state: rows i0 .. i0 + RL - 1, columns j0 .. j0 + CW - 1, held as
 // column pairs (c, c + 1).
 template <int D>

@@ -95,9 +95,9 @@ template <typename Tio>
 __device__ __forceinline__ void prologue_stage(Tio* tile, const Tio* xh, long t0, int T, int width,
                                                int d) {
   constexpr int N = Vec16<Tio>::N;
-  const int L = d / N;
+  const int L = d / N, lgL = __ffs(L) - 1;    // 16-byte pieces per row (a power of two)
   for (int i = threadIdx.x; i < (kPrologueTokens + 3) * L; i += blockDim.x) {
-    const int r = i / L, c = i - r * L;
+    const int r = i >> lgL, c = i & (L - 1);
     const long t = t0 - 3 + r;
     const bool in = t >= 0 && t < T;
     const Tio* src = in ? xh + t * width + c * N : xh;
@@ -108,26 +108,62 @@ __device__ __forceinline__ void prologue_stage(Tio* tile, const Tio* xh, long t0
   asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
 }
 
+// Vectors of 4 values: 16 bytes of fp32 or 8 of bf16.
+template <typename T4> struct Vec4;
+template <> struct Vec4<float> {
+  static __device__ __forceinline__ void load(const float* p, float (&v)[4]) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  }
+  static __device__ __forceinline__ void store(float* p, const float (&v)[4]) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+};
+template <> struct Vec4<__nv_bfloat16> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[4]) {
+    const uint2 a = *reinterpret_cast<const uint2*>(p);
+    v[0] = __uint_as_float(a.x << 16); v[1] = __uint_as_float(a.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(a.y << 16); v[3] = __uint_as_float(a.y & 0xFFFF0000u);
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[4]) {
+    __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]), h1 = __floats2bfloat162_rn(v[2], v[3]);
+    *reinterpret_cast<uint2*>(p) =
+        make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
+  }
+};
+
+// Whether every value within 2^-24 E of y rounds to the same bf16 value as y, tested as: the
+// midpoint next to y's truncation to bf16 (low 16 bits 0x8000; the cell boundary nearest y unless y
+// sits at the start of its binade) is farther than twice that.  Every other boundary is at least
+// half that distance away (the nearest one below a binade's start, where the cell below is half
+// as wide, included), so all are farther than 2^-24 E.  The scaling by 2^23 is exact; E = 0 (an
+// exact y) is decided, NaN never.
+__device__ __forceinline__ bool bf16_decided_e24(float y, float E) {
+  const float mid = __uint_as_float((__float_as_uint(y) & 0xFFFF0000u) | 0x8000u);
+  return fabsf(y - mid) * 8388608.0f > E;
+}
+
 // Prologue of the v channels (no normalisation): grid (Hv, ceil(T / kPrologueTokens), B), head
 // slots fastest, so that CTAs that run together read neighbouring parts of the same token rows;
 // block: 128 threads.  One CTA takes one head of dv channels over kPrologueTokens tokens: a head
-// row is held by L = dv / N threads (N channels of one 16-byte vector each) and the 128 / L row
-// groups take consecutive spans of tokens, carrying the conv window in registers.
+// row is held by L = dv / 4 threads (4 channels each) and the 128 / L row groups take consecutive
+// spans of tokens, carrying the conv window in registers (a ring of four rows).
 //
 // bf16 outputs: rounding to bf16 is a quantising decision, taken here as the exact result would
-// take it, i.e. as rounding the fp64 value does.  Each fp32 value y carries a bound E on its
-// distance from the exact value: the convolution's 4-term fp32 sum (at most about 4 units of
-// roundoff of sum |w x|, carried through SiLU' <= 1.1), the rounding of the exponent's argument
-// (|x| units, relative), the budgets of ex2.approx and rcp.approx and one unit per remaining
-// operation.  Values with a rounding boundary within 2E are redone in fp64 after the tile is
-// stored, from a list in shared memory (so the rare fp64 work does not diverge the common path).
+// take it, i.e. as rounding the fp64 value does.  The fp32 value s = SiLU(pre) is within
+// 2^-24 ((20 + 2 |pre|) |s| + 1.2 P) of the exact value, P = |p0| + |p1| + |p2| + |pre| the
+// magnitudes of the conv's partial sums (each of its four FMAs rounds once, by at most a unit of
+// its result, carried through SiLU' <= 1.1): the exponent's argument rounds with the constant
+// log2 e (2 |pre| units of s, relative), ex2.approx and rcp.approx are budgeted 8 units each (more
+// than the maximum errors the PTX ISA documents), the remaining operations one unit each.
+// Values whose rounding that leaves open (about 0.2 %, bf16_decided_e24) are marked in a
+// per-thread bit mask, gathered into a shared-memory list after the loop and redone in fp64 after
+// the tile is stored, so the rare fp64 work and its bookkeeping stay off the common path.
 template <typename Tio>
 __global__ void __launch_bounds__(128, 6)
 prologue_v_kernel(const Tio* __restrict__ x, const float* __restrict__ w, Tio* __restrict__ y,
                   int T, int Hv, int dv) {
-  constexpr int N = Vec16<Tio>::N;
   constexpr bool kBf16 = sizeof(Tio) == 2;
-  constexpr float u = 5.9604645e-8f;          // 2^-24, the unit roundoff of fp32
   extern __shared__ __align__(16) uint8_t pro_smem[];
   Tio* tile = reinterpret_cast<Tio*>(pro_smem);
   __shared__ uint16_t list[kPrologueList];    // undecided (token << 8 | channel)
@@ -135,51 +171,65 @@ prologue_v_kernel(const Tio* __restrict__ x, const float* __restrict__ w, Tio* _
   const int head = blockIdx.x, d = dv, width = Hv * dv;
   const long b = blockIdx.z;
   const long t0 = (long)blockIdx.y * kPrologueTokens;
-  const int L = d / N, grp = threadIdx.x / L, lc = threadIdx.x % L, ngrp = 128 / L;
+  const int L = d / 4, grp = threadIdx.x / L, lc = threadIdx.x % L, ngrp = 128 / L;
   const int tpg = kPrologueTokens / ngrp, i0 = grp * tpg;  // this row group's tokens
   if (threadIdx.x == 0) nlist = 0;
   prologue_stage(tile, x + b * T * (long)width + (long)head * d, t0, T, width, d);
-  const long c0 = (long)head * d + lc * N;    // first channel of this thread
-  float wt[N][4];
+  const long c0 = (long)head * d + lc * 4;    // first channel of this thread
+  float wk[4][4];                             // [channel][tap]
 #pragma unroll
-  for (int i = 0; i < N; ++i)                 // weights need only 4-byte alignment
+  for (int c = 0; c < 4; ++c)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) wt[i][j] = w[(c0 + i) * 4 + j];
+    for (int k = 0; k < 4; ++k) wk[c][k] = w[(c0 + c) * 4 + k];   // 4-byte alignment only
   __syncthreads();
   const long rem = T - t0;
   const int nt = rem < kPrologueTokens ? (int)rem : kPrologueTokens;
   Tio* const yt = y + (b * T + t0) * width + c0;          // this thread's channels of token t0
-  float h0[N], h1[N], h2[N];                  // the window: rows i, i + 1, i + 2 of token i
-  Vec16<Tio>::load(tile + (long)i0 * d + lc * N, h0);
-  Vec16<Tio>::load(tile + (long)(i0 + 1) * d + lc * N, h1);
-  Vec16<Tio>::load(tile + (long)(i0 + 2) * d + lc * N, h2);
-#pragma unroll 4
-  for (int tt = 0; tt < tpg; ++tt) {
-    const int i = i0 + tt;
-    float h3[N], yv_[N];
-    Vec16<Tio>::load(tile + (long)(i + 3) * d + lc * N, h3);
+  const Tio* const xr = tile + lc * 4;                    // ... of tile row 0
+  // token i reads tile rows i .. i + 3 at ring slots i .. i + 3 (mod 4): with the token loop
+  // unrolled by four no row is ever moved
+  float h[4][4];
 #pragma unroll
-    for (int j = 0; j < N; ++j) {
-      const float pre = fmaf(wt[j][3], h3[j], fmaf(wt[j][2], h2[j],
-                                                   fmaf(wt[j][1], h1[j], wt[j][0] * h0[j])));
-      // SiLU(pre) = pre / (1 + 2^(-pre log2 e))
-      const float s = pre * rcp_fast(1.0f + ex2_fast(pre * -1.4426950408889634f));
-      yv_[j] = s;
-      if constexpr (kBf16) {
-        const float A = fmaf(fabsf(wt[j][3]), fabsf(h3[j]),
-                             fmaf(fabsf(wt[j][2]), fabsf(h2[j]),
-                                  fmaf(fabsf(wt[j][1]), fabsf(h1[j]), fabsf(wt[j][0]) * fabsf(h0[j]))));
-        const float e = 2.0f * u * fmaf(21.0f + fabsf(pre), fabsf(s), 6.0f * A);
-        if (!bf16_decided(s, e)) {
-          const int k = atomicAdd(&nlist, 1);
-          if (k < kPrologueList) list[k] = (uint16_t)((i << 8) | (lc * N + j));
+  for (int r = 0; r < 3; ++r) Vec4<Tio>::load(xr + (long)(i0 + r) * d, h[r]);
+  unsigned long long umask = 0ull;            // undecided values: bit 4 (i - i0) + channel
+#pragma unroll 1
+  for (int t4 = 0; t4 < tpg; t4 += 4) {
+    unsigned m16 = 0u;
+#pragma unroll
+    for (int sl = 0; sl < 4; ++sl) {
+      if (t4 + sl >= tpg) break;              // tpg = 2 for 16-channel heads
+      const int i = i0 + t4 + sl;
+      const int r0 = sl, r1 = (sl + 1) & 3, r2 = (sl + 2) & 3, r3 = (sl + 3) & 3;
+      Vec4<Tio>::load(xr + (long)(i + 3) * d, h[r3]);
+      float yv_[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float p0 = wk[j][0] * h[r0][j];
+        const float p1 = fmaf(wk[j][1], h[r1][j], p0);
+        const float p2 = fmaf(wk[j][2], h[r2][j], p1);
+        const float pre = fmaf(wk[j][3], h[r3][j], p2);
+        // SiLU(pre) = pre / (1 + 2^(-pre log2 e))
+        const float sv = pre * rcp_fast(1.0f + ex2_fast(pre * -1.4426950408889634f));
+        yv_[j] = sv;
+        if constexpr (kBf16) {
+          // half the bound's bracket: 10 |s| + pre s + 0.6 P (pre s = |pre| |s|)
+          const float P = (fabsf(p0) + fabsf(p1)) + (fabsf(p2) + fabsf(pre));
+          const float E = fmaf(pre, sv, fmaf(P, 0.6f, 10.0f * fabsf(sv)));
+          if (!bf16_decided_e24(sv, E + E)) m16 |= 1u << (sl * 4 + j);
         }
       }
-      h0[j] = h1[j]; h1[j] = h2[j]; h2[j] = h3[j];
+      if (i < nt) Vec4<Tio>::store(yt + (long)i * width, yv_);
     }
-    if (i < nt) Vec16<Tio>::store(yt + (long)i * width, yv_);
+    umask |= (unsigned long long)m16 << (4 * t4);
   }
   if constexpr (kBf16) {
+    if (umask) {                              // into the CTA's list
+      int k = atomicAdd(&nlist, __popcll(umask));
+      for (unsigned long long m = umask; m; m &= m - 1, ++k) {
+        const int bit = __ffsll(m) - 1;
+        if (k < kPrologueList) list[k] = (uint16_t)(((i0 + (bit >> 2)) << 8) | (lc * 4 + (bit & 3)));
+      }
+    }
     __syncthreads();                          // the list is complete, the fast values stored
     const int n = nlist;
     __nv_bfloat16* yb = reinterpret_cast<__nv_bfloat16*>(y) + (b * T + t0) * width + (long)head * d;
@@ -203,18 +253,20 @@ prologue_v_kernel(const Tio* __restrict__ x, const float* __restrict__ w, Tio* _
 }
 
 // Prologue of the q and k channels (conv, SiLU, then each head row divided by its L2 norm): grid
-// (2 Hk, ceil(T / kPrologueTokens), B), q heads then k heads; the thread layout of the v kernel.
+// (2 Hk, ceil(T / kPrologueTokens), B), q heads then k heads; the thread layout of the v kernel
+// (4 channels per thread, so that the fp64 weights and window take 56 registers).
 // bf16 outputs: the convolution in fp64 (the weights widened once per thread, each input once, in
-// the window), SiLU in fp32 (expf, IEEE division: within 6 units of roundoff, plus the rounded
-// argument's 0.55 |x|), the row's sum of squares in fp32 with its roundoff bound, so that a value's
-// error is a few tens of units of roundoff at most; a row with any value whose bf16 rounding that
-// leaves open is redone whole in fp64 afterwards (the row's values share the norm).
+// the window), SiLU in fp32 (expf and a Newton-refined reciprocal: within 7 units of roundoff, plus
+// the rounded argument's 0.55 |x|), the row's sum of squares in fp32 with its roundoff bound and
+// rsqrtf, so that a value's error is a few tens of units of roundoff at most; a row with any value
+// whose bf16 rounding that leaves open is redone whole in fp64 afterwards (the row's values share
+// the norm).  No step has a data-dependent branch.
 template <typename Tio>
-__global__ void __launch_bounds__(128, 3)
+__global__ void __launch_bounds__(128, 5)
 prologue_qk_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
                    const float* __restrict__ wq, const float* __restrict__ wk,
                    Tio* __restrict__ yq, Tio* __restrict__ yk, int T, int Hk, int dk, float eps) {
-  constexpr int N = Vec16<Tio>::N;
+  constexpr int N = 4;                        // channels per thread
   constexpr bool kBf16 = sizeof(Tio) == 2;
   constexpr float u = 5.9604645e-8f;
   extern __shared__ __align__(16) uint8_t pro_smem[];
@@ -244,14 +296,14 @@ prologue_qk_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
   Tio* const yt = y + (b * T + t0) * width + c0;
   if constexpr (!kBf16) {                     // fp32 outputs: fp32 throughout
     float h0[N], h1[N], h2[N];
-    Vec16<Tio>::load(tile + (long)i0 * d + lc * N, h0);
-    Vec16<Tio>::load(tile + (long)(i0 + 1) * d + lc * N, h1);
-    Vec16<Tio>::load(tile + (long)(i0 + 2) * d + lc * N, h2);
+    Vec4<Tio>::load(tile + (long)i0 * d + lc * N, h0);
+    Vec4<Tio>::load(tile + (long)(i0 + 1) * d + lc * N, h1);
+    Vec4<Tio>::load(tile + (long)(i0 + 2) * d + lc * N, h2);
 #pragma unroll 2
     for (int tt = 0; tt < tpg; ++tt) {
       const int i = i0 + tt;
       float h3[N], yv_[N], ss = 0.f;
-      Vec16<Tio>::load(tile + (long)(i + 3) * d + lc * N, h3);
+      Vec4<Tio>::load(tile + (long)(i + 3) * d + lc * N, h3);
 #pragma unroll
       for (int j = 0; j < N; ++j) {
         const float pre = fmaf(wt[j][3], h3[j], fmaf(wt[j][2], h2[j],
@@ -264,7 +316,7 @@ prologue_qk_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
       const float inv = rsqrtf(ss + eps);
 #pragma unroll
       for (int j = 0; j < N; ++j) yv_[j] *= inv;
-      if (i < nt) Vec16<Tio>::store(yt + (long)i * width, yv_);
+      if (i < nt) Vec4<Tio>::store(yt + (long)i * width, yv_);
     }
   } else {
     double wd[N][4];                          // the weights, widened once
@@ -272,55 +324,70 @@ prologue_qk_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
     for (int j = 0; j < N; ++j)
 #pragma unroll
       for (int k = 0; k < 4; ++k) wd[j][k] = wt[j][k];
-    double d0[N], d1[N], d2[N];               // the window, widened once per input
-    {
+    // the window, widened once per input, as a ring of four rows: token i reads rows i .. i + 3
+    // at ring slots i .. i + 3 (mod 4), so with the token loop unrolled by four no row is moved
+    double dr[4][N];
+#pragma unroll
+    for (int r = 0; r < 3; ++r) {
       float f[N];
-      Vec16<Tio>::load(tile + (long)i0 * d + lc * N, f);
+      Vec4<Tio>::load(tile + (long)(i0 + r) * d + lc * N, f);
 #pragma unroll
-      for (int j = 0; j < N; ++j) d0[j] = f[j];
-      Vec16<Tio>::load(tile + (long)(i0 + 1) * d + lc * N, f);
-#pragma unroll
-      for (int j = 0; j < N; ++j) d1[j] = f[j];
-      Vec16<Tio>::load(tile + (long)(i0 + 2) * d + lc * N, f);
-#pragma unroll
-      for (int j = 0; j < N; ++j) d2[j] = f[j];
+      for (int j = 0; j < N; ++j) dr[r][j] = f[j];
     }
-    for (int tt = 0; tt < tpg; ++tt) {
-      const int i = i0 + tt;
-      float f[N], s[N], es[N], yv_[N];
-      Vec16<Tio>::load(tile + (long)(i + 3) * d + lc * N, f);
-      float ss = 0.f, se = 0.f;
+    const int lane = threadIdx.x & 31;
+    const unsigned lmask = L == 32 ? 0xffffffffu : (1u << L) - 1u;
+#pragma unroll 1
+    for (int t4 = 0; t4 < tpg; t4 += 4) {
 #pragma unroll
-      for (int j = 0; j < N; ++j) {
-        const double d3 = f[j];
-        const double acc = fma(wd[j][3], d3, fma(wd[j][2], d2[j], fma(wd[j][1], d1[j],
-                                                                      wd[j][0] * d0[j])));
-        const float pre = (float)acc;         // within half a unit of the exact sum
-        s[j] = pre / (1.0f + expf(-pre));
-        es[j] = u * fmaf(fabsf(pre), 0.6f, 7.0f * fabsf(s[j]));   // expf, +, /, rounded pre
-        ss = fmaf(s[j], s[j], ss);
-        se = fmaf(2.0f * fabsf(s[j]), es[j], se);
-        d0[j] = d1[j]; d1[j] = d2[j]; d2[j] = d3;
-      }
-      for (int o = L >> 1; o > 0; o >>= 1) {
-        ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        se += __shfl_xor_sync(0xffffffffu, se, o);
-      }
-      // sum of squares: at most (N + log2 L + 1) units of its own roundoff plus se from the
-      // values; 1/sqrt in fp32: sqrtf and the division, one unit each
-      const float den = ss + eps;
-      const float inv = 1.0f / sqrtf(den);
-      const float dinv = 0.5f * (se + (float)(N + 8) * u * ss) / den * 1.01f + 3.0f * u;
-      bool need = false;
+      for (int sl = 0; sl < 4; ++sl) {
+        if (t4 + sl >= tpg) break;            // tpg = 2 for 16-channel heads
+        const int i = i0 + t4 + sl;
+        const int r0 = sl, r1 = (sl + 1) & 3, r2 = (sl + 2) & 3, r3 = (sl + 3) & 3;
+        float f[N], s[N], es[N], yv_[N];
+        Vec4<Tio>::load(tile + (long)(i + 3) * d + lc * N, f);
+        float ss = 0.f, se = 0.f;
 #pragma unroll
-      for (int j = 0; j < N; ++j) {
-        yv_[j] = s[j] * inv;                  // fp32 product: one more unit
-        const float e = 2.0f * (fabsf(yv_[j]) * (dinv + u) + es[j] * inv);
-        need = need || !bf16_decided(yv_[j], e);
+        for (int j = 0; j < N; ++j) {
+          dr[r3][j] = f[j];
+          const double acc = fma(wd[j][3], dr[r3][j], fma(wd[j][2], dr[r2][j],
+                                                          fma(wd[j][1], dr[r1][j],
+                                                              wd[j][0] * dr[r0][j])));
+          const float pre = (float)acc;       // within half a unit of the exact sum
+          // SiLU = pre / (1 + e^-pre): expf (2 units), the sum (half a unit), 1 / den by
+          // rcp.approx and one Newton step (about half a unit; the approximation's own error
+          // enters squared) and the product (half a unit): within 7 units of s, plus the
+          // rounded argument's 0.55 |pre|
+          const float den = 1.0f + expf(-pre);
+          const float r0 = rcp_fast(den);
+          s[j] = pre * fmaf(r0, fmaf(-den, r0, 1.0f), r0);
+          es[j] = u * fmaf(fabsf(pre), 0.6f, 7.0f * fabsf(s[j]));
+          ss = fmaf(s[j], s[j], ss);
+          se = fmaf(2.0f * fabsf(s[j]), es[j], se);
+        }
+        for (int o = L >> 1; o > 0; o >>= 1) {
+          ss += __shfl_xor_sync(0xffffffffu, ss, o);
+          se += __shfl_xor_sync(0xffffffffu, se, o);
+        }
+        // sum of squares: at most (N + log2 L + 1) units of its own roundoff plus se from the
+        // values; inv = rsqrtf (within 2 ulps, 4 units) of the rounded sum: inv's relative error
+        // is at most half that of den (1 / den = inv^2 within a few units, 2 % allowed), plus 5
+        // units
+        const float den = ss + eps;
+        const float inv = rsqrtf(den);
+        const float dinv = 0.5f * (se + (float)(N + 8) * u * ss) * (inv * inv) * 1.02f + 5.0f * u;
+        bool need = false;
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+          yv_[j] = s[j] * inv;                // fp32 product: one more unit
+          const float e = 2.0f * (fabsf(yv_[j]) * (dinv + u) + es[j] * inv);
+          need = need || !bf16_decided(yv_[j], e);
+        }
+        // any lane of this row (the L lanes lane & ~(L - 1) ..) undecided
+        const unsigned bal = __ballot_sync(0xffffffffu, need);
+        if (lc == 0 && ((bal >> (lane & ~(L - 1))) & lmask) != 0)
+          list[atomicAdd(&nlist, 1)] = (uint16_t)i;               // at most one per token
+        if (i < nt) Vec4<Tio>::store(yt + (long)i * width, yv_);
       }
-      for (int o = L >> 1; o > 0; o >>= 1) need |= __shfl_xor_sync(0xffffffffu, need, o) != 0;
-      if (need && lc == 0) list[atomicAdd(&nlist, 1)] = (uint16_t)i;   // at most one per token
-      if (i < nt) Vec16<Tio>::store(yt + (long)i * width, yv_);
     }
     __syncthreads();                          // the list is complete, the fast values stored
     const int n = nlist;
@@ -347,8 +414,7 @@ prologue_qk_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
         uint32_t pk[N / 2];
 #pragma unroll
         for (int j = 0; j < N / 2; ++j) pk[j] = bf16_pair_rn(yd[2 * j] * invd, yd[2 * j + 1] * invd);
-        *reinterpret_cast<uint4*>(yb + (long)i * width + lc * N) =
-            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint2*>(yb + (long)i * width + lc * N) = make_uint2(pk[0], pk[1]);
       }
     }
   }
@@ -359,31 +425,8 @@ inline size_t prologue_smem_bytes(int d, size_t elem) {
   return (size_t)(kPrologueTokens + 3) * d * elem;
 }
 
-// One warp per row of dv <= 128 values, 4 consecutive channels per lane.  `o` may be wider than
-// z / y (the layer keeps o in fp32).
-template <typename T4> struct Vec4;
-template <> struct Vec4<float> {
-  static __device__ __forceinline__ void load(const float* p, float (&v)[4]) {
-    const float4 a = *reinterpret_cast<const float4*>(p);
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-  }
-  static __device__ __forceinline__ void store(float* p, const float (&v)[4]) {
-    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
-  }
-};
-template <> struct Vec4<__nv_bfloat16> {
-  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[4]) {
-    const uint2 a = *reinterpret_cast<const uint2*>(p);
-    v[0] = __uint_as_float(a.x << 16); v[1] = __uint_as_float(a.x & 0xFFFF0000u);
-    v[2] = __uint_as_float(a.y << 16); v[3] = __uint_as_float(a.y & 0xFFFF0000u);
-  }
-  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[4]) {
-    __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]), h1 = __floats2bfloat162_rn(v[2], v[3]);
-    *reinterpret_cast<uint2*>(p) =
-        make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
-  }
-};
-
+// The gated norm: one warp per row of dv <= 128 values, 4 consecutive channels per lane.  `o` may
+// be wider than z / y (the layer keeps o in fp32).
 template <typename To, typename Tz, typename Ty = Tz>
 __global__ void __launch_bounds__(256)
 out_norm_kernel(const To* __restrict__ o, const Tz* __restrict__ z, const float* __restrict__ w,

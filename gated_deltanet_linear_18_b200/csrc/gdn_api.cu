@@ -621,9 +621,8 @@ gdn_status gdn_prologue(const void* q_raw, const void* k_raw, const void* v_raw,
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if ((T + kPrologueTokens - 1) / kPrologueTokens > 65535) return GDN_ERR_UNSUPPORTED;
   // the q and k heads (normalised rows) on the library's high-priority stream, forked from and
-  // joined back into `stream`, beside the v heads on `stream`: the two kernels share the SMs (the
-  // q/k kernel is latency-bound at three CTAs per SM, the v kernel issue-bound); head slots
-  // fastest in each grid
+  // joined back into `stream`, beside the v heads on `stream`: the two kernels share the SMs (both
+  // are bound by instruction issue and latency, not by HBM); head slots fastest in each grid
   const unsigned tb = (unsigned)((T + kPrologueTokens - 1) / kPrologueTokens);
   const dim3 gqk(2 * Hk, tb, B), gv(Hv, tb, B);
   std::lock_guard<std::mutex> lock(tcf::split_mutex());

@@ -18,7 +18,7 @@ def layer_w(**kw):
 
 @pytest.mark.parametrize("dtype,T,dk,dv", [("f32", 70, 16, 32), ("f32", 131, 64, 64),
                                            ("bf16", 200, 128, 128), ("bf16", 3, 128, 128),
-                                           ("bf16", 1000, 64, 32)])
+                                           ("bf16", 1000, 64, 32), ("bf16", 257, 16, 16)])
 def test_prologue(orc, dtype, T, dk, dv):
     w = layer_w(B=2, T=T, Hk=2, Hv=4, dk=dk, dv=dv, dtype=dtype, seed=T)
     x = gi.make_layer_inputs(w)
@@ -40,6 +40,33 @@ def test_prologue(orc, dtype, T, dk, dv):
             rb = round_bf16(r)
             diff = np64(g) != rb
             assert not np.any(diff & (np.abs(r) > 1e-30)), int(np.count_nonzero(diff))
+
+
+def test_prologue_zero_and_cancelling_rows(orc):
+    """Rows of zeros (an exact zero output, decided without the fp64 redo) and conv windows that
+    cancel exactly or nearly (x repeated, taps of opposite sign), still bit for bit."""
+    w = layer_w(B=1, T=96, Hk=1, Hv=2, dk=128, dv=128, dtype="bf16", seed=5)
+    x = gi.make_layer_inputs(w)
+    for key in ("q_raw", "k_raw", "v_raw"):
+        t = x[key].clone()
+        t[:, 10:20] = 0                          # zero rows: windows with zeros only at 13..19
+        t[:, 40:60] = t[:, 40:41]                # constant rows: sum of taps times one value
+        x[key] = t
+    for key in ("conv_wq", "conv_wk", "conv_wv"):
+        cw = x[key].clone()
+        cw[::2, 3] = -cw[::2, 2]                 # taps 2 and 3 cancel on every other channel
+        x[key] = cw
+    d = to_dev(x)
+    q, k, v = gdn.prologue(d["q_raw"], d["k_raw"], d["v_raw"], d["conv_wq"], d["conv_wk"],
+                           d["conv_wv"], w.Hk, w.Hv, w.dk, w.dv, l2_eps=w.l2_eps)
+    torch.cuda.synchronize()
+    qr, kr, vr = orc.prologue(x["q_raw"], x["k_raw"], x["v_raw"], x["conv_wq"], x["conv_wk"],
+                              x["conv_wv"], w.Hk, w.Hv, w.dk, w.dv, w.l2_eps)
+    for g, r in ((q, qr), (k, kr), (v, vr)):
+        rb = round_bf16(r)
+        diff = np64(g) != rb
+        assert not np.any(diff & (np.abs(r) > 1e-30)), int(np.count_nonzero(diff))
+    assert np.all(np64(v)[:, 16:20] == 0)      # all four taps on zero rows
 
 
 @pytest.mark.parametrize("dtype,dv", [("f32", 16), ("f32", 128), ("bf16", 64), ("bf16", 128)])
