@@ -375,11 +375,14 @@ prologue_qk_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
         const float den = ss + eps;
         const float inv = rsqrtf(den);
         const float dinv = 0.5f * (se + (float)(N + 8) * u * ss) * (inv * inv) * 1.02f + 5.0f * u;
+        // y - y* = (s - s*) inv + s* (inv - inv*) + the product's rounding, so |y - y*| is at most
+        // es inv + |y| (dinv + u) to first order; the 10 % cover the second-order terms (products
+        // of these relative errors, below 1e-12) and |y*| against |y|
         bool need = false;
 #pragma unroll
         for (int j = 0; j < N; ++j) {
-          yv_[j] = s[j] * inv;                // fp32 product: one more unit
-          const float e = 2.0f * (fabsf(yv_[j]) * (dinv + u) + es[j] * inv);
+          yv_[j] = s[j] * inv;
+          const float e = 1.1f * (fabsf(yv_[j]) * (dinv + u) + es[j] * inv);
           need = need || !bf16_decided(yv_[j], e);
         }
         // any lane of this row (the L lanes lane & ~(L - 1) ..) undecided
