@@ -775,10 +775,15 @@ template <typename Tin>
 gdn_status prologue_bwd_one(const void* x_raw, const float* w, const float* dy, float* dx_raw,
                             float* dw, float* dpre, float* dw_part, int B, int T, int heads,
                             int d, bool normalize, float eps, cudaStream_t st) {
-  const long long rows = (long long)B * T * heads;
-  const long long blocks = (rows + 7) / 8;
-  lbwd::conv_dpre_kernel<Tin><<<(unsigned)blocks, 256, 0, st>>>(
-      static_cast<const Tin*>(x_raw), w, dy, dpre, rows, T, heads, d, normalize ? 1 : 0, eps);
+  const dim3 gd(heads, (T + lbwd::kDpreTok - 1) / lbwd::kDpreTok, B);
+  const Tin* xr = static_cast<const Tin*>(x_raw);
+  const int nz = normalize ? 1 : 0;
+  if (d == 128)
+    lbwd::conv_dpre_kernel<Tin, 4><<<gd, 128, 0, st>>>(xr, w, dy, dpre, T, heads, d, nz, eps);
+  else if (d == 64)
+    lbwd::conv_dpre_kernel<Tin, 2><<<gd, 128, 0, st>>>(xr, w, dy, dpre, T, heads, d, nz, eps);
+  else
+    lbwd::conv_dpre_kernel<Tin, 1><<<gd, 128, 0, st>>>(xr, w, dy, dpre, T, heads, d, nz, eps);
   const int C = heads * d;
   const dim3 grid((C + 127) / 128, (T + lbwd::kConvTok - 1) / lbwd::kConvTok, B);
   lbwd::conv_bwd_kernel<Tin><<<grid, 128, 0, st>>>(static_cast<const Tin*>(x_raw), w, dpre,
@@ -817,7 +822,7 @@ gdn_status layer_bwd_run(const void* q_raw, const void* k_raw, const void* v_raw
   const long long rows = (long long)tok * Hv;
   lbwd::out_norm_bwd_kernel<Tin, Tdy><<<kNormBwdCtas, 32 * lbwd::kNormWarps, 0, st>>>(
       o, static_cast<const Tin*>(z), norm_w, static_cast<const Tdy*>(dy), d_o, dz, nw, rows, dv,
-      norm_eps);
+      norm_eps, aligned16(dz) ? 1 : 0);
   lbwd::col_sum_kernel<<<(dv + 255) / 256, 256, 0, st>>>(nw, dnorm_w, (int)kNormBwdCtas, dv);
   if (launch_status() != GDN_OK) return GDN_ERR_CUDA;
   float* dqg = reinterpret_cast<float*>(ws + L.dq);

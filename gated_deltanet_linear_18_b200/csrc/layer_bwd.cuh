@@ -21,16 +21,52 @@ __device__ __forceinline__ float silu_grad(float x) {
 
 constexpr int kNormWarps = 8;
 
+// Vectors of PER consecutive values (PER in 1, 2, 4) as fp32: PER x 4 bytes of fp32 or PER x 2 of
+// bf16, read with one load (the pointer aligned to that size).
+template <int PER, typename T>
+__device__ __forceinline__ void vload(const T* p, float (&v)[PER]) {
+  if constexpr (sizeof(T) == 4) {
+    if constexpr (PER == 4) {
+      const float4 a = *reinterpret_cast<const float4*>(p);
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    } else if constexpr (PER == 2) {
+      const float2 a = *reinterpret_cast<const float2*>(p);
+      v[0] = a.x; v[1] = a.y;
+    } else {
+      v[0] = to_f(p[0]);
+    }
+  } else {
+    if constexpr (PER == 4) {
+      const uint2 a = *reinterpret_cast<const uint2*>(p);
+      v[0] = __uint_as_float(a.x << 16); v[1] = __uint_as_float(a.x & 0xFFFF0000u);
+      v[2] = __uint_as_float(a.y << 16); v[3] = __uint_as_float(a.y & 0xFFFF0000u);
+    } else if constexpr (PER == 2) {
+      const uint32_t a = *reinterpret_cast<const uint32_t*>(p);
+      v[0] = __uint_as_float(a << 16); v[1] = __uint_as_float(a & 0xFFFF0000u);
+    } else {
+      v[0] = to_f(p[0]);
+    }
+  }
+}
+template <int PER>
+__device__ __forceinline__ void vstore(float* p, const float (&v)[PER]) {
+  if constexpr (PER == 4) *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  else if constexpr (PER == 2) *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+  else p[0] = v[0];
+}
+
 // Gated RMSNorm backward, y = o inv w SiLU(z), inv = 1 / sqrt(mean(o^2) + eps), one warp per row of
-// dv <= 128 (4 columns per lane), rows strided over a fixed grid:
+// dv <= 128 (4 columns per lane, read and written as vectors), rows strided over a fixed grid:
 //   g = dy w SiLU(z);  do = inv g - o inv^3 (g . o) / dv;  dz = dy o inv w SiLU'(z);
 //   dw += dy o inv SiLU(z)  (per CTA: dw_part[blockIdx.x][dv]).
+// dz is written as one 16-byte vector per lane when dz_vec (the caller's dz 16-byte aligned), else
+// value by value.
 template <typename Tz, typename Ty>
 __global__ void __launch_bounds__(32 * kNormWarps)
 out_norm_bwd_kernel(const float* __restrict__ o, const Tz* __restrict__ z,
                     const float* __restrict__ w, const Ty* __restrict__ dy,
                     float* __restrict__ d_o, float* __restrict__ dz, float* __restrict__ dw_part,
-                    long long rows, int dv, float eps) {
+                    long long rows, int dv, float eps, int dz_vec) {
   __shared__ float part[kNormWarps][128];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, c = 4 * lane;
   const bool active = c < dv;
@@ -40,12 +76,11 @@ out_norm_bwd_kernel(const float* __restrict__ o, const Tz* __restrict__ z,
   for (long long row = (long long)blockIdx.x * kNormWarps + warp; row < rows;
        row += (long long)gridDim.x * kNormWarps) {
     float ov[4] = {0.f, 0.f, 0.f, 0.f}, zv[4] = {0.f, 0.f, 0.f, 0.f}, gv[4] = {0.f, 0.f, 0.f, 0.f};
-    if (active)
-      for (int e = 0; e < 4; ++e) {
-        ov[e] = o[row * dv + c + e];
-        zv[e] = to_f(z[row * dv + c + e]);
-        gv[e] = to_f(dy[row * dv + c + e]);
-      }
+    if (active) {
+      vload<4>(o + row * dv + c, ov);
+      vload<4>(z + row * dv + c, zv);
+      vload<4>(dy + row * dv + c, gv);
+    }
     float ss = 0.f;
     for (int e = 0; e < 4; ++e) ss = fmaf(ov[e], ov[e], ss);
     ss = warp_sum(ss);
@@ -58,11 +93,17 @@ out_norm_bwd_kernel(const float* __restrict__ o, const Tz* __restrict__ z,
       acc[e] = fmaf(gv[e] * ov[e] * inv, sz, acc[e]);
     }
     go = warp_sum(go);
-    if (active)
+    if (active) {
+      float dov[4], dzv[4];
       for (int e = 0; e < 4; ++e) {
-        d_o[row * dv + c + e] = inv * g[e] - ov[e] * inv * inv * inv * go / dv;
-        dz[row * dv + c + e] = gv[e] * ov[e] * inv * ww[e] * silu_grad(zv[e]);
+        dov[e] = inv * g[e] - ov[e] * inv * inv * inv * go / dv;
+        dzv[e] = gv[e] * ov[e] * inv * ww[e] * silu_grad(zv[e]);
       }
+      vstore<4>(d_o + row * dv + c, dov);
+      if (dz_vec) vstore<4>(dz + row * dv + c, dzv);
+      else
+        for (int e = 0; e < 4; ++e) dz[row * dv + c + e] = dzv[e];
+    }
   }
   if (active)
     for (int e = 0; e < 4; ++e) part[warp][c + e] = acc[e];
@@ -84,60 +125,97 @@ __global__ void col_sum_kernel(const float* __restrict__ part, float* __restrict
   out[j] = s;
 }
 
-// Prologue backward, step 1: the gradient at the convolution's output (pre), one warp per
-// (token, head) row of d channels (d / 32 per lane, d in {32, 64, 128}; 16: lanes 0..15).
+constexpr int kDpreTok = 64;    // tokens per CTA of conv_dpre_kernel (16 per warp)
+
+// Prologue backward, step 1: the gradient at the convolution's output (pre).  grid (heads,
+// ceil(T / kDpreTok), B), 128 threads: warp w takes 16 consecutive tokens of one head, lane l the
+// channels l PER .. l PER + PER - 1 of it (d = 32 PER; for d = 16, PER = 1 and lanes 16.. idle),
+// with the weights loaded once and the 4-tap window of raw inputs in a ring of four register rows
+// (token t reads slots t .. t + 3 mod 4, the loop unrolled by four):
 //   s = SiLU(pre);  q, k (normalize): y = s / n, n = sqrt(s . s + eps),
 //   ds = dy / n - s (s . dy) / n^3;  v: ds = dy;  dpre = ds SiLU'(pre).
-// x: raw inputs [B, T, heads * d]; dy: [B, T, heads, d] fp32; dpre: [B, T, heads * d] fp32.
-template <typename Tin>
-__global__ void __launch_bounds__(256)
+// x: raw inputs [B, T, heads * d]; dy: [B, T, heads, d] fp32; dpre: [B, T, heads * d] fp32; x, dy
+// and dpre aligned to PER values.
+template <typename Tin, int PER>
+__global__ void __launch_bounds__(128)
 conv_dpre_kernel(const Tin* __restrict__ x, const float* __restrict__ w,
-                 const float* __restrict__ dy, float* __restrict__ dpre, long long rows, int T,
-                 int heads, int d, int normalize, float eps) {
-  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);   // (b * T + t) * heads + h
-  const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  const int h = (int)(row % heads);
-  const long long bt = row / heads;
-  const int t = (int)(bt % T);
+                 const float* __restrict__ dy, float* __restrict__ dpre, int T, int heads, int d,
+                 int normalize, float eps) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int h = blockIdx.x;
+  const long b = blockIdx.z;
+  const int tb = blockIdx.y * kDpreTok + warp * (kDpreTok / 4);
   const int C = heads * d;
-  constexpr int kMax = 4;                             // channels per lane (d <= 128)
-  float pre[kMax], s[kMax], g[kMax];
-  float ss = 0.f, sd = 0.f;
-  const int per = d >= 32 ? d / 32 : 1;
-  const bool lane_on = d >= 32 || lane < d;
-  for (int e = 0; e < kMax; ++e) {
-    pre[e] = s[e] = g[e] = 0.f;
-    if (e >= per || !lane_on) continue;
-    const int ch = h * d + lane * per + e;
-    float acc = 0.f;
-    for (int j = 0; j < 4; ++j) {
-      const int u = t - 3 + j;
-      if (u >= 0) acc = fmaf(w[ch * 4 + j], to_f(x[(bt - t + u) * C + ch]), acc);
+  const bool on = lane * PER < d;
+  const int ch0 = h * d + lane * PER;         // this lane's first channel
+  float wt[PER][4];
+#pragma unroll
+  for (int e = 0; e < PER; ++e)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) wt[e][j] = on ? w[(ch0 + e) * 4 + j] : 0.f;
+  const Tin* xb = x + b * (long)T * C + ch0;
+  auto row_in = [&](int t, float (&v)[PER]) {  // raw inputs of token t (zeros outside 0 .. T - 1)
+#pragma unroll
+    for (int e = 0; e < PER; ++e) v[e] = 0.f;
+    if (on && t >= 0 && t < T) vload<PER>(xb + (long)t * C, v);
+  };
+  float r[4][PER];
+  row_in(tb - 3, r[0]);
+  row_in(tb - 2, r[1]);
+  row_in(tb - 1, r[2]);
+#pragma unroll 1
+  for (int t4 = 0; t4 < kDpreTok / 4; t4 += 4) {
+#pragma unroll
+    for (int sl = 0; sl < 4; ++sl) {
+      const int t = tb + t4 + sl;
+      if (t >= T) break;                      // uniform over the warp
+      const int r0 = sl, r1 = (sl + 1) & 3, r2 = (sl + 2) & 3, r3 = (sl + 3) & 3;
+      row_in(t, r[r3]);
+      const long row = (b * T + t) * heads + h;
+      float pre[PER], s[PER], g[PER];
+#pragma unroll
+      for (int e = 0; e < PER; ++e) g[e] = 0.f;
+      if (on) vload<PER>(dy + row * d + lane * PER, g);
+      float ss = 0.f, sd = 0.f;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) {
+        // the taps in order (w[.., 3] on token t), as the forward's sum; a zero-history tap adds
+        // nothing
+        float acc = 0.f;
+        if (t - 3 >= 0) acc = fmaf(wt[e][0], r[r0][e], acc);
+        if (t - 2 >= 0) acc = fmaf(wt[e][1], r[r1][e], acc);
+        if (t - 1 >= 0) acc = fmaf(wt[e][2], r[r2][e], acc);
+        acc = fmaf(wt[e][3], r[r3][e], acc);
+        pre[e] = acc;
+        s[e] = acc * sigm(acc);
+        ss = fmaf(s[e], s[e], ss);
+        sd = fmaf(s[e], g[e], sd);
+      }
+      float n = 1.f, n3 = 1.f;
+      if (normalize) {
+        ss = warp_sum(ss);
+        sd = warp_sum(sd);
+        n = sqrtf(ss + eps);
+        n3 = n * n * n;
+      }
+      if (on) {
+        float out[PER];
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+          const float ds = normalize ? g[e] / n - s[e] * sd / n3 : g[e];
+          out[e] = ds * silu_grad(pre[e]);
+        }
+        vstore<PER>(dpre + (b * T + t) * (long)C + ch0, out);
+      }
     }
-    pre[e] = acc;
-    s[e] = acc * sigm(acc);
-    g[e] = dy[row * d + lane * per + e];
-    ss = fmaf(s[e], s[e], ss);
-    sd = fmaf(s[e], g[e], sd);
-  }
-  float n = 1.f, n3 = 1.f;
-  if (normalize) {
-    ss = warp_sum(ss);
-    sd = warp_sum(sd);
-    n = sqrtf(ss + eps);
-    n3 = n * n * n;
-  }
-  for (int e = 0; e < per && lane_on; ++e) {
-    const float ds = normalize ? g[e] / n - s[e] * sd / n3 : g[e];
-    dpre[bt * C + h * d + lane * per + e] = ds * silu_grad(pre[e]);
   }
 }
 
 constexpr int kConvTok = 64;    // tokens per CTA of conv_bwd_kernel
 
 // Prologue backward, step 2: through the 4-tap convolution, one thread per channel of a
-// 128-channel block over kConvTok tokens:  dx[t] = sum_j w[j] dpre[t + 3 - j]  (t + 3 - j < T),
+// 128-channel block over kConvTok tokens, dpre and x in rings of four registers (each read once):
+//   dx[t] = sum_j w[j] dpre[t + 3 - j]  (t + 3 - j < T),
 //   dw[j] += dpre[t] x[t - 3 + j]  (t - 3 + j >= 0), per CTA: dw_part[cta][C][4], cta over
 //   (token tile, batch).  grid (ceil(C / 128), ceil(T / kConvTok), B).
 template <typename Tin>
@@ -155,14 +233,26 @@ conv_bwd_kernel(const Tin* __restrict__ x, const float* __restrict__ w,
   const int t1 = min(T, t0 + kConvTok);
   auto P = [&](int t) -> float { return t < T ? dpre[(b * T + t) * C + c] : 0.f; };
   auto X = [&](int t) -> float { return t >= 0 ? to_f(x[(b * T + t) * C + c]) : 0.f; };
-  for (int t = t0; t < t1; ++t) {
-    // tap j multiplies x[t - 3 + j] in the output at t, so x[t] feeds outputs t + 3 - j
-    dx[(b * T + t) * C + c] = fmaf(w0, P(t + 3), fmaf(w1, P(t + 2), fmaf(w2, P(t + 1), w3 * P(t))));
-    const float p = P(t);
-    a0 = fmaf(p, X(t - 3), a0);
-    a1 = fmaf(p, X(t - 2), a1);
-    a2 = fmaf(p, X(t - 1), a2);
-    a3 = fmaf(p, X(t), a3);
+  // p[t mod 4] = dpre[t] for t .. t + 3, xr[t mod 4] = x[t - 3 + ...] for t - 3 .. t
+  float p[4], xr[4];
+  p[0] = P(t0); p[1] = P(t0 + 1); p[2] = P(t0 + 2);
+  xr[0] = X(t0 - 3); xr[1] = X(t0 - 2); xr[2] = X(t0 - 1);
+#pragma unroll 1
+  for (int t4 = 0; t4 < kConvTok; t4 += 4) {
+#pragma unroll
+    for (int sl = 0; sl < 4; ++sl) {
+      const int t = t0 + t4 + sl;
+      if (t >= t1) break;
+      const int r0 = sl, r1 = (sl + 1) & 3, r2 = (sl + 2) & 3, r3 = (sl + 3) & 3;
+      p[r3] = P(t + 3);
+      xr[r3] = X(t);
+      // tap j multiplies x[t - 3 + j] in the output at t, so x[t] feeds outputs t + 3 - j
+      dx[(b * T + t) * C + c] = fmaf(w0, p[r3], fmaf(w1, p[r2], fmaf(w2, p[r1], w3 * p[r0])));
+      a0 = fmaf(p[r0], xr[r0], a0);
+      a1 = fmaf(p[r0], xr[r1], a1);
+      a2 = fmaf(p[r0], xr[r2], a2);
+      a3 = fmaf(p[r0], xr[r3], a3);
+    }
   }
   float* dp = dw_part + (cta * C + c) * 4;
   dp[0] = a0;
