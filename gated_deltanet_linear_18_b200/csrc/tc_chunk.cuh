@@ -1110,14 +1110,16 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         if (q == 2 && lane == 0) GDN_TRACE(c, 30 + ev);
         tc::tc_fence_after();
         const bool t_out = (long)c * C + t >= sp.len;
-#pragma unroll 1
+        // this half's 64 columns of the row in one TMEM round trip
+        float x[64];
+        tc::tmem_ld32(tx, *reinterpret_cast<float(*)[32]>(&x[0]));
+        tc::tmem_ld32(tx + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
+        tc::tmem_wait_ld();
+#pragma unroll
         for (int p = 0; p < 2; ++p) {            // value columns 32p .. 32p+31 of this half
-          float x[32];
-          tc::tmem_ld32(tx + 32 * p, x);
-          tc::tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const float* xx = x + 8 * j;
+            const float* xx = x + 32 * p + 8 * j;
             const uint4 u = p ? vr[4 + j] : vr[j];   // (no dynamic register indexing)
             const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
             float rv[8];
@@ -1235,16 +1237,17 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
           }
         };
 #pragma unroll 1
-        for (int p = 0; p < 4; ++p) {            // value columns 16p .. 16p+15 of this half
-          float x[16], y[16];
-          tmem_ld16(tx + 16 * p, x);
-          tmem_ld16(tmem + lane_off + TM_Y + tcol + 16 * p, y);
+        for (int p = 0; p < 4; p += 2) {         // value columns 16p .. 16p+31 of this half
+          float x[32], y[32];
+          tc::tmem_ld32(tx + 16 * p, x);
+          tc::tmem_ld32(tmem + lane_off + TM_Y + tcol + 16 * p, y);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; i += 2)
+          for (int i = 0; i < 32; i += 2)
             tc::f2_get(tc::fma2(tc::f2(g, g), tc::f2(x[i], x[i + 1]), tc::f2(y[i], y[i + 1])),
                        y[i], y[i + 1]);
           put16(p, y);
+          put16(p + 1, y + 16);
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
