@@ -40,6 +40,12 @@
  * Streams.  `stream` is a cudaStream_t (NULL = the legacy default stream).  Each compute call
  * validates its arguments synchronously, enqueues its kernels on `stream` and returns without
  * waiting; results are ready when the stream reaches that point.
+ * CUDA graphs.  gdn_chunk_fwd, gdn_decode_step and gdn_layer_fwd can be captured into a CUDA
+ * graph (stream capture on `stream`) and replayed, with the results of the eager calls (tested
+ * bit for bit); the work the chunked forward forks onto the library's own streams is joined back
+ * into `stream` and so captured with it.  Make one eager call of the chunked forward (or of
+ * gdn_layer_fwd or gdn_prologue) per device before the first capture: it creates the library's
+ * streams and events for the device.  A replay reuses the pointers and sizes of the captured call.
  *
  * Errors.  Calls return gdn_status and never abort, throw or trap.  GDN_ERR_INVALID_ARG: a null
  * required pointer, a non-positive size, Hv not a multiple of Hk, misalignment, or an
