@@ -82,10 +82,14 @@ def lib() -> ctypes.CDLL:
         L.gdn_wait_timeout_selftest.restype = I
         L.gdn_prologue.argtypes = [P] * 9 + [I] * 6 + [F, I, P]
         L.gdn_prologue.restype = I
+        L.gdn_prologue_ex.argtypes = [P] * 12 + [I] * 6 + [F, I, P]
+        L.gdn_prologue_ex.restype = I
         L.gdn_out_norm.argtypes = [P, P, P, P, LL, I, F, I, P]
         L.gdn_out_norm.restype = I
         L.gdn_layer_fwd.argtypes = [P] * 14 + [SZ] + [I] * 7 + [F, F, F, I, I, P]
         L.gdn_layer_fwd.restype = I
+        L.gdn_layer_fwd_ex.argtypes = [P] * 20 + [SZ] + [I] * 7 + [F, F, F, I, I, P]
+        L.gdn_layer_fwd_ex.restype = I
         L.gdn_layer_workspace_bytes.argtypes = [I] * 7 + [I]
         L.gdn_layer_fwd_static.argtypes = [P] * 13 + [I] * 7 + [F, F, F, I, I, P]
         L.gdn_layer_fwd_static.restype = I
@@ -385,21 +389,33 @@ def gates(ba, Hv: int) -> Tuple[torch.Tensor, torch.Tensor]:
     return log_alpha, beta
 
 
+def _hist_shapes(B, Hk, Hv, dk, dv, hist):
+    """Check a conv history (hq, hk, hv) of [B, 3, Hk*dk], [B, 3, Hk*dk], [B, 3, Hv*dv]."""
+    if hist is None:
+        return (None, None, None)
+    hq, hk, hv = hist
+    if hq.shape != (B, 3, Hk * dk) or hk.shape != hq.shape or hv.shape != (B, 3, Hv * dv):
+        raise ValueError("conv history shapes disagree")
+    return hq, hk, hv
+
+
 def prologue(q_raw, k_raw, v_raw, wq, wk, wv, Hk: int, Hv: int, dk: int, dv: int,
-             l2_eps: float = 1e-6):
+             l2_eps: float = 1e-6, hist=None):
     """Conv(4 taps) + SiLU + L2-normalisation of q/k heads.  Returns (q, k, v) shaped
-    [B,T,Hk,dk], [B,T,Hk,dk], [B,T,Hv,dv]."""
+    [B,T,Hk,dk], [B,T,Hk,dk], [B,T,Hv,dv].  ``hist`` (optional): the raw inputs (hq, hk, hv) of
+    the three tokens before, [B,3,Hk*dk], [B,3,Hk*dk], [B,3,Hv*dv], oldest first."""
     B, T = q_raw.shape[:2]
     _f32(wq, wk, wv)
+    hq, hk, hv = _hist_shapes(B, Hk, Hv, dk, dv, hist)
     q = torch.empty(B, T, Hk, dk, device=q_raw.device, dtype=q_raw.dtype)
     k = torch.empty_like(q)
     v = torch.empty(B, T, Hv, dv, device=q_raw.device, dtype=q_raw.dtype)
-    dev = _dev(q_raw, k_raw, v_raw, wq, wk, wv, q, k, v)
+    dev = _dev(q_raw, k_raw, v_raw, wq, wk, wv, q, k, v, hq, hk, hv)
     with torch.cuda.device(dev):
-        st = lib().gdn_prologue(_p(q_raw), _p(k_raw), _p(v_raw), _p(wq), _p(wk), _p(wv), _p(q),
-                                _p(k), _p(v), B, T, Hk, Hv, dk, dv, float(l2_eps),
-                                _io_dtype(q_raw), _stream(dev))
-    _check("gdn_prologue", st)
+        st = lib().gdn_prologue_ex(_p(q_raw), _p(k_raw), _p(v_raw), _p(hq), _p(hk), _p(hv),
+                                   _p(wq), _p(wk), _p(wv), _p(q), _p(k), _p(v), B, T, Hk, Hv, dk,
+                                   dv, float(l2_eps), _io_dtype(q_raw), _stream(dev))
+    _check("gdn_prologue_ex", st)
     return q, k, v
 
 
@@ -426,26 +442,39 @@ def layer_fwd(q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, *
               Hv: int, dk: int, dv: int, chunk: int = 64, scale: float = 1.0,
               l2_eps: float = 1e-6, norm_eps: float = 1e-5, want_state: bool = True,
               workspace: Optional[torch.Tensor] = None,
-              out_dtype: Optional[torch.dtype] = None):
+              out_dtype: Optional[torch.dtype] = None, hist=None, want_hist: bool = False):
     """Whole layer between the projections: returns (y [B,T,Hv,dv], S_T or None); y in
-    ``out_dtype`` (default the inputs' dtype; float32 for bf16 inputs)."""
+    ``out_dtype`` (default the inputs' dtype; float32 for bf16 inputs).  ``hist`` (optional): the
+    raw inputs (hq, hk, hv) of the three tokens before this call, [B,3,Hk*dk], [B,3,Hk*dk],
+    [B,3,Hv*dv], oldest first.  With ``want_hist`` the history after the call is returned too:
+    (y, S_T, (hq, hk, hv))."""
     B, T = q_raw.shape[:2]
     _f32(wq, wk, wv, log_alpha, beta, S0, norm_w)
+    hq, hk, hv = _hist_shapes(B, Hk, Hv, dk, dv, hist)
     y = torch.empty(B, T, Hv, dv, device=q_raw.device, dtype=out_dtype or q_raw.dtype)
     sT = torch.empty(B, Hv, dk, dv, device=q_raw.device, dtype=torch.float32) \
         if want_state else None
+    ho = (None, None, None)
+    if want_hist:
+        ho = (torch.empty(B, 3, Hk * dk, device=q_raw.device, dtype=q_raw.dtype),
+              torch.empty(B, 3, Hk * dk, device=q_raw.device, dtype=q_raw.dtype),
+              torch.empty(B, 3, Hv * dv, device=q_raw.device, dtype=q_raw.dtype))
     need = layer_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, q_raw.dtype)
     if workspace is None and need > 0:
         workspace = torch.empty(need, device=q_raw.device, dtype=torch.uint8)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    dev = _dev(q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, y, sT)
+    dev = _dev(q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, y, sT, hq, hk,
+               hv, *ho)
     with torch.cuda.device(dev):
-        st = lib().gdn_layer_fwd(_p(q_raw), _p(k_raw), _p(v_raw), _p(z), _p(wq), _p(wk), _p(wv),
-                                 _p(log_alpha), _p(beta), _p(S0), _p(norm_w), _p(y), _p(sT),
-                                 _p(workspace), wbytes, B, T, Hk, Hv, dk, dv, chunk,
-                                 float(scale), float(l2_eps), float(norm_eps),
-                                 _io_dtype(q_raw), _io_dtype(y), _stream(dev))
-    _check("gdn_layer_fwd", st)
+        st = lib().gdn_layer_fwd_ex(_p(q_raw), _p(k_raw), _p(v_raw), _p(z), _p(hq), _p(hk),
+                                    _p(hv), _p(wq), _p(wk), _p(wv), _p(log_alpha), _p(beta),
+                                    _p(S0), _p(norm_w), _p(y), _p(sT), _p(ho[0]), _p(ho[1]),
+                                    _p(ho[2]), _p(workspace), wbytes, B, T, Hk, Hv, dk, dv, chunk,
+                                    float(scale), float(l2_eps), float(norm_eps),
+                                    _io_dtype(q_raw), _io_dtype(y), _stream(dev))
+    _check("gdn_layer_fwd_ex", st)
+    if want_hist:
+        return y, sT, ho
     return y, sT
 
 

@@ -89,18 +89,21 @@ __device__ __forceinline__ float rcp_fast(float x) {
 constexpr int kPrologueList = 1024;     // undecided values one CTA redoes in fp64 afterwards
 
 // The staged tile of one prologue CTA: the raw rows of tokens t0 - 3 .. t0 + kPrologueTokens - 1
-// (zeros outside 0 .. T - 1) of one head of d channels, row r holding token t0 - 3 + r, brought in
-// by 16-byte asynchronous copies that are all issued at once (many tiles in flight per SM).
+// of one head of d channels, row r holding token t0 - 3 + r, brought in by 16-byte asynchronous
+// copies that are all issued at once (many tiles in flight per SM).  Tokens -3 .. -1 come from the
+// carried history hh (the raw rows of the three tokens before this call, oldest first, at the same
+// row width), or are zeros when there is none; tokens from T on are zeros.
 template <typename Tio>
-__device__ __forceinline__ void prologue_stage(Tio* tile, const Tio* xh, long t0, int T, int width,
-                                               int d) {
+__device__ __forceinline__ void prologue_stage(Tio* tile, const Tio* xh, const Tio* hh, long t0,
+                                               int T, int width, int d) {
   constexpr int N = Vec16<Tio>::N;
   const int L = d / N, lgL = __ffs(L) - 1;    // 16-byte pieces per row (a power of two)
   for (int i = threadIdx.x; i < (kPrologueTokens + 3) * L; i += blockDim.x) {
     const int r = i >> lgL, c = i & (L - 1);
     const long t = t0 - 3 + r;
-    const bool in = t >= 0 && t < T;
-    const Tio* src = in ? xh + t * width + c * N : xh;
+    const bool hist = t < 0 && hh != nullptr;
+    const bool in = (t >= 0 && t < T) || hist;
+    const Tio* src = !in ? xh : (t >= 0 ? xh + t * width + c * N : hh + (t + 3) * width + c * N);
     const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(tile + (long)r * d + c * N));
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
                  "r"(in ? 16 : 0) : "memory");
@@ -161,8 +164,8 @@ __device__ __forceinline__ bool bf16_decided_e24(float y, float E) {
 // the tile is stored, so the rare fp64 work and its bookkeeping stay off the common path.
 template <typename Tio>
 __global__ void __launch_bounds__(128, 6)
-prologue_v_kernel(const Tio* __restrict__ x, const float* __restrict__ w, Tio* __restrict__ y,
-                  int T, int Hv, int dv) {
+prologue_v_kernel(const Tio* __restrict__ x, const Tio* __restrict__ hist,
+                  const float* __restrict__ w, Tio* __restrict__ y, int T, int Hv, int dv) {
   constexpr bool kBf16 = sizeof(Tio) == 2;
   extern __shared__ __align__(16) uint8_t pro_smem[];
   Tio* tile = reinterpret_cast<Tio*>(pro_smem);
@@ -174,7 +177,8 @@ prologue_v_kernel(const Tio* __restrict__ x, const float* __restrict__ w, Tio* _
   const int L = d / 4, grp = threadIdx.x / L, lc = threadIdx.x % L, ngrp = 128 / L;
   const int tpg = kPrologueTokens / ngrp, i0 = grp * tpg;  // this row group's tokens
   if (threadIdx.x == 0) nlist = 0;
-  prologue_stage(tile, x + b * T * (long)width + (long)head * d, t0, T, width, d);
+  prologue_stage(tile, x + b * T * (long)width + (long)head * d,
+                 hist ? hist + b * 3 * (long)width + (long)head * d : nullptr, t0, T, width, d);
   const long c0 = (long)head * d + lc * 4;    // first channel of this thread
   float wk[4][4];                             // [channel][tap]
 #pragma unroll
@@ -264,6 +268,7 @@ prologue_v_kernel(const Tio* __restrict__ x, const float* __restrict__ w, Tio* _
 template <typename Tio>
 __global__ void __launch_bounds__(128, 5)
 prologue_qk_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
+                   const Tio* __restrict__ hq, const Tio* __restrict__ hk,
                    const float* __restrict__ wq, const float* __restrict__ wk,
                    Tio* __restrict__ yq, Tio* __restrict__ yk, int T, int Hk, int dk, float eps) {
   constexpr int N = 4;                        // channels per thread
@@ -276,6 +281,7 @@ prologue_qk_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
   const bool isq = blockIdx.x < Hk;
   const int head = isq ? blockIdx.x : blockIdx.x - Hk, d = dk, width = Hk * dk;
   const Tio* x = isq ? xq : xk;
+  const Tio* hist = isq ? hq : hk;
   const float* w = isq ? wq : wk;
   Tio* y = isq ? yq : yk;
   const long b = blockIdx.z;
@@ -283,7 +289,8 @@ prologue_qk_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
   const int L = d / N, grp = threadIdx.x / L, lc = threadIdx.x % L, ngrp = 128 / L;
   const int tpg = kPrologueTokens / ngrp, i0 = grp * tpg;
   if (threadIdx.x == 0) nlist = 0;
-  prologue_stage(tile, x + b * T * (long)width + (long)head * d, t0, T, width, d);
+  prologue_stage(tile, x + b * T * (long)width + (long)head * d,
+                 hist ? hist + b * 3 * (long)width + (long)head * d : nullptr, t0, T, width, d);
   const long c0 = (long)head * d + lc * N;
   float wt[N][4];
 #pragma unroll
@@ -454,6 +461,26 @@ out_norm_kernel(const To* __restrict__ o, const Tz* __restrict__ z, const float*
     for (int e = 0; e < 4; ++e) yv[e] = ov[e] * inv * ww[e] * silu_fast(zv[e]);
     Vec4<Ty>::store(y + row * dv + c, yv);
   }
+}
+
+// The conv history after a call: the raw rows of the last three tokens of [history; x] (oldest
+// first), per sequence, for `width` channels: row r is token T + r of that concatenation, from the
+// incoming history hin while T + r < 3 (zeros when there is none), else from x.  One thread per
+// 16-byte piece of a row.
+template <typename Tio>
+__global__ void conv_hist_out_kernel(const Tio* __restrict__ x, const Tio* __restrict__ hin,
+                                     Tio* __restrict__ hout, long B, int T, int width) {
+  constexpr int N = 16 / sizeof(Tio);
+  const int P = width / N;
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= B * 3 * P) return;
+  const long b = i / (3 * P);
+  const int r = (int)(i / P % 3), c = (int)(i % P);
+  const long s = (long)T + r;                 // position in [history; x]
+  uint4 v = make_uint4(0u, 0u, 0u, 0u);
+  if (s >= 3) v = reinterpret_cast<const uint4*>(x + (b * T + s - 3) * (long)width)[c];
+  else if (hin) v = reinterpret_cast<const uint4*>(hin + (b * 3 + s) * (long)width)[c];
+  reinterpret_cast<uint4*>(hout + (b * 3 + r) * (long)width)[c] = v;
 }
 
 // Gates from the in_proj_ba outputs: beta = sigmoid(b), log alpha = -softplus(-a), one thread per

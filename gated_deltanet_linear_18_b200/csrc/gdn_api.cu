@@ -604,13 +604,17 @@ gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const fl
                                                        Hk, Hv, scale, st);
 }
 
-gdn_status gdn_prologue(const void* q_raw, const void* k_raw, const void* v_raw, const float* wq,
-                        const float* wk, const float* wv, void* q, void* k, void* v, int B, int T,
-                        int Hk, int Hv, int dk, int dv, float l2_eps, gdn_dtype dtype,
-                        gdn_stream_t stream) {
+gdn_status gdn_prologue_ex(const void* q_raw, const void* k_raw, const void* v_raw,
+                           const void* hq_in, const void* hk_in, const void* hv_in,
+                           const float* wq, const float* wk, const float* wv, void* q, void* k,
+                           void* v, int B, int T, int Hk, int Hv, int dk, int dv, float l2_eps,
+                           gdn_dtype dtype, gdn_stream_t stream) {
   if (B < 0 || T < 0 || !valid_dtype(dtype) || !(l2_eps >= 0.f)) return GDN_ERR_INVALID_ARG;
   gdn_status s = validate_heads(Hk, Hv, dk, dv);
   if (s != GDN_OK) return s;
+  const void* hist[] = {hq_in, hk_in, hv_in};
+  for (const void* p : hist)
+    if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
   if ((long)B * T == 0) return GDN_OK;
   if (B > 65535 || 2L * Hk + Hv > 65535) return GDN_ERR_UNSUPPORTED;
   const void* ptrs[] = {q_raw, k_raw, v_raw, q, k, v};
@@ -632,15 +636,17 @@ gdn_status gdn_prologue(const void* q_raw, const void* k_raw, const void* v_raw,
     return GDN_ERR_CUDA;
   if (dtype == GDN_F32) {
     prologue_qk_kernel<float><<<gqk, 128, prologue_smem_bytes(dk, 4), sp->s_hi>>>(
-        (const float*)q_raw, (const float*)k_raw, wq, wk, (float*)q, (float*)k, T, Hk, dk, l2_eps);
+        (const float*)q_raw, (const float*)k_raw, (const float*)hq_in, (const float*)hk_in, wq,
+        wk, (float*)q, (float*)k, T, Hk, dk, l2_eps);
     prologue_v_kernel<float><<<gv, 128, prologue_smem_bytes(dv, 4), st>>>(
-        (const float*)v_raw, wv, (float*)v, T, Hv, dv);
+        (const float*)v_raw, (const float*)hv_in, wv, (float*)v, T, Hv, dv);
   } else {
     using bf = __nv_bfloat16;
     prologue_qk_kernel<bf><<<gqk, 128, prologue_smem_bytes(dk, 2), sp->s_hi>>>(
-        (const bf*)q_raw, (const bf*)k_raw, wq, wk, (bf*)q, (bf*)k, T, Hk, dk, l2_eps);
+        (const bf*)q_raw, (const bf*)k_raw, (const bf*)hq_in, (const bf*)hk_in, wq, wk, (bf*)q,
+        (bf*)k, T, Hk, dk, l2_eps);
     prologue_v_kernel<bf><<<gv, 128, prologue_smem_bytes(dv, 2), st>>>(
-        (const bf*)v_raw, wv, (bf*)v, T, Hv, dv);
+        (const bf*)v_raw, (const bf*)hv_in, wv, (bf*)v, T, Hv, dv);
   }
   const gdn_status ls = launch_status();
   // the caller's stream waits for the q/k kernel, also after a failed launch
@@ -648,6 +654,14 @@ gdn_status gdn_prologue(const void* q_raw, const void* k_raw, const void* v_raw,
       cudaStreamWaitEvent(st, sp->ev_hi, 0) != cudaSuccess)
     return GDN_ERR_CUDA;
   return ls;
+}
+
+gdn_status gdn_prologue(const void* q_raw, const void* k_raw, const void* v_raw, const float* wq,
+                        const float* wk, const float* wv, void* q, void* k, void* v, int B, int T,
+                        int Hk, int Hv, int dk, int dv, float l2_eps, gdn_dtype dtype,
+                        gdn_stream_t stream) {
+  return gdn_prologue_ex(q_raw, k_raw, v_raw, nullptr, nullptr, nullptr, wq, wk, wv, q, k, v, B,
+                         T, Hk, Hv, dk, dv, l2_eps, dtype, stream);
 }
 
 gdn_status gdn_out_norm(const void* o, const void* z, const float* w, void* y, long long rows,
@@ -683,19 +697,55 @@ size_t gdn_layer_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, i
   return qkv + up(tok * Hv * dv * 4) + tc;
 }
 
-gdn_status gdn_layer_fwd(const void* q_raw, const void* k_raw, const void* v_raw, const void* z,
-                         const float* wq, const float* wk, const float* wv,
-                         const float* log_alpha, const float* beta, const float* S0,
-                         const float* norm_w, void* y, float* S_T, void* workspace,
-                         size_t workspace_bytes, int B, int T, int Hk, int Hv, int dk, int dv,
-                         int chunk, float scale, float l2_eps, float norm_eps, gdn_dtype dtype,
-                         gdn_dtype y_dtype, gdn_stream_t stream) {
+// The conv history after a layer call: the last three raw rows of [history; x] for the q, k and
+// v channels (see conv_hist_out_kernel).
+static gdn_status layer_hist_out(const void* q_raw, const void* k_raw, const void* v_raw,
+                          const void* hq_in, const void* hk_in, const void* hv_in, void* hq_out,
+                          void* hk_out, void* hv_out, int B, int T, int Hk, int Hv, int dk, int dv,
+                          gdn_dtype dtype, cudaStream_t st) {
+  const void* x[] = {q_raw, k_raw, v_raw};
+  const void* hin[] = {hq_in, hk_in, hv_in};
+  void* hout[] = {hq_out, hk_out, hv_out};
+  const int width[] = {Hk * dk, Hk * dk, Hv * dv};
+  for (int i = 0; i < 3; ++i) {
+    if (!hout[i]) continue;
+    const long pieces = (long)B * 3 * width[i] / (dtype == GDN_F32 ? 4 : 8);
+    const unsigned blocks = (unsigned)((pieces + 255) / 256);
+    if (blocks == 0) continue;
+    if (dtype == GDN_F32)
+      conv_hist_out_kernel<float><<<blocks, 256, 0, st>>>(
+          (const float*)x[i], (const float*)hin[i], (float*)hout[i], B, T, width[i]);
+    else
+      conv_hist_out_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(
+          (const __nv_bfloat16*)x[i], (const __nv_bfloat16*)hin[i], (__nv_bfloat16*)hout[i], B,
+          T, width[i]);
+  }
+  return launch_status();
+}
+
+gdn_status gdn_layer_fwd_ex(const void* q_raw, const void* k_raw, const void* v_raw,
+                            const void* z, const void* hq_in, const void* hk_in,
+                            const void* hv_in, const float* wq, const float* wk, const float* wv,
+                            const float* log_alpha, const float* beta, const float* S0,
+                            const float* norm_w, void* y, float* S_T, void* hq_out,
+                            void* hk_out, void* hv_out, void* workspace, size_t workspace_bytes,
+                            int B, int T, int Hk, int Hv, int dk, int dv, int chunk, float scale,
+                            float l2_eps, float norm_eps, gdn_dtype dtype, gdn_dtype y_dtype,
+                            gdn_stream_t stream) {
   if (B < 0 || T < 0 || !valid_dtype(dtype) || !valid_dtype(y_dtype)) return GDN_ERR_INVALID_ARG;
   if (!io_pair_ok(dtype, y_dtype)) return GDN_ERR_UNSUPPORTED;
   gdn_status s = validate_heads(Hk, Hv, dk, dv);
   if (s != GDN_OK) return s;
   if (chunk <= 0 || !(norm_eps >= 0.f)) return GDN_ERR_INVALID_ARG;
   if (!supported_chunk(chunk)) return GDN_ERR_UNSUPPORTED;
+  const void* hs[] = {hq_in, hk_in, hv_in, hq_out, hk_out, hv_out};
+  for (const void* p : hs)
+    if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+  if ((hq_out && hq_out == hq_in) || (hk_out && hk_out == hk_in) ||
+      (hv_out && hv_out == hv_in))
+    return GDN_ERR_INVALID_ARG;
+  if ((long)B * T > 0 && (hq_out || hk_out || hv_out) && (!q_raw || !k_raw || !v_raw))
+    return GDN_ERR_INVALID_ARG;
   const bool tc = tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16);
   if (tc && !tc_chunk_length_ok(T)) return GDN_ERR_UNSUPPORTED;
   const size_t need = gdn_layer_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, dtype);
@@ -704,9 +754,14 @@ gdn_status gdn_layer_fwd(const void* q_raw, const void* k_raw, const void* v_raw
       return GDN_ERR_INVALID_ARG;
     if (!workspace_ok(workspace, workspace_bytes, need)) return GDN_ERR_INVALID_ARG;
   }
-  if ((long)B * T == 0)
-    return gdn_chunk_fwd(nullptr, nullptr, nullptr, nullptr, nullptr, S0, nullptr, S_T, nullptr, 0,
-                         B, T, Hk, Hv, dk, dv, chunk, scale, dtype, dtype, stream);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if ((long)B * T == 0) {
+    s = gdn_chunk_fwd(nullptr, nullptr, nullptr, nullptr, nullptr, S0, nullptr, S_T, nullptr, 0,
+                      B, T, Hk, Hv, dk, dv, chunk, scale, dtype, dtype, stream);
+    if (s != GDN_OK) return s;
+    return layer_hist_out(q_raw, k_raw, v_raw, hq_in, hk_in, hv_in, hq_out, hk_out, hv_out, B, T,
+                          Hk, Hv, dk, dv, dtype, st);
+  }
   const size_t el = dtype == GDN_F32 ? 4 : 2;
   const size_t tok = (size_t)B * T;
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
@@ -715,10 +770,9 @@ gdn_status gdn_layer_fwd(const void* q_raw, const void* k_raw, const void* v_raw
   void* kn = ws + up(tok * Hk * dk * el);
   void* vc = ws + 2 * up(tok * Hk * dk * el);
   char* rest = ws + 2 * up(tok * Hk * dk * el) + up(tok * Hv * dv * el);
-  s = gdn_prologue(q_raw, k_raw, v_raw, wq, wk, wv, qn, kn, vc, B, T, Hk, Hv, dk, dv, l2_eps,
-                   dtype, stream);
+  s = gdn_prologue_ex(q_raw, k_raw, v_raw, hq_in, hk_in, hv_in, wq, wk, wv, qn, kn, vc, B, T, Hk,
+                      Hv, dk, dv, l2_eps, dtype, stream);
   if (s != GDN_OK) return s;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // the recurrence writes o in fp32 so that the gated norm reads it unrounded
   float* o = reinterpret_cast<float*>(rest);
   void* tc_scratch = rest + up(tok * Hv * dv * 4);
@@ -737,7 +791,23 @@ gdn_status gdn_layer_fwd(const void* q_raw, const void* k_raw, const void* v_raw
   else
     out_norm_kernel<float, __nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
         (const float*)o, (const __nv_bfloat16*)z, norm_w, (__nv_bfloat16*)y, rows, dv, norm_eps);
-  return launch_status();
+  s = launch_status();
+  if (s != GDN_OK) return s;
+  return layer_hist_out(q_raw, k_raw, v_raw, hq_in, hk_in, hv_in, hq_out, hk_out, hv_out, B, T,
+                        Hk, Hv, dk, dv, dtype, st);
+}
+
+gdn_status gdn_layer_fwd(const void* q_raw, const void* k_raw, const void* v_raw, const void* z,
+                         const float* wq, const float* wk, const float* wv,
+                         const float* log_alpha, const float* beta, const float* S0,
+                         const float* norm_w, void* y, float* S_T, void* workspace,
+                         size_t workspace_bytes, int B, int T, int Hk, int Hv, int dk, int dv,
+                         int chunk, float scale, float l2_eps, float norm_eps, gdn_dtype dtype,
+                         gdn_dtype y_dtype, gdn_stream_t stream) {
+  return gdn_layer_fwd_ex(q_raw, k_raw, v_raw, z, nullptr, nullptr, nullptr, wq, wk, wv,
+                          log_alpha, beta, S0, norm_w, y, S_T, nullptr, nullptr, nullptr,
+                          workspace, workspace_bytes, B, T, Hk, Hv, dk, dv, chunk, scale, l2_eps,
+                          norm_eps, dtype, y_dtype, stream);
 }
 
 }  // extern "C"

@@ -353,7 +353,8 @@ GDN_API gdn_status gdn_gates(const void *ba, float *log_alpha, float *beta, long
  * channel; "Les briques d'un réseau de neurones", 2.: SiLU(x) = x sigmoid(x).)
  *   q_raw, k_raw [B, T, Hk*dk]; v_raw [B, T, Hv*dv]         (dtype)
  *   wq, wk [Hk*dk, 4]; wv [Hv*dv, 4] float: tap 3 multiplies the current token, tap 0 the token
- *        three steps back; positions before t = 0 are zeros (no carried conv state).
+ *        three steps back; positions before t = 0 are zeros (gdn_prologue_ex carries the
+ *        previous tokens instead).
  *   q, k [B, T, Hk, dk]; v [B, T, Hv, dv]                    (dtype, outputs)
  * bf16 outputs are the exact results rounded to the nearest bf16 (ties to even): a value whose
  * rounding the fp32 computation cannot decide within its error bound is recomputed in fp64, so
@@ -366,6 +367,23 @@ GDN_API gdn_status gdn_prologue(const void *q_raw, const void *k_raw, const void
                         void *q, void *k, void *v,
                         int B, int T, int Hk, int Hv, int dk, int dv, float l2_eps,
                         gdn_dtype dtype, gdn_stream_t stream);
+
+/*
+ * gdn_prologue continuing a sequence: the convolution at tokens 0, 1, 2 reads the raw inputs of
+ * the three tokens before the call from a carried history instead of zeros, so that a sequence
+ * run in pieces gets the outputs of one run ("Chapitre 16 - Assembler un système de type Kimi
+ * K3", 16.2: prefill in blocks, the state handed from block to block; the conv's three inputs are
+ * part of that state, as in gdn_decode_layer_step).
+ *   hq_in, hk_in [B, 3, Hk*dk]; hv_in [B, 3, Hv*dv] (dtype, 16-byte aligned): the raw inputs of
+ *        the three previous tokens, oldest first; NULL means zeros (a fresh sequence).
+ * Everything else as gdn_prologue.
+ */
+GDN_API gdn_status gdn_prologue_ex(const void *q_raw, const void *k_raw, const void *v_raw,
+                           const void *hq_in, const void *hk_in, const void *hv_in,
+                           const float *wq, const float *wk, const float *wv,
+                           void *q, void *k, void *v,
+                           int B, int T, int Hk, int Hv, int dk, int dv, float l2_eps,
+                           gdn_dtype dtype, gdn_stream_t stream);
 
 /*
  * Output gate: y = o / sqrt(mean(o^2) + eps) * w (.) SiLU(z) for each row of dv values
@@ -394,6 +412,32 @@ GDN_API gdn_status gdn_layer_fwd(const void *q_raw, const void *k_raw, const voi
                          int B, int T, int Hk, int Hv, int dk, int dv, int chunk,
                          float scale, float l2_eps, float norm_eps,
                          gdn_dtype dtype, gdn_dtype y_dtype, gdn_stream_t stream);
+
+/*
+ * gdn_layer_fwd continuing a sequence (prefill in pieces, or prefill followed by
+ * gdn_decode_layer_step): the conv reads a carried history of the three previous tokens' raw
+ * inputs, and the history after the call can be written out.  Run in pieces, with S0 = the
+ * previous piece's S_T and the history passed on, a sequence gets the outputs of one run (bit for
+ * bit when each piece but the last is a multiple of `chunk` tokens long; otherwise the pieces'
+ * chunk boundaries differ and the results differ by rounding).  ("Chapitre 16 - Assembler un
+ * système de type Kimi K3", 16.2 and 16.3: the state handed from block to block, then read and
+ * updated by decode; the conv's inputs are part of it.)
+ *   hq_in, hk_in [B, 3, Hk*dk]; hv_in [B, 3, Hv*dv] (dtype): raw inputs of the three tokens
+ *        before the call, oldest first; NULL means zeros (a fresh sequence).
+ *   hq_out, hk_out, hv_out: same shapes (dtype), written with the raw inputs of the last three
+ *        tokens of [history; this call's tokens], the history gdn_decode_layer_step or the next
+ *        piece takes; NULL skips it.  They must not overlap the _in buffers or any input.
+ * History pointers are 16-byte aligned.  Everything else as gdn_layer_fwd (same workspace size).
+ */
+GDN_API gdn_status gdn_layer_fwd_ex(const void *q_raw, const void *k_raw, const void *v_raw,
+                            const void *z, const void *hq_in, const void *hk_in,
+                            const void *hv_in, const float *wq, const float *wk, const float *wv,
+                            const float *log_alpha, const float *beta, const float *S0,
+                            const float *norm_w, void *y, float *S_T, void *hq_out,
+                            void *hk_out, void *hv_out, void *workspace, size_t workspace_bytes,
+                            int B, int T, int Hk, int Hv, int dk, int dv, int chunk, float scale,
+                            float l2_eps, float norm_eps, gdn_dtype dtype, gdn_dtype y_dtype,
+                            gdn_stream_t stream);
 
 /* Scratch bytes gdn_layer_fwd needs for these sizes (host only, no CUDA call); 0 if none. */
 GDN_API size_t gdn_layer_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, int chunk,

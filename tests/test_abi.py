@@ -293,3 +293,24 @@ def test_layer_bwd_workspace_and_gates_bwd_validation(L):
     assert L.gdn_gates_bwd(FAKE, FAKE, FAKE, FAKE, -1, 4, 1, None) == 1
     assert L.gdn_gates_bwd(None, FAKE, FAKE, FAKE, 10, 4, 1, None) == 1
     assert L.gdn_gates_bwd(FAKE, FAKE, FAKE, FAKE, 0, 4, 1, None) == 0
+
+
+def test_prologue_ex_and_layer_ex_validation(L):
+    """The conv-history calls: a misaligned history, or a history out that is the history in,
+    returns GDN_ERR_INVALID_ARG (1) before any work; null histories are allowed (fresh
+    sequences) and T = 0 with none is a no-op."""
+    bad = P(0x1008)
+    assert L.gdn_prologue_ex(FAKE, FAKE, FAKE, bad, None, None, *([FAKE] * 6), 1, 8, 2, 4, 16,
+                             16, 1e-6, 1, None) == 1
+    assert L.gdn_prologue_ex(*([FAKE] * 3), None, None, None, *([FAKE] * 6), 1, 0, 2, 4, 16, 16,
+                             1e-6, 1, None) == 0                       # T = 0
+    head = [FAKE] * 4                                   # q_raw, k_raw, v_raw, z
+    mid = [FAKE] * 9                                    # wq .. S_T
+    ws = [P(0x100000), 1 << 40]
+    sizes = [1, 8, 2, 4, 16, 16, 16, 1.0, 1e-6, 1e-5, 1, 1, None]
+    # misaligned history in / out
+    assert L.gdn_layer_fwd_ex(*head, bad, None, None, *mid, None, None, None, *ws, *sizes) == 1
+    assert L.gdn_layer_fwd_ex(*head, None, None, None, *mid, None, bad, None, *ws, *sizes) == 1
+    # a history out that is the history in
+    h = P(0x2000)
+    assert L.gdn_layer_fwd_ex(*head, None, None, h, *mid, None, None, h, *ws, *sizes) == 1
