@@ -307,6 +307,8 @@ GDN_API size_t gdn_bwd_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int
  *   workspace: gdn_layer_bwd_workspace_bytes(...) bytes, 256-byte aligned, owned by the caller.
  * dk == dv (else GDN_ERR_UNSUPPORTED); other limits as gdn_layer_fwd and gdn_bwd.  Weight
  * gradients are sums of per-CTA partial sums taken in a fixed order (reproducible bit for bit).
+ * The sequence starts fresh: the conv sees zeros before token 0, as in gdn_layer_fwd (there is
+ * no backward of gdn_layer_fwd_ex's carried history).
  */
 GDN_API gdn_status gdn_layer_bwd(const void *q_raw, const void *k_raw, const void *v_raw,
                          const void *z, const float *wq, const float *wk, const float *wv,
