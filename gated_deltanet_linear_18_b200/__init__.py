@@ -90,6 +90,11 @@ def lib() -> ctypes.CDLL:
         L.gdn_layer_fwd.restype = I
         L.gdn_layer_fwd_ex.argtypes = [P] * 20 + [SZ] + [I] * 7 + [F, F, F, I, I, P]
         L.gdn_layer_fwd_ex.restype = I
+        L.gdn_layer_fwd_varlen.argtypes = [P] * 5 + [I, I] + [P] * 16 + [SZ] + [I] * 6 + \
+            [F, F, F, I, I, P]
+        L.gdn_layer_fwd_varlen.restype = I
+        L.gdn_layer_fwd_varlen_workspace_bytes.argtypes = [I] * 9
+        L.gdn_layer_fwd_varlen_workspace_bytes.restype = SZ
         L.gdn_layer_workspace_bytes.argtypes = [I] * 7 + [I]
         L.gdn_layer_fwd_static.argtypes = [P] * 13 + [I] * 7 + [F, F, F, I, I, P]
         L.gdn_layer_fwd_static.restype = I
@@ -473,6 +478,47 @@ def layer_fwd(q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, *
                                     float(scale), float(l2_eps), float(norm_eps),
                                     _io_dtype(q_raw), _io_dtype(y), _stream(dev))
     _check("gdn_layer_fwd_ex", st)
+    if want_hist:
+        return y, sT, ho
+    return y, sT
+
+
+def layer_fwd_varlen(q_raw, k_raw, v_raw, z, cu_seqlens, max_seqlen: int, wq, wk, wv,
+                     log_alpha, beta, S0, norm_w, *, Hk: int, Hv: int, dk: int, dv: int,
+                     chunk: int = 64, scale: float = 1.0, l2_eps: float = 1e-6,
+                     norm_eps: float = 1e-5, hist=None, want_hist: bool = False,
+                     out_dtype: Optional[torch.dtype] = None):
+    """The layer over packed requests: raw q, k [total, Hk*dk], v, z [total, Hv*dv], gates
+    [total, Hv], cu_seqlens [nseq+1] int32 (device), S0 [nseq, Hv, dk, dv] or None, ``hist``
+    (hq, hk, hv) [nseq, 3, C] or None.  Returns (y [total, Hv, dv], S_T) and, with
+    ``want_hist``, the histories after the call."""
+    total = q_raw.shape[0]
+    nseq = cu_seqlens.numel() - 1
+    if cu_seqlens.dtype != torch.int32:
+        raise ValueError("cu_seqlens must be int32")
+    _f32(wq, wk, wv, log_alpha, beta, S0, norm_w)
+    hq, hk, hv = _hist_shapes(nseq, Hk, Hv, dk, dv, hist)
+    dev = q_raw.device
+    y = torch.empty(total, Hv, dv, device=dev, dtype=out_dtype or q_raw.dtype)
+    sT = torch.empty(nseq, Hv, dk, dv, device=dev, dtype=torch.float32)
+    ho = (None, None, None)
+    if want_hist:
+        ho = (torch.empty(nseq, 3, Hk * dk, device=dev, dtype=q_raw.dtype),
+              torch.empty(nseq, 3, Hk * dk, device=dev, dtype=q_raw.dtype),
+              torch.empty(nseq, 3, Hv * dv, device=dev, dtype=q_raw.dtype))
+    need = int(lib().gdn_layer_fwd_varlen_workspace_bytes(nseq, max_seqlen, total, Hk, Hv, dk, dv,
+                                                          chunk, _DTYPES[q_raw.dtype]))
+    ws = torch.empty(max(need, 1), device=dev, dtype=torch.uint8)
+    d = _dev(q_raw, k_raw, v_raw, z, cu_seqlens, wq, wk, wv, log_alpha, beta, S0, norm_w, y, sT,
+             hq, hk, hv, *ho)
+    with torch.cuda.device(d):
+        st = lib().gdn_layer_fwd_varlen(
+            _p(q_raw), _p(k_raw), _p(v_raw), _p(z), _p(cu_seqlens), nseq, int(max_seqlen), _p(hq),
+            _p(hk), _p(hv), _p(wq), _p(wk), _p(wv), _p(log_alpha), _p(beta), _p(S0), _p(norm_w),
+            _p(y), _p(sT), _p(ho[0]), _p(ho[1]), _p(ho[2]), _p(ws), need, total, Hk, Hv, dk, dv,
+            chunk, float(scale), float(l2_eps), float(norm_eps), _io_dtype(q_raw), _io_dtype(y),
+            _stream(d))
+    _check("gdn_layer_fwd_varlen", st)
     if want_hist:
         return y, sT, ho
     return y, sT

@@ -88,6 +88,21 @@ __device__ __forceinline__ float rcp_fast(float x) {
 
 constexpr int kPrologueList = 1024;     // undecided values one CTA redoes in fp64 afterwards
 
+// Rows of sequence s: of [B, T, ...] tensors (cu == nullptr), rows s T .. s T + T - 1; packed
+// (cu != nullptr), rows cu[s] .. cu[s + 1] - 1 of [T, ...] tensors (T = total rows), clamped to
+// the tensor and cut at max_len, so that malformed offsets cannot reach outside it.
+struct RowSpan {
+  long row0;
+  int len;
+};
+__device__ __forceinline__ RowSpan row_span(const int* __restrict__ cu, int s, int T,
+                                            int max_len) {
+  if (!cu) return RowSpan{(long)s * T, T};
+  const int a = min(max(cu[s], 0), T);
+  const int b = min(max(cu[s + 1], a), min(T, a + max_len));
+  return RowSpan{(long)a, b - a};
+}
+
 // The staged tile of one prologue CTA: the raw rows of tokens t0 - 3 .. t0 + kPrologueTokens - 1
 // of one head of d channels, row r holding token t0 - 3 + r, brought in by 16-byte asynchronous
 // copies that are all issued at once (many tiles in flight per SM).  Tokens -3 .. -1 come from the
@@ -165,7 +180,8 @@ __device__ __forceinline__ bool bf16_decided_e24(float y, float E) {
 template <typename Tio>
 __global__ void __launch_bounds__(128, 6)
 prologue_v_kernel(const Tio* __restrict__ x, const Tio* __restrict__ hist,
-                  const float* __restrict__ w, Tio* __restrict__ y, int T, int Hv, int dv) {
+                  const float* __restrict__ w, Tio* __restrict__ y, int T, int Hv, int dv,
+                  const int* __restrict__ cu, int max_len) {
   constexpr bool kBf16 = sizeof(Tio) == 2;
   extern __shared__ __align__(16) uint8_t pro_smem[];
   Tio* tile = reinterpret_cast<Tio*>(pro_smem);
@@ -174,11 +190,14 @@ prologue_v_kernel(const Tio* __restrict__ x, const Tio* __restrict__ hist,
   const int head = blockIdx.x, d = dv, width = Hv * dv;
   const long b = blockIdx.z;
   const long t0 = (long)blockIdx.y * kPrologueTokens;
+  const RowSpan sp = row_span(cu, (int)b, T, max_len);
+  if (t0 >= sp.len) return;                   // past this sequence's end (uniform, no barrier yet)
   const int L = d / 4, grp = threadIdx.x / L, lc = threadIdx.x % L, ngrp = 128 / L;
   const int tpg = kPrologueTokens / ngrp, i0 = grp * tpg;  // this row group's tokens
   if (threadIdx.x == 0) nlist = 0;
-  prologue_stage(tile, x + b * T * (long)width + (long)head * d,
-                 hist ? hist + b * 3 * (long)width + (long)head * d : nullptr, t0, T, width, d);
+  prologue_stage(tile, x + sp.row0 * width + (long)head * d,
+                 hist ? hist + b * 3 * (long)width + (long)head * d : nullptr, t0, sp.len, width,
+                 d);
   const long c0 = (long)head * d + lc * 4;    // first channel of this thread
   float wk[4][4];                             // [channel][tap]
 #pragma unroll
@@ -186,9 +205,9 @@ prologue_v_kernel(const Tio* __restrict__ x, const Tio* __restrict__ hist,
 #pragma unroll
     for (int k = 0; k < 4; ++k) wk[c][k] = w[(c0 + c) * 4 + k];   // 4-byte alignment only
   __syncthreads();
-  const long rem = T - t0;
+  const long rem = sp.len - t0;
   const int nt = rem < kPrologueTokens ? (int)rem : kPrologueTokens;
-  Tio* const yt = y + (b * T + t0) * width + c0;          // this thread's channels of token t0
+  Tio* const yt = y + (sp.row0 + t0) * width + c0;        // this thread's channels of token t0
   const Tio* const xr = tile + lc * 4;                    // ... of tile row 0
   // token i reads tile rows i .. i + 3 at ring slots i .. i + 3 (mod 4): with the token loop
   // unrolled by four no row is ever moved
@@ -236,7 +255,8 @@ prologue_v_kernel(const Tio* __restrict__ x, const Tio* __restrict__ hist,
     }
     __syncthreads();                          // the list is complete, the fast values stored
     const int n = nlist;
-    __nv_bfloat16* yb = reinterpret_cast<__nv_bfloat16*>(y) + (b * T + t0) * width + (long)head * d;
+    __nv_bfloat16* yb =
+        reinterpret_cast<__nv_bfloat16*>(y) + (sp.row0 + t0) * width + (long)head * d;
     const __nv_bfloat16* tb16 = reinterpret_cast<const __nv_bfloat16*>(tile);
     const float* wh = w + (long)head * d * 4;
     if (n <= kPrologueList) {
@@ -270,7 +290,8 @@ __global__ void __launch_bounds__(128, 5)
 prologue_qk_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
                    const Tio* __restrict__ hq, const Tio* __restrict__ hk,
                    const float* __restrict__ wq, const float* __restrict__ wk,
-                   Tio* __restrict__ yq, Tio* __restrict__ yk, int T, int Hk, int dk, float eps) {
+                   Tio* __restrict__ yq, Tio* __restrict__ yk, int T, int Hk, int dk, float eps,
+                   const int* __restrict__ cu, int max_len) {
   constexpr int N = 4;                        // channels per thread
   constexpr bool kBf16 = sizeof(Tio) == 2;
   constexpr float u = 5.9604645e-8f;
@@ -286,11 +307,14 @@ prologue_qk_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
   Tio* y = isq ? yq : yk;
   const long b = blockIdx.z;
   const long t0 = (long)blockIdx.y * kPrologueTokens;
+  const RowSpan sp = row_span(cu, (int)b, T, max_len);
+  if (t0 >= sp.len) return;                   // past this sequence's end (uniform, no barrier yet)
   const int L = d / N, grp = threadIdx.x / L, lc = threadIdx.x % L, ngrp = 128 / L;
   const int tpg = kPrologueTokens / ngrp, i0 = grp * tpg;
   if (threadIdx.x == 0) nlist = 0;
-  prologue_stage(tile, x + b * T * (long)width + (long)head * d,
-                 hist ? hist + b * 3 * (long)width + (long)head * d : nullptr, t0, T, width, d);
+  prologue_stage(tile, x + sp.row0 * width + (long)head * d,
+                 hist ? hist + b * 3 * (long)width + (long)head * d : nullptr, t0, sp.len, width,
+                 d);
   const long c0 = (long)head * d + lc * N;
   float wt[N][4];
 #pragma unroll
@@ -298,9 +322,9 @@ prologue_qk_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
 #pragma unroll
     for (int j = 0; j < 4; ++j) wt[i][j] = w[(c0 + i) * 4 + j];
   __syncthreads();
-  const long rem = T - t0;
+  const long rem = sp.len - t0;
   const int nt = rem < kPrologueTokens ? (int)rem : kPrologueTokens;
-  Tio* const yt = y + (b * T + t0) * width + c0;
+  Tio* const yt = y + (sp.row0 + t0) * width + c0;
   if constexpr (!kBf16) {                     // fp32 outputs: fp32 throughout
     float h0[N], h1[N], h2[N];
     Vec4<Tio>::load(tile + (long)i0 * d + lc * N, h0);
@@ -401,7 +425,8 @@ prologue_qk_kernel(const Tio* __restrict__ xq, const Tio* __restrict__ xk,
     }
     __syncthreads();                          // the list is complete, the fast values stored
     const int n = nlist;
-    __nv_bfloat16* yb = reinterpret_cast<__nv_bfloat16*>(y) + (b * T + t0) * width + (long)head * d;
+    __nv_bfloat16* yb =
+        reinterpret_cast<__nv_bfloat16*>(y) + (sp.row0 + t0) * width + (long)head * d;
     const __nv_bfloat16* tb16 = reinterpret_cast<const __nv_bfloat16*>(tile);
     const float* wh = w + (long)head * d * 4;
     // one row per group of L threads (the row's norm by shuffles over those lanes)
@@ -464,21 +489,23 @@ out_norm_kernel(const To* __restrict__ o, const Tz* __restrict__ z, const float*
 }
 
 // The conv history after a call: the raw rows of the last three tokens of [history; x] (oldest
-// first), per sequence, for `width` channels: row r is token T + r of that concatenation, from the
-// incoming history hin while T + r < 3 (zeros when there is none), else from x.  One thread per
-// 16-byte piece of a row.
+// first), per sequence, for `width` channels: with the sequence's length n, row r is token n + r of
+// that concatenation, from the incoming history hin while n + r < 3 (zeros when there is none),
+// else from x.  Sequences as in row_span.  One thread per 16-byte piece of a row.
 template <typename Tio>
 __global__ void conv_hist_out_kernel(const Tio* __restrict__ x, const Tio* __restrict__ hin,
-                                     Tio* __restrict__ hout, long B, int T, int width) {
+                                     Tio* __restrict__ hout, long B, int T, int width,
+                                     const int* __restrict__ cu, int max_len) {
   constexpr int N = 16 / sizeof(Tio);
   const int P = width / N;
   const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= B * 3 * P) return;
   const long b = i / (3 * P);
   const int r = (int)(i / P % 3), c = (int)(i % P);
-  const long s = (long)T + r;                 // position in [history; x]
+  const RowSpan sp = row_span(cu, (int)b, T, max_len);
+  const long s = (long)sp.len + r;            // position in [history; x]
   uint4 v = make_uint4(0u, 0u, 0u, 0u);
-  if (s >= 3) v = reinterpret_cast<const uint4*>(x + (b * T + s - 3) * (long)width)[c];
+  if (s >= 3) v = reinterpret_cast<const uint4*>(x + (sp.row0 + s - 3) * (long)width)[c];
   else if (hin) v = reinterpret_cast<const uint4*>(hin + (b * 3 + s) * (long)width)[c];
   reinterpret_cast<uint4*>(hout + (b * 3 + r) * (long)width)[c] = v;
 }

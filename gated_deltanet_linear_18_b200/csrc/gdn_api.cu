@@ -604,6 +604,46 @@ gdn_status gdn_decode_step(const void* q, const void* k, const void* v, const fl
                                                        Hk, Hv, scale, st);
 }
 
+// The two prologue kernels for `nseq` sequences (cu == nullptr: [nseq, T] rows; else packed rows
+// cu[s] .. cu[s + 1] - 1 of T in all, none longer than max_len), arguments already checked.  The q
+// and k heads (normalised rows) run on the library's high-priority stream, forked from and joined
+// back into `stream`, beside the v heads on `stream`: the two kernels share the SMs (both are
+// bound by instruction issue and latency, not by HBM); head slots fastest in each grid.
+static gdn_status prologue_launch(const void* q_raw, const void* k_raw, const void* v_raw,
+                                  const void* hq_in, const void* hk_in, const void* hv_in,
+                                  const float* wq, const float* wk, const float* wv, void* q,
+                                  void* k, void* v, int nseq, int T, int Hk, int Hv, int dk,
+                                  int dv, float l2_eps, gdn_dtype dtype, const int* cu,
+                                  int max_len, cudaStream_t st) {
+  const unsigned tb = (unsigned)((max_len + kPrologueTokens - 1) / kPrologueTokens);
+  const dim3 gqk(2 * Hk, tb, nseq), gv(Hv, tb, nseq);
+  std::lock_guard<std::mutex> lock(tcf::split_mutex());
+  tcf::Split* sp = tcf::split_for_device();
+  if (!sp || cudaEventRecord(sp->ev_fork, st) != cudaSuccess ||
+      cudaStreamWaitEvent(sp->s_hi, sp->ev_fork, 0) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  if (dtype == GDN_F32) {
+    prologue_qk_kernel<float><<<gqk, 128, prologue_smem_bytes(dk, 4), sp->s_hi>>>(
+        (const float*)q_raw, (const float*)k_raw, (const float*)hq_in, (const float*)hk_in, wq,
+        wk, (float*)q, (float*)k, T, Hk, dk, l2_eps, cu, max_len);
+    prologue_v_kernel<float><<<gv, 128, prologue_smem_bytes(dv, 4), st>>>(
+        (const float*)v_raw, (const float*)hv_in, wv, (float*)v, T, Hv, dv, cu, max_len);
+  } else {
+    using bf = __nv_bfloat16;
+    prologue_qk_kernel<bf><<<gqk, 128, prologue_smem_bytes(dk, 2), sp->s_hi>>>(
+        (const bf*)q_raw, (const bf*)k_raw, (const bf*)hq_in, (const bf*)hk_in, wq, wk, (bf*)q,
+        (bf*)k, T, Hk, dk, l2_eps, cu, max_len);
+    prologue_v_kernel<bf><<<gv, 128, prologue_smem_bytes(dv, 2), st>>>(
+        (const bf*)v_raw, (const bf*)hv_in, wv, (bf*)v, T, Hv, dv, cu, max_len);
+  }
+  const gdn_status ls = launch_status();
+  // the caller's stream waits for the q/k kernel, also after a failed launch
+  if (cudaEventRecord(sp->ev_hi, sp->s_hi) != cudaSuccess ||
+      cudaStreamWaitEvent(st, sp->ev_hi, 0) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  return ls;
+}
+
 gdn_status gdn_prologue_ex(const void* q_raw, const void* k_raw, const void* v_raw,
                            const void* hq_in, const void* hk_in, const void* hv_in,
                            const float* wq, const float* wk, const float* wv, void* q, void* k,
@@ -622,38 +662,10 @@ gdn_status gdn_prologue_ex(const void* q_raw, const void* k_raw, const void* v_r
     if (!p || !aligned16(p)) return GDN_ERR_INVALID_ARG;
   if (!wq || !wk || !wv || !aligned4(wq) || !aligned4(wk) || !aligned4(wv))
     return GDN_ERR_INVALID_ARG;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if ((T + kPrologueTokens - 1) / kPrologueTokens > 65535) return GDN_ERR_UNSUPPORTED;
-  // the q and k heads (normalised rows) on the library's high-priority stream, forked from and
-  // joined back into `stream`, beside the v heads on `stream`: the two kernels share the SMs (both
-  // are bound by instruction issue and latency, not by HBM); head slots fastest in each grid
-  const unsigned tb = (unsigned)((T + kPrologueTokens - 1) / kPrologueTokens);
-  const dim3 gqk(2 * Hk, tb, B), gv(Hv, tb, B);
-  std::lock_guard<std::mutex> lock(tcf::split_mutex());
-  tcf::Split* sp = tcf::split_for_device();
-  if (!sp || cudaEventRecord(sp->ev_fork, st) != cudaSuccess ||
-      cudaStreamWaitEvent(sp->s_hi, sp->ev_fork, 0) != cudaSuccess)
-    return GDN_ERR_CUDA;
-  if (dtype == GDN_F32) {
-    prologue_qk_kernel<float><<<gqk, 128, prologue_smem_bytes(dk, 4), sp->s_hi>>>(
-        (const float*)q_raw, (const float*)k_raw, (const float*)hq_in, (const float*)hk_in, wq,
-        wk, (float*)q, (float*)k, T, Hk, dk, l2_eps);
-    prologue_v_kernel<float><<<gv, 128, prologue_smem_bytes(dv, 4), st>>>(
-        (const float*)v_raw, (const float*)hv_in, wv, (float*)v, T, Hv, dv);
-  } else {
-    using bf = __nv_bfloat16;
-    prologue_qk_kernel<bf><<<gqk, 128, prologue_smem_bytes(dk, 2), sp->s_hi>>>(
-        (const bf*)q_raw, (const bf*)k_raw, (const bf*)hq_in, (const bf*)hk_in, wq, wk, (bf*)q,
-        (bf*)k, T, Hk, dk, l2_eps);
-    prologue_v_kernel<bf><<<gv, 128, prologue_smem_bytes(dv, 2), st>>>(
-        (const bf*)v_raw, (const bf*)hv_in, wv, (bf*)v, T, Hv, dv);
-  }
-  const gdn_status ls = launch_status();
-  // the caller's stream waits for the q/k kernel, also after a failed launch
-  if (cudaEventRecord(sp->ev_hi, sp->s_hi) != cudaSuccess ||
-      cudaStreamWaitEvent(st, sp->ev_hi, 0) != cudaSuccess)
-    return GDN_ERR_CUDA;
-  return ls;
+  return prologue_launch(q_raw, k_raw, v_raw, hq_in, hk_in, hv_in, wq, wk, wv, q, k, v, B, T, Hk,
+                         Hv, dk, dv, l2_eps, dtype, nullptr, T,
+                         reinterpret_cast<cudaStream_t>(stream));
 }
 
 gdn_status gdn_prologue(const void* q_raw, const void* k_raw, const void* v_raw, const float* wq,
@@ -700,9 +712,10 @@ size_t gdn_layer_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, i
 // The conv history after a layer call: the last three raw rows of [history; x] for the q, k and
 // v channels (see conv_hist_out_kernel).
 static gdn_status layer_hist_out(const void* q_raw, const void* k_raw, const void* v_raw,
-                          const void* hq_in, const void* hk_in, const void* hv_in, void* hq_out,
-                          void* hk_out, void* hv_out, int B, int T, int Hk, int Hv, int dk, int dv,
-                          gdn_dtype dtype, cudaStream_t st) {
+                                 const void* hq_in, const void* hk_in, const void* hv_in,
+                                 void* hq_out, void* hk_out, void* hv_out, int B, int T, int Hk,
+                                 int Hv, int dk, int dv, gdn_dtype dtype, cudaStream_t st,
+                                 const int* cu = nullptr, int max_len = 0) {
   const void* x[] = {q_raw, k_raw, v_raw};
   const void* hin[] = {hq_in, hk_in, hv_in};
   void* hout[] = {hq_out, hk_out, hv_out};
@@ -714,11 +727,11 @@ static gdn_status layer_hist_out(const void* q_raw, const void* k_raw, const voi
     if (blocks == 0) continue;
     if (dtype == GDN_F32)
       conv_hist_out_kernel<float><<<blocks, 256, 0, st>>>(
-          (const float*)x[i], (const float*)hin[i], (float*)hout[i], B, T, width[i]);
+          (const float*)x[i], (const float*)hin[i], (float*)hout[i], B, T, width[i], cu, max_len);
     else
       conv_hist_out_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(
           (const __nv_bfloat16*)x[i], (const __nv_bfloat16*)hin[i], (__nv_bfloat16*)hout[i], B,
-          T, width[i]);
+          T, width[i], cu, max_len);
   }
   return launch_status();
 }
@@ -808,6 +821,97 @@ gdn_status gdn_layer_fwd(const void* q_raw, const void* k_raw, const void* v_raw
                           log_alpha, beta, S0, norm_w, y, S_T, nullptr, nullptr, nullptr,
                           workspace, workspace_bytes, B, T, Hk, Hv, dk, dv, chunk, scale, l2_eps,
                           norm_eps, dtype, y_dtype, stream);
+}
+
+
+size_t gdn_layer_fwd_varlen_workspace_bytes(int nseq, int max_seqlen, int total_T, int Hk, int Hv,
+                                            int dk, int dv, int chunk, gdn_dtype dtype) {
+  if (nseq <= 0 || max_seqlen <= 0 || total_T <= 0 || !valid_dtype(dtype) ||
+      validate_heads(Hk, Hv, dk, dv) != GDN_OK ||
+      !tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16))
+    return 0;
+  const size_t tok = (size_t)total_T;
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  // normalised q, k and convolved v (bf16), the recurrence's fp32 o, the hand-over buffer
+  return 2 * up(tok * Hk * dk * 2) + up(tok * Hv * dv * 2) + up(tok * Hv * dv * 4) +
+         up(tc_chunk_varlen_scratch_bytes(nseq, max_seqlen, Hv));
+}
+
+gdn_status gdn_layer_fwd_varlen(const void* q_raw, const void* k_raw, const void* v_raw,
+                                const void* z, const int* cu_seqlens, int nseq, int max_seqlen,
+                                const void* hq_in, const void* hk_in, const void* hv_in,
+                                const float* wq, const float* wk, const float* wv,
+                                const float* log_alpha, const float* beta, const float* S0,
+                                const float* norm_w, void* y, float* S_T, void* hq_out,
+                                void* hk_out, void* hv_out, void* workspace,
+                                size_t workspace_bytes, int total_T, int Hk, int Hv, int dk,
+                                int dv, int chunk, float scale, float l2_eps, float norm_eps,
+                                gdn_dtype dtype, gdn_dtype y_dtype, gdn_stream_t stream) {
+  if (nseq < 0 || max_seqlen < 0 || total_T < 0 || !valid_dtype(dtype) || !valid_dtype(y_dtype))
+    return GDN_ERR_INVALID_ARG;
+  if (!io_pair_ok(dtype, y_dtype)) return GDN_ERR_UNSUPPORTED;
+  gdn_status s = validate_heads(Hk, Hv, dk, dv);
+  if (s != GDN_OK) return s;
+  if (chunk <= 0 || !(norm_eps >= 0.f) || !(l2_eps >= 0.f)) return GDN_ERR_INVALID_ARG;
+  if (!tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16)) return GDN_ERR_UNSUPPORTED;
+  if (nseq > 65535 || 2L * Hk + Hv > 65535) return GDN_ERR_UNSUPPORTED;
+  if (nseq == 0) return GDN_OK;
+  const void* hs[] = {hq_in, hk_in, hv_in, hq_out, hk_out, hv_out};
+  for (const void* p : hs)
+    if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+  if ((hq_out && hq_out == hq_in) || (hk_out && hk_out == hk_in) ||
+      (hv_out && hv_out == hv_in))
+    return GDN_ERR_INVALID_ARG;
+  if (!cu_seqlens || !aligned4(cu_seqlens) || !opt_aligned16(S0) || !opt_aligned16(S_T))
+    return GDN_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (total_T == 0 || max_seqlen == 0) {   // every sequence is empty: state and history pass on
+    s = gdn_chunk_fwd_varlen(nullptr, nullptr, nullptr, nullptr, nullptr, cu_seqlens, nseq, 0, S0,
+                             nullptr, S_T, nullptr, 0, 0, Hk, Hv, dk, dv, chunk, scale, dtype,
+                             dtype, stream);
+    if (s != GDN_OK) return s;
+    return layer_hist_out(q_raw, k_raw, v_raw, hq_in, hk_in, hv_in, hq_out, hk_out, hv_out, nseq,
+                          0, Hk, Hv, dk, dv, dtype, st, cu_seqlens, 0);
+  }
+  const void* ptrs[] = {q_raw, k_raw, v_raw, z, y};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return GDN_ERR_INVALID_ARG;
+  if (!wq || !wk || !wv || !norm_w || !log_alpha || !beta || !aligned4(wq) || !aligned4(wk) ||
+      !aligned4(wv) || !aligned4(norm_w) || !aligned4(log_alpha) || !aligned4(beta))
+    return GDN_ERR_INVALID_ARG;
+  if (!tc_chunk_length_ok(max_seqlen) ||
+      (max_seqlen + kPrologueTokens - 1) / kPrologueTokens > 65535)
+    return GDN_ERR_UNSUPPORTED;
+  const size_t need = gdn_layer_fwd_varlen_workspace_bytes(nseq, max_seqlen, total_T, Hk, Hv, dk,
+                                                           dv, chunk, dtype);
+  if (!workspace_ok(workspace, workspace_bytes, need)) return GDN_ERR_INVALID_ARG;
+  const size_t tok = (size_t)total_T;
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  char* ws = static_cast<char*>(workspace);
+  void* qn = ws;
+  void* kn = ws + up(tok * Hk * dk * 2);
+  void* vc = ws + 2 * up(tok * Hk * dk * 2);
+  float* o = reinterpret_cast<float*>(ws + 2 * up(tok * Hk * dk * 2) + up(tok * Hv * dv * 2));
+  void* tc_scratch = reinterpret_cast<char*>(o) + up(tok * Hv * dv * 4);
+  s = prologue_launch(q_raw, k_raw, v_raw, hq_in, hk_in, hv_in, wq, wk, wv, qn, kn, vc, nseq,
+                      total_T, Hk, Hv, dk, dv, l2_eps, dtype, cu_seqlens, max_seqlen, st);
+  if (s != GDN_OK) return s;
+  s = tc_chunk_launch_varlen(qn, kn, vc, log_alpha, beta, cu_seqlens, nseq, max_seqlen, S0, o,
+                             S_T, total_T, Hk, Hv, scale, true, tc_scratch, st);
+  if (s != GDN_OK) return s;
+  const long long rows = (long long)tok * Hv;
+  const long long blocks = (rows + 7) / 8;
+  if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+  if (y_dtype == GDN_F32)
+    out_norm_kernel<float, __nv_bfloat16, float><<<(unsigned)blocks, 256, 0, st>>>(
+        o, (const __nv_bfloat16*)z, norm_w, (float*)y, rows, dv, norm_eps);
+  else
+    out_norm_kernel<float, __nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
+        o, (const __nv_bfloat16*)z, norm_w, (__nv_bfloat16*)y, rows, dv, norm_eps);
+  s = launch_status();
+  if (s != GDN_OK) return s;
+  return layer_hist_out(q_raw, k_raw, v_raw, hq_in, hk_in, hv_in, hq_out, hk_out, hv_out, nseq,
+                        total_T, Hk, Hv, dk, dv, dtype, st, cu_seqlens, max_seqlen);
 }
 
 }  // extern "C"

@@ -441,6 +441,41 @@ GDN_API gdn_status gdn_layer_fwd_ex(const void *q_raw, const void *k_raw, const 
                             float l2_eps, float norm_eps, gdn_dtype dtype, gdn_dtype y_dtype,
                             gdn_stream_t stream);
 
+/*
+ * The whole layer over packed requests of different lengths: the serving form of
+ * gdn_layer_fwd_ex, many requests in one call, each with its own state and conv history
+ * ("Chapitre 16 - Assembler un système de type Kimi K3", 16.1-16.2: the working state belongs
+ * to the request; a prompt in blocks with the state handed on).
+ *   q_raw, k_raw [total_T, Hk*dk]; v_raw, z [total_T, Hv*dv] (dtype); y [total_T, Hv, dv]
+ *        (y_dtype); log_alpha, beta [total_T, Hv] float
+ *   cu_seqlens [nseq + 1] int32 in device memory, max_seqlen: as gdn_chunk_fwd_varlen (request s
+ *        is tokens cu[s] .. cu[s+1] - 1; empty requests allowed; offsets clamped); the conv of a
+ *        request never reads another request's tokens.
+ *   hq_in, hk_in [nseq, 3, Hk*dk]; hv_in [nseq, 3, Hv*dv] (dtype) or NULL (fresh requests);
+ *        hq_out, hk_out, hv_out: same shapes or NULL, as gdn_layer_fwd_ex, per request
+ *   S0, S_T [nseq, Hv, dk, dv] float, each may be NULL (zero states / not written)
+ *   workspace: gdn_layer_fwd_varlen_workspace_bytes(...) bytes, 256-byte aligned.
+ * y of tokens outside every request is unspecified.  Supported: bf16 inputs, dk = dv = 128,
+ * chunk 64 (y bf16 or fp32); other sizes return GDN_ERR_UNSUPPORTED.  Each request gets the
+ * results of gdn_layer_fwd_ex on it alone.
+ */
+GDN_API gdn_status gdn_layer_fwd_varlen(const void *q_raw, const void *k_raw, const void *v_raw,
+                                const void *z, const int *cu_seqlens, int nseq, int max_seqlen,
+                                const void *hq_in, const void *hk_in, const void *hv_in,
+                                const float *wq, const float *wk, const float *wv,
+                                const float *log_alpha, const float *beta, const float *S0,
+                                const float *norm_w, void *y, float *S_T, void *hq_out,
+                                void *hk_out, void *hv_out, void *workspace,
+                                size_t workspace_bytes, int total_T, int Hk, int Hv, int dk,
+                                int dv, int chunk, float scale, float l2_eps, float norm_eps,
+                                gdn_dtype dtype, gdn_dtype y_dtype, gdn_stream_t stream);
+
+/* Device scratch bytes gdn_layer_fwd_varlen needs (host only, no CUDA call); 0 for sizes it does
+ * not support. */
+GDN_API size_t gdn_layer_fwd_varlen_workspace_bytes(int nseq, int max_seqlen, int total_T,
+                                            int Hk, int Hv, int dk, int dv, int chunk,
+                                            gdn_dtype dtype);
+
 /* Scratch bytes gdn_layer_fwd needs for these sizes (host only, no CUDA call); 0 if none. */
 GDN_API size_t gdn_layer_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv, int chunk,
                                  gdn_dtype dtype);

@@ -314,3 +314,23 @@ def test_prologue_ex_and_layer_ex_validation(L):
     # a history out that is the history in
     h = P(0x2000)
     assert L.gdn_layer_fwd_ex(*head, None, None, h, *mid, None, None, h, *ws, *sizes) == 1
+
+
+def test_layer_varlen_validation(L):
+    """gdn_layer_fwd_varlen rejects unsupported sizes (2) and a missing or short workspace or
+    offsets (1) before any work; no requests is a no-op."""
+    pre = [FAKE] * 4
+    mid = [FAKE] * 3 + [None] * 3                     # conv taps; no history
+    tail = [FAKE] * 6 + [None] * 3                    # gates, S0, norm gain, y, S_T; no history out
+    sizes = [700, 2, 16, 128, 128, 64, 1.0, 1e-6, 1e-5, 1, 1, None]
+    assert L.gdn_layer_fwd_varlen(*pre, FAKE, 0, 300, *mid[3:], *mid[:3], *tail, None, 0,
+                                  *sizes) == 0        # nseq = 0
+    assert L.gdn_layer_fwd_varlen(*pre, None, 4, 300, *mid[3:], *mid[:3], *tail, P(0x100000),
+                                  1 << 40, *sizes) == 1   # no offsets
+    assert L.gdn_layer_fwd_varlen(*pre, FAKE, 4, 300, *mid[3:], *mid[:3], *tail, None, 0,
+                                  *sizes) == 1        # no workspace
+    assert L.gdn_layer_fwd_varlen(*pre, FAKE, 4, 300, *mid[3:], *mid[:3], *tail, P(0x100000),
+                                  1 << 40, 700, 2, 16, 64, 64, 64, 1.0, 1e-6, 1e-5, 1, 1,
+                                  None) == 2          # d = 64: not the tensor-core shape
+    assert L.gdn_layer_fwd_varlen_workspace_bytes(4, 300, 700, 2, 16, 128, 128, 64, 1) > 0
+    assert L.gdn_layer_fwd_varlen_workspace_bytes(4, 300, 700, 2, 16, 64, 64, 64, 1) == 0
