@@ -397,6 +397,44 @@ def bench_varlen(gdn, dev, warmup, flush, peaks, steps=10):
             f"Hk{w.Hk} Hv{w.Hv} dk{w.dk} dv{w.dv} chunk{w.chunk} {w.dtype} S0~N(0,0.02)"}
 
 
+def bench_layer_varlen(gdn, dev, warmup, flush, peaks, steps=10):
+    """The whole layer over 32 packed requests of seeded lengths U[64, 1024] with the 8:1 heads
+    (Hk16 Hv128 d128, bf16), each continuing from a nonzero state and a carried conv history:
+    the serving form of the layer (gdn_layer_fwd_varlen)."""
+    w = gi.WORKLOADS["layer_8to1"]
+    g = torch.Generator().manual_seed(12)
+    lengths = torch.randint(64, 1025, (32,), generator=g)
+    total, n, mx = int(lengths.sum()), 32, int(lengths.max())
+    cq, cv = w.Hk * w.dk, w.Hv * w.dv
+    bf = lambda *shape: torch.randn(*shape, generator=g).to(w.torch_dtype).to(dev)
+    qr, kr, vr, z = bf(total, cq), bf(total, cq), bf(total, cv), bf(total, cv)
+    hist = (bf(n, 3, cq), bf(n, 3, cq), bf(n, 3, cv))
+    wq, wk = [(torch.randn(cq, 4, generator=g) * w.conv_w_std).to(dev) for _ in range(2)]
+    wv = (torch.randn(cv, 4, generator=g) * w.conv_w_std).to(dev)
+    la = (-torch.nn.functional.softplus(torch.randn(total, w.Hv, generator=g))
+          * torch.exp(torch.rand(total, w.Hv, generator=g) * 4.0 - 5.0)).to(dev)
+    be = torch.sigmoid(torch.randn(total, w.Hv, generator=g)).to(dev)
+    S0 = (torch.randn(n, w.Hv, w.dk, w.dv, generator=g) * 0.02).to(dev)
+    nw = torch.ones(w.dv, device=dev)
+    cu = torch.cat([torch.zeros(1, dtype=torch.int64), lengths.cumsum(0)]).to(torch.int32).to(dev)
+
+    def step():
+        gdn.layer_fwd_varlen(qr, kr, vr, z, cu, mx, wq, wk, wv, la, be, S0, nw, Hk=w.Hk, Hv=w.Hv,
+                             dk=w.dk, dv=w.dv, chunk=w.chunk, hist=hist, want_hist=True)
+    ms = time_steps(step, steps, warmup, flush, 3)
+    gdn.check_error(dev)
+    t = sum(ms) / len(ms) / 1e3
+    # raw q, k, v, z in and y out (bf16), gates, states in and out, histories in and out
+    B = (total * (2 * cq * 2 + 2 * cv * 2 + cv * 2 + 8 * w.Hv) + n * w.Hv * w.dk * w.dv * 8 +
+         2 * n * 3 * (2 * cq + cv) * 2)
+    roof = roofline_block(B, fwd_flops(w.with_sizes(B=1, T=total)), t, peaks,
+                          "gdn_layer_fwd_varlen")
+    return {"value": total / t, "unit": "tokens/s", "ms_per_call": t * 1e3, "tokens": total,
+            "requests": n, "roofline_frac": roof["frac"], "roofline": roof,
+            "workload": f"layer_varlen 32 requests U[64,1024] ({total} tokens) Hk{w.Hk} Hv{w.Hv} "
+                        f"dk{w.dk} dv{w.dv} chunk{w.chunk} {w.dtype}, S0 and conv history carried"}
+
+
 def bench_gates(gdn, dev, warmup, flush, peaks, steps=20):
     """Gates from the in_proj_ba outputs on the prefill shape (B4 T2048, 48 value heads, bf16)."""
     w = gi.WORKLOADS["prefill"]
@@ -837,6 +875,7 @@ def main():
             sec["decode_layer"] = bench_decode_layer(gdn, dev, args.warmup, flush, peaks)
             sec["gates"] = bench_gates(gdn, dev, args.warmup, flush, peaks)
             sec["varlen"] = bench_varlen(gdn, dev, args.warmup, flush, peaks)
+            sec["layer_varlen"] = bench_layer_varlen(gdn, dev, args.warmup, flush, peaks)
             del d
             torch.cuda.empty_cache()
             _, xl, dl, _, sec["long_context"] = bench_prefill_like(
