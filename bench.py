@@ -4,8 +4,9 @@
 Headline: the chunked forward (gdn_chunk_fwd) on the prefill workload — B=4, T=2048, 16 key heads
 shared by 48 value heads, d_k = d_v = 128, chunk 64, bf16 q/k/v, fp32 gates and state, S0 = 0 —
 in tokens/s, with its fraction of the HBM/tensor roofline.  Secondary lines in the same JSON
-object: the decode step (256 sequences, GB/s of state traffic against the HBM peak), the long
-context forward (B1 T65536) and the fused 8:1 layer (B2 T8192 Hv128).
+object: the decode step (256 sequences, GB/s of state traffic against the HBM peak), the full-layer
+decode step, the gates, the packed prefill of 32 requests, the packed 8:1 layer, the long context
+forward (B1 T65536), the 8:1 layer (B2 T8192 Hv128), the backward pass and the layer backward.
 
 Every step runs with its inputs resident in HBM; an L2 flush (a 256 MiB write, outside the timed
 events) separates timed steps.  Device time comes from CUDA events on the launching stream.  Under
