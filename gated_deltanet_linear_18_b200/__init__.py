@@ -102,6 +102,10 @@ def lib() -> ctypes.CDLL:
         L.gdn_bwd.argtypes = [P] * 15 + [SZ] + [I] * 6 + [F, I, P]
         L.gdn_bwd.restype = I
         L.gdn_bwd_workspace_bytes.argtypes = [I] * 6
+        L.gdn_bwd_varlen.argtypes = [P] * 6 + [I, I] + [P] * 10 + [SZ] + [I] * 5 + [F, I, P]
+        L.gdn_bwd_varlen.restype = I
+        L.gdn_bwd_varlen_workspace_bytes.argtypes = [I] * 7
+        L.gdn_bwd_varlen_workspace_bytes.restype = SZ
         L.gdn_bwd_workspace_bytes.restype = SZ
         L.gdn_bwd_launches.argtypes = [I] * 6
         L.gdn_bwd_launches.restype = I
@@ -263,6 +267,35 @@ def bwd(q, k, v, log_alpha, beta, S0, dO, dS_T=None, *, scale: float = 1.0,
                            wbytes, B, T, Hk, Hv, dk, dv, float(scale), _io_dtype(q),
                            _stream(dev))
     _check("gdn_bwd", st)
+    return out
+
+
+def bwd_varlen(q, k, v, log_alpha, beta, cu_seqlens, max_seqlen: int, S0, dO, dS_T=None, *,
+               scale: float = 1.0) -> dict:
+    """gdn_bwd over packed sequences (gdn_bwd_varlen): q, k [total, Hk, dk]; v, dO [total, Hv,
+    dv]; gates [total, Hv]; cu_seqlens [nseq+1] int32 (device); S0, dS_T [nseq, Hv, dk, dv] or
+    None.  Returns fp32 dq, dk [total, Hk, dk], dv [total, Hv, dv], dlog_alpha, dbeta [total, Hv],
+    dS0 [nseq, Hv, dk, dv]."""
+    total, Hk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    nseq = cu_seqlens.numel() - 1
+    if cu_seqlens.dtype != torch.int32:
+        raise ValueError("cu_seqlens must be int32")
+    _f32(log_alpha, beta, S0, dS_T)
+    f = dict(device=q.device, dtype=torch.float32)
+    out = {"dq": torch.empty(total, Hk, dk, **f), "dk": torch.empty(total, Hk, dk, **f),
+           "dv": torch.empty(total, Hv, dv, **f), "dlog_alpha": torch.empty(total, Hv, **f),
+           "dbeta": torch.empty(total, Hv, **f), "dS0": torch.empty(nseq, Hv, dk, dv, **f)}
+    dev = _dev(q, k, v, log_alpha, beta, cu_seqlens, S0, dO, dS_T)
+    need = int(lib().gdn_bwd_varlen_workspace_bytes(nseq, int(max_seqlen), total, Hk, Hv, dk, dv))
+    ws = torch.empty(max(need, 1), device=dev, dtype=torch.uint8)
+    with torch.cuda.device(dev):
+        st = lib().gdn_bwd_varlen(_p(q), _p(k), _p(v), _p(log_alpha), _p(beta), _p(cu_seqlens),
+                                  nseq, int(max_seqlen), _p(S0), _p(dO), _p(dS_T), _p(out["dq"]),
+                                  _p(out["dk"]), _p(out["dv"]), _p(out["dlog_alpha"]),
+                                  _p(out["dbeta"]), _p(out["dS0"]), _p(ws), need, total, Hk, Hv,
+                                  dk, dv, float(scale), _io_dtype(q), _stream(dev))
+    _check("gdn_bwd_varlen", st)
     return out
 
 

@@ -120,24 +120,24 @@ __device__ __forceinline__ void load_segment(Smem<D>& sm, const Tin* __restrict_
                                              const Tin* __restrict__ k, const Tin* __restrict__ v,
                                              const Tdo* __restrict__ dO,
                                              const float* __restrict__ la,
-                                             const float* __restrict__ be, long b, int h, int hk,
-                                             int c0, int T, int Hk, int Hv, int t0, int len,
+                                             const float* __restrict__ be, long r0, int h,
+                                             int hk, int c0, int Hk, int Hv, int t0, int len,
                                              bool with_q) {
   constexpr int NT = Shape<D>::NT, DC = Shape<D>::DC;
   for (int e = threadIdx.x; e < len * D; e += NT) {
     const int j = e / D, i = e - j * D;
-    const long rk = ((b * T + t0 + j) * Hk + hk) * (long)D + i;
+    const long rk = ((r0 + t0 + j) * Hk + hk) * (long)D + i;
     sm.k[j][i] = to_f(k[rk]);
     if (with_q) sm.q[j][i] = to_f(q[rk]);
   }
   for (int e = threadIdx.x; e < len * DC; e += NT) {      // this CTA's columns c0 .. c0 + DC - 1
     const int j = e / DC, i = e - j * DC;
-    const long rv = ((b * T + t0 + j) * Hv + h) * (long)D + c0 + i;
+    const long rv = ((r0 + t0 + j) * Hv + h) * (long)D + c0 + i;
     sm.v[j][i] = to_f(v[rv]);
     if (with_q) sm.dO[j][i] = to_f(dO[rv]);
   }
   for (int j = threadIdx.x; j < len; j += NT) {
-    const long g = (b * T + t0 + j) * Hv + h;
+    const long g = (r0 + t0 + j) * Hv + h;
     sm.alpha[j] = expf(la[g]);
     sm.beta[j] = be[g];
   }
@@ -153,10 +153,13 @@ struct Tile {
 };
 
 // grid: B * Hv * NS CTAs ((b * Hv + h) * NS + column slice); block Shape<D>::NT; dynamic shared
-// memory smem_bytes<D>().  direct (one value head per key head and one slice per head): dq_out,
-// dk_out are [B, T, Hk, D] and dla_out, dbeta_out [B, T, Hv]; otherwise they are the per-slice
-// partials [B, T, Hv * NS, D] and [B, T, Hv, NS], summed afterwards by group_sum_kernel.  ckpt:
-// B * Hv * NS * ceil(T / kSeg) slices of D * DC floats, each in the CTA's own per-thread order.
+// memory smem_bytes<D>().  Sequences as in row_span: b of [B, T, ...] tensors (cu == nullptr,
+// max_len = T), or packed rows cu[b] .. cu[b + 1] - 1 of T in all (none longer than max_len);
+// token rows below are rows of those tensors.  direct (one value head per key head and one slice
+// per head): dq_out, dk_out are [rows, Hk, D] and dla_out, dbeta_out [rows, Hv]; otherwise they are
+// the per-slice partials [rows, Hv * NS, D] and [rows, Hv, NS], summed afterwards by
+// group_sum_kernel.  ckpt: B * Hv * NS * ceil(max_len / kSeg) slices of D * DC floats, each in the
+// CTA's own per-thread order.
 template <int D, typename Tin, typename Tdo = Tin>
 __global__ void __launch_bounds__(Shape<D>::NT, Shape<D>::MINB)
 bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
@@ -165,7 +168,8 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
            const float* __restrict__ dS_T, float* __restrict__ dq_out,
            float* __restrict__ dk_out, int direct, float* __restrict__ dv_out,
            float* __restrict__ dla_out, float* __restrict__ dbeta_out, float* __restrict__ dS0,
-           float* __restrict__ ckpt, int T, int Hk, int Hv, float scale) {
+           float* __restrict__ ckpt, int T, int Hk, int Hv, float scale,
+           const int* __restrict__ cu, int max_len) {
   using Sh = Shape<D>;
   constexpr int RL = Sh::RL, CW = Sh::CW, CP = CW / 2, LR = Sh::LR, NT = Sh::NT, SL = Sh::SL;
   constexpr int NS = Sh::NS, DC = Sh::DC, PPT = RL * CP;   // column pairs per thread
@@ -181,8 +185,11 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
   const int hk = h / (Hv / Hk);
   const int nqk = direct ? Hk : Hv * NS, hq = direct ? hk : h * NS + ns;   // dq, dk slot
   const int nab = direct ? 1 : NS, hab = direct ? 0 : ns;                 // dla, dbeta slot
-  const int nseg = (T + kSeg - 1) / kSeg;
-  float* const ck = ckpt + (long)blockIdx.x * nseg * D * DC;
+  const RowSpan span = row_span(cu, (int)b, T, max_len);   // this sequence's rows
+  const long r0 = span.row0;
+  const int Ts = span.len;
+  const int nseg = (Ts + kSeg - 1) / kSeg;
+  float* const ck = ckpt + (long)blockIdx.x * ((max_len + kSeg - 1) / kSeg) * D * DC;
   const long sbase = bh * (long)D * D;               // [dk][dv] slot of S0, dS_T, dS0
 
   // a state in the [dk][dv] order of S0 / dS_T / dS0 (8-byte pairs: j0 and CW are even), and in
@@ -248,9 +255,9 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
   if (S0) get_sq(S0 + sbase, M);
   else zero(M);
   for (int sg = 0; sg < nseg; ++sg) {
-    const int t0 = sg * kSeg, len = min(kSeg, T - t0);
+    const int t0 = sg * kSeg, len = min(kSeg, Ts - t0);
     __syncthreads();                                 // the previous segment's data is read
-    load_segment(sm, q, k, v, dO, log_alpha, beta, b, h, hk, c0, T, Hk, Hv, t0, len, false);
+    load_segment(sm, q, k, v, dO, log_alpha, beta, r0, h, hk, c0, Hk, Hv, t0, len, false);
     put_pt(ck + (long)sg * D * DC, M);
     __syncthreads();
     for (int j = 0; j < len; ++j) fwd_step(M, j);
@@ -272,12 +279,12 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
 #pragma unroll 4
         for (int s2 = 0; s2 < SL; ++s2) acc += f < D ? sm.pdq[hj][s2][i] : sm.pdk[hj][s2][i];
         float* dst = f < D ? dq_out : dk_out;
-        dst[((b * T + t) * nqk + hq) * (long)D + i] = acc;
+        dst[((r0 + t) * nqk + hq) * (long)D + i] = acc;
       } else {
         const bool isa = f == 2 * D;
 #pragma unroll 4
         for (int s2 = 0; s2 < SL; ++s2) acc += isa ? sm.pa[hj][s2] : sm.pb[hj][s2];
-        const long g = ((b * T + t) * Hv + h) * nab + hab;
+        const long g = ((r0 + t) * Hv + h) * nab + hab;
         if (isa) dla_out[g] = sm.alpha[j] * acc;       // alpha <G, P - beta x k^T>
         else dbeta_out[g] = acc;                       // (v - alpha x)^T Gk
       }
@@ -285,9 +292,9 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
     __syncthreads();
   };
   for (int sg = nseg - 1; sg >= 0; --sg) {
-    const int t0 = sg * kSeg, len = min(kSeg, T - t0);
+    const int t0 = sg * kSeg, len = min(kSeg, Ts - t0);
     __syncthreads();
-    load_segment(sm, q, k, v, dO, log_alpha, beta, b, h, hk, c0, T, Hk, Hv, t0, len, true);
+    load_segment(sm, q, k, v, dO, log_alpha, beta, r0, h, hk, c0, Hk, Hv, t0, len, true);
     get_pt(ck + (long)sg * D * DC, M);               // this thread's own elements
     put_pt(sm.state0, M);
     __syncthreads();
@@ -363,7 +370,7 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
         sm.pb[hj][sl] = ug;
 #pragma unroll
         for (int c = 0; c < CW; ++c)
-          dv_out[((b * T + t0 + j) * Hv + h) * (long)D + j0 + c] = be * gk[c];
+          dv_out[((r0 + t0 + j) * Hv + h) * (long)D + j0 + c] = be * gk[c];
       }
       // the gradient reaching S_{t-1}: alpha G + dx k^T
 #pragma unroll

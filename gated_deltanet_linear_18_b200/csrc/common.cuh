@@ -68,4 +68,19 @@ __device__ __forceinline__ float hsum2(f2_t r) {
   return a + b;
 }
 
+// Rows of sequence s: of [B, T, ...] tensors (cu == nullptr), rows s T .. s T + T - 1; packed
+// (cu != nullptr), rows cu[s] .. cu[s + 1] - 1 of [T, ...] tensors (T = total rows), clamped to
+// the tensor and cut at max_len, so that malformed offsets cannot reach outside it.
+struct RowSpan {
+  long row0;
+  int len;
+};
+__device__ __forceinline__ RowSpan row_span(const int* __restrict__ cu, int s, int T,
+                                            int max_len) {
+  if (!cu) return RowSpan{(long)s * T, T};
+  const int a = min(max(cu[s], 0), T);
+  const int b = min(max(cu[s + 1], a), min(T, a + max_len));
+  return RowSpan{(long)a, b - a};
+}
+
 }  // namespace gdn

@@ -88,21 +88,6 @@ __device__ __forceinline__ float rcp_fast(float x) {
 
 constexpr int kPrologueList = 1024;     // undecided values one CTA redoes in fp64 afterwards
 
-// Rows of sequence s: of [B, T, ...] tensors (cu == nullptr), rows s T .. s T + T - 1; packed
-// (cu != nullptr), rows cu[s] .. cu[s + 1] - 1 of [T, ...] tensors (T = total rows), clamped to
-// the tensor and cut at max_len, so that malformed offsets cannot reach outside it.
-struct RowSpan {
-  long row0;
-  int len;
-};
-__device__ __forceinline__ RowSpan row_span(const int* __restrict__ cu, int s, int T,
-                                            int max_len) {
-  if (!cu) return RowSpan{(long)s * T, T};
-  const int a = min(max(cu[s], 0), T);
-  const int b = min(max(cu[s + 1], a), min(T, a + max_len));
-  return RowSpan{(long)a, b - a};
-}
-
 // The staged tile of one prologue CTA: the raw rows of tokens t0 - 3 .. t0 + kPrologueTokens - 1
 // of one head of d channels, row r holding token t0 - 3 + r, brought in by 16-byte asynchronous
 // copies that are all issued at once (many tiles in flight per SM).  Tokens -3 .. -1 come from the

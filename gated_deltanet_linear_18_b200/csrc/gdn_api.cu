@@ -220,14 +220,16 @@ size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
 struct BwdLayout {
   size_t dqh = 0, dkh = 0, dah = 0, dbh = 0, total = 0;   // section offsets; total bytes
 };
-BwdLayout bwd_layout(int B, int T, int Hk, int Hv, int dk, int dv) {
+// nseq sequences of at most max_len tokens, `rows` token rows in all: checkpoints per (sequence,
+// head) for max_len tokens, per-token partials for every row.
+BwdLayout bwd_layout_rows(int nseq, int max_len, size_t rows, int Hk, int Hv, int dk, int dv) {
   BwdLayout L;
   const size_t ns = (size_t)bwd::head_slices(dk);
-  const size_t nseg = ((size_t)T + bwd::kSeg - 1) / bwd::kSeg;
-  const size_t ck = align256((size_t)B * Hv * nseg * dk * dv * sizeof(float));
+  const size_t nseg = ((size_t)max_len + bwd::kSeg - 1) / bwd::kSeg;
+  const size_t ck = align256((size_t)nseq * Hv * nseg * dk * dv * sizeof(float));
   const bool direct = Hv == Hk && ns == 1;
-  const size_t per = direct ? 0 : align256((size_t)B * T * Hv * ns * dk * sizeof(float));
-  const size_t gate = ns > 1 ? align256((size_t)B * T * Hv * ns * sizeof(float)) : 0;
+  const size_t per = direct ? 0 : align256(rows * Hv * ns * dk * sizeof(float));
+  const size_t gate = ns > 1 ? align256(rows * Hv * ns * sizeof(float)) : 0;
   L.dqh = ck;
   L.dkh = ck + per;
   L.dah = ck + 2 * per;
@@ -235,19 +237,26 @@ BwdLayout bwd_layout(int B, int T, int Hk, int Hv, int dk, int dv) {
   L.total = ck + 2 * per + 2 * gate;
   return L;
 }
+BwdLayout bwd_layout(int B, int T, int Hk, int Hv, int dk, int dv) {
+  return bwd_layout_rows(B, T, (size_t)B * T, Hk, Hv, dk, dv);
+}
 
 template <int D, typename Tin, typename Tdo = Tin>
 gdn_status bwd_launch(const void* q, const void* k, const void* v, const float* la,
                       const float* be, const float* S0, const void* dO, const float* dST,
                       float* dq, float* dk, float* dv, float* dla, float* dbeta, float* dS0,
-                      void* ws, int B, int T, int Hk, int Hv, float scale, cudaStream_t st) {
+                      void* ws, int B, int T, int Hk, int Hv, float scale, cudaStream_t st,
+                      const int* cu = nullptr, int max_len = -1) {
+  // B sequences: [B, T] rows, or (cu) packed rows of T in all, none longer than max_len
+  if (!cu) max_len = T;
+  const long rows = cu ? (long)T : (long)B * T;
   constexpr int NS = bwd::Shape<D>::NS;
   auto kern = bwd::bwd_kernel<D, Tin, Tdo>;
   const size_t smem = bwd::smem_bytes<D>();
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return GDN_ERR_CUDA;
-  const BwdLayout L = bwd_layout(B, T, Hk, Hv, D, D);
+  const BwdLayout L = bwd_layout_rows(B, max_len, (size_t)rows, Hk, Hv, D, D);
   uint8_t* w = static_cast<uint8_t*>(ws);
   const bool direct = Hv == Hk && NS == 1;
   float* dqo = direct ? dq : reinterpret_cast<float*>(w + L.dqh);
@@ -259,7 +268,7 @@ gdn_status bwd_launch(const void* q, const void* k, const void* v, const float* 
   kern<<<(unsigned)ctas, bwd::Shape<D>::NT, smem, st>>>(
       static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v), la, be,
       S0, static_cast<const Tdo*>(dO), dST, dqo, dko, direct ? 1 : 0, dv, dao, dbo, dS0,
-      reinterpret_cast<float*>(w), T, Hk, Hv, scale);
+      reinterpret_cast<float*>(w), T, Hk, Hv, scale, cu, max_len);
   if (cudaGetLastError() != cudaSuccess) return GDN_ERR_CUDA;
   auto sum = [&](const float* a_src, float* a_dst, const float* b_src, float* b_dst, long rows,
                  int G, int Dd) {
@@ -267,8 +276,8 @@ gdn_status bwd_launch(const void* q, const void* k, const void* v, const float* 
     const unsigned blocks = (unsigned)std::min<long>((n + 255) / 256, 148L * 16);
     if (blocks > 0) bwd::group_sum_kernel<<<blocks, 256, 0, st>>>(a_src, a_dst, b_src, b_dst, rows, G, Dd);
   };
-  if (!direct && T > 0) sum(dqo, dq, dko, dk, (long)B * T * Hk, (Hv / Hk) * NS, D);
-  if (NS > 1 && T > 0) sum(dao, dla, dbo, dbeta, (long)B * T * Hv, NS, 1);
+  if (!direct && rows > 0) sum(dqo, dq, dko, dk, rows * Hk, (Hv / Hk) * NS, D);
+  if (NS > 1 && rows > 0) sum(dao, dla, dbo, dbeta, rows * Hv, NS, 1);
   return launch_status();
 }
 
@@ -276,11 +285,12 @@ template <typename Tin, typename Tdo = Tin>
 gdn_status bwd_dispatch(int d, const void* q, const void* k, const void* v, const float* la,
                         const float* be, const float* S0, const void* dO, const float* dST,
                         float* dq, float* dk, float* dv, float* dla, float* dbeta, float* dS0,
-                        void* ws, int B, int T, int Hk, int Hv, float scale, cudaStream_t st) {
+                        void* ws, int B, int T, int Hk, int Hv, float scale, cudaStream_t st,
+                        const int* cu = nullptr, int max_len = -1) {
 #define GDN_BWD(D)                                                                              \
   case D:                                                                                       \
     return bwd_launch<D, Tin, Tdo>(q, k, v, la, be, S0, dO, dST, dq, dk, dv, dla, dbeta, dS0, ws, \
-                                   B, T, Hk, Hv, scale, st);
+                                   B, T, Hk, Hv, scale, st, cu, max_len);
   switch (d) {
     GDN_BWD(16)
     GDN_BWD(32)
@@ -337,6 +347,50 @@ gdn_status gdn_bwd(const void* q, const void* k, const void* v, const float* log
                                dlog_alpha, dbeta, dS0, workspace, B, T, Hk, Hv, scale, st);
   return bwd_dispatch<__nv_bfloat16>(dk_, q, k, v, log_alpha, beta, S0, dO, dS_T, dq, dk, dv,
                                      dlog_alpha, dbeta, dS0, workspace, B, T, Hk, Hv, scale, st);
+}
+
+size_t gdn_bwd_varlen_workspace_bytes(int nseq, int max_seqlen, int total_T, int Hk, int Hv,
+                                      int dk, int dv) {
+  if (nseq <= 0 || max_seqlen < 0 || total_T < 0 || validate_heads(Hk, Hv, dk, dv) != GDN_OK ||
+      dk != dv)
+    return 0;
+  return bwd_layout_rows(nseq, max_seqlen, (size_t)total_T, Hk, Hv, dk, dv).total;
+}
+
+gdn_status gdn_bwd_varlen(const void* q, const void* k, const void* v, const float* log_alpha,
+                          const float* beta, const int* cu_seqlens, int nseq, int max_seqlen,
+                          const float* S0, const void* dO, const float* dS_T, float* dq,
+                          float* dk, float* dv, float* dlog_alpha, float* dbeta, float* dS0,
+                          void* workspace, size_t workspace_bytes, int total_T, int Hk, int Hv,
+                          int dk_, int dv_, float scale, gdn_dtype dtype, gdn_stream_t stream) {
+  if (nseq < 0 || max_seqlen < 0 || total_T < 0 || !valid_dtype(dtype)) return GDN_ERR_INVALID_ARG;
+  gdn_status s = validate_heads(Hk, Hv, dk_, dv_);
+  if (s != GDN_OK) return s;
+  if (dk_ != dv_) return GDN_ERR_UNSUPPORTED;
+  if ((long)nseq * Hv * bwd::head_slices(dk_) > 0x7fffffffL) return GDN_ERR_UNSUPPORTED;
+  if (nseq == 0) return GDN_OK;
+  if (!cu_seqlens || !aligned4(cu_seqlens)) return GDN_ERR_INVALID_ARG;
+  const bool work = total_T > 0 && max_seqlen > 0;
+  if (work && (!q || !k || !v || !log_alpha || !beta || !dO || !dq || !dk || !dv ||
+               !dlog_alpha || !dbeta))
+    return GDN_ERR_INVALID_ARG;
+  if (!opt_aligned4(q) || !opt_aligned4(k) || !opt_aligned4(v) || !opt_aligned4(dO) ||
+      !opt_aligned4(log_alpha) || !opt_aligned4(beta) || !opt_aligned4(dq) ||
+      !opt_aligned4(dk) || !opt_aligned4(dlog_alpha) || !opt_aligned4(dbeta) ||
+      !opt_aligned16(dv) || !opt_aligned16(S0) || !opt_aligned16(dS_T) || !opt_aligned16(dS0))
+    return GDN_ERR_INVALID_ARG;
+  const int ml = work ? max_seqlen : 0;
+  if (!workspace_ok(workspace, workspace_bytes,
+                    bwd_layout_rows(nseq, ml, (size_t)total_T, Hk, Hv, dk_, dv_).total))
+    return GDN_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == GDN_F32)
+    return bwd_dispatch<float>(dk_, q, k, v, log_alpha, beta, S0, dO, dS_T, dq, dk, dv,
+                               dlog_alpha, dbeta, dS0, workspace, nseq, total_T, Hk, Hv, scale,
+                               st, cu_seqlens, ml);
+  return bwd_dispatch<__nv_bfloat16>(dk_, q, k, v, log_alpha, beta, S0, dO, dS_T, dq, dk, dv,
+                                     dlog_alpha, dbeta, dS0, workspace, nseq, total_T, Hk, Hv,
+                                     scale, st, cu_seqlens, ml);
 }
 
 const char* gdn_status_string(gdn_status s) {

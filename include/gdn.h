@@ -283,6 +283,31 @@ GDN_API gdn_status gdn_bwd(const void *q, const void *k, const void *v, const fl
                    void *workspace, size_t workspace_bytes, int B, int T, int Hk, int Hv,
                    int dk_, int dv_, float scale, gdn_dtype dtype, gdn_stream_t stream);
 
+/*
+ * gdn_bwd over packed sequences of different lengths: the training form of gdn_chunk_fwd_varlen,
+ * each sequence with its own S0 and its own gradients ("Chapitre 16 - Assembler un système de type
+ * Kimi K3", 16.1: the working state belongs to the request; the recurrence differentiated as in
+ * gdn_bwd).
+ *   q, k [total_T, Hk, dk]; v, dO [total_T, Hv, dv]; log_alpha, beta [total_T, Hv]
+ *   cu_seqlens [nseq + 1] int32 (device), max_seqlen: as gdn_chunk_fwd_varlen
+ *   S0, dS_T, dS0 [nseq, Hv, dk, dv] (each may be NULL as in gdn_bwd)
+ *   dq, dk [total_T, Hk, dk]; dv [total_T, Hv, dv]; dlog_alpha, dbeta [total_T, Hv]
+ *   workspace: gdn_bwd_varlen_workspace_bytes(...) bytes, 256-byte aligned.
+ * Gradients of tokens outside every sequence are unspecified.  Sizes, dtypes and the
+ * reproducibility of the sums as gdn_bwd; each sequence gets the gradients of gdn_bwd on it alone.
+ */
+GDN_API gdn_status gdn_bwd_varlen(const void *q, const void *k, const void *v,
+                          const float *log_alpha, const float *beta, const int *cu_seqlens,
+                          int nseq, int max_seqlen, const float *S0, const void *dO,
+                          const float *dS_T, float *dq, float *dk, float *dv, float *dlog_alpha,
+                          float *dbeta, float *dS0, void *workspace, size_t workspace_bytes,
+                          int total_T, int Hk, int Hv, int dk_, int dv_, float scale,
+                          gdn_dtype dtype, gdn_stream_t stream);
+
+/* Device scratch bytes gdn_bwd_varlen needs (host only, no CUDA call); 0 for invalid sizes. */
+GDN_API size_t gdn_bwd_varlen_workspace_bytes(int nseq, int max_seqlen, int total_T, int Hk,
+                                      int Hv, int dk, int dv);
+
 /* Kernels one gdn_bwd call with these sizes launches (host only, no CUDA call): the backward
  * kernel, plus the sums of the partial dq, dk and of dlog_alpha, dbeta where the call has them;
  * -1 for sizes the call rejects. */

@@ -334,3 +334,19 @@ def test_layer_varlen_validation(L):
                                   None) == 2          # d = 64: not the tensor-core shape
     assert L.gdn_layer_fwd_varlen_workspace_bytes(4, 300, 700, 2, 16, 128, 128, 64, 1) > 0
     assert L.gdn_layer_fwd_varlen_workspace_bytes(4, 300, 700, 2, 16, 64, 64, 64, 1) == 0
+
+
+def test_bwd_varlen_validation(L):
+    """gdn_bwd_varlen: missing offsets or workspace (1), unequal head sizes (2), no sequences is a
+    no-op; the workspace query follows the call."""
+    ten = [FAKE] * 5
+    outs = [FAKE] * 9
+    ws = [P(0x100000), 1 << 40]
+    tail = [300, 2, 6, 64, 64, 1.0, 1, None]
+    assert L.gdn_bwd_varlen(*ten, FAKE, 0, 100, *outs, None, 0, *tail) == 0          # nseq = 0
+    assert L.gdn_bwd_varlen(*ten, None, 3, 100, *outs, *ws, *tail) == 1              # no offsets
+    assert L.gdn_bwd_varlen(*ten, FAKE, 3, 100, *outs, None, 0, *tail) == 1          # no workspace
+    assert L.gdn_bwd_varlen(*ten, FAKE, 3, 100, *outs, *ws, 300, 2, 6, 64, 32, 1.0, 1,
+                            None) == 2                                               # dk != dv
+    assert L.gdn_bwd_varlen_workspace_bytes(3, 100, 300, 2, 6, 64, 64) > 0
+    assert L.gdn_bwd_varlen_workspace_bytes(3, 100, 300, 2, 6, 64, 32) == 0
