@@ -113,6 +113,11 @@ def lib() -> ctypes.CDLL:
         L.gdn_layer_bwd.restype = I
         L.gdn_layer_bwd_workspace_bytes.argtypes = [I] * 8
         L.gdn_layer_bwd_workspace_bytes.restype = SZ
+        L.gdn_layer_bwd_varlen.argtypes = ([P] * 5 + [I, I] + [P] * 21 + [SZ] + [I] * 6 +
+                                           [F, F, F, I, I, P])
+        L.gdn_layer_bwd_varlen.restype = I
+        L.gdn_layer_bwd_varlen_workspace_bytes.argtypes = [I] * 9
+        L.gdn_layer_bwd_varlen_workspace_bytes.restype = SZ
         L.gdn_gates_bwd.argtypes = [P, P, P, P, LL, I, I, P]
         L.gdn_gates_bwd.restype = I
         _lib = L
@@ -590,6 +595,44 @@ def layer_bwd(q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, d
             wbytes, B, T, Hk, Hv, dk, dv, chunk, float(scale), float(l2_eps), float(norm_eps),
             _io_dtype(q_raw), _io_dtype(dy), _stream(dev))
     _check("gdn_layer_bwd", st)
+    return out
+
+
+def layer_bwd_varlen(q_raw, k_raw, v_raw, z, cu_seqlens, max_seqlen: int, wq, wk, wv,
+                     log_alpha, beta, S0, norm_w, dy, dS_T=None, *, Hk: int, Hv: int, dk: int,
+                     dv: int, chunk: int = 64, scale: float = 1.0, l2_eps: float = 1e-6,
+                     norm_eps: float = 1e-5, want_dS0: bool = True) -> dict:
+    """layer_bwd over packed sequences (gdn_layer_bwd_varlen), laid out as layer_fwd_varlen's
+    inputs (no carried history): the same fp32 gradients, token tensors [total, ...] and dS0
+    [nseq, Hv, dk, dv]."""
+    total = q_raw.shape[0]
+    nseq = cu_seqlens.numel() - 1
+    if cu_seqlens.dtype != torch.int32:
+        raise ValueError("cu_seqlens must be int32")
+    _f32(wq, wk, wv, log_alpha, beta, S0, norm_w, dS_T)
+    f = dict(device=q_raw.device, dtype=torch.float32)
+    out = {"dq_raw": torch.empty(q_raw.shape, **f), "dk_raw": torch.empty(k_raw.shape, **f),
+           "dv_raw": torch.empty(v_raw.shape, **f), "dz": torch.empty(z.shape, **f),
+           "dwq": torch.empty(wq.shape, **f), "dwk": torch.empty(wk.shape, **f),
+           "dwv": torch.empty(wv.shape, **f), "dlog_alpha": torch.empty(log_alpha.shape, **f),
+           "dbeta": torch.empty(beta.shape, **f),
+           "dS0": torch.empty(nseq, Hv, dk, dv, **f) if want_dS0 else None,
+           "dnorm_w": torch.empty(norm_w.shape, **f)}
+    need = int(lib().gdn_layer_bwd_varlen_workspace_bytes(nseq, int(max_seqlen), total, Hk, Hv,
+                                                          dk, dv, chunk, _DTYPES[q_raw.dtype]))
+    dev = _dev(q_raw, k_raw, v_raw, z, cu_seqlens, wq, wk, wv, log_alpha, beta, S0, norm_w, dy,
+               dS_T)
+    ws = torch.empty(max(need, 1), device=dev, dtype=torch.uint8)
+    with torch.cuda.device(dev):
+        st = lib().gdn_layer_bwd_varlen(
+            _p(q_raw), _p(k_raw), _p(v_raw), _p(z), _p(cu_seqlens), nseq, int(max_seqlen),
+            _p(wq), _p(wk), _p(wv), _p(log_alpha), _p(beta), _p(S0), _p(norm_w), _p(dy),
+            _p(dS_T), _p(out["dq_raw"]), _p(out["dk_raw"]), _p(out["dv_raw"]), _p(out["dz"]),
+            _p(out["dwq"]), _p(out["dwk"]), _p(out["dwv"]), _p(out["dlog_alpha"]),
+            _p(out["dbeta"]), _p(out["dS0"]), _p(out["dnorm_w"]), _p(ws), need, total, Hk, Hv,
+            dk, dv, chunk, float(scale), float(l2_eps), float(norm_eps), _io_dtype(q_raw),
+            _io_dtype(dy), _stream(dev))
+    _check("gdn_layer_bwd_varlen", st)
     return out
 
 

@@ -979,19 +979,25 @@ constexpr unsigned kNormBwdCtas = 592;   // fixed grid of the norm backward (its
 struct LayerBwdLayout {
   size_t fwd = 0, d_o = 0, dq = 0, dk = 0, dv = 0, bwd = 0, dpre = 0, nw = 0, cw = 0, total = 0;
 };
+// The layer backward's workspace for B sequences of T tokens, or (packed) nseq = B sequences of
+// at most max_len tokens, T rows in all: the forward's buffers (q, k, v, fp32 o, hand-over), then
+// the backward's.
 LayerBwdLayout layer_bwd_layout(int B, int T, int Hk, int Hv, int dk, int dv, int chunk,
-                                gdn_dtype dtype) {
+                                gdn_dtype dtype, bool packed = false, int max_len = 0) {
   LayerBwdLayout L;
-  const size_t tok = (size_t)B * T;
+  if (!packed) max_len = T;
+  const size_t tok = packed ? (size_t)T : (size_t)B * T;
   const size_t C = std::max((size_t)Hk * dk, (size_t)Hv * dv);
-  const size_t tiles = (size_t)B * ((T + lbwd::kConvTok - 1) / lbwd::kConvTok);
-  size_t o = align256(gdn_layer_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, dtype));
+  const size_t tiles = (size_t)B * ((max_len + lbwd::kConvTok - 1) / lbwd::kConvTok);
+  size_t o = align256(packed ? gdn_layer_fwd_varlen_workspace_bytes(B, max_len, T, Hk, Hv, dk, dv,
+                                                                    chunk, dtype)
+                             : gdn_layer_workspace_bytes(B, T, Hk, Hv, dk, dv, chunk, dtype));
   L.fwd = 0;
   L.d_o = o;  o += align256(tok * Hv * dv * 4);
   L.dq = o;   o += align256(tok * Hk * dk * 4);
   L.dk = o;   o += align256(tok * Hk * dk * 4);
   L.dv = o;   o += align256(tok * Hv * dv * 4);
-  L.bwd = o;  o += align256(bwd_layout(B, T, Hk, Hv, dk, dv).total);
+  L.bwd = o;  o += align256(bwd_layout_rows(B, max_len, tok, Hk, Hv, dk, dv).total);
   L.dpre = o; o += align256(tok * C * 4);
   L.nw = o;   o += align256((size_t)kNormBwdCtas * dv * 4);
   L.cw = o;   o += align256(tiles * C * 4 * 4);
@@ -1002,20 +1008,25 @@ LayerBwdLayout layer_bwd_layout(int B, int T, int Hk, int Hv, int dk, int dv, in
 template <typename Tin>
 gdn_status prologue_bwd_one(const void* x_raw, const float* w, const float* dy, float* dx_raw,
                             float* dw, float* dpre, float* dw_part, int B, int T, int heads,
-                            int d, bool normalize, float eps, cudaStream_t st) {
-  const dim3 gd(heads, (T + lbwd::kDpreTok - 1) / lbwd::kDpreTok, B);
+                            int d, bool normalize, float eps, cudaStream_t st,
+                            const int* cu = nullptr, int max_len = -1) {
+  if (!cu) max_len = T;                       // B sequences of T rows, or packed (T rows in all)
+  const dim3 gd(heads, (max_len + lbwd::kDpreTok - 1) / lbwd::kDpreTok, B);
   const Tin* xr = static_cast<const Tin*>(x_raw);
   const int nz = normalize ? 1 : 0;
   if (d == 128)
-    lbwd::conv_dpre_kernel<Tin, 4><<<gd, 128, 0, st>>>(xr, w, dy, dpre, T, heads, d, nz, eps);
+    lbwd::conv_dpre_kernel<Tin, 4><<<gd, 128, 0, st>>>(xr, w, dy, dpre, T, heads, d, nz, eps, cu,
+                                                       max_len);
   else if (d == 64)
-    lbwd::conv_dpre_kernel<Tin, 2><<<gd, 128, 0, st>>>(xr, w, dy, dpre, T, heads, d, nz, eps);
+    lbwd::conv_dpre_kernel<Tin, 2><<<gd, 128, 0, st>>>(xr, w, dy, dpre, T, heads, d, nz, eps, cu,
+                                                       max_len);
   else
-    lbwd::conv_dpre_kernel<Tin, 1><<<gd, 128, 0, st>>>(xr, w, dy, dpre, T, heads, d, nz, eps);
+    lbwd::conv_dpre_kernel<Tin, 1><<<gd, 128, 0, st>>>(xr, w, dy, dpre, T, heads, d, nz, eps, cu,
+                                                       max_len);
   const int C = heads * d;
-  const dim3 grid((C + 127) / 128, (T + lbwd::kConvTok - 1) / lbwd::kConvTok, B);
+  const dim3 grid((C + 127) / 128, (max_len + lbwd::kConvTok - 1) / lbwd::kConvTok, B);
   lbwd::conv_bwd_kernel<Tin><<<grid, 128, 0, st>>>(static_cast<const Tin*>(x_raw), w, dpre,
-                                                   dx_raw, dw_part, T, C);
+                                                   dx_raw, dw_part, T, C, cu, max_len);
   lbwd::col_sum_kernel<<<(C * 4 + 255) / 256, 256, 0, st>>>(dw_part, dw, (int)(grid.y * grid.z),
                                                             C * 4);
   return launch_status();
@@ -1029,21 +1040,33 @@ gdn_status layer_bwd_run(const void* q_raw, const void* k_raw, const void* v_raw
                          float* dz, float* dwq, float* dwk, float* dwv, float* dla, float* dbeta,
                          float* dS0, float* dnorm_w, char* ws, const LayerBwdLayout& L, int B,
                          int T, int Hk, int Hv, int dk, int dv, int chunk, float scale,
-                         float l2_eps, float norm_eps, gdn_dtype dtype, gdn_stream_t stream) {
+                         float l2_eps, float norm_eps, gdn_dtype dtype, gdn_stream_t stream,
+                         const int* cu = nullptr, int max_len = -1) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const size_t el = dtype == GDN_F32 ? 4 : 2;
-  const size_t tok = (size_t)B * T;
+  const size_t tok = cu ? (size_t)T : (size_t)B * T;   // packed: B sequences, T rows in all
   void* qn = ws;
   void* kn = ws + align256(tok * Hk * dk * el);
   void* vc = ws + 2 * align256(tok * Hk * dk * el);
   char* rest = ws + 2 * align256(tok * Hk * dk * el) + align256(tok * Hv * dv * el);
   float* o = reinterpret_cast<float*>(rest);
   void* tc_scratch = rest + align256(tok * Hv * dv * 4);
-  gdn_status s = gdn_prologue(q_raw, k_raw, v_raw, wq, wk, wv, qn, kn, vc, B, T, Hk, Hv, dk, dv,
-                              l2_eps, dtype, stream);
-  if (s != GDN_OK) return s;
-  s = layer_chunk_fwd(qn, kn, vc, la, be, S0, o, nullptr, B, T, Hk, Hv, dk, dv, chunk, scale,
-                      dtype, tc_scratch, st);
+  gdn_status s;
+  if (cu) {   // packed rows: the tensor-core recurrence over the sequences' spans
+    // o of rows in no sequence stays zero, so the norm's backward adds nothing from them
+    if (cudaMemsetAsync(o, 0, tok * Hv * dv * 4, st) != cudaSuccess) return GDN_ERR_CUDA;
+    s = prologue_launch(q_raw, k_raw, v_raw, nullptr, nullptr, nullptr, wq, wk, wv, qn, kn, vc, B,
+                        T, Hk, Hv, dk, dv, l2_eps, dtype, cu, max_len, st);
+    if (s != GDN_OK) return s;
+    s = tc_chunk_launch_varlen(qn, kn, vc, la, be, cu, B, max_len, S0, o, nullptr, T, Hk, Hv,
+                               scale, true, tc_scratch, st);
+  } else {
+    s = gdn_prologue(q_raw, k_raw, v_raw, wq, wk, wv, qn, kn, vc, B, T, Hk, Hv, dk, dv, l2_eps,
+                     dtype, stream);
+    if (s != GDN_OK) return s;
+    s = layer_chunk_fwd(qn, kn, vc, la, be, S0, o, nullptr, B, T, Hk, Hv, dk, dv, chunk, scale,
+                        dtype, tc_scratch, st);
+  }
   if (s != GDN_OK) return s;
   float* d_o = reinterpret_cast<float*>(ws + L.d_o);
   float* nw = reinterpret_cast<float*>(ws + L.nw);
@@ -1057,16 +1080,18 @@ gdn_status layer_bwd_run(const void* q_raw, const void* k_raw, const void* v_raw
   float* dkg = reinterpret_cast<float*>(ws + L.dk);
   float* dvg = reinterpret_cast<float*>(ws + L.dv);
   s = bwd_dispatch<Tin, float>(dk, qn, kn, vc, la, be, S0, d_o, dS_T, dqg, dkg, dvg, dla, dbeta,
-                               dS0, ws + L.bwd, B, T, Hk, Hv, scale, st);
+                               dS0, ws + L.bwd, B, T, Hk, Hv, scale, st, cu, max_len);
   if (s != GDN_OK) return s;
   float* dpre = reinterpret_cast<float*>(ws + L.dpre);
   float* cw = reinterpret_cast<float*>(ws + L.cw);
-  s = prologue_bwd_one<Tin>(q_raw, wq, dqg, dq_raw, dwq, dpre, cw, B, T, Hk, dk, true, l2_eps, st);
+  s = prologue_bwd_one<Tin>(q_raw, wq, dqg, dq_raw, dwq, dpre, cw, B, T, Hk, dk, true, l2_eps, st,
+                            cu, max_len);
   if (s == GDN_OK)
     s = prologue_bwd_one<Tin>(k_raw, wk, dkg, dk_raw, dwk, dpre, cw, B, T, Hk, dk, true, l2_eps,
-                              st);
+                              st, cu, max_len);
   if (s == GDN_OK)
-    s = prologue_bwd_one<Tin>(v_raw, wv, dvg, dv_raw, dwv, dpre, cw, B, T, Hv, dv, false, 0.f, st);
+    s = prologue_bwd_one<Tin>(v_raw, wv, dvg, dv_raw, dwv, dpre, cw, B, T, Hv, dv, false, 0.f, st,
+                              cu, max_len);
   return s;
 }
 }  // namespace
@@ -1126,6 +1151,76 @@ gdn_status gdn_layer_bwd(const void* q_raw, const void* k_raw, const void* v_raw
       q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, dy, dS_T, dq_raw, dk_raw,
       dv_raw, dz, dwq, dwk, dwv, dlog_alpha, dbeta, dS0, dnorm_w, ws, L, B, T, Hk, Hv, dk, dv,
       chunk, scale, l2_eps, norm_eps, dtype, stream);
+}
+
+size_t gdn_layer_bwd_varlen_workspace_bytes(int nseq, int max_seqlen, int total_T, int Hk, int Hv,
+                                            int dk, int dv, int chunk, gdn_dtype dtype) {
+  if (nseq <= 0 || max_seqlen <= 0 || total_T <= 0 || validate_heads(Hk, Hv, dk, dv) != GDN_OK ||
+      dk != dv || !valid_dtype(dtype) || !tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16))
+    return 0;
+  return layer_bwd_layout(nseq, total_T, Hk, Hv, dk, dv, chunk, dtype, true, max_seqlen).total;
+}
+
+gdn_status gdn_layer_bwd_varlen(const void* q_raw, const void* k_raw, const void* v_raw,
+                                const void* z, const int* cu_seqlens, int nseq, int max_seqlen,
+                                const float* wq, const float* wk, const float* wv,
+                                const float* log_alpha, const float* beta, const float* S0,
+                                const float* norm_w, const void* dy, const float* dS_T,
+                                float* dq_raw, float* dk_raw, float* dv_raw, float* dz,
+                                float* dwq, float* dwk, float* dwv, float* dlog_alpha,
+                                float* dbeta, float* dS0, float* dnorm_w, void* workspace,
+                                size_t workspace_bytes, int total_T, int Hk, int Hv, int dk,
+                                int dv, int chunk, float scale, float l2_eps, float norm_eps,
+                                gdn_dtype dtype, gdn_dtype dy_dtype, gdn_stream_t stream) {
+  if (nseq < 0 || max_seqlen < 0 || total_T < 0 || !valid_dtype(dtype) || !valid_dtype(dy_dtype))
+    return GDN_ERR_INVALID_ARG;
+  if (!io_pair_ok(dtype, dy_dtype)) return GDN_ERR_UNSUPPORTED;
+  gdn_status s = validate_heads(Hk, Hv, dk, dv);
+  if (s != GDN_OK) return s;
+  if (chunk <= 0 || !(norm_eps >= 0.f) || !(l2_eps >= 0.f)) return GDN_ERR_INVALID_ARG;
+  if (dk != dv || !tc_chunk_supported(dk, dv, chunk, dtype == GDN_BF16)) return GDN_ERR_UNSUPPORTED;
+  if (nseq > 65535 || (long)nseq * Hv * bwd::head_slices(dk) > 0x7fffffffL ||
+      (long)total_T * Hv > 0x7fffffffL * 8L)
+    return GDN_ERR_UNSUPPORTED;
+  if (nseq == 0) return GDN_OK;
+  if (!cu_seqlens || !aligned4(cu_seqlens)) return GDN_ERR_INVALID_ARG;
+  const float* w4[] = {wq, wk, wv, norm_w};
+  float* dw4[] = {dwq, dwk, dwv, dnorm_w};
+  for (int i = 0; i < 4; ++i)
+    if (!w4[i] || !dw4[i] || !aligned4(w4[i]) || !aligned4(dw4[i])) return GDN_ERR_INVALID_ARG;
+  if (!opt_aligned16(S0) || !opt_aligned16(dS_T) || !opt_aligned16(dS0)) return GDN_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (total_T == 0 || max_seqlen == 0) {   // every sequence is empty: dS0 = dS_T, no weight grads
+    const size_t wb[] = {(size_t)Hk * dk * 16, (size_t)Hk * dk * 16, (size_t)Hv * dv * 16,
+                         (size_t)dv * 4};
+    for (int i = 0; i < 4; ++i)
+      if (cudaMemsetAsync(dw4[i], 0, wb[i], st) != cudaSuccess) return GDN_ERR_CUDA;
+    return gdn_bwd_varlen(nullptr, nullptr, nullptr, nullptr, nullptr, cu_seqlens, nseq, 0, S0,
+                          nullptr, dS_T, nullptr, nullptr, nullptr, nullptr, nullptr, dS0,
+                          nullptr, 0, 0, Hk, Hv, dk, dv, scale, dtype, stream);
+  }
+  const void* in16[] = {q_raw, k_raw, v_raw, z, dy};
+  for (const void* p : in16)
+    if (!p || !aligned16(p)) return GDN_ERR_INVALID_ARG;
+  const void* in4[] = {log_alpha, beta, dq_raw, dk_raw, dv_raw, dz, dlog_alpha, dbeta};
+  for (const void* p : in4)
+    if (!p || !aligned4(p)) return GDN_ERR_INVALID_ARG;
+  if (!tc_chunk_length_ok(max_seqlen) ||
+      (max_seqlen + kPrologueTokens - 1) / kPrologueTokens > 65535)
+    return GDN_ERR_UNSUPPORTED;
+  const LayerBwdLayout L =
+      layer_bwd_layout(nseq, total_T, Hk, Hv, dk, dv, chunk, dtype, true, max_seqlen);
+  if (!workspace_ok(workspace, workspace_bytes, L.total)) return GDN_ERR_INVALID_ARG;
+  char* ws = static_cast<char*>(workspace);
+  if (dy_dtype == GDN_F32)
+    return layer_bwd_run<__nv_bfloat16, float>(
+        q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, dy, dS_T, dq_raw, dk_raw,
+        dv_raw, dz, dwq, dwk, dwv, dlog_alpha, dbeta, dS0, dnorm_w, ws, L, nseq, total_T, Hk, Hv,
+        dk, dv, chunk, scale, l2_eps, norm_eps, dtype, stream, cu_seqlens, max_seqlen);
+  return layer_bwd_run<__nv_bfloat16, __nv_bfloat16>(
+      q_raw, k_raw, v_raw, z, wq, wk, wv, log_alpha, beta, S0, norm_w, dy, dS_T, dq_raw, dk_raw,
+      dv_raw, dz, dwq, dwk, dwv, dlog_alpha, dbeta, dS0, dnorm_w, ws, L, nseq, total_T, Hk, Hv, dk,
+      dv, chunk, scale, l2_eps, norm_eps, dtype, stream, cu_seqlens, max_seqlen);
 }
 
 gdn_status gdn_gates_bwd(const void* ba, const float* dlog_alpha, const float* dbeta, float* dba,

@@ -135,15 +135,18 @@ constexpr int kDpreTok = 64;    // tokens per CTA of conv_dpre_kernel (16 per wa
 //   s = SiLU(pre);  q, k (normalize): y = s / n, n = sqrt(s . s + eps),
 //   ds = dy / n - s (s . dy) / n^3;  v: ds = dy;  dpre = ds SiLU'(pre).
 // x: raw inputs [B, T, heads * d]; dy: [B, T, heads, d] fp32; dpre: [B, T, heads * d] fp32; x, dy
-// and dpre aligned to PER values.
+// and dpre aligned to PER values.  Sequences as in row_span (cu: packed rows of T in all, grid z
+// over the sequences, y over ceil(max_len / kDpreTok) tiles).
 template <typename Tin, int PER>
 __global__ void __launch_bounds__(128)
 conv_dpre_kernel(const Tin* __restrict__ x, const float* __restrict__ w,
                  const float* __restrict__ dy, float* __restrict__ dpre, int T, int heads, int d,
-                 int normalize, float eps) {
+                 int normalize, float eps, const int* __restrict__ cu, int max_len) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int h = blockIdx.x;
-  const long b = blockIdx.z;
+  const RowSpan sp = row_span(cu, (int)blockIdx.z, T, max_len);   // this sequence's rows
+  const long r0 = sp.row0;
+  const int Ts = sp.len;
   const int tb = blockIdx.y * kDpreTok + warp * (kDpreTok / 4);
   const int C = heads * d;
   const bool on = lane * PER < d;
@@ -153,11 +156,11 @@ conv_dpre_kernel(const Tin* __restrict__ x, const float* __restrict__ w,
   for (int e = 0; e < PER; ++e)
 #pragma unroll
     for (int j = 0; j < 4; ++j) wt[e][j] = on ? w[(ch0 + e) * 4 + j] : 0.f;
-  const Tin* xb = x + b * (long)T * C + ch0;
-  auto row_in = [&](int t, float (&v)[PER]) {  // raw inputs of token t (zeros outside 0 .. T - 1)
+  const Tin* xb = x + r0 * C + ch0;
+  auto row_in = [&](int t, float (&v)[PER]) {  // raw inputs of token t (zeros outside 0 .. Ts - 1)
 #pragma unroll
     for (int e = 0; e < PER; ++e) v[e] = 0.f;
-    if (on && t >= 0 && t < T) vload<PER>(xb + (long)t * C, v);
+    if (on && t >= 0 && t < Ts) vload<PER>(xb + (long)t * C, v);
   };
   float r[4][PER];
   row_in(tb - 3, r[0]);
@@ -168,10 +171,10 @@ conv_dpre_kernel(const Tin* __restrict__ x, const float* __restrict__ w,
 #pragma unroll
     for (int sl = 0; sl < 4; ++sl) {
       const int t = tb + t4 + sl;
-      if (t >= T) break;                      // uniform over the warp
-      const int r0 = sl, r1 = (sl + 1) & 3, r2 = (sl + 2) & 3, r3 = (sl + 3) & 3;
+      if (t >= Ts) break;                     // uniform over the warp
+      const int q0 = sl, r1 = (sl + 1) & 3, r2 = (sl + 2) & 3, r3 = (sl + 3) & 3;
       row_in(t, r[r3]);
-      const long row = (b * T + t) * heads + h;
+      const long row = (r0 + t) * heads + h;
       float pre[PER], s[PER], g[PER];
 #pragma unroll
       for (int e = 0; e < PER; ++e) g[e] = 0.f;
@@ -182,7 +185,7 @@ conv_dpre_kernel(const Tin* __restrict__ x, const float* __restrict__ w,
         // the taps in order (w[.., 3] on token t), as the forward's sum; a zero-history tap adds
         // nothing
         float acc = 0.f;
-        if (t - 3 >= 0) acc = fmaf(wt[e][0], r[r0][e], acc);
+        if (t - 3 >= 0) acc = fmaf(wt[e][0], r[q0][e], acc);
         if (t - 2 >= 0) acc = fmaf(wt[e][1], r[r1][e], acc);
         if (t - 1 >= 0) acc = fmaf(wt[e][2], r[r2][e], acc);
         acc = fmaf(wt[e][3], r[r3][e], acc);
@@ -205,7 +208,7 @@ conv_dpre_kernel(const Tin* __restrict__ x, const float* __restrict__ w,
           const float ds = normalize ? g[e] / n - s[e] * sd / n3 : g[e];
           out[e] = ds * silu_grad(pre[e]);
         }
-        vstore<PER>(dpre + (b * T + t) * (long)C + ch0, out);
+        vstore<PER>(dpre + (r0 + t) * (long)C + ch0, out);
       }
     }
   }
@@ -217,22 +220,26 @@ constexpr int kConvTok = 64;    // tokens per CTA of conv_bwd_kernel
 // 128-channel block over kConvTok tokens, dpre and x in rings of four registers (each read once):
 //   dx[t] = sum_j w[j] dpre[t + 3 - j]  (t + 3 - j < T),
 //   dw[j] += dpre[t] x[t - 3 + j]  (t - 3 + j >= 0), per CTA: dw_part[cta][C][4], cta over
-//   (token tile, batch).  grid (ceil(C / 128), ceil(T / kConvTok), B).
+//   (token tile, batch).  grid (ceil(C / 128), ceil(T / kConvTok), B); packed sequences as in
+//   conv_dpre_kernel (a tile past its sequence's end writes zero partial sums).
 template <typename Tin>
 __global__ void __launch_bounds__(128)
 conv_bwd_kernel(const Tin* __restrict__ x, const float* __restrict__ w,
                 const float* __restrict__ dpre, float* __restrict__ dx,
-                float* __restrict__ dw_part, int T, int C) {
+                float* __restrict__ dw_part, int T, int C, const int* __restrict__ cu,
+                int max_len) {
   const int c = blockIdx.x * 128 + threadIdx.x;
-  const long b = blockIdx.z;
+  const RowSpan sp = row_span(cu, (int)blockIdx.z, T, max_len);   // this sequence's rows
+  const long r0 = sp.row0;
+  const int Ts = sp.len;
   const int t0 = blockIdx.y * kConvTok;
   const long cta = (long)blockIdx.z * gridDim.y + blockIdx.y;
   if (c >= C) return;
   const float w0 = w[c * 4], w1 = w[c * 4 + 1], w2 = w[c * 4 + 2], w3 = w[c * 4 + 3];
   float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-  const int t1 = min(T, t0 + kConvTok);
-  auto P = [&](int t) -> float { return t < T ? dpre[(b * T + t) * C + c] : 0.f; };
-  auto X = [&](int t) -> float { return t >= 0 ? to_f(x[(b * T + t) * C + c]) : 0.f; };
+  const int t1 = min(Ts, t0 + kConvTok);
+  auto P = [&](int t) -> float { return t < Ts ? dpre[(r0 + t) * C + c] : 0.f; };
+  auto X = [&](int t) -> float { return t >= 0 && t < Ts ? to_f(x[(r0 + t) * C + c]) : 0.f; };
   // p[t mod 4] = dpre[t] for t .. t + 3, xr[t mod 4] = x[t - 3 + ...] for t - 3 .. t
   float p[4], xr[4];
   p[0] = P(t0); p[1] = P(t0 + 1); p[2] = P(t0 + 2);
@@ -243,15 +250,15 @@ conv_bwd_kernel(const Tin* __restrict__ x, const float* __restrict__ w,
     for (int sl = 0; sl < 4; ++sl) {
       const int t = t0 + t4 + sl;
       if (t >= t1) break;
-      const int r0 = sl, r1 = (sl + 1) & 3, r2 = (sl + 2) & 3, r3 = (sl + 3) & 3;
+      const int q0 = sl, r1 = (sl + 1) & 3, r2 = (sl + 2) & 3, r3 = (sl + 3) & 3;
       p[r3] = P(t + 3);
       xr[r3] = X(t);
       // tap j multiplies x[t - 3 + j] in the output at t, so x[t] feeds outputs t + 3 - j
-      dx[(b * T + t) * C + c] = fmaf(w0, p[r3], fmaf(w1, p[r2], fmaf(w2, p[r1], w3 * p[r0])));
-      a0 = fmaf(p[r0], xr[r0], a0);
-      a1 = fmaf(p[r0], xr[r1], a1);
-      a2 = fmaf(p[r0], xr[r2], a2);
-      a3 = fmaf(p[r0], xr[r3], a3);
+      dx[(r0 + t) * C + c] = fmaf(w0, p[r3], fmaf(w1, p[r2], fmaf(w2, p[r1], w3 * p[q0])));
+      a0 = fmaf(p[q0], xr[q0], a0);
+      a1 = fmaf(p[q0], xr[r1], a1);
+      a2 = fmaf(p[q0], xr[r2], a2);
+      a3 = fmaf(p[q0], xr[r3], a3);
     }
   }
   float* dp = dw_part + (cta * C + c) * 4;

@@ -333,7 +333,7 @@ GDN_API size_t gdn_bwd_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int
  * dk == dv (else GDN_ERR_UNSUPPORTED); other limits as gdn_layer_fwd and gdn_bwd.  Weight
  * gradients are sums of per-CTA partial sums taken in a fixed order (reproducible bit for bit).
  * The sequence starts fresh: the conv sees zeros before token 0, as in gdn_layer_fwd (there is
- * no backward of gdn_layer_fwd_ex's carried history).
+ * no backward of gdn_layer_fwd_ex's carried history).  Packed sequences: gdn_layer_bwd_varlen.
  */
 GDN_API gdn_status gdn_layer_bwd(const void *q_raw, const void *k_raw, const void *v_raw,
                          const void *z, const float *wq, const float *wk, const float *wv,
@@ -348,6 +348,40 @@ GDN_API gdn_status gdn_layer_bwd(const void *q_raw, const void *k_raw, const voi
 /* Device scratch bytes gdn_layer_bwd needs (host only, no CUDA call); 0 for invalid sizes. */
 GDN_API size_t gdn_layer_bwd_workspace_bytes(int B, int T, int Hk, int Hv, int dk, int dv,
                                              int chunk, gdn_dtype dtype);
+
+/*
+ * gdn_layer_bwd over packed sequences of different lengths: sequence s owns rows cu_seqlens[s] ..
+ * cu_seqlens[s + 1] - 1 of every token tensor (total_T rows in all, none longer than max_seqlen),
+ * as gdn_layer_fwd_varlen lays them out, and starts fresh (the conv sees zeros before its first
+ * token; there is no carried history).  Each sequence's gradients equal gdn_layer_bwd on that
+ * sequence alone up to the order of the weight gradients' sums (per-CTA partial sums over the
+ * packed tiles, taken in a fixed order).
+ *   q_raw, k_raw [total_T, Hk * dk]; v_raw, z [total_T, Hv * dv]; dy [total_T, Hv * dv] (dy_dtype)
+ *   log_alpha, beta [total_T, Hv]; S0, dS_T, dS0 [nseq, Hv, dk, dv] (nullable)
+ *   dq_raw, dk_raw [total_T, Hk * dk]; dv_raw, dz [total_T, Hv * dv]; dlog_alpha, dbeta
+ *   [total_T, Hv]; dwq, dwk [Hk * dk, 4]; dwv [Hv * dv, 4]; dnorm_w [dv] (float outputs)
+ *   workspace: gdn_layer_bwd_varlen_workspace_bytes(...) bytes, 256-byte aligned, caller-owned.
+ * The tensor-core shape only (bf16 inputs, dk = dv = 128, chunk 64; else GDN_ERR_UNSUPPORTED).
+ * Rows in no sequence (past cu_seqlens[nseq], or cut off by max_seqlen) add nothing to the
+ * weight gradients and get dz = 0; their other gradients are unspecified.  An empty sequence hands
+ * dS_T on as dS0; when every sequence is empty the weight gradients are zeros.
+ */
+GDN_API gdn_status gdn_layer_bwd_varlen(const void *q_raw, const void *k_raw, const void *v_raw,
+                         const void *z, const int *cu_seqlens, int nseq, int max_seqlen,
+                         const float *wq, const float *wk, const float *wv,
+                         const float *log_alpha, const float *beta, const float *S0,
+                         const float *norm_w, const void *dy, const float *dS_T, float *dq_raw,
+                         float *dk_raw, float *dv_raw, float *dz, float *dwq, float *dwk,
+                         float *dwv, float *dlog_alpha, float *dbeta, float *dS0, float *dnorm_w,
+                         void *workspace, size_t workspace_bytes, int total_T, int Hk, int Hv,
+                         int dk, int dv, int chunk, float scale, float l2_eps, float norm_eps,
+                         gdn_dtype dtype, gdn_dtype dy_dtype, gdn_stream_t stream);
+
+/* Device scratch bytes gdn_layer_bwd_varlen needs (host only, no CUDA call); 0 for invalid
+ * sizes. */
+GDN_API size_t gdn_layer_bwd_varlen_workspace_bytes(int nseq, int max_seqlen, int total_T, int Hk,
+                                                    int Hv, int dk, int dv, int chunk,
+                                                    gdn_dtype dtype);
 
 /*
  * Backward of gdn_gates: dba [rows, 2*Hv] float, the b gradients dbeta beta (1 - beta) then the a

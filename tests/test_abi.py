@@ -350,3 +350,26 @@ def test_bwd_varlen_validation(L):
                             None) == 2                                               # dk != dv
     assert L.gdn_bwd_varlen_workspace_bytes(3, 100, 300, 2, 6, 64, 64) > 0
     assert L.gdn_bwd_varlen_workspace_bytes(3, 100, 300, 2, 6, 64, 32) == 0
+
+
+def test_layer_bwd_varlen_validation(L):
+    """gdn_layer_bwd_varlen: no sequences is a no-op; missing offsets or workspace (1); a shape
+    off the tensor-core path or bf16 gradients of fp32 inputs (2); the workspace query follows."""
+    pre = [FAKE] * 4
+    mid = [FAKE] * 9                                  # taps, gates, S0, norm gain, dy, dS_T
+    outs = [FAKE] * 11
+    ws = [P(0x100000), 1 << 40]
+    sizes = [700, 2, 16, 128, 128, 64, 1.0, 1e-6, 1e-5, 1, 1, None]
+    assert L.gdn_layer_bwd_varlen(*pre, FAKE, 0, 300, *mid, *outs, None, 0, *sizes) == 0
+    assert L.gdn_layer_bwd_varlen(*pre, None, 4, 300, *mid, *outs, *ws, *sizes) == 1
+    assert L.gdn_layer_bwd_varlen(*pre, FAKE, 4, 300, *mid, *outs, None, 0, *sizes) == 1
+    assert L.gdn_layer_bwd_varlen(*pre, FAKE, 4, 300, *mid, *outs, *ws, 700, 2, 16, 64, 64, 64,
+                                  1.0, 1e-6, 1e-5, 1, 1, None) == 2      # d = 64
+    assert L.gdn_layer_bwd_varlen(*pre, FAKE, 4, 300, *mid, *outs, *ws, 700, 2, 16, 128, 128, 64,
+                                  1.0, 1e-6, 1e-5, 0, 1, None) == 2      # fp32 in, bf16 dy
+    assert L.gdn_layer_bwd_varlen(*pre, FAKE, 4, 300, *mid, *outs, *ws, 700, 2, 16, 128, 128, 64,
+                                  1.0, -1.0, 1e-5, 1, 1, None) == 1      # negative eps
+    big = L.gdn_layer_bwd_varlen_workspace_bytes(4, 300, 700, 2, 16, 128, 128, 64, 1)
+    assert big > L.gdn_layer_fwd_varlen_workspace_bytes(4, 300, 700, 2, 16, 128, 128, 64, 1)
+    assert L.gdn_layer_bwd_varlen_workspace_bytes(4, 300, 700, 2, 16, 64, 64, 64, 1) == 0
+    assert L.gdn_layer_bwd_varlen_workspace_bytes(4, 300, 700, 2, 16, 128, 128, 64, 0) == 0
