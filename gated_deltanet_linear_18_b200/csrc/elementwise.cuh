@@ -194,11 +194,26 @@ prologue_v_kernel(const Tio* __restrict__ x, const Tio* __restrict__ hist,
   const int nt = rem < kPrologueTokens ? (int)rem : kPrologueTokens;
   Tio* const yt = y + (sp.row0 + t0) * width + c0;        // this thread's channels of token t0
   const Tio* const xr = tile + lc * 4;                    // ... of tile row 0
+  // The four channels run as two pairs on sm_100's paired fp32 instructions (each lane the IEEE
+  // operation of the scalar form, so every value and every rounding decision is that of the
+  // scalar arithmetic): weights and window rows are held as channel pairs.
+  f2_t w2[2][4];                              // [channel pair][tap]
+#pragma unroll
+  for (int jp = 0; jp < 2; ++jp)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) w2[jp][k] = pk2(wk[2 * jp][k], wk[2 * jp + 1][k]);
   // token i reads tile rows i .. i + 3 at ring slots i .. i + 3 (mod 4): with the token loop
   // unrolled by four no row is ever moved
-  float h[4][4];
+  f2_t h[4][2];
+  auto load_row = [&](long row, f2_t (&hr)[2]) {
+    float v[4];
+    Vec4<Tio>::load(xr + row * d, v);
+    hr[0] = pk2(v[0], v[1]);
+    hr[1] = pk2(v[2], v[3]);
+  };
 #pragma unroll
-  for (int r = 0; r < 3; ++r) Vec4<Tio>::load(xr + (long)(i0 + r) * d, h[r]);
+  for (int r = 0; r < 3; ++r) load_row(i0 + r, h[r]);
+  const f2_t neg_log2e = splat2(-1.4426950408889634f), one2 = splat2(1.0f);
   unsigned long long umask = 0ull;            // undecided values: bit 4 (i - i0) + channel
 #pragma unroll 1
   for (int t4 = 0; t4 < tpg; t4 += 4) {
@@ -208,22 +223,36 @@ prologue_v_kernel(const Tio* __restrict__ x, const Tio* __restrict__ hist,
       if (t4 + sl >= tpg) break;              // tpg = 2 for 16-channel heads
       const int i = i0 + t4 + sl;
       const int r0 = sl, r1 = (sl + 1) & 3, r2 = (sl + 2) & 3, r3 = (sl + 3) & 3;
-      Vec4<Tio>::load(xr + (long)(i + 3) * d, h[r3]);
+      load_row(i + 3, h[r3]);
       float yv_[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float p0 = wk[j][0] * h[r0][j];
-        const float p1 = fmaf(wk[j][1], h[r1][j], p0);
-        const float p2 = fmaf(wk[j][2], h[r2][j], p1);
-        const float pre = fmaf(wk[j][3], h[r3][j], p2);
+      for (int jp = 0; jp < 2; ++jp) {
+        const f2_t p0 = mul2(w2[jp][0], h[r0][jp]);
+        const f2_t p1 = fma2(w2[jp][1], h[r1][jp], p0);
+        const f2_t p2 = fma2(w2[jp][2], h[r2][jp], p1);
+        const f2_t pre = fma2(w2[jp][3], h[r3][jp], p2);
         // SiLU(pre) = pre / (1 + 2^(-pre log2 e))
-        const float sv = pre * rcp_fast(1.0f + ex2_fast(pre * -1.4426950408889634f));
-        yv_[j] = sv;
+        float ea, eb, da, db, s0, s1;
+        up2(mul2(pre, neg_log2e), ea, eb);
+        up2(add2(one2, pk2(ex2_fast(ea), ex2_fast(eb))), da, db);
+        const f2_t sv = mul2(pre, pk2(rcp_fast(da), rcp_fast(db)));
+        up2(sv, s0, s1);
+        yv_[2 * jp] = s0;
+        yv_[2 * jp + 1] = s1;
         if constexpr (kBf16) {
           // half the bound's bracket: 10 |s| + pre s + 0.6 P (pre s = |pre| |s|)
-          const float P = (fabsf(p0) + fabsf(p1)) + (fabsf(p2) + fabsf(pre));
-          const float E = fmaf(pre, sv, fmaf(P, 0.6f, 10.0f * fabsf(sv)));
-          if (!bf16_decided_e24(sv, E + E)) m16 |= 1u << (sl * 4 + j);
+          float a0, a1, b0, b1, c0, c1, e0, e1;
+          up2(p0, a0, a1);
+          up2(p1, b0, b1);
+          up2(p2, c0, c1);
+          up2(pre, e0, e1);
+          const f2_t P = pk2((fabsf(a0) + fabsf(b0)) + (fabsf(c0) + fabsf(e0)),
+                             (fabsf(a1) + fabsf(b1)) + (fabsf(c1) + fabsf(e1)));
+          float E0, E1;
+          up2(fma2(pre, sv, fma2(P, splat2(0.6f), pk2(10.0f * fabsf(s0), 10.0f * fabsf(s1)))),
+              E0, E1);
+          if (!bf16_decided_e24(s0, E0 + E0)) m16 |= 1u << (sl * 4 + 2 * jp);
+          if (!bf16_decided_e24(s1, E1 + E1)) m16 |= 1u << (sl * 4 + 2 * jp + 1);
         }
       }
       if (i < nt) Vec4<Tio>::store(yt + (long)i * width, yv_);
