@@ -15,10 +15,12 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["GdnError", "lib", "library_path", "chunk_fwd", "chunk_fwd_variant",
-           "chunk_fwd_workspace_bytes", "chunk_fwd_launches", "chunk_fwd_ba", "decode_step",
-           "prologue", "out_norm", "layer_fwd", "layer_workspace_bytes", "check_error",
-           "STATUS", "VARIANTS"]
+__all__ = ["GdnError", "lib", "library_path", "STATUS", "VARIANTS", "check_error",
+           "chunk_fwd", "chunk_fwd_ba", "chunk_fwd_varlen", "chunk_fwd_variant",
+           "chunk_fwd_workspace_bytes", "chunk_fwd_launches", "decode_step", "decode_layer_step",
+           "gates", "gates_bwd", "prologue", "out_norm", "layer_fwd", "layer_fwd_varlen",
+           "layer_fwd_static", "layer_workspace_bytes", "bwd", "bwd_varlen", "bwd_workspace_bytes",
+           "bwd_launches", "layer_bwd", "layer_bwd_varlen", "layer_bwd_workspace_bytes"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_PKG, "libgdn.so")
