@@ -50,7 +50,7 @@
  * Errors.  Calls return gdn_status and never abort, throw or trap.  GDN_ERR_INVALID_ARG: a null
  * required pointer, a non-positive size, Hv not a multiple of Hk, misalignment, or an
  * unsupported enum value, or a missing, misaligned or too small workspace; nothing is enqueued.
- * GDN_ERR_UNSUPPORTED: valid sizes or dtypes this build has no kernel for (dk, dv not in {16, 32,
+ * GDN_ERR_UNSUPPORTED: valid sizes or dtypes the library has no kernel for (dk, dv not in {16, 32,
  * 64, 128}, chunk not in {16, 32, 64}, fp32 inputs with a bf16 output); nothing enqueued.
  * GDN_ERR_CUDA: a CUDA call failed (e.g. the launch); the CUDA error is left for
  * cudaGetLastError.  GDN_ERR_TIMEOUT is reported by gdn_check_error when a kernel gave up on a
