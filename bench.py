@@ -13,8 +13,8 @@ events) separates timed steps.  Device time comes from CUDA events on the launch
 torchrun each rank runs an independent replica of the workload (the path shards over sequences and
 heads with no exchange), a barrier brackets the timed region and the time is the max over ranks.
 
---impl reference times the fp64 CPU oracle (no other reference implementation is installed) on the host cores,
-on a bounded sample of the same workload per step.
+--impl reference times the fp64 CPU oracle (no other reference implementation is installed) on
+the host cores, on a bounded sample of the same workload per step.
 """
 from __future__ import annotations
 
