@@ -474,22 +474,12 @@ inline size_t prologue_smem_bytes(int d, size_t elem) {
   return (size_t)(kPrologueTokens + 3) * d * elem;
 }
 
-// The gated norm: one warp per row of dv <= 128 values, 4 consecutive channels per lane.  `o` may
-// be wider than z / y (the layer keeps o in fp32).
-template <typename To, typename Tz, typename Ty = Tz>
-__global__ void __launch_bounds__(256)
-out_norm_kernel(const To* __restrict__ o, const Tz* __restrict__ z, const float* __restrict__ w,
-                Ty* __restrict__ y, long long rows, int dv, float eps) {
-  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  const int c = 4 * lane;
-  const bool active = c < dv;
-  float ov[4] = {0.f, 0.f, 0.f, 0.f}, zv[4] = {0.f, 0.f, 0.f, 0.f};
-  if (active) {
-    Vec4<To>::load(o + row * dv + c, ov);
-    Vec4<Tz>::load(z + row * dv + c, zv);
-  }
+// The gated norm of one row from the lane's 4 values of o and z (zeros on lanes past dv): the
+// row's sum of squares over the warp, then y = o / rms(o) * w * SiLU(z) on the lane's channels.
+template <typename Ty>
+__device__ __forceinline__ void out_norm_row(const float (&ov)[4], const float (&zv)[4],
+                                             const float* __restrict__ w, Ty* yrow, int c,
+                                             bool active, int dv, float eps) {
   float ss = (ov[0] * ov[0] + ov[1] * ov[1]) + (ov[2] * ov[2] + ov[3] * ov[3]);
   ss = warp_sum(ss);
   const float inv = rsqrtf(ss / dv + eps);
@@ -498,8 +488,37 @@ out_norm_kernel(const To* __restrict__ o, const Tz* __restrict__ z, const float*
     float yv[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) yv[e] = ov[e] * inv * ww[e] * silu_fast(zv[e]);
-    Vec4<Ty>::store(y + row * dv + c, yv);
+    Vec4<Ty>::store(yrow + c, yv);
   }
+}
+
+// The gated norm over rows of dv <= 128 values, 4 consecutive channels per lane: each warp takes
+// two consecutive rows and loads both before it reduces either (twice the loads in flight of a
+// row per warp); blocks of kNormThreads threads cover 8 rows.  `o` may be wider than z / y (the
+// layer keeps o in fp32).
+constexpr int kNormThreads = 128;
+template <typename To, typename Tz, typename Ty = Tz>
+__global__ void __launch_bounds__(kNormThreads)
+out_norm_kernel(const To* __restrict__ o, const Tz* __restrict__ z, const float* __restrict__ w,
+                Ty* __restrict__ y, long long rows, int dv, float eps) {
+  const long long row0 = (long long)blockIdx.x * 8 + (threadIdx.x >> 5) * 2;
+  if (row0 >= rows) return;
+  const int c = 4 * (threadIdx.x & 31);
+  const bool active = c < dv;
+  const int nr = row0 + 1 < rows ? 2 : 1;    // (uniform over the warp)
+  float ov[2][4], zv[2][4];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) ov[r][e] = zv[r][e] = 0.f;
+    if (active && r < nr) {
+      Vec4<To>::load(o + (row0 + r) * dv + c, ov[r]);
+      Vec4<Tz>::load(z + (row0 + r) * dv + c, zv[r]);
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < 2; ++r)
+    if (r < nr) out_norm_row(ov[r], zv[r], w, y + (row0 + r) * dv, c, active, dv, eps);
 }
 
 // The conv history after a call: the raw rows of the last three tokens of [history; x] (oldest

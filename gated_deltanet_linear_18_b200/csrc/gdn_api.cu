@@ -741,10 +741,10 @@ gdn_status gdn_out_norm(const void* o, const void* z, const float* w, void* y, l
   if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == GDN_F32)
-    out_norm_kernel<float, float><<<(unsigned)blocks, 256, 0, st>>>(
+    out_norm_kernel<float, float><<<(unsigned)blocks, kNormThreads, 0, st>>>(
         (const float*)o, (const float*)z, w, (float*)y, rows, dv, eps);
   else
-    out_norm_kernel<__nv_bfloat16, __nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
+    out_norm_kernel<__nv_bfloat16, __nv_bfloat16><<<(unsigned)blocks, kNormThreads, 0, st>>>(
         (const __nv_bfloat16*)o, (const __nv_bfloat16*)z, w, (__nv_bfloat16*)y, rows, dv, eps);
   return launch_status();
 }
@@ -850,13 +850,13 @@ gdn_status gdn_layer_fwd_ex(const void* q_raw, const void* k_raw, const void* v_
   const long long blocks = (rows + 7) / 8;
   if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
   if (dtype == GDN_F32)
-    out_norm_kernel<float, float><<<(unsigned)blocks, 256, 0, st>>>(
+    out_norm_kernel<float, float><<<(unsigned)blocks, kNormThreads, 0, st>>>(
         (const float*)o, (const float*)z, norm_w, (float*)y, rows, dv, norm_eps);
   else if (y_dtype == GDN_F32)
-    out_norm_kernel<float, __nv_bfloat16, float><<<(unsigned)blocks, 256, 0, st>>>(
+    out_norm_kernel<float, __nv_bfloat16, float><<<(unsigned)blocks, kNormThreads, 0, st>>>(
         (const float*)o, (const __nv_bfloat16*)z, norm_w, (float*)y, rows, dv, norm_eps);
   else
-    out_norm_kernel<float, __nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
+    out_norm_kernel<float, __nv_bfloat16><<<(unsigned)blocks, kNormThreads, 0, st>>>(
         (const float*)o, (const __nv_bfloat16*)z, norm_w, (__nv_bfloat16*)y, rows, dv, norm_eps);
   s = launch_status();
   if (s != GDN_OK) return s;
@@ -957,10 +957,10 @@ gdn_status gdn_layer_fwd_varlen(const void* q_raw, const void* k_raw, const void
   const long long blocks = (rows + 7) / 8;
   if (blocks > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
   if (y_dtype == GDN_F32)
-    out_norm_kernel<float, __nv_bfloat16, float><<<(unsigned)blocks, 256, 0, st>>>(
+    out_norm_kernel<float, __nv_bfloat16, float><<<(unsigned)blocks, kNormThreads, 0, st>>>(
         o, (const __nv_bfloat16*)z, norm_w, (float*)y, rows, dv, norm_eps);
   else
-    out_norm_kernel<float, __nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
+    out_norm_kernel<float, __nv_bfloat16><<<(unsigned)blocks, kNormThreads, 0, st>>>(
         o, (const __nv_bfloat16*)z, norm_w, (__nv_bfloat16*)y, rows, dv, norm_eps);
   s = launch_status();
   if (s != GDN_OK) return s;
